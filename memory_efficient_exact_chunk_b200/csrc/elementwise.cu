@@ -1,0 +1,512 @@
+// Row-wise and element-wise kernels of the decoder layer: RMSNorm forward/backward, RoPE,
+// SwiGLU, chunk gather/scatter, deterministic column sums, embedding.  All are HBM-bound:
+// coalesced accesses along the feature dimension, one CTA per row (or grid-stride), fp32
+// arithmetic, warp-shuffle reductions.
+#include "sbp_internal.cuh"
+
+namespace sbp {
+
+namespace {
+
+constexpr int kRowThreads = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = 0.f;
+  const int nw = blockDim.x >> 5;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+// ---------------------------------------------------------------- RMSNorm forward
+__global__ void rmsnorm_fwd_kernel(int64_t cols, int xdt, const void* __restrict__ x, int gdt,
+                                   const void* __restrict__ g, int ydt, void* __restrict__ y,
+                                   float* __restrict__ rstd, float eps) {
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  const int64_t base = r * cols;
+  float ss = 0.f;
+  for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+    const float v = ld_dt(x, xdt, base + c);
+    ss = fmaf(v, v, ss);
+  }
+  ss = block_sum(ss, red);
+  const float rs = rsqrtf(ss / (float)cols + eps);
+  for (int64_t c = threadIdx.x; c < cols; c += blockDim.x)
+    st_dt(y, ydt, base + c, ld_dt(x, xdt, base + c) * rs * ld_dt(g, gdt, c));
+  if (rstd && threadIdx.x == 0) rstd[r] = rs;
+}
+
+// ---------------------------------------------------------------- RMSNorm backward
+// Each CTA handles rows r = blockIdx.x, blockIdx.x + gridDim.x, ...; its dg partial goes to
+// partial[blockIdx.x, :] and a second kernel sums the partials in a fixed order.
+constexpr int kBwdBlocks = 296;
+
+__global__ void rmsnorm_bwd_kernel(int64_t rows, int64_t cols, int xdt,
+                                   const void* __restrict__ x, int gdt,
+                                   const void* __restrict__ g, const float* __restrict__ rstd,
+                                   const float* __restrict__ dy, const float* __restrict__ base,
+                                   float* __restrict__ out, int accumulate,
+                                   float* __restrict__ partial) {
+  __shared__ float red[32];
+  extern __shared__ float dgs[];  // [cols]
+  for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) dgs[c] = 0.f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int64_t o = r * cols;
+    const float rs = rstd[r];
+    float dot = 0.f;
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+      const float xh = ld_dt(x, xdt, o + c) * rs;
+      const float u = dy[o + c] * ld_dt(g, gdt, c);
+      dot = fmaf(xh, u, dot);
+    }
+    dot = block_sum(dot, red) / (float)cols;
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+      const float xh = ld_dt(x, xdt, o + c) * rs;
+      const float d = dy[o + c];
+      const float u = d * ld_dt(g, gdt, c);
+      float v = rs * (u - xh * dot);
+      if (base) v += base[o + c];
+      if (accumulate) v += out[o + c];
+      out[o + c] = v;
+      dgs[c] = fmaf(d, xh, dgs[c]);
+    }
+  }
+  __syncthreads();
+  for (int64_t c = threadIdx.x; c < cols; c += blockDim.x)
+    partial[(int64_t)blockIdx.x * cols + c] = dgs[c];
+}
+
+__global__ void colsum_partials_kernel(int64_t nparts, int64_t cols,
+                                       const float* __restrict__ partial,
+                                       float* __restrict__ dst) {
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  float s = 0.f;
+  for (int64_t p = 0; p < nparts; ++p) s += partial[p * cols + c];
+  dst[c] += s;
+}
+
+// column partial sums of a [rows, cols] fp32 matrix: CTA b sums rows b, b + grid, ...
+__global__ void colsum_stage1_kernel(int64_t rows, int64_t cols, const float* __restrict__ src,
+                                     float* __restrict__ partial) {
+  const int64_t c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  float s = 0.f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) s += src[r * cols + c];
+  partial[(int64_t)blockIdx.x * cols + c] = s;
+}
+constexpr int kColsumParts = 64;
+
+// ---------------------------------------------------------------- RoPE
+__global__ void rope_table_kernel(int64_t T, int64_t half, double theta, float* cosb,
+                                  float* sinb) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * half) return;
+  const int64_t t = i / half, j = i % half;
+  const double inv_freq = pow(theta, -(2.0 * (double)j) / (double)(2 * half));
+  const double a = (double)t * inv_freq;
+  cosb[i] = (float)cos(a);
+  sinb[i] = (float)sin(a);
+}
+
+// one thread per (row, head, pair j): rotates (x_j, x_{j+half})
+__global__ void qkv_post_kernel(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H,
+                                int64_t Hkv, int64_t hd, const float* __restrict__ qkv, int dt,
+                                void* __restrict__ q, void* __restrict__ Kp,
+                                void* __restrict__ Vp, const float* __restrict__ cosb,
+                                const float* __restrict__ sinb) {
+  const int64_t half = hd / 2;
+  const int64_t heads = H + 2 * Hkv;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * heads * half) return;
+  const int64_t j = i % half;
+  const int64_t hh = (i / half) % heads;
+  const int64_t r = i / (half * heads);
+  const int64_t b = r / Tc, t = s + r % Tc;
+  const int64_t width = heads * hd;
+  const float x1 = qkv[r * width + hh * hd + j];
+  const float x2 = qkv[r * width + hh * hd + j + half];
+  if (hh < H + Hkv) {
+    const float c = cosb[t * half + j], sn = sinb[t * half + j];
+    const float y1 = x1 * c - x2 * sn;
+    const float y2 = x2 * c + x1 * sn;
+    if (hh < H) {
+      const int64_t o = r * H * hd + hh * hd;
+      st_dt(q, dt, o + j, y1);
+      st_dt(q, dt, o + j + half, y2);
+    } else {
+      const int64_t o = (b * T + t) * Hkv * hd + (hh - H) * hd;
+      st_dt(Kp, dt, o + j, y1);
+      st_dt(Kp, dt, o + j + half, y2);
+    }
+  } else {
+    const int64_t o = (b * T + t) * Hkv * hd + (hh - H - Hkv) * hd;
+    st_dt(Vp, dt, o + j, x1);
+    st_dt(Vp, dt, o + j + half, x2);
+  }
+}
+
+// inverse rotation (transpose): (d1, d2) -> (d1 c + d2 s, d2 c - d1 s)
+__global__ void rope_inv_kernel(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd,
+                                float* __restrict__ x, const float* __restrict__ cosb,
+                                const float* __restrict__ sinb) {
+  const int64_t half = hd / 2;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * heads * half) return;
+  const int64_t j = i % half;
+  const int64_t hh = (i / half) % heads;
+  const int64_t r = i / (half * heads);
+  const int64_t t = s + r % Tc;
+  const int64_t o = r * heads * hd + hh * hd;
+  const float d1 = x[o + j], d2 = x[o + j + half];
+  const float c = cosb[t * half + j], sn = sinb[t * half + j];
+  x[o + j] = d1 * c + d2 * sn;
+  x[o + j + half] = d2 * c - d1 * sn;
+}
+
+__global__ void gather_rope_inv_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s,
+                                       int64_t heads, int64_t hd, const float* __restrict__ src,
+                                       float* __restrict__ dst, const float* __restrict__ cosb,
+                                       const float* __restrict__ sinb) {
+  const int64_t half = hd / 2;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * Tc * heads * half) return;
+  const int64_t j = i % half;
+  const int64_t hh = (i / half) % heads;
+  const int64_t r = i / (half * heads);
+  const int64_t b = r / Tc, t = s + r % Tc;
+  const int64_t so = (b * T + t) * heads * hd + hh * hd;
+  const int64_t o = r * heads * hd + hh * hd;
+  const float d1 = src[so + j], d2 = src[so + j + half];
+  const float c = cosb[t * half + j], sn = sinb[t * half + j];
+  dst[o + j] = d1 * c + d2 * sn;
+  dst[o + j + half] = d2 * c - d1 * sn;
+}
+
+// ---------------------------------------------------------------- SwiGLU
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
+
+__global__ void swiglu_fwd_kernel(int64_t R, int64_t f, int dt, const void* __restrict__ gu,
+                                  void* __restrict__ m) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * f) return;
+  const int64_t r = i / f, c = i % f;
+  const float gv = ld_dt(gu, dt, r * 2 * f + c);
+  const float uv = ld_dt(gu, dt, r * 2 * f + f + c);
+  st_dt(m, dt, i, gv * sigmoidf_(gv) * uv);
+}
+
+__global__ void swiglu_bwd_kernel(int64_t R, int64_t f, int dt, const void* __restrict__ gu,
+                                  const float* __restrict__ dm, void* __restrict__ dgu) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * f) return;
+  const int64_t r = i / f, c = i % f;
+  const float gv = ld_dt(gu, dt, r * 2 * f + c);
+  const float uv = ld_dt(gu, dt, r * 2 * f + f + c);
+  const float sg = sigmoidf_(gv);
+  const float d = dm[i];
+  st_dt(dgu, dt, r * 2 * f + c, d * uv * sg * (1.f + gv * (1.f - sg)));
+  st_dt(dgu, dt, r * 2 * f + f + c, d * gv * sg);
+}
+
+// ---------------------------------------------------------------- gather / scatter
+__global__ void gather_chunk_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                                    int dt, const void* __restrict__ src, void* __restrict__ dst) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * Tc * cols) return;
+  const int64_t c = i % cols, r = i / cols;
+  const int64_t b = r / Tc, t = s + r % Tc;
+  const int64_t so = (b * T + t) * cols + c;
+  if (dt == DT_BF16)
+    static_cast<__nv_bfloat16*>(dst)[i] = static_cast<const __nv_bfloat16*>(src)[so];
+  else
+    static_cast<float*>(dst)[i] = static_cast<const float*>(src)[so];
+}
+
+__global__ void scatter_chunk_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                                     int dt, const void* __restrict__ src, void* __restrict__ dst,
+                                     int accumulate) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * Tc * cols) return;
+  const int64_t c = i % cols, r = i / cols;
+  const int64_t b = r / Tc, t = s + r % Tc;
+  const int64_t o = (b * T + t) * cols + c;
+  if (dt == DT_BF16) {
+    static_cast<__nv_bfloat16*>(dst)[o] = static_cast<const __nv_bfloat16*>(src)[i];
+  } else {
+    const float v = static_cast<const float*>(src)[i];
+    float* d = static_cast<float*>(dst);
+    d[o] = accumulate ? d[o] + v : v;
+  }
+}
+
+__global__ void add_residual_kernel(int64_t n, int xdt, const void* __restrict__ x,
+                                    const float* __restrict__ z, int ydt, void* __restrict__ y) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  st_dt(y, ydt, i, ld_dt(x, xdt, i) + z[i]);
+}
+
+__global__ void copy_cast_kernel(int64_t n, int sdt, const void* __restrict__ src, int ddt,
+                                 void* __restrict__ dst) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  st_dt(dst, ddt, i, ld_dt(src, sdt, i));
+}
+
+// ---------------------------------------------------------------- embedding
+// ids outside [0, vocab) produce a zero row (and are skipped by the backward)
+__global__ void embed_fwd_kernel(int64_t rows, int64_t cols, int64_t vocab, int dt,
+                                 const int* __restrict__ ids, const void* __restrict__ table,
+                                 void* __restrict__ y) {
+  const int64_t r = blockIdx.x;
+  const int64_t v = ids[r];
+  const bool ok = v >= 0 && v < vocab;
+  for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+    if (dt == DT_BF16)
+      static_cast<__nv_bfloat16*>(y)[r * cols + c] =
+          ok ? static_cast<const __nv_bfloat16*>(table)[v * cols + c] : __float2bfloat16_rn(0.f);
+    else
+      static_cast<float*>(y)[r * cols + c] = ok ? static_cast<const float*>(table)[v * cols + c]
+                                                : 0.f;
+  }
+}
+
+// Deterministic embedding backward: counting sort of rows by id (stable), then one CTA per
+// distinct id sums its rows in row order.
+__global__ void embed_count_kernel(int64_t rows, int64_t vocab, const int* __restrict__ ids,
+                                   int* cnt) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < rows && ids[r] >= 0 && ids[r] < vocab) atomicAdd(&cnt[ids[r]], 1);
+}
+// exclusive scan of cnt[0..vocab) into off (single CTA, 1024 threads, sequential chunks)
+__global__ void scan_kernel(int64_t n, const int* __restrict__ cnt, int* __restrict__ off) {
+  __shared__ int part[1024];
+  const int64_t per = (n + blockDim.x - 1) / blockDim.x;
+  const int64_t b = threadIdx.x * per, e = imin(n, b + per);
+  int s = 0;
+  for (int64_t i = b; i < e; ++i) s += cnt[i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) { const int t = part[i]; part[i] = a; a += t; }
+  }
+  __syncthreads();
+  int a = part[threadIdx.x];
+  for (int64_t i = b; i < e; ++i) { off[i] = a; a += cnt[i]; }
+}
+// rows of each id land in their segment in arbitrary order (atomics); the accumulate kernel
+// restores row order inside the segment before summing, so the sum is deterministic.
+__global__ void embed_place_kernel(int64_t rows, int64_t vocab, const int* __restrict__ ids,
+                                   int* __restrict__ pos, int* __restrict__ order) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < rows && ids[r] >= 0 && ids[r] < vocab) order[atomicAdd(&pos[ids[r]], 1)] = (int)r;
+}
+constexpr int kSegSort = 2048;
+__global__ void embed_accum_kernel(int64_t rows, int64_t cols, const int* __restrict__ ids,
+                                   const int* __restrict__ off0, const int* __restrict__ cnt,
+                                   const int* __restrict__ order, const float* __restrict__ dy,
+                                   float* __restrict__ dtable) {
+  __shared__ int seg[kSegSort];
+  __shared__ int srt[kSegSort];
+  const int64_t v = blockIdx.x;
+  const int n = cnt[v];
+  if (n == 0) return;
+  if (n <= kSegSort) {
+    const int o = off0[v];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) seg[i] = order[o + i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      int rank = 0;
+      const int a = seg[i];
+      for (int j = 0; j < n; ++j) rank += (seg[j] < a);
+      srt[rank] = a;
+    }
+    __syncthreads();
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+      float s = 0.f;
+      for (int k = 0; k < n; ++k) s += dy[(int64_t)srt[k] * cols + c];
+      dtable[v * cols + c] += s;
+    }
+  } else {
+    // very frequent id: walk all rows in order
+    for (int64_t c0 = 0; c0 < cols; c0 += blockDim.x) {
+      const int64_t c = c0 + threadIdx.x;
+      float s = 0.f;
+      for (int64_t r = 0; r < rows; ++r)
+        if (ids[r] == (int)v && c < cols) s += dy[r * cols + c];
+      if (c < cols) dtable[v * cols + c] += s;
+    }
+  }
+}
+
+inline unsigned nblk(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
+
+}  // namespace
+
+cudaError_t rmsnorm_fwd(int64_t rows, int64_t cols, int xdt, const void* x, int gdt,
+                        const void* g, int ydt, void* y, float* rstd, float eps,
+                        cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  rmsnorm_fwd_kernel<<<(unsigned)rows, kRowThreads, 0, st>>>(cols, xdt, x, gdt, g, ydt, y, rstd,
+                                                             eps);
+  return cudaGetLastError();
+}
+
+size_t rmsnorm_bwd_partial_floats(int64_t cols) { return (size_t)kBwdBlocks * cols; }
+
+cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int gdt,
+                        const void* g, const float* rstd, const float* dy, const float* base,
+                        float* out, int accumulate, float* dg, float* partial,
+                        cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const size_t smem = (size_t)cols * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(rmsnorm_bwd_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  rmsnorm_bwd_kernel<<<kBwdBlocks, kRowThreads, smem, st>>>(rows, cols, xdt, x, gdt, g, rstd, dy,
+                                                            base, out, accumulate, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (dg) {
+    colsum_partials_kernel<<<nblk(cols, 256), 256, 0, st>>>(kBwdBlocks, cols, partial, dg);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+cudaError_t rope_table(int64_t T, int64_t hd, double theta, float* cosb, float* sinb,
+                       cudaStream_t st) {
+  const int64_t n = T * (hd / 2);
+  if (n <= 0) return cudaSuccess;
+  rope_table_kernel<<<nblk(n, 256), 256, 0, st>>>(T, hd / 2, theta, cosb, sinb);
+  return cudaGetLastError();
+}
+
+cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int64_t Hkv,
+                     int64_t hd, const float* qkv, int dt, void* q, void* Kp, void* Vp,
+                     const float* cosb, const float* sinb, cudaStream_t st) {
+  const int64_t n = R * (H + 2 * Hkv) * (hd / 2);
+  if (n <= 0) return cudaSuccess;
+  qkv_post_kernel<<<nblk(n, 256), 256, 0, st>>>(R, Tc, s, T, H, Hkv, hd, qkv, dt, q, Kp, Vp,
+                                                cosb, sinb);
+  return cudaGetLastError();
+}
+
+cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd, float* x,
+                         const float* cosb, const float* sinb, cudaStream_t st) {
+  const int64_t n = R * heads * (hd / 2);
+  if (n <= 0) return cudaSuccess;
+  rope_inv_kernel<<<nblk(n, 256), 256, 0, st>>>(R, Tc, s, heads, hd, x, cosb, sinb);
+  return cudaGetLastError();
+}
+
+cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t heads,
+                            int64_t hd, const float* src, float* dst, const float* cosb,
+                            const float* sinb, cudaStream_t st) {
+  const int64_t n = B * Tc * heads * (hd / 2);
+  if (n <= 0) return cudaSuccess;
+  gather_rope_inv_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, heads, hd, src, dst, cosb,
+                                                       sinb);
+  return cudaGetLastError();
+}
+
+cudaError_t swiglu_fwd(int64_t R, int64_t f, int dt, const void* gu, void* m, cudaStream_t st) {
+  if (R * f <= 0) return cudaSuccess;
+  swiglu_fwd_kernel<<<nblk(R * f, 256), 256, 0, st>>>(R, f, dt, gu, m);
+  return cudaGetLastError();
+}
+
+cudaError_t swiglu_bwd(int64_t R, int64_t f, int dt, const void* gu, const float* dm, void* dgu,
+                       cudaStream_t st) {
+  if (R * f <= 0) return cudaSuccess;
+  swiglu_bwd_kernel<<<nblk(R * f, 256), 256, 0, st>>>(R, f, dt, gu, dm, dgu);
+  return cudaGetLastError();
+}
+
+cudaError_t gather_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
+                         const void* src, void* dst, cudaStream_t st) {
+  const int64_t n = B * Tc * cols;
+  if (n <= 0) return cudaSuccess;
+  gather_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, dt, src, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t scatter_chunk_f32(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                              const float* src, float* dst, int accumulate, cudaStream_t st) {
+  const int64_t n = B * Tc * cols;
+  if (n <= 0) return cudaSuccess;
+  scatter_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, DT_F32, src, dst,
+                                                     accumulate);
+  return cudaGetLastError();
+}
+
+cudaError_t scatter_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
+                          const void* src, void* dst, cudaStream_t st) {
+  const int64_t n = B * Tc * cols;
+  if (n <= 0) return cudaSuccess;
+  scatter_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, dt, src, dst, 0);
+  return cudaGetLastError();
+}
+
+size_t colsum_partial_floats(int64_t cols) { return (size_t)kColsumParts * cols; }
+
+cudaError_t colsum_acc(int64_t rows, int64_t cols, const float* src, float* dst, float* partial,
+                       cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  dim3 g1(kColsumParts, nblk(cols, 256));
+  colsum_stage1_kernel<<<g1, 256, 0, st>>>(rows, cols, src, partial);
+  colsum_partials_kernel<<<nblk(cols, 256), 256, 0, st>>>(kColsumParts, cols, partial, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int ydt, void* y,
+                         cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  add_residual_kernel<<<nblk(n, 256), 256, 0, st>>>(n, xdt, x, z, ydt, y);
+  return cudaGetLastError();
+}
+
+cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  copy_cast_kernel<<<nblk(n, 256), 256, 0, st>>>(n, sdt, src, ddt, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t embed_fwd(int64_t rows, int64_t cols, int64_t vocab, int dt, const int* ids,
+                      const void* table, void* y, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  embed_fwd_kernel<<<(unsigned)rows, 256, 0, st>>>(rows, cols, vocab, dt, ids, table, y);
+  return cudaGetLastError();
+}
+
+size_t embed_bwd_ws_ints(int64_t rows, int64_t vocab) { return (size_t)(3 * vocab + rows); }
+
+cudaError_t embed_bwd(int64_t rows, int64_t cols, int64_t vocab, const int* ids, const float* dy,
+                      float* dtable, int* ws, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  int* cnt = ws;
+  int* off = ws + vocab;
+  int* pos = ws + 2 * vocab;
+  int* order = ws + 3 * vocab;
+  cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int) * vocab, st);
+  if (e != cudaSuccess) return e;
+  embed_count_kernel<<<nblk(rows, 256), 256, 0, st>>>(rows, vocab, ids, cnt);
+  scan_kernel<<<1, 1024, 0, st>>>(vocab, cnt, off);
+  e = cudaMemcpyAsync(pos, off, sizeof(int) * vocab, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return e;
+  embed_place_kernel<<<nblk(rows, 256), 256, 0, st>>>(rows, vocab, ids, pos, order);
+  embed_accum_kernel<<<(unsigned)vocab, 128, 0, st>>>(rows, cols, ids, off, cnt, order, dy,
+                                                       dtable);
+  return cudaGetLastError();
+}
+
+}  // namespace sbp

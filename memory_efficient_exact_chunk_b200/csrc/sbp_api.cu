@@ -1,0 +1,571 @@
+// C ABI of libsbp (declared in include/sbp.h): argument checks, workspace carving and the
+// host-side chunk loops that queue the kernels on the caller's stream.
+//
+// Sources: "StreamBP: Memory-Efficient Backpropagation" (skill page), sections Core Concept,
+// Architecture Overview and Implementation; "StreamBP: Memory-Efficient Exact Backpropagation
+// for Long Sequence Training of LLMs" (paper page), Abstract.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "sbp.h"
+#include "sbp_internal.cuh"
+
+using namespace sbp;
+
+namespace {
+
+thread_local std::string g_err;
+
+sbp_status fail(sbp_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define SBP_CK(expr)                                                                 \
+  do {                                                                               \
+    cudaError_t e_ = (expr);                                                         \
+    if (e_ != cudaSuccess)                                                           \
+      return fail(SBP_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));     \
+  } while (0)
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Bump allocator over the caller's workspace (dry run when base == nullptr).
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+  void* take_bytes(size_t n) { return take<char>(n); }
+};
+
+// ------------------------------------------------------------------------ chunk bounds
+inline int64_t chunk_size(int64_t T, int D) { return T / D; }
+inline void chunk_range(int64_t T, int D, int i, int64_t& s, int64_t& e) {
+  const int64_t c = chunk_size(T, D);
+  s = (int64_t)i * c;
+  e = (i < D - 1) ? (int64_t)(i + 1) * c : T;
+}
+inline int64_t chunk_max(int64_t T, int D) { return T - (int64_t)(D - 1) * chunk_size(T, D); }
+
+// ------------------------------------------------------------------------ LM head plan
+constexpr int64_t kVocabBlock = 8192;
+
+struct CePlan {
+  int* status;
+  int* idx;
+  int* count;
+  void* hc;
+  int* yc;
+  float *wc, *zy, *lse, *row_loss, *pmax, *psum;
+  void* G;
+  int64_t Rmax, tiles, Vb;
+};
+
+void ce_carve(Carver& c, int64_t N, int64_t d, int64_t V, int D, int dt, CePlan& p) {
+  p.status = static_cast<int*>(c.take_bytes(kStatusBytes));
+  p.Rmax = chunk_max(N, D);
+  p.tiles = gemm_lse_tiles(V);
+  p.Vb = V < kVocabBlock ? V : kVocabBlock;
+  p.idx = c.take<int>(p.Rmax);
+  p.count = c.take<int>(64);
+  p.hc = c.take_bytes((size_t)p.Rmax * d * dt_size(dt));
+  p.yc = c.take<int>(p.Rmax);
+  p.wc = c.take<float>(p.Rmax);
+  p.zy = c.take<float>(p.Rmax);
+  p.lse = c.take<float>(p.Rmax);
+  p.row_loss = c.take<float>(p.Rmax);
+  p.pmax = c.take<float>((size_t)p.Rmax * p.tiles);
+  p.psum = c.take<float>((size_t)p.Rmax * p.tiles);
+  p.G = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
+}
+
+// ------------------------------------------------------------------------ layer plan
+struct LayerPlan {
+  int* status;
+  float *cosb, *sinb;
+  void *Kp, *Vp;
+  float *dKp, *dVp;
+  void *xg, *n1, *q, *o, *n2, *gu, *m, *dgu, *dO;
+  float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dm, *dn2, *dh, *delta, *dq, *dn1, *dxg;
+  float *dkpre, *dvg, *rpart, *cpart;
+  int64_t R;
+};
+
+void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
+  const int dt = L.dtype;
+  const size_t es = dt_size(dt);
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
+  const int64_t dq = L.n_heads * L.head_dim, dkv = L.n_kv_heads * L.head_dim;
+  const int64_t R = B * chunk_max(T, L.num_chunks);
+  p.R = R;
+  p.status = static_cast<int*>(c.take_bytes(kStatusBytes));
+  p.cosb = c.take<float>((size_t)T * (L.head_dim / 2));
+  p.sinb = c.take<float>((size_t)T * (L.head_dim / 2));
+  p.Kp = c.take_bytes((size_t)B * T * dkv * es);
+  p.Vp = c.take_bytes((size_t)B * T * dkv * es);
+  p.dKp = c.take<float>((size_t)B * T * dkv);
+  p.dVp = c.take<float>((size_t)B * T * dkv);
+  p.xg = c.take_bytes((size_t)R * d * es);
+  p.dyg = c.take<float>((size_t)R * d);
+  p.n1 = c.take_bytes((size_t)R * d * es);
+  p.rstd1 = c.take<float>(R);
+  p.qkv = c.take<float>((size_t)R * (dq + 2 * dkv));
+  p.q = c.take_bytes((size_t)R * dq * es);
+  p.o = c.take_bytes((size_t)R * dq * es);
+  p.alse = c.take<float>((size_t)R * L.n_heads);
+  p.hbuf = c.take<float>((size_t)R * d);
+  p.n2 = c.take_bytes((size_t)R * d * es);
+  p.rstd2 = c.take<float>(R);
+  p.gu = c.take_bytes((size_t)R * 2 * f * es);
+  p.m = c.take_bytes((size_t)R * f * es);
+  p.dm = c.take<float>((size_t)R * f);
+  p.dgu = c.take_bytes((size_t)R * 2 * f * es);
+  p.dn2 = c.take<float>((size_t)R * d);
+  p.dh = c.take<float>((size_t)R * d);
+  p.dO = c.take_bytes((size_t)R * dq * es);
+  p.delta = c.take<float>((size_t)R * L.n_heads);
+  p.dq = c.take<float>((size_t)R * dq);
+  p.dn1 = c.take<float>((size_t)R * d);
+  p.dxg = c.take<float>((size_t)R * d);
+  p.dkpre = c.take<float>((size_t)R * dkv);
+  p.dvg = c.take<float>((size_t)R * dkv);
+  p.rpart = c.take<float>(rmsnorm_bwd_partial_floats(d));
+  int64_t wmax = dq > dkv ? dq : dkv;
+  p.cpart = c.take<float>(colsum_partial_floats(wmax));
+}
+
+// GEMM descriptor helpers.  Matrices are row-major with the given leading dimension.
+//   "N" operand (no transpose): A(m,k) = A[m*ld + k]   /  B(k,n) = B[k*ld + n]
+//   "T" operand (transposed)  : A(m,k) = A[k*ld + m]   /  B(k,n) = B[n*ld + k]
+GemmDesc mk_gemm(int64_t M, int64_t N, int64_t K, int adt, const void* A, bool a_t, int64_t lda,
+                 int bdt, const void* B, bool b_t, int64_t ldb, int cdt, void* C, int64_t ldc,
+                 int epi) {
+  GemmDesc g;
+  g.M = M; g.N = N; g.K = K;
+  g.adt = adt; g.A = A;
+  if (!a_t) { g.sam = lda; g.sak = 1; } else { g.sam = 1; g.sak = lda; }
+  g.bdt = bdt; g.B = B;
+  if (!b_t) { g.sbk = ldb; g.sbn = 1; } else { g.sbk = 1; g.sbn = ldb; }
+  g.cdt = cdt; g.C = C; g.ldc = ldc;
+  g.epi = epi;
+  return g;
+}
+
+sbp_status check_layer_cfg(const sbp_layer_cfg* L) {
+  if (!L) return fail(SBP_ERR_INVALID_ARG, "cfg is NULL");
+  if (L->batch <= 0 || L->seq_len <= 0 || L->d_model <= 0 || L->n_heads <= 0 ||
+      L->n_kv_heads <= 0 || L->head_dim <= 0 || L->ffn <= 0)
+    return fail(SBP_ERR_INVALID_ARG, "all layer dimensions must be positive");
+  if (L->num_chunks < 1 || (int64_t)L->num_chunks > L->seq_len)
+    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= seq_len (got %d, T=%lld)",
+                L->num_chunks, (long long)L->seq_len);
+  if (L->n_heads % L->n_kv_heads != 0)
+    return fail(SBP_ERR_INVALID_ARG, "n_heads %% n_kv_heads != 0");
+  if (L->dtype != SBP_F32 && L->dtype != SBP_BF16)
+    return fail(SBP_ERR_INVALID_ARG, "unknown dtype %d", L->dtype);
+  if (L->head_dim % 2 != 0 || L->head_dim > 256)
+    return fail(SBP_ERR_UNSUPPORTED, "head_dim must be even and <= 256");
+  if (!(L->rms_eps >= 0.f)) return fail(SBP_ERR_INVALID_ARG, "rms_eps must be >= 0");
+  if (!(L->rope_theta > 0.0)) return fail(SBP_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (L->dtype == SBP_BF16) {
+    const int64_t dq = L->n_heads * L->head_dim, dkv = L->n_kv_heads * L->head_dim;
+    if (L->d_model % 8 || dq % 8 || dkv % 8 || L->ffn % 8)
+      return fail(SBP_ERR_UNSUPPORTED, "bf16 needs d_model, heads*head_dim, ffn % 8 == 0");
+  }
+  return SBP_OK;
+}
+
+sbp_status check_weights(const sbp_layer_weights* w, bool* has_bias) {
+  if (!w) return fail(SBP_ERR_INVALID_ARG, "weights is NULL");
+  const void* req[] = {w->ln1_g, w->wq, w->wk, w->wv, w->wo, w->ln2_g, w->w_gate, w->w_up,
+                       w->w_down};
+  for (const void* p : req) {
+    if (!p) return fail(SBP_ERR_INVALID_ARG, "a required weight pointer is NULL");
+    if (!aligned16(p)) return fail(SBP_ERR_INVALID_ARG, "weight pointer not 16-byte aligned");
+  }
+  const int nb = (w->bq != nullptr) + (w->bk != nullptr) + (w->bv != nullptr);
+  if (nb != 0 && nb != 3) return fail(SBP_ERR_INVALID_ARG, "bq/bk/bv must be all set or all NULL");
+  *has_bias = nb == 3;
+  return SBP_OK;
+}
+
+// Forward recompute of one chunk: fills n1, rstd1, q, K/V prefix rows, o, alse, hbuf (= h),
+// n2, rstd2, gu and m.  xg holds the chunk's gathered input.
+sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& w,
+                               const LayerPlan& p, int64_t s, int64_t Tc, cudaStream_t st) {
+  const int dt = L.dtype;
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
+  const int64_t H = L.n_heads, Hkv = L.n_kv_heads, hd = L.head_dim;
+  const int64_t dq = H * hd, dkv = Hkv * hd, W3 = dq + 2 * dkv;
+  const int64_t R = B * Tc;
+  SBP_CK(rmsnorm_fwd(R, d, dt, p.xg, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+  {
+    GemmDesc g = mk_gemm(R, dq, d, dt, p.n1, false, d, dt, w.wq, true, d, DT_F32, p.qkv, W3,
+                         EPI_STORE);
+    g.bias = w.bq; g.bias_dt = dt;
+    SBP_CK(gemm(g, st));
+    g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
+                EPI_STORE);
+    g.bias = w.bk; g.bias_dt = dt;
+    SBP_CK(gemm(g, st));
+    g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wv, true, d, DT_F32, p.qkv + dq + dkv, W3,
+                EPI_STORE);
+    g.bias = w.bv; g.bias_dt = dt;
+    SBP_CK(gemm(g, st));
+  }
+  SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
+  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, st));
+  SBP_CK(copy_cast(R * d, dt, p.xg, DT_F32, p.hbuf, st));
+  SBP_CK(gemm(mk_gemm(R, d, dq, dt, p.o, false, dq, dt, w.wo, true, dq, DT_F32, p.hbuf, d,
+                      EPI_ACC), st));
+  SBP_CK(rmsnorm_fwd(R, d, DT_F32, p.hbuf, dt, w.ln2_g, dt, p.n2, p.rstd2, L.rms_eps, st));
+  SBP_CK(gemm(mk_gemm(R, f, d, dt, p.n2, false, d, dt, w.w_gate, true, d, dt, p.gu, 2 * f,
+                      EPI_STORE), st));
+  SBP_CK(gemm(mk_gemm(R, f, d, dt, p.n2, false, d, dt, w.w_up, true, d, dt,
+                      static_cast<char*>(p.gu) + f * dt_size(dt), 2 * f, EPI_STORE), st));
+  SBP_CK(swiglu_fwd(R, f, dt, p.gu, p.m, st));
+  return SBP_OK;
+}
+
+sbp_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return fail(SBP_ERR_INVALID_ARG, "workspace is NULL");
+  if (((uintptr_t)ws & 255u) != 0) return fail(SBP_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (have < need)
+    return fail(SBP_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", have, need);
+  return SBP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sbp_last_error(void) { return g_err.c_str(); }
+
+const char* sbp_version(void) { return "sbp 0.1 (sm_100a)"; }
+
+sbp_status sbp_chunk_bounds(int64_t seq_len, int num_chunks, int64_t* bounds) {
+  if (!bounds) return fail(SBP_ERR_INVALID_ARG, "bounds is NULL");
+  if (num_chunks < 1 || seq_len < 1 || (int64_t)num_chunks > seq_len)
+    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= seq_len");
+  for (int i = 0; i < num_chunks; ++i) {
+    int64_t s, e;
+    chunk_range(seq_len, num_chunks, i, s, e);
+    bounds[i] = s;
+    if (i == num_chunks - 1) bounds[num_chunks] = e;
+  }
+  return SBP_OK;
+}
+
+sbp_status sbp_get_device_status(void* workspace, void* stream) {
+  if (!workspace) return fail(SBP_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  SBP_CK(cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st));
+  SBP_CK(cudaStreamSynchronize(st));
+  SBP_CK(cudaMemsetAsync(workspace, 0, sizeof(int), st));
+  if (h == DEV_OK) return SBP_OK;
+  if (h == DEV_BAD_TARGET)
+    return fail(SBP_ERR_BAD_TARGET, "a target outside [0, vocab) had a nonzero loss weight");
+  if (h == DEV_TIMEOUT) return fail(SBP_ERR_DEVICE_TIMEOUT, "a device-side wait gave up");
+  return fail(SBP_ERR_CUDA, "unknown device status %d", h);
+}
+
+// ------------------------------------------------------------------------------- LM head
+size_t sbp_lmhead_ce_workspace_size(int64_t n_tokens, int64_t hidden, int64_t vocab,
+                                    int num_chunks, sbp_dtype dt) {
+  if (n_tokens <= 0 || hidden <= 0 || vocab <= 0 || num_chunks < 1 ||
+      (int64_t)num_chunks > n_tokens)
+    return 0;
+  Carver c(nullptr);
+  CePlan p;
+  ce_carve(c, n_tokens, hidden, vocab, num_chunks, dt, p);
+  return c.off;
+}
+
+sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt,
+                                         const void* hidden_states, const void* weight,
+                                         const int32_t* targets, const float* loss_weights,
+                                         float* loss_out, float* d_hidden, float* d_weight,
+                                         void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  if (N <= 0 || d <= 0 || V <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (D < 1 || (int64_t)D > N)
+    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= n_tokens");
+  if (dt != SBP_F32 && dt != SBP_BF16) return fail(SBP_ERR_INVALID_ARG, "unknown dtype");
+  if (dt == SBP_BF16 && d % 8 != 0) return fail(SBP_ERR_UNSUPPORTED, "bf16 needs hidden % 8 == 0");
+  const void* ptrs[] = {hidden_states, weight, targets, loss_weights, loss_out, d_hidden,
+                        d_weight};
+  for (const void* q : ptrs) {
+    if (!q) return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "a pointer is not 16-byte aligned");
+  }
+  const size_t need = sbp_lmhead_ce_workspace_size(N, d, V, D, dt);
+  if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  CePlan p;
+  ce_carve(c, N, d, V, D, dt, p);
+  SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
+  for (int i = 0; i < D; ++i) {
+    int64_t s, e;
+    chunk_range(N, D, i, s, e);
+    const int64_t Rc = e - s;
+    SBP_CK(ce_compact(s, e, V, targets, loss_weights, p.idx, p.count, p.status, st));
+    SBP_CK(ce_gather(Rc, d, dt, hidden_states, p.idx, p.count, targets, loss_weights, p.hc, p.yc,
+                     p.wc, p.zy, p.lse, st));
+    SBP_CK(zero_rows(s, e, d, d_hidden, st));
+    // pass 1: per-row log-sum-exp over the vocabulary (logits stay in GEMM tiles)
+    GemmDesc g = mk_gemm(Rc, V, d, dt, p.hc, false, d, dt, weight, true, d, DT_F32, nullptr, 0,
+                         EPI_LSE);
+    g.dynM = p.count; g.tgt = p.yc; g.col0 = 0; g.pmax = p.pmax; g.psum = p.psum;
+    g.pld = p.tiles; g.zy = p.zy;
+    SBP_CK(gemm(g, st));
+    SBP_CK(ce_finish(Rc, p.tiles, p.pmax, p.psum, p.tiles, p.count, p.wc, p.zy, p.lse,
+                     p.row_loss, loss_out, i == 0, st));
+    // pass 2, one vocabulary block at a time: G = w (softmax - onehot), dH += G W_b,
+    // dW_b += G^T H
+    for (int64_t vb = 0; vb < V; vb += p.Vb) {
+      const int64_t nb = (V - vb) < p.Vb ? (V - vb) : p.Vb;
+      const char* Wb = static_cast<const char*>(weight) + vb * d * dt_size(dt);
+      GemmDesc gg = mk_gemm(Rc, nb, d, dt, p.hc, false, d, dt, Wb, true, d, dt, p.G, nb,
+                            EPI_CEGRAD);
+      gg.dynM = p.count; gg.lse = p.lse; gg.tgt = p.yc; gg.wt = p.wc; gg.col0 = vb;
+      SBP_CK(gemm(gg, st));
+      GemmDesc gh = mk_gemm(Rc, d, nb, dt, p.G, false, nb, dt, Wb, false, d, DT_F32, d_hidden,
+                            d, vb == 0 ? EPI_STORE : EPI_ACC);
+      gh.dynM = p.count; gh.crow = p.idx;
+      SBP_CK(gemm(gh, st));
+      GemmDesc gw = mk_gemm(nb, d, Rc, dt, p.G, true, nb, dt, p.hc, false, d, DT_F32,
+                            d_weight + vb * d, d, EPI_ACC);
+      gw.dynK = p.count;
+      SBP_CK(gemm(gw, st));
+    }
+  }
+  return SBP_OK;
+}
+
+// ------------------------------------------------------------------------------- layer
+size_t sbp_decoder_layer_workspace_size(const sbp_layer_cfg* cfg) {
+  if (check_layer_cfg(cfg) != SBP_OK) return 0;
+  Carver c(nullptr);
+  LayerPlan p;
+  layer_carve(c, *cfg, p);
+  return c.off;
+}
+
+sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
+                                             const sbp_layer_weights* w, const void* x,
+                                             const float* dy, float* dx,
+                                             const sbp_layer_grads* gr, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+  if (sbp_status s = check_layer_cfg(cfg)) return s;
+  bool has_bias = false;
+  if (sbp_status s = check_weights(w, &has_bias)) return s;
+  if (!gr) return fail(SBP_ERR_INVALID_ARG, "grads is NULL");
+  {
+    float* req[] = {gr->ln1_g, gr->wq, gr->wk, gr->wv, gr->wo, gr->ln2_g, gr->w_gate, gr->w_up,
+                    gr->w_down};
+    for (float* q : req)
+      if (!q || !aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "grad pointer NULL or misaligned");
+    const int nb = (gr->bq != nullptr) + (gr->bk != nullptr) + (gr->bv != nullptr);
+    if ((has_bias && nb != 3) || (!has_bias && nb != 0))
+      return fail(SBP_ERR_INVALID_ARG, "bias grads must be set exactly when biases are");
+  }
+  const void* io[] = {x, dy, dx};
+  for (const void* q : io)
+    if (!q || !aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "x/dy/dx NULL or misaligned");
+  const sbp_layer_cfg& L = *cfg;
+  const size_t need = sbp_decoder_layer_workspace_size(cfg);
+  if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  LayerPlan p;
+  layer_carve(c, L, p);
+  const int dt = L.dtype;
+  const size_t es = dt_size(dt);
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
+  const int64_t H = L.n_heads, Hkv = L.n_kv_heads, hd = L.head_dim;
+  const int64_t dq = H * hd, dkv = Hkv * hd;
+  const int D = L.num_chunks;
+
+  SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
+  SBP_CK(rope_table(T, hd, L.rope_theta, p.cosb, p.sinb, st));
+  SBP_CK(cudaMemsetAsync(p.dKp, 0, sizeof(float) * (size_t)B * T * dkv, st));
+  SBP_CK(cudaMemsetAsync(p.dVp, 0, sizeof(float) * (size_t)B * T * dkv, st));
+
+  for (int i = 0; i < D; ++i) {
+    int64_t s, e;
+    chunk_range(T, D, i, s, e);
+    const int64_t Tc = e - s, R = B * Tc;
+    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+    SBP_CK(gather_chunk(B, T, Tc, s, d, DT_F32, dy, p.dyg, st));
+    if (sbp_status r = layer_chunk_forward(L, *w, p, s, Tc, st)) return r;
+    // ---- MLP backward
+    SBP_CK(gemm(mk_gemm(R, f, d, DT_F32, p.dyg, false, d, dt, w->w_down, false, f, DT_F32, p.dm,
+                        f, EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(d, f, R, DT_F32, p.dyg, true, d, dt, p.m, false, f, DT_F32, gr->w_down,
+                        f, EPI_ACC), st));
+    SBP_CK(swiglu_bwd(R, f, dt, p.gu, p.dm, p.dgu, st));
+    const char* dU = static_cast<const char*>(p.dgu) + f * es;
+    SBP_CK(gemm(mk_gemm(R, d, f, dt, p.dgu, false, 2 * f, dt, w->w_gate, false, d, DT_F32, p.dn2,
+                        d, EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(R, d, f, dt, dU, false, 2 * f, dt, w->w_up, false, d, DT_F32, p.dn2, d,
+                        EPI_ACC), st));
+    SBP_CK(gemm(mk_gemm(f, d, R, dt, p.dgu, true, 2 * f, dt, p.n2, false, d, DT_F32, gr->w_gate,
+                        d, EPI_ACC), st));
+    SBP_CK(gemm(mk_gemm(f, d, R, dt, dU, true, 2 * f, dt, p.n2, false, d, DT_F32, gr->w_up, d,
+                        EPI_ACC), st));
+    SBP_CK(rmsnorm_bwd(R, d, DT_F32, p.hbuf, dt, w->ln2_g, p.rstd2, p.dn2, p.dyg, p.dh, 0,
+                       gr->ln2_g, p.rpart, st));
+    // ---- attention output projection backward
+    SBP_CK(gemm(mk_gemm(R, dq, d, DT_F32, p.dh, false, d, dt, w->wo, false, dq, dt, p.dO, dq,
+                        EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(d, dq, R, DT_F32, p.dh, true, d, dt, p.o, false, dq, DT_F32, gr->wo, dq,
+                        EPI_ACC), st));
+    // ---- attention backward over the causal prefix; dK/dV accumulate in fp32
+    SBP_CK(attn_bwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.dO, p.alse, p.delta,
+                    p.dq, p.dKp, p.dVp, st));
+    SBP_CK(rope_inv_f32(R, Tc, s, H, hd, p.dq, p.cosb, p.sinb, st));
+    // ---- q projection backward
+    SBP_CK(gemm(mk_gemm(R, d, dq, DT_F32, p.dq, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
+                        EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(dq, d, R, DT_F32, p.dq, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
+                        EPI_ACC), st));
+    if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
+    SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, p.dxg, 0, gr->ln1_g,
+                       p.rpart, st));
+    SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 0, st));
+  }
+  // ---- K/V projection backward, chunk by chunk, once every later chunk has added its dK/dV
+  for (int j = 0; j < D; ++j) {
+    int64_t s, e;
+    chunk_range(T, D, j, s, e);
+    const int64_t Tc = e - s, R = B * Tc;
+    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+    SBP_CK(rmsnorm_fwd(R, d, dt, p.xg, dt, w->ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+    SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
+    SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
+    SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
+                        p.dn1, d, EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32, p.dn1,
+                        d, EPI_ACC), st));
+    SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d, DT_F32,
+                        gr->wk, d, EPI_ACC), st));
+    SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d, DT_F32, gr->wv,
+                        d, EPI_ACC), st));
+    if (has_bias) {
+      SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
+      SBP_CK(colsum_acc(R, dkv, p.dvg, gr->bv, p.cpart, st));
+    }
+    SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, p.dxg, 0,
+                       gr->ln1_g, p.rpart, st));
+    SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 1, st));
+  }
+  return SBP_OK;
+}
+
+sbp_status sbp_decoder_layer_forward_stream(const sbp_layer_cfg* cfg,
+                                            const sbp_layer_weights* w, const void* x, void* y,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  if (sbp_status s = check_layer_cfg(cfg)) return s;
+  bool has_bias = false;
+  if (sbp_status s = check_weights(w, &has_bias)) return s;
+  if (!x || !y || !aligned16(x) || !aligned16(y))
+    return fail(SBP_ERR_INVALID_ARG, "x/y NULL or misaligned");
+  const sbp_layer_cfg& L = *cfg;
+  const size_t need = sbp_decoder_layer_workspace_size(cfg);
+  if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  LayerPlan p;
+  layer_carve(c, L, p);
+  const int dt = L.dtype;
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
+  SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
+  SBP_CK(rope_table(T, L.head_dim, L.rope_theta, p.cosb, p.sinb, st));
+  for (int i = 0; i < L.num_chunks; ++i) {
+    int64_t s, e;
+    chunk_range(T, L.num_chunks, i, s, e);
+    const int64_t Tc = e - s, R = B * Tc;
+    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+    if (sbp_status r = layer_chunk_forward(L, *w, p, s, Tc, st)) return r;
+    SBP_CK(gemm(mk_gemm(R, d, f, dt, p.m, false, f, dt, w->w_down, true, f, DT_F32, p.hbuf, d,
+                        EPI_ACC), st));
+    SBP_CK(copy_cast(R * d, DT_F32, p.hbuf, dt, p.xg, st));
+    SBP_CK(scatter_chunk(B, T, Tc, s, d, dt, p.xg, y, st));
+  }
+  return SBP_OK;
+}
+
+// ------------------------------------------------------------------------------- support
+sbp_status sbp_rmsnorm_forward(int64_t rows, int64_t cols, sbp_dtype dt, float eps,
+                               const void* x, const void* g, void* y, float* rstd,
+                               void* stream) {
+  if (rows <= 0 || cols <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (!x || !g || !y) return fail(SBP_ERR_INVALID_ARG, "x/g/y is NULL");
+  SBP_CK(rmsnorm_fwd(rows, cols, dt, x, dt, g, dt, y, rstd, eps,
+                     static_cast<cudaStream_t>(stream)));
+  return SBP_OK;
+}
+
+size_t sbp_rmsnorm_backward_workspace_size(int64_t rows, int64_t cols) {
+  (void)rows;
+  return rmsnorm_bwd_partial_floats(cols) * sizeof(float);
+}
+
+sbp_status sbp_rmsnorm_backward(int64_t rows, int64_t cols, sbp_dtype dt, const void* x,
+                                const void* g, const float* rstd, const float* dy, float* dx,
+                                int accumulate, float* dg, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (rows <= 0 || cols <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (!x || !g || !rstd || !dy || !dx || !workspace)
+    return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (workspace_bytes < sbp_rmsnorm_backward_workspace_size(rows, cols))
+    return fail(SBP_ERR_WORKSPACE, "workspace too small");
+  SBP_CK(rmsnorm_bwd(rows, cols, dt, x, dt, g, rstd, dy, nullptr, dx, accumulate, dg,
+                     static_cast<float*>(workspace), static_cast<cudaStream_t>(stream)));
+  return SBP_OK;
+}
+
+sbp_status sbp_embedding_forward(int64_t rows, int64_t cols, int64_t vocab, sbp_dtype dt,
+                                 const int32_t* ids, const void* table, void* y, void* stream) {
+  if (rows <= 0 || cols <= 0 || vocab <= 0) return fail(SBP_ERR_INVALID_ARG, "bad sizes");
+  if (!ids || !table || !y) return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+  SBP_CK(embed_fwd(rows, cols, vocab, dt, ids, table, y, static_cast<cudaStream_t>(stream)));
+  return SBP_OK;
+}
+
+size_t sbp_embedding_backward_workspace_size(int64_t rows, int64_t vocab) {
+  return embed_bwd_ws_ints(rows, vocab) * sizeof(int);
+}
+
+sbp_status sbp_embedding_backward(int64_t rows, int64_t cols, int64_t vocab,
+                                  const int32_t* ids, const float* dy, float* d_table,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (rows <= 0 || cols <= 0 || vocab <= 0) return fail(SBP_ERR_INVALID_ARG, "bad sizes");
+  if (!ids || !dy || !d_table || !workspace)
+    return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (workspace_bytes < sbp_embedding_backward_workspace_size(rows, vocab))
+    return fail(SBP_ERR_WORKSPACE, "workspace too small");
+  SBP_CK(embed_bwd(rows, cols, vocab, ids, dy, d_table, static_cast<int*>(workspace),
+                   static_cast<cudaStream_t>(stream)));
+  return SBP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+// Internal declarations shared by the libsbp translation units (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace sbp {
+
+enum Dt : int { DT_F32 = 0, DT_BF16 = 1 };
+
+inline size_t dt_size(int dt) { return dt == DT_BF16 ? 2 : 4; }
+__host__ __device__ __forceinline__ int64_t imin(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t imax(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Device status word kept in the first bytes of every workspace.
+enum : int { DEV_OK = 0, DEV_BAD_TARGET = 6, DEV_TIMEOUT = 5 };
+constexpr size_t kStatusBytes = 256;
+
+// ---------------------------------------------------------------------------------------------
+// scalar load/store helpers
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float ld_f(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void st_f(float* p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void st_f(__nv_bfloat16* p, int64_t i, float v) {
+  p[i] = __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ float ld_dt(const void* p, int dt, int64_t i) {
+  return dt == DT_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i])
+                       : static_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void st_dt(void* p, int dt, int64_t i, float v) {
+  if (dt == DT_BF16)
+    static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else
+    static_cast<float*>(p)[i] = v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ---------------------------------------------------------------------------------------------
+// GEMM:  C[m, n] (op)= alpha * sum_k A(m, k) * B(k, n)  with element strides
+//   A(m, k) = A[m * sam + k * sak],  B(k, n) = B[k * sbk + n * sbn],  C row-major (ldc).
+// Epilogues:
+//   EPI_STORE  : C = alpha * acc (+ bias[n])
+//   EPI_ACC    : C += alpha * acc (+ bias[n])
+//   EPI_LSE    : per row and column tile, partial max / sum-exp of acc over the tile's columns
+//                (pmax/psum[m * pld + tile]); zy[m] = acc at column tgt[m] - col0 if in tile.
+//   EPI_CEGRAD : C = wt[m] * (exp(acc - lse[m]) - [col0 + n == tgt[m]])  (cross-entropy
+//                gradient of the logits), stored in the C dtype.
+// dynM / dynK (nullable) give the true M / K on the device (<= the static M / K).
+// crow (nullable) maps row m of the result to row crow[m] of C.
+// ---------------------------------------------------------------------------------------------
+enum Epi : int { EPI_STORE = 0, EPI_ACC = 1, EPI_LSE = 2, EPI_CEGRAD = 3 };
+
+struct GemmDesc {
+  int64_t M = 0, N = 0, K = 0;
+  const int* dynM = nullptr;
+  const int* dynK = nullptr;
+  int adt = DT_F32, bdt = DT_F32, cdt = DT_F32;
+  const void* A = nullptr;
+  int64_t sam = 0, sak = 0;
+  const void* B = nullptr;
+  int64_t sbk = 0, sbn = 0;
+  void* C = nullptr;
+  int64_t ldc = 0;
+  const int* crow = nullptr;
+  const void* bias = nullptr;
+  int bias_dt = DT_F32;
+  int epi = EPI_STORE;
+  float alpha = 1.f;
+  // cross-entropy epilogue parameters
+  const float* lse = nullptr;
+  const int* tgt = nullptr;
+  const float* wt = nullptr;
+  int64_t col0 = 0;
+  float* pmax = nullptr;
+  float* psum = nullptr;
+  int64_t pld = 0;
+  float* zy = nullptr;
+};
+
+// Number of column tiles the EPI_LSE epilogue writes per row (its partial buffers' width).
+int64_t gemm_lse_tiles(int64_t N);
+
+cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------------
+// element-wise / row kernels (elementwise.cu)
+// ---------------------------------------------------------------------------------------------
+// y = rmsnorm(x) * g ; rstd (nullable).  x dtype xdt, g/y dtype ydt.
+cudaError_t rmsnorm_fwd(int64_t rows, int64_t cols, int xdt, const void* x, int gdt,
+                        const void* g, int ydt, void* y, float* rstd, float eps,
+                        cudaStream_t st);
+// out = (base ? base : 0) + (accumulate ? out : 0) + rmsnorm_bwd(dy); dg += (deterministic).
+// partial: workspace of rmsnorm_bwd_partial_floats(cols) floats.
+size_t rmsnorm_bwd_partial_floats(int64_t cols);
+cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int gdt,
+                        const void* g, const float* rstd, const float* dy, const float* base,
+                        float* out, int accumulate, float* dg, float* partial, cudaStream_t st);
+// cos/sin tables [T, hd/2] fp32 from fp64 angles pos * theta^(-2j/hd).
+cudaError_t rope_table(int64_t T, int64_t hd, double theta, float* cosb, float* sinb,
+                       cudaStream_t st);
+// QKV post-processing of one chunk: qkv [R, dq + 2 dkv] fp32 (R = B * Tc rows, row r is token
+// s + r % Tc of sequence r / Tc) -> q [R, dq] (RoPE'd, dt), K/V prefix [B, T, dkv] (dt).
+cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int64_t Hkv,
+                     int64_t hd, const float* qkv, int dt, void* q, void* Kp, void* Vp,
+                     const float* cosb, const float* sinb, cudaStream_t st);
+// In-place inverse RoPE on x [R, heads, hd] fp32 with position(r) = s + r % Tc.
+cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd, float* x,
+                         const float* cosb, const float* sinb, cudaStream_t st);
+// dK prefix rows of chunk [s, s + Tc) for all sequences -> dst [B * Tc, dkv] fp32 with RoPE^-1.
+cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t heads,
+                            int64_t hd, const float* src, float* dst, const float* cosb,
+                            const float* sinb, cudaStream_t st);
+// m = silu(g) * u from gu [R, 2f] (g = cols [0, f), u = [f, 2f)), dtype dt.
+cudaError_t swiglu_fwd(int64_t R, int64_t f, int dt, const void* gu, void* m, cudaStream_t st);
+// dgu [R, 2f] (dt) from dm [R, f] fp32 and gu.
+cudaError_t swiglu_bwd(int64_t R, int64_t f, int dt, const void* gu, const float* dm, void* dgu,
+                       cudaStream_t st);
+// Row gather/scatter between [B, T, cols] and a chunk buffer [B * Tc, cols].
+cudaError_t gather_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
+                         const void* src, void* dst, cudaStream_t st);
+cudaError_t scatter_chunk_f32(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                              const float* src, float* dst, int accumulate, cudaStream_t st);
+cudaError_t scatter_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
+                          const void* src, void* dst, cudaStream_t st);
+// dst[c] += sum_r src[r, c] (deterministic; partial of colsum_partial_floats(cols) floats).
+size_t colsum_partial_floats(int64_t cols);
+cudaError_t colsum_acc(int64_t rows, int64_t cols, const float* src, float* dst, float* partial,
+                       cudaStream_t st);
+// y = x + z (dt out) with x dt, z fp32: used for residual outputs.
+cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int ydt, void* y,
+                         cudaStream_t st);
+cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st);
+
+// LM head helpers (lmhead.cu)
+// Stable compaction of chunk rows [s, e) with w != 0 (and a valid target) into idx[0..n),
+// count[0] = n; bad targets with w != 0 raise the device status.
+cudaError_t ce_compact(int64_t s, int64_t e, int64_t V, const int* tgt, const float* w,
+                       int* idx, int* count, int* status, cudaStream_t st);
+// hc[r] = h[idx[r]] (r < n), rows [n, Rmax) = 0; wc, yc likewise (0 / -1); zy = 0, lse = 0.
+cudaError_t ce_gather(int64_t Rmax, int64_t d, int dt, const void* h, const int* idx,
+                      const int* count, const int* tgt, const float* w, void* hc, int* yc,
+                      float* wc, float* zy, float* lse, cudaStream_t st);
+// lse[r] from partials; loss (= if first else +=) sum_r wc[r] (lse[r] - zy[r]).
+cudaError_t ce_finish(int64_t Rmax, int64_t tiles, const float* pmax, const float* psum,
+                      int64_t pld, const int* count, const float* wc, const float* zy,
+                      float* lse, float* row_loss, float* loss, int first, cudaStream_t st);
+// out rows idx[r] (r < n) of d_hidden chunk: zero rows [s, e) of dh first.
+cudaError_t zero_rows(int64_t s, int64_t e, int64_t d, float* dh, cudaStream_t st);
+
+// attention (attention.cu)
+// Forward for chunk queries q [B*Tc, H, hd] at positions s.. over prefix keys [0, s + Tc).
+cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
+                     int64_t hd, int dt, const void* q, const void* Kp, const void* Vp, void* o,
+                     float* lse, cudaStream_t st);
+// Backward: dq [B*Tc, H, hd] fp32 (overwritten); dKp/dVp [B, T, Hkv, hd] fp32 (+= rows < s+Tc).
+cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
+                     int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
+                     const void* o, const void* dO, const float* lse, float* delta, float* dq,
+                     float* dKp, float* dVp, cudaStream_t st);
+
+// embedding (elementwise.cu)
+cudaError_t embed_fwd(int64_t rows, int64_t cols, int64_t vocab, int dt, const int* ids,
+                      const void* table, void* y, cudaStream_t st);
+cudaError_t embed_bwd(int64_t rows, int64_t cols, int64_t vocab, const int* ids, const float* dy,
+                      float* dtable, int* ws, cudaStream_t st);
+size_t embed_bwd_ws_ints(int64_t rows, int64_t vocab);
+
+}  // namespace sbp

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI (no kernel launch): the library loads, exports every symbol
+that include/sbp.h declares, and rejects bad arguments before queueing any work."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from memory_efficient_exact_chunk_b200 import build as sbp_build
+from memory_efficient_exact_chunk_b200 import sbp
+from oracle import sbp_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x100000  # an aligned address that is never dereferenced (argument checks fail first)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sbp_build.build()
+    return sbp.load()
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "sbp.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbp_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = header_symbols()
+    assert "sbp_lmhead_ce_backward_stream" in syms and "sbp_decoder_layer_backward_stream" in syms
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) <= set(sbp.EXPORTS) | set(syms)
+    assert lib.sbp_version().decode().startswith("sbp")
+
+
+def test_chunk_bounds_matches_oracle(lib):
+    for T in (1, 7, 10, 256, 32768, 65536):
+        for D in (1, 2, 3, 7, 8, 16):
+            if D > T:
+                with pytest.raises(sbp.SbpError):
+                    sbp.chunk_bounds(T, D)
+                continue
+            assert sbp.chunk_bounds(T, D) == O.chunk_bounds(T, D)
+
+
+def test_workspace_sizes(lib):
+    assert sbp.lmhead_ce_workspace_size(1024, 64, 1000, 4, sbp.SBP_BF16) > 0
+    assert sbp.lmhead_ce_workspace_size(1024, 64, 1000, 0, sbp.SBP_BF16) == 0
+    assert sbp.lmhead_ce_workspace_size(4, 64, 1000, 5, sbp.SBP_BF16) == 0
+    cfg = sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 4)
+    w4 = sbp.layer_workspace_size(cfg)
+    assert w4 > 0
+    cfg1 = sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 1)
+    assert sbp.layer_workspace_size(cfg1) > w4          # per-chunk buffers scale with T / D
+    bad = sbp.layer_cfg(1, 256, 64, 4, 3, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 4)
+    assert sbp.layer_workspace_size(bad) == 0
+
+
+def _lm_call(lib, **kw):
+    a = dict(N=64, d=64, V=100, D=2, dt=sbp.SBP_F32, h=FAKE, W=FAKE, y=FAKE, w=FAKE, loss=FAKE,
+             dH=FAKE, dW=FAKE, ws=FAKE, wsb=1 << 40)
+    a.update(kw)
+    return lib.sbp_lmhead_ce_backward_stream(a["N"], a["d"], a["V"], a["D"], a["dt"], a["h"],
+                                             a["W"], a["y"], a["w"], a["loss"], a["dH"], a["dW"],
+                                             a["ws"], a["wsb"], None)
+
+
+def test_lmhead_argument_errors(lib):
+    assert _lm_call(lib, h=None) == 1
+    assert _lm_call(lib, dW=None) == 1
+    assert _lm_call(lib, D=0) == 1
+    assert _lm_call(lib, D=65) == 1
+    assert _lm_call(lib, N=0) == 1
+    assert _lm_call(lib, dt=7) == 1
+    assert _lm_call(lib, h=FAKE + 4) == 1                      # misaligned
+    assert _lm_call(lib, dt=sbp.SBP_BF16, d=60) == 2            # unsupported width
+    assert _lm_call(lib, wsb=16) == 3                            # workspace too small
+    assert _lm_call(lib, ws=FAKE + 16) == 1                      # workspace misaligned
+    assert "workspace" in lib.sbp_last_error().decode()
+
+
+def test_layer_argument_errors(lib):
+    cfg = sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 4)
+    names = sbp.WEIGHT_FIELDS
+    w = sbp.LayerWeights(**{n: (FAKE if n not in ("bq", "bk", "bv") else None) for n in names})
+    g = sbp.LayerGrads(**{n: (FAKE if n not in ("bq", "bk", "bv") else None) for n in names})
+
+    def call(c=cfg, w=w, g=g, x=FAKE, dy=FAKE, dx=FAKE, ws=FAKE, wsb=1 << 40):
+        return lib.sbp_decoder_layer_backward_stream(C.byref(c), C.byref(w), x, dy, dx,
+                                                     C.byref(g), ws, wsb, None)
+
+    assert call(x=None) == 1
+    assert call(wsb=1024) == 3
+    bad = sbp.layer_cfg(1, 256, 64, 4, 3, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 4)
+    assert call(c=bad) == 1                                      # n_heads % n_kv_heads
+    assert call(c=sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 257)) == 1
+    assert call(c=sbp.layer_cfg(1, 256, 64, 4, 4, 15, 172, 1e-6, 1e4, sbp.SBP_F32, 4)) == 2
+    assert call(c=sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_BF16, 4)) == 2
+    wb = sbp.LayerWeights(**{n: FAKE for n in names})
+    assert call(w=wb) == 1                                        # biases without bias grads
+    w1 = sbp.LayerWeights(**{n: (FAKE if n != "bk" else None) for n in names})
+    assert call(w=w1) == 1                                        # partial bias set

@@ -1,0 +1,106 @@
+"""GPU parity of sbp_decoder_layer_backward_stream (and the chunked forward) against the fp64
+oracle, through the C ABI.  Tolerances: relative Frobenius 1e-5 (fp32), 1e-2 (bf16) per
+tensor; D = 1 vs D > 1 within 1e-5."""
+import numpy as np
+import pytest
+
+from oracle import sbp_oracle as O
+from memory_efficient_exact_chunk_b200 import synth
+from tests.helpers import f64, oracle_cfg, rel_fro, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 1e-2}
+NAMES = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up", "w_down")
+
+
+def _gpu_layer(L, W, x, dy, D, dtype, forward=False):
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    B, T, d = x.shape
+    code = sbp.SBP_BF16 if dtype == "bf16" else sbp.SBP_F32
+    cfg = sbp.layer_cfg(B, T, d, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn, L.rms_eps,
+                        L.rope_theta, code, D)
+    Wd = {n: (to_dev(W[n], dtype) if W.get(n) is not None else None) for n in NAMES}
+    xd = to_dev(x, dtype)
+    if forward:
+        y = torch.full(xd.shape, float("nan"), dtype=xd.dtype, device="cuda")
+        sbp.decoder_layer_forward(cfg, Wd, xd, y)
+        torch.cuda.synchronize()
+        return to_np(y)
+    dyd = to_dev(dy, "f32")
+    dx = torch.full((B, T, d), float("nan"), device="cuda")
+    g = {n: (torch.zeros(W[n].shape, device="cuda") if W.get(n) is not None else None)
+         for n in NAMES}
+    ws = sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, g)
+    sbp.device_status(ws)
+    torch.cuda.synchronize()
+    return to_np(dx), {n: to_np(v) for n, v in g.items() if v is not None}
+
+
+def _oracle(L, W, x, dy):
+    cfg = oracle_cfg(O, L)
+    W64 = {n: f64(W.get(n)) for n in NAMES}
+    return O.decoder_layer_backward(cfg, W64, f64(x), f64(dy))
+
+
+def _check(L, W, x, dy, D, dtype, tol=None):
+    tol = tol or TOL[dtype]
+    dx, g = _gpu_layer(L, W, x, dy, D, dtype)
+    dx0, g0 = _oracle(L, W, x, dy)
+    errs = {"dx": rel_fro(dx, dx0)}
+    for n in g:
+        errs[n] = rel_fro(g[n], g0[n])
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (errs, tol)
+    return dx, g
+
+
+TINY = synth.LayerShape(64, 4, 4, 16, 172, 1e-6, 10000.0)           # the fp32 tiny model
+GQA = synth.LayerShape(128, 4, 2, 32, 200, 1e-5, 500000.0)
+QWEN_LIKE = synth.LayerShape(128, 4, 1, 32, 160, 1e-6, 1e6, qkv_bias=True)
+
+
+@pytest.mark.parametrize("D", [1, 4, 5])
+def test_layer_fp32_tiny(D):
+    W, x, dy = synth.layer_inputs(0, TINY, 1, 256, bf16=False, dy_std=1.0)
+    _check(TINY, W, x, dy, D, "f32")
+
+
+@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 200, 3), (QWEN_LIKE, 1, 256, 4)])
+def test_layer_fp32_gqa_bias_ragged(L, B, T, D):
+    W, x, dy = synth.layer_inputs(1, L, B, T, bf16=False, dy_std=1.0, gamma_std=0.1)
+    _check(L, W, x, dy, D, "f32")
+
+
+@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 256, 4), (QWEN_LIKE, 2, 384, 3)])
+def test_layer_bf16(L, B, T, D):
+    W, x, dy = synth.layer_inputs(2, L, B, T, bf16=True, dy_std=1e-3, gamma_std=0.1)
+    _check(L, W, x, dy, D, "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layer_d_invariance(dtype):
+    L = GQA
+    W, x, dy = synth.layer_inputs(3, L, 2, 512, bf16=(dtype == "bf16"), dy_std=1e-3)
+    dx1, g1 = _gpu_layer(L, W, x, dy, 1, dtype)
+    for D in (2, 4, 8):
+        dxD, gD = _gpu_layer(L, W, x, dy, D, dtype)
+        assert rel_fro(dxD, dx1) <= 1e-5, D
+        for n in g1:
+            assert rel_fro(gD[n], g1[n]) <= 1e-5, (D, n, rel_fro(gD[n], g1[n]))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layer_forward(dtype):
+    L = QWEN_LIKE
+    W, x, _ = synth.layer_inputs(4, L, 2, 256, bf16=(dtype == "bf16"))
+    y = _gpu_layer(L, W, x, None, 4, dtype, forward=True)
+    y0 = O.decoder_layer_forward(oracle_cfg(O, L), {n: f64(W.get(n)) for n in NAMES}, f64(x))
+    assert rel_fro(y, y0) <= (1e-6 if dtype == "f32" else 4e-3)
+
+
+def test_layer_llama_width_reduced_t():
+    """Llama-3-8B layer widths (d 4096, 32/8 heads of 128, MLP 14336) on T = 256, D = 2."""
+    W, x, dy = synth.layer_inputs(5, synth.LLAMA3_8B, 1, 256, bf16=True, dy_std=1e-3)
+    _check(synth.LLAMA3_8B, W, x, dy, 2, "bf16")
