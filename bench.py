@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the streamed exact backward (StreamBP) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sbp|reference]
+                    [--workload lmhead_ce_32k|llama3_8b_layer_32k] [--chunks D] [--no-sweep]
+
+Default workload: the chunked LM-head + cross-entropy backward of a 32K-token SFT sequence
+(hidden 3584 = an RMSNorm output ~ N(0,1), vocabulary 152064, weight ~ N(0, 0.02), uniform
+targets, first 30 % of tokens loss-masked), bf16 operands with fp32 accumulation, D = 8.
+One step = one call of sbp_lmhead_ce_backward_stream over the whole sequence (all chunks).
+Inputs are resident in HBM and larger than L2 (the 1.09 GB LM-head weight is streamed by
+every chunk), so no explicit L2 flush is used.  Prints ONE JSON line on rank 0.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own independent sequence
+(weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "streamed backward tokens/s (1 B200) vs D; tensor-pipe % of peak; peak act. GB"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for ln in fh:
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+def lmhead_workload(T):
+    from memory_efficient_exact_chunk_b200 import synth
+    wl = synth.WORKLOADS["lmhead_ce_32k"]
+    return wl, T or wl.seq_len
+
+
+def traffic_from_profiles(kernel_src: str, workload: str):
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, if the kernel source has
+    not changed since (the summary stores a hash of the kernel's source file)."""
+    path = os.path.join(ROOT, "profiles", f"{workload}_gemm_tc.md")
+    src = os.path.join(ROOT, "memory_efficient_exact_chunk_b200", "csrc", kernel_src)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    txt = open(path).read()
+    mh = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", txt)
+    mb = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", txt)
+    if not (mh and mb) or mh.group(1) != h:
+        return None
+    return float(mb.group(1))
+
+
+def run_lmhead(args, rank, world, device):
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp, synth
+    wl = synth.WORKLOADS["lmhead_ce_32k"]
+    T, d, V = wl.seq_len, wl.hidden, wl.vocab
+    D = args.chunks or wl.num_chunks
+    h, W, y, w = synth.lmhead_inputs(1000 + rank, T, d, V, bf16=True, from_frac=wl.loss_from_frac)
+    n_valid = int(np.count_nonzero(w))
+    hd = torch.from_numpy(h).to(torch.bfloat16).to(device)
+    Wd = torch.from_numpy(W).to(torch.bfloat16).to(device)
+    del W
+    yd = torch.from_numpy(y).to(device)
+    wd = torch.from_numpy(w).to(device)
+    loss = torch.zeros(1, device=device)
+    dH = torch.empty(T, d, device=device)
+    dW = torch.zeros(V, d, device=device)
+    torch.cuda.synchronize()
+    resident = torch.cuda.memory_allocated(device)
+
+    def make_ws(Dc):
+        return sbp.workspace(sbp.lmhead_ce_workspace_size(T, d, V, Dc, sbp.SBP_BF16), device)
+
+    ws = make_ws(D)
+    step = lambda: sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW, ws=ws)
+    flops_step = 8.0 * n_valid * d * V          # executed design: lse pass + 3 products
+    flops_min = 6.0 * n_valid * d * V           # logits + dH + dW
+    res = timed(args, step, world, device, profile=True)
+    sbp.device_status(ws)
+    torch.cuda.reset_peak_memory_stats(device)
+    step()
+    torch.cuda.synchronize()
+    peak_alloc = torch.cuda.max_memory_allocated(device)
+    out = {
+        "tokens_per_step": T, "n_loss_tokens": n_valid, "flops_step": flops_step,
+        "flops_min_step": flops_min, "res": res, "ws_bytes": ws.numel(),
+        "peak_act_gb": (peak_alloc - resident) / 1e9, "D": D,
+        "config": {"workload": "lmhead_ce_32k", "batch": 1, "seq_len": T, "hidden": d,
+                   "vocab": V, "num_chunks": D, "loss_mask": "first 30% of tokens",
+                   "n_loss_tokens": n_valid,
+                   "l2": "inputs larger than L2 (1.09 GB LM-head weight re-read per chunk)"},
+    }
+    # ---- D sweep (tokens/s and workspace vs D)
+    if args.sweep and rank == 0 and world == 1:
+        sweep = []
+        for Dc in (1, 2, 4, 8, 16):
+            wsc = make_ws(Dc)
+            stepc = lambda: sbp.lmhead_ce_backward(hd, Wd, yd, wd, Dc, loss, dH, dW, ws=wsc)
+            r = timed(argparse.Namespace(steps=2, warmup=1), stepc, 1, device, profile=False)
+            sweep.append({"D": Dc, "tokens_per_s": T / (r["ms"] / 1e3),
+                          "ms_per_step": r["ms"], "workspace_gb": wsc.numel() / 1e9})
+            del wsc
+        out["sweep"] = sweep
+    # ---- end to end through the C ABI from pinned host buffers
+    if args.e2e:
+        hh = torch.from_numpy(h).to(torch.bfloat16).pin_memory()
+        yh = torch.from_numpy(y).pin_memory()
+        wh = torch.from_numpy(w).pin_memory()
+        lh = torch.zeros(1).pin_memory()
+        stream = torch.cuda.current_stream(device)
+
+        def e2e_step():
+            hd.copy_(hh, non_blocking=True)
+            yd.copy_(yh, non_blocking=True)
+            wd.copy_(wh, non_blocking=True)
+            sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW, ws=ws, stream=stream)
+            lh.copy_(loss, non_blocking=True)
+
+        r = timed(args, e2e_step, world, device, profile=False)
+        out["e2e"] = {"value": T * world / (r["ms"] / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": hh.numel() * 2 + yh.numel() * 4 + wh.numel() * 4,
+                      "d2h_bytes_per_step": 4}
+    return out
+
+
+def timed(args, step, world, device, profile):
+    """W warm-up steps, then K timed steps between a barrier + synchronize on both sides;
+    device time from CUDA events on the launching stream, max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from memory_efficient_exact_chunk_b200 import sbp
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    clk = ClockSampler(device.index or 0) if profile else None
+    if clk:
+        clk.start()
+        time.sleep(0.3)
+    n0 = sbp.launch_count()
+    if profile:
+        sbp.profile_begin()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize(device)
+    prof = sbp.profile_end() if profile else None
+    launches = sbp.launch_count() - n0
+    clocks = clk.stop() if clk else None
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+        dist.barrier()
+    return {"ms_total": ms, "ms": ms / args.steps, "prof": prof, "launches": launches,
+            "clocks": clocks}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_lmhead_sample(n_rows: int, seed: int = 5):
+    """The fp64 oracle on n_rows rows of the 32K workload's shapes (full hidden / vocab)."""
+    from memory_efficient_exact_chunk_b200 import synth
+    from oracle import sbp_oracle as O
+    wl = synth.WORKLOADS["lmhead_ce_32k"]
+    h, W, y, w = synth.lmhead_inputs(seed, n_rows, wl.hidden, wl.vocab, bf16=True, from_frac=0.0)
+    t0 = time.perf_counter()
+    O.lmhead_ce_forward_backward(h, W, y, w)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(n_rows=48):
+    dt = oracle_lmhead_sample(n_rows)
+    return {"value": n_rows / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n_rows} loss tokens of the 32K LM-head workload (hidden 3584, vocab "
+                      f"152064), fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    n_rows = 16
+    oracle_lmhead_sample(4)                       # warm the BLAS threads
+    for _ in range(args.warmup):
+        oracle_lmhead_sample(n_rows)
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_lmhead_sample(n_rows)
+    value = n_rows * args.steps / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "lmhead_ce_32k", "batch": 1, "seq_len": 32768, "hidden": 3584,
+                   "vocab": 152064, "num_chunks": 8},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                         "kind": "oracle",
+                         "sample": f"{n_rows} loss tokens per step of the 32K LM-head workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sbp", choices=["sbp", "reference"])
+    ap.add_argument("--workload", default="lmhead_ce_32k", choices=["lmhead_ce_32k"])
+    ap.add_argument("--chunks", type=int, default=0)
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from memory_efficient_exact_chunk_b200 import sbp
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    sbp.load()
+    out = run_lmhead(args, rank, world, device)
+    res = out["res"]
+    peaks, peak_src = load_peaks()
+    prof = res["prof"]["gemm_tc"]
+    tc_ms = prof["ms"]
+    n_l = max(prof["launches"], 1)
+    achieved = (out["flops_step"] * args.steps) / (tc_ms / 1e3) / 1e12 if tc_ms > 0 else 0.0
+    peak = float(peaks["bf16_tflops_sustained"])
+    traffic = traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k")
+    line = {
+        "metric": METRIC,
+        "value": out["tokens_per_step"] * world / (res["ms"] / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": out["config"],
+        "roofline": {
+            "bound": "tensor", "kernel": "gemm_tc_kernel (tcgen05, all GEMM launches of a step)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak if peak else None,
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "flops_per_launch": out["flops_step"] / (n_l / args.steps),
+            "launch_ms": tc_ms / n_l, "launches_per_step": n_l / args.steps,
+            "share_of_step": tc_ms / res["ms_total"] if res["ms_total"] else None,
+            "achieved_min_flops": (out["flops_min_step"] * args.steps) / (tc_ms / 1e3) / 1e12
+            if tc_ms > 0 else 0.0,
+            "traffic": traffic,
+        },
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+        "peak_act_gb": out["peak_act_gb"],
+        "workspace_gb": out["ws_bytes"] / 1e9,
+    }
+    if "sweep" in out:
+        line["sweep"] = out["sweep"]
+    if "e2e" in out:
+        line["e2e"] = out["e2e"]
+    if args.cpu and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,36 @@
+/*
+ * sbp_debug.h -- test hooks of libsbp (not part of the streamed-backward API).
+ *
+ * The paper has no counterpart: these calls exist so that the tests can check a single
+ * building block of the library (the GEMM engine) against a reference, path by path.
+ */
+#ifndef SBP_DEBUG_H_
+#define SBP_DEBUG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sbp.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * C[m, n] (+)= sum_k op(A)[m, k] * op(B)[k, n] with bf16 A and B and fp32 C, all row-major:
+ *   a_trans = 0: A is [M, K] with leading dimension lda;  1: A is [K, M] (op(A) = A^T)
+ *   b_trans = 0: B is [K, N] with leading dimension ldb;  1: B is [N, K] (op(B) = B^T)
+ * C is [M, N] with leading dimension ldc; accumulate = 0 overwrites, 1 adds.
+ * path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores (SBP_ERR_UNSUPPORTED if the layout is
+ * not one the tensor-core kernel takes).  `workspace` (>= 256 bytes, device) receives the
+ * device status word (see sbp_get_device_status).  Device pointers, queued on `stream`.
+ */
+sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int a_trans,
+                               int64_t lda, const void* B, int b_trans, int64_t ldb, float* C,
+                               int64_t ldc, int accumulate, int path, void* workspace,
+                               void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SBP_DEBUG_H_ */

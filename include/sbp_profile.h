@@ -1,0 +1,37 @@
+/*
+ * sbp_profile.h -- launch accounting and GEMM timing of libsbp (instrumentation; the paper
+ * has no counterpart).
+ *
+ * While profiling is on, every GEMM the library queues is bracketed by two CUDA events on its
+ * own stream, so that a caller can read the device time of the dominant kernels of a timed
+ * region.  Profiling is process-wide and off by default.
+ */
+#ifndef SBP_PROFILE_H_
+#define SBP_PROFILE_H_
+
+#include "sbp.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { SBP_PROF_GEMM_TC = 0, SBP_PROF_GEMM_SIMT = 1, SBP_PROF_KINDS = 2 };
+
+typedef struct {
+  long long launches[SBP_PROF_KINDS]; /* launches per kind (tensor-core GEMM, CUDA-core GEMM) */
+  double ms[SBP_PROF_KINDS];          /* summed device time per kind, milliseconds            */
+} sbp_profile;
+
+/* Number of kernels the library has launched in this process (all kinds). */
+long long sbp_launch_count(void);
+
+/* Start recording GEMM launches (clears earlier records). */
+sbp_status sbp_profile_begin(void);
+
+/* Stop recording, synchronise on the recorded events and fill `out` (may be NULL). */
+sbp_status sbp_profile_end(sbp_profile* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SBP_PROFILE_H_ */

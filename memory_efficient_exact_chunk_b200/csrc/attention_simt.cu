@@ -182,11 +182,11 @@ cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int
   const int64_t w = B * Tc * H;
   if (w <= 0) return cudaSuccess;
   if (dt == DT_BF16)
-    attn_fwd_kernel<__nv_bfloat16><<<warps_blocks(w), 256, 0, st>>>(
+    launch(attn_fwd_kernel<__nv_bfloat16>, warps_blocks(w), 256, 0, st, 
         B, T, Tc, s, H, Hkv, (int)hd, (const __nv_bfloat16*)q, (const __nv_bfloat16*)Kp,
         (const __nv_bfloat16*)Vp, (__nv_bfloat16*)o, lse);
   else
-    attn_fwd_kernel<float><<<warps_blocks(w), 256, 0, st>>>(
+    launch(attn_fwd_kernel<float>, warps_blocks(w), 256, 0, st, 
         B, T, Tc, s, H, Hkv, (int)hd, (const float*)q, (const float*)Kp, (const float*)Vp,
         (float*)o, lse);
   return cudaGetLastError();
@@ -199,10 +199,10 @@ static void attn_bwd_launch(int64_t B, int64_t Tn, int64_t Tc, int64_t s, int64_
                             float* dq, float* dKp, float* dVp, cudaStream_t st) {
   const int64_t w = B * Tc * H;
   const int64_t w2 = B * (s + Tc) * Hkv;
-  attn_bwd_dq_kernel<T><<<warps_blocks(w), 256, 0, st>>>(
+  launch(attn_bwd_dq_kernel<T>, warps_blocks(w), 256, 0, st, 
       B, Tn, Tc, s, H, Hkv, (int)hd, (const T*)q, (const T*)Kp, (const T*)Vp, (const T*)o,
       (const T*)dO, lse, delta, dq);
-  attn_bwd_dkv_kernel<T><<<warps_blocks(w2), 256, 0, st>>>(
+  launch(attn_bwd_dkv_kernel<T>, warps_blocks(w2), 256, 0, st, 
       B, Tn, Tc, s, H, Hkv, (int)hd, (const T*)q, (const T*)Kp, (const T*)Vp, (const T*)dO, lse,
       delta, dKp, dVp);
 }

@@ -252,6 +252,18 @@ __global__ void add_residual_kernel(int64_t n, int xdt, const void* __restrict__
   st_dt(y, ydt, i, ld_dt(x, xdt, i) + z[i]);
 }
 
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi): a 16-bit-mantissa operand for the tensor
+// cores, used where a value's fp32 rounding depends on the chunking (the fp32 dK/dV sums)
+__global__ void split_bf16_kernel(int64_t n, const float* __restrict__ x,
+                                  __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = x[i];
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[i] = h;
+  lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
 __global__ void copy_cast_kernel(int64_t n, int sdt, const void* __restrict__ src, int ddt,
                                  void* __restrict__ dst) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -354,7 +366,7 @@ cudaError_t rmsnorm_fwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
                         const void* g, int ydt, void* y, float* rstd, float eps,
                         cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  rmsnorm_fwd_kernel<<<(unsigned)rows, kRowThreads, 0, st>>>(cols, xdt, x, gdt, g, ydt, y, rstd,
+  launch(rmsnorm_fwd_kernel, (unsigned)rows, kRowThreads, 0, st, cols, xdt, x, gdt, g, ydt, y, rstd,
                                                              eps);
   return cudaGetLastError();
 }
@@ -372,12 +384,12 @@ cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  rmsnorm_bwd_kernel<<<kBwdBlocks, kRowThreads, smem, st>>>(rows, cols, xdt, x, gdt, g, rstd, dy,
+  launch(rmsnorm_bwd_kernel, kBwdBlocks, kRowThreads, smem, st, rows, cols, xdt, x, gdt, g, rstd, dy,
                                                             base, out, accumulate, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (dg) {
-    colsum_partials_kernel<<<nblk(cols, 256), 256, 0, st>>>(kBwdBlocks, cols, partial, dg);
+    launch(colsum_partials_kernel, nblk(cols, 256), 256, 0, st, kBwdBlocks, cols, partial, dg);
     e = cudaGetLastError();
   }
   return e;
@@ -387,7 +399,7 @@ cudaError_t rope_table(int64_t T, int64_t hd, double theta, float* cosb, float* 
                        cudaStream_t st) {
   const int64_t n = T * (hd / 2);
   if (n <= 0) return cudaSuccess;
-  rope_table_kernel<<<nblk(n, 256), 256, 0, st>>>(T, hd / 2, theta, cosb, sinb);
+  launch(rope_table_kernel, nblk(n, 256), 256, 0, st, T, hd / 2, theta, cosb, sinb);
   return cudaGetLastError();
 }
 
@@ -396,7 +408,7 @@ cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int
                      const float* cosb, const float* sinb, cudaStream_t st) {
   const int64_t n = R * (H + 2 * Hkv) * (hd / 2);
   if (n <= 0) return cudaSuccess;
-  qkv_post_kernel<<<nblk(n, 256), 256, 0, st>>>(R, Tc, s, T, H, Hkv, hd, qkv, dt, q, Kp, Vp,
+  launch(qkv_post_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, T, H, Hkv, hd, qkv, dt, q, Kp, Vp,
                                                 cosb, sinb);
   return cudaGetLastError();
 }
@@ -405,7 +417,7 @@ cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_
                          const float* cosb, const float* sinb, cudaStream_t st) {
   const int64_t n = R * heads * (hd / 2);
   if (n <= 0) return cudaSuccess;
-  rope_inv_kernel<<<nblk(n, 256), 256, 0, st>>>(R, Tc, s, heads, hd, x, cosb, sinb);
+  launch(rope_inv_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, heads, hd, x, cosb, sinb);
   return cudaGetLastError();
 }
 
@@ -414,21 +426,21 @@ cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t
                             const float* sinb, cudaStream_t st) {
   const int64_t n = B * Tc * heads * (hd / 2);
   if (n <= 0) return cudaSuccess;
-  gather_rope_inv_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, heads, hd, src, dst, cosb,
+  launch(gather_rope_inv_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, heads, hd, src, dst, cosb,
                                                        sinb);
   return cudaGetLastError();
 }
 
 cudaError_t swiglu_fwd(int64_t R, int64_t f, int dt, const void* gu, void* m, cudaStream_t st) {
   if (R * f <= 0) return cudaSuccess;
-  swiglu_fwd_kernel<<<nblk(R * f, 256), 256, 0, st>>>(R, f, dt, gu, m);
+  launch(swiglu_fwd_kernel, nblk(R * f, 256), 256, 0, st, R, f, dt, gu, m);
   return cudaGetLastError();
 }
 
 cudaError_t swiglu_bwd(int64_t R, int64_t f, int dt, const void* gu, const float* dm, void* dgu,
                        cudaStream_t st) {
   if (R * f <= 0) return cudaSuccess;
-  swiglu_bwd_kernel<<<nblk(R * f, 256), 256, 0, st>>>(R, f, dt, gu, dm, dgu);
+  launch(swiglu_bwd_kernel, nblk(R * f, 256), 256, 0, st, R, f, dt, gu, dm, dgu);
   return cudaGetLastError();
 }
 
@@ -436,7 +448,7 @@ cudaError_t gather_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t co
                          const void* src, void* dst, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
-  gather_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, dt, src, dst);
+  launch(gather_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, dt, src, dst);
   return cudaGetLastError();
 }
 
@@ -444,7 +456,7 @@ cudaError_t scatter_chunk_f32(int64_t B, int64_t T, int64_t Tc, int64_t s, int64
                               const float* src, float* dst, int accumulate, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
-  scatter_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, DT_F32, src, dst,
+  launch(scatter_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, DT_F32, src, dst,
                                                      accumulate);
   return cudaGetLastError();
 }
@@ -453,7 +465,7 @@ cudaError_t scatter_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t c
                           const void* src, void* dst, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
-  scatter_chunk_kernel<<<nblk(n, 256), 256, 0, st>>>(B, T, Tc, s, cols, dt, src, dst, 0);
+  launch(scatter_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, dt, src, dst, 0);
   return cudaGetLastError();
 }
 
@@ -463,28 +475,35 @@ cudaError_t colsum_acc(int64_t rows, int64_t cols, const float* src, float* dst,
                        cudaStream_t st) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   dim3 g1(kColsumParts, nblk(cols, 256));
-  colsum_stage1_kernel<<<g1, 256, 0, st>>>(rows, cols, src, partial);
-  colsum_partials_kernel<<<nblk(cols, 256), 256, 0, st>>>(kColsumParts, cols, partial, dst);
+  launch(colsum_stage1_kernel, g1, 256, 0, st, rows, cols, src, partial);
+  launch(colsum_partials_kernel, nblk(cols, 256), 256, 0, st, kColsumParts, cols, partial, dst);
   return cudaGetLastError();
 }
 
 cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int ydt, void* y,
                          cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  add_residual_kernel<<<nblk(n, 256), 256, 0, st>>>(n, xdt, x, z, ydt, y);
+  launch(add_residual_kernel, nblk(n, 256), 256, 0, st, n, xdt, x, z, ydt, y);
+  return cudaGetLastError();
+}
+
+cudaError_t split_bf16(int64_t n, const float* x, void* hi, void* lo, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  launch(split_bf16_kernel, nblk(n, 256), 256, 0, st, n, x, static_cast<__nv_bfloat16*>(hi),
+                                                  static_cast<__nv_bfloat16*>(lo));
   return cudaGetLastError();
 }
 
 cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  copy_cast_kernel<<<nblk(n, 256), 256, 0, st>>>(n, sdt, src, ddt, dst);
+  launch(copy_cast_kernel, nblk(n, 256), 256, 0, st, n, sdt, src, ddt, dst);
   return cudaGetLastError();
 }
 
 cudaError_t embed_fwd(int64_t rows, int64_t cols, int64_t vocab, int dt, const int* ids,
                       const void* table, void* y, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  embed_fwd_kernel<<<(unsigned)rows, 256, 0, st>>>(rows, cols, vocab, dt, ids, table, y);
+  launch(embed_fwd_kernel, (unsigned)rows, 256, 0, st, rows, cols, vocab, dt, ids, table, y);
   return cudaGetLastError();
 }
 
@@ -499,12 +518,12 @@ cudaError_t embed_bwd(int64_t rows, int64_t cols, int64_t vocab, const int* ids,
   int* order = ws + 3 * vocab;
   cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int) * vocab, st);
   if (e != cudaSuccess) return e;
-  embed_count_kernel<<<nblk(rows, 256), 256, 0, st>>>(rows, vocab, ids, cnt);
-  scan_kernel<<<1, 1024, 0, st>>>(vocab, cnt, off);
+  launch(embed_count_kernel, nblk(rows, 256), 256, 0, st, rows, vocab, ids, cnt);
+  launch(scan_kernel, 1, 1024, 0, st, vocab, cnt, off);
   e = cudaMemcpyAsync(pos, off, sizeof(int) * vocab, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return e;
-  embed_place_kernel<<<nblk(rows, 256), 256, 0, st>>>(rows, vocab, ids, pos, order);
-  embed_accum_kernel<<<(unsigned)vocab, 128, 0, st>>>(rows, cols, ids, off, cnt, order, dy,
+  launch(embed_place_kernel, nblk(rows, 256), 256, 0, st, rows, vocab, ids, pos, order);
+  launch(embed_accum_kernel, (unsigned)vocab, 128, 0, st, rows, cols, ids, off, cnt, order, dy,
                                                        dtable);
   return cudaGetLastError();
 }

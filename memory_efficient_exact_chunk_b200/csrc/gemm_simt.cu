@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
   const int64_t N = g.N;
   const int64_t m0 = (int64_t)blockIdx.y * BM;
   const int64_t n0 = (int64_t)blockIdx.x * BN;
-  if (m0 >= M) return;
+  if (m0 >= (g.epi == EPI_CEGRAD ? g.M : M)) return;
 
   const TA* A = static_cast<const TA*>(g.A);
   const TB* B = static_cast<const TB*>(g.B);
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t m = m0 + ty + 16 * i;
-      if (m >= M) continue;
+      if (m >= g.M) continue;
       const float w = g.wt[m];
       const float l = g.lse[m];
       const int y = g.tgt[m];
@@ -143,13 +143,13 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t st) {
   dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + BM - 1) / BM));
   if (grid.y > 65535u) return cudaErrorInvalidValue;
   if (g.adt == DT_F32 && g.bdt == DT_F32)
-    gemm_simt_kernel<float, float><<<grid, 256, 0, st>>>(g);
+    launch(gemm_simt_kernel<float, float>, grid, 256, 0, st, g);
   else if (g.adt == DT_BF16 && g.bdt == DT_BF16)
-    gemm_simt_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(g);
+    launch(gemm_simt_kernel<__nv_bfloat16, __nv_bfloat16>, grid, 256, 0, st, g);
   else if (g.adt == DT_F32 && g.bdt == DT_BF16)
-    gemm_simt_kernel<float, __nv_bfloat16><<<grid, 256, 0, st>>>(g);
+    launch(gemm_simt_kernel<float, __nv_bfloat16>, grid, 256, 0, st, g);
   else
-    gemm_simt_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(g);
+    launch(gemm_simt_kernel<__nv_bfloat16, float>, grid, 256, 0, st, g);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,449 @@
+// Persistent bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+//   C[m, n] (op)= sum_k A(m, k) B(k, n),   A, B bf16 in either K-major or MN-major layout,
+//   fp32 accumulation in TMEM, fused epilogues (store / accumulate fp32 or bf16, column bias,
+//   row remap, cross-entropy log-sum-exp partials, cross-entropy logit gradient).
+//
+// CTA tile 128 x 256 x 64, 4-stage TMA -> shared-memory ring, warp-specialised:
+//   warp 0      : TMA producer (one lane)
+//   warp 1      : TMEM allocator + MMA issuer (one lane), M=128 N=256 K=16 instructions
+//   warps 2..5  : epilogue, TMEM -> registers -> global (each warp owns 32 TMEM lanes)
+// The accumulator is double-buffered in TMEM (2 x 256 columns) so the epilogue of tile i
+// overlaps the main loop of tile i+1.  One CTA per SM, grid = min(tiles, SMs).
+// Every mbarrier wait is bounded; on timeout the CTA raises the device status word, drains its
+// own TMA copies and MMAs (bounded), frees TMEM and exits.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "sbp_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace sbp {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+constexpr int TMEM_COLS = 2 * BN;                    // double-buffered accumulator
+constexpr int kThreads = 192;
+constexpr int kGroupM = 8;                           // tile rasterisation group
+
+struct TcArgs {
+  GemmDesc g;
+  int a_mn, b_mn;
+  int nM, nN;
+  int* err;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int nM, int nN, int& mt, int& nt) {
+  const int per_group = kGroupM * nN;
+  const int group = t / per_group;
+  const int first_m = group * kGroupM;
+  const int gsz = min(nM - first_m, kGroupM);
+  const int r = t % per_group;
+  mt = first_m + r % gsz;
+  nt = r / gsz;
+}
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
+  uint4 pk;
+  __nv_bfloat162 t0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 t1 = __floats2bfloat162_rn(v[2], v[3]);
+  __nv_bfloat162 t2 = __floats2bfloat162_rn(v[4], v[5]);
+  __nv_bfloat162 t3 = __floats2bfloat162_rn(v[6], v[7]);
+  pk.x = *reinterpret_cast<uint32_t*>(&t0);
+  pk.y = *reinterpret_cast<uint32_t*>(&t1);
+  pk.z = *reinterpret_cast<uint32_t*>(&t2);
+  pk.w = *reinterpret_cast<uint32_t*>(&t3);
+  *reinterpret_cast<uint4*>(p) = pk;
+}
+
+// Store / accumulate 32 consecutive values v[0..31] of row `row` starting at column n.
+__device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int64_t n, int64_t N,
+                                            float (&v)[32]) {
+  if (g.bias) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (n + j < N) v[j] += ld_dt(g.bias, g.bias_dt, n + j);
+  }
+  const int64_t off = row * g.ldc + n;
+  if (n + 32 <= N) {
+    if (g.cdt == DT_F32) {
+      float* c = static_cast<float*>(g.C) + off;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 x = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        if (g.epi == EPI_ACC) {
+          const float4 o = *reinterpret_cast<const float4*>(c + j);
+          x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+        }
+        *reinterpret_cast<float4*>(c + j) = x;
+      }
+    } else {
+      __nv_bfloat16* c = static_cast<__nv_bfloat16*>(g.C) + off;
+      if (g.epi == EPI_ACC) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += __bfloat162float(c[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) store8_bf16(c + j, v + j);
+    }
+  } else {
+    for (int j = 0; j < 32 && n + j < N; ++j) {
+      float x = v[j];
+      if (g.epi == EPI_ACC) x += ld_dt(g.C, g.cdt, off + j);
+      st_dt(g.C, g.cdt, off + j, x);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2];
+  __shared__ uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GemmDesc& g = args.g;
+  volatile int* abort_flag = &abort_sh;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full_bar[s], 1);
+      tc::mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull_bar[a], 1);
+      tc::mbar_init(&tempty_bar[a], 4);
+    }
+    tc::mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tmap(&tmA);
+    tc::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  const int64_t M = g.dynM ? (int64_t)*g.dynM : g.M;
+  const int64_t K = g.dynK ? (int64_t)*g.dynK : g.K;
+  const int64_t N = g.N;
+  const int nk = (int)((K + BK - 1) / BK);
+  const int ntiles = args.nM * args.nN;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_coords(t, args.nM, args.nN, mt, nt);
+        const int m0 = mt * BM, n0 = nt * BN;
+        if (m0 >= M) continue;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          tc::mbar_expect_tx(&full_bar[s], STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (!args.a_mn) {
+            tc::tma_load_2d(sa, &tmA, &full_bar[s], k0, m0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j)
+              tc::tma_load_2d(sa + j * 8192, &tmA, &full_bar[s], m0 + 64 * j, k0);
+          }
+          if (!args.b_mn) {
+            tc::tma_load_2d(sb, &tmB, &full_bar[s], k0, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tc::tma_load_2d(sb + j * 8192, &tmB, &full_bar[s], n0 + 64 * j, k0);
+          }
+          issued_mask |= 1u << s;
+          issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // wind down: wait (bounded) for this CTA's own copies still in flight
+        const uint64_t t0 = tc::globaltimer_ns();
+        for (int q = 0; q < STAGES; ++q) {
+          if (!(issued_mask & (1u << q))) continue;
+          const uint32_t p = (issued_phase >> q) & 1u;
+          while (!tc::mbar_try_wait(&full_bar[q], p) &&
+                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, args.a_mn, args.b_mn);
+      const uint32_t smem_base = tc::smem_u32(smem);
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_coords(t, args.nM, args.nN, mt, nt);
+        if ((int64_t)mt * BM >= M) continue;
+        if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t sa = smem_base + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                          : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                          : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc::mma_f16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc::mma_commit(&empty_bar[s]);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc::mma_commit(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      if (issued) {
+        // make sure every MMA of this CTA has completed before TMEM is released
+        tc::mma_commit(&drain_bar);
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(&drain_bar, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int mt, nt;
+      tile_coords(t, args.nM, args.nN, mt, nt);
+      const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
+      if (m0 >= M) continue;
+      if (!tc::mbar_wait(&tfull_bar[acc], aph, abort_flag)) break;
+      tc::fence_after_sync();
+      const int64_t m = m0 + row_in_tile;
+      // the logit-gradient epilogue also writes the zero rows between the live row count and
+      // the buffer's row count, so that a later product over those rows reads zeros
+      const bool row_ok = m < (g.epi == EPI_CEGRAD ? g.M : M);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (g.epi == EPI_LSE) {
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t r0[32], r1[32];
+          tc::tmem_ld32(tbase + c, r0);
+          tc::tmem_ld32(tbase + c + 32, r1);
+          tc::tmem_ld_wait();
+          const int64_t nc = n0 + c;
+          if (!row_ok || nc >= N) continue;
+          const int ncols = (int)imin(64, N - nc);
+          float mx = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
+            if (j < ncols) mx = fmaxf(mx, a);
+            if (j + 32 < ncols) mx = fmaxf(mx, b);
+          }
+          float sm = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
+            if (j < ncols) sm += expf(a - mx);
+            if (j + 32 < ncols) sm += expf(b - mx);
+          }
+          const int64_t tile = nc / 64;
+          g.pmax[m * g.pld + tile] = mx;
+          g.psum[m * g.pld + tile] = sm;
+          const int64_t y = (int64_t)g.tgt[m] - g.col0 - nc;
+          if (y >= 0 && y < ncols) {
+            float z = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (y == j) z = u2f(r0[j]);
+              if (y == j + 32) z = u2f(r1[j]);
+            }
+            g.zy[m] = nk ? z : 0.f;
+          }
+        }
+      } else {
+        float w = 0.f, l = 0.f;
+        int64_t ycol = -1;
+        int64_t crow = m;
+        if (row_ok) {
+          if (g.epi == EPI_CEGRAD) {
+            w = g.wt[m];
+            l = g.lse[m];
+            ycol = (int64_t)g.tgt[m] - g.col0;
+          } else if (g.crow) {
+            crow = g.crow[m];
+          }
+        }
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tc::tmem_ld32(tbase + c, r);
+          tc::tmem_ld_wait();
+          const int64_t nc = n0 + c;
+          if (!row_ok || nc >= N) continue;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = nk ? u2f(r[j]) : 0.f;
+          if (g.epi == EPI_CEGRAD) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float p = expf(v[j] - l);
+              if (nc + j == ycol) p -= 1.f;
+              v[j] = w * p;
+            }
+          } else if (g.alpha != 1.f) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= g.alpha;
+          }
+          epi_store32(g, crow, nc, N, v);
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; aph ^= 1u; }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (threadIdx.x == 0 && abort_sh && args.err) atomicExch(args.err, DEV_TIMEOUT);
+  if (warp == 1) tc::tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  });
+  return n;
+}
+
+// 2-D bf16 tensor map: inner dimension `inner` (contiguous), outer dimension `outer` with a
+// stride of `ld` elements; box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+              int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+// Can the tensor-core kernel take this GEMM?
+bool gemm_tc_supported(const GemmDesc& g) {
+  if (g.adt != DT_BF16 || g.bdt != DT_BF16) return false;
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return false;
+  const bool a_k = g.sak == 1 && g.sam % 8 == 0 && g.sam > 0;
+  const bool a_m = g.sam == 1 && g.sak % 8 == 0 && g.sak > 0;
+  const bool b_k = g.sbk == 1 && g.sbn % 8 == 0 && g.sbn > 0;
+  const bool b_n = g.sbn == 1 && g.sbk % 8 == 0 && g.sbk > 0;
+  if (!(a_k || a_m) || !(b_k || b_n)) return false;
+  if (!al16(g.A) || !al16(g.B)) return false;
+  if (g.epi == EPI_STORE || g.epi == EPI_ACC || g.epi == EPI_CEGRAD) {
+    if (!al16(g.C) || g.ldc % 8 != 0) return false;
+  }
+  if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX)
+    return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st) {
+  TcArgs args;
+  args.g = g;
+  args.a_mn = (g.sak == 1) ? 0 : 1;
+  args.b_mn = (g.sbk == 1) ? 0 : 1;
+  args.nM = (int)((g.M + BM - 1) / BM);
+  args.nN = (int)((g.N + BN - 1) / BN);
+  args.err = err;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (!args.a_mn) ok = make_map(&ma, g.A, g.K, g.M, g.sam, BM);     // rows of K
+  else ok = make_map(&ma, g.A, g.M, g.K, g.sak, 64);               // k-rows of M
+  if (!ok) return cudaErrorInvalidValue;
+  if (!args.b_mn) ok = make_map(&mb, g.B, g.K, g.N, g.sbn, BN);
+  else ok = make_map(&mb, g.B, g.N, g.K, g.sbk, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = args.nM * args.nN;
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  launch(gemm_tc_kernel, grid, kThreads, SMEM_BYTES, st, ma, mb, args);
+  return cudaGetLastError();
+}
+
+}  // namespace sbp

@@ -120,7 +120,7 @@ __global__ void ce_loss_kernel(const int* __restrict__ count, const float* __res
 
 cudaError_t ce_compact(int64_t s, int64_t e, int64_t V, const int* tgt, const float* w, int* idx,
                        int* count, int* status, cudaStream_t st) {
-  ce_compact_kernel<<<1, 1024, 0, st>>>(s, e, V, tgt, w, idx, count, status);
+  launch(ce_compact_kernel, 1, 1024, 0, st, s, e, V, tgt, w, idx, count, status);
   return cudaGetLastError();
 }
 
@@ -128,7 +128,7 @@ cudaError_t ce_gather(int64_t Rmax, int64_t d, int dt, const void* h, const int*
                       const int* count, const int* tgt, const float* w, void* hc, int* yc,
                       float* wc, float* zy, float* lse, cudaStream_t st) {
   if (Rmax <= 0) return cudaSuccess;
-  ce_gather_kernel<<<(unsigned)Rmax, 256, 0, st>>>(d, dt, h, idx, count, tgt, w, hc, yc, wc, zy,
+  launch(ce_gather_kernel, (unsigned)Rmax, 256, 0, st, d, dt, h, idx, count, tgt, w, hc, yc, wc, zy,
                                                    lse);
   return cudaGetLastError();
 }
@@ -137,9 +137,9 @@ cudaError_t ce_finish(int64_t Rmax, int64_t tiles, const float* pmax, const floa
                       int64_t pld, const int* count, const float* wc, const float* zy,
                       float* lse, float* row_loss, float* loss, int first, cudaStream_t st) {
   if (Rmax > 0)
-    ce_lse_kernel<<<(unsigned)((Rmax * 32 + 255) / 256), 256, 0, st>>>(
+    launch(ce_lse_kernel, (unsigned)((Rmax * 32 + 255) / 256), 256, 0, st, 
         Rmax, tiles, pmax, psum, pld, count, wc, zy, lse, row_loss);
-  ce_loss_kernel<<<1, 1024, 0, st>>>(count, row_loss, loss, first);
+  launch(ce_loss_kernel, 1, 1024, 0, st, count, row_loss, loss, first);
   return cudaGetLastError();
 }
 

@@ -10,6 +10,7 @@
 #include <string>
 
 #include "sbp.h"
+#include "sbp_debug.h"
 #include "sbp_internal.cuh"
 
 using namespace sbp;
@@ -17,6 +18,9 @@ using namespace sbp;
 namespace {
 
 thread_local std::string g_err;
+// status word of the workspace of the entry point running on this thread (GEMMs raise their
+// bounded-wait timeouts there)
+thread_local int* tl_status = nullptr;
 
 sbp_status fail(sbp_status s, const char* fmt, ...) {
   char buf[512];
@@ -102,6 +106,8 @@ struct LayerPlan {
   void *xg, *n1, *q, *o, *n2, *gu, *m, *dgu, *dO;
   float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dm, *dn2, *dh, *delta, *dq, *dn1, *dxg;
   float *dkpre, *dvg, *rpart, *cpart;
+  // bf16 operand copies of fp32 gradients (bf16 path only)
+  void *dyg16, *dh16, *dq16, *khi, *klo, *vhi, *vlo;
   int64_t R;
 };
 
@@ -146,6 +152,16 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.rpart = c.take<float>(rmsnorm_bwd_partial_floats(d));
   int64_t wmax = dq > dkv ? dq : dkv;
   p.cpart = c.take<float>(colsum_partial_floats(wmax));
+  p.dyg16 = p.dh16 = p.dq16 = p.khi = p.klo = p.vhi = p.vlo = nullptr;
+  if (dt == DT_BF16) {
+    p.dyg16 = c.take_bytes((size_t)R * d * 2);
+    p.dh16 = c.take_bytes((size_t)R * d * 2);
+    p.dq16 = c.take_bytes((size_t)R * dq * 2);
+    p.khi = c.take_bytes((size_t)R * dkv * 2);
+    p.klo = c.take_bytes((size_t)R * dkv * 2);
+    p.vhi = c.take_bytes((size_t)R * dkv * 2);
+    p.vlo = c.take_bytes((size_t)R * dkv * 2);
+  }
 }
 
 // GEMM descriptor helpers.  Matrices are row-major with the given leading dimension.
@@ -162,6 +178,7 @@ GemmDesc mk_gemm(int64_t M, int64_t N, int64_t K, int adt, const void* A, bool a
   if (!b_t) { g.sbk = ldb; g.sbn = 1; } else { g.sbk = 1; g.sbn = ldb; }
   g.cdt = cdt; g.C = C; g.ldc = ldc;
   g.epi = epi;
+  g.err = tl_status;
   return g;
 }
 
@@ -319,6 +336,7 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D,
   Carver c(workspace);
   CePlan p;
   ce_carve(c, N, d, V, D, dt, p);
+  tl_status = p.status;
   SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
   for (int i = 0; i < D; ++i) {
     int64_t s, e;
@@ -403,6 +421,7 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
   const int64_t dq = H * hd, dkv = Hkv * hd;
   const int D = L.num_chunks;
 
+  tl_status = p.status;
   SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
   SBP_CK(rope_table(T, hd, L.rope_theta, p.cosb, p.sinb, st));
   SBP_CK(cudaMemsetAsync(p.dKp, 0, sizeof(float) * (size_t)B * T * dkv, st));
@@ -415,11 +434,20 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
     SBP_CK(gather_chunk(B, T, Tc, s, d, DT_F32, dy, p.dyg, st));
     if (sbp_status r = layer_chunk_forward(L, *w, p, s, Tc, st)) return r;
-    // ---- MLP backward
-    SBP_CK(gemm(mk_gemm(R, f, d, DT_F32, p.dyg, false, d, dt, w->w_down, false, f, DT_F32, p.dm,
-                        f, EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(d, f, R, DT_F32, p.dyg, true, d, dt, p.m, false, f, DT_F32, gr->w_down,
-                        f, EPI_ACC), st));
+    // ---- MLP backward.  fp32 gradients enter the tensor cores as bf16 operands (rounded
+    // per element, so the rounding does not depend on the chunking).
+    const bool b16 = dt == DT_BF16;
+    const void* dY = p.dyg;
+    int dYdt = DT_F32;
+    if (b16) {
+      SBP_CK(copy_cast(R * d, DT_F32, p.dyg, DT_BF16, p.dyg16, st));
+      dY = p.dyg16;
+      dYdt = DT_BF16;
+    }
+    SBP_CK(gemm(mk_gemm(R, f, d, dYdt, dY, false, d, dt, w->w_down, false, f, DT_F32, p.dm, f,
+                        EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(d, f, R, dYdt, dY, true, d, dt, p.m, false, f, DT_F32, gr->w_down, f,
+                        EPI_ACC), st));
     SBP_CK(swiglu_bwd(R, f, dt, p.gu, p.dm, p.dgu, st));
     const char* dU = static_cast<const char*>(p.dgu) + f * es;
     SBP_CK(gemm(mk_gemm(R, d, f, dt, p.dgu, false, 2 * f, dt, w->w_gate, false, d, DT_F32, p.dn2,
@@ -433,18 +461,32 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     SBP_CK(rmsnorm_bwd(R, d, DT_F32, p.hbuf, dt, w->ln2_g, p.rstd2, p.dn2, p.dyg, p.dh, 0,
                        gr->ln2_g, p.rpart, st));
     // ---- attention output projection backward
-    SBP_CK(gemm(mk_gemm(R, dq, d, DT_F32, p.dh, false, d, dt, w->wo, false, dq, dt, p.dO, dq,
+    const void* dH = p.dh;
+    int dHdt = DT_F32;
+    if (b16) {
+      SBP_CK(copy_cast(R * d, DT_F32, p.dh, DT_BF16, p.dh16, st));
+      dH = p.dh16;
+      dHdt = DT_BF16;
+    }
+    SBP_CK(gemm(mk_gemm(R, dq, d, dHdt, dH, false, d, dt, w->wo, false, dq, dt, p.dO, dq,
                         EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(d, dq, R, DT_F32, p.dh, true, d, dt, p.o, false, dq, DT_F32, gr->wo, dq,
+    SBP_CK(gemm(mk_gemm(d, dq, R, dHdt, dH, true, d, dt, p.o, false, dq, DT_F32, gr->wo, dq,
                         EPI_ACC), st));
     // ---- attention backward over the causal prefix; dK/dV accumulate in fp32
     SBP_CK(attn_bwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.dO, p.alse, p.delta,
                     p.dq, p.dKp, p.dVp, st));
     SBP_CK(rope_inv_f32(R, Tc, s, H, hd, p.dq, p.cosb, p.sinb, st));
     // ---- q projection backward
-    SBP_CK(gemm(mk_gemm(R, d, dq, DT_F32, p.dq, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
+    const void* dQ = p.dq;
+    int dQdt = DT_F32;
+    if (b16) {
+      SBP_CK(copy_cast(R * dq, DT_F32, p.dq, DT_BF16, p.dq16, st));
+      dQ = p.dq16;
+      dQdt = DT_BF16;
+    }
+    SBP_CK(gemm(mk_gemm(R, d, dq, dQdt, dQ, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
                         EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(dq, d, R, DT_F32, p.dq, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
+    SBP_CK(gemm(mk_gemm(dq, d, R, dQdt, dQ, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
                         EPI_ACC), st));
     if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
     SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, p.dxg, 0, gr->ln1_g,
@@ -460,14 +502,30 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     SBP_CK(rmsnorm_fwd(R, d, dt, p.xg, dt, w->ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
     SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
     SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
-    SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
-                        p.dn1, d, EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32, p.dn1,
-                        d, EPI_ACC), st));
-    SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d, DT_F32,
-                        gr->wk, d, EPI_ACC), st));
-    SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d, DT_F32, gr->wv,
-                        d, EPI_ACC), st));
+    if (dt == DT_BF16) {
+      // dK/dV are fp32 sums over chunks; their bf16 operands carry a hi + lo pair so that the
+      // products do not depend on where the fp32 sum happened to round
+      SBP_CK(split_bf16(R * dkv, p.dkpre, p.khi, p.klo, st));
+      SBP_CK(split_bf16(R * dkv, p.dvg, p.vhi, p.vlo, st));
+      const void* parts[4] = {p.khi, p.klo, p.vhi, p.vlo};
+      const void* wts[4] = {w->wk, w->wk, w->wv, w->wv};
+      float* grs[4] = {gr->wk, gr->wk, gr->wv, gr->wv};
+      for (int k = 0; k < 4; ++k) {
+        SBP_CK(gemm(mk_gemm(R, d, dkv, DT_BF16, parts[k], false, dkv, dt, wts[k], false, d,
+                            DT_F32, p.dn1, d, k == 0 ? EPI_STORE : EPI_ACC), st));
+        SBP_CK(gemm(mk_gemm(dkv, d, R, DT_BF16, parts[k], true, dkv, dt, p.n1, false, d, DT_F32,
+                            grs[k], d, EPI_ACC), st));
+      }
+    } else {
+      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
+                          p.dn1, d, EPI_STORE), st));
+      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32,
+                          p.dn1, d, EPI_ACC), st));
+      SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d, DT_F32,
+                          gr->wk, d, EPI_ACC), st));
+      SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d, DT_F32,
+                          gr->wv, d, EPI_ACC), st));
+    }
     if (has_bias) {
       SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
       SBP_CK(colsum_acc(R, dkv, p.dvg, gr->bv, p.cpart, st));
@@ -497,6 +555,7 @@ sbp_status sbp_decoder_layer_forward_stream(const sbp_layer_cfg* cfg,
   layer_carve(c, L, p);
   const int dt = L.dtype;
   const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
+  tl_status = p.status;
   SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
   SBP_CK(rope_table(T, L.head_dim, L.rope_theta, p.cosb, p.sinb, st));
   for (int i = 0; i < L.num_chunks; ++i) {
@@ -565,6 +624,25 @@ sbp_status sbp_embedding_backward(int64_t rows, int64_t cols, int64_t vocab,
     return fail(SBP_ERR_WORKSPACE, "workspace too small");
   SBP_CK(embed_bwd(rows, cols, vocab, ids, dy, d_table, static_cast<int*>(workspace),
                    static_cast<cudaStream_t>(stream)));
+  return SBP_OK;
+}
+
+// ------------------------------------------------------------------------------- debug
+sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int a_trans,
+                               int64_t lda, const void* B, int b_trans, int64_t ldb, float* C,
+                               int64_t ldc, int accumulate, int path, void* workspace,
+                               void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (!A || !B || !C || !workspace) return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
+  if (path < 0 || path > 2) return fail(SBP_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tl_status = static_cast<int*>(workspace);
+  GemmDesc g = mk_gemm(M, N, K, DT_BF16, A, a_trans != 0, lda, DT_BF16, B, b_trans != 0, ldb,
+                       DT_F32, C, ldc, accumulate ? EPI_ACC : EPI_STORE);
+  g.path = path;
+  if (path == 2 && !gemm_tc_supported(g))
+    return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
+  SBP_CK(gemm(g, st));
   return SBP_OK;
 }
 

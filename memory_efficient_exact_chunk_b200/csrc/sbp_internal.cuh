@@ -6,7 +6,27 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <utility>
+
 namespace sbp {
+
+// ---------------------------------------------------------------------------------------------
+// launch accounting (profile.cu): every kernel of the library goes through launch(), which
+// counts it; the profiler (sbp_profile.h) reads the count and times GEMM launches with events.
+// ---------------------------------------------------------------------------------------------
+void prof_count_launch();
+bool prof_enabled();
+enum ProfKind : int { PROF_GEMM_TC = 0, PROF_GEMM_SIMT = 1, PROF_KINDS = 2 };
+// events bracketing one launch of `kind` on `st` (no-ops unless profiling)
+void prof_mark_begin(int kind, cudaStream_t st);
+void prof_mark_end(int kind, cudaStream_t st);
+
+template <typename... KArgs, typename... Args>
+inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args&&... args) {
+  prof_count_launch();
+  kernel<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+}
 
 enum Dt : int { DT_F32 = 0, DT_BF16 = 1 };
 
@@ -91,12 +111,17 @@ struct GemmDesc {
   float* psum = nullptr;
   int64_t pld = 0;
   float* zy = nullptr;
+  // device status word raised on a bounded-wait timeout (nullable)
+  int* err = nullptr;
+  // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores only
+  int path = 0;
 };
 
 // Number of column tiles the EPI_LSE epilogue writes per row (its partial buffers' width).
 int64_t gemm_lse_tiles(int64_t N);
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
+bool gemm_tc_supported(const GemmDesc& g);
 
 // ---------------------------------------------------------------------------------------------
 // element-wise / row kernels (elementwise.cu)
@@ -146,6 +171,8 @@ cudaError_t colsum_acc(int64_t rows, int64_t cols, const float* src, float* dst,
 cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int ydt, void* y,
                          cudaStream_t st);
 cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st);
+// hi = bf16(x), lo = bf16(x - hi)
+cudaError_t split_bf16(int64_t n, const float* x, void* hi, void* lo, cudaStream_t st);
 
 // LM head helpers (lmhead.cu)
 // Stable compaction of chunk rows [s, e) with w != 0 (and a valid target) into idx[0..n),

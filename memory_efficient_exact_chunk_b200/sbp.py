@@ -24,7 +24,8 @@ EXPORTS = [
     "sbp_decoder_layer_workspace_size", "sbp_decoder_layer_backward_stream",
     "sbp_decoder_layer_forward_stream", "sbp_rmsnorm_forward",
     "sbp_rmsnorm_backward_workspace_size", "sbp_rmsnorm_backward", "sbp_embedding_forward",
-    "sbp_embedding_backward_workspace_size", "sbp_embedding_backward",
+    "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
+    "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -35,6 +36,10 @@ class SbpError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"{STATUS.get(code, code)}: {msg}")
         self.code = code
+
+
+class Profile(C.Structure):
+    _fields_ = [("launches", C.c_longlong * 2), ("ms", C.c_double * 2)]
 
 
 class LayerCfg(C.Structure):
@@ -90,6 +95,10 @@ def load(path: Optional[str] = None):
     lib.sbp_embedding_backward_workspace_size.restype = sz
     lib.sbp_embedding_backward_workspace_size.argtypes = [i64, i64]
     lib.sbp_embedding_backward.argtypes = [i64, i64, i64, vp, vp, vp, vp, sz, vp]
+    lib.sbp_debug_gemm_bf16.argtypes = [i64, i64, i64, vp, C.c_int, i64, vp, C.c_int, i64, vp, i64,
+                                         C.c_int, C.c_int, vp, vp]
+    lib.sbp_launch_count.restype = C.c_longlong
+    lib.sbp_profile_end.argtypes = [C.POINTER(Profile)]
     _lib = lib
     return lib
 
@@ -237,3 +246,34 @@ def embedding_backward(ids, dy2d, d_table, ws=None, stream=None):
     _check(load().sbp_embedding_backward(rows, cols, V, _ptr(ids), _ptr(dy2d), _ptr(d_table),
                                          _ptr(ws), ws.numel(), _stream(stream)))
     return ws
+
+
+# ----------------------------------------------------------------------------- test hooks
+def debug_gemm_bf16(A, a_trans, B, b_trans, C, accumulate=False, path=0, ws=None, stream=None):
+    """C (+)= op(A) op(B) with bf16 A/B and fp32 C (see include/sbp_debug.h)."""
+    M = A.shape[1] if a_trans else A.shape[0]
+    K = A.shape[0] if a_trans else A.shape[1]
+    N = B.shape[0] if b_trans else B.shape[1]
+    if ws is None:
+        ws = workspace(256, C.device)
+        ws.zero_()
+    _check(load().sbp_debug_gemm_bf16(M, N, K, _ptr(A), int(a_trans), A.stride(0), _ptr(B),
+                                      int(b_trans), B.stride(0), _ptr(C), C.stride(0),
+                                      int(accumulate), int(path), _ptr(ws), _stream(stream)))
+    return ws
+
+
+# ----------------------------------------------------------------------------- profiling
+def launch_count() -> int:
+    return int(load().sbp_launch_count())
+
+
+def profile_begin():
+    _check(load().sbp_profile_begin())
+
+
+def profile_end() -> dict:
+    p = Profile()
+    _check(load().sbp_profile_end(C.byref(p)))
+    return {"gemm_tc": {"launches": p.launches[0], "ms": p.ms[0]},
+            "gemm_simt": {"launches": p.launches[1], "ms": p.ms[1]}}

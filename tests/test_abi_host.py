@@ -21,7 +21,8 @@ def lib():
 
 
 def header_symbols():
-    txt = open(os.path.join(ROOT, "include", "sbp.h")).read()
+    txt = "".join(open(os.path.join(ROOT, "include", f)).read()
+                  for f in sorted(os.listdir(os.path.join(ROOT, "include"))) if f.endswith(".h"))
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
     return sorted(set(re.findall(r"\b(sbp_[a-z0-9_]+)\s*\(", txt)))
 

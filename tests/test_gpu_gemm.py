@@ -1,0 +1,52 @@
+"""GPU check of the GEMM engine (tensor-core tcgen05 kernel and CUDA-core kernel) against a
+plain PyTorch fp64 product of the same bf16 operands, for every operand layout."""
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+def _ref(A, at, B, bt):
+    a = A.double().cpu()
+    b = B.double().cpu()
+    a = a.t() if at else a
+    b = b.t() if bt else b
+    return a @ b
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("at,bt", [(0, 1), (0, 0), (1, 1), (1, 0)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 328, 136), (64, 8, 520), (392, 1032, 3584),
+                                   (8, 512, 8)])
+def test_gemm_layouts(path, at, bt, M, N, K):
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    A = torch.randn((K, M) if at else (M, K), generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn((N, K) if bt else (K, N), generator=g).to(torch.bfloat16).cuda()
+    C0 = torch.randn(M, N, generator=g).cuda()
+    C = torch.full((M, N), float("nan"), device="cuda")
+    ws = sbp.debug_gemm_bf16(A, at, B, bt, C, path=path)
+    sbp.device_status(ws)
+    ref = _ref(A, at, B, bt)
+    err = ((C.double().cpu() - ref).norm() / ref.norm()).item()
+    assert err <= 1e-5, err
+    C1 = C0.clone()
+    sbp.debug_gemm_bf16(A, at, B, bt, C1, accumulate=True, path=path, ws=ws)
+    sbp.device_status(ws)
+    ref1 = ref + C0.double().cpu()
+    err = ((C1.double().cpu() - ref1).norm() / ref1.norm()).item()
+    assert err <= 1e-5, err
+
+
+def test_gemm_tensor_core_rejects_unaligned_layout():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    A = torch.randn(64, 20).to(torch.bfloat16).cuda()     # leading dimension 20: not a multiple of 8
+    B = torch.randn(20, 64).to(torch.bfloat16).cuda()
+    C = torch.zeros(64, 64, device="cuda")
+    with pytest.raises(sbp.SbpError) as ei:
+        sbp.debug_gemm_bf16(A, 0, B, 0, C, path=2)
+    assert ei.value.code == 2
+    sbp.debug_gemm_bf16(A, 0, B, 0, C, path=0)               # automatic: CUDA cores
+    ref = _ref(A, 0, B, 0)
+    assert ((C.double().cpu() - ref).norm() / ref.norm()).item() <= 1e-5
