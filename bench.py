@@ -126,7 +126,7 @@ def run_lmhead(args, rank, world, device):
     import torch
     from memory_efficient_exact_chunk_b200 import sbp, synth
     wl = synth.WORKLOADS["lmhead_ce_32k"]
-    T, d, V = wl.seq_len, wl.hidden, wl.vocab
+    T, d, V = (args.tokens or wl.seq_len), wl.hidden, wl.vocab
     D = args.chunks or wl.num_chunks
     h, W, y, w = synth.lmhead_inputs(1000 + rank, T, d, V, bf16=True, from_frac=wl.loss_from_frac)
     n_valid = int(np.count_nonzero(w))
@@ -158,7 +158,8 @@ def run_lmhead(args, rank, world, device):
         "tokens_per_step": T, "n_loss_tokens": n_valid, "flops_step": flops_step,
         "flops_min_step": flops_min, "res": res, "ws_bytes": ws.numel(),
         "peak_act_gb": (peak_alloc - resident) / 1e9, "D": D,
-        "config": {"workload": "lmhead_ce_32k", "batch": 1, "seq_len": T, "hidden": d,
+        "config": {"workload": "lmhead_ce_32k" if T == wl.seq_len else f"lmhead_ce_{T}",
+                   "batch": 1, "seq_len": T, "hidden": d,
                    "vocab": V, "num_chunks": D, "loss_mask": "first 30% of tokens",
                    "n_loss_tokens": n_valid,
                    "l2": "inputs larger than L2 (1.09 GB LM-head weight re-read per chunk)"},
@@ -253,7 +254,7 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(n_rows=48):
+def cpu_baseline(n_rows=384):
     dt = oracle_lmhead_sample(n_rows)
     return {"value": n_rows / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{n_rows} loss tokens of the 32K LM-head workload (hidden 3584, vocab "
@@ -297,6 +298,8 @@ def main():
     ap.add_argument("--impl", default="sbp", choices=["sbp", "reference"])
     ap.add_argument("--workload", default="lmhead_ce_32k", choices=["lmhead_ce_32k"])
     ap.add_argument("--chunks", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the sequence length (small cases for profiling)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
