@@ -268,6 +268,11 @@ sbp_status check_ws(void* ws, size_t have, size_t need) {
 
 }  // namespace
 
+namespace sbp {
+// Lets other translation units of the library report a message through sbp_last_error().
+void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+}  // namespace sbp
+
 extern "C" {
 
 const char* sbp_last_error(void) { return g_err.c_str(); }

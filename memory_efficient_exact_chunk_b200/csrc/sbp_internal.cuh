@@ -30,6 +30,9 @@ inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 enum Dt : int { DT_F32 = 0, DT_BF16 = 1 };
 
+// Message returned by sbp_last_error() on this thread (sbp_api.cu).
+void set_last_error(const char* msg);
+
 inline size_t dt_size(int dt) { return dt == DT_BF16 ? 2 : 4; }
 __host__ __device__ __forceinline__ int64_t imin(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t imax(int64_t a, int64_t b) { return a > b ? a : b; }

@@ -25,7 +25,7 @@ EXPORTS = [
     "sbp_decoder_layer_forward_stream", "sbp_rmsnorm_forward",
     "sbp_rmsnorm_backward_workspace_size", "sbp_rmsnorm_backward", "sbp_embedding_forward",
     "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
-    "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end",
+    "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -97,6 +97,8 @@ def load(path: Optional[str] = None):
     lib.sbp_embedding_backward.argtypes = [i64, i64, i64, vp, vp, vp, vp, sz, vp]
     lib.sbp_debug_gemm_bf16.argtypes = [i64, i64, i64, vp, C.c_int, i64, vp, C.c_int, i64, vp, i64,
                                          C.c_int, C.c_int, vp, vp]
+    lib.sbp_lmhead_ce_backward_noalloc.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
+        [vp]
     lib.sbp_launch_count.restype = C.c_longlong
     lib.sbp_profile_end.argtypes = [C.POINTER(Profile)]
     _lib = lib
@@ -168,6 +170,18 @@ def lmhead_ce_backward(hidden_states, weight, targets, loss_weights, num_chunks,
         _ptr(loss_weights), _ptr(loss_out), _ptr(d_hidden), _ptr(d_weight), _ptr(ws),
         ws.numel(), _stream(stream)))
     return ws
+
+
+def lmhead_ce_backward_noalloc(hidden_states, weight, targets, loss_weights, num_chunks, loss_out,
+                               d_hidden, d_weight, stream=None):
+    """As lmhead_ce_backward, with the library's own fixed scratch instead of a workspace
+    (include/sbp_noalloc.h): nothing is allocated, sizes above the scratch are rejected."""
+    N, d = hidden_states.shape
+    V = weight.shape[0]
+    _check(load().sbp_lmhead_ce_backward_noalloc(
+        N, d, V, num_chunks, _dtype_code(hidden_states), _ptr(hidden_states), _ptr(weight),
+        _ptr(targets), _ptr(loss_weights), _ptr(loss_out), _ptr(d_hidden), _ptr(d_weight),
+        _stream(stream)))
 
 
 # ----------------------------------------------------------------------------- decoder layer
