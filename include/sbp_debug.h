@@ -30,6 +30,18 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
                                int64_t ldc, int accumulate, int path, void* workspace,
                                void* stream);
 
+/*
+ * Causal GQA attention forward of one query chunk over its key prefix (bf16):
+ *   q  [B * Tc, H, hd]  (chunk rows; row r is position s + r % Tc of sequence r / Tc)
+ *   Kp, Vp [B, T, Hkv, hd] (keys/values of whole sequences; positions < s + Tc are read)
+ *   o  [B * Tc, H, hd] bf16 out;  lse [B * Tc, H] fp32 out (natural log of the softmax sum)
+ * path: 0 automatic, 1 CUDA cores, 2 tensor cores (head_dim 128 only).
+ */
+sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H,
+                                   int64_t Hkv, int64_t hd, const void* q, const void* Kp,
+                                   const void* Vp, void* o, float* lse, int path, void* workspace,
+                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

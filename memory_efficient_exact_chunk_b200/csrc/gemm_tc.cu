@@ -253,7 +253,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tile_coords(t, args.nM, args.nN, mt, nt);
       const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
       if (m0 >= M) continue;
-      if (!tc::mbar_wait(&tfull_bar[acc], aph, abort_flag)) break;
+      if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) break;
       tc::fence_after_sync();
       const int64_t m = m0 + row_in_tile;
       // the logit-gradient epilogue also writes the zero rows between the live row count and

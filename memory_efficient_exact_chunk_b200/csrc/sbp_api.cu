@@ -271,6 +271,7 @@ sbp_status check_ws(void* ws, size_t have, size_t need) {
 namespace sbp {
 // Lets other translation units of the library report a message through sbp_last_error().
 void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+int* status_word() { return tl_status; }
 }  // namespace sbp
 
 extern "C" {
@@ -648,6 +649,23 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
   if (path == 2 && !gemm_tc_supported(g))
     return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
   SBP_CK(gemm(g, st));
+  return SBP_OK;
+}
+
+sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H,
+                                   int64_t Hkv, int64_t hd, const void* q, const void* Kp,
+                                   const void* Vp, void* o, float* lse, int path, void* workspace,
+                                   void* stream) {
+  if (B <= 0 || T <= 0 || Tc <= 0 || s < 0 || s + Tc > T || H <= 0 || Hkv <= 0 || H % Hkv ||
+      hd <= 0 || hd % 2 || hd > 256)
+    return fail(SBP_ERR_INVALID_ARG, "bad attention sizes");
+  if (!q || !Kp || !Vp || !o || !lse || !workspace) return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
+  if (path < 0 || path > 2) return fail(SBP_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+  if (path == 2 && !attn_tc_supported(hd, DT_BF16, q, Kp, Vp, o))
+    return fail(SBP_ERR_UNSUPPORTED, "the tensor-core attention needs head_dim 128 and aligned rows");
+  tl_status = static_cast<int*>(workspace);
+  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, lse,
+                  static_cast<cudaStream_t>(stream), path));
   return SBP_OK;
 }
 

@@ -32,6 +32,9 @@ enum Dt : int { DT_F32 = 0, DT_BF16 = 1 };
 
 // Message returned by sbp_last_error() on this thread (sbp_api.cu).
 void set_last_error(const char* msg);
+// Device status word of the workspace of the entry point running on this thread (sbp_api.cu);
+// kernels with bounded waits raise their timeouts there.
+int* status_word();
 
 inline size_t dt_size(int dt) { return dt == DT_BF16 ? 2 : 4; }
 __host__ __device__ __forceinline__ int64_t imin(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -193,11 +196,18 @@ cudaError_t ce_finish(int64_t Rmax, int64_t tiles, const float* pmax, const floa
 // out rows idx[r] (r < n) of d_hidden chunk: zero rows [s, e) of dh first.
 cudaError_t zero_rows(int64_t s, int64_t e, int64_t d, float* dh, cudaStream_t st);
 
-// attention (attention.cu)
+// attention: tensor-core forward (attn_tc.cu, head_dim 128, bf16) and CUDA-core kernels
+// (attention_simt.cu, any even head_dim <= 256, fp32 or bf16).  attn_fwd/attn_bwd dispatch;
+// path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores.
+bool attn_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
+                       const void* o);
+cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
+                        const void* q, const void* Kp, const void* Vp, void* o, float* lse,
+                        int* err, cudaStream_t st);
 // Forward for chunk queries q [B*Tc, H, hd] at positions s.. over prefix keys [0, s + Tc).
 cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp, void* o,
-                     float* lse, cudaStream_t st);
+                     float* lse, cudaStream_t st, int path = 0);
 // Backward: dq [B*Tc, H, hd] fp32 (overwritten); dKp/dVp [B, T, Hkv, hd] fp32 (+= rows < s+Tc).
 cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,

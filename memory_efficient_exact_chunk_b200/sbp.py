@@ -26,6 +26,7 @@ EXPORTS = [
     "sbp_rmsnorm_backward_workspace_size", "sbp_rmsnorm_backward", "sbp_embedding_forward",
     "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
     "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
+    "sbp_debug_attn_fwd_bf16",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -99,6 +100,7 @@ def load(path: Optional[str] = None):
                                          C.c_int, C.c_int, vp, vp]
     lib.sbp_lmhead_ce_backward_noalloc.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp]
+    lib.sbp_debug_attn_fwd_bf16.argtypes = [i64] * 7 + [vp] * 5 + [C.c_int, vp, vp]
     lib.sbp_launch_count.restype = C.c_longlong
     lib.sbp_profile_end.argtypes = [C.POINTER(Profile)]
     _lib = lib
@@ -291,3 +293,18 @@ def profile_end() -> dict:
     _check(load().sbp_profile_end(C.byref(p)))
     return {"gemm_tc": {"launches": p.launches[0], "ms": p.ms[0]},
             "gemm_simt": {"launches": p.launches[1], "ms": p.ms[1]}}
+
+
+def debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=0, ws=None, stream=None):
+    """Attention forward of a chunk (include/sbp_debug.h); q/o [B*Tc, H, hd], Kp/Vp
+    [B, T, Hkv, hd] bf16, lse [B*Tc, H] fp32."""
+    B, T, Hkv, hd = Kp.shape
+    R, H, _ = q.shape
+    Tc = R // B
+    if ws is None:
+        ws = workspace(256, q.device)
+        ws.zero_()
+    _check(load().sbp_debug_attn_fwd_bf16(B, T, Tc, s, H, Hkv, hd, _ptr(q), _ptr(Kp), _ptr(Vp),
+                                          _ptr(o), _ptr(lse), int(path), _ptr(ws),
+                                          _stream(stream)))
+    return ws

@@ -73,15 +73,19 @@ def test_layer_fp32_gqa_bias_ragged(L, B, T, D):
     _check(L, W, x, dy, D, "f32")
 
 
-@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 256, 4), (QWEN_LIKE, 2, 384, 3)])
+HD128 = synth.LayerShape(256, 4, 2, 128, 512, 1e-5, 500000.0)
+HD128_BIAS = synth.LayerShape(256, 4, 1, 128, 384, 1e-6, 1e6, qkv_bias=True)
+
+
+@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 256, 4), (QWEN_LIKE, 2, 384, 3), (HD128, 2, 384, 3),
+                                     (HD128, 1, 300, 5), (HD128_BIAS, 2, 256, 2)])
 def test_layer_bf16(L, B, T, D):
     W, x, dy = synth.layer_inputs(2, L, B, T, bf16=True, dy_std=1e-3, gamma_std=0.1)
     _check(L, W, x, dy, D, "bf16")
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_layer_d_invariance(dtype):
-    L = GQA
+@pytest.mark.parametrize("dtype,L", [("f32", GQA), ("bf16", GQA), ("bf16", HD128)])
+def test_layer_d_invariance(dtype, L):
     W, x, dy = synth.layer_inputs(3, L, 2, 512, bf16=(dtype == "bf16"), dy_std=1e-3)
     dx1, g1 = _gpu_layer(L, W, x, dy, 1, dtype)
     for D in (2, 4, 8):
