@@ -213,8 +213,12 @@ static void attn_bwd_launch(int64_t B, int64_t Tn, int64_t Tc, int64_t s, int64_
 cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
                      const void* o, const void* dO, const float* lse, float* delta, float* dq,
-                     float* dKp, float* dVp, cudaStream_t st) {
+                     float* dKp, float* dVp, cudaStream_t st, int path) {
   if (B * Tc * H <= 0) return cudaSuccess;
+  if (path != 1 && attn_bwd_tc_supported(hd, dt, q, Kp, Vp, o, dO, dq))
+    return attn_bwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, dO, lse, delta, dq, dKp, dVp,
+                       status_word(), st);
+  if (path == 2) return cudaErrorNotSupported;
   if (dt == DT_BF16)
     attn_bwd_launch<__nv_bfloat16>(B, T, Tc, s, H, Hkv, hd, q, Kp, Vp, o, dO, lse, delta, dq, dKp,
                                    dVp, st);

@@ -107,7 +107,7 @@ struct LayerPlan {
   float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dm, *dn2, *dh, *delta, *dq, *dn1, *dxg;
   float *dkpre, *dvg, *rpart, *cpart;
   // bf16 operand copies of fp32 gradients (bf16 path only)
-  void *dyg16, *dh16, *dq16, *khi, *klo, *vhi, *vlo;
+  void *dyg16, *dh16, *dq16, *dqlo, *khi, *klo, *vhi, *vlo;
   int64_t R;
 };
 
@@ -152,11 +152,12 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.rpart = c.take<float>(rmsnorm_bwd_partial_floats(d));
   int64_t wmax = dq > dkv ? dq : dkv;
   p.cpart = c.take<float>(colsum_partial_floats(wmax));
-  p.dyg16 = p.dh16 = p.dq16 = p.khi = p.klo = p.vhi = p.vlo = nullptr;
+  p.dyg16 = p.dh16 = p.dq16 = p.dqlo = p.khi = p.klo = p.vhi = p.vlo = nullptr;
   if (dt == DT_BF16) {
     p.dyg16 = c.take_bytes((size_t)R * d * 2);
     p.dh16 = c.take_bytes((size_t)R * d * 2);
     p.dq16 = c.take_bytes((size_t)R * dq * 2);
+    p.dqlo = c.take_bytes((size_t)R * dq * 2);
     p.khi = c.take_bytes((size_t)R * dkv * 2);
     p.klo = c.take_bytes((size_t)R * dkv * 2);
     p.vhi = c.take_bytes((size_t)R * dkv * 2);
@@ -432,6 +433,10 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
   SBP_CK(rope_table(T, hd, L.rope_theta, p.cosb, p.sinb, st));
   SBP_CK(cudaMemsetAsync(p.dKp, 0, sizeof(float) * (size_t)B * T * dkv, st));
   SBP_CK(cudaMemsetAsync(p.dVp, 0, sizeof(float) * (size_t)B * T * dkv, st));
+  // key/value rows past the current prefix are read (and masked) by the last key tile of a
+  // query tile: give them finite contents
+  SBP_CK(cudaMemsetAsync(p.Kp, 0, es * (size_t)B * T * dkv, st));
+  SBP_CK(cudaMemsetAsync(p.Vp, 0, es * (size_t)B * T * dkv, st));
 
   for (int i = 0; i < D; ++i) {
     int64_t s, e;
@@ -483,17 +488,23 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
                     p.dq, p.dKp, p.dVp, st));
     SBP_CK(rope_inv_f32(R, Tc, s, H, hd, p.dq, p.cosb, p.sinb, st));
     // ---- q projection backward
-    const void* dQ = p.dq;
-    int dQdt = DT_F32;
     if (b16) {
-      SBP_CK(copy_cast(R * dq, DT_F32, p.dq, DT_BF16, p.dq16, st));
-      dQ = p.dq16;
-      dQdt = DT_BF16;
+      // dQ is a sum over key tiles accumulated with atomics (order not fixed): it enters the
+      // tensor cores as a hi + lo bf16 pair so that its rounding does not show in the result
+      SBP_CK(split_bf16(R * dq, p.dq, p.dq16, p.dqlo, st));
+      const void* parts[2] = {p.dq16, p.dqlo};
+      for (int k = 0; k < 2; ++k) {
+        SBP_CK(gemm(mk_gemm(R, d, dq, DT_BF16, parts[k], false, dq, dt, w->wq, false, d, DT_F32,
+                            p.dn1, d, k == 0 ? EPI_STORE : EPI_ACC), st));
+        SBP_CK(gemm(mk_gemm(dq, d, R, DT_BF16, parts[k], true, dq, dt, p.n1, false, d, DT_F32,
+                            gr->wq, d, EPI_ACC), st));
+      }
+    } else {
+      SBP_CK(gemm(mk_gemm(R, d, dq, DT_F32, p.dq, false, dq, dt, w->wq, false, d, DT_F32, p.dn1,
+                          d, EPI_STORE), st));
+      SBP_CK(gemm(mk_gemm(dq, d, R, DT_F32, p.dq, true, dq, dt, p.n1, false, d, DT_F32, gr->wq,
+                          d, EPI_ACC), st));
     }
-    SBP_CK(gemm(mk_gemm(R, d, dq, dQdt, dQ, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
-                        EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(dq, d, R, dQdt, dQ, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
-                        EPI_ACC), st));
     if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
     SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, p.dxg, 0, gr->ln1_g,
                        p.rpart, st));
@@ -564,6 +575,11 @@ sbp_status sbp_decoder_layer_forward_stream(const sbp_layer_cfg* cfg,
   tl_status = p.status;
   SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
   SBP_CK(rope_table(T, L.head_dim, L.rope_theta, p.cosb, p.sinb, st));
+  {
+    const size_t kvb = dt_size(dt) * (size_t)B * T * L.n_kv_heads * L.head_dim;
+    SBP_CK(cudaMemsetAsync(p.Kp, 0, kvb, st));
+    SBP_CK(cudaMemsetAsync(p.Vp, 0, kvb, st));
+  }
   for (int i = 0; i < L.num_chunks; ++i) {
     int64_t s, e;
     chunk_range(T, L.num_chunks, i, s, e);
@@ -665,6 +681,26 @@ sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, 
     return fail(SBP_ERR_UNSUPPORTED, "the tensor-core attention needs head_dim 128 and aligned rows");
   tl_status = static_cast<int*>(workspace);
   SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, lse,
+                  static_cast<cudaStream_t>(stream), path));
+  return SBP_OK;
+}
+
+sbp_status sbp_debug_attn_bwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H,
+                                   int64_t Hkv, int64_t hd, const void* q, const void* Kp,
+                                   const void* Vp, const void* o, const void* dO,
+                                   const float* lse, float* dq, float* dKp, float* dVp,
+                                   int path, void* workspace, void* stream) {
+  if (B <= 0 || T <= 0 || Tc <= 0 || s < 0 || s + Tc > T || H <= 0 || Hkv <= 0 || H % Hkv ||
+      hd <= 0 || hd % 2 || hd > 256)
+    return fail(SBP_ERR_INVALID_ARG, "bad attention sizes");
+  if (!q || !Kp || !Vp || !o || !dO || !lse || !dq || !dKp || !dVp || !workspace)
+    return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
+  if (path < 0 || path > 2) return fail(SBP_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+  if (path == 2 && !attn_bwd_tc_supported(hd, DT_BF16, q, Kp, Vp, o, dO, dq))
+    return fail(SBP_ERR_UNSUPPORTED, "the tensor-core attention needs head_dim 128 and aligned rows");
+  tl_status = static_cast<int*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  SBP_CK(attn_bwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, dO, lse, delta, dq, dKp, dVp,
                   static_cast<cudaStream_t>(stream), path));
   return SBP_OK;
 }

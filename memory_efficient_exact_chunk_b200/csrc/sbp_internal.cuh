@@ -212,7 +212,13 @@ cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int
 cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
                      const void* o, const void* dO, const float* lse, float* delta, float* dq,
-                     float* dKp, float* dVp, cudaStream_t st);
+                     float* dKp, float* dVp, cudaStream_t st, int path = 0);
+bool attn_bwd_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
+                           const void* o, const void* dO, const float* dq);
+cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
+                        const void* q, const void* Kp, const void* Vp, const void* o,
+                        const void* dO, const float* lse, float* delta, float* dq, float* dKp,
+                        float* dVp, int* err, cudaStream_t st);
 
 // embedding (elementwise.cu)
 cudaError_t embed_fwd(int64_t rows, int64_t cols, int64_t vocab, int dt, const int* ids,

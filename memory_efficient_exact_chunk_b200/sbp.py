@@ -26,7 +26,7 @@ EXPORTS = [
     "sbp_rmsnorm_backward_workspace_size", "sbp_rmsnorm_backward", "sbp_embedding_forward",
     "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
     "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
-    "sbp_debug_attn_fwd_bf16",
+    "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -101,6 +101,7 @@ def load(path: Optional[str] = None):
     lib.sbp_lmhead_ce_backward_noalloc.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp]
     lib.sbp_debug_attn_fwd_bf16.argtypes = [i64] * 7 + [vp] * 5 + [C.c_int, vp, vp]
+    lib.sbp_debug_attn_bwd_bf16.argtypes = [i64] * 7 + [vp] * 9 + [C.c_int, vp, vp]
     lib.sbp_launch_count.restype = C.c_longlong
     lib.sbp_profile_end.argtypes = [C.POINTER(Profile)]
     _lib = lib
@@ -307,4 +308,17 @@ def debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=0, ws=None, stream=None):
     _check(load().sbp_debug_attn_fwd_bf16(B, T, Tc, s, H, Hkv, hd, _ptr(q), _ptr(Kp), _ptr(Vp),
                                           _ptr(o), _ptr(lse), int(path), _ptr(ws),
                                           _stream(stream)))
+    return ws
+
+
+def debug_attn_bwd_bf16(q, Kp, Vp, o, dO, lse, dq, dKp, dVp, s, path=0, stream=None):
+    """Attention backward of a chunk (include/sbp_debug.h)."""
+    B, T, Hkv, hd = Kp.shape
+    R, H, _ = q.shape
+    Tc = R // B
+    ws = workspace(256 + 4 * R * H, q.device)
+    ws.zero_()
+    _check(load().sbp_debug_attn_bwd_bf16(B, T, Tc, s, H, Hkv, hd, _ptr(q), _ptr(Kp), _ptr(Vp),
+                                          _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dKp),
+                                          _ptr(dVp), int(path), _ptr(ws), _stream(stream)))
     return ws

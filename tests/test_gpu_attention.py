@@ -74,3 +74,59 @@ def test_attention_forward_tc_chunking_is_bitwise_neutral():
         sbp.debug_attn_fwd_bf16(q[s:e].contiguous(), Kp, Vp, o, l, s, path=2)
         torch.cuda.synchronize()
         assert torch.equal(o, o_full[s:e]) and torch.equal(l, l_full[s:e]), (s, e)
+
+
+@pytest.mark.parametrize("B,T,s,Tc,H,Hkv", [
+    (1, 256, 0, 256, 2, 1),
+    (2, 384, 128, 128, 4, 2),
+    (1, 300, 100, 150, 2, 2),      # ragged chunk and sequence
+    (1, 640, 256, 384, 4, 1),
+])
+def test_attention_backward_tc(B, T, s, Tc, H, Hkv):
+    """dQ, dK, dV of the chunk queries against fp64 autograd of the same bf16 operands."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(7 * T + s + H)
+    hd = 128
+    q = torch.randn(B * Tc, H, hd, generator=g).to(torch.bfloat16).cuda()
+    Kp = torch.randn(B, T, Hkv, hd, generator=g).to(torch.bfloat16).cuda()
+    Vp = torch.randn(B, T, Hkv, hd, generator=g).to(torch.bfloat16).cuda()
+    dO = torch.randn(B * Tc, H, hd, generator=g).to(torch.bfloat16).cuda()
+    o = torch.empty(B * Tc, H, hd, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B * Tc, H, device="cuda")
+    sbp.debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=2)
+    # fp64 autograd reference
+    qr = q.double().cpu().requires_grad_()
+    kr = Kp.double().cpu().requires_grad_()
+    vr = Vp.double().cpu().requires_grad_()
+    out, _ = _reference_autograd(qr, kr, vr, s)
+    out.backward(dO.double().cpu())
+    for path in (2, 1):
+        dq = torch.full((B * Tc, H, hd), float("nan"), device="cuda")
+        dK = torch.zeros(B, T, Hkv, hd, device="cuda")
+        dV = torch.zeros(B, T, Hkv, hd, device="cuda")
+        ws = sbp.debug_attn_bwd_bf16(q, Kp, Vp, o, dO, lse, dq, dK, dV, s, path=path)
+        sbp.device_status(ws)
+        for got, want, name in ((dq, qr.grad, "dq"), (dK, kr.grad, "dK"), (dV, vr.grad, "dV")):
+            err = ((got.double().cpu() - want).norm() / want.norm()).item()
+            assert err <= 1e-2, (path, name, err)
+        assert torch.all(dK[:, s + Tc:] == 0) and torch.all(dV[:, s + Tc:] == 0)
+
+
+def _reference_autograd(q, Kp, Vp, s):
+    import torch
+    B, T, Hkv, hd = Kp.shape
+    R, H, _ = q.shape
+    Tc = R // B
+    grp = H // Hkv
+    outs = []
+    for b in range(B):
+        qb = q[b * Tc:(b + 1) * Tc]
+        kb = Kp[b, :s + Tc].repeat_interleave(grp, 1)
+        vb = Vp[b, :s + Tc].repeat_interleave(grp, 1)
+        sc = torch.einsum("thd,uhd->htu", qb, kb) / math.sqrt(hd)
+        tpos = torch.arange(s, s + Tc)[:, None]
+        upos = torch.arange(s + Tc)[None, :]
+        sc = sc.masked_fill(upos > tpos, float("-inf"))
+        outs.append(torch.einsum("htu,uhd->thd", torch.softmax(sc, -1), vb))
+    return torch.cat(outs), None
