@@ -197,6 +197,87 @@ def run_lmhead(args, rank, world, device):
     return out
 
 
+def run_layer(args, rank, world, device, sweep=False):
+    """One Llama-3-8B-shaped decoder layer (d 4096, 32/8 heads of 128, MLP 14336, theta 5e5),
+    bf16, T = 32768, D = 8: one step = one sbp_decoder_layer_backward_stream call."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp, synth
+    wl = synth.WORKLOADS["llama3_8b_layer_32k"]
+    L = wl.layer
+    B, T = wl.batch, (args.layer_tokens or wl.seq_len)
+    D = args.layer_chunks or wl.num_chunks
+    W, x, dy = synth.layer_inputs(2000 + rank, L, B, T, bf16=True, dy_std=1e-3)
+    names = sbp.WEIGHT_FIELDS
+    Wd = {n: (torch.from_numpy(W[n]).to(torch.bfloat16).to(device) if W.get(n) is not None
+              else None) for n in names}
+    P = sum(int(np.prod(W[n].shape)) for n in ("wq", "wk", "wv", "wo", "w_gate", "w_up",
+                                              "w_down"))
+    del W
+    xd = torch.from_numpy(x).to(torch.bfloat16).to(device)
+    dyd = torch.from_numpy(dy).to(device)
+    del x, dy
+    dx = torch.empty(B, T, L.d_model, device=device)
+    grads = {n: (torch.zeros(Wd[n].shape, device=device) if Wd.get(n) is not None else None)
+             for n in names}
+    torch.cuda.synchronize()
+    resident = torch.cuda.memory_allocated(device)
+
+    def cfg_for(Dc):
+        return sbp.layer_cfg(B, T, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
+                             L.rms_eps, L.rope_theta, sbp.SBP_BF16, Dc)
+
+    cfg = cfg_for(D)
+    ws = sbp.workspace(sbp.layer_workspace_size(cfg), device)
+    step = lambda: sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, grads, ws=ws)
+    lin_flops = 6.0 * P * B * T
+    att_flops = 14.0 * L.head_dim * L.n_heads * B * T * (T + 1) / 2
+    largs = argparse.Namespace(steps=max(1, min(args.steps, 3)), warmup=args.warmup)
+    res = timed(largs, step, world, device, profile=True)
+    sbp.device_status(ws)
+    torch.cuda.reset_peak_memory_stats(device)
+    step()
+    torch.cuda.synchronize()
+    peak = torch.cuda.max_memory_allocated(device) - resident
+    prof = res["prof"]
+    k = largs.steps
+
+    def tf(flops, ms):
+        return flops * k / (ms / 1e3) / 1e12 if ms > 0 else None
+
+    out = {
+        "workload": "llama3_8b_layer_32k" if T == wl.seq_len else f"llama3_8b_layer_{T}",
+        "value": B * T * world / (res["ms"] / 1e3), "unit": "tokens/s",
+        "ms_per_step": res["ms"], "steps": k, "num_chunks": D,
+        "config": {"batch": B, "seq_len": T, "d_model": L.d_model, "n_heads": L.n_heads,
+                   "n_kv_heads": L.n_kv_heads, "head_dim": L.head_dim, "ffn": L.ffn,
+                   "num_chunks": D, "linear_params": P},
+        "flops_step": {"linear_6P": lin_flops, "attention_14hd": att_flops},
+        "achieved_tflops_step": (lin_flops + att_flops) / (res["ms"] / 1e3) / 1e12,
+        "kernels": {n: {"launches_per_step": v["launches"] / k, "ms_per_step": v["ms"] / k,
+                        "share": v["ms"] / res["ms_total"] if res["ms_total"] else None}
+                    for n, v in prof.items() if v["launches"]},
+        "gemm_tc_tflops": tf(lin_flops, prof["gemm_tc"]["ms"]),
+        "attn_tflops": tf(att_flops, prof["attn_fwd"]["ms"] + prof["attn_bwd"]["ms"]),
+        "attn_fwd_tflops": tf(4.0 / 14.0 * att_flops, prof["attn_fwd"]["ms"]),
+        "attn_bwd_tflops": tf(10.0 / 14.0 * att_flops, prof["attn_bwd"]["ms"]),
+        "gpu_launches": res["launches"], "clocks": res["clocks"],
+        "peak_act_gb": peak / 1e9, "workspace_gb": ws.numel() / 1e9,
+    }
+    if sweep and rank == 0 and world == 1:
+        sw = []
+        for Dc in (1, 2, 4, 8, 16):
+            c2 = cfg_for(Dc)
+            del ws
+            torch.cuda.empty_cache()
+            ws = sbp.workspace(sbp.layer_workspace_size(c2), device)
+            st2 = lambda: sbp.decoder_layer_backward(c2, Wd, xd, dyd, dx, grads, ws=ws)
+            r = timed(argparse.Namespace(steps=1, warmup=1), st2, 1, device, profile=False)
+            sw.append({"D": Dc, "tokens_per_s": B * T / (r["ms"] / 1e3), "ms_per_step": r["ms"],
+                       "workspace_gb": ws.numel() / 1e9})
+        out["sweep"] = sw
+    return out
+
+
 def timed(args, step, world, device, profile):
     """W warm-up steps, then K timed steps between a barrier + synchronize on both sides;
     device time from CUDA events on the launching stream, max over ranks."""
@@ -254,8 +335,8 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(n_rows=384):
-    dt = oracle_lmhead_sample(n_rows)
+def cpu_baseline(n_rows=2048):
+    dt = sum(oracle_lmhead_sample(512, seed=5 + i) for i in range(n_rows // 512))
     return {"value": n_rows / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{n_rows} loss tokens of the 32K LM-head workload (hidden 3584, vocab "
                       f"152064), fp64 numpy, {dt:.1f} s"}
@@ -289,6 +370,32 @@ def run_reference(args, rank, world):
     return 0
 
 
+def layer_main(args, rank, world, device):
+    """The decoder-layer workload as the line's own workload (no LM head)."""
+    import torch.distributed as dist
+    peaks, peak_src = load_peaks()
+    o = run_layer(args, rank, world, device, sweep=args.sweep)
+    att = o["attn_tflops"] or 0.0
+    line = {
+        "metric": METRIC, "value": o["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": o["steps"], "warmup": args.warmup, "ms_per_step": o["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": dict(workload=o["workload"], **o["config"]),
+        "layer": o, "cpu_baseline": None,
+        "roofline": {"bound": "tensor", "kernel": "attention backward + forward (tcgen05)",
+                     "achieved": att, "peak": float(peaks["bf16_tflops_sustained"]),
+                     "unit": "TFLOP/s", "frac": att / float(peaks["bf16_tflops_sustained"]),
+                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None},
+        "gpu_launches": o["gpu_launches"], "clocks": o["clocks"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -296,13 +403,18 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sbp", choices=["sbp", "reference"])
-    ap.add_argument("--workload", default="lmhead_ce_32k", choices=["lmhead_ce_32k"])
+    ap.add_argument("--workload", default="lmhead_ce_32k",
+                    choices=["lmhead_ce_32k", "llama3_8b_layer_32k"])
     ap.add_argument("--chunks", type=int, default=0)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the sequence length (small cases for profiling)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--no-layer", dest="layer", action="store_false",
+                    help="skip the decoder-layer measurement added to the line")
+    ap.add_argument("--layer-tokens", type=int, default=0)
+    ap.add_argument("--layer-chunks", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -322,6 +434,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     sbp.load()
+    if args.workload == "llama3_8b_layer_32k":
+        return layer_main(args, rank, world, device)
     out = run_lmhead(args, rank, world, device)
     res = out["res"]
     peaks, peak_src = load_peaks()
@@ -358,6 +472,8 @@ def main():
     }
     if "sweep" in out:
         line["sweep"] = out["sweep"]
+    if args.layer:
+        line["also"] = [run_layer(args, rank, world, device, sweep=args.sweep)]
     if "e2e" in out:
         line["e2e"] = out["e2e"]
     if args.cpu and rank == 0 and world == 1:

@@ -2,9 +2,9 @@
  * sbp_profile.h -- launch accounting and GEMM timing of libsbp (instrumentation; the paper
  * has no counterpart).
  *
- * While profiling is on, every GEMM the library queues is bracketed by two CUDA events on its
- * own stream, so that a caller can read the device time of the dominant kernels of a timed
- * region.  Profiling is process-wide and off by default.
+ * While profiling is on, every GEMM and attention call the library queues is bracketed by two
+ * CUDA events on its own stream, so that a caller can read the device time of the dominant
+ * kernels of a timed region.  Profiling is process-wide and off by default.
  */
 #ifndef SBP_PROFILE_H_
 #define SBP_PROFILE_H_
@@ -15,10 +15,16 @@
 extern "C" {
 #endif
 
-enum { SBP_PROF_GEMM_TC = 0, SBP_PROF_GEMM_SIMT = 1, SBP_PROF_KINDS = 2 };
+enum {
+  SBP_PROF_GEMM_TC = 0,   /* tcgen05 GEMM                               */
+  SBP_PROF_GEMM_SIMT = 1, /* CUDA-core GEMM                             */
+  SBP_PROF_ATTN_FWD = 2,  /* attention forward of a chunk (either path) */
+  SBP_PROF_ATTN_BWD = 3,  /* attention backward of a chunk (either path) */
+  SBP_PROF_KINDS = 4
+};
 
 typedef struct {
-  long long launches[SBP_PROF_KINDS]; /* launches per kind (tensor-core GEMM, CUDA-core GEMM) */
+  long long launches[SBP_PROF_KINDS]; /* timed calls per kind                                  */
   double ms[SBP_PROF_KINDS];          /* summed device time per kind, milliseconds            */
 } sbp_profile;
 

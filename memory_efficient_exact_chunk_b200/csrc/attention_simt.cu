@@ -181,9 +181,14 @@ cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int
                      float* lse, cudaStream_t st, int path) {
   const int64_t w = B * Tc * H;
   if (w <= 0) return cudaSuccess;
-  if (path != 1 && attn_tc_supported(hd, dt, q, Kp, Vp, o))
-    return attn_fwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, lse, status_word(), st);
+  if (path != 1 && attn_tc_supported(hd, dt, q, Kp, Vp, o)) {
+    prof_mark_begin(PROF_ATTN_FWD, st);
+    const cudaError_t e = attn_fwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, lse, status_word(), st);
+    prof_mark_end(PROF_ATTN_FWD, st);
+    return e;
+  }
   if (path == 2) return cudaErrorNotSupported;
+  prof_mark_begin(PROF_ATTN_FWD, st);
   if (dt == DT_BF16)
     launch(attn_fwd_kernel<__nv_bfloat16>, warps_blocks(w), 256, 0, st, 
         B, T, Tc, s, H, Hkv, (int)hd, (const __nv_bfloat16*)q, (const __nv_bfloat16*)Kp,
@@ -192,6 +197,7 @@ cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int
     launch(attn_fwd_kernel<float>, warps_blocks(w), 256, 0, st, 
         B, T, Tc, s, H, Hkv, (int)hd, (const float*)q, (const float*)Kp, (const float*)Vp,
         (float*)o, lse);
+  prof_mark_end(PROF_ATTN_FWD, st);
   return cudaGetLastError();
 }
 
@@ -215,16 +221,22 @@ cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int
                      const void* o, const void* dO, const float* lse, float* delta, float* dq,
                      float* dKp, float* dVp, cudaStream_t st, int path) {
   if (B * Tc * H <= 0) return cudaSuccess;
-  if (path != 1 && attn_bwd_tc_supported(hd, dt, q, Kp, Vp, o, dO, dq))
-    return attn_bwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, dO, lse, delta, dq, dKp, dVp,
-                       status_word(), st);
+  if (path != 1 && attn_bwd_tc_supported(hd, dt, q, Kp, Vp, o, dO, dq)) {
+    prof_mark_begin(PROF_ATTN_BWD, st);
+    const cudaError_t e = attn_bwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, dO, lse, delta, dq, dKp,
+                                      dVp, status_word(), st);
+    prof_mark_end(PROF_ATTN_BWD, st);
+    return e;
+  }
   if (path == 2) return cudaErrorNotSupported;
+  prof_mark_begin(PROF_ATTN_BWD, st);
   if (dt == DT_BF16)
     attn_bwd_launch<__nv_bfloat16>(B, T, Tc, s, H, Hkv, hd, q, Kp, Vp, o, dO, lse, delta, dq, dKp,
                                    dVp, st);
   else
     attn_bwd_launch<float>(B, T, Tc, s, H, Hkv, hd, q, Kp, Vp, o, dO, lse, delta, dq, dKp, dVp,
                            st);
+  prof_mark_end(PROF_ATTN_BWD, st);
   return cudaGetLastError();
 }
 

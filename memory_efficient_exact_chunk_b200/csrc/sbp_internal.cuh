@@ -16,7 +16,8 @@ namespace sbp {
 // ---------------------------------------------------------------------------------------------
 void prof_count_launch();
 bool prof_enabled();
-enum ProfKind : int { PROF_GEMM_TC = 0, PROF_GEMM_SIMT = 1, PROF_KINDS = 2 };
+enum ProfKind : int { PROF_GEMM_TC = 0, PROF_GEMM_SIMT = 1, PROF_ATTN_FWD = 2, PROF_ATTN_BWD = 3,
+                       PROF_KINDS = 4 };
 // events bracketing one launch of `kind` on `st` (no-ops unless profiling)
 void prof_mark_begin(int kind, cudaStream_t st);
 void prof_mark_end(int kind, cudaStream_t st);

@@ -40,7 +40,7 @@ class SbpError(RuntimeError):
 
 
 class Profile(C.Structure):
-    _fields_ = [("launches", C.c_longlong * 2), ("ms", C.c_double * 2)]
+    _fields_ = [("launches", C.c_longlong * 4), ("ms", C.c_double * 4)]
 
 
 class LayerCfg(C.Structure):
@@ -292,8 +292,8 @@ def profile_begin():
 def profile_end() -> dict:
     p = Profile()
     _check(load().sbp_profile_end(C.byref(p)))
-    return {"gemm_tc": {"launches": p.launches[0], "ms": p.ms[0]},
-            "gemm_simt": {"launches": p.launches[1], "ms": p.ms[1]}}
+    names = ("gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd")
+    return {n: {"launches": p.launches[i], "ms": p.ms[i]} for i, n in enumerate(names)}
 
 
 def debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=0, ws=None, stream=None):
