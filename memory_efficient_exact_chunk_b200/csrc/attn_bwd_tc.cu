@@ -14,7 +14,9 @@
 // an accumulator.
 //
 // Warp roles: warp 0 TMA producer (K, V once; Q and dO per pair), warp 1 TMEM owner + MMA
-// issuer, warps 2..5 element-wise + TMEM read-out (thread = key row, or query row for dQ).
+// issuer, warps 2..9 element-wise + TMEM read-out (thread = key row, or query row for dQ; the
+// warp's lane quarter is fixed by its index mod 4, the two warps of a quarter split the 128
+// columns in halves).
 #include <cuda.h>
 
 #include <mutex>
@@ -31,7 +33,8 @@ constexpr int BT = 128;                     // keys per key tile, queries per qu
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
 constexpr int SMEM_BYTES = 6 * TILE + 1024;  // K, V, Q, dO, P^T, dS^T + alignment
-constexpr int kThreads = 192;
+constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
+constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 384;
 
@@ -55,10 +58,15 @@ __device__ __forceinline__ void st_unit(uint8_t* tile, int r, int u, uint4 v) {
   const int chunk = u >> 3, uu = u & 7;
   *reinterpret_cast<uint4*>(tile + chunk * CHUNK + r * 128 + ((uu ^ (r & 7)) << 4)) = v;
 }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Bounded barrier of the four element-wise warps (an mbarrier with one arrival per warp that
+// Bounded barrier of the element-wise warps (an mbarrier with one arrival per warp that
 // completes once per use), so that a warp that gave up on a wait cannot strand the others.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t parity, int lane,
                                            volatile int* abort_flag) {
@@ -76,7 +84,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __shared__ uint64_t sync_a, sync_b;
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
-  __shared__ float lse_s[BT], delta_s[BT];
+  __shared__ __align__(16) float lse_s[BT];
+  __shared__ __align__(16) float delta_s[BT];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -107,12 +116,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc::mbar_init(&qd_full, 1);
     tc::mbar_init(&qd_empty, 1);
     tc::mbar_init(&sdp_full, 1);
-    tc::mbar_init(&ds_full, 4);
+    tc::mbar_init(&ds_full, kEwWarps);
     tc::mbar_init(&mma2_done, 1);
-    tc::mbar_init(&dq_free, 4);
+    tc::mbar_init(&dq_free, kEwWarps);
     tc::mbar_init(&drain, 1);
-    tc::mbar_init(&sync_a, 4);
-    tc::mbar_init(&sync_b, 4);
+    tc::mbar_init(&sync_a, kEwWarps);
+    tc::mbar_init(&sync_b, kEwWarps);
     abort_sh = 0;
     tc::fence_barrier_init();
   }
@@ -212,20 +221,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (npairs > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;                // column half of this warp
     const int r = q4 * 32 + lane;                    // TMEM lane = key row (or query row)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const int64_t kpos = k_lo + r;
+    const int kpos = (int)(k_lo + r);
     const float scale_log2 = a.scale * 1.4426950408889634f;
-    const int tid = threadIdx.x - 64;                // 0..127
+    const int tid = threadIdx.x - 64;                // 0..255
+    const int e32 = (int)e;
     bool ok = true;
     for (int j = 0; j < npairs; ++j) {
       const uint32_t ph = (uint32_t)j & 1u;
       int64_t hh, qi;
       pair_coords(j, hh, qi);
-      const int64_t q0 = a.s + qi * BT;              // absolute position of query column 0
-      // per-query statistics of this pair (thread tid loads query column tid)
+      const int q0 = (int)(a.s + qi * BT);           // absolute position of query column 0
+      // no masking needed when every key of the tile precedes every (valid) query of the tile
+      const bool full = (k_lo + BT - 1 <= q0) && (qi * BT + BT <= a.Tc);
+      // per-query statistics of this pair (thread tid < 128 loads query column tid)
       if (!group_sync(&sync_a, ph, lane, abort_flag)) { ok = false; break; }
-      {
+      if (tid < BT) {
         const int64_t ql = qi * BT + tid;           // position within the chunk
         const bool qv = ql < a.Tc;
         const int64_t gi = (b * a.Tc + ql) * a.H + hh;
@@ -236,27 +249,37 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (!tc::mbar_wait_warp(&sdp_full, ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;                 // 32-column slice
         uint32_t rs[32], rd[32];
         tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rs);
         tc::tmem_ld32(tmem + lane_off + C_DP + c * 32, rd);
         tc::tmem_ld_wait();
         uint32_t pp[16], dd[16];
+        const float4* l4 = reinterpret_cast<const float4*>(lse_s + c * 32);
+        const float4* d4 = reinterpret_cast<const float4*>(delta_s + c * 32);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pv[2], dv[2];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 lv = l4[i4], dv = d4[i4];
+          const float la[4] = {lv.x, lv.y, lv.z, lv.w};
+          const float da[4] = {dv.x, dv.y, dv.z, dv.w};
+          float p[4], g[4];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int col = c * 32 + i + k;
-            const int64_t qpos = q0 + col;
-            const bool live = (kpos <= qpos) && (qpos < e) && (kpos < e);
-            const float p = exp2f(__uint_as_float(rs[i + k]) * scale_log2 - lse_s[col]);
-            const float ds = p * (__uint_as_float(rd[i + k]) - delta_s[col]);
-            pv[k] = live ? p : 0.f;
-            dv[k] = live ? ds : 0.f;
+          for (int k = 0; k < 4; ++k) {
+            const int i = i4 * 4 + k;
+            p[k] = ex2(fmaf(__uint_as_float(rs[i]), scale_log2, -la[k]));
+            g[k] = p[k] * (__uint_as_float(rd[i]) - da[k]);
+            if (!full) {
+              const int qpos = q0 + c * 32 + i;
+              const bool live = (kpos <= qpos) && (qpos < e32);
+              p[k] = live ? p[k] : 0.f;
+              g[k] = live ? g[k] : 0.f;
+            }
           }
-          pp[i >> 1] = pack2(pv[0], pv[1]);
-          dd[i >> 1] = pack2(dv[0], dv[1]);
+          pp[i4 * 2] = pack2(p[0], p[1]);
+          pp[i4 * 2 + 1] = pack2(p[2], p[3]);
+          dd[i4 * 2] = pack2(g[0], g[1]);
+          dd[i4 * 2 + 1] = pack2(g[2], g[3]);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -276,7 +299,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const bool qv = ql < a.Tc;
         float* dqp = a.dq + ((b * a.Tc + ql) * a.H + hh) * HD;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;
           uint32_t rq[32];
           tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rq);
           tc::tmem_ld_wait();
@@ -298,10 +322,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     // dK, dV of this key tile: add into the fp32 prefix accumulators (single owner)
     if (ok) {
-      const bool kv = kpos < e;
+      const bool kv = kpos < e32;
       const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;
         uint32_t rk[32], rv[32];
         tc::tmem_ld32(tmem + lane_off + C_DK + c * 32, rk);
         tc::tmem_ld32(tmem + lane_off + C_DV + c * 32, rv);

@@ -47,7 +47,11 @@ struct FwdArgs {
   int* err;
 };
 
-__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -251,16 +255,28 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s_empty[sb]);
-      // scale into the exp2 domain, causal mask
+      // scale into the exp2 domain; only tiles that reach past the first query need the
+      // causal mask
       const int64_t k0 = (int64_t)j * BKV;
-      float mx = -INFINITY;
+      const bool diag = k0 + BKV - 1 > q_lo;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (diag) {
+        const int lim = (int)(t - k0);             // keys k0 + i with i > lim are masked
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float x = sv[i] * a.scale_log2;
-        if (k0 + i > t) x = -INFINITY;
-        sv[i] = x;
-        mx = fmaxf(mx, x);
+        for (int i = 0; i < 128; ++i) {
+          const float x = (i <= lim) ? sv[i] * a.scale_log2 : -INFINITY;
+          sv[i] = x;
+          m4[i & 3] = fmaxf(m4[i & 3], x);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float x = sv[i] * a.scale_log2;
+          sv[i] = x;
+          m4[i & 3] = fmaxf(m4[i & 3], x);
+        }
       }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       float corr = 1.f;
       bool rescale = false;
       if (mx > m_ref + kRescaleThreshold) {
@@ -270,15 +286,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         m_ref = mn;
         l *= corr;
       }
-      float sum = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const float p0 = fast_exp2(sv[2 * i] - m_ref);
         const float p1 = fast_exp2(sv[2 * i + 1] - m_ref);
-        sum += p0 + p1;
+        s4[i & 3] += p0 + p1;
         pk[i] = pack_bf16(p0, p1);
       }
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       l += sum;
       // P_j may overwrite P_{j-1} (and O may be rescaled) once O += P_{j-1} V_{j-1} is done
       if (j >= 1) {
@@ -333,7 +350,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
       }
-      if (row_ok) a.lse[grow * a.H + h] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (row_ok) a.lse[grow * a.H + h] = (m_ref + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
