@@ -4,9 +4,12 @@
 // One CTA owns (sequence b, KV head g, 128-key tile kt) and loops over the query heads of g's
 // group and the chunk's query tiles that can see those keys.  Per (query head, query tile):
 //   S^T  = K Q^T            (TMEM cols [0,128))      dP^T = V dO^T   (TMEM cols [128,256))
-//   P^T  = exp(S^T * scale - lse), dS^T = P^T (dP^T - delta)   -> bf16 tiles in shared memory
+//   P^T  = exp(S^T * scale - lse) -> bf16, written back into TMEM over the dP^T columns the
+//          same warp has already read (the A operand of the next product, read from TMEM)
+//   dS^T = P^T (dP^T - delta)     -> bf16 tile in shared memory
 //   dV  += P^T dO           (TMEM cols [256,384))    dK  += dS^T Q   (TMEM cols [384,512))
 //   dQ   = dS K             (TMEM cols [0,128) again) -> added to the fp32 dQ in global memory
+// Q and dO go through a two-stage ring, so the next pair's tiles load during this pair.
 // dK and dV stay in TMEM for the whole loop and are added once into the fp32 prefix
 // accumulators (single owner: deterministic); dQ receives one vector atomic add per query tile
 // and key tile.  Entries with key > query, queries outside the chunk and keys outside the
@@ -32,7 +35,8 @@ constexpr int HD = 128;
 constexpr int BT = 128;                     // keys per key tile, queries per query tile
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
-constexpr int SMEM_BYTES = 6 * TILE + 1024;  // K, V, Q, dO, P^T, dS^T + alignment
+constexpr int QD_STAGES = 2;
+constexpr int SMEM_BYTES = (3 + 2 * QD_STAGES) * TILE + 1024;  // K, V, dS^T, 2 x (Q, dO)
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
@@ -58,6 +62,29 @@ __device__ __forceinline__ void st_unit(uint8_t* tile, int r, int u, uint4 v) {
   const int chunk = u >> 3, uu = u & 7;
   *reinterpret_cast<uint4*>(tile + chunk * CHUNK + r * 128 + ((uu ^ (r & 7)) << 4)) = v;
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, f32 accumulate (A: 128 lanes x K/2 columns of
+// packed bf16 pairs, K-major).
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -80,7 +107,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                    const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t kv_full, qd_full, qd_empty, sdp_full, ds_full, mma2_done, dq_free, drain;
+  __shared__ uint64_t kv_full, qd_full[QD_STAGES], qd_empty[QD_STAGES], sdp_full, ds_full,
+      mma2_done, dq_free, drain;
   __shared__ uint64_t sync_a, sync_b;
   __shared__ uint32_t tmem_sh;
   __shared__ int abort_sh;
@@ -91,10 +119,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + TILE;
-  uint8_t* sQ = sV + TILE;
-  uint8_t* sdO = sQ + TILE;
-  uint8_t* sPt = sdO + TILE;
-  uint8_t* sdSt = sPt + TILE;
+  uint8_t* sdSt = sV + TILE;
+  uint8_t* sQ0 = sdSt + TILE;                    // stage st: Q at sQ0 + 2 st TILE, dO after it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
 
@@ -113,8 +139,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&kv_full, 1);
-    tc::mbar_init(&qd_full, 1);
-    tc::mbar_init(&qd_empty, 1);
+    for (int i = 0; i < QD_STAGES; ++i) {
+      tc::mbar_init(&qd_full[i], 1);
+      tc::mbar_init(&qd_empty[i], 1);
+    }
     tc::mbar_init(&sdp_full, 1);
     tc::mbar_init(&ds_full, kEwWarps);
     tc::mbar_init(&mma2_done, 1);
@@ -153,20 +181,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int j = 0; j < npairs; ++j) {
         int64_t hh, qi;
         pair_coords(j, hh, qi);
-        if (!tc::mbar_wait(&qd_empty, ((uint32_t)j & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        const int st = j % QD_STAGES;
+        const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
+        if (!tc::mbar_wait(&qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* sQ = sQ0 + 2 * st * TILE;
+        uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + qi * BT);
-        tc::mbar_expect_tx(&qd_full, 2 * TILE);
-        tc::tma_load_3d(sQ, &tmQ, &qd_full, 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sQ + CHUNK, &tmQ, &qd_full, 64, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO, &tmdO, &qd_full, 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO + CHUNK, &tmdO, &qd_full, 64, (int32_t)hh, qrow);
+        tc::mbar_expect_tx(&qd_full[st], 2 * TILE);
+        tc::tma_load_3d(sQ, &tmQ, &qd_full[st], 0, (int32_t)hh, qrow);
+        tc::tma_load_3d(sQ + CHUNK, &tmQ, &qd_full[st], 64, (int32_t)hh, qrow);
+        tc::tma_load_3d(sdO, &tmdO, &qd_full[st], 0, (int32_t)hh, qrow);
+        tc::tma_load_3d(sdO + CHUNK, &tmdO, &qd_full[st], 64, (int32_t)hh, qrow);
         issued = j + 1;
       }
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-        if (issued > 0)
-          while (!tc::mbar_try_wait(&qd_full, (uint32_t)(issued - 1) & 1u) &&
+        for (int j = issued > QD_STAGES ? issued - QD_STAGES : 0; j < issued; ++j)
+          while (!tc::mbar_try_wait(&qd_full[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }
     }
@@ -176,13 +208,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t id_kk = tc::idesc_bf16_f32(128, 128, 0, 0);   // A K-major, B K-major
       const uint32_t id_km = tc::idesc_bf16_f32(128, 128, 0, 1);   // A K-major, B MN-major
       const uint32_t id_mm = tc::idesc_bf16_f32(128, 128, 1, 1);   // A MN-major, B MN-major
-      const uint32_t aK = tc::smem_u32(sK), aV = tc::smem_u32(sV), aQ = tc::smem_u32(sQ),
-                     adO = tc::smem_u32(sdO), aPt = tc::smem_u32(sPt), adS = tc::smem_u32(sdSt);
+      const uint32_t aK = tc::smem_u32(sK), aV = tc::smem_u32(sV), adS = tc::smem_u32(sdSt),
+                     aQ0 = tc::smem_u32(sQ0);
       bool ok = tc::mbar_wait(&kv_full, 0, abort_flag);
       bool issued = false;
       for (int j = 0; j < npairs && ok; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
-        if (!tc::mbar_wait(&qd_full, ph, abort_flag)) { ok = false; break; }
+        const int st = j % QD_STAGES;
+        const uint32_t sph = (uint32_t)(j / QD_STAGES) & 1u;
+        const uint32_t aQ = aQ0 + 2 * st * TILE, adO = aQ + TILE;
+        if (!tc::mbar_wait(&qd_full[st], sph, abort_flag)) { ok = false; break; }
         if (j >= 1 && !tc::mbar_wait(&dq_free, ph ^ 1u, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
@@ -202,15 +237,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;   // K-major operand step
           const uint32_t offm = kk * 2048;                            // MN-major operand step
           const uint32_t acc = (j | kk) != 0;
-          tc::mma_f16_ss(tmem + C_DV, tc::smem_desc_sw128(aPt + offk, 16, 1024),
-                         tc::smem_desc_sw128(adO + offm, CHUNK, 1024), id_km, acc);
+          // P^T (packed bf16) sits in TMEM: queries 64h.. of half h at C_DP + 64 h
+          const uint32_t pcol = C_DP + 64 * (kk >> 2) + 8 * (kk & 3);
+          mma_f16_ts(tmem + C_DV, tmem + pcol, tc::smem_desc_sw128(adO + offm, CHUNK, 1024),
+                     id_km, acc);
           tc::mma_f16_ss(tmem + C_DK, tc::smem_desc_sw128(adS + offk, 16, 1024),
                          tc::smem_desc_sw128(aQ + offm, CHUNK, 1024), id_km, acc);
           tc::mma_f16_ss(tmem + C_S, tc::smem_desc_sw128(adS + offm, CHUNK, 1024),
                          tc::smem_desc_sw128(aK + offm, CHUNK, 1024), id_mm, kk != 0);
         }
         tc::mma_commit(&mma2_done);
-        tc::mma_commit(&qd_empty);
+        tc::mma_commit(&qd_empty[st]);
       }
       if (issued) {
         tc::mma_commit(&drain);
@@ -281,12 +318,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           dd[i4 * 2] = pack2(g[0], g[1]);
           dd[i4 * 2 + 1] = pack2(g[2], g[3]);
         }
+        // packed P over dP^T columns this warp has already read (queries 32 cc .. of its half)
+        tmem_st16(tmem + lane_off + C_DP + 64 * half + 16 * cc, pp);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          st_unit(sPt, r, c * 4 + u, make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]));
+        for (int u = 0; u < 4; ++u)
           st_unit(sdSt, r, c * 4 + u, make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
-        }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
