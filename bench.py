@@ -278,6 +278,82 @@ def run_layer(args, rank, world, device, sweep=False):
     return out
 
 
+def run_stack(args, rank, world, device):
+    """Four Llama-3-8B-shaped layers + untied LM head (vocab 128256), bf16, T = 65536, D = 16,
+    targets = next token, mean CE over the last 75 % of tokens.  Weights are drawn on the
+    device from a seeded generator (N(0, 0.02), gains 1).  The forward (layer-input
+    checkpoints) and the streamed backward are timed separately; the metric is the backward."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp, stack, synth
+    wl = synth.WORKLOADS["llama3_8b_stack4_64k"]
+    L, B, T, V = wl.layer, wl.batch, (args.stack_tokens or wl.seq_len), wl.vocab
+    D = wl.num_chunks
+    gen = torch.Generator(device=device).manual_seed(3000 + rank)
+
+    def rnd(*shape):
+        return (torch.randn(*shape, generator=gen, device=device) * 0.02).to(torch.bfloat16)
+
+    d, dq, dkv, f = L.d_model, L.n_heads * L.head_dim, L.n_kv_heads * L.head_dim, L.ffn
+    layers = []
+    for _ in range(wl.n_layers):
+        layers.append({"ln1_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+                       "wq": rnd(dq, d), "wk": rnd(dkv, d), "wv": rnd(dkv, d), "wo": rnd(d, dq),
+                       "ln2_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+                       "w_gate": rnd(f, d), "w_up": rnd(f, d), "w_down": rnd(d, f),
+                       "bq": None, "bk": None, "bv": None})
+    embed = rnd(V, d)
+    lm_w = rnd(V, d)
+    final_g = torch.ones(d, dtype=torch.bfloat16, device=device)
+    rng = np.random.default_rng(3000 + rank)
+    ids = synth.token_ids(rng, B, T, V)
+    y = synth.shifted_targets(ids)
+    w = synth.loss_weights("shifted_tail", B, T, from_frac=wl.loss_from_frac)
+    n_loss = int(np.count_nonzero(w))
+    ids_d = torch.from_numpy(ids.reshape(-1)).to(device)
+    y_d = torch.from_numpy(y.reshape(-1)).to(device)
+    w_d = torch.from_numpy(w.reshape(-1)).to(device)
+    cfg = sbp.layer_cfg(B, T, d, L.n_heads, L.n_kv_heads, L.head_dim, f, L.rms_eps,
+                        L.rope_theta, sbp.SBP_BF16, D)
+    ws = stack.Workspaces(device)
+    grads = stack.zero_grads(layers, lm_w, final_g, device, embed_shape=embed.shape)
+    state = {}
+
+    def fwd():
+        state["ck"] = stack.stack_forward(cfg, embed, layers, final_g, ids_d, ws)
+
+    def bwd():
+        xs, hf, rstd = state["ck"]
+        stack.stack_backward_from(cfg, layers, final_g, lm_w, ids_d, y_d, w_d, xs, hf, rstd, ws,
+                                  grads=grads)
+
+    fwd()
+    sargs = argparse.Namespace(steps=1, warmup=args.warmup)
+    rb = timed(sargs, bwd, world, device, profile=True)
+    rf = timed(argparse.Namespace(steps=1, warmup=1), fwd, world, device, profile=False)
+    P = sum(int(layers[0][n].numel()) for n in ("wq", "wk", "wv", "wo", "w_gate", "w_up",
+                                                "w_down"))
+    lin = 6.0 * P * B * T * wl.n_layers
+    att = 14.0 * L.head_dim * L.n_heads * B * T * (T + 1) / 2 * wl.n_layers
+    head = 8.0 * n_loss * d * V
+    prof = rb["prof"]
+    return {
+        "workload": wl.name if T == wl.seq_len else f"llama3_8b_stack4_{T}",
+        "value": B * T * world / (rb["ms"] / 1e3), "unit": "tokens/s",
+        "ms_per_step": rb["ms"], "forward_ms": rf["ms"],
+        "fwd_bwd_tokens_per_s": B * T * world / ((rb["ms"] + rf["ms"]) / 1e3),
+        "config": {"batch": B, "seq_len": T, "n_layers": wl.n_layers, "vocab": V,
+                   "num_chunks": D, "n_loss_tokens": n_loss},
+        "flops_step": {"layers_linear_6P": lin, "layers_attention_14hd": att,
+                       "lmhead_8NdV": head},
+        "achieved_tflops_step": (lin + att + head) / (rb["ms"] / 1e3) / 1e12,
+        "kernels": {n: {"launches_per_step": v["launches"], "ms_per_step": v["ms"],
+                        "share": v["ms"] / rb["ms_total"] if rb["ms_total"] else None}
+                    for n, v in prof.items() if v["launches"]},
+        "gpu_launches": rb["launches"], "clocks": rb["clocks"],
+        "workspace_gb": sum(t.numel() for t in ws.bufs.values()) / 1e9,
+    }
+
+
 def timed(args, step, world, device, profile):
     """W warm-up steps, then K timed steps between a barrier + synchronize on both sides;
     device time from CUDA events on the launching stream, max over ranks."""
@@ -414,6 +490,9 @@ def main():
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the decoder-layer measurement added to the line")
     ap.add_argument("--layer-tokens", type=int, default=0)
+    ap.add_argument("--no-stack", dest="stack", action="store_false",
+                    help="skip the 4-layer stack measurement added to the line")
+    ap.add_argument("--stack-tokens", type=int, default=0)
     ap.add_argument("--layer-chunks", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -472,8 +551,15 @@ def main():
     }
     if "sweep" in out:
         line["sweep"] = out["sweep"]
+    also = []
     if args.layer:
-        line["also"] = [run_layer(args, rank, world, device, sweep=args.sweep)]
+        also.append(run_layer(args, rank, world, device, sweep=args.sweep))
+    if args.stack:
+        import torch
+        torch.cuda.empty_cache()
+        also.append(run_stack(args, rank, world, device))
+    if also:
+        line["also"] = also
     if "e2e" in out:
         line["e2e"] = out["e2e"]
     if args.cpu and rank == 0 and world == 1:

@@ -21,57 +21,92 @@ class StackResult:
     grads: Dict[str, object]    # lm_head, final_g, embed, layers: List[dict]
 
 
-def stack_backward(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, lm_w, ids, targets,
-                   loss_weights, stream=None, keep_workspace: dict | None = None) -> StackResult:
-    """ids/targets int32 [B*T]; loss_weights fp32 [B*T]; weights on the device in cfg.dtype.
-    Returns the loss and fp32 gradients (freshly zeroed, then accumulated by the library)."""
-    import torch
-    dev = embed.device
-    B, T, d = cfg.batch, cfg.seq_len, cfg.d_model
-    N = B * T
-    V = lm_w.shape[0]
-    wdt = embed.dtype
-    ws_cache = keep_workspace if keep_workspace is not None else {}
+class Workspaces:
+    """Device buffers reused across calls (grown on demand)."""
 
-    def ws(name, nbytes):
-        t = ws_cache.get(name)
+    def __init__(self, device):
+        self.device = device
+        self.bufs = {}
+
+    def get(self, name, nbytes):
+        t = self.bufs.get(name)
         if t is None or t.numel() < nbytes:
-            t = sbp.workspace(nbytes, dev)
-            ws_cache[name] = t
+            t = sbp.workspace(nbytes, self.device)
+            self.bufs[name] = t
         return t
 
-    lws = ws("layer", sbp.layer_workspace_size(cfg))
-    # ---- forward: keep the input of every layer
-    xs = [torch.empty(N, d, dtype=wdt, device=dev)]
+
+def stack_forward(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, ids, ws: Workspaces,
+                  stream=None):
+    """Embedding and L chunked layer forwards; returns the layer inputs (checkpoints), the
+    final-norm output and its rstd."""
+    import torch
+    dev = embed.device
+    N = cfg.batch * cfg.seq_len
+    d = cfg.d_model
+    xs = [torch.empty(N, d, dtype=embed.dtype, device=dev)]
     sbp.embedding_forward(ids, embed, xs[0], stream=stream)
+    lws = ws.get("layer", sbp.layer_workspace_size(cfg))
     for W in layers:
-        y = torch.empty(N, d, dtype=wdt, device=dev)
+        y = torch.empty(N, d, dtype=embed.dtype, device=dev)
         sbp.decoder_layer_forward(cfg, W, xs[-1], y, ws=lws, stream=stream)
         xs.append(y)
-    hf = torch.empty(N, d, dtype=wdt, device=dev)
+    hf = torch.empty(N, d, dtype=embed.dtype, device=dev)
     rstd = torch.empty(N, dtype=torch.float32, device=dev)
     sbp.rmsnorm_forward(xs[-1], final_g, cfg.rms_eps, hf, rstd, stream=stream)
-    # ---- backward
+    return xs, hf, rstd
+
+
+def stack_backward_from(cfg: sbp.LayerCfg, layers: List[dict], final_g, lm_w, ids, targets,
+                        loss_weights, xs, hf, rstd, ws: Workspaces, grads=None, stream=None):
+    """The streamed backward of the stack from its checkpoints.  `grads` (optional) holds fp32
+    gradient buffers to accumulate into (the layout StackResult.grads uses); else fresh zeros."""
+    import torch
+    dev = hf.device
+    N, d = hf.shape
+    V = lm_w.shape[0]
+    if grads is None:
+        grads = zero_grads(layers, lm_w, final_g, dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     dhf = torch.empty(N, d, dtype=torch.float32, device=dev)
-    dlm = torch.zeros(V, d, dtype=torch.float32, device=dev)
-    cws = ws("lmhead", sbp.lmhead_ce_workspace_size(N, d, V, cfg.num_chunks,
-                                                    sbp._dtype_code(hf)))
-    sbp.lmhead_ce_backward(hf, lm_w, targets, loss_weights, cfg.num_chunks, loss, dhf, dlm,
-                           ws=cws, stream=stream)
-    dfg = torch.zeros(d, dtype=torch.float32, device=dev)
+    cws = ws.get("lmhead", sbp.lmhead_ce_workspace_size(N, d, V, cfg.num_chunks,
+                                                        sbp._dtype_code(hf)))
+    sbp.lmhead_ce_backward(hf, lm_w, targets, loss_weights, cfg.num_chunks, loss, dhf,
+                           grads["lm_head"], ws=cws, stream=stream)
     dx = torch.empty(N, d, dtype=torch.float32, device=dev)
-    sbp.rmsnorm_backward(xs[-1], final_g, rstd, dhf, dx, dfg, ws=ws("rms", 0), stream=stream)
-    layer_grads: List[dict] = [None] * len(layers)
+    sbp.rmsnorm_backward(xs[-1], final_g, rstd, dhf, dx, grads["final_g"],
+                         ws=ws.get("rms", 0), stream=stream)
+    lws = ws.get("layer", sbp.layer_workspace_size(cfg))
+    dxn = dhf                                        # reuse the buffer: dhf is consumed
     for li in range(len(layers) - 1, -1, -1):
-        W = layers[li]
-        g = {n: (torch.zeros(W[n].shape, dtype=torch.float32, device=dev)
-                 if W.get(n) is not None else None) for n in sbp.WEIGHT_FIELDS}
-        dxn = torch.empty(N, d, dtype=torch.float32, device=dev)
-        sbp.decoder_layer_backward(cfg, W, xs[li], dx, dxn, g, ws=lws, stream=stream)
-        layer_grads[li] = g
-        dx = dxn
-    dE = torch.zeros(embed.shape, dtype=torch.float32, device=dev)
-    sbp.embedding_backward(ids, dx, dE, ws=ws("embed", 0), stream=stream)
-    return StackResult(loss, {"lm_head": dlm, "final_g": dfg, "embed": dE,
-                              "layers": layer_grads})
+        sbp.decoder_layer_backward(cfg, layers[li], xs[li], dx, dxn, grads["layers"][li],
+                                   ws=lws, stream=stream)
+        dx, dxn = dxn, dx
+    sbp.embedding_backward(ids, dx, grads["embed"], ws=ws.get("embed", 0), stream=stream)
+    return StackResult(loss, grads)
+
+
+def zero_grads(layers, lm_w, final_g, dev, embed_shape=None):
+    import torch
+    g = {"lm_head": torch.zeros(lm_w.shape, dtype=torch.float32, device=dev),
+         "final_g": torch.zeros(final_g.shape, dtype=torch.float32, device=dev),
+         "layers": [{n: (torch.zeros(W[n].shape, dtype=torch.float32, device=dev)
+                         if W.get(n) is not None else None) for n in sbp.WEIGHT_FIELDS}
+                    for W in layers]}
+    if embed_shape is not None:
+        g["embed"] = torch.zeros(embed_shape, dtype=torch.float32, device=dev)
+    return g
+
+
+def stack_backward(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, lm_w, ids, targets,
+                   loss_weights, stream=None, keep_workspace: dict | None = None) -> StackResult:
+    """Forward (checkpoints only) and streamed backward of the whole stack.
+    ids/targets int32 [B*T]; loss_weights fp32 [B*T]; weights on the device in cfg.dtype.
+    Returns the loss and fp32 gradients (freshly zeroed, then accumulated by the library)."""
+    ws = Workspaces(embed.device)
+    if keep_workspace is not None:
+        ws.bufs = keep_workspace
+    xs, hf, rstd = stack_forward(cfg, embed, layers, final_g, ids, ws, stream=stream)
+    grads = zero_grads(layers, lm_w, final_g, embed.device, embed_shape=embed.shape)
+    return stack_backward_from(cfg, layers, final_g, lm_w, ids, targets, loss_weights, xs, hf,
+                               rstd, ws, grads=grads, stream=stream)
