@@ -22,6 +22,173 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
+// ---------------------------------------------------------------- 8-wide vector access
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+  uint4 q;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = q;
+}
+
+// RMSNorm forward, 8 columns per access (cols % 8 == 0, 16-byte aligned rows)
+template <typename TX, typename TG, typename TY>
+__global__ void rmsnorm_fwd_vec_kernel(int64_t cols, const TX* __restrict__ x,
+                                       const TG* __restrict__ g, TY* __restrict__ y,
+                                       float* __restrict__ rstd, float eps) {
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  const TX* xr = x + r * cols;
+  float ss = 0.f;
+  for (int64_t c = 8 * threadIdx.x; c < cols; c += 8 * blockDim.x) {
+    float v[8];
+    load8(xr + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
+  }
+  ss = block_sum(ss, red);
+  const float rs = rsqrtf(ss / (float)cols + eps);
+  for (int64_t c = 8 * threadIdx.x; c < cols; c += 8 * blockDim.x) {
+    float v[8], gv[8];
+    load8(xr + c, v);
+    load8(g + c, gv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = v[i] * rs * gv[i];
+    store8(y + r * cols + c, v);
+  }
+  if (rstd && threadIdx.x == 0) rstd[r] = rs;
+}
+
+// RMSNorm backward, 8 columns per access; each thread keeps the dg partial of its columns in
+// registers (at most kVecChunks 8-column chunks per thread).
+constexpr int kVecChunks = 4;
+template <typename TX, typename TG>
+__global__ void rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __restrict__ x,
+                                       const TG* __restrict__ g, const float* __restrict__ rstd,
+                                       const float* __restrict__ dy,
+                                       const float* __restrict__ base, float* __restrict__ out,
+                                       int accumulate, float* __restrict__ partial) {
+  __shared__ float red[32];
+  float dg[kVecChunks][8];
+  float gv[kVecChunks][8];
+#pragma unroll
+  for (int k = 0; k < kVecChunks; ++k) {
+    const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dg[k][i] = 0.f;
+    if (c < cols) load8(g + c, gv[k]);
+  }
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int64_t o = r * cols;
+    const float rs = rstd[r];
+    float xh[kVecChunks][8], u[kVecChunks][8];
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kVecChunks; ++k) {
+      const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+      if (c >= cols) continue;
+      float xv[8], dv[8];
+      load8(x + o + c, xv);
+      load8(dy + o + c, dv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        xh[k][i] = xv[i] * rs;
+        u[k][i] = dv[i] * gv[k][i];
+        dot = fmaf(xh[k][i], u[k][i], dot);
+        dg[k][i] = fmaf(dv[i], xh[k][i], dg[k][i]);
+      }
+    }
+    dot = block_sum(dot, red) / (float)cols;
+#pragma unroll
+    for (int k = 0; k < kVecChunks; ++k) {
+      const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+      if (c >= cols) continue;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = rs * (u[k][i] - xh[k][i] * dot);
+      if (base) {
+        float b[8];
+        load8(base + o + c, b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += b[i];
+      }
+      if (accumulate) {
+        float b[8];
+        load8(out + o + c, b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += b[i];
+      }
+      store8(out + o + c, v);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kVecChunks; ++k) {
+    const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+    if (c < cols) store8(partial + (int64_t)blockIdx.x * cols + c, dg[k]);
+  }
+}
+
+// y = x (cast), 8 per thread
+template <typename TS, typename TD>
+__global__ void copy_cast_vec_kernel(int64_t n8, const TS* __restrict__ src, TD* __restrict__ dst) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  float v[8];
+  load8(src + 8 * i, v);
+  store8(dst + 8 * i, v);
+}
+
+__global__ void split_bf16_vec_kernel(int64_t n8, const float* __restrict__ x,
+                                      __nv_bfloat16* __restrict__ hi,
+                                      __nv_bfloat16* __restrict__ lo) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  float v[8], h[8], l[8];
+  load8(x + 8 * i, v);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    h[k] = __bfloat162float(__float2bfloat16_rn(v[k]));
+    l[k] = v[k] - h[k];
+  }
+  store8(hi + 8 * i, h);
+  store8(lo + 8 * i, l);
+}
+
+__global__ void swiglu_fwd_vec_kernel(int64_t R, int64_t f, const __nv_bfloat16* __restrict__ gu,
+                                      __nv_bfloat16* __restrict__ m) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // 8-column group
+  const int64_t f8 = f / 8;
+  if (i >= R * f8) return;
+  const int64_t r = i / f8, c = 8 * (i % f8);
+  float gv[8], uv[8], o[8];
+  load8(gu + r * 2 * f + c, gv);
+  load8(gu + r * 2 * f + f + c, uv);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) o[k] = gv[k] / (1.f + expf(-gv[k])) * uv[k];
+  store8(m + r * f + c, o);
+}
+
+inline bool al16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // ---------------------------------------------------------------- RMSNorm forward
 __global__ void rmsnorm_fwd_kernel(int64_t cols, int xdt, const void* __restrict__ x, int gdt,
                                    const void* __restrict__ g, int ydt, void* __restrict__ y,
@@ -366,6 +533,18 @@ cudaError_t rmsnorm_fwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
                         const void* g, int ydt, void* y, float* rstd, float eps,
                         cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  if (cols % 8 == 0 && gdt == DT_BF16 && ydt == DT_BF16 && al16p(x) && al16p(g) && al16p(y)) {
+    const auto* gb = static_cast<const __nv_bfloat16*>(g);
+    auto* yb = static_cast<__nv_bfloat16*>(y);
+    if (xdt == DT_BF16)
+      launch(rmsnorm_fwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>,
+             dim3((unsigned)rows), dim3(kRowThreads), 0, st, cols,
+             static_cast<const __nv_bfloat16*>(x), gb, yb, rstd, eps);
+    else
+      launch(rmsnorm_fwd_vec_kernel<float, __nv_bfloat16, __nv_bfloat16>, dim3((unsigned)rows),
+             dim3(kRowThreads), 0, st, cols, static_cast<const float*>(x), gb, yb, rstd, eps);
+    return cudaGetLastError();
+  }
   launch(rmsnorm_fwd_kernel, (unsigned)rows, kRowThreads, 0, st, cols, xdt, x, gdt, g, ydt, y, rstd,
                                                              eps);
   return cudaGetLastError();
@@ -378,6 +557,23 @@ cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
                         float* out, int accumulate, float* dg, float* partial,
                         cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  if (cols % 8 == 0 && cols <= 8 * kRowThreads * kVecChunks && gdt == DT_BF16 && al16p(x) &&
+      al16p(g) && al16p(dy) && al16p(out) && (!base || al16p(base))) {
+    const auto* gb = static_cast<const __nv_bfloat16*>(g);
+    if (xdt == DT_BF16)
+      launch(rmsnorm_bwd_vec_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(kBwdBlocks),
+             dim3(kRowThreads), 0, st, rows, cols, static_cast<const __nv_bfloat16*>(x), gb,
+             rstd, dy, base, out, accumulate, partial);
+    else
+      launch(rmsnorm_bwd_vec_kernel<float, __nv_bfloat16>, dim3(kBwdBlocks), dim3(kRowThreads),
+             0, st, rows, cols, static_cast<const float*>(x), gb, rstd, dy, base, out,
+             accumulate, partial);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || !dg) return e;
+    launch(colsum_partials_kernel, dim3(nblk(cols, 256)), dim3(256), 0, st, (int64_t)kBwdBlocks,
+           cols, (const float*)partial, dg);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)cols * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(rmsnorm_bwd_kernel,
@@ -433,6 +629,12 @@ cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t
 
 cudaError_t swiglu_fwd(int64_t R, int64_t f, int dt, const void* gu, void* m, cudaStream_t st) {
   if (R * f <= 0) return cudaSuccess;
+  if (dt == DT_BF16 && f % 8 == 0 && al16p(gu) && al16p(m)) {
+    const int64_t n = R * (f / 8);
+    launch(swiglu_fwd_vec_kernel, dim3(nblk(n, 256)), dim3(256), 0, st, R, f,
+           static_cast<const __nv_bfloat16*>(gu), static_cast<__nv_bfloat16*>(m));
+    return cudaGetLastError();
+  }
   launch(swiglu_fwd_kernel, nblk(R * f, 256), 256, 0, st, R, f, dt, gu, m);
   return cudaGetLastError();
 }
@@ -489,6 +691,11 @@ cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int 
 
 cudaError_t split_bf16(int64_t n, const float* x, void* hi, void* lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
+  if (n % 8 == 0 && al16p(x) && al16p(hi) && al16p(lo)) {
+    launch(split_bf16_vec_kernel, dim3(nblk(n / 8, 256)), dim3(256), 0, st, n / 8, x,
+           static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+    return cudaGetLastError();
+  }
   launch(split_bf16_kernel, nblk(n, 256), 256, 0, st, n, x, static_cast<__nv_bfloat16*>(hi),
                                                   static_cast<__nv_bfloat16*>(lo));
   return cudaGetLastError();
@@ -496,6 +703,23 @@ cudaError_t split_bf16(int64_t n, const float* x, void* hi, void* lo, cudaStream
 
 cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
+  if (n % 8 == 0 && al16p(src) && al16p(dst)) {
+    const int64_t n8 = n / 8;
+    const dim3 grid(nblk(n8, 256)), blk(256);
+    if (sdt == DT_F32 && ddt == DT_BF16)
+      launch(copy_cast_vec_kernel<float, __nv_bfloat16>, grid, blk, 0, st, n8,
+             static_cast<const float*>(src), static_cast<__nv_bfloat16*>(dst));
+    else if (sdt == DT_BF16 && ddt == DT_F32)
+      launch(copy_cast_vec_kernel<__nv_bfloat16, float>, grid, blk, 0, st, n8,
+             static_cast<const __nv_bfloat16*>(src), static_cast<float*>(dst));
+    else if (sdt == DT_F32 && ddt == DT_F32)
+      launch(copy_cast_vec_kernel<float, float>, grid, blk, 0, st, n8,
+             static_cast<const float*>(src), static_cast<float*>(dst));
+    else
+      launch(copy_cast_vec_kernel<__nv_bfloat16, __nv_bfloat16>, grid, blk, 0, st, n8,
+             static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst));
+    return cudaGetLastError();
+  }
   launch(copy_cast_kernel, nblk(n, 256), 256, 0, st, n, sdt, src, ddt, dst);
   return cudaGetLastError();
 }

@@ -93,6 +93,25 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
     }
     return;
   }
+  if (g.epi == EPI_SWIGLU_BWD) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t m = m0 + ty + 16 * i;
+      if (m >= M) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t n = n0 + tx + 16 * j;
+        if (n >= N) continue;
+        const float dm = g.alpha * acc[i][j];
+        const float gv = ld_dt(g.aux, g.cdt, m * g.aux_ld + n);
+        const float uv = ld_dt(g.aux, g.cdt, m * g.aux_ld + g.aux_off + n);
+        const float sg = 1.f / (1.f + expf(-gv));
+        st_dt(g.C, g.cdt, m * g.ldc + n, dm * uv * sg * (1.f + gv * (1.f - sg)));
+        st_dt(g.C, g.cdt, m * g.ldc + g.aux_off + n, dm * gv * sg);
+      }
+    }
+    return;
+  }
   if (g.epi == EPI_CEGRAD) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

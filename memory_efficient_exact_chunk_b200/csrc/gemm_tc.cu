@@ -103,6 +103,45 @@ __device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int6
   }
 }
 
+__device__ __forceinline__ float silu_grad_parts(float dm, float gv, float uv, float* du) {
+  const float sg = 1.f / (1.f + __expf(-gv));
+  *du = dm * gv * sg;
+  return dm * uv * sg * (1.f + gv * (1.f - sg));
+}
+
+// SwiGLU backward for 32 consecutive columns: v = dM, g / u from aux (bf16), results to C (bf16).
+__device__ __forceinline__ void epi_swiglu_bwd32(const GemmDesc& g, int64_t m, int64_t n,
+                                                 int64_t N, const float (&v)[32]) {
+  const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(g.aux) + m * g.aux_ld + n;
+  const __nv_bfloat16* up = gp + g.aux_off;
+  __nv_bfloat16* dgp = static_cast<__nv_bfloat16*>(g.C) + m * g.ldc + n;
+  __nv_bfloat16* dup = dgp + g.aux_off;
+  if (n + 32 <= N) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 gq = *reinterpret_cast<const uint4*>(gp + 8 * q);
+      const uint4 uq = *reinterpret_cast<const uint4*>(up + 8 * q);
+      const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
+      const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&uq);
+      float dg[8], du[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dg[i] = silu_grad_parts(v[8 * q + i], __bfloat162float(gb[i]), __bfloat162float(ub[i]),
+                                &du[i]);
+      store8_bf16(dgp + 8 * q, dg);
+      store8_bf16(dup + 8 * q, du);
+    }
+  } else {
+    for (int i = 0; i < 32 && n + i < N; ++i) {
+      float du;
+      const float dg = silu_grad_parts(v[i], __bfloat162float(gp[i]), __bfloat162float(up[i]),
+                                       &du);
+      dgp[i] = __float2bfloat16_rn(dg);
+      dup[i] = __float2bfloat16_rn(du);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcArgs args) {
@@ -319,6 +358,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = nk ? u2f(r[j]) : 0.f;
+          if (g.epi == EPI_SWIGLU_BWD) {
+            epi_swiglu_bwd32(g, m, nc, N, v);
+            continue;
+          }
           if (g.epi == EPI_CEGRAD) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -409,9 +452,13 @@ bool gemm_tc_supported(const GemmDesc& g) {
   const bool b_n = g.sbn == 1 && g.sbk % 8 == 0 && g.sbk > 0;
   if (!(a_k || a_m) || !(b_k || b_n)) return false;
   if (!al16(g.A) || !al16(g.B)) return false;
-  if (g.epi == EPI_STORE || g.epi == EPI_ACC || g.epi == EPI_CEGRAD) {
+  if (g.epi == EPI_STORE || g.epi == EPI_ACC || g.epi == EPI_CEGRAD ||
+      g.epi == EPI_SWIGLU_BWD) {
     if (!al16(g.C) || g.ldc % 8 != 0) return false;
   }
+  if (g.epi == EPI_SWIGLU_BWD &&
+      (g.cdt != DT_BF16 || !al16(g.aux) || g.aux_ld % 8 != 0 || g.aux_off % 8 != 0))
+    return false;
   if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX)
     return false;
   return encode_fn() != nullptr;

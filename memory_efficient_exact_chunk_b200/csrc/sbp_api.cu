@@ -104,7 +104,7 @@ struct LayerPlan {
   void *Kp, *Vp;
   float *dKp, *dVp;
   void *xg, *n1, *q, *o, *n2, *gu, *m, *dgu, *dO;
-  float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dm, *dn2, *dh, *delta, *dq, *dn1, *dxg;
+  float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dn2, *dh, *delta, *dq, *dn1, *dxg;
   float *dkpre, *dvg, *rpart, *cpart;
   // bf16 operand copies of fp32 gradients (bf16 path only)
   void *dyg16, *dh16, *dq16, *dqlo, *khi, *klo, *vhi, *vlo;
@@ -138,7 +138,6 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.rstd2 = c.take<float>(R);
   p.gu = c.take_bytes((size_t)R * 2 * f * es);
   p.m = c.take_bytes((size_t)R * f * es);
-  p.dm = c.take<float>((size_t)R * f);
   p.dgu = c.take_bytes((size_t)R * 2 * f * es);
   p.dn2 = c.take<float>((size_t)R * d);
   p.dh = c.take<float>((size_t)R * d);
@@ -222,15 +221,16 @@ sbp_status check_weights(const sbp_layer_weights* w, bool* has_bias) {
 }
 
 // Forward recompute of one chunk: fills n1, rstd1, q, K/V prefix rows, o, alse, hbuf (= h),
-// n2, rstd2, gu and m.  xg holds the chunk's gathered input.
+// n2, rstd2, gu and m.  xc is the chunk's input rows [B * Tc, d] (contiguous).
 sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& w,
-                               const LayerPlan& p, int64_t s, int64_t Tc, cudaStream_t st) {
+                               const LayerPlan& p, const void* xc, int64_t s, int64_t Tc,
+                               cudaStream_t st) {
   const int dt = L.dtype;
   const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
   const int64_t H = L.n_heads, Hkv = L.n_kv_heads, hd = L.head_dim;
   const int64_t dq = H * hd, dkv = Hkv * hd, W3 = dq + 2 * dkv;
   const int64_t R = B * Tc;
-  SBP_CK(rmsnorm_fwd(R, d, dt, p.xg, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+  SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
   {
     GemmDesc g = mk_gemm(R, dq, d, dt, p.n1, false, d, dt, w.wq, true, d, DT_F32, p.qkv, W3,
                          EPI_STORE);
@@ -247,7 +247,7 @@ sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& 
   }
   SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
   SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, st));
-  SBP_CK(copy_cast(R * d, dt, p.xg, DT_F32, p.hbuf, st));
+  SBP_CK(copy_cast(R * d, dt, xc, DT_F32, p.hbuf, st));
   SBP_CK(gemm(mk_gemm(R, d, dq, dt, p.o, false, dq, dt, w.wo, true, dq, DT_F32, p.hbuf, d,
                       EPI_ACC), st));
   SBP_CK(rmsnorm_fwd(R, d, DT_F32, p.hbuf, dt, w.ln2_g, dt, p.n2, p.rstd2, L.rms_eps, st));
@@ -442,24 +442,40 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     int64_t s, e;
     chunk_range(T, D, i, s, e);
     const int64_t Tc = e - s, R = B * Tc;
-    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
-    SBP_CK(gather_chunk(B, T, Tc, s, d, DT_F32, dy, p.dyg, st));
-    if (sbp_status r = layer_chunk_forward(L, *w, p, s, Tc, st)) return r;
+    // a single sequence's chunk is contiguous: use it in place, no gather / scatter
+    const void* xc = static_cast<const char*>(x) + s * d * es;
+    const float* dyc = dy + s * d;
+    float* dxc = dx + s * d;
+    if (B > 1) {
+      SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+      SBP_CK(gather_chunk(B, T, Tc, s, d, DT_F32, dy, p.dyg, st));
+      xc = p.xg;
+      dyc = p.dyg;
+      dxc = p.dxg;
+    }
+    if (sbp_status r = layer_chunk_forward(L, *w, p, xc, s, Tc, st)) return r;
     // ---- MLP backward.  fp32 gradients enter the tensor cores as bf16 operands (rounded
     // per element, so the rounding does not depend on the chunking).
     const bool b16 = dt == DT_BF16;
-    const void* dY = p.dyg;
+    const void* dY = dyc;
     int dYdt = DT_F32;
     if (b16) {
-      SBP_CK(copy_cast(R * d, DT_F32, p.dyg, DT_BF16, p.dyg16, st));
+      SBP_CK(copy_cast(R * d, DT_F32, dyc, DT_BF16, p.dyg16, st));
       dY = p.dyg16;
       dYdt = DT_BF16;
     }
-    SBP_CK(gemm(mk_gemm(R, f, d, dYdt, dY, false, d, dt, w->w_down, false, f, DT_F32, p.dm, f,
-                        EPI_STORE), st));
+    {
+      // dM = dY W_d with the SwiGLU backward fused into the product's epilogue:
+      // (dG, dU) = dM * (u sigma'(g) ..., silu(g)) written straight into dgu
+      GemmDesc gd = mk_gemm(R, f, d, dYdt, dY, false, d, dt, w->w_down, false, f, dt, p.dgu,
+                            2 * f, EPI_SWIGLU_BWD);
+      gd.aux = p.gu;
+      gd.aux_ld = 2 * f;
+      gd.aux_off = f;
+      SBP_CK(gemm(gd, st));
+    }
     SBP_CK(gemm(mk_gemm(d, f, R, dYdt, dY, true, d, dt, p.m, false, f, DT_F32, gr->w_down, f,
                         EPI_ACC), st));
-    SBP_CK(swiglu_bwd(R, f, dt, p.gu, p.dm, p.dgu, st));
     const char* dU = static_cast<const char*>(p.dgu) + f * es;
     SBP_CK(gemm(mk_gemm(R, d, f, dt, p.dgu, false, 2 * f, dt, w->w_gate, false, d, DT_F32, p.dn2,
                         d, EPI_STORE), st));
@@ -469,7 +485,7 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
                         d, EPI_ACC), st));
     SBP_CK(gemm(mk_gemm(f, d, R, dt, dU, true, 2 * f, dt, p.n2, false, d, DT_F32, gr->w_up, d,
                         EPI_ACC), st));
-    SBP_CK(rmsnorm_bwd(R, d, DT_F32, p.hbuf, dt, w->ln2_g, p.rstd2, p.dn2, p.dyg, p.dh, 0,
+    SBP_CK(rmsnorm_bwd(R, d, DT_F32, p.hbuf, dt, w->ln2_g, p.rstd2, p.dn2, dyc, p.dh, 0,
                        gr->ln2_g, p.rpart, st));
     // ---- attention output projection backward
     const void* dH = p.dh;
@@ -506,17 +522,21 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
                           d, EPI_ACC), st));
     }
     if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
-    SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, p.dxg, 0, gr->ln1_g,
+    SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, dxc, 0, gr->ln1_g,
                        p.rpart, st));
-    SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 0, st));
+    if (B > 1) SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 0, st));
   }
   // ---- K/V projection backward, chunk by chunk, once every later chunk has added its dK/dV
   for (int j = 0; j < D; ++j) {
     int64_t s, e;
     chunk_range(T, D, j, s, e);
     const int64_t Tc = e - s, R = B * Tc;
-    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
-    SBP_CK(rmsnorm_fwd(R, d, dt, p.xg, dt, w->ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+    const void* xc = static_cast<const char*>(x) + s * d * es;
+    if (B > 1) {
+      SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+      xc = p.xg;
+    }
+    SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w->ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
     SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
     SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
     if (dt == DT_BF16) {
@@ -547,9 +567,14 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
       SBP_CK(colsum_acc(R, dkv, p.dvg, gr->bv, p.cpart, st));
     }
-    SBP_CK(rmsnorm_bwd(R, d, dt, p.xg, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, p.dxg, 0,
-                       gr->ln1_g, p.rpart, st));
-    SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 1, st));
+    if (B > 1) {
+      SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, p.dxg, 0,
+                         gr->ln1_g, p.rpart, st));
+      SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 1, st));
+    } else {
+      SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, dx + s * d, 1,
+                         gr->ln1_g, p.rpart, st));
+    }
   }
   return SBP_OK;
 }
@@ -584,12 +609,21 @@ sbp_status sbp_decoder_layer_forward_stream(const sbp_layer_cfg* cfg,
     int64_t s, e;
     chunk_range(T, L.num_chunks, i, s, e);
     const int64_t Tc = e - s, R = B * Tc;
-    SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
-    if (sbp_status r = layer_chunk_forward(L, *w, p, s, Tc, st)) return r;
+    const void* xc = static_cast<const char*>(x) + s * d * dt_size(dt);
+    if (B > 1) {
+      SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+      xc = p.xg;
+    }
+    if (sbp_status r = layer_chunk_forward(L, *w, p, xc, s, Tc, st)) return r;
     SBP_CK(gemm(mk_gemm(R, d, f, dt, p.m, false, f, dt, w->w_down, true, f, DT_F32, p.hbuf, d,
                         EPI_ACC), st));
-    SBP_CK(copy_cast(R * d, DT_F32, p.hbuf, dt, p.xg, st));
-    SBP_CK(scatter_chunk(B, T, Tc, s, d, dt, p.xg, y, st));
+    if (B > 1) {
+      SBP_CK(copy_cast(R * d, DT_F32, p.hbuf, dt, p.xg, st));
+      SBP_CK(scatter_chunk(B, T, Tc, s, d, dt, p.xg, y, st));
+    } else {
+      SBP_CK(copy_cast(R * d, DT_F32, p.hbuf, dt, static_cast<char*>(y) + s * d * dt_size(dt),
+                       st));
+    }
   }
   return SBP_OK;
 }

@@ -88,10 +88,13 @@ __device__ __forceinline__ float warp_max(float v) {
 //                (pmax/psum[m * pld + tile]); zy[m] = acc at column tgt[m] - col0 if in tile.
 //   EPI_CEGRAD : C = wt[m] * (exp(acc - lse[m]) - [col0 + n == tgt[m]])  (cross-entropy
 //                gradient of the logits), stored in the C dtype.
+//   EPI_SWIGLU_BWD : acc = dM (gradient of m = silu(g) u); with g = aux[m, n] and
+//                u = aux[m, aux_off + n] (aux row stride aux_ld, C dtype):
+//                C[m, n] = dM u silu'(g),  C[m, aux_off + n] = dM silu(g).
 // dynM / dynK (nullable) give the true M / K on the device (<= the static M / K).
 // crow (nullable) maps row m of the result to row crow[m] of C.
 // ---------------------------------------------------------------------------------------------
-enum Epi : int { EPI_STORE = 0, EPI_ACC = 1, EPI_LSE = 2, EPI_CEGRAD = 3 };
+enum Epi : int { EPI_STORE = 0, EPI_ACC = 1, EPI_LSE = 2, EPI_CEGRAD = 3, EPI_SWIGLU_BWD = 4 };
 
 struct GemmDesc {
   int64_t M = 0, N = 0, K = 0;
@@ -118,6 +121,9 @@ struct GemmDesc {
   float* psum = nullptr;
   int64_t pld = 0;
   float* zy = nullptr;
+  // SwiGLU-backward epilogue operand
+  const void* aux = nullptr;
+  int64_t aux_ld = 0, aux_off = 0;
   // device status word raised on a bounded-wait timeout (nullable)
   int* err = nullptr;
   // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores only
