@@ -45,7 +45,8 @@ sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, 
 /*
  * Backward of sbp_debug_attn_fwd_bf16 given its o and lse and the upstream dO [B*Tc, H, hd]
  * (bf16): dq [B*Tc, H, hd] fp32 is overwritten; dKp, dVp [B, T, Hkv, hd] fp32 are accumulated
- * (+=) for key positions < s + Tc.  `workspace` needs 256 + 4 * B * Tc * H bytes.
+ * (+=) for key positions < s + Tc.  `workspace` needs 256 + 8 * H * B * ceil(Tc / 128) * 128
+ * bytes (and at least 256 + 4 * B * Tc * H).
  */
 sbp_status sbp_debug_attn_bwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H,
                                    int64_t Hkv, int64_t hd, const void* q, const void* Kp,

@@ -1,25 +1,26 @@
 // Causal GQA attention backward of one query chunk over its key prefix on the tcgen05 tensor
-// cores (head_dim 128, bf16 operands, fp32 accumulation).
+// cores (head_dim 128, bf16 operands, fp32 accumulation), as two kernels that each keep their
+// accumulator in TMEM and write it once (no atomics; both results are deterministic and do not
+// depend on how the sequence was chunked):
 //
-// One CTA owns (sequence b, KV head g, 128-key tile kt) and loops over the query heads of g's
-// group and the chunk's query tiles that can see those keys.  Per (query head, query tile):
-//   S^T  = K Q^T            (TMEM cols [0,128))      dP^T = V dO^T   (TMEM cols [128,256))
-//   P^T  = exp(S^T * scale - lse) -> bf16, written back into TMEM over the dP^T columns the
-//          same warp has already read (the A operand of the next product, read from TMEM)
+// dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile) and loops over the query
+// heads of g's group and the chunk's query tiles that can see those keys.  Per pair:
+//   S^T  = K Q^T  (TMEM [0,128))            dP^T = V dO^T  (TMEM [128,256))
+//   P^T  = exp(S^T * scale - lse) -> bf16, written back into TMEM over dP^T columns the same
+//          warp has already read (the A operand of the dV product, read from TMEM)
 //   dS^T = P^T (dP^T - delta)     -> bf16 tile in shared memory
-//   dV  += P^T dO           (TMEM cols [256,384))    dK  += dS^T Q   (TMEM cols [384,512))
-//   dQ   = dS K             (TMEM cols [0,128) again) -> added to the fp32 dQ in global memory
-// Q and dO go through a two-stage ring, so the next pair's tiles load during this pair.
-// dK and dV stay in TMEM for the whole loop and are added once into the fp32 prefix
-// accumulators (single owner: deterministic); dQ receives one vector atomic add per query tile
-// and key tile.  Entries with key > query, queries outside the chunk and keys outside the
-// prefix are masked by selection (not by multiplication), so stale values there never reach
-// an accumulator.
+//   dV  += P^T dO (TMEM [256,384))          dK  += dS^T Q  (TMEM [384,512))
+// then dK, dV are added once into the fp32 prefix accumulators (single owner).
 //
-// Warp roles: warp 0 TMA producer (K, V once; Q and dO per pair), warp 1 TMEM owner + MMA
-// issuer, warps 2..9 element-wise + TMEM read-out (thread = key row, or query row for dQ; the
-// warp's lane quarter is fixed by its index mod 4, the two warps of a quarter split the 128
-// columns in halves).
+// dQ kernel: one CTA owns (sequence b, query head h, 128-query tile) and loops over the key
+// tiles of its causal prefix:  S = Q K^T, dP = dO V^T, dS = P (dP - delta) -> shared memory,
+// dQ += dS K (TMEM), stored once at the end.
+//
+// Entries with key > query, queries outside the chunk and keys outside the prefix are masked
+// by selection (not by multiplication), so stale values never reach an accumulator.
+// Warp roles (both kernels): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..9
+// element-wise (the warp's TMEM lane quarter is its index mod 4; the two warps of a quarter
+// split the 128 columns in halves).
 #include <cuda.h>
 
 #include <mutex>
@@ -36,18 +37,37 @@ constexpr int BT = 128;                     // keys per key tile, queries per qu
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
 constexpr int QD_STAGES = 2;
-constexpr int SMEM_BYTES = (3 + 2 * QD_STAGES) * TILE + 1024;  // K, V, dS^T, 2 x (Q, dO)
+// All shared state lives in the dynamic allocation (no static shared memory), whose start is
+// 1024-byte aligned as the 128-byte swizzle needs: the tiles first, then the statistics and
+// the barriers.
+struct KvShared {
+  float stat[2 /*QD_STAGES*/][2][BT];   // per stage: lse (log2 units), delta
+  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full, ds_full, mma2_done, drain;
+  uint32_t tmem;
+  int abort;
+};
+constexpr int KV_TILES_BYTES = (3 + 2 * QD_STAGES) * TILE;        // K, V, dS^T, 2 x (Q, dO)
+constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
+constexpr int KV_RING = 2;                                         // K/V stages of the dQ kernel
+struct QShared {
+  uint64_t qd_full, kv_full[KV_RING], kv_empty[KV_RING], sdp_full, ds_full, dq_done, drain;
+  uint32_t tmem;
+  int abort;
+};
+constexpr int Q_TILES_BYTES = (3 + 2 * KV_RING) * TILE;           // Q, dO, dS, 2 x (K, V)
+constexpr int Q_SMEM_BYTES = Q_TILES_BYTES + (int)sizeof(QShared);
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 384;
+constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 384, C_DQ = 256;
 
 struct BwdArgs {
   int64_t B, T, Tc, s, H, Hkv;
   int nq, nkt;
-  const float* lse;     // [B*Tc, H] natural log
-  const float* delta;   // [B*Tc, H]
-  float* dq;            // [B*Tc, H, HD] fp32, accumulated
+  int64_t Tcp;          // Tc rounded up to the query tile
+  const float* lse_t;   // [H, B, Tcp] log2 units, zero padded
+  const float* delta_t; // [H, B, Tcp], zero padded
+  float* dq;            // [B*Tc, H, HD] fp32, overwritten (dQ kernel)
   float* dKp;           // [B, T, Hkv, HD] fp32, accumulated
   float* dVp;
   float scale;          // 1 / sqrt(hd)
@@ -93,36 +113,19 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Bounded barrier of the element-wise warps (an mbarrier with one arrival per warp that
-// completes once per use), so that a warp that gave up on a wait cannot strand the others.
-__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t parity, int lane,
-                                           volatile int* abort_flag) {
-  __syncwarp();
-  if (lane == 0) tc::mbar_arrive(bar);
-  return tc::mbar_wait_warp(bar, parity, abort_flag);
-}
-
+// ================================================================== dK / dV kernel
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                    const BwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t kv_full, qd_full[QD_STAGES], qd_empty[QD_STAGES], sdp_full, ds_full,
-      mma2_done, dq_free, drain;
-  __shared__ uint64_t sync_a, sync_b;
-  __shared__ uint32_t tmem_sh;
-  __shared__ int abort_sh;
-  __shared__ __align__(16) float lse_s[BT];
-  __shared__ __align__(16) float delta_s[BT];
-
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  KvShared& sh = *reinterpret_cast<KvShared*>(smem_raw + KV_TILES_BYTES);
+  uint8_t* sK = smem_raw;
   uint8_t* sV = sK + TILE;
   uint8_t* sdSt = sV + TILE;
   uint8_t* sQ0 = sdSt + TILE;                    // stage st: Q at sQ0 + 2 st TILE, dO after it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  volatile int* abort_flag = &abort_sh;
+  volatile int* abort_flag = &sh.abort;
 
   // work decomposition: early key tiles (the most query tiles) first
   const int kt = (int)(blockIdx.x % a.nkt);
@@ -132,35 +135,33 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int64_t e = a.s + a.Tc;                  // prefix end
   const int64_t k_lo = (int64_t)kt * BT;
   // first query tile whose last row can see key k_lo
-  int64_t i0 = (k_lo - a.s - (BT - 1) + (BT - 1)) / BT;
-  if (k_lo - a.s - (BT - 1) <= 0) i0 = 0;
+  const int64_t i0 = (k_lo - a.s - (BT - 1) <= 0) ? 0 : (k_lo - a.s) / BT;
   const int nqt = (int)(a.nq - i0);              // query tiles per head
-  const int npairs = nqt > 0 ? (int)(grp * nqt) : 0;
+  // the swizzled tiles need a 1024-byte aligned base: refuse to run (status raised) otherwise
+  const bool misaligned = (tc::smem_u32(smem_raw) & 1023u) != 0;
+  const int npairs = (nqt > 0 && !misaligned) ? (int)(grp * nqt) : 0;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&kv_full, 1);
+    tc::mbar_init(&sh.kv_full, 1);
     for (int i = 0; i < QD_STAGES; ++i) {
-      tc::mbar_init(&qd_full[i], 1);
-      tc::mbar_init(&qd_empty[i], 1);
+      tc::mbar_init(&sh.qd_full[i], 1);
+      tc::mbar_init(&sh.qd_empty[i], 1);
     }
-    tc::mbar_init(&sdp_full, 1);
-    tc::mbar_init(&ds_full, kEwWarps);
-    tc::mbar_init(&mma2_done, 1);
-    tc::mbar_init(&dq_free, kEwWarps);
-    tc::mbar_init(&drain, 1);
-    tc::mbar_init(&sync_a, kEwWarps);
-    tc::mbar_init(&sync_b, kEwWarps);
-    abort_sh = 0;
+    tc::mbar_init(&sh.sdp_full, 1);
+    tc::mbar_init(&sh.ds_full, kEwWarps);
+    tc::mbar_init(&sh.mma2_done, 1);
+    tc::mbar_init(&sh.drain, 1);
+    sh.abort = 0;
     tc::fence_barrier_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(&tmem_sh, TMEM_COLS);
+    tc::tmem_alloc(&sh.tmem, TMEM_COLS);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = tmem_sh;
+  const uint32_t tmem = sh.tmem;
 
   auto pair_coords = [&](int j, int64_t& hh, int64_t& qi) {
     hh = g * grp + j / nqt;
@@ -171,11 +172,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0 && npairs > 0) {
       // ---------------------------------------------------------------- producer
       const int32_t krow = (int32_t)(b * a.T + k_lo);
-      tc::mbar_expect_tx(&kv_full, 2 * TILE);
-      tc::tma_load_3d(sK, &tmK, &kv_full, 0, (int32_t)g, krow);
-      tc::tma_load_3d(sK + CHUNK, &tmK, &kv_full, 64, (int32_t)g, krow);
-      tc::tma_load_3d(sV, &tmV, &kv_full, 0, (int32_t)g, krow);
-      tc::tma_load_3d(sV + CHUNK, &tmV, &kv_full, 64, (int32_t)g, krow);
+      tc::mbar_expect_tx(&sh.kv_full, 2 * TILE);
+      tc::tma_load_3d(sK, &tmK, &sh.kv_full, 0, (int32_t)g, krow);
+      tc::tma_load_3d(sK + CHUNK, &tmK, &sh.kv_full, 64, (int32_t)g, krow);
+      tc::tma_load_3d(sV, &tmV, &sh.kv_full, 0, (int32_t)g, krow);
+      tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full, 64, (int32_t)g, krow);
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < npairs; ++j) {
@@ -183,22 +184,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         pair_coords(j, hh, qi);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
-        if (!tc::mbar_wait(&qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + qi * BT);
-        tc::mbar_expect_tx(&qd_full[st], 2 * TILE);
-        tc::tma_load_3d(sQ, &tmQ, &qd_full[st], 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sQ + CHUNK, &tmQ, &qd_full[st], 64, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO, &tmdO, &qd_full[st], 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO + CHUNK, &tmdO, &qd_full[st], 64, (int32_t)hh, qrow);
+        tc::mbar_expect_tx(&sh.qd_full[st], 2 * TILE + 2 * BT * 4);
+        const int64_t srow = (hh * a.B + b) * a.Tcp + qi * BT;
+        tc::bulk_load(&sh.stat[st][0][0], a.lse_t + srow, BT * 4, &sh.qd_full[st]);
+        tc::bulk_load(&sh.stat[st][1][0], a.delta_t + srow, BT * 4, &sh.qd_full[st]);
+        tc::tma_load_3d(sQ, &tmQ, &sh.qd_full[st], 0, (int32_t)hh, qrow);
+        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.qd_full[st], 64, (int32_t)hh, qrow);
+        tc::tma_load_3d(sdO, &tmdO, &sh.qd_full[st], 0, (int32_t)hh, qrow);
+        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)hh, qrow);
         issued = j + 1;
       }
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
-        while (!tc::mbar_try_wait(&kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+        while (!tc::mbar_try_wait(&sh.kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
         for (int j = issued > QD_STAGES ? issued - QD_STAGES : 0; j < issued; ++j)
-          while (!tc::mbar_try_wait(&qd_full[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u) &&
+          while (!tc::mbar_try_wait(&sh.qd_full[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }
     }
@@ -207,18 +211,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // ---------------------------------------------------------------- MMA issuer
       const uint32_t id_kk = tc::idesc_bf16_f32(128, 128, 0, 0);   // A K-major, B K-major
       const uint32_t id_km = tc::idesc_bf16_f32(128, 128, 0, 1);   // A K-major, B MN-major
-      const uint32_t id_mm = tc::idesc_bf16_f32(128, 128, 1, 1);   // A MN-major, B MN-major
       const uint32_t aK = tc::smem_u32(sK), aV = tc::smem_u32(sV), adS = tc::smem_u32(sdSt),
                      aQ0 = tc::smem_u32(sQ0);
-      bool ok = tc::mbar_wait(&kv_full, 0, abort_flag);
+      bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag);
       bool issued = false;
       for (int j = 0; j < npairs && ok; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
         const int st = j % QD_STAGES;
         const uint32_t sph = (uint32_t)(j / QD_STAGES) & 1u;
         const uint32_t aQ = aQ0 + 2 * st * TILE, adO = aQ + TILE;
-        if (!tc::mbar_wait(&qd_full[st], sph, abort_flag)) { ok = false; break; }
-        if (j >= 1 && !tc::mbar_wait(&dq_free, ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.qd_full[st], sph, abort_flag)) { ok = false; break; }
+        // the previous pair's dV / dK products must have read P^T (TMEM) and dS^T (smem)
+        if (j >= 1 && !tc::mbar_wait(&sh.mma2_done, ph ^ 1u, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
@@ -229,11 +233,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                          tc::smem_desc_sw128(adO + off, 16, 1024), id_kk, kk != 0);
         }
         issued = true;
-        tc::mma_commit(&sdp_full);
-        if (!tc::mbar_wait(&ds_full, ph, abort_flag)) { ok = false; break; }
+        tc::mma_commit(&sh.sdp_full);
+        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = queries for dV, dK; keys for dQ
+        for (int kk = 0; kk < 8; ++kk) {   // K = queries
           const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;   // K-major operand step
           const uint32_t offm = kk * 2048;                            // MN-major operand step
           const uint32_t acc = (j | kk) != 0;
@@ -243,27 +247,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                      id_km, acc);
           tc::mma_f16_ss(tmem + C_DK, tc::smem_desc_sw128(adS + offk, 16, 1024),
                          tc::smem_desc_sw128(aQ + offm, CHUNK, 1024), id_km, acc);
-          tc::mma_f16_ss(tmem + C_S, tc::smem_desc_sw128(adS + offm, CHUNK, 1024),
-                         tc::smem_desc_sw128(aK + offm, CHUNK, 1024), id_mm, kk != 0);
         }
-        tc::mma_commit(&mma2_done);
-        tc::mma_commit(&qd_empty[st]);
+        tc::mma_commit(&sh.mma2_done);
+        tc::mma_commit(&sh.qd_empty[st]);
       }
       if (issued) {
-        tc::mma_commit(&drain);
+        tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
-        while (!tc::mbar_try_wait(&drain, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+        while (!tc::mbar_try_wait(&sh.drain, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }
     }
   } else if (npairs > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
     const int half = (warp - 2) >> 2;                // column half of this warp
-    const int r = q4 * 32 + lane;                    // TMEM lane = key row (or query row)
+    const int r = q4 * 32 + lane;                    // TMEM lane = key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int kpos = (int)(k_lo + r);
     const float scale_log2 = a.scale * 1.4426950408889634f;
-    const int tid = threadIdx.x - 64;                // 0..255
     const int e32 = (int)e;
     bool ok = true;
     for (int j = 0; j < npairs; ++j) {
@@ -273,17 +274,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int q0 = (int)(a.s + qi * BT);           // absolute position of query column 0
       // no masking needed when every key of the tile precedes every (valid) query of the tile
       const bool full = (k_lo + BT - 1 <= q0) && (qi * BT + BT <= a.Tc);
-      // per-query statistics of this pair (thread tid < 128 loads query column tid)
-      if (!group_sync(&sync_a, ph, lane, abort_flag)) { ok = false; break; }
-      if (tid < BT) {
-        const int64_t ql = qi * BT + tid;           // position within the chunk
-        const bool qv = ql < a.Tc;
-        const int64_t gi = (b * a.Tc + ql) * a.H + hh;
-        lse_s[tid] = qv ? a.lse[gi] * 1.4426950408889634f : 0.f;
-        delta_s[tid] = qv ? a.delta[gi] : 0.f;
+      const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
+      const float* lse_s = sh.stat[st][0];
+      const float* delta_s = sh.stat[st][1];
+      // acquire the bulk copies of this stage (already complete once the scores are ready)
+      if (!tc::mbar_wait_warp(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+        ok = false;
+        break;
       }
-      if (!group_sync(&sync_b, ph, lane, abort_flag)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(&sdp_full, ph, abort_flag)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&sh.sdp_full, ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
@@ -300,23 +299,23 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const float4 lv = l4[i4], dv = d4[i4];
           const float la[4] = {lv.x, lv.y, lv.z, lv.w};
           const float da[4] = {dv.x, dv.y, dv.z, dv.w};
-          float p[4], g[4];
+          float p[4], gg[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int i = i4 * 4 + k;
             p[k] = ex2(fmaf(__uint_as_float(rs[i]), scale_log2, -la[k]));
-            g[k] = p[k] * (__uint_as_float(rd[i]) - da[k]);
+            gg[k] = p[k] * (__uint_as_float(rd[i]) - da[k]);
             if (!full) {
               const int qpos = q0 + c * 32 + i;
               const bool live = (kpos <= qpos) && (qpos < e32);
               p[k] = live ? p[k] : 0.f;
-              g[k] = live ? g[k] : 0.f;
+              gg[k] = live ? gg[k] : 0.f;
             }
           }
           pp[i4 * 2] = pack2(p[0], p[1]);
           pp[i4 * 2 + 1] = pack2(p[2], p[3]);
-          dd[i4 * 2] = pack2(g[0], g[1]);
-          dd[i4 * 2 + 1] = pack2(g[2], g[3]);
+          dd[i4 * 2] = pack2(gg[0], gg[1]);
+          dd[i4 * 2 + 1] = pack2(gg[2], gg[3]);
         }
         // packed P over dP^T columns this warp has already read (queries 32 cc .. of its half)
         tmem_st16(tmem + lane_off + C_DP + 64 * half + 16 * cc, pp);
@@ -328,38 +327,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&ds_full);
-      // dQ of this query tile: TMEM lane r = query row r
-      if (!tc::mbar_wait_warp(&mma2_done, ph, abort_flag)) { ok = false; break; }
-      tc::fence_after_sync();
-      {
-        const int64_t ql = qi * BT + r;
-        const bool qv = ql < a.Tc;
-        float* dqp = a.dq + ((b * a.Tc + ql) * a.H + hh) * HD;
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;
-          uint32_t rq[32];
-          tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rq);
-          tc::tmem_ld_wait();
-          if (qv) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 v = make_float4(__uint_as_float(rq[i]) * a.scale,
-                                     __uint_as_float(rq[i + 1]) * a.scale,
-                                     __uint_as_float(rq[i + 2]) * a.scale,
-                                     __uint_as_float(rq[i + 3]) * a.scale);
-              atomicAdd(reinterpret_cast<float4*>(dqp + c * 32 + i), v);
-            }
-          }
-        }
-      }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&dq_free);
+      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
     }
     // dK, dV of this key tile: add into the fp32 prefix accumulators (single owner)
-    if (ok) {
+    if (ok && tc::mbar_wait_warp(&sh.mma2_done, (uint32_t)(npairs - 1) & 1u, abort_flag)) {
+      tc::fence_after_sync();
       const bool kv = kpos < e32;
       const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
 #pragma unroll 1
@@ -394,27 +366,255 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (threadIdx.x == 0 && abort_sh && a.err) atomicExch(a.err, DEV_TIMEOUT);
+  if (threadIdx.x == 0 && (sh.abort || misaligned) && a.err) atomicExch(a.err, DEV_TIMEOUT);
   if (warp == 1) {
     __syncwarp();
     tc::tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
-// delta[r, h] = sum_d dO[r, h, d] * O[r, h, d]  (one warp per (row, head))
-__global__ void attn_delta_kernel(int64_t rows_heads, const __nv_bfloat16* __restrict__ dO,
-                                  const __nv_bfloat16* __restrict__ o, float* __restrict__ delta) {
+// ================================================================== dQ kernel
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  QShared& sh = *reinterpret_cast<QShared*>(smem_raw + Q_TILES_BYTES);
+  uint8_t* sQ = smem_raw;
+  uint8_t* sdO = sQ + TILE;
+  uint8_t* sdS = sdO + TILE;
+  uint8_t* sKV0 = sdS + TILE;                    // ring stage st: K at sKV0 + 2 st TILE, V after
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &sh.abort;
+
+  // heavy (late) query tiles first
+  const int qt = a.nq - 1 - (int)(blockIdx.x % a.nq);
+  const int64_t h = (blockIdx.x / a.nq) % a.H;
+  const int64_t b = blockIdx.x / (a.nq * a.H);
+  const int64_t g = h / (a.H / a.Hkv);
+  const int64_t q_lo = a.s + (int64_t)qt * BT;                  // absolute position of row 0
+  const int64_t q_hi = a.s + imin((int64_t)(qt + 1) * BT, a.Tc);  // one past the last valid row
+  const bool misaligned = (tc::smem_u32(smem_raw) & 1023u) != 0;
+  const int nkv = misaligned ? 0 : (int)((q_hi + BT - 1) / BT);  // key tiles 0 .. nkv-1
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&sh.qd_full, 1);
+    for (int i = 0; i < KV_RING; ++i) {
+      tc::mbar_init(&sh.kv_full[i], 1);
+      tc::mbar_init(&sh.kv_empty[i], 1);
+    }
+    tc::mbar_init(&sh.sdp_full, 1);
+    tc::mbar_init(&sh.ds_full, kEwWarps);
+    tc::mbar_init(&sh.dq_done, 1);
+    tc::mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sh.tmem, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sh.tmem;
+
+  if (warp == 0) {
+    if (lane == 0 && nkv > 0) {
+      // ---------------------------------------------------------------- producer
+      const int32_t qrow = (int32_t)(b * a.Tc + (int64_t)qt * BT);
+      tc::mbar_expect_tx(&sh.qd_full, 2 * TILE);
+      tc::tma_load_3d(sQ, &tmQ, &sh.qd_full, 0, (int32_t)h, qrow);
+      tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.qd_full, 64, (int32_t)h, qrow);
+      tc::tma_load_3d(sdO, &tmdO, &sh.qd_full, 0, (int32_t)h, qrow);
+      tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full, 64, (int32_t)h, qrow);
+      bool ok = true;
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j % KV_RING;
+        const uint32_t ph = (uint32_t)(j / KV_RING) & 1u;
+        if (!tc::mbar_wait(&sh.kv_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* sK = sKV0 + 2 * st * TILE;
+        uint8_t* sV = sK + TILE;
+        const int32_t krow = (int32_t)(b * a.T + (int64_t)j * BT);
+        tc::mbar_expect_tx(&sh.kv_full[st], 2 * TILE);
+        tc::tma_load_3d(sK, &tmK, &sh.kv_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sK + CHUNK, &tmK, &sh.kv_full[st], 64, (int32_t)g, krow);
+        tc::tma_load_3d(sV, &tmV, &sh.kv_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full[st], 64, (int32_t)g, krow);
+        issued = j + 1;
+      }
+      if (!ok) {
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(&sh.qd_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+        for (int j = issued > KV_RING ? issued - KV_RING : 0; j < issued; ++j)
+          while (!tc::mbar_try_wait(&sh.kv_full[j % KV_RING], (uint32_t)(j / KV_RING) & 1u) &&
+                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nkv > 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      const uint32_t id_kk = tc::idesc_bf16_f32(128, 128, 0, 0);   // A K-major, B K-major
+      const uint32_t id_km = tc::idesc_bf16_f32(128, 128, 0, 1);   // A K-major, B MN-major
+      const uint32_t aQ = tc::smem_u32(sQ), adO = tc::smem_u32(sdO), adS = tc::smem_u32(sdS),
+                     aKV0 = tc::smem_u32(sKV0);
+      bool ok = tc::mbar_wait(&sh.qd_full, 0, abort_flag);
+      bool issued = false;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const uint32_t ph = (uint32_t)j & 1u;
+        const int st = j % KV_RING;
+        const uint32_t sph = (uint32_t)(j / KV_RING) & 1u;
+        const uint32_t aK = aKV0 + 2 * st * TILE, aV = aK + TILE;
+        if (!tc::mbar_wait(&sh.kv_full[st], sph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        // S and dP of this key tile (the element-wise warps have read the previous ones:
+        // ds_full of the previous tile was waited below)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
+          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+          tc::mma_f16_ss(tmem + C_S, tc::smem_desc_sw128(aQ + off, 16, 1024),
+                         tc::smem_desc_sw128(aK + off, 16, 1024), id_kk, kk != 0);
+          tc::mma_f16_ss(tmem + C_DP, tc::smem_desc_sw128(adO + off, 16, 1024),
+                         tc::smem_desc_sw128(aV + off, 16, 1024), id_kk, kk != 0);
+        }
+        issued = true;
+        tc::mma_commit(&sh.sdp_full);
+        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = keys: dQ += dS K
+          const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;
+          tc::mma_f16_ss(tmem + C_DQ, tc::smem_desc_sw128(adS + offk, 16, 1024),
+                         tc::smem_desc_sw128(aK + kk * 2048, CHUNK, 1024), id_km,
+                         (j | kk) != 0);
+        }
+        tc::mma_commit(&sh.dq_done);
+        tc::mma_commit(&sh.kv_empty[st]);
+      }
+      if (issued) {
+        tc::mma_commit(&sh.drain);
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(&sh.drain, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+      }
+    }
+  } else if (nkv > 0) {
+    // ------------------------------------------------------------------ element-wise warps
+    const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = q4 * 32 + lane;                    // TMEM lane = query row
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const int t = (int)(q_lo + r);                   // absolute query position
+    const bool qv = t < q_hi;
+    const int64_t srow = (h * a.B + b) * a.Tcp + (int64_t)qt * BT + r;
+    const float lse_r = a.lse_t[srow];               // log2 units (0 in the padding)
+    const float dl_r = a.delta_t[srow];
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const uint32_t ph = (uint32_t)j & 1u;
+      const int k0 = j * BT;
+      const bool diag = k0 + BT - 1 > (int)q_lo;     // some key may follow some query
+      if (!tc::mbar_wait_warp(&sh.sdp_full, ph, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      uint32_t dd[2][16];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;
+        uint32_t rs[32], rd[32];
+        tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rs);
+        tc::tmem_ld32(tmem + lane_off + C_DP + c * 32, rd);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float gg[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const float p = ex2(fmaf(__uint_as_float(rs[i + k]), scale_log2, -lse_r));
+            float v = p * (__uint_as_float(rd[i + k]) - dl_r);
+            if (diag) v = (k0 + c * 32 + i + k <= t && qv) ? v : 0.f;
+            else v = qv ? v : 0.f;
+            gg[k] = v;
+          }
+          dd[cc][i >> 1] = pack2(gg[0], gg[1]);
+        }
+      }
+      // dS may overwrite the previous tile's dS once its dQ product has read it
+      if (j >= 1) {
+        if (!tc::mbar_wait_warp(&sh.dq_done, ph ^ 1u, abort_flag)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_unit(sdS, r, c * 4 + u,
+                  make_uint4(dd[cc][4 * u], dd[cc][4 * u + 1], dd[cc][4 * u + 2], dd[cc][4 * u + 3]));
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
+    }
+    // dQ of this query tile, written once
+    if (ok && tc::mbar_wait_warp(&sh.dq_done, (uint32_t)(nkv - 1) & 1u, abort_flag)) {
+      tc::fence_after_sync();
+      float* dqp = a.dq + ((b * a.Tc + (t - a.s)) * a.H + h) * HD;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;
+        uint32_t rq[32];
+        tc::tmem_ld32(tmem + lane_off + C_DQ + c * 32, rq);
+        tc::tmem_ld_wait();
+        if (qv) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dqp + c * 32 + i) =
+                make_float4(__uint_as_float(rq[i]) * a.scale, __uint_as_float(rq[i + 1]) * a.scale,
+                            __uint_as_float(rq[i + 2]) * a.scale,
+                            __uint_as_float(rq[i + 3]) * a.scale);
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (threadIdx.x == 0 && (sh.abort || misaligned) && a.err) atomicExch(a.err, DEV_TIMEOUT);
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Per (row, head): delta = sum_d dO * O and lse in log2 units, written head-major into
+// [H, B, Tcp] rows padded to whole query tiles (padding = 0), so that the backward kernel can
+// bulk-copy the 128 values of a query tile.  One warp per (row, head) of the chunk.
+__global__ void attn_stats_kernel(int64_t B, int64_t Tc, int64_t Tcp, int64_t H,
+                                  const __nv_bfloat16* __restrict__ dO,
+                                  const __nv_bfloat16* __restrict__ o,
+                                  const float* __restrict__ lse, float* __restrict__ lse_t,
+                                  float* __restrict__ delta_t) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (w >= rows_heads) return;
-  const __nv_bfloat16* a = dO + w * HD;
-  const __nv_bfloat16* c = o + w * HD;
-  float s = 0.f;
+  if (w >= H * B * Tcp) return;
+  const int64_t t = w % Tcp, b = (w / Tcp) % B, h = w / (Tcp * B);
+  float s = 0.f, l = 0.f;
+  if (t < Tc) {
+    const int64_t rh = (b * Tc + t) * H + h;
+    const __nv_bfloat16* pa = dO + rh * HD;
+    const __nv_bfloat16* pc = o + rh * HD;
 #pragma unroll
-  for (int i = 0; i < HD / 32; ++i)
-    s = fmaf(__bfloat162float(a[lane + 32 * i]), __bfloat162float(c[lane + 32 * i]), s);
-  s = warp_sum(s);
-  if (lane == 0) delta[w] = s;
+    for (int i = 0; i < HD / 32; ++i)
+      s = fmaf(__bfloat162float(pa[lane + 32 * i]), __bfloat162float(pc[lane + 32 * i]), s);
+    s = warp_sum(s);
+    l = lse[rh] * 1.4426950408889634f;
+  }
+  if (lane == 0) {
+    delta_t[w] = s;
+    lse_t[w] = l;
+  }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -457,10 +657,15 @@ bool attn_bwd_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, co
          encode_fn_bwd() != nullptr;
 }
 
+size_t attn_bwd_tc_stats_floats(int64_t B, int64_t Tc, int64_t H) {
+  return (size_t)2 * H * B * ((Tc + BT - 1) / BT) * BT;
+}
+
+// stats: scratch of attn_bwd_tc_stats_floats() floats (16-byte aligned).
 // dq [B*Tc, H, HD] fp32 is overwritten; dKp/dVp [B, T, Hkv, HD] fp32 accumulate rows < s + Tc.
 cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                         const void* q, const void* Kp, const void* Vp, const void* o,
-                        const void* dO, const float* lse, float* delta, float* dq, float* dKp,
+                        const void* dO, const float* lse, float* stats, float* dq, float* dKp,
                         float* dVp, int* err, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
   if (!map3(&mq, q, H, B * Tc) || !map3(&mk, Kp, Hkv, B * T) || !map3(&mv, Vp, Hkv, B * T) ||
@@ -469,29 +674,36 @@ cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES);
+    attr = cudaFuncSetAttribute(attn_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                KV_SMEM_BYTES);
+    if (attr == cudaSuccess)
+      attr = cudaFuncSetAttribute(attn_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  Q_SMEM_BYTES);
   });
   if (attr != cudaSuccess) return attr;
-  const int64_t rh = B * Tc * H;
-  cudaError_t e = cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)rh * HD, st);
-  if (e != cudaSuccess) return e;
-  launch(attn_delta_kernel, dim3((unsigned)((rh * 32 + 255) / 256)), dim3(256), 0, st, rh,
-         static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), delta);
+  const int64_t Tcp = ((Tc + BT - 1) / BT) * BT;
+  float* lse_t = stats;
+  float* delta_t = stats + H * B * Tcp;
+  const int64_t nw = H * B * Tcp;
+  launch(attn_stats_kernel, dim3((unsigned)((nw * 32 + 255) / 256)), dim3(256), 0, st, B, Tc,
+         Tcp, H, static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o),
+         lse, lse_t, delta_t);
   BwdArgs a;
   a.B = B; a.T = T; a.Tc = Tc; a.s = s; a.H = H; a.Hkv = Hkv;
   a.nq = (int)((Tc + BT - 1) / BT);
   a.nkt = (int)((s + Tc + BT - 1) / BT);
-  a.lse = lse;
-  a.delta = delta;
+  a.Tcp = Tcp;
+  a.lse_t = lse_t;
+  a.delta_t = delta_t;
   a.dq = dq;
   a.dKp = dKp;
   a.dVp = dVp;
   a.scale = 1.f / sqrtf((float)HD);
   a.err = err;
-  const int64_t grid = B * Hkv * a.nkt;
-  launch(attn_bwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)SMEM_BYTES, st, mq, mk,
-         mv, mdo, a);
+  launch(attn_bwd_kv_kernel, dim3((unsigned)(B * Hkv * a.nkt)), dim3(kThreads),
+         (size_t)KV_SMEM_BYTES, st, mq, mk, mv, mdo, a);
+  launch(attn_bwd_q_kernel, dim3((unsigned)(B * H * a.nq)), dim3(kThreads),
+         (size_t)Q_SMEM_BYTES, st, mq, mk, mv, mdo, a);
   return cudaGetLastError();
 }
 

@@ -107,7 +107,7 @@ struct LayerPlan {
   float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dn2, *dh, *delta, *dq, *dn1, *dxg;
   float *dkpre, *dvg, *rpart, *cpart;
   // bf16 operand copies of fp32 gradients (bf16 path only)
-  void *dyg16, *dh16, *dq16, *dqlo, *khi, *klo, *vhi, *vlo;
+  void *dyg16, *dh16, *dq16, *khi, *klo, *vhi, *vlo;
   int64_t R;
 };
 
@@ -142,7 +142,7 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.dn2 = c.take<float>((size_t)R * d);
   p.dh = c.take<float>((size_t)R * d);
   p.dO = c.take_bytes((size_t)R * dq * es);
-  p.delta = c.take<float>((size_t)R * L.n_heads);
+  p.delta = c.take<float>(attn_bwd_scratch_floats(B, chunk_max(T, L.num_chunks), L.n_heads));
   p.dq = c.take<float>((size_t)R * dq);
   p.dn1 = c.take<float>((size_t)R * d);
   p.dxg = c.take<float>((size_t)R * d);
@@ -151,12 +151,11 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.rpart = c.take<float>(rmsnorm_bwd_partial_floats(d));
   int64_t wmax = dq > dkv ? dq : dkv;
   p.cpart = c.take<float>(colsum_partial_floats(wmax));
-  p.dyg16 = p.dh16 = p.dq16 = p.dqlo = p.khi = p.klo = p.vhi = p.vlo = nullptr;
+  p.dyg16 = p.dh16 = p.dq16 = p.khi = p.klo = p.vhi = p.vlo = nullptr;
   if (dt == DT_BF16) {
     p.dyg16 = c.take_bytes((size_t)R * d * 2);
     p.dh16 = c.take_bytes((size_t)R * d * 2);
     p.dq16 = c.take_bytes((size_t)R * dq * 2);
-    p.dqlo = c.take_bytes((size_t)R * dq * 2);
     p.khi = c.take_bytes((size_t)R * dkv * 2);
     p.klo = c.take_bytes((size_t)R * dkv * 2);
     p.vhi = c.take_bytes((size_t)R * dkv * 2);
@@ -504,23 +503,19 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
                     p.dq, p.dKp, p.dVp, st));
     SBP_CK(rope_inv_f32(R, Tc, s, H, hd, p.dq, p.cosb, p.sinb, st));
     // ---- q projection backward
+    // dQ of a query row is a fixed-order sum over its key tiles (the same at every D), so a
+    // plain per-element bf16 rounding is D-independent
+    const void* dQ = p.dq;
+    int dQdt = DT_F32;
     if (b16) {
-      // dQ is a sum over key tiles accumulated with atomics (order not fixed): it enters the
-      // tensor cores as a hi + lo bf16 pair so that its rounding does not show in the result
-      SBP_CK(split_bf16(R * dq, p.dq, p.dq16, p.dqlo, st));
-      const void* parts[2] = {p.dq16, p.dqlo};
-      for (int k = 0; k < 2; ++k) {
-        SBP_CK(gemm(mk_gemm(R, d, dq, DT_BF16, parts[k], false, dq, dt, w->wq, false, d, DT_F32,
-                            p.dn1, d, k == 0 ? EPI_STORE : EPI_ACC), st));
-        SBP_CK(gemm(mk_gemm(dq, d, R, DT_BF16, parts[k], true, dq, dt, p.n1, false, d, DT_F32,
-                            gr->wq, d, EPI_ACC), st));
-      }
-    } else {
-      SBP_CK(gemm(mk_gemm(R, d, dq, DT_F32, p.dq, false, dq, dt, w->wq, false, d, DT_F32, p.dn1,
-                          d, EPI_STORE), st));
-      SBP_CK(gemm(mk_gemm(dq, d, R, DT_F32, p.dq, true, dq, dt, p.n1, false, d, DT_F32, gr->wq,
-                          d, EPI_ACC), st));
+      SBP_CK(copy_cast(R * dq, DT_F32, p.dq, DT_BF16, p.dq16, st));
+      dQ = p.dq16;
+      dQdt = DT_BF16;
     }
+    SBP_CK(gemm(mk_gemm(R, d, dq, dQdt, dQ, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
+                        EPI_STORE), st));
+    SBP_CK(gemm(mk_gemm(dq, d, R, dQdt, dQ, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
+                        EPI_ACC), st));
     if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
     SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, dxc, 0, gr->ln1_g,
                        p.rpart, st));
@@ -734,6 +729,7 @@ sbp_status sbp_debug_attn_bwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, 
     return fail(SBP_ERR_UNSUPPORTED, "the tensor-core attention needs head_dim 128 and aligned rows");
   tl_status = static_cast<int*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  // (the caller provides kStatusBytes + 4 * attn_bwd_scratch_floats(B, Tc, H) bytes)
   SBP_CK(attn_bwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, dO, lse, delta, dq, dKp, dVp,
                   static_cast<cudaStream_t>(stream), path));
   return SBP_OK;

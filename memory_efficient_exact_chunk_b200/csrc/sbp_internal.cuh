@@ -215,7 +215,8 @@ cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
 cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp, void* o,
                      float* lse, cudaStream_t st, int path = 0);
-// Backward: dq [B*Tc, H, hd] fp32 (overwritten); dKp/dVp [B, T, Hkv, hd] fp32 (+= rows < s+Tc).
+// Backward: dq [B*Tc, H, hd] fp32 (overwritten); dKp/dVp [B, T, Hkv, hd] fp32 (+= rows < s+Tc);
+// delta: scratch of attn_bwd_scratch_floats() floats.
 cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
                      const void* o, const void* dO, const float* lse, float* delta, float* dq,
@@ -224,8 +225,15 @@ bool attn_bwd_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, co
                            const void* o, const void* dO, const float* dq);
 cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                         const void* q, const void* Kp, const void* Vp, const void* o,
-                        const void* dO, const float* lse, float* delta, float* dq, float* dKp,
+                        const void* dO, const float* lse, float* stats, float* dq, float* dKp,
                         float* dVp, int* err, cudaStream_t st);
+// scratch floats of the tensor-core backward's per-query statistics
+size_t attn_bwd_tc_stats_floats(int64_t B, int64_t Tc, int64_t H);
+// scratch floats attn_bwd needs in its `delta` argument (either path)
+inline size_t attn_bwd_scratch_floats(int64_t B, int64_t Tc, int64_t H) {
+  const size_t a = (size_t)B * Tc * H, b = attn_bwd_tc_stats_floats(B, Tc, H);
+  return a > b ? a : b;
+}
 
 // embedding (elementwise.cu)
 cudaError_t embed_fwd(int64_t rows, int64_t cols, int64_t vocab, int dt, const int* ids,

@@ -316,7 +316,8 @@ def debug_attn_bwd_bf16(q, Kp, Vp, o, dO, lse, dq, dKp, dVp, s, path=0, stream=N
     B, T, Hkv, hd = Kp.shape
     R, H, _ = q.shape
     Tc = R // B
-    ws = workspace(256 + 4 * R * H, q.device)
+    tcp = (Tc + 127) // 128 * 128
+    ws = workspace(256 + max(4 * R * H, 8 * H * B * tcp), q.device)
     ws.zero_()
     _check(load().sbp_debug_attn_bwd_bf16(B, T, Tc, s, H, Hkv, hd, _ptr(q), _ptr(Kp), _ptr(Vp),
                                           _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dKp),
