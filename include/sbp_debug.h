@@ -21,8 +21,9 @@ extern "C" {
  *   a_trans = 0: A is [M, K] with leading dimension lda;  1: A is [K, M] (op(A) = A^T)
  *   b_trans = 0: B is [K, N] with leading dimension ldb;  1: B is [N, K] (op(B) = B^T)
  * C is [M, N] with leading dimension ldc; accumulate = 0 overwrites, 1 adds.
- * path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores (SBP_ERR_UNSUPPORTED if the layout is
- * not one the tensor-core kernel takes).  `workspace` (>= 256 bytes, device) receives the
+ * path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores (either kernel), 3 = tensor cores with
+ * one CTA per 128 x 256 tile, 4 = tensor cores with a CTA pair per 256 x 256 tile
+ * (SBP_ERR_UNSUPPORTED for 2..4 if the layout is not one the tensor-core kernels take).  `workspace` (>= 256 bytes, device) receives the
  * device status word (see sbp_get_device_status).  Device pointers, queued on `stream`.
  */
 sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int a_trans,

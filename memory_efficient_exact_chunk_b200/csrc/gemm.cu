@@ -6,14 +6,23 @@ namespace sbp {
 
 cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t st);
 cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st);
+cudaError_t gemm_tc_pair(const GemmDesc& g, int* err, cudaStream_t st);
+
+// The CTA-pair kernel needs enough 256 x 256 tiles to occupy every SM pair.
+static bool use_pair(const GemmDesc& g) {
+  const int64_t tiles = ((g.M + 255) / 256) * ((g.N + 255) / 256);
+  return g.path != 3 && tiles >= 74;
+}
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
   const bool tc = g.path != 1 && gemm_tc_supported(g);
-  if (!tc && g.path == 2) return cudaErrorNotSupported;
+  if (!tc && g.path >= 2) return cudaErrorNotSupported;
   const int kind = tc ? PROF_GEMM_TC : PROF_GEMM_SIMT;
   prof_mark_begin(kind, st);
-  const cudaError_t e = tc ? gemm_tc(g, g.err, st) : gemm_simt(g, st);
+  const cudaError_t e = tc ? ((g.path == 4 || (g.path == 0 && use_pair(g))) ? gemm_tc_pair(g, g.err, st)
+                                                                            : gemm_tc(g, g.err, st))
+                           : gemm_simt(g, st);
   prof_mark_end(kind, st);
   return e;
 }

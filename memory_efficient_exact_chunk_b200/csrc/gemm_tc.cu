@@ -142,6 +142,92 @@ __device__ __forceinline__ void epi_swiglu_bwd32(const GemmDesc& g, int64_t m, i
   }
 }
 
+// Epilogue of one accumulator tile for the calling thread's row m: columns [n0, n0 + BN) of the
+// tile are read from TMEM at tbase (this warp's lane quarter, accumulator base column).
+__device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase, int64_t m,
+                                              int64_t n0, int64_t M, int64_t N, int nk) {
+  // the logit-gradient epilogue also writes the zero rows between the live row count and
+  // the buffer's row count, so that a later product over those rows reads zeros
+  const bool row_ok = m < (g.epi == EPI_CEGRAD ? g.M : M);
+  if (g.epi == EPI_LSE) {
+    for (int c = 0; c < BN; c += 64) {
+      uint32_t r0[32], r1[32];
+      tc::tmem_ld32(tbase + c, r0);
+      tc::tmem_ld32(tbase + c + 32, r1);
+      tc::tmem_ld_wait();
+      const int64_t nc = n0 + c;
+      if (!row_ok || nc >= N) continue;
+      const int ncols = (int)imin(64, N - nc);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
+        if (j < ncols) mx = fmaxf(mx, a);
+        if (j + 32 < ncols) mx = fmaxf(mx, b);
+      }
+      float sm = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
+        if (j < ncols) sm += expf(a - mx);
+        if (j + 32 < ncols) sm += expf(b - mx);
+      }
+      const int64_t tile = nc / 64;
+      g.pmax[m * g.pld + tile] = mx;
+      g.psum[m * g.pld + tile] = sm;
+      const int64_t y = (int64_t)g.tgt[m] - g.col0 - nc;
+      if (y >= 0 && y < ncols) {
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (y == j) z = u2f(r0[j]);
+          if (y == j + 32) z = u2f(r1[j]);
+        }
+        g.zy[m] = nk ? z : 0.f;
+      }
+    }
+  } else {
+    float w = 0.f, l = 0.f;
+    int64_t ycol = -1;
+    int64_t crow = m;
+    if (row_ok) {
+      if (g.epi == EPI_CEGRAD) {
+        w = g.wt[m];
+        l = g.lse[m];
+        ycol = (int64_t)g.tgt[m] - g.col0;
+      } else if (g.crow) {
+        crow = g.crow[m];
+      }
+    }
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tc::tmem_ld32(tbase + c, r);
+      tc::tmem_ld_wait();
+      const int64_t nc = n0 + c;
+      if (!row_ok || nc >= N) continue;
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = nk ? u2f(r[j]) : 0.f;
+      if (g.epi == EPI_SWIGLU_BWD) {
+        epi_swiglu_bwd32(g, m, nc, N, v);
+        continue;
+      }
+      if (g.epi == EPI_CEGRAD) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float p = expf(v[j] - l);
+          if (nc + j == ycol) p -= 1.f;
+          v[j] = w * p;
+        }
+      } else if (g.alpha != 1.f) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= g.alpha;
+      }
+      epi_store32(g, crow, nc, N, v);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcArgs args) {
@@ -295,87 +381,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) break;
       tc::fence_after_sync();
       const int64_t m = m0 + row_in_tile;
-      // the logit-gradient epilogue also writes the zero rows between the live row count and
-      // the buffer's row count, so that a later product over those rows reads zeros
-      const bool row_ok = m < (g.epi == EPI_CEGRAD ? g.M : M);
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (g.epi == EPI_LSE) {
-        for (int c = 0; c < BN; c += 64) {
-          uint32_t r0[32], r1[32];
-          tc::tmem_ld32(tbase + c, r0);
-          tc::tmem_ld32(tbase + c + 32, r1);
-          tc::tmem_ld_wait();
-          const int64_t nc = n0 + c;
-          if (!row_ok || nc >= N) continue;
-          const int ncols = (int)imin(64, N - nc);
-          float mx = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
-            if (j < ncols) mx = fmaxf(mx, a);
-            if (j + 32 < ncols) mx = fmaxf(mx, b);
-          }
-          float sm = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
-            if (j < ncols) sm += expf(a - mx);
-            if (j + 32 < ncols) sm += expf(b - mx);
-          }
-          const int64_t tile = nc / 64;
-          g.pmax[m * g.pld + tile] = mx;
-          g.psum[m * g.pld + tile] = sm;
-          const int64_t y = (int64_t)g.tgt[m] - g.col0 - nc;
-          if (y >= 0 && y < ncols) {
-            float z = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (y == j) z = u2f(r0[j]);
-              if (y == j + 32) z = u2f(r1[j]);
-            }
-            g.zy[m] = nk ? z : 0.f;
-          }
-        }
-      } else {
-        float w = 0.f, l = 0.f;
-        int64_t ycol = -1;
-        int64_t crow = m;
-        if (row_ok) {
-          if (g.epi == EPI_CEGRAD) {
-            w = g.wt[m];
-            l = g.lse[m];
-            ycol = (int64_t)g.tgt[m] - g.col0;
-          } else if (g.crow) {
-            crow = g.crow[m];
-          }
-        }
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tc::tmem_ld32(tbase + c, r);
-          tc::tmem_ld_wait();
-          const int64_t nc = n0 + c;
-          if (!row_ok || nc >= N) continue;
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = nk ? u2f(r[j]) : 0.f;
-          if (g.epi == EPI_SWIGLU_BWD) {
-            epi_swiglu_bwd32(g, m, nc, N, v);
-            continue;
-          }
-          if (g.epi == EPI_CEGRAD) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float p = expf(v[j] - l);
-              if (nc + j == ycol) p -= 1.f;
-              v[j] = w * p;
-            }
-          } else if (g.alpha != 1.f) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= g.alpha;
-          }
-          epi_store32(g, crow, nc, N, v);
-        }
-      }
+      epilogue_tile(g, tbase, m, n0, M, N, nk);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tempty_bar[acc]);
@@ -388,6 +395,195 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   tc::fence_after_sync();
   if (threadIdx.x == 0 && abort_sh && args.err) atomicExch(args.err, DEV_TIMEOUT);
   if (warp == 1) tc::tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+
+// ============================================================================ CTA-pair kernel
+// The same GEMM on 256 x 256 tiles computed by a pair of CTAs (a 2-CTA cluster) with
+// tcgen05.mma.cta_group::2: each CTA stages 128 rows of A and 128 rows (N/2) of B per k-block,
+// the even CTA issues M=256 N=256 MMAs that read both CTAs' shared memory, and each CTA keeps
+// its 128 accumulator rows in its own TMEM.  Shared-memory traffic per MMA is half that of the
+// single-CTA kernel, which is what lets the tensor cores run closer to their peak.
+constexpr int BM2 = 256, STAGES2 = 6;
+constexpr int A2_BYTES = 128 * BK * 2;              // 16 KB per CTA
+constexpr int B2_BYTES = 128 * BK * 2;              // 16 KB per CTA (half of N)
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const TcArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full_bar[STAGES2], empty_bar[STAGES2], tfull_bar[2], tempty_bar[2];
+  __shared__ uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GemmDesc& g = args.g;
+  volatile int* abort_flag = &abort_sh;
+  const uint32_t rank = tc::cluster_ctarank();      // 0 = leader (issues the MMAs)
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      tc::mbar_init(&full_bar[s], 1);
+      tc::mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull_bar[a], 1);
+      tc::mbar_init(&tempty_bar[a], 8);      // 4 epilogue warps in each CTA of the pair
+    }
+    tc::mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tmap(&tmA);
+    tc::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc_pair(&tmem_base_sh, TMEM_COLS);
+    tc::tmem_relinquish_pair();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::cluster_sync();                        // barriers of both CTAs initialised
+  tc::fence_after_sync();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  const int64_t M = g.dynM ? (int64_t)*g.dynM : g.M;
+  const int64_t K = g.dynK ? (int64_t)*g.dynK : g.K;
+  const int64_t N = g.N;
+  const int nk = (int)((K + BK - 1) / BK);
+  const int ntiles = args.nM * args.nN;      // nM counts 256-row tiles here
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = cluster; t < ntiles && ok; t += nclusters) {
+        int mt, nt;
+        tile_coords(t, args.nM, args.nN, mt, nt);
+        const int m0 = mt * BM2, n0 = nt * BN;
+        if (m0 >= M) continue;
+        const int ma = m0 + 128 * (int)rank, nb = n0 + 128 * (int)rank;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + s * STAGE2_BYTES;
+          uint8_t* sb = sa + A2_BYTES;
+          const uint32_t fb = tc::mapa(tc::smem_u32(&full_bar[s]), 0);
+          if (rank == 0) tc::mbar_expect_tx(&full_bar[s], 2 * STAGE2_BYTES);
+          const int k0 = kb * BK;
+          if (!args.a_mn) {
+            tc::tma_load_2d_pair(sa, &tmA, fb, k0, ma);
+          } else {
+            tc::tma_load_2d_pair(sa, &tmA, fb, ma, k0);
+            tc::tma_load_2d_pair(sa + 8192, &tmA, fb, ma + 64, k0);
+          }
+          if (!args.b_mn) {
+            tc::tma_load_2d_pair(sb, &tmB, fb, k0, nb);
+          } else {
+            tc::tma_load_2d_pair(sb, &tmB, fb, nb, k0);
+            tc::tma_load_2d_pair(sb + 8192, &tmB, fb, nb + 64, k0);
+          }
+          issued_mask |= 1u << s;
+          issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
+          if (++s == STAGES2) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        // wind down: wait (bounded) for the pair's copies in flight on this CTA's barriers
+        const uint64_t t0 = tc::globaltimer_ns();
+        for (int q = 0; q < STAGES2; ++q) {
+          if (!(issued_mask & (1u << q))) continue;
+          const uint32_t p = (issued_phase >> q) & 1u;
+          while (!tc::mbar_try_wait(&full_bar[q], p) &&
+                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(BM2, BN, args.a_mn, args.b_mn);
+      const uint32_t smem_base = tc::smem_u32(smem);
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = cluster; t < ntiles && ok; t += nclusters) {
+        int mt, nt;
+        tile_coords(t, args.nM, args.nN, mt, nt);
+        if ((int64_t)mt * BM2 >= M) continue;
+        if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t sa = smem_base + s * STAGE2_BYTES;
+          const uint32_t sb = sa + A2_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                          : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                          : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc::mma_f16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc::mma_commit_pair(&empty_bar[s], 0x3);
+          if (++s == STAGES2) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc::mma_commit_pair(&tfull_bar[acc], 0x3);
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      if (issued) {
+        tc::mma_commit_pair(&drain_bar, 0x1);
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(&drain_bar, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t te_leader = tc::mapa(tc::smem_u32(&tempty_bar[0]), 0);
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = cluster; t < ntiles; t += nclusters) {
+      int mt, nt;
+      tile_coords(t, args.nM, args.nN, mt, nt);
+      const int64_t m0 = (int64_t)mt * BM2, n0 = (int64_t)nt * BN;
+      if (m0 >= M) continue;
+      if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) break;
+      tc::fence_after_sync();
+      const int64_t m = m0 + 128 * rank + row_in_tile;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_tile(g, tbase, m, n0, M, N, nk);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(te_leader + (uint32_t)(acc * sizeof(uint64_t)));
+      if (++acc == 2) { acc = 0; aph ^= 1u; }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::cluster_sync();                        // no CTA leaves while its peer may still signal it
+  tc::fence_after_sync();
+  if (threadIdx.x == 0 && abort_sh && args.err) atomicExch(args.err, DEV_TIMEOUT);
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -491,6 +687,50 @@ cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st) {
   const int grid = tiles < sm_count() ? tiles : sm_count();
   launch(gemm_tc_kernel, grid, kThreads, SMEM_BYTES, st, ma, mb, args);
   return cudaGetLastError();
+}
+
+
+// The CTA-pair kernel: 256 x 256 tiles; B boxes hold 128 rows (half of N) per CTA.
+cudaError_t gemm_tc_pair(const GemmDesc& g, int* err, cudaStream_t st) {
+  TcArgs args;
+  args.g = g;
+  args.a_mn = (g.sak == 1) ? 0 : 1;
+  args.b_mn = (g.sbk == 1) ? 0 : 1;
+  args.nM = (int)((g.M + BM2 - 1) / BM2);
+  args.nN = (int)((g.N + BN - 1) / BN);
+  args.err = err;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (!args.a_mn) ok = make_map(&ma, g.A, g.K, g.M, g.sam, 128);
+  else ok = make_map(&ma, g.A, g.M, g.K, g.sak, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  if (!args.b_mn) ok = make_map(&mb, g.B, g.K, g.N, g.sbn, 128);
+  else ok = make_map(&mb, g.B, g.N, g.K, g.sbk, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SMEM2_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = args.nM * args.nN;
+  const int pairs = sm_count() / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM2_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  prof_count_launch();
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, mb, args);
 }
 
 }  // namespace sbp

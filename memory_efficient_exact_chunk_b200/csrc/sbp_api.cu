@@ -685,13 +685,13 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
                                void* stream) {
   if (M <= 0 || N <= 0 || K <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
   if (!A || !B || !C || !workspace) return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
-  if (path < 0 || path > 2) return fail(SBP_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+  if (path < 0 || path > 4) return fail(SBP_ERR_INVALID_ARG, "path must be 0 .. 4");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   tl_status = static_cast<int*>(workspace);
   GemmDesc g = mk_gemm(M, N, K, DT_BF16, A, a_trans != 0, lda, DT_BF16, B, b_trans != 0, ldb,
                        DT_F32, C, ldc, accumulate ? EPI_ACC : EPI_STORE);
   g.path = path;
-  if (path == 2 && !gemm_tc_supported(g))
+  if (path >= 2 && !gemm_tc_supported(g))
     return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
   SBP_CK(gemm(g, st));
   return SBP_OK;

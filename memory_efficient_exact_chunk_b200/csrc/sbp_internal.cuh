@@ -126,7 +126,8 @@ struct GemmDesc {
   int64_t aux_ld = 0, aux_off = 0;
   // device status word raised on a bounded-wait timeout (nullable)
   int* err = nullptr;
-  // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores only
+  // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores (either kernel),
+  // 3 = tensor cores, single-CTA kernel, 4 = tensor cores, CTA-pair kernel
   int path = 0;
 };
 

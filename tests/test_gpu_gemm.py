@@ -13,10 +13,10 @@ def _ref(A, at, B, bt):
     return a @ b
 
 
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 3, 4])
 @pytest.mark.parametrize("at,bt", [(0, 1), (0, 0), (1, 1), (1, 0)])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 328, 136), (64, 8, 520), (392, 1032, 3584),
-                                   (8, 512, 8)])
+                                   (8, 512, 8), (1000, 776, 520)])
 def test_gemm_layouts(path, at, bt, M, N, K):
     import torch
     from memory_efficient_exact_chunk_b200 import sbp
@@ -44,9 +44,27 @@ def test_gemm_tensor_core_rejects_unaligned_layout():
     A = torch.randn(64, 20).to(torch.bfloat16).cuda()     # leading dimension 20: not a multiple of 8
     B = torch.randn(20, 64).to(torch.bfloat16).cuda()
     C = torch.zeros(64, 64, device="cuda")
-    with pytest.raises(sbp.SbpError) as ei:
-        sbp.debug_gemm_bf16(A, 0, B, 0, C, path=2)
-    assert ei.value.code == 2
+    for path in (2, 3, 4):
+        with pytest.raises(sbp.SbpError) as ei:
+            sbp.debug_gemm_bf16(A, 0, B, 0, C, path=path)
+        assert ei.value.code == 2
     sbp.debug_gemm_bf16(A, 0, B, 0, C, path=0)               # automatic: CUDA cores
     ref = _ref(A, 0, B, 0)
     assert ((C.double().cpu() - ref).norm() / ref.norm()).item() <= 1e-5
+
+
+def test_gemm_pair_kernel_large_ragged_accumulate():
+    """A product big enough for the automatic choice of the CTA-pair kernel, ragged edges."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(11)
+    M, N, K = 4000, 4616, 1032
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16).cuda()
+    ref = _ref(A, 0, B, 0)
+    for path in (0, 4):
+        C = torch.full((M, N), float("nan"), device="cuda")
+        ws = sbp.debug_gemm_bf16(A, 0, B, 0, C, path=path)
+        sbp.device_status(ws)
+        err = ((C.double().cpu() - ref).norm() / ref.norm()).item()
+        assert err <= 1e-5, (path, err)
