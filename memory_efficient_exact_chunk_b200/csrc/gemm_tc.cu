@@ -7,7 +7,8 @@
 // CTA tile 128 x 256 x 64, 4-stage TMA -> shared-memory ring, warp-specialised:
 //   warp 0      : TMA producer (one lane)
 //   warp 1      : TMEM allocator + MMA issuer (one lane), M=128 N=256 K=16 instructions
-//   warps 2..5  : epilogue, TMEM -> registers -> global (each warp owns 32 TMEM lanes)
+//   warps 2..9  : epilogue, TMEM -> registers -> global (each warp owns 32 TMEM lanes and half
+//                 of the tile's columns)
 // The accumulator is double-buffered in TMEM (2 x 256 columns) so the epilogue of tile i
 // overlaps the main loop of tile i+1.  One CTA per SM, grid = min(tiles, SMs).
 // Every mbarrier wait is bounded; on timeout the CTA raises the device status word, drains its
@@ -29,7 +30,8 @@ constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 constexpr int TMEM_COLS = 2 * BN;                    // double-buffered accumulator
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                        // 4 TMEM lane quarters x 2 column halves
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kGroupM = 8;                           // tile rasterisation group
 
 struct TcArgs {
@@ -142,15 +144,18 @@ __device__ __forceinline__ void epi_swiglu_bwd32(const GemmDesc& g, int64_t m, i
   }
 }
 
-// Epilogue of one accumulator tile for the calling thread's row m: columns [n0, n0 + BN) of the
-// tile are read from TMEM at tbase (this warp's lane quarter, accumulator base column).
+// Epilogue of one accumulator tile for the calling thread's row m: tile columns
+// [c_lo, c_lo + BN / 2) (this warp's half) starting at global column n0, read from TMEM at
+// tbase (this warp's lane quarter, accumulator base column).
 __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase, int64_t m,
-                                              int64_t n0, int64_t M, int64_t N, int nk) {
+                                              int64_t n0, int64_t M, int64_t N, int nk,
+                                              int c_lo) {
+  const int c_hi = c_lo + BN / 2;
   // the logit-gradient epilogue also writes the zero rows between the live row count and
   // the buffer's row count, so that a later product over those rows reads zeros
   const bool row_ok = m < (g.epi == EPI_CEGRAD ? g.M : M);
   if (g.epi == EPI_LSE) {
-    for (int c = 0; c < BN; c += 64) {
+    for (int c = c_lo; c < c_hi; c += 64) {
       uint32_t r0[32], r1[32];
       tc::tmem_ld32(tbase + c, r0);
       tc::tmem_ld32(tbase + c + 32, r1);
@@ -165,12 +170,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
         if (j < ncols) mx = fmaxf(mx, a);
         if (j + 32 < ncols) mx = fmaxf(mx, b);
       }
+      const float mxl = mx * tc::kLog2e;
       float sm = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float a = nk ? u2f(r0[j]) : 0.f, b = nk ? u2f(r1[j]) : 0.f;
-        if (j < ncols) sm += expf(a - mx);
-        if (j + 32 < ncols) sm += expf(b - mx);
+        if (j < ncols) sm += tc::ex2_approx(fmaf(a, tc::kLog2e, -mxl));
+        if (j + 32 < ncols) sm += tc::ex2_approx(fmaf(b, tc::kLog2e, -mxl));
       }
       const int64_t tile = nc / 64;
       g.pmax[m * g.pld + tile] = mx;
@@ -199,7 +205,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
         crow = g.crow[m];
       }
     }
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c_lo; c < c_hi; c += 32) {
       uint32_t r[32];
       tc::tmem_ld32(tbase + c, r);
       tc::tmem_ld_wait();
@@ -213,9 +219,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
         continue;
       }
       if (g.epi == EPI_CEGRAD) {
+        const float ll = l * tc::kLog2e;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          float p = expf(v[j] - l);
+          float p = tc::ex2_approx(fmaf(v[j], tc::kLog2e, -ll));
           if (nc + j == ycol) p -= 1.f;
           v[j] = w * p;
         }
@@ -250,7 +257,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tfull_bar[a], 1);
-      tc::mbar_init(&tempty_bar[a], 4);
+      tc::mbar_init(&tempty_bar[a], kEpiWarps);
     }
     tc::mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -368,9 +375,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row_in_tile = q * 32 + lane;
+    const int c_lo = ((warp - 2) >> 2) * (BN / 2);
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -382,7 +390,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc::fence_after_sync();
       const int64_t m = m0 + row_in_tile;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile(g, tbase, m, n0, M, N, nk);
+      epilogue_tile(g, tbase, m, n0, M, N, nk, c_lo);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tempty_bar[acc]);
@@ -434,7 +442,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tfull_bar[a], 1);
-      tc::mbar_init(&tempty_bar[a], 8);      // 4 epilogue warps in each CTA of the pair
+      tc::mbar_init(&tempty_bar[a], 2 * kEpiWarps);   // epilogue warps of both CTAs
     }
     tc::mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -552,9 +560,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
+    const int c_lo = ((warp - 2) >> 2) * (BN / 2);
     const uint32_t te_leader = tc::mapa(tc::smem_u32(&tempty_bar[0]), 0);
     int acc = 0;
     uint32_t aph = 0;
@@ -567,7 +576,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       tc::fence_after_sync();
       const int64_t m = m0 + 128 * rank + row_in_tile;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile(g, tbase, m, n0, M, N, nk);
+      epilogue_tile(g, tbase, m, n0, M, N, nk, c_lo);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive_cluster(te_leader + (uint32_t)(acc * sizeof(uint64_t)));
