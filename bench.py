@@ -354,6 +354,18 @@ def run_stack(args, rank, world, device):
     }
 
 
+def max_over_ranks(ms: float, world: int) -> float:
+    """The slowest rank's time (all ranks get it); plain value when there is one rank."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def timed(args, step, world, device, profile):
     """W warm-up steps, then K timed steps between a barrier + synchronize on both sides;
     device time from CUDA events on the launching stream, max over ranks."""
@@ -384,9 +396,7 @@ def timed(args, step, world, device, profile):
     clocks = clk.stop() if clk else None
     ms = ev0.elapsed_time(ev1)
     if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+        ms = max_over_ranks(ms, world)
         dist.barrier()
     return {"ms_total": ms, "ms": ms / args.steps, "prof": prof, "launches": launches,
             "clocks": clocks}

@@ -23,13 +23,17 @@ extern "C" {
  * C is [M, N] with leading dimension ldc; accumulate = 0 overwrites, 1 adds.
  * path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores (either kernel), 3 = tensor cores with
  * one CTA per 128 x 256 tile, 4 = tensor cores with a CTA pair per 256 x 256 tile
- * (SBP_ERR_UNSUPPORTED for 2..4 if the layout is not one the tensor-core kernels take).  `workspace` (>= 256 bytes, device) receives the
- * device status word (see sbp_get_device_status).  Device pointers, queued on `stream`.
+ * (SBP_ERR_UNSUPPORTED for 2..4 if the layout is not one the tensor-core kernels
+ * take).  kblk = 0 sums all of K in one accumulator; kblk > 0 (a multiple of 64, else
+ * SBP_ERR_INVALID_ARG) adds the partial products of consecutive K blocks of that length into
+ * C one after another, in fp32 (the rounding the weight-gradient products over tokens use).
+ * `workspace` (>= 256 bytes, device) receives the device status word (see
+ * sbp_get_device_status).  Device pointers, queued on `stream`.
  */
 sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int a_trans,
                                int64_t lda, const void* B, int b_trans, int64_t ldb, float* C,
-                               int64_t ldc, int accumulate, int path, void* workspace,
-                               void* stream);
+                               int64_t ldc, int accumulate, int path, int64_t kblk,
+                               void* workspace, void* stream);
 
 /*
  * Causal GQA attention forward of one query chunk over its key prefix (bf16):

@@ -10,7 +10,10 @@
 //          warp has already read (the A operand of the dV product, read from TMEM)
 //   dS^T = P^T (dP^T - delta)     -> bf16 tile in shared memory
 //   dV  += P^T dO (TMEM [256,384))          dK  += dS^T Q  (TMEM [384,512))
-// then dK, dV are added once into the fp32 prefix accumulators (single owner).
+// The query tiles are taken in blocks of a fixed number of tiles counted from the chunk start
+// (all heads of the group within a block); after each block dK, dV are added into the fp32
+// prefix accumulators (single owner, no atomics).  A chunk whose length is a multiple of the
+// block therefore adds exactly the partial sums the same queries give inside a longer chunk.
 //
 // dQ kernel: one CTA owns (sequence b, query head h, 128-query tile) and loops over the key
 // tiles of its causal prefix:  S = Q K^T, dP = dO V^T, dS = P (dP - delta) -> shared memory,
@@ -42,7 +45,7 @@ constexpr int QD_STAGES = 2;
 // the barriers.
 struct KvShared {
   float stat[2 /*QD_STAGES*/][2][BT];   // per stage: lse (log2 units), delta
-  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full, ds_full, mma2_done, drain;
+  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full, ds_full, mma2_done, kv_free, drain;
   uint32_t tmem;
   int abort;
 };
@@ -64,6 +67,7 @@ constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 384, C_DQ = 256;
 struct BwdArgs {
   int64_t B, T, Tc, s, H, Hkv;
   int nq, nkt;
+  int qb;               // query tiles per dK/dV accumulation block
   int64_t Tcp;          // Tc rounded up to the query tile
   const float* lse_t;   // [H, B, Tcp] log2 units, zero padded
   const float* delta_t; // [H, B, Tcp], zero padded
@@ -114,6 +118,36 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // ================================================================== dK / dV kernel
+// Pair j of a key tile's work: query head hh of the group and query tile qi (from i0 to
+// nq - 1), ordered block by block (qb tiles, counted from the chunk start) and head-major
+// inside a block; first / last: the pair opens / closes its block.
+struct PairPos {
+  int64_t hh, qi;
+  bool first, last;
+};
+__device__ __forceinline__ PairPos pair_at(int j, int64_t g, int64_t grp, int64_t i0, int64_t nq,
+                                           int64_t qb) {
+  const int64_t e0 = imin((i0 / qb + 1) * qb, nq);    // end of the first block
+  int64_t qs, nbt, w;
+  if (j < grp * (e0 - i0)) {
+    qs = i0;
+    nbt = e0 - i0;
+    w = j;
+  } else {
+    const int64_t jj = j - grp * (e0 - i0);
+    const int64_t fb = jj / (grp * qb);
+    qs = e0 + fb * qb;
+    nbt = imin(qb, nq - qs);
+    w = jj - fb * grp * qb;
+  }
+  PairPos p;
+  p.hh = g * grp + w / nbt;
+  p.qi = qs + w % nbt;
+  p.first = w == 0;
+  p.last = w == grp * nbt - 1;
+  return p;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -150,6 +184,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc::mbar_init(&sh.sdp_full, 1);
     tc::mbar_init(&sh.ds_full, kEwWarps);
     tc::mbar_init(&sh.mma2_done, 1);
+    tc::mbar_init(&sh.kv_free, kEwWarps);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
     tc::fence_barrier_init();
@@ -164,8 +199,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t tmem = sh.tmem;
 
   auto pair_coords = [&](int j, int64_t& hh, int64_t& qi) {
-    hh = g * grp + j / nqt;
-    qi = i0 + j % nqt;
+    const PairPos pp = pair_at(j, g, grp, i0, a.nq, a.qb);
+    hh = pp.hh;
+    qi = pp.qi;
   };
 
   if (warp == 0) {
@@ -215,7 +251,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                      aQ0 = tc::smem_u32(sQ0);
       bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag);
       bool issued = false;
+      int nflush = 0;
       for (int j = 0; j < npairs && ok; ++j) {
+        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
         const uint32_t ph = (uint32_t)j & 1u;
         const int st = j % QD_STAGES;
         const uint32_t sph = (uint32_t)(j / QD_STAGES) & 1u;
@@ -235,12 +273,17 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         issued = true;
         tc::mma_commit(&sh.sdp_full);
         if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
+        // a new block overwrites dK / dV: the element-wise warps must have added the last one
+        if (pos.first && j > 0) {
+          if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
+          ++nflush;
+        }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = queries
           const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;   // K-major operand step
           const uint32_t offm = kk * 2048;                            // MN-major operand step
-          const uint32_t acc = (j | kk) != 0;
+          const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
           // P^T (packed bf16) sits in TMEM: queries 64h.. of half h at C_DP + 64 h
           const uint32_t pcol = C_DP + 64 * (kk >> 2) + 8 * (kk & 3);
           mma_f16_ts(tmem + C_DV, tmem + pcol, tc::smem_desc_sw128(adO + offm, CHUNK, 1024),
@@ -266,11 +309,13 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int kpos = (int)(k_lo + r);
     const float scale_log2 = a.scale * 1.4426950408889634f;
     const int e32 = (int)e;
+    const bool kv = kpos < e32;
+    const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
     bool ok = true;
     for (int j = 0; j < npairs; ++j) {
       const uint32_t ph = (uint32_t)j & 1u;
-      int64_t hh, qi;
-      pair_coords(j, hh, qi);
+      const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
+      const int64_t qi = pos.qi;
       const int q0 = (int)(a.s + qi * BT);           // absolute position of query column 0
       // no masking needed when every key of the tile precedes every (valid) query of the tile
       const bool full = (k_lo + BT - 1 <= q0) && (qi * BT + BT <= a.Tc);
@@ -328,12 +373,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sh.ds_full);
-    }
-    // dK, dV of this key tile: add into the fp32 prefix accumulators (single owner)
-    if (ok && tc::mbar_wait_warp(&sh.mma2_done, (uint32_t)(npairs - 1) & 1u, abort_flag)) {
+      if (!pos.last) continue;
+      // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner)
+      if (!tc::mbar_wait_warp(&sh.mma2_done, ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
-      const bool kv = kpos < e32;
-      const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int c = half * 2 + cc;
@@ -360,6 +403,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
       }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0 && j + 1 < npairs) tc::mbar_arrive(&sh.kv_free);
     }
   }
 
@@ -688,10 +734,13 @@ cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   launch(attn_stats_kernel, dim3((unsigned)((nw * 32 + 255) / 256)), dim3(256), 0, st, B, Tc,
          Tcp, H, static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o),
          lse, lse_t, delta_t);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   BwdArgs a;
   a.B = B; a.T = T; a.Tc = Tc; a.s = s; a.H = H; a.Hkv = Hkv;
   a.nq = (int)((Tc + BT - 1) / BT);
   a.nkt = (int)((s + Tc + BT - 1) / BT);
+  a.qb = (int)(kTokenBlock / BT);
   a.Tcp = Tcp;
   a.lse_t = lse_t;
   a.delta_t = delta_t;
@@ -700,11 +749,28 @@ cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   a.dVp = dVp;
   a.scale = 1.f / sqrtf((float)HD);
   a.err = err;
+  // the two kernels are independent: the key-tile kernel (whose CTAs carry very unequal
+  // amounts of work) runs on a side stream so that the query-tile kernel fills its tail
+  SidePool* sp = side_pool();
+  cudaStream_t kv_st = st;
+  std::unique_lock<std::recursive_mutex> lk;
+  if (sp) {
+    lk = std::unique_lock<std::recursive_mutex>(sp->mu);
+    e = cudaEventRecord(sp->ev[14], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sp->s[2], sp->ev[14], 0);
+    if (e != cudaSuccess) return e;
+    kv_st = sp->s[2];
+  }
   launch(attn_bwd_kv_kernel, dim3((unsigned)(B * Hkv * a.nkt)), dim3(kThreads),
-         (size_t)KV_SMEM_BYTES, st, mq, mk, mv, mdo, a);
+         (size_t)KV_SMEM_BYTES, kv_st, mq, mk, mv, mdo, a);
   launch(attn_bwd_q_kernel, dim3((unsigned)(B * H * a.nq)), dim3(kThreads),
          (size_t)Q_SMEM_BYTES, st, mq, mk, mv, mdo, a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess && sp) {
+    e = cudaEventRecord(sp->ev[15], kv_st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sp->ev[15], 0);
+  }
+  return e;
 }
 
 }  // namespace sbp

@@ -16,6 +16,8 @@ static bool use_pair(const GemmDesc& g) {
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
+  if (g.kblk < 0 || (g.kblk > 0 && (g.kblk % 64 != 0 || (g.epi != EPI_STORE && g.epi != EPI_ACC))))
+    return cudaErrorInvalidValue;
   const bool tc = g.path != 1 && gemm_tc_supported(g);
   if (!tc && g.path >= 2) return cudaErrorNotSupported;
   const int kind = tc ? PROF_GEMM_TC : PROF_GEMM_SIMT;

@@ -29,11 +29,11 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
   const bool a_kmajor = (g.sak == 1);
   const bool b_nmajor = (g.sbn == 1);
 
-  float acc[4][4];
+  float acc[4][4], tot[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = tot[i][j] = 0.f;
 
   for (int64_t k0 = 0; k0 < K; k0 += BK) {
     // A tile [BM x BK]
@@ -72,6 +72,19 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
     __syncthreads();
+    // K blocks (kblk, a multiple of BK): partial sums restart at each block boundary
+    if (g.kblk > 0 && ((k0 + BK) % g.kblk == 0 || k0 + BK >= K)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { tot[i][j] += acc[i][j]; acc[i][j] = 0.f; }
+    }
+  }
+  if (g.kblk > 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = tot[i][j];
   }
 
   if (g.epi == EPI_STORE || g.epi == EPI_ACC) {

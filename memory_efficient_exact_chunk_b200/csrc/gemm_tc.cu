@@ -66,10 +66,12 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = pk;
 }
 
-// Store / accumulate 32 consecutive values v[0..31] of row `row` starting at column n.
+// Store / accumulate 32 consecutive values v[0..31] of row `row` starting at column n.  A
+// later K block (blk > 0) always accumulates and does not add the bias again.
 __device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int64_t n, int64_t N,
-                                            float (&v)[32]) {
-  if (g.bias) {
+                                            float (&v)[32], int blk) {
+  const bool accum = g.epi == EPI_ACC || blk > 0;
+  if (g.bias && blk == 0) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       if (n + j < N) v[j] += ld_dt(g.bias, g.bias_dt, n + j);
@@ -81,7 +83,7 @@ __device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int6
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
         float4 x = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        if (g.epi == EPI_ACC) {
+        if (accum) {
           const float4 o = *reinterpret_cast<const float4*>(c + j);
           x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
         }
@@ -89,7 +91,7 @@ __device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int6
       }
     } else {
       __nv_bfloat16* c = static_cast<__nv_bfloat16*>(g.C) + off;
-      if (g.epi == EPI_ACC) {
+      if (accum) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += __bfloat162float(c[j]);
       }
@@ -99,7 +101,7 @@ __device__ __forceinline__ void epi_store32(const GemmDesc& g, int64_t row, int6
   } else {
     for (int j = 0; j < 32 && n + j < N; ++j) {
       float x = v[j];
-      if (g.epi == EPI_ACC) x += ld_dt(g.C, g.cdt, off + j);
+      if (accum) x += ld_dt(g.C, g.cdt, off + j);
       st_dt(g.C, g.cdt, off + j, x);
     }
   }
@@ -146,10 +148,11 @@ __device__ __forceinline__ void epi_swiglu_bwd32(const GemmDesc& g, int64_t m, i
 
 // Epilogue of one accumulator tile for the calling thread's row m: tile columns
 // [c_lo, c_lo + BN / 2) (this warp's half) starting at global column n0, read from TMEM at
-// tbase (this warp's lane quarter, accumulator base column).
+// tbase (this warp's lane quarter, accumulator base column).  nk = the k-steps summed into
+// the accumulator (0: it holds nothing); blk = the index of its K block (see kblk).
 __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase, int64_t m,
                                               int64_t n0, int64_t M, int64_t N, int nk,
-                                              int c_lo) {
+                                              int c_lo, int blk) {
   const int c_hi = c_lo + BN / 2;
   // the logit-gradient epilogue also writes the zero rows between the live row count and
   // the buffer's row count, so that a later product over those rows reads zeros
@@ -230,7 +233,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] *= g.alpha;
       }
-      epi_store32(g, crow, nc, N, v);
+      epi_store32(g, crow, nc, N, v, blk);
     }
   }
 }
@@ -279,6 +282,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int64_t N = g.N;
   const int nk = (int)((K + BK - 1) / BK);
   const int ntiles = args.nM * args.nN;
+  // k-steps per K block and blocks per tile (one block, possibly empty, when kblk == 0)
+  const int kpb = g.kblk > 0 ? (int)(g.kblk / BK) : (nk > 0 ? nk : 1);
+  const int nblk = nk > 0 ? (nk + kpb - 1) / kpb : 1;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -342,29 +348,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         int mt, nt;
         tile_coords(t, args.nM, args.nN, mt, nt);
         if ((int64_t)mt * BM >= M) continue;
-        if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+        for (int b = 0; b < nblk && ok; ++b) {
+          if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
           tc::fence_after_sync();
-          const uint32_t sa = smem_base + s * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          const int kb0 = b * kpb, kb1 = imin(nk, kb0 + kpb);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint32_t sa = smem_base + s * STAGE_BYTES;
+            const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
-                                          : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                          : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
-            tc::mma_f16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                            : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                            : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
+              tc::mma_f16_ss(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0 ? 1u : 0u);
+            }
+            issued = true;
+            tc::mma_commit(&empty_bar[s]);
+            if (++s == STAGES) { s = 0; ph ^= 1u; }
           }
-          issued = true;
-          tc::mma_commit(&empty_bar[s]);
-          if (++s == STAGES) { s = 0; ph ^= 1u; }
+          if (!ok) break;
+          tc::mma_commit(&tfull_bar[acc]);
+          if (++acc == 2) { acc = 0; aph ^= 1u; }
         }
-        if (!ok) break;
-        tc::mma_commit(&tfull_bar[acc]);
-        if (++acc == 2) { acc = 0; aph ^= 1u; }
       }
       if (issued) {
         // make sure every MMA of this CTA has completed before TMEM is released
@@ -386,15 +395,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tile_coords(t, args.nM, args.nN, mt, nt);
       const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
       if (m0 >= M) continue;
-      if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) break;
-      tc::fence_after_sync();
-      const int64_t m = m0 + row_in_tile;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile(g, tbase, m, n0, M, N, nk, c_lo);
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&tempty_bar[acc]);
-      if (++acc == 2) { acc = 0; aph ^= 1u; }
+      bool ok = true;
+      for (int b = 0; b < nblk; ++b) {
+        if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const int64_t m = m0 + row_in_tile;
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+        epilogue_tile(g, tbase, m, n0, M, N, imin(nk - b * kpb, kpb), c_lo, b);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&tempty_bar[acc]);
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      if (!ok) break;
     }
   }
 
@@ -465,6 +478,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int64_t N = g.N;
   const int nk = (int)((K + BK - 1) / BK);
   const int ntiles = args.nM * args.nN;      // nM counts 256-row tiles here
+  const int kpb = g.kblk > 0 ? (int)(g.kblk / BK) : (nk > 0 ? nk : 1);
+  const int nblk = nk > 0 ? (nk + kpb - 1) / kpb : 1;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -528,29 +543,32 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         int mt, nt;
         tile_coords(t, args.nM, args.nN, mt, nt);
         if ((int64_t)mt * BM2 >= M) continue;
-        if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+        for (int b = 0; b < nblk && ok; ++b) {
+          if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
           tc::fence_after_sync();
-          const uint32_t sa = smem_base + s * STAGE2_BYTES;
-          const uint32_t sb = sa + A2_BYTES;
+          const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+          const int kb0 = b * kpb, kb1 = imin(nk, kb0 + kpb);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint32_t sa = smem_base + s * STAGE2_BYTES;
+            const uint32_t sb = sa + A2_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
-                                          : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                          : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
-            tc::mma_f16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                            : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                            : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
+              tc::mma_f16_ss_pair(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0 ? 1u : 0u);
+            }
+            issued = true;
+            tc::mma_commit_pair(&empty_bar[s], 0x3);
+            if (++s == STAGES2) { s = 0; ph ^= 1u; }
           }
-          issued = true;
-          tc::mma_commit_pair(&empty_bar[s], 0x3);
-          if (++s == STAGES2) { s = 0; ph ^= 1u; }
+          if (!ok) break;
+          tc::mma_commit_pair(&tfull_bar[acc], 0x3);
+          if (++acc == 2) { acc = 0; aph ^= 1u; }
         }
-        if (!ok) break;
-        tc::mma_commit_pair(&tfull_bar[acc], 0x3);
-        if (++acc == 2) { acc = 0; aph ^= 1u; }
       }
       if (issued) {
         tc::mma_commit_pair(&drain_bar, 0x1);
@@ -572,15 +590,19 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       tile_coords(t, args.nM, args.nN, mt, nt);
       const int64_t m0 = (int64_t)mt * BM2, n0 = (int64_t)nt * BN;
       if (m0 >= M) continue;
-      if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) break;
-      tc::fence_after_sync();
-      const int64_t m = m0 + 128 * rank + row_in_tile;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile(g, tbase, m, n0, M, N, nk, c_lo);
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive_cluster(te_leader + (uint32_t)(acc * sizeof(uint64_t)));
-      if (++acc == 2) { acc = 0; aph ^= 1u; }
+      bool ok = true;
+      for (int b = 0; b < nblk; ++b) {
+        if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const int64_t m = m0 + 128 * rank + row_in_tile;
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+        epilogue_tile(g, tbase, m, n0, M, N, imin(nk - b * kpb, kpb), c_lo, b);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive_cluster(te_leader + (uint32_t)(acc * sizeof(uint64_t)));
+        if (++acc == 2) { acc = 0; aph ^= 1u; }
+      }
+      if (!ok) break;
     }
   }
 

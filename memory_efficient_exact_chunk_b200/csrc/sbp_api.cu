@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "sbp.h"
@@ -75,7 +76,7 @@ struct CePlan {
   void* hc;
   int* yc;
   float *wc, *zy, *lse, *row_loss, *pmax, *psum;
-  void* G;
+  void* G[2];   // double-buffered logit-gradient block
   int64_t Rmax, tiles, Vb;
 };
 
@@ -94,7 +95,8 @@ void ce_carve(Carver& c, int64_t N, int64_t d, int64_t V, int D, int dt, CePlan&
   p.row_loss = c.take<float>(p.Rmax);
   p.pmax = c.take<float>((size_t)p.Rmax * p.tiles);
   p.psum = c.take<float>((size_t)p.Rmax * p.tiles);
-  p.G = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
+  p.G[0] = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
+  p.G[1] = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
 }
 
 // ------------------------------------------------------------------------ layer plan
@@ -178,6 +180,12 @@ GemmDesc mk_gemm(int64_t M, int64_t N, int64_t K, int adt, const void* A, bool a
   g.cdt = cdt; g.C = C; g.ldc = ldc;
   g.epi = epi;
   g.err = tl_status;
+  return g;
+}
+
+// A product that sums over tokens (a weight gradient): K blocks of kTokenBlock rows.
+GemmDesc over_tokens(GemmDesc g) {
+  g.kblk = kTokenBlock;
   return g;
 }
 
@@ -360,24 +368,48 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D,
     SBP_CK(gemm(g, st));
     SBP_CK(ce_finish(Rc, p.tiles, p.pmax, p.psum, p.tiles, p.count, p.wc, p.zy, p.lse,
                      p.row_loss, loss_out, i == 0, st));
-    // pass 2, one vocabulary block at a time: G = w (softmax - onehot), dH += G W_b,
-    // dW_b += G^T H
-    for (int64_t vb = 0; vb < V; vb += p.Vb) {
+    // pass 2, one vocabulary block at a time: G = w (softmax - onehot) on the caller's stream,
+    // then dH += G W_b and dW_b += G^T H on the two side streams while the next block's G is
+    // formed in the other buffer (dH stays in vocabulary order on its stream).
+    SidePool* sp = side_pool();
+    if (!sp) return fail(SBP_ERR_CUDA, "could not create the side streams");
+    std::lock_guard<std::recursive_mutex> side_lock(sp->mu);
+    SBP_CK(cudaEventRecord(sp->ev[0], st));
+    SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[0], 0));
+    SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[0], 0));
+    int blk = 0;
+    for (int64_t vb = 0; vb < V; vb += p.Vb, ++blk) {
+      const int buf = blk & 1;
       const int64_t nb = (V - vb) < p.Vb ? (V - vb) : p.Vb;
       const char* Wb = static_cast<const char*>(weight) + vb * d * dt_size(dt);
-      GemmDesc gg = mk_gemm(Rc, nb, d, dt, p.hc, false, d, dt, Wb, true, d, dt, p.G, nb,
+      if (blk >= 2) {   // the products of block blk - 2 have read this buffer
+        SBP_CK(cudaStreamWaitEvent(st, sp->ev[3 + buf], 0));
+        SBP_CK(cudaStreamWaitEvent(st, sp->ev[5 + buf], 0));
+      }
+      GemmDesc gg = mk_gemm(Rc, nb, d, dt, p.hc, false, d, dt, Wb, true, d, dt, p.G[buf], nb,
                             EPI_CEGRAD);
       gg.dynM = p.count; gg.lse = p.lse; gg.tgt = p.yc; gg.wt = p.wc; gg.col0 = vb;
       SBP_CK(gemm(gg, st));
-      GemmDesc gh = mk_gemm(Rc, d, nb, dt, p.G, false, nb, dt, Wb, false, d, DT_F32, d_hidden,
-                            d, vb == 0 ? EPI_STORE : EPI_ACC);
+      SBP_CK(cudaEventRecord(sp->ev[1 + buf], st));
+      SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[1 + buf], 0));
+      GemmDesc gh = mk_gemm(Rc, d, nb, dt, p.G[buf], false, nb, dt, Wb, false, d, DT_F32,
+                            d_hidden, d, vb == 0 ? EPI_STORE : EPI_ACC);
       gh.dynM = p.count; gh.crow = p.idx;
-      SBP_CK(gemm(gh, st));
-      GemmDesc gw = mk_gemm(nb, d, Rc, dt, p.G, true, nb, dt, p.hc, false, d, DT_F32,
+      SBP_CK(gemm(gh, sp->s[0]));
+      SBP_CK(cudaEventRecord(sp->ev[3 + buf], sp->s[0]));
+      SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[1 + buf], 0));
+      GemmDesc gw = mk_gemm(nb, d, Rc, dt, p.G[buf], true, nb, dt, p.hc, false, d, DT_F32,
                             d_weight + vb * d, d, EPI_ACC);
       gw.dynK = p.count;
-      SBP_CK(gemm(gw, st));
+      gw.kblk = kTokenBlock;
+      SBP_CK(gemm(gw, sp->s[1]));
+      SBP_CK(cudaEventRecord(sp->ev[5 + buf], sp->s[1]));
     }
+    // join: the next chunk reuses the compacted rows and the row map
+    SBP_CK(cudaEventRecord(sp->ev[3], sp->s[0]));
+    SBP_CK(cudaEventRecord(sp->ev[5], sp->s[1]));
+    SBP_CK(cudaStreamWaitEvent(st, sp->ev[3], 0));
+    SBP_CK(cudaStreamWaitEvent(st, sp->ev[5], 0));
   }
   return SBP_OK;
 }
@@ -437,6 +469,24 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
   SBP_CK(cudaMemsetAsync(p.Kp, 0, es * (size_t)B * T * dkv, st));
   SBP_CK(cudaMemsetAsync(p.Vp, 0, es * (size_t)B * T * dkv, st));
 
+  // Weight-gradient products run on two side streams next to the chain of data gradients on
+  // the caller's stream; each chunk ends with a join (its buffers are reused by the next one).
+  SidePool* sp = side_pool();
+  if (!sp) return fail(SBP_ERR_CUDA, "could not create the side streams");
+  std::lock_guard<std::recursive_mutex> side_lock(sp->mu);
+  auto fork_to = [&](int k, int ev) -> cudaError_t {
+    cudaError_t e = cudaEventRecord(sp->ev[ev], st);
+    return e == cudaSuccess ? cudaStreamWaitEvent(sp->s[k], sp->ev[ev], 0) : e;
+  };
+  auto join_all = [&]() -> cudaError_t {
+    cudaError_t e = cudaEventRecord(sp->ev[12], sp->s[0]);
+    if (e == cudaSuccess) e = cudaEventRecord(sp->ev[13], sp->s[1]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sp->ev[12], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sp->ev[13], 0);
+    return e;
+  };
+  cudaStream_t s0 = sp->s[0], s1 = sp->s[1];
+
   for (int i = 0; i < D; ++i) {
     int64_t s, e;
     chunk_range(T, D, i, s, e);
@@ -463,6 +513,9 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       dY = p.dyg16;
       dYdt = DT_BF16;
     }
+    SBP_CK(fork_to(0, 8));
+    SBP_CK(gemm(over_tokens(mk_gemm(d, f, R, dYdt, dY, true, d, dt, p.m, false, f, DT_F32,
+                                    gr->w_down, f, EPI_ACC)), s0));
     {
       // dM = dY W_d with the SwiGLU backward fused into the product's epilogue:
       // (dG, dU) = dM * (u sigma'(g) ..., silu(g)) written straight into dgu
@@ -473,17 +526,16 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       gd.aux_off = f;
       SBP_CK(gemm(gd, st));
     }
-    SBP_CK(gemm(mk_gemm(d, f, R, dYdt, dY, true, d, dt, p.m, false, f, DT_F32, gr->w_down, f,
-                        EPI_ACC), st));
     const char* dU = static_cast<const char*>(p.dgu) + f * es;
     SBP_CK(gemm(mk_gemm(R, d, f, dt, p.dgu, false, 2 * f, dt, w->w_gate, false, d, DT_F32, p.dn2,
                         d, EPI_STORE), st));
     SBP_CK(gemm(mk_gemm(R, d, f, dt, dU, false, 2 * f, dt, w->w_up, false, d, DT_F32, p.dn2, d,
                         EPI_ACC), st));
-    SBP_CK(gemm(mk_gemm(f, d, R, dt, p.dgu, true, 2 * f, dt, p.n2, false, d, DT_F32, gr->w_gate,
-                        d, EPI_ACC), st));
-    SBP_CK(gemm(mk_gemm(f, d, R, dt, dU, true, 2 * f, dt, p.n2, false, d, DT_F32, gr->w_up, d,
-                        EPI_ACC), st));
+    SBP_CK(fork_to(1, 9));
+    SBP_CK(gemm(over_tokens(mk_gemm(f, d, R, dt, p.dgu, true, 2 * f, dt, p.n2, false, d, DT_F32,
+                                    gr->w_gate, d, EPI_ACC)), s1));
+    SBP_CK(gemm(over_tokens(mk_gemm(f, d, R, dt, dU, true, 2 * f, dt, p.n2, false, d, DT_F32,
+                                    gr->w_up, d, EPI_ACC)), s1));
     SBP_CK(rmsnorm_bwd(R, d, DT_F32, p.hbuf, dt, w->ln2_g, p.rstd2, p.dn2, dyc, p.dh, 0,
                        gr->ln2_g, p.rpart, st));
     // ---- attention output projection backward
@@ -494,10 +546,11 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       dH = p.dh16;
       dHdt = DT_BF16;
     }
+    SBP_CK(fork_to(0, 10));
+    SBP_CK(gemm(over_tokens(mk_gemm(d, dq, R, dHdt, dH, true, d, dt, p.o, false, dq, DT_F32,
+                                    gr->wo, dq, EPI_ACC)), s0));
     SBP_CK(gemm(mk_gemm(R, dq, d, dHdt, dH, false, d, dt, w->wo, false, dq, dt, p.dO, dq,
                         EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(d, dq, R, dHdt, dH, true, d, dt, p.o, false, dq, DT_F32, gr->wo, dq,
-                        EPI_ACC), st));
     // ---- attention backward over the causal prefix; dK/dV accumulate in fp32
     SBP_CK(attn_bwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.dO, p.alse, p.delta,
                     p.dq, p.dKp, p.dVp, st));
@@ -512,14 +565,16 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       dQ = p.dq16;
       dQdt = DT_BF16;
     }
+    SBP_CK(fork_to(1, 11));
+    SBP_CK(gemm(over_tokens(mk_gemm(dq, d, R, dQdt, dQ, true, dq, dt, p.n1, false, d, DT_F32,
+                                    gr->wq, d, EPI_ACC)), s1));
+    if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, s1));
     SBP_CK(gemm(mk_gemm(R, d, dq, dQdt, dQ, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
                         EPI_STORE), st));
-    SBP_CK(gemm(mk_gemm(dq, d, R, dQdt, dQ, true, dq, dt, p.n1, false, d, DT_F32, gr->wq, d,
-                        EPI_ACC), st));
-    if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, st));
     SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, dxc, 0, gr->ln1_g,
                        p.rpart, st));
     if (B > 1) SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 0, st));
+    SBP_CK(join_all());
   }
   // ---- K/V projection backward, chunk by chunk, once every later chunk has added its dK/dV
   for (int j = 0; j < D; ++j) {
@@ -542,21 +597,22 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       const void* parts[4] = {p.khi, p.klo, p.vhi, p.vlo};
       const void* wts[4] = {w->wk, w->wk, w->wv, w->wv};
       float* grs[4] = {gr->wk, gr->wk, gr->wv, gr->wv};
-      for (int k = 0; k < 4; ++k) {
+      SBP_CK(fork_to(0, 8));
+      for (int k = 0; k < 4; ++k)
+        SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_BF16, parts[k], true, dkv, dt, p.n1, false,
+                                        d, DT_F32, grs[k], d, EPI_ACC)), s0));
+      for (int k = 0; k < 4; ++k)
         SBP_CK(gemm(mk_gemm(R, d, dkv, DT_BF16, parts[k], false, dkv, dt, wts[k], false, d,
                             DT_F32, p.dn1, d, k == 0 ? EPI_STORE : EPI_ACC), st));
-        SBP_CK(gemm(mk_gemm(dkv, d, R, DT_BF16, parts[k], true, dkv, dt, p.n1, false, d, DT_F32,
-                            grs[k], d, EPI_ACC), st));
-      }
     } else {
       SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
                           p.dn1, d, EPI_STORE), st));
       SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32,
                           p.dn1, d, EPI_ACC), st));
-      SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d, DT_F32,
-                          gr->wk, d, EPI_ACC), st));
-      SBP_CK(gemm(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d, DT_F32,
-                          gr->wv, d, EPI_ACC), st));
+      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d,
+                                      DT_F32, gr->wk, d, EPI_ACC)), st));
+      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d,
+                                      DT_F32, gr->wv, d, EPI_ACC)), st));
     }
     if (has_bias) {
       SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
@@ -570,6 +626,7 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, dx + s * d, 1,
                          gr->ln1_g, p.rpart, st));
     }
+    SBP_CK(join_all());
   }
   return SBP_OK;
 }
@@ -681,16 +738,19 @@ sbp_status sbp_embedding_backward(int64_t rows, int64_t cols, int64_t vocab,
 // ------------------------------------------------------------------------------- debug
 sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int a_trans,
                                int64_t lda, const void* B, int b_trans, int64_t ldb, float* C,
-                               int64_t ldc, int accumulate, int path, void* workspace,
-                               void* stream) {
+                               int64_t ldc, int accumulate, int path, int64_t kblk,
+                               void* workspace, void* stream) {
   if (M <= 0 || N <= 0 || K <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
   if (!A || !B || !C || !workspace) return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
   if (path < 0 || path > 4) return fail(SBP_ERR_INVALID_ARG, "path must be 0 .. 4");
+  if (kblk < 0 || kblk % 64 != 0)
+    return fail(SBP_ERR_INVALID_ARG, "kblk must be 0 or a positive multiple of 64");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   tl_status = static_cast<int*>(workspace);
   GemmDesc g = mk_gemm(M, N, K, DT_BF16, A, a_trans != 0, lda, DT_BF16, B, b_trans != 0, ldb,
                        DT_F32, C, ldc, accumulate ? EPI_ACC : EPI_STORE);
   g.path = path;
+  g.kblk = kblk;
   if (path >= 2 && !gemm_tc_supported(g))
     return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
   SBP_CK(gemm(g, st));

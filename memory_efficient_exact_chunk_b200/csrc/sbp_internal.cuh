@@ -6,9 +6,25 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <mutex>
 #include <utility>
 
 namespace sbp {
+
+// ---------------------------------------------------------------------------------------------
+// side streams (streams.cu): kSideStreams streams and kSideEvents events per device; `mu` is
+// held while one call queues work on them (keeps the event record / wait order of a call).
+// Events 0..7: LM head, 8..13: decoder layer, 14..15: attention backward.  Streams 0, 1:
+// products next to the caller's stream, 2: the attention backward's key-tile kernel.
+// ---------------------------------------------------------------------------------------------
+constexpr int kSideStreams = 3, kSideEvents = 16;
+struct SidePool {
+  std::recursive_mutex mu;
+  cudaStream_t s[kSideStreams] = {};
+  cudaEvent_t ev[kSideEvents] = {};
+  bool ok = false;
+};
+SidePool* side_pool();
 
 // ---------------------------------------------------------------------------------------------
 // launch accounting (profile.cu): every kernel of the library goes through launch(), which
@@ -124,6 +140,12 @@ struct GemmDesc {
   // SwiGLU-backward epilogue operand
   const void* aux = nullptr;
   int64_t aux_ld = 0, aux_off = 0;
+  // > 0: the accumulator is flushed into C after every kblk elements of K (a multiple of 64),
+  // so C is a left-to-right fp32 sum of partial products over consecutive K blocks that
+  // start at the GEMM's first K row.  Used on the reductions over tokens (weight gradients):
+  // a chunk whose length is a multiple of kblk then rounds exactly as the same tokens do
+  // inside a longer chunk.  Only with EPI_STORE / EPI_ACC.
+  int64_t kblk = 0;
   // device status word raised on a bounded-wait timeout (nullable)
   int* err = nullptr;
   // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores (either kernel),
@@ -133,6 +155,9 @@ struct GemmDesc {
 
 // Number of column tiles the EPI_LSE epilogue writes per row (its partial buffers' width).
 int64_t gemm_lse_tiles(int64_t N);
+
+// K-block length of every product that sums over tokens (weight gradients, see kblk).
+constexpr int64_t kTokenBlock = 1024;
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
 bool gemm_tc_supported(const GemmDesc& g);

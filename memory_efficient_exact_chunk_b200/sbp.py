@@ -97,7 +97,7 @@ def load(path: Optional[str] = None):
     lib.sbp_embedding_backward_workspace_size.argtypes = [i64, i64]
     lib.sbp_embedding_backward.argtypes = [i64, i64, i64, vp, vp, vp, vp, sz, vp]
     lib.sbp_debug_gemm_bf16.argtypes = [i64, i64, i64, vp, C.c_int, i64, vp, C.c_int, i64, vp, i64,
-                                         C.c_int, C.c_int, vp, vp]
+                                         C.c_int, C.c_int, i64, vp, vp]
     lib.sbp_lmhead_ce_backward_noalloc.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp]
     lib.sbp_debug_attn_fwd_bf16.argtypes = [i64] * 7 + [vp] * 5 + [C.c_int, vp, vp]
@@ -266,7 +266,8 @@ def embedding_backward(ids, dy2d, d_table, ws=None, stream=None):
 
 
 # ----------------------------------------------------------------------------- test hooks
-def debug_gemm_bf16(A, a_trans, B, b_trans, C, accumulate=False, path=0, ws=None, stream=None):
+def debug_gemm_bf16(A, a_trans, B, b_trans, C, accumulate=False, path=0, kblk=0, ws=None,
+                    stream=None):
     """C (+)= op(A) op(B) with bf16 A/B and fp32 C (see include/sbp_debug.h)."""
     M = A.shape[1] if a_trans else A.shape[0]
     K = A.shape[0] if a_trans else A.shape[1]
@@ -276,7 +277,8 @@ def debug_gemm_bf16(A, a_trans, B, b_trans, C, accumulate=False, path=0, ws=None
         ws.zero_()
     _check(load().sbp_debug_gemm_bf16(M, N, K, _ptr(A), int(a_trans), A.stride(0), _ptr(B),
                                       int(b_trans), B.stride(0), _ptr(C), C.stride(0),
-                                      int(accumulate), int(path), _ptr(ws), _stream(stream)))
+                                      int(accumulate), int(path), int(kblk), _ptr(ws),
+                                      _stream(stream)))
     return ws
 
 

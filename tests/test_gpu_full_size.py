@@ -1,0 +1,87 @@
+"""Checks at the full sizes the bench times (32K-token LM head, 32K-token Llama-3-8B layer), in
+the bench's launch configuration.  The oracle cannot run these sizes whole, so the checks are:
+sampled rows of d_hidden (each row depends only on its own hidden state) against the oracle,
+and D = 1 vs D = 8 agreement within 1e-5 for every output (the exactness of the chunking)."""
+import numpy as np
+import pytest
+
+from oracle import sbp_oracle as O
+from memory_efficient_exact_chunk_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel(a, b):
+    import torch
+    return ((a.double() - b.double()).norm() / b.double().norm().clamp_min(1e-300)).item()
+
+
+def test_lmhead_full_size():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    wl = synth.WORKLOADS["lmhead_ce_32k"]
+    T, d, V = wl.seq_len, wl.hidden, wl.vocab
+    h, W, y, w = synth.lmhead_inputs(77, T, d, V, bf16=True, from_frac=wl.loss_from_frac)
+    hd = torch.from_numpy(h).to(torch.bfloat16).cuda()
+    Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
+    yd = torch.from_numpy(y).cuda()
+    wd = torch.from_numpy(w).cuda()
+    out = {}
+    for D in (wl.num_chunks, 1):
+        loss = torch.zeros(1, device="cuda")
+        dH = torch.full((T, d), float("nan"), device="cuda")
+        dW = torch.zeros(V, d, device="cuda")
+        ws = sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW)
+        sbp.device_status(ws)
+        out[D] = (loss, dH, dW)
+        del ws
+    (l8, dH8, dW8), (l1, dH1, dW1) = out[wl.num_chunks], out[1]
+    errs = {"loss": abs(l8.item() - l1.item()) / abs(l1.item()), "dH": _rel(dH8, dH1),
+            "dW": _rel(dW8, dW1)}
+    assert all(v <= 1e-5 for v in errs.values()), errs
+    # sampled rows against the oracle (masked rows must be exactly zero)
+    masked = np.flatnonzero(w == 0)
+    live = np.flatnonzero(w != 0)
+    rng = np.random.default_rng(0)
+    rows = list(rng.choice(live, 5, replace=False)) + [int(live[0]), int(live[-1])]
+    W64 = W.astype(np.float64)
+    for r in rows:
+        _, dh0, _, _ = O.lmhead_ce_forward_backward(h[r:r + 1], W64, y[r:r + 1], w[r:r + 1])
+        got = dH8[r].double().cpu().numpy()
+        err = np.linalg.norm(got - dh0[0]) / np.linalg.norm(dh0[0])
+        assert err <= 1e-2, (r, err)
+    assert torch.all(dH8[torch.from_numpy(masked[:1000]).cuda()] == 0)
+
+
+def test_llama_layer_full_size_chunk_invariance():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    wl = synth.WORKLOADS["llama3_8b_layer_32k"]
+    L, B, T = wl.layer, wl.batch, wl.seq_len
+    W, x, dy = synth.layer_inputs(78, L, B, T, bf16=True, dy_std=1e-3)
+    names = sbp.WEIGHT_FIELDS
+    Wd = {n: (torch.from_numpy(W[n]).to(torch.bfloat16).cuda() if W.get(n) is not None else None)
+          for n in names}
+    xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    dyd = torch.from_numpy(dy).cuda()
+    res = {}
+    for D in (wl.num_chunks, 1):
+        cfg = sbp.layer_cfg(B, T, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
+                            L.rms_eps, L.rope_theta, sbp.SBP_BF16, D)
+        dx = torch.full((B, T, L.d_model), float("nan"), device="cuda")
+        g = {n: (torch.zeros(Wd[n].shape, device="cuda") if Wd.get(n) is not None else None)
+             for n in names}
+        ws = sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, g)
+        sbp.device_status(ws)
+        res[D] = (dx, g)
+        del ws
+        torch.cuda.empty_cache()
+    dx8, g8 = res[wl.num_chunks]
+    dx1, g1 = res[1]
+    assert torch.isfinite(dx8).all()
+    errs = {"dx": _rel(dx8, dx1)}
+    for n, v in g1.items():
+        if v is not None:
+            errs[n] = _rel(g8[n], v)
+    bad = {k: v for k, v in errs.items() if not v <= 1e-5}
+    assert not bad, errs

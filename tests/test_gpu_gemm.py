@@ -68,3 +68,41 @@ def test_gemm_pair_kernel_large_ragged_accumulate():
         sbp.device_status(ws)
         err = ((C.double().cpu() - ref).norm() / ref.norm()).item()
         assert err <= 1e-5, (path, err)
+
+
+@pytest.mark.parametrize("path", [1, 3, 4])
+@pytest.mark.parametrize("at", [0, 1])
+@pytest.mark.parametrize("K", [3072, 2504])
+def test_gemm_k_blocks_match_sliced_products(path, at, K):
+    """kblk: C equals, bit for bit, the same product taken as consecutive K slices of kblk
+    rows added into C one after another (the rounding a chunked token sum sees), and stays
+    within the fp32 bound of the exact product."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(K + at)
+    M, N, kb = 264, 520, 1024
+    A = torch.randn((K, M) if at else (M, K), generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16).cuda()
+    C = torch.full((M, N), float("nan"), device="cuda")
+    ws = sbp.debug_gemm_bf16(A, at, B, 0, C, path=path, kblk=kb)
+    sbp.device_status(ws)
+    Cs = torch.full((M, N), float("nan"), device="cuda")
+    for k0 in range(0, K, kb):
+        k1 = min(K, k0 + kb)
+        As = A[k0:k1] if at else A[:, k0:k1]
+        sbp.debug_gemm_bf16(As, at, B[k0:k1], 0, Cs, accumulate=k0 > 0, path=path, ws=ws)
+    sbp.device_status(ws)
+    assert torch.equal(C, Cs)
+    ref = _ref(A, at, B, 0)
+    assert ((C.double().cpu() - ref).norm() / ref.norm()).item() <= 1e-5
+
+
+def test_gemm_k_block_argument_checked():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    A = torch.zeros(64, 128, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(128, 64, dtype=torch.bfloat16, device="cuda")
+    C = torch.zeros(64, 64, device="cuda")
+    with pytest.raises(sbp.SbpError) as ei:
+        sbp.debug_gemm_bf16(A, 0, B, 0, C, kblk=100)
+    assert ei.value.code == 1
