@@ -26,6 +26,9 @@ enum {
 typedef struct {
   long long launches[SBP_PROF_KINDS]; /* timed calls per kind                                  */
   double ms[SBP_PROF_KINDS];          /* summed device time per kind, milliseconds            */
+  double busy_ms[SBP_PROF_KINDS];     /* device time during which at least one call of the kind
+                                         ran (the union of its intervals: calls the library runs
+                                         side by side on several streams are counted once)      */
 } sbp_profile;
 
 /* Number of kernels the library has launched in this process (all kinds). */

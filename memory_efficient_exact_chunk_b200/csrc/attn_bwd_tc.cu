@@ -114,6 +114,9 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -316,6 +319,14 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t ph = (uint32_t)j & 1u;
       const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
       const int64_t qi = pos.qi;
+      if (pos.first && kv) {
+        // bring this row's dK / dV accumulator lines into L2 ahead of the block's flush
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          prefetch_l2(a.dKp + ko + half * 64 + u * 32);
+          prefetch_l2(a.dVp + ko + half * 64 + u * 32);
+        }
+      }
       const int q0 = (int)(a.s + qi * BT);           // absolute position of query column 0
       // no masking needed when every key of the tile precedes every (valid) query of the tile
       const bool full = (k_lo + BT - 1 <= q0) && (qi * BT + BT <= a.Tc);
@@ -740,7 +751,7 @@ cudaError_t attn_bwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   a.B = B; a.T = T; a.Tc = Tc; a.s = s; a.H = H; a.Hkv = Hkv;
   a.nq = (int)((Tc + BT - 1) / BT);
   a.nkt = (int)((s + Tc + BT - 1) / BT);
-  a.qb = (int)(kTokenBlock / BT);
+  a.qb = (int)(kKvTokenBlock / BT);
   a.Tcp = Tcp;
   a.lse_t = lse_t;
   a.delta_t = delta_t;

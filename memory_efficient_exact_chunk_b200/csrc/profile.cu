@@ -1,6 +1,8 @@
 // Launch accounting and GEMM timing (the C interface is in include/sbp_profile.h).
-// While profiling is on, each GEMM launch is bracketed by two CUDA events on its own stream;
-// sbp_profile_end() synchronises, sums the elapsed times per kernel kind and frees the events.
+// While profiling is on, each GEMM / attention call is bracketed by two CUDA events on its own
+// stream; sbp_profile_end() synchronises, sums the elapsed times per kernel kind, measures the
+// union of each kind's intervals (calls on side streams overlap) and recycles the events.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -77,18 +79,45 @@ sbp_status sbp_profile_end(sbp_profile* out) {
     for (int k = 0; k < PROF_KINDS; ++k) {
       out->launches[k] = 0;
       out->ms[k] = 0.0;
+      out->busy_ms[k] = 0.0;
     }
   }
   sbp_status st = SBP_OK;
+  // intervals on one time axis: milliseconds from the first mark's start (may be negative
+  // for a call on another stream that started earlier)
+  std::vector<std::pair<double, double>> iv[PROF_KINDS];
   for (const Mark& m : g_marks) {
-    float ms = 0.f;
+    float ms = 0.f, t0 = 0.f;
     if (cudaEventSynchronize(m.b) != cudaSuccess ||
-        cudaEventElapsedTime(&ms, m.a, m.b) != cudaSuccess)
+        cudaEventElapsedTime(&ms, m.a, m.b) != cudaSuccess ||
+        cudaEventElapsedTime(&t0, g_marks.front().a, m.a) != cudaSuccess)
       st = SBP_ERR_CUDA;
     if (out && m.kind >= 0 && m.kind < PROF_KINDS) {
       out->launches[m.kind] += 1;
       out->ms[m.kind] += ms;
+      iv[m.kind].push_back({(double)t0, (double)t0 + (double)ms});
     }
+  }
+  if (out) {
+    for (int k = 0; k < PROF_KINDS; ++k) {
+      std::sort(iv[k].begin(), iv[k].end());
+      double busy = 0.0, lo = 0.0, hi = 0.0;
+      bool open = false;
+      for (const auto& x : iv[k]) {
+        if (open && x.first <= hi) {
+          hi = std::max(hi, x.second);
+          continue;
+        }
+        if (open) busy += hi - lo;
+        lo = x.first;
+        hi = x.second;
+        open = true;
+      }
+      if (open) busy += hi - lo;
+      out->busy_ms[k] = busy;
+    }
+  }
+  for (const Mark& m : g_marks) {
     g_pool.push_back(m.a);
     g_pool.push_back(m.b);
   }

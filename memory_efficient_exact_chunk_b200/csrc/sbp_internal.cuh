@@ -143,8 +143,8 @@ struct GemmDesc {
   // > 0: the accumulator is flushed into C after every kblk elements of K (a multiple of 64),
   // so C is a left-to-right fp32 sum of partial products over consecutive K blocks that
   // start at the GEMM's first K row.  Used on the reductions over tokens (weight gradients):
-  // a chunk whose length is a multiple of kblk then rounds exactly as the same tokens do
-  // inside a longer chunk.  Only with EPI_STORE / EPI_ACC.
+  // no accumulator sums more than kblk tokens, and a chunk whose length is a multiple of kblk
+  // rounds exactly as the same tokens do inside a longer chunk.  Only with EPI_STORE / EPI_ACC.
   int64_t kblk = 0;
   // device status word raised on a bounded-wait timeout (nullable)
   int* err = nullptr;
@@ -156,8 +156,15 @@ struct GemmDesc {
 // Number of column tiles the EPI_LSE epilogue writes per row (its partial buffers' width).
 int64_t gemm_lse_tiles(int64_t N);
 
-// K-block length of every product that sums over tokens (weight gradients, see kblk).
-constexpr int64_t kTokenBlock = 1024;
+// Longest run of tokens one tensor-core accumulator sums before its partial sum is added
+// into the fp32 result in a plain fp32 add: kTokenBlock for the weight-gradient products
+// (GemmDesc::kblk), kKvTokenBlock for the attention dK/dV sums over queries (which add all
+// query heads of a KV group, so their accumulators see four to eight times more terms per
+// token).  The accumulator's own rounding error grows with the number of terms it has added;
+// these blocks bound it, and a chunk whose length is a multiple of the block adds the same
+// partial sums as a longer chunk.
+constexpr int64_t kTokenBlock = 4096;
+constexpr int64_t kKvTokenBlock = 1024;
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
 bool gemm_tc_supported(const GemmDesc& g);

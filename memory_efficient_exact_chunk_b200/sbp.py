@@ -40,7 +40,8 @@ class SbpError(RuntimeError):
 
 
 class Profile(C.Structure):
-    _fields_ = [("launches", C.c_longlong * 4), ("ms", C.c_double * 4)]
+    _fields_ = [("launches", C.c_longlong * 4), ("ms", C.c_double * 4),
+                ("busy_ms", C.c_double * 4)]
 
 
 class LayerCfg(C.Structure):
@@ -295,7 +296,8 @@ def profile_end() -> dict:
     p = Profile()
     _check(load().sbp_profile_end(C.byref(p)))
     names = ("gemm_tc", "gemm_simt", "attn_fwd", "attn_bwd")
-    return {n: {"launches": p.launches[i], "ms": p.ms[i]} for i, n in enumerate(names)}
+    return {n: {"launches": p.launches[i], "ms": p.ms[i], "busy_ms": p.busy_ms[i]}
+            for i, n in enumerate(names)}
 
 
 def debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=0, ws=None, stream=None):

@@ -27,7 +27,7 @@ def test_lmhead_full_size():
     yd = torch.from_numpy(y).cuda()
     wd = torch.from_numpy(w).cuda()
     out = {}
-    for D in (wl.num_chunks, 1):
+    for D in (wl.num_chunks, 2 * wl.num_chunks, 1):
         loss = torch.zeros(1, device="cuda")
         dH = torch.full((T, d), float("nan"), device="cuda")
         dW = torch.zeros(V, d, device="cuda")
@@ -35,10 +35,14 @@ def test_lmhead_full_size():
         sbp.device_status(ws)
         out[D] = (loss, dH, dW)
         del ws
-    (l8, dH8, dW8), (l1, dH1, dW1) = out[wl.num_chunks], out[1]
-    errs = {"loss": abs(l8.item() - l1.item()) / abs(l1.item()), "dH": _rel(dH8, dH1),
-            "dW": _rel(dW8, dW1)}
-    assert all(v <= 1e-5 for v in errs.values()), errs
+    l1, dH1, dW1 = out[1]
+    for D in (wl.num_chunks, 2 * wl.num_chunks):
+        lD, dHD, dWD = out[D]
+        errs = {"loss": abs(lD.item() - l1.item()) / abs(l1.item()), "dH": _rel(dHD, dH1),
+                "dW": _rel(dWD, dW1)}
+        print(f"lmhead D={D} vs D=1:", errs)
+        assert all(v <= 1e-5 for v in errs.values()), (D, errs)
+    l8, dH8, dW8 = out[wl.num_chunks]
     # sampled rows against the oracle (masked rows must be exactly zero)
     masked = np.flatnonzero(w == 0)
     live = np.flatnonzero(w != 0)
@@ -65,7 +69,7 @@ def test_llama_layer_full_size_chunk_invariance():
     xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
     dyd = torch.from_numpy(dy).cuda()
     res = {}
-    for D in (wl.num_chunks, 1):
+    for D in (wl.num_chunks, 2 * wl.num_chunks, 1):
         cfg = sbp.layer_cfg(B, T, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
                             L.rms_eps, L.rope_theta, sbp.SBP_BF16, D)
         dx = torch.full((B, T, L.d_model), float("nan"), device="cuda")
@@ -76,12 +80,14 @@ def test_llama_layer_full_size_chunk_invariance():
         res[D] = (dx, g)
         del ws
         torch.cuda.empty_cache()
-    dx8, g8 = res[wl.num_chunks]
     dx1, g1 = res[1]
-    assert torch.isfinite(dx8).all()
-    errs = {"dx": _rel(dx8, dx1)}
-    for n, v in g1.items():
-        if v is not None:
-            errs[n] = _rel(g8[n], v)
-    bad = {k: v for k, v in errs.items() if not v <= 1e-5}
-    assert not bad, errs
+    for D in (wl.num_chunks, 2 * wl.num_chunks):
+        dxD, gD = res[D]
+        assert torch.isfinite(dxD).all()
+        errs = {"dx": _rel(dxD, dx1)}
+        for n, v in g1.items():
+            if v is not None:
+                errs[n] = _rel(gD[n], v)
+        print(f"layer D={D} vs D=1:", errs)
+        bad = {k: v for k, v in errs.items() if not v <= 1e-5}
+        assert not bad, (D, errs)
