@@ -4,26 +4,31 @@
 // depend on how the sequence was chunked):
 //
 // dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile) and loops over the query
-// heads of g's group and the chunk's query tiles that can see those keys.  Per pair:
-//   S^T  = K Q^T  (TMEM [0,128))            dP^T = V dO^T  (TMEM [128,256))
-//   P^T  = exp(S^T * scale - lse) -> bf16, written back into TMEM over dP^T columns the same
-//          warp has already read (the A operand of the dV product, read from TMEM)
-//   dS^T = P^T (dP^T - delta)     -> bf16 tile in shared memory
-//   dV  += P^T dO (TMEM [256,384))          dK  += dS^T Q  (TMEM [384,512))
+// heads of g's group and the chunk's query tiles that can see those keys.  Each (head, query
+// tile) pair is taken as two halves of 64 queries; per half h:
+//   S^T_h  = K Q_h^T   (TMEM c_s(h), 64 columns)     dP^T_h = V dO_h^T  (TMEM c_dp(h))
+//   P^T_h  = exp(S^T_h * scale - lse) -> bf16, written back into TMEM over the dP^T_h columns
+//            the same warp has already read (the A operand of the dV product)
+//   dS^T_h = P^T_h (dP^T_h - delta)    -> bf16, shared-memory buffer h
+//   dV    += P^T_h dO_h (TMEM [256,384))            dK += dS^T_h Q_h (TMEM [384,512))
+// The two halves have their own TMEM columns and dS^T buffers, so the tensor cores compute the
+// scores of one half (and the dV / dK products of the other) while the element-wise warps
+// turn the scores of a half into P^T and dS^T.
 // The query tiles are taken in blocks of a fixed number of tiles counted from the chunk start
 // (all heads of the group within a block); after each block dK, dV are added into the fp32
 // prefix accumulators (single owner, no atomics).  A chunk whose length is a multiple of the
 // block therefore adds exactly the partial sums the same queries give inside a longer chunk.
 //
 // dQ kernel: one CTA owns (sequence b, query head h, 128-query tile) and loops over the key
-// tiles of its causal prefix:  S = Q K^T, dP = dO V^T, dS = P (dP - delta) -> shared memory,
-// dQ += dS K (TMEM), stored once at the end.
+// tiles of its causal prefix, each as two halves of 64 keys:  S_h = Q K_h^T, dP_h = dO V_h^T,
+// dS_h = P_h (dP_h - delta) -> shared-memory buffer h, dQ += dS_h K_h (TMEM), stored once at
+// the end; the halves are pipelined the same way.
 //
 // Entries with key > query, queries outside the chunk and keys outside the prefix are masked
 // by selection (not by multiplication), so stale values never reach an accumulator.
 // Warp roles (both kernels): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..9
 // element-wise (the warp's TMEM lane quarter is its index mod 4; the two warps of a quarter
-// split the 128 columns in halves).
+// split the 64 columns of a half).
 #include <cuda.h>
 
 #include <mutex>
@@ -45,7 +50,7 @@ constexpr int QD_STAGES = 2;
 // the barriers.
 struct KvShared {
   float stat[2 /*QD_STAGES*/][2][BT];   // per stage: lse (log2 units), delta
-  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full, ds_full, mma2_done, kv_free, drain;
+  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full[2], ds_full[2], kvacc_done, kv_free, drain;
   uint32_t tmem;
   int abort;
 };
@@ -53,7 +58,7 @@ constexpr int KV_TILES_BYTES = (3 + 2 * QD_STAGES) * TILE;        // K, V, dS^T,
 constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
 constexpr int KV_RING = 2;                                         // K/V stages of the dQ kernel
 struct QShared {
-  uint64_t qd_full, kv_full[KV_RING], kv_empty[KV_RING], sdp_full, ds_full, dq_done, drain;
+  uint64_t qd_full, kv_full[KV_RING], kv_empty[KV_RING], sdp_full[2], ds_full[2], dq_done, drain;
   uint32_t tmem;
   int abort;
 };
@@ -62,7 +67,13 @@ constexpr int Q_SMEM_BYTES = Q_TILES_BYTES + (int)sizeof(QShared);
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 384, C_DQ = 256;
+// TMEM columns: half h of a tile keeps its scores at c_s(h) and their gradient at c_dp(h)
+// (64 columns each); the fp32 accumulators dV, dK (key-tile kernel) or dQ (query-tile kernel)
+// take the upper columns.
+constexpr uint32_t C_DV = 256, C_DK = 384, C_DQ = 256;
+__device__ __forceinline__ uint32_t c_s(int h) { return 128u * (uint32_t)h; }
+__device__ __forceinline__ uint32_t c_dp(int h) { return 128u * (uint32_t)h + 64u; }
+constexpr int HALF = TILE / 4;              // 64 rows x 128 bytes: a 64-row slice of a chunk
 
 struct BwdArgs {
   int64_t B, T, Tc, s, H, Hkv;
@@ -159,7 +170,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   KvShared& sh = *reinterpret_cast<KvShared*>(smem_raw + KV_TILES_BYTES);
   uint8_t* sK = smem_raw;
   uint8_t* sV = sK + TILE;
-  uint8_t* sdSt = sV + TILE;
+  uint8_t* sdSt = sV + TILE;                     // half h: dS^T [128 keys x 64 queries] at h*CHUNK
   uint8_t* sQ0 = sdSt + TILE;                    // stage st: Q at sQ0 + 2 st TILE, dO after it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
@@ -184,9 +195,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::mbar_init(&sh.qd_full[i], 1);
       tc::mbar_init(&sh.qd_empty[i], 1);
     }
-    tc::mbar_init(&sh.sdp_full, 1);
-    tc::mbar_init(&sh.ds_full, kEwWarps);
-    tc::mbar_init(&sh.mma2_done, 1);
+    for (int h = 0; h < 2; ++h) {
+      tc::mbar_init(&sh.sdp_full[h], 1);
+      tc::mbar_init(&sh.ds_full[h], kEwWarps);
+    }
+    tc::mbar_init(&sh.kvacc_done, 1);
     tc::mbar_init(&sh.kv_free, kEwWarps);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -201,12 +214,6 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc::fence_after_sync();
   const uint32_t tmem = sh.tmem;
 
-  auto pair_coords = [&](int j, int64_t& hh, int64_t& qi) {
-    const PairPos pp = pair_at(j, g, grp, i0, a.nq, a.qb);
-    hh = pp.hh;
-    qi = pp.qi;
-  };
-
   if (warp == 0) {
     if (lane == 0 && npairs > 0) {
       // ---------------------------------------------------------------- producer
@@ -219,22 +226,21 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < npairs; ++j) {
-        int64_t hh, qi;
-        pair_coords(j, hh, qi);
+        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
         if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
-        const int32_t qrow = (int32_t)(b * a.Tc + qi * BT);
+        const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
         tc::mbar_expect_tx(&sh.qd_full[st], 2 * TILE + 2 * BT * 4);
-        const int64_t srow = (hh * a.B + b) * a.Tcp + qi * BT;
+        const int64_t srow = (pos.hh * a.B + b) * a.Tcp + pos.qi * BT;
         tc::bulk_load(&sh.stat[st][0][0], a.lse_t + srow, BT * 4, &sh.qd_full[st]);
         tc::bulk_load(&sh.stat[st][1][0], a.delta_t + srow, BT * 4, &sh.qd_full[st]);
-        tc::tma_load_3d(sQ, &tmQ, &sh.qd_full[st], 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.qd_full[st], 64, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO, &tmdO, &sh.qd_full[st], 0, (int32_t)hh, qrow);
-        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)hh, qrow);
+        tc::tma_load_3d(sQ, &tmQ, &sh.qd_full[st], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sdO, &tmdO, &sh.qd_full[st], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
         issued = j + 1;
       }
       if (!ok) {
@@ -248,54 +254,78 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 1) {
     if (lane == 0 && npairs > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t id_kk = tc::idesc_bf16_f32(128, 128, 0, 0);   // A K-major, B K-major
-      const uint32_t id_km = tc::idesc_bf16_f32(128, 128, 0, 1);   // A K-major, B MN-major
+      // Two 64-query halves per pair, each with its own S^T / dP^T columns and dS^T buffer,
+      // so the scores of one half are computed while the element-wise warps work on the other.
+      const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);     // S^T, dP^T: N = 64 queries
+      const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dV, dK: B MN-major
       const uint32_t aK = tc::smem_u32(sK), aV = tc::smem_u32(sV), adS = tc::smem_u32(sdSt),
                      aQ0 = tc::smem_u32(sQ0);
       bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag);
       bool issued = false;
-      int nflush = 0;
-      for (int j = 0; j < npairs && ok; ++j) {
-        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
-        const uint32_t ph = (uint32_t)j & 1u;
-        const int st = j % QD_STAGES;
-        const uint32_t sph = (uint32_t)(j / QD_STAGES) & 1u;
-        const uint32_t aQ = aQ0 + 2 * st * TILE, adO = aQ + TILE;
-        if (!tc::mbar_wait(&sh.qd_full[st], sph, abort_flag)) { ok = false; break; }
-        // the previous pair's dV / dK products must have read P^T (TMEM) and dS^T (smem)
-        if (j >= 1 && !tc::mbar_wait(&sh.mma2_done, ph ^ 1u, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
+      // S^T_h = K Q_h^T and dP^T_h = V dO_h^T of pair j's half h
+      auto scores = [&](int j, int h) {
+        const uint32_t aQ = aQ0 + 2 * (j % QD_STAGES) * TILE, adO = aQ + TILE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
           const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + C_S, tc::smem_desc_sw128(aK + off, 16, 1024),
-                         tc::smem_desc_sw128(aQ + off, 16, 1024), id_kk, kk != 0);
-          tc::mma_f16_ss(tmem + C_DP, tc::smem_desc_sw128(aV + off, 16, 1024),
-                         tc::smem_desc_sw128(adO + off, 16, 1024), id_kk, kk != 0);
+          tc::mma_f16_ss(tmem + c_s(h), tc::smem_desc_sw128(aK + off, 16, 1024),
+                         tc::smem_desc_sw128(aQ + h * HALF + off, 16, 1024), id_s, kk != 0);
+          tc::mma_f16_ss(tmem + c_dp(h), tc::smem_desc_sw128(aV + off, 16, 1024),
+                         tc::smem_desc_sw128(adO + h * HALF + off, 16, 1024), id_s, kk != 0);
         }
+        tc::mma_commit(&sh.sdp_full[h]);
+      };
+      // dV += P^T_h dO_h (P^T from TMEM), dK += dS^T_h Q_h; `first`: the block's first product
+      auto grads = [&](int j, int h, bool first) {
+        const uint32_t aQ = aQ0 + 2 * (j % QD_STAGES) * TILE, adO = aQ + TILE;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries of the half
+          const uint32_t offm = (4 * h + kk) * 2048;                  // MN-major operand step
+          const uint32_t acc = (!first || kk != 0) ? 1u : 0u;
+          // packed P^T of queries 32 w.. of half h sits at c_dp(h) + 32 w (w = column half)
+          const uint32_t pcol = c_dp(h) + 32 * (kk >> 1) + 8 * (kk & 1);
+          mma_f16_ts(tmem + C_DV, tmem + pcol, tc::smem_desc_sw128(adO + offm, CHUNK, 1024),
+                     id_g, acc);
+          tc::mma_f16_ss(tmem + C_DK, tc::smem_desc_sw128(adS + h * CHUNK + kk * 32, 16, 1024),
+                         tc::smem_desc_sw128(aQ + offm, CHUNK, 1024), id_g, acc);
+        }
+      };
+      int nflush = 0;
+      if (ok && tc::mbar_wait(&sh.qd_full[0], 0, abort_flag)) {
+        tc::fence_after_sync();
+        scores(0, 0);
+        scores(0, 1);
         issued = true;
-        tc::mma_commit(&sh.sdp_full);
-        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
+      } else {
+        ok = false;
+      }
+      for (int j = 0; j < npairs && ok; ++j) {
+        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
+        const uint32_t ph = (uint32_t)j & 1u;
+        if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
         // a new block overwrites dK / dV: the element-wise warps must have added the last one
         if (pos.first && j > 0) {
           if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
           ++nflush;
         }
         tc::fence_after_sync();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = queries
-          const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;   // K-major operand step
-          const uint32_t offm = kk * 2048;                            // MN-major operand step
-          const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
-          // P^T (packed bf16) sits in TMEM: queries 64h.. of half h at C_DP + 64 h
-          const uint32_t pcol = C_DP + 64 * (kk >> 2) + 8 * (kk & 3);
-          mma_f16_ts(tmem + C_DV, tmem + pcol, tc::smem_desc_sw128(adO + offm, CHUNK, 1024),
-                     id_km, acc);
-          tc::mma_f16_ss(tmem + C_DK, tc::smem_desc_sw128(adS + offk, 16, 1024),
-                         tc::smem_desc_sw128(aQ + offm, CHUNK, 1024), id_km, acc);
+        grads(j, 0, pos.first);
+        const bool more = j + 1 < npairs;
+        if (more) {
+          const int st1 = (j + 1) % QD_STAGES;
+          if (!tc::mbar_wait(&sh.qd_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          scores(j + 1, 0);
         }
-        tc::mma_commit(&sh.mma2_done);
-        tc::mma_commit(&sh.qd_empty[st]);
+        if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        grads(j, 1, false);
+        tc::mma_commit(&sh.kvacc_done);
+        tc::mma_commit(&sh.qd_empty[j % QD_STAGES]);
+        if (more) scores(j + 1, 1);
       }
       if (issued) {
         tc::mma_commit(&sh.drain);
@@ -306,7 +336,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (npairs > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
-    const int half = (warp - 2) >> 2;                // column half of this warp
+    const int wh = (warp - 2) >> 2;                  // column half: queries 32 wh .. of a half
     const int r = q4 * 32 + lane;                    // TMEM lane = key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int kpos = (int)(k_lo + r);
@@ -315,41 +345,40 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const bool kv = kpos < e32;
     const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
     bool ok = true;
-    for (int j = 0; j < npairs; ++j) {
+    for (int j = 0; j < npairs && ok; ++j) {
       const uint32_t ph = (uint32_t)j & 1u;
       const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
-      const int64_t qi = pos.qi;
       if (pos.first && kv) {
         // bring this row's dK / dV accumulator lines into L2 ahead of the block's flush
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          prefetch_l2(a.dKp + ko + half * 64 + u * 32);
-          prefetch_l2(a.dVp + ko + half * 64 + u * 32);
+          prefetch_l2(a.dKp + ko + wh * 64 + u * 32);
+          prefetch_l2(a.dVp + ko + wh * 64 + u * 32);
         }
       }
-      const int q0 = (int)(a.s + qi * BT);           // absolute position of query column 0
-      // no masking needed when every key of the tile precedes every (valid) query of the tile
-      const bool full = (k_lo + BT - 1 <= q0) && (qi * BT + BT <= a.Tc);
       const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
-      const float* lse_s = sh.stat[st][0];
-      const float* delta_s = sh.stat[st][1];
       // acquire the bulk copies of this stage (already complete once the scores are ready)
       if (!tc::mbar_wait_warp(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
         break;
       }
-      if (!tc::mbar_wait_warp(&sh.sdp_full, ph, abort_flag)) { ok = false; break; }
-      tc::fence_after_sync();
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = half * 2 + cc;                 // 32-column slice
+      for (int h = 0; h < 2; ++h) {
+        const int qoff = 64 * h + 32 * wh;             // this warp's queries within the tile
+        const int q0 = (int)(a.s + pos.qi * BT) + qoff;  // absolute position of its first query
+        // no masking needed when every key of the tile precedes every (valid) query here
+        const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 32 <= a.Tc);
+        const float* lse_s = sh.stat[st][0] + qoff;
+        const float* delta_s = sh.stat[st][1] + qoff;
+        if (!tc::mbar_wait_warp(&sh.sdp_full[h], ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
         uint32_t rs[32], rd[32];
-        tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rs);
-        tc::tmem_ld32(tmem + lane_off + C_DP + c * 32, rd);
+        tc::tmem_ld32(tmem + lane_off + c_s(h) + 32 * wh, rs);
+        tc::tmem_ld32(tmem + lane_off + c_dp(h) + 32 * wh, rd);
         tc::tmem_ld_wait();
         uint32_t pp[16], dd[16];
-        const float4* l4 = reinterpret_cast<const float4*>(lse_s + c * 32);
-        const float4* d4 = reinterpret_cast<const float4*>(delta_s + c * 32);
+        const float4* l4 = reinterpret_cast<const float4*>(lse_s);
+        const float4* d4 = reinterpret_cast<const float4*>(delta_s);
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 lv = l4[i4], dv = d4[i4];
@@ -362,7 +391,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             p[k] = ex2(fmaf(__uint_as_float(rs[i]), scale_log2, -la[k]));
             gg[k] = p[k] * (__uint_as_float(rd[i]) - da[k]);
             if (!full) {
-              const int qpos = q0 + c * 32 + i;
+              const int qpos = q0 + i;
               const bool live = (kpos <= qpos) && (qpos < e32);
               p[k] = live ? p[k] : 0.f;
               gg[k] = live ? gg[k] : 0.f;
@@ -373,24 +402,27 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           dd[i4 * 2] = pack2(gg[0], gg[1]);
           dd[i4 * 2 + 1] = pack2(gg[2], gg[3]);
         }
-        // packed P over dP^T columns this warp has already read (queries 32 cc .. of its half)
-        tmem_st16(tmem + lane_off + C_DP + 64 * half + 16 * cc, pp);
+        // packed P^T over the dP^T columns this warp has just read
+        tmem_st16(tmem + lane_off + c_dp(h) + 32 * wh, pp);
+        // dS^T of this half (the previous pair's dK product of this half has read the buffer:
+        // its completion precedes the scores this warp has waited for)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          st_unit(sdSt, r, c * 4 + u, make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
+          st_unit(sdSt + h * CHUNK, r, 4 * wh + u,
+                  make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sh.ds_full[h]);
       }
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
-      if (!pos.last) continue;
+      if (!ok || !pos.last) continue;
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner)
-      if (!tc::mbar_wait_warp(&sh.mma2_done, ph, abort_flag)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&sh.kvacc_done, ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
-        const int c = half * 2 + cc;
+        const int c = wh * 2 + cc;
         uint32_t rk[32], rv[32];
         tc::tmem_ld32(tmem + lane_off + C_DK + c * 32, rk);
         tc::tmem_ld32(tmem + lane_off + C_DV + c * 32, rv);
@@ -439,7 +471,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   QShared& sh = *reinterpret_cast<QShared*>(smem_raw + Q_TILES_BYTES);
   uint8_t* sQ = smem_raw;
   uint8_t* sdO = sQ + TILE;
-  uint8_t* sdS = sdO + TILE;
+  uint8_t* sdS = sdO + TILE;                     // half h: dS [128 queries x 64 keys] at h*CHUNK
   uint8_t* sKV0 = sdS + TILE;                    // ring stage st: K at sKV0 + 2 st TILE, V after
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
@@ -460,8 +492,10 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       tc::mbar_init(&sh.kv_full[i], 1);
       tc::mbar_init(&sh.kv_empty[i], 1);
     }
-    tc::mbar_init(&sh.sdp_full, 1);
-    tc::mbar_init(&sh.ds_full, kEwWarps);
+    for (int hh = 0; hh < 2; ++hh) {
+      tc::mbar_init(&sh.sdp_full[hh], 1);
+      tc::mbar_init(&sh.ds_full[hh], kEwWarps);
+    }
     tc::mbar_init(&sh.dq_done, 1);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -512,43 +546,65 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else if (warp == 1) {
     if (lane == 0 && nkv > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t id_kk = tc::idesc_bf16_f32(128, 128, 0, 0);   // A K-major, B K-major
-      const uint32_t id_km = tc::idesc_bf16_f32(128, 128, 0, 1);   // A K-major, B MN-major
+      // Two 64-key halves per key tile, each with its own S / dP columns and dS buffer.
+      const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);     // S, dP: N = 64 keys
+      const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dQ: B MN-major
       const uint32_t aQ = tc::smem_u32(sQ), adO = tc::smem_u32(sdO), adS = tc::smem_u32(sdS),
                      aKV0 = tc::smem_u32(sKV0);
-      bool ok = tc::mbar_wait(&sh.qd_full, 0, abort_flag);
-      bool issued = false;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const uint32_t ph = (uint32_t)j & 1u;
-        const int st = j % KV_RING;
-        const uint32_t sph = (uint32_t)(j / KV_RING) & 1u;
-        const uint32_t aK = aKV0 + 2 * st * TILE, aV = aK + TILE;
-        if (!tc::mbar_wait(&sh.kv_full[st], sph, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-        // S and dP of this key tile (the element-wise warps have read the previous ones:
-        // ds_full of the previous tile was waited below)
+      // S_h = Q K_h^T and dP_h = dO V_h^T of key tile j's half hh
+      auto scores = [&](int j, int hh) {
+        const uint32_t aK = aKV0 + 2 * (j % KV_RING) * TILE, aV = aK + TILE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
           const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + C_S, tc::smem_desc_sw128(aQ + off, 16, 1024),
-                         tc::smem_desc_sw128(aK + off, 16, 1024), id_kk, kk != 0);
-          tc::mma_f16_ss(tmem + C_DP, tc::smem_desc_sw128(adO + off, 16, 1024),
-                         tc::smem_desc_sw128(aV + off, 16, 1024), id_kk, kk != 0);
+          tc::mma_f16_ss(tmem + c_s(hh), tc::smem_desc_sw128(aQ + off, 16, 1024),
+                         tc::smem_desc_sw128(aK + hh * HALF + off, 16, 1024), id_s, kk != 0);
+          tc::mma_f16_ss(tmem + c_dp(hh), tc::smem_desc_sw128(adO + off, 16, 1024),
+                         tc::smem_desc_sw128(aV + hh * HALF + off, 16, 1024), id_s, kk != 0);
         }
-        issued = true;
-        tc::mma_commit(&sh.sdp_full);
-        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
+        tc::mma_commit(&sh.sdp_full[hh]);
+      };
+      // dQ += dS_h K_h
+      auto dq_prod = [&](int j, int hh) {
+        const uint32_t aK = aKV0 + 2 * (j % KV_RING) * TILE;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = keys: dQ += dS K
-          const uint32_t offk = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + C_DQ, tc::smem_desc_sw128(adS + offk, 16, 1024),
-                         tc::smem_desc_sw128(aK + kk * 2048, CHUNK, 1024), id_km,
-                         (j | kk) != 0);
+        for (int kk = 0; kk < 4; ++kk) {   // K = 64 keys of the half
+          tc::mma_f16_ss(tmem + C_DQ, tc::smem_desc_sw128(adS + hh * CHUNK + kk * 32, 16, 1024),
+                         tc::smem_desc_sw128(aK + (4 * hh + kk) * 2048, CHUNK, 1024), id_g,
+                         (j | hh | kk) != 0 ? 1u : 0u);
         }
-        tc::mma_commit(&sh.dq_done);
-        tc::mma_commit(&sh.kv_empty[st]);
+      };
+      bool ok = tc::mbar_wait(&sh.qd_full, 0, abort_flag) &&
+                tc::mbar_wait(&sh.kv_full[0], 0, abort_flag);
+      bool issued = false;
+      if (ok) {
+        tc::fence_after_sync();
+        scores(0, 0);
+        scores(0, 1);
+        issued = true;
       }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const uint32_t ph = (uint32_t)j & 1u;
+        if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        dq_prod(j, 0);
+        const bool more = j + 1 < nkv;
+        if (more) {
+          const int st1 = (j + 1) % KV_RING;
+          if (!tc::mbar_wait(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          scores(j + 1, 0);
+        }
+        if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        dq_prod(j, 1);
+        tc::mma_commit(&sh.kv_empty[j % KV_RING]);
+        if (more) scores(j + 1, 1);
+      }
+      if (ok) tc::mma_commit(&sh.dq_done);
       if (issued) {
         tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
@@ -558,7 +614,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else if (nkv > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int wh = (warp - 2) >> 2;                  // column half: keys 32 wh .. of a half
     const int r = q4 * 32 + lane;                    // TMEM lane = query row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int t = (int)(q_lo + r);                   // absolute query position
@@ -568,20 +624,19 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const float dl_r = a.delta_t[srow];
     const float scale_log2 = a.scale * 1.4426950408889634f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; j < nkv && ok; ++j) {
       const uint32_t ph = (uint32_t)j & 1u;
-      const int k0 = j * BT;
-      const bool diag = k0 + BT - 1 > (int)q_lo;     // some key may follow some query
-      if (!tc::mbar_wait_warp(&sh.sdp_full, ph, abort_flag)) { ok = false; break; }
-      tc::fence_after_sync();
-      uint32_t dd[2][16];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = half * 2 + cc;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int k0 = j * BT + 64 * hh + 32 * wh;   // this warp's first key
+        const bool diag = k0 + 31 > (int)q_lo;       // some key may follow some query
+        if (!tc::mbar_wait_warp(&sh.sdp_full[hh], ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
         uint32_t rs[32], rd[32];
-        tc::tmem_ld32(tmem + lane_off + C_S + c * 32, rs);
-        tc::tmem_ld32(tmem + lane_off + C_DP + c * 32, rd);
+        tc::tmem_ld32(tmem + lane_off + c_s(hh) + 32 * wh, rs);
+        tc::tmem_ld32(tmem + lane_off + c_dp(hh) + 32 * wh, rd);
         tc::tmem_ld_wait();
+        uint32_t dd[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           float gg[2];
@@ -589,37 +644,31 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           for (int k = 0; k < 2; ++k) {
             const float p = ex2(fmaf(__uint_as_float(rs[i + k]), scale_log2, -lse_r));
             float v = p * (__uint_as_float(rd[i + k]) - dl_r);
-            if (diag) v = (k0 + c * 32 + i + k <= t && qv) ? v : 0.f;
+            if (diag) v = (k0 + i + k <= t && qv) ? v : 0.f;
             else v = qv ? v : 0.f;
             gg[k] = v;
           }
-          dd[cc][i >> 1] = pack2(gg[0], gg[1]);
+          dd[i >> 1] = pack2(gg[0], gg[1]);
         }
-      }
-      // dS may overwrite the previous tile's dS once its dQ product has read it
-      if (j >= 1) {
-        if (!tc::mbar_wait_warp(&sh.dq_done, ph ^ 1u, abort_flag)) { ok = false; break; }
-      }
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = half * 2 + cc;
+        // dS of this half (the previous tile's dQ product of this half has read the buffer:
+        // its completion precedes the scores this warp has waited for)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          st_unit(sdS, r, c * 4 + u,
-                  make_uint4(dd[cc][4 * u], dd[cc][4 * u + 1], dd[cc][4 * u + 2], dd[cc][4 * u + 3]));
+          st_unit(sdS + hh * CHUNK, r, 4 * wh + u,
+                  make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sh.ds_full[hh]);
       }
-      fence_proxy_async_smem();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
     }
     // dQ of this query tile, written once
-    if (ok && tc::mbar_wait_warp(&sh.dq_done, (uint32_t)(nkv - 1) & 1u, abort_flag)) {
+    if (ok && tc::mbar_wait_warp(&sh.dq_done, 0, abort_flag)) {
       tc::fence_after_sync();
       float* dqp = a.dq + ((b * a.Tc + (t - a.s)) * a.H + h) * HD;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
-        const int c = half * 2 + cc;
+        const int c = wh * 2 + cc;
         uint32_t rq[32];
         tc::tmem_ld32(tmem + lane_off + C_DQ + c * 32, rq);
         tc::tmem_ld_wait();
