@@ -99,6 +99,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def fit_inverse_d(sweep):
+    """Least-squares fit of the activation memory against D: workspace_gb ~ a / D + b.  a is
+    the part that shrinks with the chunk (O(T/D)), b the part that does not (for the layer,
+    the K/V prefix and the fp32 dK/dV accumulators)."""
+    if not sweep or len(sweep) < 2:
+        return None
+    x = np.array([1.0 / r["D"] for r in sweep])
+    y = np.array([r["workspace_gb"] for r in sweep])
+    A = np.stack([x, np.ones_like(x)], 1)
+    (a, b), *_ = np.linalg.lstsq(A, y, rcond=None)
+    res = y - A @ np.array([a, b])
+    return {"a_gb": float(a), "b_gb": float(b),
+            "max_abs_residual_gb": float(np.max(np.abs(res)))}
+
+
 # ----------------------------------------------------------------------------- workloads
 def lmhead_workload(T):
     from memory_efficient_exact_chunk_b200 import synth
@@ -175,6 +190,7 @@ def run_lmhead(args, rank, world, device):
                           "ms_per_step": r["ms"], "workspace_gb": wsc.numel() / 1e9})
             del wsc
         out["sweep"] = sweep
+        out["memory_fit"] = fit_inverse_d(sweep)
     # ---- end to end through the C ABI from pinned host buffers
     if args.e2e:
         hh = torch.from_numpy(h).to(torch.bfloat16).pin_memory()
@@ -276,18 +292,25 @@ def run_layer(args, rank, world, device, sweep=False):
             sw.append({"D": Dc, "tokens_per_s": B * T / (r["ms"] / 1e3), "ms_per_step": r["ms"],
                        "workspace_gb": ws.numel() / 1e9})
         out["sweep"] = sw
+        out["memory_fit"] = fit_inverse_d(sw)
     return out
 
 
-def run_stack(args, rank, world, device):
-    """Four Llama-3-8B-shaped layers + untied LM head (vocab 128256), bf16, T = 65536, D = 16,
-    targets = next token, mean CE over the last 75 % of tokens.  Weights are drawn on the
-    device from a seeded generator (N(0, 0.02), gains 1).  The forward (layer-input
-    checkpoints) and the streamed backward are timed separately; the metric is the backward."""
+def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k"):
+    """A decoder stack + untied LM head, bf16, through the streamed entry points:
+    llama3_8b_stack4_64k: four Llama-3-8B-shaped layers, vocabulary 128256, T = 65536, D = 16,
+        targets = next token, mean CE over the last 75 % of tokens;
+    qwen25_7b_stack2_grpo: two Qwen2.5-7B-shaped layers (QKV bias), vocabulary 152064,
+        8 sequences of 16384 tokens, D = 8, GRPO loss (per-sequence advantage N(0, 1) over
+        the response tokens after a 2048-token prompt).
+    Weights are drawn on the device from a seeded generator (N(0, 0.02), gains 1).  The
+    forward (layer-input checkpoints) and the streamed backward are timed separately; the
+    metric is the backward."""
     import torch
     from memory_efficient_exact_chunk_b200 import sbp, stack, synth
-    wl = synth.WORKLOADS["llama3_8b_stack4_64k"]
-    L, B, T, V = wl.layer, wl.batch, (args.stack_tokens or wl.seq_len), wl.vocab
+    wl = synth.WORKLOADS[name]
+    L, B, V = wl.layer, wl.batch, wl.vocab
+    T = (args.stack_tokens or wl.seq_len) if name.startswith("llama") else wl.seq_len
     D = wl.num_chunks
     gen = torch.Generator(device=device).manual_seed(3000 + rank)
 
@@ -297,18 +320,24 @@ def run_stack(args, rank, world, device):
     d, dq, dkv, f = L.d_model, L.n_heads * L.head_dim, L.n_kv_heads * L.head_dim, L.ffn
     layers = []
     for _ in range(wl.n_layers):
+        bias = L.qkv_bias
         layers.append({"ln1_g": torch.ones(d, dtype=torch.bfloat16, device=device),
                        "wq": rnd(dq, d), "wk": rnd(dkv, d), "wv": rnd(dkv, d), "wo": rnd(d, dq),
                        "ln2_g": torch.ones(d, dtype=torch.bfloat16, device=device),
                        "w_gate": rnd(f, d), "w_up": rnd(f, d), "w_down": rnd(d, f),
-                       "bq": None, "bk": None, "bv": None})
+                       "bq": rnd(dq) if bias else None, "bk": rnd(dkv) if bias else None,
+                       "bv": rnd(dkv) if bias else None})
     embed = rnd(V, d)
     lm_w = rnd(V, d)
     final_g = torch.ones(d, dtype=torch.bfloat16, device=device)
     rng = np.random.default_rng(3000 + rank)
     ids = synth.token_ids(rng, B, T, V)
     y = synth.shifted_targets(ids)
-    w = synth.loss_weights("shifted_tail", B, T, from_frac=wl.loss_from_frac)
+    if wl.loss == "grpo":
+        adv = rng.standard_normal(B)
+        w = synth.loss_weights("grpo", B, T, prompt_len=wl.prompt_len, advantages=adv)
+    else:
+        w = synth.loss_weights("shifted_tail", B, T, from_frac=wl.loss_from_frac)
     n_loss = int(np.count_nonzero(w))
     ids_d = torch.from_numpy(ids.reshape(-1)).to(device)
     y_d = torch.from_numpy(y.reshape(-1)).to(device)
@@ -338,7 +367,7 @@ def run_stack(args, rank, world, device):
     head = 8.0 * n_loss * d * V
     prof = rb["prof"]
     return {
-        "workload": wl.name if T == wl.seq_len else f"llama3_8b_stack4_{T}",
+        "workload": wl.name if T == wl.seq_len else f"{wl.name[:-4]}_{T}",
         "value": B * T * world / (rb["ms"] / 1e3), "unit": "tokens/s",
         "ms_per_step": rb["ms"], "forward_ms": rf["ms"],
         "fwd_bwd_tokens_per_s": B * T * world / ((rb["ms"] + rf["ms"]) / 1e3),
@@ -566,13 +595,15 @@ def main():
     }
     if "sweep" in out:
         line["sweep"] = out["sweep"]
+        line["memory_fit"] = out["memory_fit"]
     also = []
     if args.layer:
         also.append(run_layer(args, rank, world, device, sweep=args.sweep))
     if args.stack:
         import torch
-        torch.cuda.empty_cache()
-        also.append(run_stack(args, rank, world, device))
+        for name in ("llama3_8b_stack4_64k", "qwen25_7b_stack2_grpo"):
+            torch.cuda.empty_cache()
+            also.append(run_stack(args, rank, world, device, name))
     if also:
         line["also"] = also
     if "e2e" in out:
