@@ -409,3 +409,71 @@ def stack_forward_backward(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, 
     np.add.at(dE, ids.reshape(-1), dxl.reshape(B * T, -1))
     grads["embed"] = dE
     return loss, grads
+
+
+# ----------------------------------------------------------------------------------------------
+# DPO.  [paper] Abstract and [skill] Core Concept ("Multiple Objectives") and Practical
+# Guidance ("Loss Objectives") name DPO among the objectives StreamBP serves; the pages give no
+# formula.  Reading (listed in the design doc): the standard DPO objective on P pairs of sequences,
+#     loss = (1/P) sum_p -log sigmoid(beta * Delta_p),
+#     Delta_p = (logp(chosen_p) - ref(chosen_p)) - (logp(rejected_p) - ref(rejected_p)),
+# where logp(seq) is the sum of the token log-probabilities (= -CE) over the response tokens
+# (mask 1) and ref(.) are the reference model's sums, given.  Sequences are laid out
+# [chosen_0, rejected_0, chosen_1, rejected_1, ...], seq_len tokens each.  Because loss depends
+# on the network only through the per-token CE, its gradient is the gradient of sum_t w_t CE_t
+# with w_t = dloss / dCE_t, which is what the streamed backward takes as loss weights.
+# ----------------------------------------------------------------------------------------------
+def lmhead_token_ce(hidden, weight, targets, mask):
+    """Per-token cross-entropy lse(h W^T) - (h W^T)[y] [N]; 0 where mask == 0."""
+    h = np.asarray(hidden, F64)
+    W = np.asarray(weight, F64)
+    y = np.asarray(targets, np.int64)
+    m = np.asarray(mask, F64)
+    if np.any((y < 0) & (m != 0)):
+        raise ValueError("ignored target inside the mask")
+    z = h @ W.T
+    zmax = np.max(z, axis=1, keepdims=True)
+    lse = (zmax + np.log(np.sum(np.exp(z - zmax), axis=1, keepdims=True)))[:, 0]
+    z_y = z[np.arange(len(y)), np.where(y >= 0, y, 0)]
+    return np.where(m != 0, lse - z_y, 0.0)
+
+
+def _log_sigmoid(x):
+    x = np.asarray(x, F64)
+    return np.where(x >= 0, -np.log1p(np.exp(-x)), x - np.log1p(np.exp(x)))
+
+
+def dpo_objective(token_ce, mask, ref_logp, beta: float, n_pairs: int, seq_len: int):
+    """Returns (loss, w [2P*seq_len], seq_logp [2P]) with w_t = dloss / dCE_t."""
+    ce = np.asarray(token_ce, F64).reshape(2 * n_pairs, seq_len)
+    m = np.asarray(mask, F64).reshape(2 * n_pairs, seq_len)
+    ref = np.asarray(ref_logp, F64).reshape(2 * n_pairs)
+    logp = -np.sum(m * ce, axis=1)                       # sequence log-probabilities
+    delta = (logp[0::2] - ref[0::2]) - (logp[1::2] - ref[1::2])
+    loss = float(-np.mean(_log_sigmoid(beta * delta)))
+    # d loss / d Delta_p = -(beta / P) sigmoid(-beta Delta_p); d Delta / d CE_t = -1 on the
+    # chosen sequence's response tokens and +1 on the rejected one's
+    coef = beta * np.exp(_log_sigmoid(-beta * delta)) / n_pairs
+    sign = np.tile(np.array([1.0, -1.0]), n_pairs)       # chosen, rejected, ...
+    w = m * (np.repeat(coef, 2) * sign)[:, None]
+    return loss, w.reshape(-1), logp
+
+
+def stack_dpo(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, targets, mask, ref_logp,
+              beta: float, num_chunks: Optional[int] = None):
+    """DPO step on the small stack: forward for the sequence log-probabilities, the per-token
+    weights, then the (optionally chunked) backward with those weights.  ids/targets/mask
+    [2P, T].  Returns (dpo loss, grads, w)."""
+    ids = np.asarray(ids, np.int64)
+    B, T = ids.shape
+    E = np.asarray(embed, F64)
+    x = E[ids]
+    for W in layers:
+        x = decoder_layer_forward(cfg, W, x)
+    hf, _ = rmsnorm_forward(x, final_g, cfg.rms_eps)
+    ce = lmhead_token_ce(hf.reshape(B * T, -1), lm_w, np.asarray(targets).reshape(-1),
+                         np.asarray(mask).reshape(-1))
+    loss, w, _ = dpo_objective(ce, mask, ref_logp, beta, B // 2, T)
+    _, grads = stack_forward_backward(cfg, embed, layers, final_g, lm_w, ids, targets,
+                                      w.reshape(B, T), num_chunks)
+    return loss, grads, w

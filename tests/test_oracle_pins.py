@@ -364,3 +364,85 @@ def test_stack_finite_differences_and_chunks():
         assert np.isclose(loss2, loss, rtol=1e-13)
         assert np.allclose(g2["embed"], g["embed"], rtol=1e-11, atol=1e-14)
         assert np.allclose(g2["layers"][0]["wk"], g["layers"][0]["wk"], rtol=1e-11, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# DPO (the third objective the pages name; the standard DPO loss is the reading taken)
+def test_dpo_policy_equal_to_reference_closed_form():
+    """Delta = 0 for every pair: loss = ln 2 and w = +-beta / (2P) on the response tokens."""
+    rng = np.random.default_rng(40)
+    P, T, beta = 3, 5, 0.3
+    ce = np.abs(rng.standard_normal(2 * P * T))
+    m = (rng.random(2 * P * T) > 0.3).astype(np.float64)
+    ref = -(m * ce).reshape(2 * P, T).sum(1)
+    loss, w, logp = O.dpo_objective(ce, m, ref, beta, P, T)
+    assert np.isclose(loss, np.log(2.0), rtol=1e-15)
+    sign = np.repeat(np.tile([1.0, -1.0], P), T)
+    assert np.allclose(w, m * sign * beta / (2 * P), rtol=1e-15, atol=0)
+    assert np.allclose(logp, ref, rtol=1e-15)
+
+
+def test_dpo_swapping_roles_changes_loss_by_mean_beta_delta():
+    """softplus(x) - softplus(-x) = x: exchanging chosen and rejected raises the loss by
+    mean_p(beta Delta_p); sigmoid(x) + sigmoid(-x) = 1: the weights of a token before and after
+    the exchange have opposite signs and magnitudes adding up to beta / P."""
+    rng = np.random.default_rng(41)
+    P, T, beta = 4, 3, 0.7
+    ce = np.abs(rng.standard_normal(2 * P * T))
+    m = np.ones(2 * P * T)
+    ref = rng.standard_normal(2 * P) - 5.0
+    loss, w, logp = O.dpo_objective(ce, m, ref, beta, P, T)
+    perm = np.arange(2 * P).reshape(P, 2)[:, ::-1].reshape(-1)
+    loss_s, w_s, _ = O.dpo_objective(ce.reshape(2 * P, T)[perm].reshape(-1), m,
+                                     ref[perm], beta, P, T)
+    delta = (logp[0::2] - ref[0::2]) - (logp[1::2] - ref[1::2])
+    assert np.isclose(loss_s - loss, np.mean(beta * delta), rtol=1e-12)
+    ws = w_s.reshape(2 * P, T)[perm]
+    wo = w.reshape(2 * P, T)
+    assert np.all(np.sign(ws) == -np.sign(wo))
+    assert np.allclose(np.abs(ws) + np.abs(wo), beta / P, rtol=1e-14)
+
+
+def test_dpo_gradient_finite_differences_through_lm_head():
+    """The weights w_t = dloss/dCE_t turn the LM-head backward into the DPO gradient: dH and
+    dW from lmhead_ce_forward_backward(h, W, y, w) match central differences of the DPO loss."""
+    rng = np.random.default_rng(42)
+    P, T, d, V, beta = 2, 3, 4, 7, 0.5
+    N = 2 * P * T
+    h = rng.standard_normal((N, d))
+    W = rng.standard_normal((V, d))
+    y = rng.integers(0, V, N)
+    m = np.ones(N)
+    m[0::T] = 0.0                                    # first token of each sequence: prompt
+    ref = rng.standard_normal(2 * P) - 4.0
+
+    def loss_of():
+        return O.dpo_objective(O.lmhead_token_ce(h, W, y, m), m, ref, beta, P, T)[0]
+
+    _, w, _ = O.dpo_objective(O.lmhead_token_ce(h, W, y, m), m, ref, beta, P, T)
+    _, dH, dW, _ = O.lmhead_ce_forward_backward(h, W, y, w)
+    _fd_check(loss_of, h, [(1, 0), (4, 3), (7, 2), (11, 1)], dH)
+    _fd_check(loss_of, W, [(y[2], 1), (0, 0), (5, 3)], dW)
+
+
+def test_stack_dpo_finite_differences_and_chunks():
+    cfg = tiny_cfg(H=2, Hkv=1, hd=4, d=8, f=12)
+    rng = np.random.default_rng(43)
+    V, P, T, beta = 10, 1, 6, 0.4
+    layers = [tiny_weights(cfg, seed=44)]
+    E = rng.standard_normal((V, cfg.d_model))
+    fg = 1 + 0.1 * rng.standard_normal(cfg.d_model)
+    lm = 0.5 * rng.standard_normal((V, cfg.d_model))
+    ids = rng.integers(0, V, (2 * P, T))
+    ys = synth.shifted_targets(ids)
+    m = np.zeros((2 * P, T))
+    m[:, 2:T - 1] = 1.0                              # response predictions (last has no target)
+    ref = np.array([-9.0, -11.0])
+    f = lambda: O.stack_dpo(cfg, E, layers, fg, lm, ids, ys, m, ref, beta)[0]
+    loss, g, w = O.stack_dpo(cfg, E, layers, fg, lm, ids, ys, m, ref, beta)
+    _fd_check(f, lm, [(ys[0, 3], 1), (2, 5)], g["lm_head"])
+    _fd_check(f, layers[0]["wv"], [(1, 2), (3, 7)], g["layers"][0]["wv"])
+    _fd_check(f, E, [(ids[1, 1], 0)], g["embed"])
+    loss2, g2, _ = O.stack_dpo(cfg, E, layers, fg, lm, ids, ys, m, ref, beta, num_chunks=3)
+    assert np.isclose(loss2, loss, rtol=1e-15)
+    assert np.allclose(g2["layers"][0]["wq"], g["layers"][0]["wq"], rtol=1e-11, atol=1e-14)
