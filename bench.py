@@ -296,6 +296,83 @@ def run_layer(args, rank, world, device, sweep=False):
     return out
 
 
+def run_dpo_stack(args, rank, world, device, name="qwen25_7b_stack2_dpo"):
+    """A DPO step on the Qwen2.5-7B-shaped 2-layer stack: 4 (chosen, rejected) pairs of 16384
+    tokens (2048-token prompts), D = 8, beta 0.1.  One step = forward (layer-input checkpoints),
+    streamed LM-head forward for the sequence log-probabilities, DPO loss and weights, streamed
+    backward; all of it is timed.  The reference log-probabilities are the policy's own plus
+    N(0, 1) per sequence (computed once before timing)."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp, stack, synth
+    wl = synth.WORKLOADS[name]
+    L, B, T, V, D = wl.layer, wl.batch, wl.seq_len, wl.vocab, wl.num_chunks
+    beta = float(wl.extra["beta"])
+    gen = torch.Generator(device=device).manual_seed(4000 + rank)
+
+    def rnd(*shape):
+        return (torch.randn(*shape, generator=gen, device=device) * 0.02).to(torch.bfloat16)
+
+    d, dq, dkv, f = L.d_model, L.n_heads * L.head_dim, L.n_kv_heads * L.head_dim, L.ffn
+    layers = [{"ln1_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+               "wq": rnd(dq, d), "wk": rnd(dkv, d), "wv": rnd(dkv, d), "wo": rnd(d, dq),
+               "ln2_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+               "w_gate": rnd(f, d), "w_up": rnd(f, d), "w_down": rnd(d, f),
+               "bq": rnd(dq), "bk": rnd(dkv), "bv": rnd(dkv)} for _ in range(wl.n_layers)]
+    embed, lm_w = rnd(V, d), rnd(V, d)
+    final_g = torch.ones(d, dtype=torch.bfloat16, device=device)
+    rng = np.random.default_rng(4000 + rank)
+    ids = synth.token_ids(rng, B, T, V)
+    y = synth.shifted_targets(ids)
+    m = np.zeros((B, T), np.float32)
+    m[:, wl.prompt_len - 1:T - 1] = 1.0
+    ids_d = torch.from_numpy(ids.reshape(-1)).to(device)
+    y_d = torch.from_numpy(y.reshape(-1)).to(device)
+    m_d = torch.from_numpy(m.reshape(-1)).to(device)
+    cfg = sbp.layer_cfg(B, T, d, L.n_heads, L.n_kv_heads, L.head_dim, f, L.rms_eps, L.rope_theta,
+                        sbp.SBP_BF16, D)
+    ws = stack.Workspaces(device)
+    grads = stack.zero_grads(layers, lm_w, final_g, device, embed_shape=embed.shape)
+    # reference = the policy's sequence log-probabilities + N(0, 1)
+    xs, hf, _ = stack.stack_forward(cfg, embed, layers, final_g, ids_d, ws)
+    ce = torch.empty(B * T, device=device)
+    sbp.lmhead_ce_forward(hf, lm_w, y_d, m_d, D, ce)
+    logp = -(m_d * ce).view(B, T).sum(1)
+    ref = (logp + torch.randn(B, generator=gen, device=device)).float().contiguous()
+    del xs, hf
+    state = {}
+
+    def step():
+        state["r"] = stack.stack_dpo_step(cfg, embed, layers, final_g, lm_w, ids_d, y_d, m_d, ref,
+                                          beta, ws, grads=grads)
+
+    r = timed(argparse.Namespace(steps=1, warmup=args.warmup), step, world, device,
+              profile=True)
+    P = sum(int(layers[0][n].numel()) for n in ("wq", "wk", "wv", "wo", "w_gate", "w_up",
+                                                "w_down"))
+    n_loss = int(m.sum())
+    fwd_lin = 2.0 * P * B * T * wl.n_layers
+    lin = 6.0 * P * B * T * wl.n_layers
+    att = (14.0 + 4.0) * L.head_dim * L.n_heads * B * T * (T + 1) / 2 * wl.n_layers
+    head = (8.0 + 2.0) * n_loss * d * V          # backward + the log-probability forward
+    prof = r["prof"]
+    return {
+        "workload": wl.name, "value": B * T * world / (r["ms"] / 1e3), "unit": "tokens/s",
+        "ms_per_step": r["ms"], "dpo_loss": float(state["r"].loss.item()),
+        "config": {"batch": B, "pairs": B // 2, "seq_len": T, "n_layers": wl.n_layers,
+                   "vocab": V, "num_chunks": D, "prompt_len": wl.prompt_len, "beta": beta,
+                   "n_loss_tokens": n_loss},
+        "flops_step": {"layers_forward_2P": fwd_lin, "layers_linear_6P": lin,
+                       "layers_attention_18hd": att, "lmhead_10NdV": head},
+        "achieved_tflops_step": (fwd_lin + lin + att + head) / (r["ms"] / 1e3) / 1e12,
+        "kernels": {n: {"launches_per_step": v["launches"], "ms_per_step": v["ms"],
+                        "busy_ms_per_step": v["busy_ms"],
+                        "share": v["busy_ms"] / r["ms_total"] if r["ms_total"] else None}
+                    for n, v in prof.items() if v["launches"]},
+        "gpu_launches": r["launches"], "clocks": r["clocks"],
+        "workspace_gb": sum(t.numel() for t in ws.bufs.values()) / 1e9,
+    }
+
+
 def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k"):
     """A decoder stack + untied LM head, bf16, through the streamed entry points:
     llama3_8b_stack4_64k: four Llama-3-8B-shaped layers, vocabulary 128256, T = 65536, D = 16,
@@ -604,6 +681,8 @@ def main():
         for name in ("llama3_8b_stack4_64k", "qwen25_7b_stack2_grpo"):
             torch.cuda.empty_cache()
             also.append(run_stack(args, rank, world, device, name))
+        torch.cuda.empty_cache()
+        also.append(run_dpo_stack(args, rank, world, device))
     if also:
         line["also"] = also
     if "e2e" in out:

@@ -132,35 +132,45 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // ================================================================== dK / dV kernel
-// Pair j of a key tile's work: query head hh of the group and query tile qi (from i0 to
-// nq - 1), ordered block by block (qb tiles, counted from the chunk start) and head-major
-// inside a block; first / last: the pair opens / closes its block.
+// The work of a key tile, pair by pair: (query head hh of the group, query tile qi) for the
+// query tiles i0 .. nq - 1, ordered block by block (qb tiles, counted from the chunk start)
+// and head-major inside a block; first / last: the pair opens / closes its block.  Every role
+// of the CTA walks the same sequence with its own iterator (no divisions per pair).
 struct PairPos {
   int64_t hh, qi;
   bool first, last;
 };
-__device__ __forceinline__ PairPos pair_at(int j, int64_t g, int64_t grp, int64_t i0, int64_t nq,
-                                           int64_t qb) {
-  const int64_t e0 = imin((i0 / qb + 1) * qb, nq);    // end of the first block
-  int64_t qs, nbt, w;
-  if (j < grp * (e0 - i0)) {
+struct PairIter {
+  int qs, nbt, hi, t;       // block start tile, tiles in the block, head in group, tile in block
+  int grp, qb, nq;
+  __device__ __forceinline__ void init(int i0, int nq_, int grp_, int qb_) {
+    grp = grp_;
+    qb = qb_;
+    nq = nq_;
     qs = i0;
-    nbt = e0 - i0;
-    w = j;
-  } else {
-    const int64_t jj = j - grp * (e0 - i0);
-    const int64_t fb = jj / (grp * qb);
-    qs = e0 + fb * qb;
-    nbt = imin(qb, nq - qs);
-    w = jj - fb * grp * qb;
+    nbt = min((i0 / qb + 1) * qb, nq) - i0;
+    hi = 0;
+    t = 0;
   }
-  PairPos p;
-  p.hh = g * grp + w / nbt;
-  p.qi = qs + w % nbt;
-  p.first = w == 0;
-  p.last = w == grp * nbt - 1;
-  return p;
-}
+  __device__ __forceinline__ PairPos pos(int64_t g) const {
+    PairPos p;
+    p.hh = g * grp + hi;
+    p.qi = qs + t;
+    p.first = hi == 0 && t == 0;
+    p.last = hi == grp - 1 && t == nbt - 1;
+    return p;
+  }
+  __device__ __forceinline__ void next() {
+    if (++t == nbt) {
+      t = 0;
+      if (++hi == grp) {
+        hi = 0;
+        qs += nbt;
+        nbt = min(qb, nq - qs);
+      }
+    }
+  }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -225,8 +235,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full, 64, (int32_t)g, krow);
       bool ok = true;
       int issued = 0;
-      for (int j = 0; j < npairs; ++j) {
-        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
+      PairIter it;
+      it.init((int)i0, a.nq, (int)grp, a.qb);
+      for (int j = 0; j < npairs; ++j, it.next()) {
+        const PairPos pos = it.pos(g);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
         if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
@@ -299,8 +311,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       } else {
         ok = false;
       }
-      for (int j = 0; j < npairs && ok; ++j) {
-        const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
+      PairIter it;
+      it.init((int)i0, a.nq, (int)grp, a.qb);
+      for (int j = 0; j < npairs && ok; ++j, it.next()) {
+        const PairPos pos = it.pos(g);
         const uint32_t ph = (uint32_t)j & 1u;
         if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
         // a new block overwrites dK / dV: the element-wise warps must have added the last one
@@ -345,9 +359,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const bool kv = kpos < e32;
     const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
     bool ok = true;
-    for (int j = 0; j < npairs && ok; ++j) {
+    PairIter it;
+    it.init((int)i0, a.nq, (int)grp, a.qb);
+    for (int j = 0; j < npairs && ok; ++j, it.next()) {
       const uint32_t ph = (uint32_t)j & 1u;
-      const PairPos pos = pair_at(j, g, grp, i0, a.nq, a.qb);
+      const PairPos pos = it.pos(g);
       if (pos.first && kv) {
         // bring this row's dK / dV accumulator lines into L2 ahead of the block's flush
 #pragma unroll

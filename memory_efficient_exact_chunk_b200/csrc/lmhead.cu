@@ -116,7 +116,26 @@ __global__ void ce_loss_kernel(const int* __restrict__ count, const float* __res
   }
 }
 
+__global__ void ce_token_scatter_kernel(int64_t Rmax, const int* __restrict__ idx,
+                                        const int* __restrict__ count,
+                                        const float* __restrict__ lse,
+                                        const float* __restrict__ zy, float* __restrict__ token_ce) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= Rmax || r >= count[0]) return;
+  token_ce[idx[r]] = lse[r] - zy[r];
+}
+
 }  // namespace
+
+cudaError_t ce_token_scatter(int64_t s, int64_t e, int64_t Rmax, const int* idx, const int* count,
+                             const float* lse, const float* zy, float* token_ce, cudaStream_t st) {
+  if (e <= s) return cudaSuccess;
+  cudaError_t err = cudaMemsetAsync(token_ce + s, 0, sizeof(float) * (size_t)(e - s), st);
+  if (err != cudaSuccess || Rmax <= 0) return err;
+  launch(ce_token_scatter_kernel, (unsigned)((Rmax + 255) / 256), 256, 0, st, Rmax, idx, count,
+         lse, zy, token_ce);
+  return cudaGetLastError();
+}
 
 cudaError_t ce_compact(int64_t s, int64_t e, int64_t V, const int* tgt, const float* w, int* idx,
                        int* count, int* status, cudaStream_t st) {

@@ -12,6 +12,7 @@
 
 #include "sbp.h"
 #include "sbp_debug.h"
+#include "sbp_dpo.h"
 #include "sbp_internal.cuh"
 
 using namespace sbp;
@@ -76,6 +77,7 @@ struct CePlan {
   void* hc;
   int* yc;
   float *wc, *zy, *lse, *row_loss, *pmax, *psum;
+  float* loss_tmp;   // loss accumulator when the caller passes none (forward entry)
   void* G[2];   // double-buffered logit-gradient block
   int64_t Rmax, tiles, Vb;
 };
@@ -95,6 +97,7 @@ void ce_carve(Carver& c, int64_t N, int64_t d, int64_t V, int D, int dt, CePlan&
   p.row_loss = c.take<float>(p.Rmax);
   p.pmax = c.take<float>((size_t)p.Rmax * p.tiles);
   p.psum = c.take<float>((size_t)p.Rmax * p.tiles);
+  p.loss_tmp = c.take<float>(64);
   p.G[0] = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
   p.G[1] = c.take_bytes((size_t)p.Rmax * p.Vb * dt_size(dt));
 }
@@ -411,6 +414,80 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D,
     SBP_CK(cudaStreamWaitEvent(st, sp->ev[3], 0));
     SBP_CK(cudaStreamWaitEvent(st, sp->ev[5], 0));
   }
+  return SBP_OK;
+}
+
+sbp_status sbp_lmhead_ce_forward_stream(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt,
+                                        const void* hidden_states, const void* weight,
+                                        const int32_t* targets, const float* loss_weights,
+                                        float* token_ce, float* loss_out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (N <= 0 || d <= 0 || V <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (D < 1 || (int64_t)D > N)
+    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= n_tokens");
+  if (dt != SBP_F32 && dt != SBP_BF16) return fail(SBP_ERR_INVALID_ARG, "unknown dtype");
+  if (dt == SBP_BF16 && d % 8 != 0) return fail(SBP_ERR_UNSUPPORTED, "bf16 needs hidden % 8 == 0");
+  const void* ptrs[] = {hidden_states, weight, targets, loss_weights, token_ce};
+  for (const void* q : ptrs) {
+    if (!q) return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "a pointer is not 16-byte aligned");
+  }
+  const size_t need = sbp_lmhead_ce_workspace_size(N, d, V, D, dt);
+  if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  CePlan p;
+  ce_carve(c, N, d, V, D, dt, p);
+  tl_status = p.status;
+  SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
+  float* lo = loss_out ? loss_out : p.loss_tmp;
+  for (int i = 0; i < D; ++i) {
+    int64_t s, e;
+    chunk_range(N, D, i, s, e);
+    const int64_t Rc = e - s;
+    SBP_CK(ce_compact(s, e, V, targets, loss_weights, p.idx, p.count, p.status, st));
+    SBP_CK(ce_gather(Rc, d, dt, hidden_states, p.idx, p.count, targets, loss_weights, p.hc, p.yc,
+                     p.wc, p.zy, p.lse, st));
+    // per-row log-sum-exp over the vocabulary (logits stay in GEMM tiles), as in the backward
+    GemmDesc g = mk_gemm(Rc, V, d, dt, p.hc, false, d, dt, weight, true, d, DT_F32, nullptr, 0,
+                         EPI_LSE);
+    g.dynM = p.count; g.tgt = p.yc; g.col0 = 0; g.pmax = p.pmax; g.psum = p.psum;
+    g.pld = p.tiles; g.zy = p.zy;
+    SBP_CK(gemm(g, st));
+    SBP_CK(ce_finish(Rc, p.tiles, p.pmax, p.psum, p.tiles, p.count, p.wc, p.zy, p.lse,
+                     p.row_loss, lo, i == 0, st));
+    SBP_CK(ce_token_scatter(s, e, Rc, p.idx, p.count, p.lse, p.zy, token_ce, st));
+  }
+  return SBP_OK;
+}
+
+// ------------------------------------------------------------------------------- DPO
+size_t sbp_dpo_workspace_size(int64_t P) {
+  if (P < 1) return 0;
+  Carver c(nullptr);
+  c.take_bytes(kStatusBytes);
+  c.take<float>(2 * P);     // sequence log-probabilities when the caller keeps none
+  c.take<float>(P);         // per-pair loss terms
+  return c.off;
+}
+
+sbp_status sbp_dpo_token_weights(int64_t P, int64_t T, const float* token_ce,
+                                 const float* mask, const float* ref_logp, float beta,
+                                 float* loss_out, float* seq_logp, float* weights,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (P < 1 || T < 1) return fail(SBP_ERR_INVALID_ARG, "n_pairs and seq_len must be positive");
+  if (!(beta > 0.f)) return fail(SBP_ERR_INVALID_ARG, "beta must be positive");
+  if (!token_ce || !mask || !ref_logp || !loss_out || !weights)
+    return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (sbp_status s = check_ws(workspace, workspace_bytes, sbp_dpo_workspace_size(P))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  int* status = static_cast<int*>(c.take_bytes(kStatusBytes));
+  float* lp_tmp = c.take<float>(2 * P);
+  float* terms = c.take<float>(P);
+  SBP_CK(cudaMemsetAsync(status, 0, sizeof(int), st));
+  SBP_CK(dpo_weights(P, T, token_ce, mask, ref_logp, beta, seq_logp ? seq_logp : lp_tmp, terms,
+                     loss_out, weights, st));
   return SBP_OK;
 }
 

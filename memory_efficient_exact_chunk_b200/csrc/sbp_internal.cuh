@@ -235,6 +235,13 @@ cudaError_t ce_finish(int64_t Rmax, int64_t tiles, const float* pmax, const floa
                       float* lse, float* row_loss, float* loss, int first, cudaStream_t st);
 // out rows idx[r] (r < n) of d_hidden chunk: zero rows [s, e) of dh first.
 cudaError_t zero_rows(int64_t s, int64_t e, int64_t d, float* dh, cudaStream_t st);
+// token_ce[s, e) = 0, then token_ce[idx[r]] = lse[r] - zy[r] for the chunk's r < *count
+cudaError_t ce_token_scatter(int64_t s, int64_t e, int64_t Rmax, const int* idx, const int* count,
+                             const float* lse, const float* zy, float* token_ce, cudaStream_t st);
+// DPO: sequence log-probabilities, per-pair loss terms, the loss and the per-token weights
+cudaError_t dpo_weights(int64_t P, int64_t T, const float* token_ce, const float* mask,
+                        const float* ref_logp, float beta, float* seq_logp, float* terms,
+                        float* loss, float* weights, cudaStream_t st);
 
 // attention: tensor-core forward (attn_tc.cu, head_dim 128, bf16) and CUDA-core kernels
 // (attention_simt.cu, any even head_dim <= 256, fp32 or bf16).  attn_fwd/attn_bwd dispatch;

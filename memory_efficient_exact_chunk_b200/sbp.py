@@ -26,7 +26,8 @@ EXPORTS = [
     "sbp_rmsnorm_backward_workspace_size", "sbp_rmsnorm_backward", "sbp_embedding_forward",
     "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
     "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
-    "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16",
+    "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16", "sbp_lmhead_ce_forward_stream",
+    "sbp_dpo_workspace_size", "sbp_dpo_token_weights",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -81,6 +82,11 @@ def load(path: Optional[str] = None):
     lib.sbp_lmhead_ce_workspace_size.argtypes = [i64, i64, i64, C.c_int, C.c_int]
     lib.sbp_lmhead_ce_backward_stream.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp, sz, vp]
+    lib.sbp_lmhead_ce_forward_stream.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 6 + \
+        [vp, sz, vp]
+    lib.sbp_dpo_workspace_size.restype = sz
+    lib.sbp_dpo_workspace_size.argtypes = [i64]
+    lib.sbp_dpo_token_weights.argtypes = [i64, i64, vp, vp, vp, C.c_float, vp, vp, vp, vp, sz, vp]
     lib.sbp_decoder_layer_workspace_size.restype = sz
     lib.sbp_decoder_layer_workspace_size.argtypes = [C.POINTER(LayerCfg)]
     lib.sbp_decoder_layer_backward_stream.argtypes = [C.POINTER(LayerCfg),
@@ -173,6 +179,39 @@ def lmhead_ce_backward(hidden_states, weight, targets, loss_weights, num_chunks,
         N, d, V, num_chunks, dt, _ptr(hidden_states), _ptr(weight), _ptr(targets),
         _ptr(loss_weights), _ptr(loss_out), _ptr(d_hidden), _ptr(d_weight), _ptr(ws),
         ws.numel(), _stream(stream)))
+    return ws
+
+
+def lmhead_ce_forward(hidden_states, weight, targets, loss_weights, num_chunks, token_ce,
+                      loss_out=None, ws=None, stream=None):
+    """token_ce[t] = CE_t where loss_weights[t] != 0, else 0 (include/sbp_dpo.h); loss_out[0]
+    (optional) = sum_t w_t CE_t."""
+    N, d = hidden_states.shape
+    V = weight.shape[0]
+    dt = _dtype_code(hidden_states)
+    need = lmhead_ce_workspace_size(N, d, V, num_chunks, dt)
+    if ws is None:
+        ws = workspace(need, hidden_states.device)
+    _check(load().sbp_lmhead_ce_forward_stream(
+        N, d, V, num_chunks, dt, _ptr(hidden_states), _ptr(weight), _ptr(targets),
+        _ptr(loss_weights), _ptr(token_ce), _ptr(loss_out) if loss_out is not None else None,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def dpo_workspace_size(n_pairs: int) -> int:
+    return int(load().sbp_dpo_workspace_size(n_pairs))
+
+
+def dpo_token_weights(n_pairs, seq_len, token_ce, response_mask, ref_logp, beta, loss_out,
+                      weights, seq_logp=None, ws=None, stream=None):
+    """DPO loss into loss_out[0] and per-token loss weights (include/sbp_dpo.h)."""
+    if ws is None:
+        ws = workspace(dpo_workspace_size(n_pairs), token_ce.device)
+    _check(load().sbp_dpo_token_weights(
+        n_pairs, seq_len, _ptr(token_ce), _ptr(response_mask), _ptr(ref_logp), float(beta),
+        _ptr(loss_out), _ptr(seq_logp) if seq_logp is not None else None, _ptr(weights),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return ws
 
 

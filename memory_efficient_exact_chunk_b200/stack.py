@@ -110,3 +110,34 @@ def stack_backward(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, lm_w, 
     grads = zero_grads(layers, lm_w, final_g, embed.device, embed_shape=embed.shape)
     return stack_backward_from(cfg, layers, final_g, lm_w, ids, targets, loss_weights, xs, hf,
                                rstd, ws, grads=grads, stream=stream)
+
+
+def stack_dpo_step(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, lm_w, ids, targets,
+                   response_mask, ref_logp, beta: float, ws: Workspaces, grads=None, stream=None):
+    """One DPO step on 2P sequences laid out [chosen_0, rejected_0, ...] (include/sbp_dpo.h):
+    the forward keeps the layer inputs, the streamed LM-head forward gives the per-token CE, the
+    DPO loss and the per-token weights w_t = d loss / d CE_t follow, and the streamed backward
+    runs with those weights.  response_mask [2P*T] fp32, ref_logp [2P] fp32 (device).  Returns
+    the DPO loss (device [1]) and the fp32 gradients (accumulated into `grads` if given)."""
+    import torch
+    dev = embed.device
+    B, T = cfg.batch, cfg.seq_len
+    if B % 2:
+        raise ValueError("DPO needs an even number of sequences (chosen, rejected pairs)")
+    N = B * T
+    xs, hf, rstd = stack_forward(cfg, embed, layers, final_g, ids, ws, stream=stream)
+    V, d = lm_w.shape
+    token_ce = torch.empty(N, dtype=torch.float32, device=dev)
+    cws = ws.get("lmhead", sbp.lmhead_ce_workspace_size(N, d, V, cfg.num_chunks,
+                                                        sbp._dtype_code(hf)))
+    sbp.lmhead_ce_forward(hf, lm_w, targets, response_mask, cfg.num_chunks, token_ce, ws=cws,
+                          stream=stream)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    w = torch.empty(N, dtype=torch.float32, device=dev)
+    sbp.dpo_token_weights(B // 2, T, token_ce, response_mask, ref_logp, beta, loss, w,
+                          ws=ws.get("dpo", sbp.dpo_workspace_size(B // 2)), stream=stream)
+    if grads is None:
+        grads = zero_grads(layers, lm_w, final_g, dev, embed_shape=embed.shape)
+    r = stack_backward_from(cfg, layers, final_g, lm_w, ids, targets, w, xs, hf, rstd, ws,
+                            grads=grads, stream=stream)
+    return StackResult(loss, r.grads)

@@ -76,6 +76,10 @@ WORKLOADS = {
                                      loss_from_frac=0.25),
     "qwen25_7b_stack2_grpo": Workload("qwen25_7b_stack2_grpo", 8, 16384, 8, "bf16", QWEN25_7B,
                                       2, vocab=152064, loss="grpo", prompt_len=2048),
+    # DPO on the same shapes: 4 (chosen, rejected) pairs of 16384 tokens, 2048-token prompts
+    "qwen25_7b_stack2_dpo": Workload("qwen25_7b_stack2_dpo", 8, 16384, 8, "bf16", QWEN25_7B,
+                                     2, vocab=152064, loss="dpo", prompt_len=2048,
+                                     extra={"beta": 0.1}),
 }
 
 

@@ -103,3 +103,28 @@ def test_layer_argument_errors(lib):
     assert call(w=wb) == 1                                        # biases without bias grads
     w1 = sbp.LayerWeights(**{n: (FAKE if n != "bk" else None) for n in names})
     assert call(w=w1) == 1                                        # partial bias set
+
+
+def test_lmhead_forward_and_dpo_argument_errors(lib):
+    """Checked on the host before anything is queued (no GPU needed)."""
+    def fwd(N=1024, d=64, V=1000, D=4, dt=sbp.SBP_F32, h=FAKE, W=FAKE, y=FAKE, w=FAKE, ce=FAKE,
+            ws=FAKE, wsb=1 << 40):
+        return lib.sbp_lmhead_ce_forward_stream(N, d, V, D, dt, h, W, y, w, ce, None, ws, wsb,
+                                                None)
+    assert fwd(ce=None) == 1
+    assert fwd(N=0) == 1
+    assert fwd(D=2000) == 1
+    assert fwd(dt=sbp.SBP_BF16, d=60) == 2
+    assert fwd(wsb=16) == 3
+    assert sbp.dpo_workspace_size(0) == 0 and sbp.dpo_workspace_size(4) >= 256
+
+    def dpo(P=2, T=8, ce=FAKE, m=FAKE, ref=FAKE, beta=0.1, loss=FAKE, w=FAKE, ws=FAKE,
+            wsb=1 << 20):
+        return lib.sbp_dpo_token_weights(P, T, ce, m, ref, beta, loss, None, w, ws, wsb, None)
+    assert dpo(P=0) == 1
+    assert dpo(T=0) == 1
+    assert dpo(beta=0.0) == 1
+    assert dpo(beta=-1.0) == 1
+    assert dpo(ref=None) == 1
+    assert dpo(w=None) == 1
+    assert dpo(wsb=8) == 3
