@@ -85,9 +85,9 @@ sbp_status sbp_get_device_status(void* workspace, void* stream);
  * of n_tokens / num_chunks rows at a time.  The objective's normaliser (1 / #loss tokens for
  * mean-CE SFT, A_s / #tokens for GRPO) is folded into w by the caller, so the result does not
  * depend on num_chunks.  Rows with w_t == 0 are skipped (their d_hidden row is 0).  Logits are
- * formed tile by tile in on-chip memory; the only logit-sized intermediate is the bf16/fp32
- * gradient tile G of one vocabulary block (<= rows_per_chunk x 8192 elements) in the
- * workspace, sized to stay L2-resident.
+ * formed tile by tile in on-chip memory; the only logit-sized intermediates are the bf16/fp32
+ * gradient blocks G of one vocabulary block (<= rows_per_chunk x 16384 elements, two of them so
+ * that one is formed while the products consume the other) in the workspace.
  *
  *   n_tokens       number of rows N (all sequences of a batch flattened)
  *   hidden         d (multiple of 8)

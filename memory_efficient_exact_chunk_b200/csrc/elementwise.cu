@@ -79,19 +79,20 @@ __global__ void rmsnorm_fwd_vec_kernel(int64_t cols, const TX* __restrict__ x,
 }
 
 // RMSNorm backward, 8 columns per access; each thread keeps the dg partial of its columns in
-// registers (at most kVecChunks 8-column chunks per thread).
+// registers (NCH <= kVecChunks 8-column chunks per thread, sized to the row so that three CTAs
+// fit on an SM).
 constexpr int kVecChunks = 4;
-template <typename TX, typename TG>
-__global__ void rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __restrict__ x,
-                                       const TG* __restrict__ g, const float* __restrict__ rstd,
-                                       const float* __restrict__ dy,
-                                       const float* __restrict__ base, float* __restrict__ out,
-                                       int accumulate, float* __restrict__ partial) {
+template <typename TX, typename TG, int NCH>
+__global__ void __launch_bounds__(256, NCH <= 2 ? 3 : 2)
+rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __restrict__ x,
+                       const TG* __restrict__ g, const float* __restrict__ rstd,
+                       const float* __restrict__ dy, const float* __restrict__ base,
+                       float* __restrict__ out, int accumulate, float* __restrict__ partial) {
   __shared__ float red[32];
-  float dg[kVecChunks][8];
-  float gv[kVecChunks][8];
+  float dg[NCH][8];
+  float gv[NCH][8];
 #pragma unroll
-  for (int k = 0; k < kVecChunks; ++k) {
+  for (int k = 0; k < NCH; ++k) {
     const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
 #pragma unroll
     for (int i = 0; i < 8; ++i) dg[k][i] = 0.f;
@@ -100,10 +101,10 @@ __global__ void rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __r
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const int64_t o = r * cols;
     const float rs = rstd[r];
-    float xh[kVecChunks][8], u[kVecChunks][8];
+    float xh[NCH][8], u[NCH][8];
     float dot = 0.f;
 #pragma unroll
-    for (int k = 0; k < kVecChunks; ++k) {
+    for (int k = 0; k < NCH; ++k) {
       const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
       if (c >= cols) continue;
       float xv[8], dv[8];
@@ -119,7 +120,7 @@ __global__ void rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __r
     }
     dot = block_sum(dot, red) / (float)cols;
 #pragma unroll
-    for (int k = 0; k < kVecChunks; ++k) {
+    for (int k = 0; k < NCH; ++k) {
       const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
       if (c >= cols) continue;
       float v[8];
@@ -141,7 +142,7 @@ __global__ void rmsnorm_bwd_vec_kernel(int64_t rows, int64_t cols, const TX* __r
     }
   }
 #pragma unroll
-  for (int k = 0; k < kVecChunks; ++k) {
+  for (int k = 0; k < NCH; ++k) {
     const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
     if (c < cols) store8(partial + (int64_t)blockIdx.x * cols + c, dg[k]);
   }
@@ -211,7 +212,7 @@ __global__ void rmsnorm_fwd_kernel(int64_t cols, int xdt, const void* __restrict
 // ---------------------------------------------------------------- RMSNorm backward
 // Each CTA handles rows r = blockIdx.x, blockIdx.x + gridDim.x, ...; its dg partial goes to
 // partial[blockIdx.x, :] and a second kernel sums the partials in a fixed order.
-constexpr int kBwdBlocks = 296;
+constexpr int kBwdBlocks = 444;   // 3 per SM
 
 __global__ void rmsnorm_bwd_kernel(int64_t rows, int64_t cols, int xdt,
                                    const void* __restrict__ x, int gdt,
@@ -560,14 +561,31 @@ cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
   if (cols % 8 == 0 && cols <= 8 * kRowThreads * kVecChunks && gdt == DT_BF16 && al16p(x) &&
       al16p(g) && al16p(dy) && al16p(out) && (!base || al16p(base))) {
     const auto* gb = static_cast<const __nv_bfloat16*>(g);
-    if (xdt == DT_BF16)
-      launch(rmsnorm_bwd_vec_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(kBwdBlocks),
-             dim3(kRowThreads), 0, st, rows, cols, static_cast<const __nv_bfloat16*>(x), gb,
-             rstd, dy, base, out, accumulate, partial);
-    else
-      launch(rmsnorm_bwd_vec_kernel<float, __nv_bfloat16>, dim3(kBwdBlocks), dim3(kRowThreads),
-             0, st, rows, cols, static_cast<const float*>(x), gb, rstd, dy, base, out,
-             accumulate, partial);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* xf = static_cast<const float*>(x);
+    const dim3 grid(kBwdBlocks), block(kRowThreads);
+    const int nch = (int)((cols + 8 * kRowThreads - 1) / (8 * kRowThreads));
+    if (xdt == DT_BF16) {
+      if (nch <= 1)
+        launch(rmsnorm_bwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, 1>, grid, block, 0, st, rows,
+               cols, xb, gb, rstd, dy, base, out, accumulate, partial);
+      else if (nch == 2)
+        launch(rmsnorm_bwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, 2>, grid, block, 0, st, rows,
+               cols, xb, gb, rstd, dy, base, out, accumulate, partial);
+      else
+        launch(rmsnorm_bwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, kVecChunks>, grid, block, 0,
+               st, rows, cols, xb, gb, rstd, dy, base, out, accumulate, partial);
+    } else {
+      if (nch <= 1)
+        launch(rmsnorm_bwd_vec_kernel<float, __nv_bfloat16, 1>, grid, block, 0, st, rows, cols,
+               xf, gb, rstd, dy, base, out, accumulate, partial);
+      else if (nch == 2)
+        launch(rmsnorm_bwd_vec_kernel<float, __nv_bfloat16, 2>, grid, block, 0, st, rows, cols,
+               xf, gb, rstd, dy, base, out, accumulate, partial);
+      else
+        launch(rmsnorm_bwd_vec_kernel<float, __nv_bfloat16, kVecChunks>, grid, block, 0, st,
+               rows, cols, xf, gb, rstd, dy, base, out, accumulate, partial);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !dg) return e;
     launch(colsum_partials_kernel, dim3(nblk(cols, 256)), dim3(256), 0, st, (int64_t)kBwdBlocks,

@@ -68,7 +68,7 @@ inline void chunk_range(int64_t T, int D, int i, int64_t& s, int64_t& e) {
 inline int64_t chunk_max(int64_t T, int D) { return T - (int64_t)(D - 1) * chunk_size(T, D); }
 
 // ------------------------------------------------------------------------ LM head plan
-constexpr int64_t kVocabBlock = 8192;
+constexpr int64_t kVocabBlock = 16384;
 
 struct CePlan {
   int* status;

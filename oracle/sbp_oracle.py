@@ -225,11 +225,16 @@ def layer_forward_rows(cfg: LayerConfig, W: Dict[str, np.ndarray], x_prefix: np.
     return y, cache
 
 
-def layer_backward_rows(cfg: LayerConfig, W: Dict[str, np.ndarray], cache, dy_rows: np.ndarray):
+def layer_backward_rows(cfg: LayerConfig, W: Dict[str, np.ndarray], cache, dy_rows: np.ndarray,
+                        sum_scales: Optional[Dict[str, np.ndarray]] = None):
     """Backward of layer_forward_rows for upstream dy on the query rows.
 
     Returns (dx_prefix [Tk, d], grads dict).  Gradient flows to earlier rows only through the
-    attention keys/values (the causal prefix)."""
+    attention keys/values (the causal prefix).  If ``sum_scales`` is given, the column sums of
+    the absolute summands of the bias gradients (sum_t |dq_pre|, |dk_pre|, |dv|) are added to
+    it: the scale against which the rounding error of those sums is measured (the bias
+    gradients are sums with heavy cancellation: without RoPE, sum_t dk_t is exactly 0 because
+    softmax is invariant to a shift shared by all keys)."""
     H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
     c = cache
     Tk = c["x_prefix"].shape[0]
@@ -264,6 +269,9 @@ def layer_backward_rows(cfg: LayerConfig, W: Dict[str, np.ndarray], cache, dy_ro
     grads["bq"] = dq_pre.sum(axis=0)
     grads["bk"] = dk_pre.sum(axis=0)
     grads["bv"] = dv.sum(axis=0)
+    if sum_scales is not None:
+        for k, v in (("bq", dq_pre), ("bk", dk_pre), ("bv", dv)):
+            sum_scales[k] = sum_scales.get(k, 0.0) + np.abs(v).sum(axis=0)
     dx, grads["ln1_g"] = rmsnorm_backward(dn1, c["x_prefix"], W["ln1_g"], c["r1"])
     dx[rows] += dh
     return dx, grads
@@ -285,17 +293,17 @@ def decoder_layer_forward(cfg: LayerConfig, W, x):
     return np.stack([layer_forward_rows(cfg, W, x[b], 0)[0] for b in range(x.shape[0])])
 
 
-def decoder_layer_backward(cfg: LayerConfig, W, x, dy):
+def decoder_layer_backward(cfg: LayerConfig, W, x, dy, sum_scales=None):
     """Plain (unchunked) backward of the layer: returns (dx [B,T,d], grads).  This is the
     'full BP' that StreamBP must reproduce exactly ([skill] Architecture Overview, Exact
-    Gradients; [paper] Abstract)."""
+    Gradients; [paper] Abstract).  ``sum_scales``: see layer_backward_rows."""
     x = np.asarray(x, F64)
     dy = np.asarray(dy, F64)
     grads = _zero_grads(cfg, W)
     dx = np.zeros_like(x)
     for b in range(x.shape[0]):
         _, cache = layer_forward_rows(cfg, W, x[b], 0)
-        dxb, gb = layer_backward_rows(cfg, W, cache, dy[b])
+        dxb, gb = layer_backward_rows(cfg, W, cache, dy[b], sum_scales)
         dx[b] = dxb
         for k in grads:
             grads[k] += gb[k]
@@ -371,16 +379,24 @@ def lmhead_ce_backward_chunked(hidden, weight, targets, loss_weights, num_chunks
 # A small stack: embedding -> L decoder layers -> final RMSNorm -> untied LM head -> sum w CE.
 # ----------------------------------------------------------------------------------------------
 def stack_forward_backward(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, targets,
-                           loss_weights, num_chunks: Optional[int] = None):
+                           loss_weights, num_chunks: Optional[int] = None, store=None,
+                           sum_scales: Optional[List[dict]] = None):
     """ids/targets/loss_weights [B, T].  Returns (loss, grads dict).  With ``num_chunks`` the
-    layer and LM-head backwards use the chunked loops; otherwise the plain ones."""
+    layer and LM-head backwards use the chunked loops; otherwise the plain ones.  ``store``
+    (optional): the storage format of the layer-input checkpoints and of the final-norm output
+    (e.g. a rounding to bf16 when the model is kept in bf16), applied where they are stored;
+    the arithmetic stays fp64.  ``sum_scales`` (optional list): receives one dict per layer
+    with the absolute-summand scales of its bias gradients (unchunked mode; see
+    layer_backward_rows)."""
     ids = np.asarray(ids, np.int64)
     B, T = ids.shape
     E = np.asarray(embed, F64)
+    keep = store if store is not None else (lambda a: a)
     xs = [E[ids]]
     for W in layers:
-        xs.append(decoder_layer_forward(cfg, W, xs[-1]))
+        xs.append(keep(decoder_layer_forward(cfg, W, xs[-1])))
     hf, rf = rmsnorm_forward(xs[-1], final_g, cfg.rms_eps)
+    hf = keep(hf)
     hflat = hf.reshape(B * T, -1)
     tflat = np.asarray(targets).reshape(-1)
     wflat = np.asarray(loss_weights, F64).reshape(-1)
@@ -400,7 +416,10 @@ def stack_forward_backward(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, 
     layer_grads = []
     for li in range(len(layers) - 1, -1, -1):
         if num_chunks is None:
-            dxl, g = decoder_layer_backward(cfg, layers[li], xs[li], dxl)
+            sc = {} if sum_scales is not None else None
+            dxl, g = decoder_layer_backward(cfg, layers[li], xs[li], dxl, sc)
+            if sum_scales is not None:
+                sum_scales.insert(0, sc)
         else:
             dxl, g = decoder_layer_backward_chunked(cfg, layers[li], xs[li], dxl, num_chunks)
         layer_grads.append(g)
@@ -460,20 +479,22 @@ def dpo_objective(token_ce, mask, ref_logp, beta: float, n_pairs: int, seq_len: 
 
 
 def stack_dpo(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, targets, mask, ref_logp,
-              beta: float, num_chunks: Optional[int] = None):
+              beta: float, num_chunks: Optional[int] = None, store=None):
     """DPO step on the small stack: forward for the sequence log-probabilities, the per-token
     weights, then the (optionally chunked) backward with those weights.  ids/targets/mask
-    [2P, T].  Returns (dpo loss, grads, w)."""
+    [2P, T].  ``store`` as in stack_forward_backward.  Returns (dpo loss, grads, w)."""
     ids = np.asarray(ids, np.int64)
     B, T = ids.shape
     E = np.asarray(embed, F64)
+    keep = store if store is not None else (lambda a: a)
     x = E[ids]
     for W in layers:
-        x = decoder_layer_forward(cfg, W, x)
+        x = keep(decoder_layer_forward(cfg, W, x))
     hf, _ = rmsnorm_forward(x, final_g, cfg.rms_eps)
+    hf = keep(hf)
     ce = lmhead_token_ce(hf.reshape(B * T, -1), lm_w, np.asarray(targets).reshape(-1),
                          np.asarray(mask).reshape(-1))
     loss, w, _ = dpo_objective(ce, mask, ref_logp, beta, B // 2, T)
     _, grads = stack_forward_backward(cfg, embed, layers, final_g, lm_w, ids, targets,
-                                      w.reshape(B, T), num_chunks)
+                                      w.reshape(B, T), num_chunks, store)
     return loss, grads, w

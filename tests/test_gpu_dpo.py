@@ -108,11 +108,17 @@ def _gpu_dpo(L, inp, D, dtype, beta):
     return to_np(r.loss)[0], out
 
 
-def _oracle_dpo(L, inp, beta):
+def _bf16_store(a):
+    """The bf16 model keeps its layer-input checkpoints and the final-norm output in bf16."""
+    return synth.bf16_round(np.asarray(a, np.float32)).astype(np.float64)
+
+
+def _oracle_dpo(L, inp, beta, bf16):
     layers, E, fg, lm, ids, y, m, ref = inp
     loss, g, _ = O.stack_dpo(oracle_cfg(O, L), f64(E),
                              [{n: f64(W.get(n)) for n in NAMES} for W in layers], f64(fg),
-                             f64(lm), ids, y, f64(m), f64(ref), beta)
+                             f64(lm), ids, y, f64(m), f64(ref), beta,
+                             store=_bf16_store if bf16 else None)
     out = {"lm_head": g["lm_head"], "final_g": g["final_g"], "embed": g["embed"]}
     for n, v in g["layers"][0].items():
         out[f"L0.{n}"] = v
@@ -127,7 +133,7 @@ def test_stack_dpo_step_matches_oracle(dtype, L, P, T, D, tol):
     inp = _dpo_inputs(7, L, 600, P, T, dtype == "bf16")
     beta = 0.5
     loss, g = _gpu_dpo(L, inp, D, dtype, beta)
-    l0, g0 = _oracle_dpo(L, inp, beta)
+    l0, g0 = _oracle_dpo(L, inp, beta, dtype == "bf16")
     assert abs(loss - l0) <= tol * abs(l0), (loss, l0)
     errs = {k: rel_fro(v, g0[k]) for k, v in g.items()}
     bad = {k: v for k, v in errs.items() if not v <= tol}

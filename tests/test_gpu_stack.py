@@ -46,18 +46,35 @@ def run_gpu(L, layers, E, fg, lm, ids, y, w, D, dtype):
             [{n: to_np(v) for n, v in lg.items() if v is not None} for lg in g["layers"]])
 
 
+def _bf16_store(a):
+    """The bf16 model keeps its layer-input checkpoints and the final-norm output in bf16."""
+    return synth.bf16_round(np.asarray(a, np.float32)).astype(np.float64)
+
+
 def check(L, stack_in, D, dtype, tol):
     layers, E, fg, lm, ids, y, w = stack_in
     loss, dlm, dfg, dE, dls = run_gpu(L, layers, E, fg, lm, ids, y, w, D, dtype)
+    scales = []
     l0, g0 = O.stack_forward_backward(oracle_cfg(O, L), f64(E),
                                       [{n: f64(W.get(n)) for n in NAMES} for W in layers],
-                                      f64(fg), f64(lm), ids, y, f64(w))
+                                      f64(fg), f64(lm), ids, y, f64(w),
+                                      store=_bf16_store if dtype == "bf16" else None,
+                                      sum_scales=scales)
     assert abs(loss - l0) <= tol * abs(l0)
     errs = {"lm_head": rel_fro(dlm, g0["lm_head"]), "final_g": rel_fro(dfg, g0["final_g"]),
             "embed": rel_fro(dE, g0["embed"])}
     for i, lg in enumerate(dls):
         for n, v in lg.items():
-            errs[f"L{i}.{n}"] = rel_fro(v, g0["layers"][i][n])
+            if n in ("bq", "bk", "bv"):
+                # a bias gradient is a column sum over tokens with heavy cancellation (softmax
+                # is shift invariant: without RoPE sum_t dk_t = 0), so its rounding error is
+                # measured against the sum of the absolute summands, the error scale of a sum
+                ref = g0["layers"][i][n]
+                errs[f"L{i}.{n}"] = float(np.linalg.norm(f64(v) - ref) /
+                                          np.linalg.norm(scales[i][n]))
+            else:
+                errs[f"L{i}.{n}"] = rel_fro(v, g0["layers"][i][n])
+    print("stack errors:", {k: float(f"{v:.3g}") for k, v in errs.items()})
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, bad
 
@@ -73,7 +90,7 @@ def test_tiny_fp32_stack_full_size():
 def test_bf16_gqa_stack_shifted_targets():
     L = synth.LayerShape(128, 4, 2, 32, 192, 1e-5, 500000.0)
     s = make_stack(1, L, 2, 700, 1, 256, "bf16", "shifted_tail", from_frac=0.25)
-    check(L, s, 4, "bf16", 2e-2)
+    check(L, s, 4, "bf16", 1e-2)
 
 
 def test_bf16_grpo_batched_stack():
@@ -83,4 +100,4 @@ def test_bf16_grpo_batched_stack():
     layers, E, fg, lm, ids, y, _ = make_stack(2, L, 2, V, B, T, "bf16", "shifted_tail",
                                               from_frac=0.25)
     w = synth.loss_weights("grpo", B, T, prompt_len=32, advantages=rng.standard_normal(B))
-    check(L, (layers, E, fg, lm, ids, y, w), 4, "bf16", 2e-2)
+    check(L, (layers, E, fg, lm, ids, y, w), 4, "bf16", 1e-2)
