@@ -274,32 +274,44 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                      aQ0 = tc::smem_u32(sQ0);
       bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag);
       bool issued = false;
+      // Shared-memory descriptors built once; a k-step adds its byte offset / 16 to the start
+      // address field (the tiles sit below 256 KB, so the field cannot carry over).  This keeps
+      // the single issuing thread fast enough for the 128 x 64 x 16 products.
+      const uint64_t dK = tc::smem_desc_sw128(aK, 16, 1024), dV = tc::smem_desc_sw128(aV, 16, 1024);
+      const uint64_t dS = tc::smem_desc_sw128(adS, 16, 1024);
+      // the two Q/dO stages differ by a constant: stage 1's start address field is stage 0's
+      // plus 2 TILE / 16 (selected, not indexed, so the descriptors stay in registers)
+      static_assert(QD_STAGES == 2, "stage descriptors are selected between two stages");
+      const uint64_t dQk0 = tc::smem_desc_sw128(aQ0, 16, 1024);
+      const uint64_t dOk0 = tc::smem_desc_sw128(aQ0 + TILE, 16, 1024);
+      const uint64_t dQm0 = tc::smem_desc_sw128(aQ0, CHUNK, 1024);
+      const uint64_t dOm0 = tc::smem_desc_sw128(aQ0 + TILE, CHUNK, 1024);
+      constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
       // S^T_h = K Q_h^T and dP^T_h = V dO_h^T of pair j's half h
       auto scores = [&](int j, int h) {
-        const uint32_t aQ = aQ0 + 2 * (j % QD_STAGES) * TILE, adO = aQ + TILE;
+        const uint64_t so = (j & 1) ? kStage : 0;
+        const uint64_t bq = dQk0 + so + (uint64_t)((h * HALF) >> 4);
+        const uint64_t bo = dOk0 + so + (uint64_t)((h * HALF) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + c_s(h), tc::smem_desc_sw128(aK + off, 16, 1024),
-                         tc::smem_desc_sw128(aQ + h * HALF + off, 16, 1024), id_s, kk != 0);
-          tc::mma_f16_ss(tmem + c_dp(h), tc::smem_desc_sw128(aV + off, 16, 1024),
-                         tc::smem_desc_sw128(adO + h * HALF + off, 16, 1024), id_s, kk != 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(tmem + c_s(h), dK + off, bq + off, id_s, kk != 0);
+          tc::mma_f16_ss(tmem + c_dp(h), dV + off, bo + off, id_s, kk != 0);
         }
         tc::mma_commit(&sh.sdp_full[h]);
       };
       // dV += P^T_h dO_h (P^T from TMEM), dK += dS^T_h Q_h; `first`: the block's first product
       auto grads = [&](int j, int h, bool first) {
-        const uint32_t aQ = aQ0 + 2 * (j % QD_STAGES) * TILE, adO = aQ + TILE;
+        const uint64_t so = (j & 1) ? kStage : 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries of the half
-          const uint32_t offm = (4 * h + kk) * 2048;                  // MN-major operand step
+          const uint64_t offm = so + (uint64_t)(((4 * h + kk) * 2048) >> 4);  // MN-major k-step
           const uint32_t acc = (!first || kk != 0) ? 1u : 0u;
           // packed P^T of queries 32 w.. of half h sits at c_dp(h) + 32 w (w = column half)
           const uint32_t pcol = c_dp(h) + 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_f16_ts(tmem + C_DV, tmem + pcol, tc::smem_desc_sw128(adO + offm, CHUNK, 1024),
-                     id_g, acc);
-          tc::mma_f16_ss(tmem + C_DK, tc::smem_desc_sw128(adS + h * CHUNK + kk * 32, 16, 1024),
-                         tc::smem_desc_sw128(aQ + offm, CHUNK, 1024), id_g, acc);
+          mma_f16_ts(tmem + C_DV, tmem + pcol, dOm0 + offm, id_g, acc);
+          tc::mma_f16_ss(tmem + C_DK, dS + (uint64_t)((h * CHUNK + kk * 32) >> 4), dQm0 + offm,
+                         id_g, acc);
         }
       };
       int nflush = 0;
@@ -444,21 +456,30 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::tmem_ld32(tmem + lane_off + C_DV + c * 32, rv);
         tc::tmem_ld_wait();
         if (kv) {
+          // all loads first (one memory latency), then the adds and the stores
+          float4* pk = reinterpret_cast<float4*>(a.dKp + ko + c * 32);
+          float4* pv = reinterpret_cast<float4*>(a.dVp + ko + c * 32);
+          float4 x[8], y[8];
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4* pk = reinterpret_cast<float4*>(a.dKp + ko + c * 32 + i);
-            float4* pv = reinterpret_cast<float4*>(a.dVp + ko + c * 32 + i);
-            float4 x = *pk, y = *pv;
-            x.x += __uint_as_float(rk[i]) * a.scale;
-            x.y += __uint_as_float(rk[i + 1]) * a.scale;
-            x.z += __uint_as_float(rk[i + 2]) * a.scale;
-            x.w += __uint_as_float(rk[i + 3]) * a.scale;
-            y.x += __uint_as_float(rv[i]);
-            y.y += __uint_as_float(rv[i + 1]);
-            y.z += __uint_as_float(rv[i + 2]);
-            y.w += __uint_as_float(rv[i + 3]);
-            *pk = x;
-            *pv = y;
+          for (int i = 0; i < 8; ++i) {
+            x[i] = pk[i];
+            y[i] = pv[i];
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            x[i].x += __uint_as_float(rk[4 * i]) * a.scale;
+            x[i].y += __uint_as_float(rk[4 * i + 1]) * a.scale;
+            x[i].z += __uint_as_float(rk[4 * i + 2]) * a.scale;
+            x[i].w += __uint_as_float(rk[4 * i + 3]) * a.scale;
+            y[i].x += __uint_as_float(rv[4 * i]);
+            y[i].y += __uint_as_float(rv[4 * i + 1]);
+            y[i].z += __uint_as_float(rv[4 * i + 2]);
+            y[i].w += __uint_as_float(rv[4 * i + 3]);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            pk[i] = x[i];
+            pv[i] = y[i];
           }
         }
       }
@@ -567,26 +588,34 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dQ: B MN-major
       const uint32_t aQ = tc::smem_u32(sQ), adO = tc::smem_u32(sdO), adS = tc::smem_u32(sdS),
                      aKV0 = tc::smem_u32(sKV0);
+      // descriptors built once; k-steps add their offset / 16 (see the key-tile kernel)
+      const uint64_t dQ = tc::smem_desc_sw128(aQ, 16, 1024), dO = tc::smem_desc_sw128(adO, 16, 1024);
+      const uint64_t dS = tc::smem_desc_sw128(adS, 16, 1024);
+      static_assert(KV_RING == 2, "stage descriptors are selected between two stages");
+      const uint64_t dKk0 = tc::smem_desc_sw128(aKV0, 16, 1024);
+      const uint64_t dVk0 = tc::smem_desc_sw128(aKV0 + TILE, 16, 1024);
+      const uint64_t dKm0 = tc::smem_desc_sw128(aKV0, CHUNK, 1024);
+      constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
       // S_h = Q K_h^T and dP_h = dO V_h^T of key tile j's half hh
       auto scores = [&](int j, int hh) {
-        const uint32_t aK = aKV0 + 2 * (j % KV_RING) * TILE, aV = aK + TILE;
+        const uint64_t so = (j & 1) ? kStage : 0;
+        const uint64_t bk = dKk0 + so + (uint64_t)((hh * HALF) >> 4);
+        const uint64_t bv = dVk0 + so + (uint64_t)((hh * HALF) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + c_s(hh), tc::smem_desc_sw128(aQ + off, 16, 1024),
-                         tc::smem_desc_sw128(aK + hh * HALF + off, 16, 1024), id_s, kk != 0);
-          tc::mma_f16_ss(tmem + c_dp(hh), tc::smem_desc_sw128(adO + off, 16, 1024),
-                         tc::smem_desc_sw128(aV + hh * HALF + off, 16, 1024), id_s, kk != 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(tmem + c_s(hh), dQ + off, bk + off, id_s, kk != 0);
+          tc::mma_f16_ss(tmem + c_dp(hh), dO + off, bv + off, id_s, kk != 0);
         }
         tc::mma_commit(&sh.sdp_full[hh]);
       };
       // dQ += dS_h K_h
       auto dq_prod = [&](int j, int hh) {
-        const uint32_t aK = aKV0 + 2 * (j % KV_RING) * TILE;
+        const uint64_t so = (j & 1) ? kStage : 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {   // K = 64 keys of the half
-          tc::mma_f16_ss(tmem + C_DQ, tc::smem_desc_sw128(adS + hh * CHUNK + kk * 32, 16, 1024),
-                         tc::smem_desc_sw128(aK + (4 * hh + kk) * 2048, CHUNK, 1024), id_g,
+          tc::mma_f16_ss(tmem + C_DQ, dS + (uint64_t)((hh * CHUNK + kk * 32) >> 4),
+                         dKm0 + so + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_g,
                          (j | hh | kk) != 0 ? 1u : 0u);
         }
       };
