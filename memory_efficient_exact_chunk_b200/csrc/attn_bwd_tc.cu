@@ -50,7 +50,7 @@ constexpr int QD_STAGES = 2;
 // the barriers.
 struct KvShared {
   float stat[2 /*QD_STAGES*/][2][BT];   // per stage: lse (log2 units), delta
-  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full[2], ds_full[2], kvacc_done, kv_free, drain;
+  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full[2], ds_full[2], kv_free, drain;
   uint32_t tmem;
   int abort;
 };
@@ -209,7 +209,6 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::mbar_init(&sh.sdp_full[h], 1);
       tc::mbar_init(&sh.ds_full[h], kEwWarps);
     }
-    tc::mbar_init(&sh.kvacc_done, 1);
     tc::mbar_init(&sh.kv_free, kEwWarps);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -349,7 +348,6 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
         grads(j, 1, false);
-        tc::mma_commit(&sh.kvacc_done);
         tc::mma_commit(&sh.qd_empty[j % QD_STAGES]);
         if (more) scores(j + 1, 1);
       }
@@ -446,7 +444,12 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (!ok || !pos.last) continue;
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner)
-      if (!tc::mbar_wait_warp(&sh.kvacc_done, ph, abort_flag)) { ok = false; break; }
+      // the release of this pair's Q/dO stage is committed after its last dK / dV product
+      if (!tc::mbar_wait_warp(&sh.qd_empty[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u,
+                              abort_flag)) {
+        ok = false;
+        break;
+      }
       tc::fence_after_sync();
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
