@@ -201,11 +201,12 @@ def run_lmhead(args, rank, world, device):
         lh = torch.zeros(1).pin_memory()
         stream = torch.cuda.current_stream(device)
 
+        wsh = sbp.workspace(sbp.lmhead_ce_workspace_size_host(T, d, V, D, sbp.SBP_BF16), device)
+
         def e2e_step():
-            hd.copy_(hh, non_blocking=True)
-            yd.copy_(yh, non_blocking=True)
-            wd.copy_(wh, non_blocking=True)
-            sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW, ws=ws, stream=stream)
+            # the public entry for host-resident inputs: the library stages each chunk's rows
+            # while the previous chunk computes; the loss is read back
+            sbp.lmhead_ce_backward_host(hh, Wd, yh, wh, D, loss, dH, dW, ws=wsh, stream=stream)
             lh.copy_(loss, non_blocking=True)
 
         r = timed(args, e2e_step, world, device, profile=False)

@@ -114,6 +114,27 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t n_tokens, int64_t hidden, int64
                                          float* loss_out, float* d_hidden, float* d_weight,
                                          void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The same backward with the per-token inputs in HOST memory: hidden_states_host [N, d] (dt),
+ * targets_host [N] and loss_weights_host [N] are host pointers (page-locked for the copies to
+ * overlap the computation; pageable memory works but serialises).  Each chunk's rows are
+ * copied into one of two staging blocks of the workspace on a library side stream while the
+ * previous chunk computes, so only the first chunk's copy is exposed.  weight, loss_out,
+ * d_hidden, d_weight and workspace are device memory as above; the results are identical to
+ * sbp_lmhead_ce_backward_stream's.  The host buffers must stay valid and unchanged until
+ * `stream` has passed this call.  Workspace: sbp_lmhead_ce_workspace_size_host(...) bytes
+ * (the device workspace plus two staging blocks of rows_per_chunk rows).
+ */
+size_t sbp_lmhead_ce_workspace_size_host(int64_t n_tokens, int64_t hidden, int64_t vocab,
+                                         int num_chunks, sbp_dtype dt);
+sbp_status sbp_lmhead_ce_backward_stream_host(int64_t n_tokens, int64_t hidden, int64_t vocab,
+                                              int num_chunks, sbp_dtype dt,
+                                              const void* hidden_states_host, const void* weight,
+                                              const int32_t* targets_host,
+                                              const float* loss_weights_host, float* loss_out,
+                                              float* d_hidden, float* d_weight, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------------
  * Causal decoder layer (pre-norm Llama/Qwen block):
  *   n1 = RMSNorm(x; ln1_g);  q,k,v = n1 W_{q,k,v}^T (+ b_{q,k,v});  RoPE(q), RoPE(k)

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 
@@ -285,6 +286,158 @@ void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
 int* status_word() { return tl_status; }
 }  // namespace sbp
 
+namespace {
+
+// Host-resident per-token inputs of the LM-head backward: each chunk's rows are copied into one
+// of two staging blocks of the workspace on a side stream while the previous chunk computes.
+struct HostIn {
+  const char* h;          // [N, d] host
+  const int32_t* y;       // [N] host
+  const float* w;         // [N] host
+  char* sh[2];            // staging blocks [Rmax, d]
+  int32_t* sy[2];
+  float* sw[2];
+};
+
+void host_carve(Carver& c, int64_t N, int64_t d, int D, int dt, HostIn& hin) {
+  const int64_t Rmax = chunk_max(N, D);
+  for (int b = 0; b < 2; ++b) {
+    hin.sh[b] = static_cast<char*>(c.take_bytes((size_t)Rmax * d * dt_size(dt)));
+    hin.sy[b] = c.take<int32_t>(Rmax);
+    hin.sw[b] = c.take<float>(Rmax);
+  }
+}
+
+sbp_status lmhead_check(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt,
+                        std::initializer_list<const void*> ptrs) {
+  if (N <= 0 || d <= 0 || V <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (D < 1 || (int64_t)D > N)
+    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= n_tokens");
+  if (dt != SBP_F32 && dt != SBP_BF16) return fail(SBP_ERR_INVALID_ARG, "unknown dtype");
+  if (dt == SBP_BF16 && d % 8 != 0) return fail(SBP_ERR_UNSUPPORTED, "bf16 needs hidden % 8 == 0");
+  for (const void* q : ptrs) {
+    if (!q) return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "a pointer is not 16-byte aligned");
+  }
+  return SBP_OK;
+}
+
+// Rows [s, e) of a chunk staged at `base` (row s at base[0]) addressed by their global row index.
+template <typename T>
+const T* as_global_rows(const void* base, int64_t s, int64_t row_bytes) {
+  return reinterpret_cast<const T*>(reinterpret_cast<uintptr_t>(base) -
+                                    (uintptr_t)(s * row_bytes));
+}
+
+sbp_status lmhead_backward_run(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt,
+                               const void* hidden_states, const void* weight,
+                               const int32_t* targets, const float* loss_weights,
+                               float* loss_out, float* d_hidden, float* d_weight, CePlan& p,
+                               const HostIn* hin, cudaStream_t st) {
+  const int64_t es = dt_size(dt);
+  SidePool* sp = side_pool();
+  if (!sp) return fail(SBP_ERR_CUDA, "could not create the side streams");
+  std::lock_guard<std::recursive_mutex> side_lock(sp->mu);
+  // staging: ev[16 + b] = block b holds its chunk, ev[18 + b] = block b has been gathered
+  auto stage = [&](int i) -> cudaError_t {
+    int64_t s0, e0;
+    chunk_range(N, D, i, s0, e0);
+    const int b = i & 1;
+    cudaError_t e = cudaSuccess;
+    if (i >= 2) e = cudaStreamWaitEvent(sp->s[2], sp->ev[18 + b], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(hin->sh[b], hin->h + s0 * d * es, (size_t)(e0 - s0) * d * es,
+                          cudaMemcpyHostToDevice, sp->s[2]);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(hin->sy[b], hin->y + s0, sizeof(int32_t) * (size_t)(e0 - s0),
+                          cudaMemcpyHostToDevice, sp->s[2]);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(hin->sw[b], hin->w + s0, sizeof(float) * (size_t)(e0 - s0),
+                          cudaMemcpyHostToDevice, sp->s[2]);
+    if (e == cudaSuccess) e = cudaEventRecord(sp->ev[16 + b], sp->s[2]);
+    return e;
+  };
+  if (hin) {
+    SBP_CK(cudaEventRecord(sp->ev[7], st));        // the side stream starts after the caller
+    SBP_CK(cudaStreamWaitEvent(sp->s[2], sp->ev[7], 0));
+    SBP_CK(stage(0));
+    if (D > 1) SBP_CK(stage(1));
+  }
+  for (int i = 0; i < D; ++i) {
+    int64_t s, e;
+    chunk_range(N, D, i, s, e);
+    const int64_t Rc = e - s;
+    const void* hid = hidden_states;
+    const int32_t* tg = targets;
+    const float* lw = loss_weights;
+    if (hin) {
+      const int b = i & 1;
+      SBP_CK(cudaStreamWaitEvent(st, sp->ev[16 + b], 0));
+      hid = as_global_rows<char>(hin->sh[b], s, d * es);
+      tg = as_global_rows<int32_t>(hin->sy[b], s, sizeof(int32_t));
+      lw = as_global_rows<float>(hin->sw[b], s, sizeof(float));
+    }
+    SBP_CK(ce_compact(s, e, V, tg, lw, p.idx, p.count, p.status, st));
+    SBP_CK(ce_gather(Rc, d, dt, hid, p.idx, p.count, tg, lw, p.hc, p.yc, p.wc, p.zy, p.lse, st));
+    if (hin) {
+      // the chunk's rows now live in the compacted buffers: its staging block may be refilled
+      SBP_CK(cudaEventRecord(sp->ev[18 + (i & 1)], st));
+      if (i + 2 < D) SBP_CK(stage(i + 2));
+    }
+    SBP_CK(zero_rows(s, e, d, d_hidden, st));
+    // pass 1: per-row log-sum-exp over the vocabulary (logits stay in GEMM tiles)
+    GemmDesc g = mk_gemm(Rc, V, d, dt, p.hc, false, d, dt, weight, true, d, DT_F32, nullptr, 0,
+                         EPI_LSE);
+    g.dynM = p.count; g.tgt = p.yc; g.col0 = 0; g.pmax = p.pmax; g.psum = p.psum;
+    g.pld = p.tiles; g.zy = p.zy;
+    SBP_CK(gemm(g, st));
+    SBP_CK(ce_finish(Rc, p.tiles, p.pmax, p.psum, p.tiles, p.count, p.wc, p.zy, p.lse,
+                     p.row_loss, loss_out, i == 0, st));
+    // pass 2, one vocabulary block at a time: G = w (softmax - onehot) on the caller's stream,
+    // then dH += G W_b and dW_b += G^T H on the two side streams while the next block's G is
+    // formed in the other buffer (dH stays in vocabulary order on its stream).
+    SBP_CK(cudaEventRecord(sp->ev[0], st));
+    SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[0], 0));
+    SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[0], 0));
+    int blk = 0;
+    for (int64_t vb = 0; vb < V; vb += p.Vb, ++blk) {
+      const int buf = blk & 1;
+      const int64_t nb = (V - vb) < p.Vb ? (V - vb) : p.Vb;
+      const char* Wb = static_cast<const char*>(weight) + vb * d * dt_size(dt);
+      if (blk >= 2) {   // the products of block blk - 2 have read this buffer
+        SBP_CK(cudaStreamWaitEvent(st, sp->ev[3 + buf], 0));
+        SBP_CK(cudaStreamWaitEvent(st, sp->ev[5 + buf], 0));
+      }
+      GemmDesc gg = mk_gemm(Rc, nb, d, dt, p.hc, false, d, dt, Wb, true, d, dt, p.G[buf], nb,
+                            EPI_CEGRAD);
+      gg.dynM = p.count; gg.lse = p.lse; gg.tgt = p.yc; gg.wt = p.wc; gg.col0 = vb;
+      SBP_CK(gemm(gg, st));
+      SBP_CK(cudaEventRecord(sp->ev[1 + buf], st));
+      SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[1 + buf], 0));
+      GemmDesc gh = mk_gemm(Rc, d, nb, dt, p.G[buf], false, nb, dt, Wb, false, d, DT_F32,
+                            d_hidden, d, vb == 0 ? EPI_STORE : EPI_ACC);
+      gh.dynM = p.count; gh.crow = p.idx;
+      SBP_CK(gemm(gh, sp->s[0]));
+      SBP_CK(cudaEventRecord(sp->ev[3 + buf], sp->s[0]));
+      SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[1 + buf], 0));
+      GemmDesc gw = mk_gemm(nb, d, Rc, dt, p.G[buf], true, nb, dt, p.hc, false, d, DT_F32,
+                            d_weight + vb * d, d, EPI_ACC);
+      gw.dynK = p.count;
+      gw.kblk = kTokenBlock;
+      SBP_CK(gemm(gw, sp->s[1]));
+      SBP_CK(cudaEventRecord(sp->ev[5 + buf], sp->s[1]));
+    }
+    // join: the next chunk reuses the compacted rows and the row map
+    SBP_CK(cudaEventRecord(sp->ev[3], sp->s[0]));
+    SBP_CK(cudaEventRecord(sp->ev[5], sp->s[1]));
+    SBP_CK(cudaStreamWaitEvent(st, sp->ev[3], 0));
+    SBP_CK(cudaStreamWaitEvent(st, sp->ev[5], 0));
+  }
+  return SBP_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* sbp_last_error(void) { return g_err.c_str(); }
@@ -336,17 +489,9 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D,
                                          float* loss_out, float* d_hidden, float* d_weight,
                                          void* workspace, size_t workspace_bytes,
                                          void* stream) {
-  if (N <= 0 || d <= 0 || V <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
-  if (D < 1 || (int64_t)D > N)
-    return fail(SBP_ERR_INVALID_ARG, "need 1 <= num_chunks <= n_tokens");
-  if (dt != SBP_F32 && dt != SBP_BF16) return fail(SBP_ERR_INVALID_ARG, "unknown dtype");
-  if (dt == SBP_BF16 && d % 8 != 0) return fail(SBP_ERR_UNSUPPORTED, "bf16 needs hidden % 8 == 0");
-  const void* ptrs[] = {hidden_states, weight, targets, loss_weights, loss_out, d_hidden,
-                        d_weight};
-  for (const void* q : ptrs) {
-    if (!q) return fail(SBP_ERR_INVALID_ARG, "a required pointer is NULL");
-    if (!aligned16(q)) return fail(SBP_ERR_INVALID_ARG, "a pointer is not 16-byte aligned");
-  }
+  if (sbp_status r = lmhead_check(N, d, V, D, dt, {hidden_states, weight, targets, loss_weights,
+                                                   loss_out, d_hidden, d_weight}))
+    return r;
   const size_t need = sbp_lmhead_ce_workspace_size(N, d, V, D, dt);
   if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -355,66 +500,45 @@ sbp_status sbp_lmhead_ce_backward_stream(int64_t N, int64_t d, int64_t V, int D,
   ce_carve(c, N, d, V, D, dt, p);
   tl_status = p.status;
   SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
-  for (int i = 0; i < D; ++i) {
-    int64_t s, e;
-    chunk_range(N, D, i, s, e);
-    const int64_t Rc = e - s;
-    SBP_CK(ce_compact(s, e, V, targets, loss_weights, p.idx, p.count, p.status, st));
-    SBP_CK(ce_gather(Rc, d, dt, hidden_states, p.idx, p.count, targets, loss_weights, p.hc, p.yc,
-                     p.wc, p.zy, p.lse, st));
-    SBP_CK(zero_rows(s, e, d, d_hidden, st));
-    // pass 1: per-row log-sum-exp over the vocabulary (logits stay in GEMM tiles)
-    GemmDesc g = mk_gemm(Rc, V, d, dt, p.hc, false, d, dt, weight, true, d, DT_F32, nullptr, 0,
-                         EPI_LSE);
-    g.dynM = p.count; g.tgt = p.yc; g.col0 = 0; g.pmax = p.pmax; g.psum = p.psum;
-    g.pld = p.tiles; g.zy = p.zy;
-    SBP_CK(gemm(g, st));
-    SBP_CK(ce_finish(Rc, p.tiles, p.pmax, p.psum, p.tiles, p.count, p.wc, p.zy, p.lse,
-                     p.row_loss, loss_out, i == 0, st));
-    // pass 2, one vocabulary block at a time: G = w (softmax - onehot) on the caller's stream,
-    // then dH += G W_b and dW_b += G^T H on the two side streams while the next block's G is
-    // formed in the other buffer (dH stays in vocabulary order on its stream).
-    SidePool* sp = side_pool();
-    if (!sp) return fail(SBP_ERR_CUDA, "could not create the side streams");
-    std::lock_guard<std::recursive_mutex> side_lock(sp->mu);
-    SBP_CK(cudaEventRecord(sp->ev[0], st));
-    SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[0], 0));
-    SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[0], 0));
-    int blk = 0;
-    for (int64_t vb = 0; vb < V; vb += p.Vb, ++blk) {
-      const int buf = blk & 1;
-      const int64_t nb = (V - vb) < p.Vb ? (V - vb) : p.Vb;
-      const char* Wb = static_cast<const char*>(weight) + vb * d * dt_size(dt);
-      if (blk >= 2) {   // the products of block blk - 2 have read this buffer
-        SBP_CK(cudaStreamWaitEvent(st, sp->ev[3 + buf], 0));
-        SBP_CK(cudaStreamWaitEvent(st, sp->ev[5 + buf], 0));
-      }
-      GemmDesc gg = mk_gemm(Rc, nb, d, dt, p.hc, false, d, dt, Wb, true, d, dt, p.G[buf], nb,
-                            EPI_CEGRAD);
-      gg.dynM = p.count; gg.lse = p.lse; gg.tgt = p.yc; gg.wt = p.wc; gg.col0 = vb;
-      SBP_CK(gemm(gg, st));
-      SBP_CK(cudaEventRecord(sp->ev[1 + buf], st));
-      SBP_CK(cudaStreamWaitEvent(sp->s[0], sp->ev[1 + buf], 0));
-      GemmDesc gh = mk_gemm(Rc, d, nb, dt, p.G[buf], false, nb, dt, Wb, false, d, DT_F32,
-                            d_hidden, d, vb == 0 ? EPI_STORE : EPI_ACC);
-      gh.dynM = p.count; gh.crow = p.idx;
-      SBP_CK(gemm(gh, sp->s[0]));
-      SBP_CK(cudaEventRecord(sp->ev[3 + buf], sp->s[0]));
-      SBP_CK(cudaStreamWaitEvent(sp->s[1], sp->ev[1 + buf], 0));
-      GemmDesc gw = mk_gemm(nb, d, Rc, dt, p.G[buf], true, nb, dt, p.hc, false, d, DT_F32,
-                            d_weight + vb * d, d, EPI_ACC);
-      gw.dynK = p.count;
-      gw.kblk = kTokenBlock;
-      SBP_CK(gemm(gw, sp->s[1]));
-      SBP_CK(cudaEventRecord(sp->ev[5 + buf], sp->s[1]));
-    }
-    // join: the next chunk reuses the compacted rows and the row map
-    SBP_CK(cudaEventRecord(sp->ev[3], sp->s[0]));
-    SBP_CK(cudaEventRecord(sp->ev[5], sp->s[1]));
-    SBP_CK(cudaStreamWaitEvent(st, sp->ev[3], 0));
-    SBP_CK(cudaStreamWaitEvent(st, sp->ev[5], 0));
-  }
-  return SBP_OK;
+  return lmhead_backward_run(N, d, V, D, dt, hidden_states, weight, targets, loss_weights,
+                             loss_out, d_hidden, d_weight, p, nullptr, st);
+}
+
+size_t sbp_lmhead_ce_workspace_size_host(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt) {
+  if (sbp_lmhead_ce_workspace_size(N, d, V, D, dt) == 0) return 0;
+  Carver c(nullptr);
+  CePlan p;
+  ce_carve(c, N, d, V, D, dt, p);
+  HostIn hin;
+  host_carve(c, N, d, D, dt, hin);
+  return c.off;
+}
+
+sbp_status sbp_lmhead_ce_backward_stream_host(int64_t N, int64_t d, int64_t V, int D,
+                                              sbp_dtype dt, const void* hidden_states_host,
+                                              const void* weight, const int32_t* targets_host,
+                                              const float* loss_weights_host, float* loss_out,
+                                              float* d_hidden, float* d_weight, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (sbp_status r = lmhead_check(N, d, V, D, dt, {hidden_states_host, weight, targets_host,
+                                                   loss_weights_host, loss_out, d_hidden,
+                                                   d_weight}))
+    return r;
+  const size_t need = sbp_lmhead_ce_workspace_size_host(N, d, V, D, dt);
+  if (sbp_status s = check_ws(workspace, workspace_bytes, need)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  CePlan p;
+  ce_carve(c, N, d, V, D, dt, p);
+  HostIn hin;
+  host_carve(c, N, d, D, dt, hin);
+  hin.h = static_cast<const char*>(hidden_states_host);
+  hin.y = targets_host;
+  hin.w = loss_weights_host;
+  tl_status = p.status;
+  SBP_CK(cudaMemsetAsync(p.status, 0, sizeof(int), st));
+  return lmhead_backward_run(N, d, V, D, dt, nullptr, weight, nullptr, nullptr, loss_out,
+                             d_hidden, d_weight, p, &hin, st);
 }
 
 sbp_status sbp_lmhead_ce_forward_stream(int64_t N, int64_t d, int64_t V, int D, sbp_dtype dt,

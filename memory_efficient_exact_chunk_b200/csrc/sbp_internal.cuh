@@ -14,10 +14,11 @@ namespace sbp {
 // ---------------------------------------------------------------------------------------------
 // side streams (streams.cu): kSideStreams streams and kSideEvents events per device; `mu` is
 // held while one call queues work on them (keeps the event record / wait order of a call).
-// Events 0..7: LM head, 8..13: decoder layer, 14..15: attention backward.  Streams 0, 1:
-// products next to the caller's stream, 2: the attention backward's key-tile kernel.
+// Events 0..7: LM head, 8..13: decoder layer, 14..15: attention backward, 16..19: LM-head
+// input staging from host memory.  Streams 0, 1: products next to the caller's stream,
+// 2: the attention backward's key-tile kernel and the LM head's host-to-device staging.
 // ---------------------------------------------------------------------------------------------
-constexpr int kSideStreams = 3, kSideEvents = 16;
+constexpr int kSideStreams = 3, kSideEvents = 20;
 struct SidePool {
   std::recursive_mutex mu;
   cudaStream_t s[kSideStreams] = {};

@@ -27,7 +27,8 @@ EXPORTS = [
     "sbp_embedding_backward_workspace_size", "sbp_embedding_backward", "sbp_debug_gemm_bf16",
     "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
     "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16", "sbp_lmhead_ce_forward_stream",
-    "sbp_dpo_workspace_size", "sbp_dpo_token_weights",
+    "sbp_dpo_workspace_size", "sbp_dpo_token_weights", "sbp_lmhead_ce_workspace_size_host",
+    "sbp_lmhead_ce_backward_stream_host",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -82,6 +83,10 @@ def load(path: Optional[str] = None):
     lib.sbp_lmhead_ce_workspace_size.argtypes = [i64, i64, i64, C.c_int, C.c_int]
     lib.sbp_lmhead_ce_backward_stream.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp, sz, vp]
+    lib.sbp_lmhead_ce_workspace_size_host.restype = sz
+    lib.sbp_lmhead_ce_workspace_size_host.argtypes = [i64, i64, i64, C.c_int, C.c_int]
+    lib.sbp_lmhead_ce_backward_stream_host.argtypes = [i64, i64, i64, C.c_int, C.c_int] + \
+        [vp] * 7 + [vp, sz, vp]
     lib.sbp_lmhead_ce_forward_stream.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 6 + \
         [vp, sz, vp]
     lib.sbp_dpo_workspace_size.restype = sz
@@ -180,6 +185,27 @@ def lmhead_ce_backward(hidden_states, weight, targets, loss_weights, num_chunks,
         _ptr(loss_weights), _ptr(loss_out), _ptr(d_hidden), _ptr(d_weight), _ptr(ws),
         ws.numel(), _stream(stream)))
     return ws
+
+
+def lmhead_ce_backward_host(hidden_states_host, weight, targets_host, loss_weights_host,
+                            num_chunks, loss_out, d_hidden, d_weight, ws=None, stream=None):
+    """sbp_lmhead_ce_backward_stream_host: hidden states, targets and loss weights in (pinned)
+    host memory, staged chunk by chunk by the library; everything else on the device."""
+    N, d = hidden_states_host.shape
+    V = weight.shape[0]
+    dt = _dtype_code(hidden_states_host)
+    if ws is None:
+        ws = workspace(int(load().sbp_lmhead_ce_workspace_size_host(N, d, V, num_chunks, dt)),
+                       weight.device)
+    _check(load().sbp_lmhead_ce_backward_stream_host(
+        N, d, V, num_chunks, dt, _ptr(hidden_states_host), _ptr(weight), _ptr(targets_host),
+        _ptr(loss_weights_host), _ptr(loss_out), _ptr(d_hidden), _ptr(d_weight), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return ws
+
+
+def lmhead_ce_workspace_size_host(N, d, V, D, dt) -> int:
+    return int(load().sbp_lmhead_ce_workspace_size_host(N, d, V, D, dt))
 
 
 def lmhead_ce_forward(hidden_states, weight, targets, loss_weights, num_chunks, token_ce,

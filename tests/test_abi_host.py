@@ -128,3 +128,17 @@ def test_lmhead_forward_and_dpo_argument_errors(lib):
     assert dpo(ref=None) == 1
     assert dpo(w=None) == 1
     assert dpo(wsb=8) == 3
+
+
+def test_lmhead_host_entry_argument_errors(lib):
+    def call(N=1024, d=64, V=1000, D=4, dt=sbp.SBP_BF16, h=FAKE, W=FAKE, y=FAKE, w=FAKE,
+             loss=FAKE, dH=FAKE, dW=FAKE, ws=FAKE, wsb=1 << 40):
+        return lib.sbp_lmhead_ce_backward_stream_host(N, d, V, D, dt, h, W, y, w, loss, dH, dW, ws,
+                                                      wsb, None)
+    assert call(h=None) == 1
+    assert call(N=0) == 1
+    assert call(D=0) == 1
+    assert call(d=60) == 2
+    assert call(wsb=64) == 3
+    assert (sbp.lmhead_ce_workspace_size_host(1024, 64, 1000, 4, sbp.SBP_BF16) >
+            sbp.lmhead_ce_workspace_size(1024, 64, 1000, 4, sbp.SBP_BF16) > 0)

@@ -6,7 +6,7 @@ import pytest
 
 from oracle import sbp_oracle as O
 from memory_efficient_exact_chunk_b200 import synth
-from tests.helpers import rel_fro, to_dev, to_np
+from tests.helpers import f64, rel_fro, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -99,3 +99,57 @@ def test_lmhead_full_width_reduced_rows():
     assert abs(loss - l0) <= 1e-2 * abs(l0)
     assert rel_fro(dH, dH0) <= 1e-2
     assert rel_fro(dW, dW0) <= 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_lmhead_one_row_chunks(dtype):
+    """D = N: one row per chunk (the degenerate decomposition) equals the oracle and D = 1."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    N, d, V = 45, 64, 700
+    h, W, y, w = synth.lmhead_inputs(46, N, d, V, bf16=(dtype == "bf16"), from_frac=0.3)
+    hd, Wd = to_dev(h, dtype), to_dev(W, dtype)
+    yd, wd = torch.from_numpy(y).cuda(), torch.from_numpy(w).cuda()
+    out = {}
+    for D in (N, 1):
+        loss = torch.zeros(1, device="cuda")
+        dH = torch.full((N, d), float("nan"), device="cuda")
+        dW = torch.zeros(V, d, device="cuda")
+        ws = sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW)
+        sbp.device_status(ws)
+        out[D] = (to_np(loss)[0], to_np(dH), to_np(dW))
+    l0, dH0, dW0, _ = O.lmhead_ce_forward_backward(f64(h), f64(W), y, w)
+    tol = 1e-5 if dtype == "f32" else 1e-2
+    lN, dHN, dWN = out[N]
+    assert abs(lN - l0) <= tol * abs(l0)
+    assert rel_fro(dHN, dH0) <= tol and rel_fro(dWN, dW0) <= tol
+    l1, dH1, dW1 = out[1]
+    assert abs(lN - l1) <= 1e-6 * abs(l1)
+    assert rel_fro(dHN, dH1) <= 1e-5 and rel_fro(dWN, dW1) <= 1e-5
+
+
+@pytest.mark.parametrize("D", [1, 3, 8])
+def test_lmhead_host_inputs_match_device_entry(D):
+    """sbp_lmhead_ce_backward_stream_host (inputs in pinned host memory, staged by chunk on a
+    side stream) gives bit for bit the results of the device-input entry."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    N, d, V = 1500, 128, 3000
+    h, W, y, w = synth.lmhead_inputs(47, N, d, V, bf16=True, from_frac=0.25)
+    hd, Wd = to_dev(h, "bf16"), to_dev(W, "bf16")
+    yd, wd = torch.from_numpy(y).cuda(), torch.from_numpy(w).cuda()
+    hh = hd.cpu().pin_memory()
+    yh, wh = torch.from_numpy(y).pin_memory(), torch.from_numpy(w).pin_memory()
+    res = []
+    for host in (False, True):
+        loss = torch.zeros(1, device="cuda")
+        dH = torch.full((N, d), float("nan"), device="cuda")
+        dW = torch.zeros(V, d, device="cuda")
+        if host:
+            ws = sbp.lmhead_ce_backward_host(hh, Wd, yh, wh, D, loss, dH, dW)
+        else:
+            ws = sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss, dH, dW)
+        sbp.device_status(ws)
+        res.append((loss.cpu(), dH.cpu(), dW.cpu()))
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)
