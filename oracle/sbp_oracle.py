@@ -18,7 +18,7 @@ method reaches, up to rounding order, the plain unchunked backward, the oracle i
 definition written out (functions without ``chunked`` in their name) plus a literal chunked
 loop (``*_chunked``) that is used only to show that the decomposition changes nothing.
 
-Readings of the pages where they are silent or garbled (each one is listed in the design doc):
+Readings of the pages where they are silent or garbled:
   * nn.Linear layout y = x W^T, W[out, in] ([skill] Implementation writes y = x W; the
     gradients are the same up to a transpose).
   * Rotate-half RoPE with absolute positions, inv_freq_j = theta^(-2j/hd); angles in fp64.
@@ -433,7 +433,7 @@ def stack_forward_backward(cfg: LayerConfig, embed, layers, final_g, lm_w, ids, 
 # ----------------------------------------------------------------------------------------------
 # DPO.  [paper] Abstract and [skill] Core Concept ("Multiple Objectives") and Practical
 # Guidance ("Loss Objectives") name DPO among the objectives StreamBP serves; the pages give no
-# formula.  Reading (listed in the design doc): the standard DPO objective on P pairs of sequences,
+# formula.  Reading taken: the standard DPO objective on P pairs of sequences,
 #     loss = (1/P) sum_p -log sigmoid(beta * Delta_p),
 #     Delta_p = (logp(chosen_p) - ref(chosen_p)) - (logp(rejected_p) - ref(rejected_p)),
 # where logp(seq) is the sum of the token log-probabilities (= -CE) over the response tokens
