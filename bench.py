@@ -124,14 +124,18 @@ def lmhead_workload(T):
 
 def traffic_from_profiles(kernel_src: str, workload: str):
     """DRAM bytes per launch recorded by an ncu capture in profiles/, if neither the kernel
-    source nor the host code that shapes its launches (sbp_api.cu) has changed since (the
-    summary stores a hash of the two files)."""
+    source nor the vocabulary block that shapes the LM head's launches has changed since (the
+    summary stores a hash of the kernel file and of the block constant)."""
     path = os.path.join(ROOT, "profiles", f"{workload}_gemm_tc.md")
     csrc = os.path.join(ROOT, "memory_efficient_exact_chunk_b200", "csrc")
-    srcs = [os.path.join(csrc, kernel_src), os.path.join(csrc, "sbp_api.cu")]
-    if not (os.path.exists(path) and all(os.path.exists(p) for p in srcs)):
+    src, api = os.path.join(csrc, kernel_src), os.path.join(csrc, "sbp_api.cu")
+    if not (os.path.exists(path) and os.path.exists(src) and os.path.exists(api)):
         return None
-    h = hashlib.sha256(b"".join(open(p, "rb").read() for p in srcs)).hexdigest()[:16]
+    blk = re.search(r"constexpr int64_t kVocabBlock = (\d+);", open(api).read())
+    if not blk:
+        return None
+    h = hashlib.sha256(open(src, "rb").read() +
+                       f"kVocabBlock={blk.group(1)}".encode()).hexdigest()[:16]
     txt = open(path).read()
     mh = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", txt)
     mb = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", txt)
