@@ -186,18 +186,25 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                      aP = tc::smem_u32(sP);
       bool ok = tc::mbar_wait(&q_full, 0, abort_flag);
       bool issued = false;
+      // shared-memory descriptors built once; a k-step or a ring stage adds its byte offset / 16
+      // to the start address field (the tiles sit below 256 KB, so the field cannot carry over)
+      static_assert(KV_STAGES == 2, "stage descriptors are selected between two stages");
+      const uint64_t dQ = tc::smem_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = tc::smem_desc_sw128(aK, 16, 1024);
+      const uint64_t dP = tc::smem_desc_sw128(aP, 16, 1024);
+      const uint64_t dV0 = tc::smem_desc_sw128(aV, CHUNK_BYTES, 1024);
+      constexpr uint64_t kStage = (uint64_t)(TILE_BYTES >> 4);
       auto do_pv = [&](int jj) -> bool {
         const int st = jj % KV_STAGES;
         const uint32_t ph = (uint32_t)(jj / KV_STAGES) & 1u;
         if (!tc::mbar_wait(&p_full, (uint32_t)jj & 1u, abort_flag)) return false;
         if (!tc::mbar_wait(&v_full[st], ph, abort_flag)) return false;
         tc::fence_after_sync();
-        const uint32_t vb = aV + st * TILE_BYTES;
+        const uint64_t vb = dV0 + (st ? kStage : 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = tc::smem_desc_sw128(aP + (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32,
-                                                  16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(vb + kk * 2048, CHUNK_BYTES, 1024);
+          const uint64_t ad = dP + (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
+          const uint64_t bd = vb + (uint64_t)((kk * 2048) >> 4);
           tc::mma_f16_ss(tmem + O_COL, ad, bd, id_o, (jj | kk) != 0 ? 1u : 0u);
         }
         tc::mma_commit(&pv_done);
@@ -212,12 +219,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!tc::mbar_wait(&k_full[st], ph, abort_flag)) { ok = false; break; }
         if (!tc::mbar_wait(&s_empty[sb], sph ^ 1u, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
-        const uint32_t kb = aK + st * TILE_BYTES;
+        const uint64_t kb = dK0 + (st ? kStage : 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + (uint32_t)(sb * 128), tc::smem_desc_sw128(aQ + off, 16, 1024),
-                         tc::smem_desc_sw128(kb + off, 16, 1024), id_s, kk != 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(tmem + (uint32_t)(sb * 128), dQ + off, kb + off, id_s, kk != 0 ? 1u : 0u);
         }
         issued = true;
         tc::mma_commit(&s_full[sb]);
