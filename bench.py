@@ -288,6 +288,18 @@ def run_layer(args, rank, world, device, sweep=False):
         "gpu_launches": res["launches"], "clocks": res["clocks"],
         "peak_act_gb": peak / 1e9, "workspace_gb": ws.numel() / 1e9,
     }
+    # the same step with the chunks in reverse order (K/V prefix first, K/V projection
+    # backward fused into each chunk's iteration)
+    rstep = lambda: sbp.decoder_layer_backward_reverse(cfg, Wd, xd, dyd, dx, grads, ws=ws)
+    rr = timed(largs, rstep, world, device, profile=True)
+    sbp.device_status(ws)
+    out["reverse_order"] = {
+        "value": B * T * world / (rr["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": rr["ms"],
+        "steps": k, "num_chunks": D, "gpu_launches": rr["launches"], "clocks": rr["clocks"],
+        "kernels": {n: {"launches_per_step": v["launches"] / k,
+                        "busy_ms_per_step": v["busy_ms"] / k}
+                    for n, v in rr["prof"].items() if v["launches"]},
+    }
     if sweep and rank == 0 and world == 1:
         sw = []
         for Dc in (1, 2, 4, 8, 16):

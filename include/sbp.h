@@ -183,6 +183,25 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
                                              size_t workspace_bytes, void* stream);
 
 /*
+ * The same backward with the chunks visited in reverse order (the pages fix the per-chunk
+ * computation, not the order of the chunk loop: [skill] Implementation, the streamed layer
+ * backward with gradient accumulation).  The K/V prefix of the whole sequence is computed
+ * first (RMSNorm-1 and the K/V projections, chunk by chunk); then chunks D-1 .. 0 are
+ * recomputed and backpropagated.  When chunk i is reached, every chunk whose queries attend to
+ * its keys has been done, so its dK/dV rows are final and its K/V projection backward runs in
+ * the same iteration, on the RMSNorm-1 rows already computed for its forward: no pass after
+ * the loop, and one RMSNorm-1 backward per chunk.  Arguments, layouts, workspace size
+ * (sbp_decoder_layer_workspace_size), accumulation and errors are those of
+ * sbp_decoder_layer_backward_stream; the results are equal up to the order of fp32 sums.
+ */
+sbp_status sbp_decoder_layer_backward_stream_reverse(const sbp_layer_cfg* cfg,
+                                                     const sbp_layer_weights* w, const void* x,
+                                                     const float* dy, float* dx,
+                                                     const sbp_layer_grads* grads,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     void* stream);
+
+/*
  * Forward of one decoder layer, chunk by chunk (activation memory O(T/D) apart from the
  * O(T * n_kv_heads * head_dim) K/V prefix).  Used to produce the layer-input checkpoints of a
  * stack ([skill] Core Concept: StreamBP is compared with, and sits on, gradient

@@ -282,19 +282,20 @@ __global__ void rope_table_kernel(int64_t T, int64_t half, double theta, float* 
   sinb[i] = (float)sin(a);
 }
 
-// one thread per (row, head, pair j): rotates (x_j, x_{j+half})
+// one thread per (row, head, pair j): rotates (x_j, x_{j+half}); heads h_lo .. h_hi - 1 of the
+// combined q | k | v head index
 __global__ void qkv_post_kernel(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H,
-                                int64_t Hkv, int64_t hd, const float* __restrict__ qkv, int dt,
-                                void* __restrict__ q, void* __restrict__ Kp,
-                                void* __restrict__ Vp, const float* __restrict__ cosb,
-                                const float* __restrict__ sinb) {
+                                int64_t Hkv, int64_t hd, int64_t h_lo, int64_t nh,
+                                const float* __restrict__ qkv, int dt, void* __restrict__ q,
+                                void* __restrict__ Kp, void* __restrict__ Vp,
+                                const float* __restrict__ cosb, const float* __restrict__ sinb) {
   const int64_t half = hd / 2;
   const int64_t heads = H + 2 * Hkv;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= R * heads * half) return;
+  if (i >= R * nh * half) return;
   const int64_t j = i % half;
-  const int64_t hh = (i / half) % heads;
-  const int64_t r = i / (half * heads);
+  const int64_t hh = h_lo + (i / half) % nh;
+  const int64_t r = i / (half * nh);
   const int64_t b = r / Tc, t = s + r % Tc;
   const int64_t width = heads * hd;
   const float x1 = qkv[r * width + hh * hd + j];
@@ -619,11 +620,13 @@ cudaError_t rope_table(int64_t T, int64_t hd, double theta, float* cosb, float* 
 
 cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int64_t Hkv,
                      int64_t hd, const float* qkv, int dt, void* q, void* Kp, void* Vp,
-                     const float* cosb, const float* sinb, cudaStream_t st) {
-  const int64_t n = R * (H + 2 * Hkv) * (hd / 2);
+                     const float* cosb, const float* sinb, cudaStream_t st, int part) {
+  const int64_t h_lo = part == QKV_KV ? H : 0;
+  const int64_t h_hi = part == QKV_Q ? H : H + 2 * Hkv;
+  const int64_t n = R * (h_hi - h_lo) * (hd / 2);
   if (n <= 0) return cudaSuccess;
-  launch(qkv_post_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, T, H, Hkv, hd, qkv, dt, q, Kp, Vp,
-                                                cosb, sinb);
+  launch(qkv_post_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, T, H, Hkv, hd, h_lo, h_hi - h_lo,
+         qkv, dt, q, Kp, Vp, cosb, sinb);
   return cudaGetLastError();
 }
 

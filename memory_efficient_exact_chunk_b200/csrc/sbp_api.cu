@@ -231,11 +231,35 @@ sbp_status check_weights(const sbp_layer_weights* w, bool* has_bias) {
   return SBP_OK;
 }
 
+// RMSNorm-1 and the K/V projections of one chunk: fills n1, rstd1 and the chunk's rows of the
+// K/V prefix.  xc is the chunk's input rows [B * Tc, d] (contiguous).
+sbp_status layer_chunk_kv(const sbp_layer_cfg& L, const sbp_layer_weights& w, const LayerPlan& p,
+                          const void* xc, int64_t s, int64_t Tc, cudaStream_t st) {
+  const int dt = L.dtype;
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model;
+  const int64_t H = L.n_heads, Hkv = L.n_kv_heads, hd = L.head_dim;
+  const int64_t dq = H * hd, dkv = Hkv * hd, W3 = dq + 2 * dkv;
+  const int64_t R = B * Tc;
+  SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+  GemmDesc g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
+                       EPI_STORE);
+  g.bias = w.bk; g.bias_dt = dt;
+  SBP_CK(gemm(g, st));
+  g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wv, true, d, DT_F32, p.qkv + dq + dkv, W3,
+              EPI_STORE);
+  g.bias = w.bv; g.bias_dt = dt;
+  SBP_CK(gemm(g, st));
+  SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st,
+                  QKV_KV));
+  return SBP_OK;
+}
+
 // Forward recompute of one chunk: fills n1, rstd1, q, K/V prefix rows, o, alse, hbuf (= h),
-// n2, rstd2, gu and m.  xc is the chunk's input rows [B * Tc, d] (contiguous).
+// n2, rstd2, gu and m.  xc is the chunk's input rows [B * Tc, d] (contiguous).  With
+// kv_ready the whole K/V prefix is already in place: only the query projection is computed.
 sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& w,
                                const LayerPlan& p, const void* xc, int64_t s, int64_t Tc,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool kv_ready = false) {
   const int dt = L.dtype;
   const int64_t B = L.batch, T = L.seq_len, d = L.d_model, f = L.ffn;
   const int64_t H = L.n_heads, Hkv = L.n_kv_heads, hd = L.head_dim;
@@ -247,16 +271,21 @@ sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& 
                          EPI_STORE);
     g.bias = w.bq; g.bias_dt = dt;
     SBP_CK(gemm(g, st));
-    g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
-                EPI_STORE);
+  }
+  if (kv_ready) {
+    SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st,
+                    QKV_Q));
+  } else {
+    GemmDesc g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
+                         EPI_STORE);
     g.bias = w.bk; g.bias_dt = dt;
     SBP_CK(gemm(g, st));
     g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wv, true, d, DT_F32, p.qkv + dq + dkv, W3,
                 EPI_STORE);
     g.bias = w.bv; g.bias_dt = dt;
     SBP_CK(gemm(g, st));
+    SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
   }
-  SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
   SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, st));
   SBP_CK(copy_cast(R * d, dt, xc, DT_F32, p.hbuf, st));
   SBP_CK(gemm(mk_gemm(R, d, dq, dt, p.o, false, dq, dt, w.wo, true, dq, DT_F32, p.hbuf, d,
@@ -624,11 +653,15 @@ size_t sbp_decoder_layer_workspace_size(const sbp_layer_cfg* cfg) {
   return c.off;
 }
 
-sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
-                                             const sbp_layer_weights* w, const void* x,
-                                             const float* dy, float* dx,
-                                             const sbp_layer_grads* gr, void* workspace,
-                                             size_t workspace_bytes, void* stream) {
+// The streamed layer backward in either chunk order.  Forward order (chunks 0 .. D-1) grows the
+// K/V prefix chunk by chunk and backpropagates the K/V projections after the loop, once every
+// later chunk has added its dK/dV.  Reverse order (D-1 .. 0) computes the whole K/V prefix
+// first; when chunk i is reached every chunk that attends to its keys is done, so its K/V
+// projection backward runs inside the same iteration, on the n1 rows already in place.
+static sbp_status layer_backward_run(const sbp_layer_cfg* cfg, const sbp_layer_weights* w,
+                                     const void* x, const float* dy, float* dx,
+                                     const sbp_layer_grads* gr, void* workspace,
+                                     size_t workspace_bytes, void* stream, bool reverse) {
   if (sbp_status s = check_layer_cfg(cfg)) return s;
   bool has_bias = false;
   if (sbp_status s = check_weights(w, &has_bias)) return s;
@@ -665,10 +698,12 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
   SBP_CK(rope_table(T, hd, L.rope_theta, p.cosb, p.sinb, st));
   SBP_CK(cudaMemsetAsync(p.dKp, 0, sizeof(float) * (size_t)B * T * dkv, st));
   SBP_CK(cudaMemsetAsync(p.dVp, 0, sizeof(float) * (size_t)B * T * dkv, st));
-  // key/value rows past the current prefix are read (and masked) by the last key tile of a
-  // query tile: give them finite contents
-  SBP_CK(cudaMemsetAsync(p.Kp, 0, es * (size_t)B * T * dkv, st));
-  SBP_CK(cudaMemsetAsync(p.Vp, 0, es * (size_t)B * T * dkv, st));
+  if (!reverse) {
+    // key/value rows past the current prefix are read (and masked) by the last key tile of a
+    // query tile: give them finite contents
+    SBP_CK(cudaMemsetAsync(p.Kp, 0, es * (size_t)B * T * dkv, st));
+    SBP_CK(cudaMemsetAsync(p.Vp, 0, es * (size_t)B * T * dkv, st));
+  }
 
   // Weight-gradient products run on two side streams next to the chain of data gradients on
   // the caller's stream; each chunk ends with a join (its buffers are reused by the next one).
@@ -688,7 +723,62 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
   };
   cudaStream_t s0 = sp->s[0], s1 = sp->s[1];
 
-  for (int i = 0; i < D; ++i) {
+  // K/V projection backward of the chunk [s, s + Tc) once its dK/dV rows are final (n1 holds
+  // that chunk's RMSNorm-1 output): dW_k, dW_v (and the bias sums) accumulate, and
+  // dK_pre W_k + dV W_v is stored into dn1 or, with acc, added to it.
+  auto kv_backward = [&](int64_t s, int64_t Tc, bool acc) -> sbp_status {
+    const int64_t R = B * Tc;
+    SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
+    SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
+    if (dt == DT_BF16) {
+      // dK/dV are fp32 sums over chunks; their bf16 operands carry a hi + lo pair so that the
+      // products do not depend on where the fp32 sum happened to round
+      SBP_CK(split_bf16(R * dkv, p.dkpre, p.khi, p.klo, st));
+      SBP_CK(split_bf16(R * dkv, p.dvg, p.vhi, p.vlo, st));
+      const void* parts[4] = {p.khi, p.klo, p.vhi, p.vlo};
+      const void* wts[4] = {w->wk, w->wk, w->wv, w->wv};
+      float* grs[4] = {gr->wk, gr->wk, gr->wv, gr->wv};
+      SBP_CK(fork_to(0, 8));
+      for (int k = 0; k < 4; ++k)
+        SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_BF16, parts[k], true, dkv, dt, p.n1, false,
+                                        d, DT_F32, grs[k], d, EPI_ACC)), s0));
+      for (int k = 0; k < 4; ++k)
+        SBP_CK(gemm(mk_gemm(R, d, dkv, DT_BF16, parts[k], false, dkv, dt, wts[k], false, d,
+                            DT_F32, p.dn1, d, k == 0 && !acc ? EPI_STORE : EPI_ACC), st));
+    } else {
+      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
+                          p.dn1, d, acc ? EPI_ACC : EPI_STORE), st));
+      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32,
+                          p.dn1, d, EPI_ACC), st));
+      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d,
+                                      DT_F32, gr->wk, d, EPI_ACC)), st));
+      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d,
+                                      DT_F32, gr->wv, d, EPI_ACC)), st));
+    }
+    if (has_bias) {
+      SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
+      SBP_CK(colsum_acc(R, dkv, p.dvg, gr->bv, p.cpart, st));
+    }
+    return SBP_OK;
+  };
+
+  if (reverse) {
+    // the K/V prefix of the whole sequence, chunk by chunk
+    for (int j = 0; j < D; ++j) {
+      int64_t s, e;
+      chunk_range(T, D, j, s, e);
+      const int64_t Tc = e - s;
+      const void* xc = static_cast<const char*>(x) + s * d * es;
+      if (B > 1) {
+        SBP_CK(gather_chunk(B, T, Tc, s, d, dt, x, p.xg, st));
+        xc = p.xg;
+      }
+      if (sbp_status r = layer_chunk_kv(L, *w, p, xc, s, Tc, st)) return r;
+    }
+  }
+
+  for (int ii = 0; ii < D; ++ii) {
+    const int i = reverse ? D - 1 - ii : ii;
     int64_t s, e;
     chunk_range(T, D, i, s, e);
     const int64_t Tc = e - s, R = B * Tc;
@@ -703,7 +793,7 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       dyc = p.dyg;
       dxc = p.dxg;
     }
-    if (sbp_status r = layer_chunk_forward(L, *w, p, xc, s, Tc, st)) return r;
+    if (sbp_status r = layer_chunk_forward(L, *w, p, xc, s, Tc, st, reverse)) return r;
     // ---- MLP backward.  fp32 gradients enter the tensor cores as bf16 operands (rounded
     // per element, so the rounding does not depend on the chunking).
     const bool b16 = dt == DT_BF16;
@@ -772,11 +862,15 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     if (has_bias) SBP_CK(colsum_acc(R, dq, p.dq, gr->bq, p.cpart, s1));
     SBP_CK(gemm(mk_gemm(R, d, dq, dQdt, dQ, false, dq, dt, w->wq, false, d, DT_F32, p.dn1, d,
                         EPI_STORE), st));
+    // in reverse order this chunk's dK/dV rows are final: its K/V part joins dn1 here
+    if (reverse)
+      if (sbp_status r = kv_backward(s, Tc, true)) return r;
     SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, p.dh, dxc, 0, gr->ln1_g,
                        p.rpart, st));
     if (B > 1) SBP_CK(scatter_chunk_f32(B, T, Tc, s, d, p.dxg, dx, 0, st));
     SBP_CK(join_all());
   }
+  if (reverse) return SBP_OK;
   // ---- K/V projection backward, chunk by chunk, once every later chunk has added its dK/dV
   for (int j = 0; j < D; ++j) {
     int64_t s, e;
@@ -788,37 +882,7 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
       xc = p.xg;
     }
     SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w->ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
-    SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
-    SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
-    if (dt == DT_BF16) {
-      // dK/dV are fp32 sums over chunks; their bf16 operands carry a hi + lo pair so that the
-      // products do not depend on where the fp32 sum happened to round
-      SBP_CK(split_bf16(R * dkv, p.dkpre, p.khi, p.klo, st));
-      SBP_CK(split_bf16(R * dkv, p.dvg, p.vhi, p.vlo, st));
-      const void* parts[4] = {p.khi, p.klo, p.vhi, p.vlo};
-      const void* wts[4] = {w->wk, w->wk, w->wv, w->wv};
-      float* grs[4] = {gr->wk, gr->wk, gr->wv, gr->wv};
-      SBP_CK(fork_to(0, 8));
-      for (int k = 0; k < 4; ++k)
-        SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_BF16, parts[k], true, dkv, dt, p.n1, false,
-                                        d, DT_F32, grs[k], d, EPI_ACC)), s0));
-      for (int k = 0; k < 4; ++k)
-        SBP_CK(gemm(mk_gemm(R, d, dkv, DT_BF16, parts[k], false, dkv, dt, wts[k], false, d,
-                            DT_F32, p.dn1, d, k == 0 ? EPI_STORE : EPI_ACC), st));
-    } else {
-      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dkpre, false, dkv, dt, w->wk, false, d, DT_F32,
-                          p.dn1, d, EPI_STORE), st));
-      SBP_CK(gemm(mk_gemm(R, d, dkv, DT_F32, p.dvg, false, dkv, dt, w->wv, false, d, DT_F32,
-                          p.dn1, d, EPI_ACC), st));
-      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dkpre, true, dkv, dt, p.n1, false, d,
-                                      DT_F32, gr->wk, d, EPI_ACC)), st));
-      SBP_CK(gemm(over_tokens(mk_gemm(dkv, d, R, DT_F32, p.dvg, true, dkv, dt, p.n1, false, d,
-                                      DT_F32, gr->wv, d, EPI_ACC)), st));
-    }
-    if (has_bias) {
-      SBP_CK(colsum_acc(R, dkv, p.dkpre, gr->bk, p.cpart, st));
-      SBP_CK(colsum_acc(R, dkv, p.dvg, gr->bv, p.cpart, st));
-    }
+    if (sbp_status r = kv_backward(s, Tc, false)) return r;
     if (B > 1) {
       SBP_CK(rmsnorm_bwd(R, d, dt, xc, dt, w->ln1_g, p.rstd1, p.dn1, nullptr, p.dxg, 0,
                          gr->ln1_g, p.rpart, st));
@@ -830,6 +894,23 @@ sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
     SBP_CK(join_all());
   }
   return SBP_OK;
+}
+
+sbp_status sbp_decoder_layer_backward_stream(const sbp_layer_cfg* cfg,
+                                             const sbp_layer_weights* w, const void* x,
+                                             const float* dy, float* dx,
+                                             const sbp_layer_grads* gr, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+  return layer_backward_run(cfg, w, x, dy, dx, gr, workspace, workspace_bytes, stream, false);
+}
+
+sbp_status sbp_decoder_layer_backward_stream_reverse(const sbp_layer_cfg* cfg,
+                                                     const sbp_layer_weights* w, const void* x,
+                                                     const float* dy, float* dx,
+                                                     const sbp_layer_grads* gr,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     void* stream) {
+  return layer_backward_run(cfg, w, x, dy, dx, gr, workspace, workspace_bytes, stream, true);
 }
 
 sbp_status sbp_decoder_layer_forward_stream(const sbp_layer_cfg* cfg,

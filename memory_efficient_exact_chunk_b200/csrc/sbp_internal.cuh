@@ -188,9 +188,13 @@ cudaError_t rope_table(int64_t T, int64_t hd, double theta, float* cosb, float* 
                        cudaStream_t st);
 // QKV post-processing of one chunk: qkv [R, dq + 2 dkv] fp32 (R = B * Tc rows, row r is token
 // s + r % Tc of sequence r / Tc) -> q [R, dq] (RoPE'd, dt), K/V prefix [B, T, dkv] (dt).
+// `part` restricts it to the query heads (QKV_Q) or to the key/value heads (QKV_KV); columns of
+// qkv outside that part are not read.
+enum { QKV_ALL = 0, QKV_Q = 1, QKV_KV = 2 };
 cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int64_t Hkv,
                      int64_t hd, const float* qkv, int dt, void* q, void* Kp, void* Vp,
-                     const float* cosb, const float* sinb, cudaStream_t st);
+                     const float* cosb, const float* sinb, cudaStream_t st,
+                     int part = QKV_ALL);
 // In-place inverse RoPE on x [R, heads, hd] fp32 with position(r) = s + r % Tc.
 cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd, float* x,
                          const float* cosb, const float* sinb, cudaStream_t st);

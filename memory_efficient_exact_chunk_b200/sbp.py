@@ -28,7 +28,7 @@ EXPORTS = [
     "sbp_launch_count", "sbp_profile_begin", "sbp_profile_end", "sbp_lmhead_ce_backward_noalloc",
     "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16", "sbp_lmhead_ce_forward_stream",
     "sbp_dpo_workspace_size", "sbp_dpo_token_weights", "sbp_lmhead_ce_workspace_size_host",
-    "sbp_lmhead_ce_backward_stream_host",
+    "sbp_lmhead_ce_backward_stream_host", "sbp_decoder_layer_backward_stream_reverse",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -97,6 +97,8 @@ def load(path: Optional[str] = None):
     lib.sbp_decoder_layer_backward_stream.argtypes = [C.POINTER(LayerCfg),
                                                       C.POINTER(LayerWeights), vp, vp, vp,
                                                       C.POINTER(LayerGrads), vp, sz, vp]
+    lib.sbp_decoder_layer_backward_stream_reverse.argtypes = \
+        lib.sbp_decoder_layer_backward_stream.argtypes
     lib.sbp_decoder_layer_forward_stream.argtypes = [C.POINTER(LayerCfg),
                                                      C.POINTER(LayerWeights), vp, vp, vp, sz, vp]
     lib.sbp_rmsnorm_forward.argtypes = [i64, i64, C.c_int, C.c_float, vp, vp, vp, vp, vp]
@@ -269,7 +271,7 @@ def layer_workspace_size(cfg: LayerCfg) -> int:
     return load().sbp_decoder_layer_workspace_size(C.byref(cfg))
 
 
-def decoder_layer_backward(cfg: LayerCfg, weights, x, dy, dx, grads, ws=None, stream=None):
+def _layer_backward(fn, cfg, weights, x, dy, dx, grads, ws, stream):
     need = layer_workspace_size(cfg)
     if need == 0:
         raise SbpError(1, "invalid layer configuration")
@@ -277,10 +279,21 @@ def decoder_layer_backward(cfg: LayerCfg, weights, x, dy, dx, grads, ws=None, st
         ws = workspace(need, x.device)
     w = _struct(LayerWeights, weights)
     g = _struct(LayerGrads, grads)
-    _check(load().sbp_decoder_layer_backward_stream(C.byref(cfg), C.byref(w), _ptr(x), _ptr(dy),
-                                                    _ptr(dx), C.byref(g), _ptr(ws), ws.numel(),
-                                                    _stream(stream)))
+    _check(fn(C.byref(cfg), C.byref(w), _ptr(x), _ptr(dy), _ptr(dx), C.byref(g), _ptr(ws),
+              ws.numel(), _stream(stream)))
     return ws
+
+
+def decoder_layer_backward(cfg: LayerCfg, weights, x, dy, dx, grads, ws=None, stream=None):
+    return _layer_backward(load().sbp_decoder_layer_backward_stream, cfg, weights, x, dy, dx,
+                           grads, ws, stream)
+
+
+def decoder_layer_backward_reverse(cfg: LayerCfg, weights, x, dy, dx, grads, ws=None,
+                                   stream=None):
+    """The layer backward with the chunks visited from last to first."""
+    return _layer_backward(load().sbp_decoder_layer_backward_stream_reverse, cfg, weights, x, dy,
+                           dx, grads, ws, stream)
 
 
 def decoder_layer_forward(cfg: LayerCfg, weights, x, y, ws=None, stream=None):

@@ -82,15 +82,17 @@ def test_lmhead_argument_errors(lib):
     assert "workspace" in lib.sbp_last_error().decode()
 
 
-def test_layer_argument_errors(lib):
+@pytest.mark.parametrize("entry", ["sbp_decoder_layer_backward_stream",
+                                   "sbp_decoder_layer_backward_stream_reverse"])
+def test_layer_argument_errors(lib, entry):
     cfg = sbp.layer_cfg(1, 256, 64, 4, 4, 16, 172, 1e-6, 1e4, sbp.SBP_F32, 4)
     names = sbp.WEIGHT_FIELDS
     w = sbp.LayerWeights(**{n: (FAKE if n not in ("bq", "bk", "bv") else None) for n in names})
     g = sbp.LayerGrads(**{n: (FAKE if n not in ("bq", "bk", "bv") else None) for n in names})
+    fn = getattr(lib, entry)
 
     def call(c=cfg, w=w, g=g, x=FAKE, dy=FAKE, dx=FAKE, ws=FAKE, wsb=1 << 40):
-        return lib.sbp_decoder_layer_backward_stream(C.byref(c), C.byref(w), x, dy, dx,
-                                                     C.byref(g), ws, wsb, None)
+        return fn(C.byref(c), C.byref(w), x, dy, dx, C.byref(g), ws, wsb, None)
 
     assert call(x=None) == 1
     assert call(wsb=1024) == 3

@@ -69,19 +69,21 @@ def test_llama_layer_full_size_chunk_invariance():
     xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
     dyd = torch.from_numpy(dy).cuda()
     res = {}
-    for D in (wl.num_chunks, 2 * wl.num_chunks, 1):
+    for D in (wl.num_chunks, 2 * wl.num_chunks, 1, -wl.num_chunks):
+        # D < 0: |D| chunks in reverse order
         cfg = sbp.layer_cfg(B, T, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
-                            L.rms_eps, L.rope_theta, sbp.SBP_BF16, D)
+                            L.rms_eps, L.rope_theta, sbp.SBP_BF16, abs(D))
         dx = torch.full((B, T, L.d_model), float("nan"), device="cuda")
         g = {n: (torch.zeros(Wd[n].shape, device="cuda") if Wd.get(n) is not None else None)
              for n in names}
-        ws = sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, g)
+        run = sbp.decoder_layer_backward_reverse if D < 0 else sbp.decoder_layer_backward
+        ws = run(cfg, Wd, xd, dyd, dx, g)
         sbp.device_status(ws)
         res[D] = (dx, g)
         del ws
         torch.cuda.empty_cache()
     dx1, g1 = res[1]
-    for D in (wl.num_chunks, 2 * wl.num_chunks):
+    for D in (wl.num_chunks, 2 * wl.num_chunks, -wl.num_chunks):
         dxD, gD = res[D]
         assert torch.isfinite(dxD).all()
         errs = {"dx": _rel(dxD, dx1)}

@@ -1,5 +1,6 @@
-"""GPU parity of sbp_decoder_layer_backward_stream (and the chunked forward) against the fp64
-oracle, through the C ABI.  Tolerances: relative Frobenius 1e-5 (fp32), 1e-2 (bf16) per
+"""GPU parity of sbp_decoder_layer_backward_stream, its reverse chunk order
+(sbp_decoder_layer_backward_stream_reverse) and the chunked forward against the fp64 oracle,
+through the C ABI.  Tolerances: relative Frobenius 1e-5 (fp32), 1e-2 (bf16) per
 tensor; D = 1 vs D > 1 within 1e-5."""
 import numpy as np
 import pytest
@@ -14,7 +15,7 @@ TOL = {"f32": 1e-5, "bf16": 1e-2}
 NAMES = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up", "w_down")
 
 
-def _gpu_layer(L, W, x, dy, D, dtype, forward=False):
+def _gpu_layer(L, W, x, dy, D, dtype, forward=False, reverse=False):
     import torch
     from memory_efficient_exact_chunk_b200 import sbp
     B, T, d = x.shape
@@ -32,7 +33,8 @@ def _gpu_layer(L, W, x, dy, D, dtype, forward=False):
     dx = torch.full((B, T, d), float("nan"), device="cuda")
     g = {n: (torch.zeros(W[n].shape, device="cuda") if W.get(n) is not None else None)
          for n in NAMES}
-    ws = sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, g)
+    run = sbp.decoder_layer_backward_reverse if reverse else sbp.decoder_layer_backward
+    ws = run(cfg, Wd, xd, dyd, dx, g)
     sbp.device_status(ws)
     torch.cuda.synchronize()
     return to_np(dx), {n: to_np(v) for n, v in g.items() if v is not None}
@@ -44,9 +46,9 @@ def _oracle(L, W, x, dy, sum_scales=None):
     return O.decoder_layer_backward(cfg, W64, f64(x), f64(dy), sum_scales)
 
 
-def _check(L, W, x, dy, D, dtype, tol=None):
+def _check(L, W, x, dy, D, dtype, tol=None, reverse=False):
     tol = tol or TOL[dtype]
-    dx, g = _gpu_layer(L, W, x, dy, D, dtype)
+    dx, g = _gpu_layer(L, W, x, dy, D, dtype, reverse=reverse)
     scales = {}
     dx0, g0 = _oracle(L, W, x, dy, scales)
     errs = {"dx": rel_fro(dx, dx0)}
@@ -129,3 +131,35 @@ def test_layer_one_token_chunks(dtype, L, B, T):
     assert rel_fro(dxT, dx1) <= 1e-5
     for n in g1:
         assert rel_fro(gT[n], g1[n]) <= 1e-5, n
+
+
+# ---- reverse chunk order: the K/V prefix first, chunks D-1 .. 0, K/V projection backward fused
+@pytest.mark.parametrize("L,B,T,D", [(TINY, 1, 256, 4), (GQA, 2, 200, 3), (QWEN_LIKE, 1, 256, 4)])
+def test_layer_reverse_fp32(L, B, T, D):
+    W, x, dy = synth.layer_inputs(7, L, B, T, bf16=False, dy_std=1.0, gamma_std=0.1)
+    _check(L, W, x, dy, D, "f32", reverse=True)
+
+
+@pytest.mark.parametrize("L,B,T,D", [(QWEN_LIKE, 2, 384, 3), (HD128, 1, 300, 5),
+                                     (HD128_BIAS, 2, 256, 2)])
+def test_layer_reverse_bf16(L, B, T, D):
+    W, x, dy = synth.layer_inputs(8, L, B, T, bf16=True, dy_std=1e-3, gamma_std=0.1)
+    _check(L, W, x, dy, D, "bf16", reverse=True)
+
+
+@pytest.mark.parametrize("dtype,L", [("f32", GQA), ("bf16", HD128), ("bf16", HD128_BIAS)])
+def test_layer_reverse_matches_forward_order(dtype, L):
+    """Reverse order at D = 1, 4, 8 against forward order at D = 1: the same gradient up to
+    the order of fp32 sums (1e-5)."""
+    W, x, dy = synth.layer_inputs(9, L, 2, 512, bf16=(dtype == "bf16"), dy_std=1e-3)
+    dx1, g1 = _gpu_layer(L, W, x, dy, 1, dtype)
+    for D in (1, 4, 8):
+        dxD, gD = _gpu_layer(L, W, x, dy, D, dtype, reverse=True)
+        assert rel_fro(dxD, dx1) <= 1e-5, D
+        for n in g1:
+            assert rel_fro(gD[n], g1[n]) <= 1e-5, (D, n, rel_fro(gD[n], g1[n]))
+
+
+def test_layer_reverse_one_token_chunks():
+    W, x, dy = synth.layer_inputs(10, GQA, 1, 37, bf16=False, dy_std=1.0, gamma_std=0.1)
+    _check(GQA, W, x, dy, 37, "f32", reverse=True)

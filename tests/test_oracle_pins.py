@@ -240,6 +240,30 @@ def test_layer_chunked_equals_unchunked(D):
         assert rel(g0[k], g1[k]) <= 1e-12, k
 
 
+@pytest.mark.parametrize("D", [2, 3, 12])
+def test_layer_reverse_order_rows_final_early(D):
+    """The reading behind the reverse chunk order: visiting chunks D-1 .. 0, the input-gradient
+    rows of chunk i (and so its dK/dV rows) are final as soon as chunk i is done, because only
+    chunks j >= i attend to its keys.  Checked against the unchunked backward; the reverse sum
+    itself equals it too."""
+    cfg = tiny_cfg()
+    W = tiny_weights(cfg, seed=21, bias=True)
+    rng = np.random.default_rng(22)
+    B, T = 2, 12
+    x = rng.standard_normal((B, T, cfg.d_model))
+    dy = rng.standard_normal((B, T, cfg.d_model))
+    dx0, g0 = O.decoder_layer_backward(cfg, W, x, dy)
+    rel = lambda a, b: np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+    for b in range(B):
+        dx = np.zeros((T, cfg.d_model))
+        for (s, e) in reversed(O.chunk_bounds(T, D)):
+            _, cache = O.layer_forward_rows(cfg, W, x[b, :e], s)
+            dxp, _ = O.layer_backward_rows(cfg, W, cache, dy[b, s:e])
+            dx[:e] += dxp
+            assert rel(dx[s:e], dx0[b, s:e]) <= 1e-12, (b, s, e)
+        assert rel(dx, dx0[b]) <= 1e-12
+
+
 # ------------------------------------------------------------------------------------------
 # LM head + CE
 # ------------------------------------------------------------------------------------------
