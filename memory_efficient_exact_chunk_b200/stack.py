@@ -58,9 +58,13 @@ def stack_forward(cfg: sbp.LayerCfg, embed, layers: List[dict], final_g, ids, ws
 
 
 def stack_backward_from(cfg: sbp.LayerCfg, layers: List[dict], final_g, lm_w, ids, targets,
-                        loss_weights, xs, hf, rstd, ws: Workspaces, grads=None, stream=None):
+                        loss_weights, xs, hf, rstd, ws: Workspaces, grads=None, stream=None,
+                        on_final=None):
     """The streamed backward of the stack from its checkpoints.  `grads` (optional) holds fp32
-    gradient buffers to accumulate into (the layout StackResult.grads uses); else fresh zeros."""
+    gradient buffers to accumulate into (the layout StackResult.grads uses); else fresh zeros.
+    `on_final` (optional) is called with "head" once the LM-head and final-norm gradients are
+    queued, "layer{l}" after layer l's backward and "embed" at the end: the points after which
+    the work on the stream leaves that gradient unchanged."""
     import torch
     dev = hf.device
     N, d = hf.shape
@@ -76,13 +80,19 @@ def stack_backward_from(cfg: sbp.LayerCfg, layers: List[dict], final_g, lm_w, id
     dx = torch.empty(N, d, dtype=torch.float32, device=dev)
     sbp.rmsnorm_backward(xs[-1], final_g, rstd, dhf, dx, grads["final_g"],
                          ws=ws.get("rms", 0), stream=stream)
+    if on_final:
+        on_final("head")
     lws = ws.get("layer", sbp.layer_workspace_size(cfg))
     dxn = dhf                                        # reuse the buffer: dhf is consumed
     for li in range(len(layers) - 1, -1, -1):
         sbp.decoder_layer_backward(cfg, layers[li], xs[li], dx, dxn, grads["layers"][li],
                                    ws=lws, stream=stream)
+        if on_final:
+            on_final(f"layer{li}")
         dx, dxn = dxn, dx
     sbp.embedding_backward(ids, dx, grads["embed"], ws=ws.get("embed", 0), stream=stream)
+    if on_final:
+        on_final("embed")
     return StackResult(loss, grads)
 
 
