@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g) {
   const int64_t m0 = (int64_t)blockIdx.y * BM;
   const int64_t n0 = (int64_t)blockIdx.x * BN;
   if (m0 >= (g.epi == EPI_CEGRAD ? g.M : M)) return;
+  if (K <= 0 && g.epi == EPI_ACC && !g.bias) return;     // C += 0: C stays as it is
 
   const TA* A = static_cast<const TA*>(g.A);
   const TB* B = static_cast<const TB*>(g.B);

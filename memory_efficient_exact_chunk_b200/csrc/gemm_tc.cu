@@ -20,6 +20,17 @@
 #include "sbp_internal.cuh"
 #include "tc_ptx.cuh"
 
+// Cycle accounting of the pair kernel, compiled in only with -DSBP_GEMM_TIMING (the build's
+// --timing library): per launch, CTAs 0/1 print the producer's time waiting for free ring
+// stages, the MMA issuer's time waiting for operands and for a free accumulator, and the
+// epilogue's time waiting for a full accumulator and working.  Off by default: no cost.
+#ifdef SBP_GEMM_TIMING
+#include <cstdio>
+#define SBP_TIMED(...) __VA_ARGS__
+#else
+#define SBP_TIMED(...)
+#endif
+
 namespace sbp {
 
 namespace {
@@ -52,6 +63,16 @@ __device__ __forceinline__ void tile_coords(int t, int nM, int nN, int& mt, int&
 }
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// True when a launch has nothing to write: no live rows (every tile would be skipped), or
+// C += A B over an empty K range (the weight gradient of a chunk without loss rows), which
+// leaves C as it is.  The same for every CTA, so the grid (and a CTA pair) returns together,
+// before any barrier or TMEM is set up.
+__device__ __forceinline__ bool nothing_to_do(const GemmDesc& g) {
+  const int64_t M = g.dynM ? (int64_t)*g.dynM : g.M;
+  const int64_t K = g.dynK ? (int64_t)*g.dynK : g.K;
+  return M <= 0 || (K <= 0 && g.epi == EPI_ACC && !g.bias);
+}
 
 __device__ __forceinline__ void store8_bf16(__nv_bfloat16* p, const float* v) {
   uint4 pk;
@@ -252,6 +273,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmDesc& g = args.g;
   volatile int* abort_flag = &abort_sh;
+  if (nothing_to_do(g)) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -445,6 +467,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmDesc& g = args.g;
   volatile int* abort_flag = &abort_sh;
+  if (nothing_to_do(g)) return;
   const uint32_t rank = tc::cluster_ctarank();      // 0 = leader (issues the MMAs)
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
 
@@ -488,14 +511,18 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       uint32_t ph = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
+      SBP_TIMED(long long w_empty = 0, tp0 = clock64(), c0; int ntl = 0;)
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
         int mt, nt;
         tile_coords(t, args.nM, args.nN, mt, nt);
         const int m0 = mt * BM2, n0 = nt * BN;
         if (m0 >= M) continue;
+        SBP_TIMED(++ntl;)
         const int ma = m0 + 128 * (int)rank, nb = n0 + 128 * (int)rank;
         for (int kb = 0; kb < nk; ++kb) {
+          SBP_TIMED(c0 = clock64();)
           if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          SBP_TIMED(w_empty += clock64() - c0;)
           uint8_t* sa = smem + s * STAGE2_BYTES;
           uint8_t* sb = sa + A2_BYTES;
           const uint32_t fb = tc::mapa(tc::smem_u32(&full_bar[s]), 0);
@@ -518,6 +545,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           if (++s == STAGES2) { s = 0; ph ^= 1u; }
         }
       }
+      SBP_TIMED(if (blockIdx.x < 2) printf(
+          "SBPT PROD cta %d M %lld N %lld K %lld epi %d tiles %d total %lld w_empty %lld\n",
+          (int)blockIdx.x, (long long)M, (long long)N, (long long)K, g.epi, ntl,
+          clock64() - tp0, w_empty);)
       if (!ok && rank == 0) {
         // wind down: wait (bounded) for the pair's copies in flight on this CTA's barriers
         const uint64_t t0 = tc::globaltimer_ns();
@@ -539,17 +570,22 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       uint32_t ph = 0, aph = 0;
       bool ok = true;
       bool issued = false;
+      SBP_TIMED(long long w_full = 0, w_temp = 0, ti0 = clock64(), c0; int nkbt = 0;)
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
         int mt, nt;
         tile_coords(t, args.nM, args.nN, mt, nt);
         if ((int64_t)mt * BM2 >= M) continue;
         for (int b = 0; b < nblk && ok; ++b) {
+          SBP_TIMED(c0 = clock64();)
           if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
+          SBP_TIMED(w_temp += clock64() - c0;)
           tc::fence_after_sync();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
           const int kb0 = b * kpb, kb1 = imin(nk, kb0 + kpb);
           for (int kb = kb0; kb < kb1; ++kb) {
+            SBP_TIMED(c0 = clock64();)
             if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+            SBP_TIMED(w_full += clock64() - c0; ++nkbt;)
             tc::fence_after_sync();
             const uint32_t sa = smem_base + s * STAGE2_BYTES;
             const uint32_t sb = sa + A2_BYTES;
@@ -576,6 +612,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         while (!tc::mbar_try_wait(&drain_bar, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
         }
       }
+      SBP_TIMED(if (blockIdx.x == 0) printf(
+          "SBPT ISSUE M %lld N %lld K %lld epi %d kblocks %d total %lld w_full %lld w_tempty %lld\n",
+          (long long)M, (long long)N, (long long)K, g.epi, nkbt, clock64() - ti0, w_full,
+          w_temp);)
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..9)
@@ -585,6 +625,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const uint32_t te_leader = tc::mapa(tc::smem_u32(&tempty_bar[0]), 0);
     int acc = 0;
     uint32_t aph = 0;
+    SBP_TIMED(long long w_tf = 0, t_ep = 0, te0 = clock64(), c0;)
     for (int t = cluster; t < ntiles; t += nclusters) {
       int mt, nt;
       tile_coords(t, args.nM, args.nN, mt, nt);
@@ -592,11 +633,15 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       if (m0 >= M) continue;
       bool ok = true;
       for (int b = 0; b < nblk; ++b) {
+        SBP_TIMED(c0 = clock64();)
         if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) { ok = false; break; }
+        SBP_TIMED(w_tf += clock64() - c0;)
         tc::fence_after_sync();
         const int64_t m = m0 + 128 * rank + row_in_tile;
         const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+        SBP_TIMED(c0 = clock64();)
         epilogue_tile(g, tbase, m, n0, M, N, imin(nk - b * kpb, kpb), c_lo, b);
+        SBP_TIMED(t_ep += clock64() - c0;)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive_cluster(te_leader + (uint32_t)(acc * sizeof(uint64_t)));
@@ -604,6 +649,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       }
       if (!ok) break;
     }
+    SBP_TIMED(if (blockIdx.x == 0 && (warp == 2 || warp == 9) && lane == 0) printf(
+        "SBPT EPI warp %d M %lld N %lld K %lld epi %d total %lld w_tfull %lld work %lld\n", warp,
+        (long long)M, (long long)N, (long long)K, g.epi, clock64() - te0, w_tf, t_ep);)
   }
 
   tc::fence_before_sync();

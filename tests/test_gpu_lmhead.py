@@ -67,6 +67,26 @@ def test_lmhead_d_invariance_and_accumulate(dtype):
     assert rel_fro(got[2] - prior, base[2]) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_lmhead_masked_chunks_keep_prior_dw(dtype):
+    """Chunks without loss rows launch products with no live rows and a dW product over an
+    empty K range; those return at once and must leave the caller's d_weight as it is."""
+    N, d, V = 2048, 256, 5000
+    h, W, y, w = _inputs(12, N, d, V, dtype, frac=0.6)    # chunks 0 and 1 fully masked at D=4
+    assert not np.any(w[:1024]) and np.any(w[1024:1536])
+    prior = (np.random.default_rng(4).standard_normal((V, d)) * 1e-3).astype(np.float32)
+    loss1, dH1, dW1 = _run(h, W, y, w, 1, dtype, dW0=prior)
+    loss4, dH4, dW4 = _run(h, W, y, w, 4, dtype, dW0=prior)
+    l0, dH0, dW0, _ = O.lmhead_ce_forward_backward(f64(h), f64(W), y, w)
+    assert rel_fro(dW4 - prior, dW0) <= TOL[dtype] and rel_fro(dH4, dH0) <= TOL[dtype]
+    assert rel_fro(dW4, dW1) <= 1e-5 and rel_fro(dH4, dH1) <= 1e-5
+    assert abs(loss4 - loss1) <= 1e-5 * abs(loss1)
+    # a fully masked input: nothing but the loss (0) and dH (0) is written
+    z = np.zeros_like(w)
+    lz, dHz, dWz = _run(h, W, y, z, 4, dtype, dW0=prior)
+    assert lz == 0.0 and np.all(dHz == 0.0) and np.array_equal(dWz, prior)
+
+
 def test_lmhead_all_masked_chunk_and_bad_target():
     import torch
     from memory_efficient_exact_chunk_b200 import sbp
