@@ -470,3 +470,109 @@ def test_stack_dpo_finite_differences_and_chunks():
     loss2, g2, _ = O.stack_dpo(cfg, E, layers, fg, lm, ids, ys, m, ref, beta, num_chunks=3)
     assert np.isclose(loss2, loss, rtol=1e-15)
     assert np.allclose(g2["layers"][0]["wq"], g["layers"][0]["wq"], rtol=1e-11, atol=1e-14)
+
+
+# ------------------------------------------------------------------------------------------
+# The hand-written chain rule against reverse-mode autograd: a torch fp64 forward written here
+# from the definition (RMSNorm, projections with bias, rotate-half RoPE at absolute positions,
+# causal GQA softmax attention, residual, SwiGLU MLP; embedding, final RMSNorm, untied LM head,
+# sum_t w_t CE_t), differentiated by torch.autograd.  Agreement to 1e-10 catches terms too
+# small for finite differences to see.
+# ------------------------------------------------------------------------------------------
+def _t(a):
+    return None if a is None else torch.tensor(np.asarray(a, np.float64), requires_grad=True)
+
+
+def _torch_layer(cfg, Wt, x):
+    B, T, d = x.shape
+    H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+
+    def rms(v, g):
+        return v * torch.rsqrt((v * v).mean(-1, keepdim=True) + cfg.rms_eps) * g
+
+    def lin(v, w, b):
+        out = v @ w.T
+        return out if b is None else out + b
+
+    n1 = rms(x, Wt["ln1_g"])
+    q = lin(n1, Wt["wq"], Wt["bq"]).reshape(B, T, H, hd)
+    k = lin(n1, Wt["wk"], Wt["bk"]).reshape(B, T, Hkv, hd)
+    v = lin(n1, Wt["wv"], Wt["bv"]).reshape(B, T, Hkv, hd)
+    half = hd // 2
+    inv = cfg.rope_theta ** (-(2.0 * torch.arange(half, dtype=torch.float64)) / hd)
+    ang = torch.arange(T, dtype=torch.float64)[:, None] * inv[None, :]
+    ang = torch.cat([ang, ang], dim=1)
+    cos, sin = torch.cos(ang)[None, :, None, :], torch.sin(ang)[None, :, None, :]
+
+    def rot(u):
+        return u * cos + torch.cat([-u[..., half:], u[..., :half]], dim=-1) * sin
+
+    q, k = rot(q), rot(k)
+    k = k.repeat_interleave(H // Hkv, dim=2)
+    v = v.repeat_interleave(H // Hkv, dim=2)
+    s = torch.einsum("bthd,buhd->bhtu", q, k) / math.sqrt(hd)
+    future = torch.triu(torch.ones(T, T, dtype=torch.bool), diagonal=1)
+    p = torch.softmax(s.masked_fill(future, float("-inf")), dim=-1)
+    a = torch.einsum("bhtu,buhd->bthd", p, v).reshape(B, T, H * hd)
+    h = x + a @ Wt["wo"].T
+    n2 = rms(h, Wt["ln2_g"])
+    g = n2 @ Wt["w_gate"].T
+    return h + (g * torch.sigmoid(g) * (n2 @ Wt["w_up"].T)) @ Wt["w_down"].T
+
+
+def _rel(a, b):
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(np.asarray(a, np.float64) - b) / max(np.linalg.norm(b), 1e-300))
+
+
+@pytest.mark.parametrize("bias", [True, False])
+def test_layer_backward_matches_autograd(bias):
+    cfg = tiny_cfg(H=4, Hkv=2, hd=8, d=16, f=24)
+    W = tiny_weights(cfg, seed=31, bias=bias)
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((2, 11, cfg.d_model))
+    dy = rng.standard_normal((2, 11, cfg.d_model))
+    dx0, g0 = O.decoder_layer_backward(cfg, W, x, dy)
+    Wt = {n: _t(W.get(n)) for n in O.WEIGHT_NAMES}
+    xt = _t(x)
+    y = _torch_layer(cfg, Wt, xt)
+    assert _rel(y.detach().numpy(), O.decoder_layer_forward(cfg, W, x)) <= 1e-12
+    (y * torch.from_numpy(dy)).sum().backward()
+    assert _rel(dx0, xt.grad.numpy()) <= 1e-10
+    for n in O.WEIGHT_NAMES:
+        if Wt[n] is not None:
+            assert _rel(g0[n], Wt[n].grad.numpy()) <= 1e-10, n
+
+
+def test_stack_backward_matches_autograd():
+    cfg = tiny_cfg(H=4, Hkv=1, hd=4, d=16, f=20)
+    rng = np.random.default_rng(33)
+    B, T, V = 2, 9, 23
+    layers = [tiny_weights(cfg, seed=34 + i, bias=(i == 0)) for i in range(2)]
+    E = rng.standard_normal((V, cfg.d_model))
+    fg = 1.0 + 0.2 * rng.standard_normal(cfg.d_model)
+    lm = 0.5 * rng.standard_normal((V, cfg.d_model))
+    ids = rng.integers(0, V, (B, T))
+    targets = np.concatenate([ids[:, 1:], -np.ones((B, 1), np.int64)], axis=1)
+    w = np.where(targets >= 0, rng.standard_normal((B, T)), 0.0)     # signed, GRPO-like
+    loss0, g0 = O.stack_forward_backward(cfg, E, layers, fg, lm, ids, targets, w)
+    Et, fgt, lmt = _t(E), _t(fg), _t(lm)
+    Lt = [{n: _t(W.get(n)) for n in O.WEIGHT_NAMES} for W in layers]
+    x = Et[torch.from_numpy(ids)]
+    for Wt in Lt:
+        x = _torch_layer(cfg, Wt, x)
+    hf = x * torch.rsqrt((x * x).mean(-1, keepdim=True) + cfg.rms_eps) * fgt
+    z = (hf @ lmt.T).reshape(B * T, V)
+    y = torch.from_numpy(np.where(targets >= 0, targets, 0).reshape(-1))
+    ce = torch.logsumexp(z, dim=-1) - z[torch.arange(B * T), y]
+    loss = (torch.from_numpy(w.reshape(-1)) * ce).sum()
+    loss.backward()
+    lt = float(loss.detach())
+    assert abs(loss0 - lt) <= 1e-12 * max(1.0, abs(lt))
+    assert _rel(g0["lm_head"], lmt.grad.numpy()) <= 1e-10
+    assert _rel(g0["final_g"], fgt.grad.numpy()) <= 1e-10
+    assert _rel(g0["embed"], Et.grad.numpy()) <= 1e-10
+    for i, Wt in enumerate(Lt):
+        for n in O.WEIGHT_NAMES:
+            if Wt[n] is not None:
+                assert _rel(g0["layers"][i][n], Wt[n].grad.numpy()) <= 1e-10, (i, n)
