@@ -34,6 +34,18 @@
 #include <mutex>
 
 #include "sbp_internal.cuh"
+
+// Cycle accounting of the dK/dV kernel, compiled in only with -DSBP_ATTN_TIMING (the build's
+// --timing library): CTA 0 prints, per launch, the producer's cycles waiting for a free Q/dO
+// stage, the MMA issuer's cycles waiting for dS / Q,dO / the accumulator flush and issuing,
+// and two element-wise warps' cycles waiting for Q,dO and for the scores, working, and
+// flushing.  Off by default: no cost.
+#ifdef SBP_ATTN_TIMING
+#include <cstdio>
+#define SBP_ATTN_TIMED(...) __VA_ARGS__
+#else
+#define SBP_ATTN_TIMED(...)
+#endif
 #include "tc_ptx.cuh"
 
 namespace sbp {
@@ -234,13 +246,16 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full, 64, (int32_t)g, krow);
       bool ok = true;
       int issued = 0;
+      SBP_ATTN_TIMED(long long w_empty = 0, tp0 = clock64(), c0;)
       PairIter it;
       it.init((int)i0, a.nq, (int)grp, a.qb);
       for (int j = 0; j < npairs; ++j, it.next()) {
         const PairPos pos = it.pos(g);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
+        SBP_ATTN_TIMED(c0 = clock64();)
         if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        SBP_ATTN_TIMED(w_empty += clock64() - c0;)
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
@@ -254,6 +269,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
         issued = j + 1;
       }
+      SBP_ATTN_TIMED(if (blockIdx.x == 0) printf(
+          "SBPT KVPROD s %lld Tc %lld pairs %d total %lld w_empty %lld\n", (long long)a.s,
+          (long long)a.Tc, npairs, clock64() - tp0, w_empty);)
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
@@ -314,6 +332,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       };
       int nflush = 0;
+      SBP_ATTN_TIMED(long long w_ds = 0, w_qd = 0, w_free = 0, t_iss = 0, ti0 = clock64(), c0;)
       if (ok && tc::mbar_wait(&sh.qd_full[0], 0, abort_flag)) {
         tc::fence_after_sync();
         scores(0, 0);
@@ -327,30 +346,48 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int j = 0; j < npairs && ok; ++j, it.next()) {
         const PairPos pos = it.pos(g);
         const uint32_t ph = (uint32_t)j & 1u;
+        SBP_ATTN_TIMED(c0 = clock64();)
         if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
+        SBP_ATTN_TIMED(w_ds += clock64() - c0;)
         // a new block overwrites dK / dV: the element-wise warps must have added the last one
         if (pos.first && j > 0) {
+          SBP_ATTN_TIMED(c0 = clock64();)
           if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
+          SBP_ATTN_TIMED(w_free += clock64() - c0;)
           ++nflush;
         }
         tc::fence_after_sync();
+        SBP_ATTN_TIMED(c0 = clock64();)
         grads(j, 0, pos.first);
+        SBP_ATTN_TIMED(t_iss += clock64() - c0;)
         const bool more = j + 1 < npairs;
         if (more) {
           const int st1 = (j + 1) % QD_STAGES;
+          SBP_ATTN_TIMED(c0 = clock64();)
           if (!tc::mbar_wait(&sh.qd_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
             ok = false;
             break;
           }
+          SBP_ATTN_TIMED(w_qd += clock64() - c0;)
           tc::fence_after_sync();
+          SBP_ATTN_TIMED(c0 = clock64();)
           scores(j + 1, 0);
+          SBP_ATTN_TIMED(t_iss += clock64() - c0;)
         }
+        SBP_ATTN_TIMED(c0 = clock64();)
         if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
+        SBP_ATTN_TIMED(w_ds += clock64() - c0;)
         tc::fence_after_sync();
+        SBP_ATTN_TIMED(c0 = clock64();)
         grads(j, 1, false);
         tc::mma_commit(&sh.qd_empty[j % QD_STAGES]);
         if (more) scores(j + 1, 1);
+        SBP_ATTN_TIMED(t_iss += clock64() - c0;)
       }
+      SBP_ATTN_TIMED(if (blockIdx.x == 0) printf(
+          "SBPT KVISSUE s %lld Tc %lld pairs %d total %lld w_ds %lld w_qd %lld w_free %lld "
+          "issue %lld\n", (long long)a.s, (long long)a.Tc, npairs, clock64() - ti0, w_ds, w_qd,
+          w_free, t_iss);)
       if (issued) {
         tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
@@ -369,6 +406,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const bool kv = kpos < e32;
     const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
     bool ok = true;
+    SBP_ATTN_TIMED(long long w_q = 0, w_sdp = 0, t_work = 0, t_flush = 0, te0 = clock64(), c0;)
     PairIter it;
     it.init((int)i0, a.nq, (int)grp, a.qb);
     for (int j = 0; j < npairs && ok; ++j, it.next()) {
@@ -384,10 +422,12 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
       // acquire the bulk copies of this stage (already complete once the scores are ready)
+      SBP_ATTN_TIMED(c0 = clock64();)
       if (!tc::mbar_wait_warp(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
         break;
       }
+      SBP_ATTN_TIMED(w_q += clock64() - c0;)
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         const int qoff = 64 * h + 32 * wh;             // this warp's queries within the tile
@@ -396,7 +436,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 32 <= a.Tc);
         const float* lse_s = sh.stat[st][0] + qoff;
         const float* delta_s = sh.stat[st][1] + qoff;
+        SBP_ATTN_TIMED(c0 = clock64();)
         if (!tc::mbar_wait_warp(&sh.sdp_full[h], ph, abort_flag)) { ok = false; break; }
+        SBP_ATTN_TIMED(w_sdp += clock64() - c0; c0 = clock64();)
         tc::fence_after_sync();
         uint32_t rs[32], rd[32];
         tc::tmem_ld32(tmem + lane_off + c_s(h) + 32 * wh, rs);
@@ -441,8 +483,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sh.ds_full[h]);
+        SBP_ATTN_TIMED(t_work += clock64() - c0;)
       }
       if (!ok || !pos.last) continue;
+      SBP_ATTN_TIMED(c0 = clock64();)
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner)
       // the release of this pair's Q/dO stage is committed after its last dK / dV product
       if (!tc::mbar_wait_warp(&sh.qd_empty[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u,
@@ -489,7 +533,12 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0 && j + 1 < npairs) tc::mbar_arrive(&sh.kv_free);
+      SBP_ATTN_TIMED(t_flush += clock64() - c0;)
     }
+    SBP_ATTN_TIMED(if (blockIdx.x == 0 && (warp == 2 || warp == 9) && lane == 0) printf(
+        "SBPT KVEW warp %d s %lld Tc %lld pairs %d total %lld w_qd %lld w_sdp %lld work %lld "
+        "flush %lld\n", warp, (long long)a.s, (long long)a.Tc, npairs, clock64() - te0, w_q,
+        w_sdp, t_work, t_flush);)
   }
 
   tc::fence_before_sync();

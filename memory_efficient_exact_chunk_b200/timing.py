@@ -1,15 +1,20 @@
-"""Cycle accounting of the pair GEMM on the LM-head CE backward, from the instrumented library.
+"""Cycle accounting of the pair GEMM and of the attention dK/dV kernel, from the instrumented
+library (libsbp_timing.so, built with SBP_GEMM_TIMING and SBP_ATTN_TIMING).
 
     python -m memory_efficient_exact_chunk_b200.build --timing
-    python -m memory_efficient_exact_chunk_b200.gemm_timing run > timing.log
-    python -m memory_efficient_exact_chunk_b200.gemm_timing summarize timing.log
+    python -m memory_efficient_exact_chunk_b200.timing lmhead > lmhead_timing.log
+    python -m memory_efficient_exact_chunk_b200.timing layer > layer_timing.log
+    python -m memory_efficient_exact_chunk_b200.timing summarize lmhead_timing.log
+    python -m memory_efficient_exact_chunk_b200.timing summarize layer_timing.log
 
-`run` loads libsbp_timing.so (the pair kernel built with SBP_GEMM_TIMING) and runs the LM-head
-CE backward twice (32768 tokens, D = 8, the bench's inputs); every pair-GEMM launch prints, for
-CTA 0 (and CTA 1 for the producer): the producer's cycles waiting for a free ring stage, the MMA
-issuer's cycles waiting for operands (full stage) and for a free accumulator, and two epilogue
-warps' cycles waiting for a full accumulator and working.  `summarize` keeps the second call
-(warm) and averages per launch shape.  Measurement only: the product library is not involved.
+`lmhead` runs the LM-head CE backward twice (32768 tokens, D = 8, the bench's inputs); every
+pair-GEMM launch prints, for CTA 0 (and CTA 1 for the producer): the producer's cycles waiting
+for a free ring stage, the MMA issuer's cycles waiting for operands (full stage) and for a free
+accumulator, and two epilogue warps' cycles waiting for a full accumulator and working.
+`layer` runs the Llama-3-8B-shaped layer backward twice (16384 tokens, D = 2); the dK/dV
+kernel's CTA 0 prints its producer's, MMA issuer's and two element-wise warps' accounts (and
+the layer's GEMMs print theirs).  `summarize` keeps the second call (warm) of each kind and
+averages per launch shape.  Measurement only: the product library is not involved.
 """
 from __future__ import annotations
 
@@ -18,13 +23,18 @@ import os
 import sys
 
 
-def run(tokens: int = 0, chunks: int = 0):
-    import torch
-    from . import build, sbp, synth
+def _load():
+    from . import build, sbp
     if not os.path.exists(build.LIB_TIMING):
         raise RuntimeError("libsbp_timing.so missing: python -m "
                            "memory_efficient_exact_chunk_b200.build --timing")
-    sbp.load(build.LIB_TIMING)
+    return sbp.load(build.LIB_TIMING)
+
+
+def run_lmhead(tokens: int = 0, chunks: int = 0):
+    import torch
+    from . import sbp, synth
+    _load()
     wl = synth.WORKLOADS["lmhead_ce_32k"]
     T, d, V = tokens or wl.seq_len, wl.hidden, wl.vocab
     D = chunks or wl.num_chunks
@@ -44,6 +54,31 @@ def run(tokens: int = 0, chunks: int = 0):
     print(f"SBPT DONE T {T} D {D} loss {float(loss.item()):.6f}", flush=True)
 
 
+def run_layer(tokens: int = 16384, chunks: int = 2):
+    import torch
+    from . import sbp, synth
+    _load()
+    wl = synth.WORKLOADS["llama3_8b_layer_32k"]
+    L, B, T, D = wl.layer, wl.batch, tokens, chunks
+    W, x, dy = synth.layer_inputs(2000, L, B, T, bf16=True, dy_std=1e-3)
+    dev = "cuda"
+    Wd = {n: (torch.from_numpy(W[n]).to(torch.bfloat16).to(dev) if W.get(n) is not None
+              else None) for n in sbp.WEIGHT_FIELDS}
+    xd = torch.from_numpy(x).to(torch.bfloat16).to(dev)
+    dyd = torch.from_numpy(dy).to(dev)
+    dx = torch.empty(B, T, L.d_model, device=dev)
+    grads = {n: (torch.zeros(Wd[n].shape, device=dev) if Wd.get(n) is not None else None)
+             for n in sbp.WEIGHT_FIELDS}
+    cfg = sbp.layer_cfg(B, T, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
+                        L.rms_eps, L.rope_theta, sbp.SBP_BF16, D)
+    ws = sbp.workspace(sbp.layer_workspace_size(cfg), dev)
+    for _ in range(2):
+        sbp.decoder_layer_backward(cfg, Wd, xd, dyd, dx, grads, ws=ws)
+        torch.cuda.synchronize()
+        sbp.device_status(ws)
+    print(f"SBPT DONE T {T} D {D}", flush=True)
+
+
 def _fields(line):
     t = line.split()[2:]
     return dict(zip(t[0::2], t[1::2]))
@@ -52,7 +87,7 @@ def _fields(line):
 def summarize(path: str) -> str:
     lines = [l.strip() for l in open(path) if l.startswith("SBPT ")]
     out = []
-    kinds = {"ISSUE": [], "PROD": [], "EPI": []}
+    kinds = {"ISSUE": [], "PROD": [], "EPI": [], "KVISSUE": [], "KVPROD": [], "KVEW": []}
     for l in lines:
         k = l.split()[1]
         if k in kinds:
@@ -115,12 +150,44 @@ def summarize(path: str) -> str:
         n, tot, wt, wk = eagg[key]
         out.append(f"| {key[0]} | {key[1]} | {names.get(key[2], key[2])} | {n} | "
                    f"{100 * wk / tot:.0f} % |")
+    if kinds["KVISSUE"]:
+        out.append("")
+        out.extend(_summarize_kv(kinds))
     return "\n".join(out)
 
 
+def _summarize_kv(kinds) -> list:
+    """Per (head, 128-query tile) pair averages of the dK/dV kernel's CTA 0, per launch."""
+    out = ["Attention dK/dV kernel, CTA 0 (one 128-key tile of one KV head), cycles per "
+           "(query head, 128-query tile) pair",
+           "| chunk start | Tc | pairs | total | MMA issuer: wait dS | wait Q/dO | wait flush | "
+           "issuing | element-wise: wait scores | working | flushing | producer: wait stage |",
+           "|---:|---:|---:|---:|---:|---:|---:|---:|---:|---:|---:|---:|"]
+    ew = collections.defaultdict(list)
+    for f in kinds["KVEW"]:
+        ew[(f["s"], f["Tc"])].append(f)
+    prod = {(f["s"], f["Tc"]): f for f in kinds["KVPROD"]}
+    for f in kinds["KVISSUE"]:
+        n = int(f["pairs"])
+        if n == 0:
+            continue
+        key = (f["s"], f["Tc"])
+        e = ew.get(key, [])
+        avg = lambda name: sum(int(x[name]) for x in e) / max(1, len(e)) / n
+        p = prod.get(key)
+        out.append(f"| {f['s']} | {f['Tc']} | {n} | {int(f['total']) / n:.0f} | "
+                   f"{int(f['w_ds']) / n:.0f} | {int(f['w_qd']) / n:.0f} | "
+                   f"{int(f['w_free']) / n:.0f} | {int(f['issue']) / n:.0f} | "
+                   f"{avg('w_sdp'):.0f} | {avg('work'):.0f} | {avg('flush'):.0f} | "
+                   f"{(int(p['w_empty']) / n if p else float('nan')):.0f} |")
+    return out
+
+
 if __name__ == "__main__":
-    if len(sys.argv) >= 2 and sys.argv[1] == "run":
-        run()
+    if len(sys.argv) >= 2 and sys.argv[1] == "lmhead":
+        run_lmhead()
+    elif len(sys.argv) >= 2 and sys.argv[1] == "layer":
+        run_layer()
     elif len(sys.argv) == 3 and sys.argv[1] == "summarize":
         print(summarize(sys.argv[2]))
     else:
