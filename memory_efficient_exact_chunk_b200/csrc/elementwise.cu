@@ -249,14 +249,26 @@ __global__ void rmsnorm_bwd_kernel(int64_t rows, int64_t cols, int xdt,
     partial[(int64_t)blockIdx.x * cols + c] = dgs[c];
 }
 
-__global__ void colsum_partials_kernel(int64_t nparts, int64_t cols,
-                                       const float* __restrict__ partial,
-                                       float* __restrict__ dst) {
-  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
+// dst[c] += sum_p partial[p, c].  A CTA of 256 threads takes 32 columns; its 8 warps sum
+// interleaved eighths of the partial rows, and warp 0 adds the eight sums in a fixed order.
+constexpr int kColsumCols = 32, kColsumGroups = 8;
+__global__ void __launch_bounds__(kColsumCols * kColsumGroups)
+colsum_partials_kernel(int64_t nparts, int64_t cols, const float* __restrict__ partial,
+                       float* __restrict__ dst) {
+  __shared__ float red[kColsumGroups][kColsumCols];
+  const int lc = threadIdx.x % kColsumCols, grp = threadIdx.x / kColsumCols;
+  const int64_t c = (int64_t)blockIdx.x * kColsumCols + lc;
   float s = 0.f;
-  for (int64_t p = 0; p < nparts; ++p) s += partial[p * cols + c];
-  dst[c] += s;
+  if (c < cols)
+    for (int64_t p = grp; p < nparts; p += kColsumGroups) s += partial[p * cols + c];
+  red[grp][lc] = s;
+  __syncthreads();
+  if (grp == 0 && c < cols) {
+    float t = red[0][lc];
+#pragma unroll
+    for (int g2 = 1; g2 < kColsumGroups; ++g2) t += red[g2][lc];
+    dst[c] += t;
+  }
 }
 
 // column partial sums of a [rows, cols] fp32 matrix: CTA b sums rows b, b + grid, ...
@@ -282,79 +294,90 @@ __global__ void rope_table_kernel(int64_t T, int64_t half, double theta, float* 
   sinb[i] = (float)sin(a);
 }
 
-// one thread per (row, head, pair j): rotates (x_j, x_{j+half}); heads h_lo .. h_hi - 1 of the
-// combined q | k | v head index
-__global__ void qkv_post_kernel(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H,
-                                int64_t Hkv, int64_t hd, int64_t h_lo, int64_t nh,
-                                const float* __restrict__ qkv, int dt, void* __restrict__ q,
-                                void* __restrict__ Kp, void* __restrict__ Vp,
-                                const float* __restrict__ cosb, const float* __restrict__ sinb) {
-  const int64_t half = hd / 2;
-  const int64_t heads = H + 2 * Hkv;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= R * nh * half) return;
-  const int64_t j = i % half;
-  const int64_t hh = h_lo + (i / half) % nh;
-  const int64_t r = i / (half * nh);
+// One CTA per row r (token s + r % Tc of sequence r / Tc); its threads stride over the
+// (head, pair j) slots of heads h_lo .. h_lo + nh - 1 of the combined q | k | v head index and
+// rotate (x_j, x_{j+half}) of q and k; v is copied.  Per-element index math is 32-bit.
+__global__ void qkv_post_kernel(int64_t Tc, int64_t s, int64_t T, int H, int Hkv, int hd,
+                                int h_lo, int nh, const float* __restrict__ qkv, int dt,
+                                void* __restrict__ q, void* __restrict__ Kp,
+                                void* __restrict__ Vp, const float* __restrict__ cosb,
+                                const float* __restrict__ sinb) {
+  const int64_t r = blockIdx.x;
+  const int half = hd / 2;
+  const int heads = H + 2 * Hkv;
   const int64_t b = r / Tc, t = s + r % Tc;
-  const int64_t width = heads * hd;
-  const float x1 = qkv[r * width + hh * hd + j];
-  const float x2 = qkv[r * width + hh * hd + j + half];
-  if (hh < H + Hkv) {
-    const float c = cosb[t * half + j], sn = sinb[t * half + j];
-    const float y1 = x1 * c - x2 * sn;
-    const float y2 = x2 * c + x1 * sn;
-    if (hh < H) {
-      const int64_t o = r * H * hd + hh * hd;
-      st_dt(q, dt, o + j, y1);
-      st_dt(q, dt, o + j + half, y2);
+  const float* row = qkv + r * (int64_t)heads * hd;
+  const float* cr = cosb + t * half;
+  const float* sr = sinb + t * half;
+  const int64_t qo = r * (int64_t)H * hd;               // this row in q [R, H * hd]
+  const int64_t ko = (b * T + t) * (int64_t)Hkv * hd;   // this token in the K/V prefix
+  const int n = nh * half;
+  for (int p = threadIdx.x; p < n; p += blockDim.x) {
+    const int hq = p / half;
+    const int j = p - hq * half;
+    const int hh = h_lo + hq;
+    const float x1 = row[hh * hd + j], x2 = row[hh * hd + j + half];
+    if (hh < H + Hkv) {
+      const float c = cr[j], sn = sr[j];
+      const float y1 = x1 * c - x2 * sn;
+      const float y2 = x2 * c + x1 * sn;
+      if (hh < H) {
+        st_dt(q, dt, qo + hh * hd + j, y1);
+        st_dt(q, dt, qo + hh * hd + j + half, y2);
+      } else {
+        st_dt(Kp, dt, ko + (hh - H) * hd + j, y1);
+        st_dt(Kp, dt, ko + (hh - H) * hd + j + half, y2);
+      }
     } else {
-      const int64_t o = (b * T + t) * Hkv * hd + (hh - H) * hd;
-      st_dt(Kp, dt, o + j, y1);
-      st_dt(Kp, dt, o + j + half, y2);
+      st_dt(Vp, dt, ko + (hh - H - Hkv) * hd + j, x1);
+      st_dt(Vp, dt, ko + (hh - H - Hkv) * hd + j + half, x2);
     }
-  } else {
-    const int64_t o = (b * T + t) * Hkv * hd + (hh - H - Hkv) * hd;
-    st_dt(Vp, dt, o + j, x1);
-    st_dt(Vp, dt, o + j + half, x2);
   }
 }
 
-// inverse rotation (transpose): (d1, d2) -> (d1 c + d2 s, d2 c - d1 s)
-__global__ void rope_inv_kernel(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd,
-                                float* __restrict__ x, const float* __restrict__ cosb,
-                                const float* __restrict__ sinb) {
-  const int64_t half = hd / 2;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= R * heads * half) return;
-  const int64_t j = i % half;
-  const int64_t hh = (i / half) % heads;
-  const int64_t r = i / (half * heads);
+// inverse rotation (transpose): (d1, d2) -> (d1 c + d2 s, d2 c - d1 s).  One CTA per row r
+// of x [R, heads, hd] (position s + r % Tc); threads stride over its (head, pair) slots.
+__global__ void rope_inv_kernel(int64_t Tc, int64_t s, int heads, int hd, float* __restrict__ x,
+                                const float* __restrict__ cosb, const float* __restrict__ sinb) {
+  const int64_t r = blockIdx.x;
+  const int half = hd / 2;
   const int64_t t = s + r % Tc;
-  const int64_t o = r * heads * hd + hh * hd;
-  const float d1 = x[o + j], d2 = x[o + j + half];
-  const float c = cosb[t * half + j], sn = sinb[t * half + j];
-  x[o + j] = d1 * c + d2 * sn;
-  x[o + j + half] = d2 * c - d1 * sn;
+  float* row = x + r * (int64_t)heads * hd;
+  const float* cr = cosb + t * half;
+  const float* sr = sinb + t * half;
+  const int n = heads * half;
+  for (int p = threadIdx.x; p < n; p += blockDim.x) {
+    const int hh = p / half;
+    const int j = p - hh * half;
+    float* o = row + hh * hd;
+    const float d1 = o[j], d2 = o[j + half];
+    const float c = cr[j], sn = sr[j];
+    o[j] = d1 * c + d2 * sn;
+    o[j + half] = d2 * c - d1 * sn;
+  }
 }
 
-__global__ void gather_rope_inv_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s,
-                                       int64_t heads, int64_t hd, const float* __restrict__ src,
-                                       float* __restrict__ dst, const float* __restrict__ cosb,
+// dst row r [heads, hd] = inverse rotation of src [B, T, heads, hd] at (r / Tc, s + r % Tc)
+__global__ void gather_rope_inv_kernel(int64_t T, int64_t Tc, int64_t s, int heads, int hd,
+                                       const float* __restrict__ src, float* __restrict__ dst,
+                                       const float* __restrict__ cosb,
                                        const float* __restrict__ sinb) {
-  const int64_t half = hd / 2;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * Tc * heads * half) return;
-  const int64_t j = i % half;
-  const int64_t hh = (i / half) % heads;
-  const int64_t r = i / (half * heads);
+  const int64_t r = blockIdx.x;
+  const int half = hd / 2;
   const int64_t b = r / Tc, t = s + r % Tc;
-  const int64_t so = (b * T + t) * heads * hd + hh * hd;
-  const int64_t o = r * heads * hd + hh * hd;
-  const float d1 = src[so + j], d2 = src[so + j + half];
-  const float c = cosb[t * half + j], sn = sinb[t * half + j];
-  dst[o + j] = d1 * c + d2 * sn;
-  dst[o + j + half] = d2 * c - d1 * sn;
+  const float* srow = src + (b * T + t) * (int64_t)heads * hd;
+  float* drow = dst + r * (int64_t)heads * hd;
+  const float* cr = cosb + t * half;
+  const float* sr = sinb + t * half;
+  const int n = heads * half;
+  for (int p = threadIdx.x; p < n; p += blockDim.x) {
+    const int hh = p / half;
+    const int j = p - hh * half;
+    const float d1 = srow[hh * hd + j], d2 = srow[hh * hd + j + half];
+    const float c = cr[j], sn = sr[j];
+    drow[hh * hd + j] = d1 * c + d2 * sn;
+    drow[hh * hd + j + half] = d2 * c - d1 * sn;
+  }
 }
 
 // ---------------------------------------------------------------- SwiGLU
@@ -589,7 +612,8 @@ cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !dg) return e;
-    launch(colsum_partials_kernel, dim3(nblk(cols, 256)), dim3(256), 0, st, (int64_t)kBwdBlocks,
+    launch(colsum_partials_kernel, dim3(nblk(cols, kColsumCols)),
+           dim3(kColsumCols * kColsumGroups), 0, st, (int64_t)kBwdBlocks,
            cols, (const float*)partial, dg);
     return cudaGetLastError();
   }
@@ -604,7 +628,8 @@ cudaError_t rmsnorm_bwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (dg) {
-    launch(colsum_partials_kernel, nblk(cols, 256), 256, 0, st, kBwdBlocks, cols, partial, dg);
+    launch(colsum_partials_kernel, nblk(cols, kColsumCols), kColsumCols * kColsumGroups, 0, st,
+           kBwdBlocks, cols, partial, dg);
     e = cudaGetLastError();
   }
   return e;
@@ -623,28 +648,27 @@ cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int
                      const float* cosb, const float* sinb, cudaStream_t st, int part) {
   const int64_t h_lo = part == QKV_KV ? H : 0;
   const int64_t h_hi = part == QKV_Q ? H : H + 2 * Hkv;
-  const int64_t n = R * (h_hi - h_lo) * (hd / 2);
-  if (n <= 0) return cudaSuccess;
-  launch(qkv_post_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, T, H, Hkv, hd, h_lo, h_hi - h_lo,
-         qkv, dt, q, Kp, Vp, cosb, sinb);
+  if (R <= 0 || h_hi <= h_lo || hd < 2) return cudaSuccess;
+  launch(qkv_post_kernel, dim3((unsigned)R), dim3(256), 0, st, Tc, s, T, (int)H, (int)Hkv,
+         (int)hd, (int)h_lo, (int)(h_hi - h_lo), qkv, dt, q, Kp, Vp, cosb, sinb);
   return cudaGetLastError();
 }
 
 cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd, float* x,
                          const float* cosb, const float* sinb, cudaStream_t st) {
-  const int64_t n = R * heads * (hd / 2);
-  if (n <= 0) return cudaSuccess;
-  launch(rope_inv_kernel, nblk(n, 256), 256, 0, st, R, Tc, s, heads, hd, x, cosb, sinb);
+  if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
+  launch(rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, Tc, s, (int)heads, (int)hd, x,
+         cosb, sinb);
   return cudaGetLastError();
 }
 
 cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t heads,
                             int64_t hd, const float* src, float* dst, const float* cosb,
                             const float* sinb, cudaStream_t st) {
-  const int64_t n = B * Tc * heads * (hd / 2);
-  if (n <= 0) return cudaSuccess;
-  launch(gather_rope_inv_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, heads, hd, src, dst, cosb,
-                                                       sinb);
+  const int64_t R = B * Tc;
+  if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
+  launch(gather_rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, T, Tc, s, (int)heads,
+         (int)hd, src, dst, cosb, sinb);
   return cudaGetLastError();
 }
 
@@ -699,7 +723,8 @@ cudaError_t colsum_acc(int64_t rows, int64_t cols, const float* src, float* dst,
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   dim3 g1(kColsumParts, nblk(cols, 256));
   launch(colsum_stage1_kernel, g1, 256, 0, st, rows, cols, src, partial);
-  launch(colsum_partials_kernel, nblk(cols, 256), 256, 0, st, kColsumParts, cols, partial, dst);
+  launch(colsum_partials_kernel, nblk(cols, kColsumCols), kColsumCols * kColsumGroups, 0, st,
+         kColsumParts, cols, partial, dst);
   return cudaGetLastError();
 }
 
