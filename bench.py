@@ -569,14 +569,15 @@ def run_reference(args, rank, world):
     value = n_rows * args.steps / t
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "lmhead_ce_32k", "batch": 1, "seq_len": 32768, "hidden": 3584,
                    "vocab": 152064, "num_chunks": 8},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
                          "kind": "oracle",
-                         "sample": f"{n_rows} loss tokens per step of the 32K LM-head workload"},
+                         "sample": f"{n_rows} loss tokens per step of the 32K LM-head workload, "
+                                   "on the host cores of rank 0 (no GPU work)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
