@@ -28,7 +28,12 @@ def _load():
     if not os.path.exists(build.LIB_TIMING):
         raise RuntimeError("libsbp_timing.so missing: python -m "
                            "memory_efficient_exact_chunk_b200.build --timing")
-    return sbp.load(build.LIB_TIMING)
+    lib = sbp.load(build.LIB_TIMING)
+    # load() keeps the first library a process opened: refuse to time the product one
+    if os.path.realpath(lib._name) != os.path.realpath(build.LIB_TIMING):
+        raise RuntimeError(f"{lib._name} is already loaded in this process; run the timing "
+                           "workload in a fresh process")
+    return lib
 
 
 def run_lmhead(tokens: int = 0, chunks: int = 0):
