@@ -144,3 +144,28 @@ def test_lmhead_host_entry_argument_errors(lib):
     assert call(wsb=64) == 3
     assert (sbp.lmhead_ce_workspace_size_host(1024, 64, 1000, 4, sbp.SBP_BF16) >
             sbp.lmhead_ce_workspace_size(1024, 64, 1000, 4, sbp.SBP_BF16) > 0)
+
+
+def test_workspace_falls_as_one_over_d_at_bench_shapes(lib):
+    """The O(T/D) claim, from the library's own sizing at the bench's full shapes (no GPU):
+    the LM head's workspace is a / D (everything in it is per chunk), the layer's a / D + b with
+    b the O(T d_kv) K/V prefix and fp32 dK/dV (R13)."""
+    import numpy as np
+    from memory_efficient_exact_chunk_b200 import synth
+    Ds = (1, 2, 4, 8, 16)
+    wl = synth.WORKLOADS["lmhead_ce_32k"]
+    lm = [sbp.lmhead_ce_workspace_size(wl.seq_len, wl.hidden, wl.vocab, D, sbp.SBP_BF16)
+          for D in Ds]
+    prod = [w * D for w, D in zip(lm, Ds)]
+    assert max(prod) / min(prod) < 1.001, prod
+    wl = synth.WORKLOADS["llama3_8b_layer_32k"]
+    L = wl.layer
+    lay = [sbp.layer_workspace_size(sbp.layer_cfg(wl.batch, wl.seq_len, L.d_model, L.n_heads,
+                                                  L.n_kv_heads, L.head_dim, L.ffn, L.rms_eps,
+                                                  L.rope_theta, sbp.SBP_BF16, D)) for D in Ds]
+    A = np.array([[1.0 / D, 1.0] for D in Ds])
+    (a, b), *_ = np.linalg.lstsq(A, np.array(lay, dtype=np.float64), rcond=None)
+    assert np.max(np.abs(A @ np.array([a, b]) - lay)) < 1e-6 * lay[0]
+    # b is the whole-sequence part: bf16 K/V prefix plus fp32 dK/dV, 12 bytes per K/V element
+    kv = wl.batch * wl.seq_len * L.n_kv_heads * L.head_dim
+    assert 12 * kv <= b < 12 * kv * 1.1, (b, 12 * kv)
