@@ -75,29 +75,37 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as fh:
-            for ln in fh:
-                f = [x.strip() for x in ln.split(",")]
-                if len(f) < 9:
-                    continue
-                try:
-                    sm.append(float(f[1]))
-                    mx = float(f[2])
-                except ValueError:
-                    continue
-                for nm, v in zip(names, f[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
+            out = parse_clocks(fh)
         try:
             os.remove(self.path)
         except OSError:
             pass
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return out
+
+
+def parse_clocks(lines):
+    """Median SM clock, the maximum clock and the throttle reasons seen in nvidia-smi records
+    of ClockSampler.FIELDS (csv, no header, no units); None without a usable record."""
+    sm, mx, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        f = [x.strip() for x in ln.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            clk, top = float(f[1]), float(f[2])
+        except ValueError:
+            continue
+        sm.append(clk)
+        mx = top
+        for nm, v in zip(names, f[5:9]):
+            if v.lower() == "active":
+                reasons.add(nm)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
 
 
 def fit_inverse_d(sweep):

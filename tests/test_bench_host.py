@@ -43,3 +43,39 @@ def test_committed_traffic_matches_the_kernel_file():
     gemm_tc.cu the DRAM-traffic capture in profiles/ has to be taken again (until then the
     bench line reports traffic null)."""
     assert bench.traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k") is not None
+
+
+def test_parse_clocks_reasons_and_median():
+    rec = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1500, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 10, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    c = bench.parse_clocks(rec)
+    assert c == {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    hot = rec[:1] + ["0, 900, 1965, 500, 0x8, Not Active, Active, Not Active, Not Active"]
+    assert bench.parse_clocks(hot)["reasons"] == ["hw_thermal_slowdown"]
+    assert bench.parse_clocks(["x"]) is None and bench.parse_clocks([]) is None
+
+
+def test_clock_sampler_stop_reads_and_removes_its_file(tmp_path):
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "clocks.csv")
+    with open(s.path, "w") as fh:
+        fh.write("0, 1800, 1965, 900, 0x4, Not Active, Not Active, Not Active, Active\n")
+
+    class Done:                       # a sampler process that has already exited
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s.proc = Done()
+    s.fh = open(str(tmp_path / "unused"), "w")
+    assert s.stop() == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                        "samples": 1}
+    assert not (tmp_path / "clocks.csv").exists()
