@@ -153,6 +153,21 @@ def attention_forward(q, k, v, q_start: int = 0):
     return out, p
 
 
+def attention_logsumexp(q, k, q_start: int = 0):
+    """Log of the softmax normaliser of each causal score row, lse [Tq, H]:
+    lse[t, h] = log sum_{u <= q_start + t} exp(q_t,h . k_u,g / sqrt(hd)), g = h // (H / Hkv).
+    The statistic a flash-style attention keeps from its forward so that the backward can
+    rebuild P = exp(S - lse) ([skill] Architecture Overview: the forward is recomputed per
+    chunk and its statistics reused by that chunk's backward)."""
+    Tq, H, hd = q.shape
+    Tk, Hkv, _ = k.shape
+    kk = np.repeat(k, H // Hkv, axis=1)
+    s = np.einsum("thd,uhd->htu", q, kk) / math.sqrt(hd)
+    s = np.where(np.arange(Tk)[None, :] <= q_start + np.arange(Tq)[:, None], s, -np.inf)
+    m = np.max(s, axis=-1, keepdims=True)
+    return (m[..., 0] + np.log(np.sum(np.exp(s - m), axis=-1))).T
+
+
 def attention_backward(dout, q, k, v, p):
     """Chain rule of attention_forward.  Returns (dq, dk, dv) with dk/dv summed per KV head."""
     Tq, H, hd = q.shape

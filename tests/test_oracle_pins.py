@@ -164,6 +164,29 @@ def test_attention_special_cases():
     assert np.allclose(out[:, 0], want, atol=1e-13) and np.allclose(out[:, 1], want, atol=1e-13)
 
 
+def test_attention_logsumexp_closed_forms():
+    """lse of a causal score row, pinned by closed forms: one key gives the score itself
+    (q.k / sqrt(hd): catches the scale); keys equal per KV head give score + log(t + 1) (the
+    causal count of keys seen by query t, offset by q_start: catches the mask) with head h
+    reading KV head h // (H / Hkv) (catches the GQA mapping)."""
+    rng = np.random.default_rng(11)
+    hd = 8
+    q = rng.standard_normal((1, 2, hd))
+    k = rng.standard_normal((1, 1, hd))
+    lse = O.attention_logsumexp(q, k)
+    assert np.allclose(lse[0], [q[0, 0] @ k[0, 0] / math.sqrt(hd), q[0, 1] @ k[0, 0] / math.sqrt(hd)],
+                       rtol=1e-14, atol=1e-15)
+    T, H, Hkv, q0 = 6, 4, 2, 3
+    kv = rng.standard_normal((Hkv, hd))
+    k = np.tile(kv[None], (q0 + T, 1, 1))
+    q = rng.standard_normal((T, H, hd))
+    lse = O.attention_logsumexp(q, k, q_start=q0)
+    for t in range(T):
+        for h in range(H):
+            want = q[t, h] @ kv[h // (H // Hkv)] / math.sqrt(hd) + math.log(q0 + t + 1)
+            assert abs(lse[t, h] - want) <= 1e-12 * max(1.0, abs(want)), (t, h)
+
+
 # ------------------------------------------------------------------------------------------
 # Layer: residual structure, finite differences, causality, chunk invariance
 # ------------------------------------------------------------------------------------------
