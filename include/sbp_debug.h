@@ -36,6 +36,21 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
                                void* workspace, void* stream);
 
 /*
+ * Test of the bounded waits (failure detection without a GPU fault).  Launches the single-CTA
+ * tensor-core GEMM of C = A B^T (A [M, K], B [N, K], both bf16 row-major with leading
+ * dimension K; C [M, N] fp32) with its producer told to issue no copy at all and every
+ * mbarrier wait bounded by `wait_limit_ns` (1e5 .. 2e9 ns, else SBP_ERR_INVALID_ARG).  The MMA
+ * issuer's first operand wait therefore runs out with no copy and no MMA in flight; the kernel
+ * takes its timeout exit (every role winds down, TMEM is freed) and raises SBP_ERR_DEVICE_TIMEOUT
+ * in the status word at the start of `workspace` (>= 256 bytes, zeroed by the caller), which
+ * sbp_get_device_status reports.  C is not written.  The same launch path as a normal GEMM,
+ * so a context that passes this call keeps working.  Device pointers, queued on `stream`.
+ */
+sbp_status sbp_debug_gemm_stall_bf16(int64_t M, int64_t N, int64_t K, const void* A,
+                                     const void* B, float* C, int64_t wait_limit_ns,
+                                     void* workspace, void* stream);
+
+/*
  * Causal GQA attention forward of one query chunk over its key prefix (bf16):
  *   q  [B * Tc, H, hd]  (chunk rows; row r is position s + r % Tc of sequence r / Tc)
  *   Kp, Vp [B, T, Hkv, hd] (keys/values of whole sequences; positions < s + Tc are read)

@@ -307,6 +307,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   // k-steps per K block and blocks per tile (one block, possibly empty, when kblk == 0)
   const int kpb = g.kblk > 0 ? (int)(g.kblk / BK) : (nk > 0 ? nk : 1);
   const int nblk = nk > 0 ? (nk + kpb - 1) / kpb : 1;
+  const bool stall = g.stall_wait_ns > 0;
+  const uint64_t wait_ns = stall ? (uint64_t)g.stall_wait_ns : tc::kWaitLimitNs;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -315,13 +317,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t ph = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int t = blockIdx.x; t < ntiles && ok && !stall; t += gridDim.x) {
         int mt, nt;
         tile_coords(t, args.nM, args.nN, mt, nt);
         const int m0 = mt * BM, n0 = nt * BN;
         if (m0 >= M) continue;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, wait_ns)) { ok = false; break; }
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           tc::mbar_expect_tx(&full_bar[s], STAGE_BYTES);
@@ -371,12 +373,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tile_coords(t, args.nM, args.nN, mt, nt);
         if ((int64_t)mt * BM >= M) continue;
         for (int b = 0; b < nblk && ok; ++b) {
-          if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, wait_ns)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
           const int kb0 = b * kpb, kb1 = imin(nk, kb0 + kpb);
           for (int kb = kb0; kb < kb1; ++kb) {
-            if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
+            if (!tc::mbar_wait(&full_bar[s], ph, abort_flag, wait_ns)) { ok = false; break; }
             tc::fence_after_sync();
             const uint32_t sa = smem_base + s * STAGE_BYTES;
             const uint32_t sb = sa + A_BYTES;
@@ -419,7 +421,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (m0 >= M) continue;
       bool ok = true;
       for (int b = 0; b < nblk; ++b) {
-        if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&tfull_bar[acc], aph, abort_flag, wait_ns)) { ok = false; break; }
         tc::fence_after_sync();
         const int64_t m = m0 + row_in_tile;
         const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);

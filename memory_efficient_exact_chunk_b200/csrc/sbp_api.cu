@@ -1039,6 +1039,25 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
   return SBP_OK;
 }
 
+sbp_status sbp_debug_gemm_stall_bf16(int64_t M, int64_t N, int64_t K, const void* A,
+                                     const void* B, float* C, int64_t wait_limit_ns,
+                                     void* workspace, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(SBP_ERR_INVALID_ARG, "sizes must be positive");
+  if (!A || !B || !C || !workspace) return fail(SBP_ERR_INVALID_ARG, "NULL pointer");
+  if (wait_limit_ns < 100000 || wait_limit_ns > 2000000000)
+    return fail(SBP_ERR_INVALID_ARG, "wait_limit_ns must be in [1e5, 2e9]");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  tl_status = static_cast<int*>(workspace);
+  GemmDesc g = mk_gemm(M, N, K, DT_BF16, A, false, K, DT_BF16, B, true, K, DT_F32, C, N,
+                       EPI_STORE);
+  g.path = 3;
+  g.stall_wait_ns = wait_limit_ns;
+  if (!gemm_tc_supported(g))
+    return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
+  SBP_CK(gemm(g, st));
+  return SBP_OK;
+}
+
 sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H,
                                    int64_t Hkv, int64_t hd, const void* q, const void* Kp,
                                    const void* Vp, void* o, float* lse, int path, void* workspace,

@@ -152,6 +152,11 @@ struct GemmDesc {
   // 0 = pick automatically, 1 = CUDA cores only, 2 = tensor cores (either kernel),
   // 3 = tensor cores, single-CTA kernel, 4 = tensor cores, CTA-pair kernel
   int path = 0;
+  // Test hook of the bounded waits (set only by sbp_debug_gemm_stall_bf16): > 0 makes the
+  // single-CTA kernel's producer issue no copy at all and bounds every wait by this many ns,
+  // so the MMA issuer's first operand wait runs out with no copy or MMA in flight and the
+  // kernel takes its timeout exit (status word raised, TMEM freed).
+  int64_t stall_wait_ns = 0;
 };
 
 // Number of column tiles the EPI_LSE epilogue writes per row (its partial buffers' width).

@@ -29,6 +29,7 @@ EXPORTS = [
     "sbp_debug_attn_fwd_bf16", "sbp_debug_attn_bwd_bf16", "sbp_lmhead_ce_forward_stream",
     "sbp_dpo_workspace_size", "sbp_dpo_token_weights", "sbp_lmhead_ce_workspace_size_host",
     "sbp_lmhead_ce_backward_stream_host", "sbp_decoder_layer_backward_stream_reverse",
+    "sbp_debug_gemm_stall_bf16",
 ]
 
 WEIGHT_FIELDS = ("ln1_g", "wq", "wk", "wv", "bq", "bk", "bv", "wo", "ln2_g", "w_gate", "w_up",
@@ -114,6 +115,7 @@ def load(path: Optional[str] = None):
                                          C.c_int, C.c_int, i64, vp, vp]
     lib.sbp_lmhead_ce_backward_noalloc.argtypes = [i64, i64, i64, C.c_int, C.c_int] + [vp] * 7 + \
         [vp]
+    lib.sbp_debug_gemm_stall_bf16.argtypes = [i64, i64, i64, vp, vp, vp, i64, vp, vp]
     lib.sbp_debug_attn_fwd_bf16.argtypes = [i64] * 7 + [vp] * 5 + [C.c_int, vp, vp]
     lib.sbp_debug_attn_bwd_bf16.argtypes = [i64] * 7 + [vp] * 9 + [C.c_int, vp, vp]
     lib.sbp_launch_count.restype = C.c_longlong
@@ -358,6 +360,20 @@ def debug_gemm_bf16(A, a_trans, B, b_trans, C, accumulate=False, path=0, kblk=0,
                                       int(b_trans), B.stride(0), _ptr(C), C.stride(0),
                                       int(accumulate), int(path), int(kblk), _ptr(ws),
                                       _stream(stream)))
+    return ws
+
+
+def debug_gemm_stall_bf16(A, B, C, wait_limit_ns, ws=None, stream=None):
+    """The single-CTA GEMM of C = A B^T with no operand copies issued, so that its bounded
+    waits run out after wait_limit_ns (include/sbp_debug.h); returns the workspace whose
+    status word the kernel raises."""
+    M, K = A.shape
+    N = B.shape[0]
+    if ws is None:
+        ws = workspace(256, C.device)
+        ws.zero_()
+    _check(load().sbp_debug_gemm_stall_bf16(M, N, K, _ptr(A), _ptr(B), _ptr(C),
+                                            int(wait_limit_ns), _ptr(ws), _stream(stream)))
     return ws
 
 

@@ -169,3 +169,21 @@ def test_workspace_falls_as_one_over_d_at_bench_shapes(lib):
     # b is the whole-sequence part: bf16 K/V prefix plus fp32 dK/dV, 12 bytes per K/V element
     kv = wl.batch * wl.seq_len * L.n_kv_heads * L.head_dim
     assert 12 * kv <= b < 12 * kv * 1.1, (b, 12 * kv)
+
+
+def test_noalloc_invalid_sizes_are_argument_errors(lib):
+    """Invalid sizes reach the caller as SBP_ERR_INVALID_ARG before any device or symbol
+    lookup (this host has no GPU, so a lookup would fail with SBP_ERR_CUDA instead)."""
+    for n, d, V, D in ((0, 64, 100, 1), (10, 0, 100, 1), (10, 64, 0, 1), (10, 64, 100, 0),
+                       (10, 64, 100, 11)):
+        rc = lib.sbp_lmhead_ce_backward_noalloc(n, d, V, D, sbp.SBP_BF16, *([None] * 8))
+        assert rc == 1, (n, d, V, D, rc)
+        assert "invalid sizes" in lib.sbp_last_error().decode()
+
+
+def test_stall_hook_argument_errors(lib):
+    f = lib.sbp_debug_gemm_stall_bf16
+    assert f(0, 256, 64, FAKE, FAKE, FAKE, 10**6, FAKE, None) == 1
+    assert f(128, 256, 64, None, FAKE, FAKE, 10**6, FAKE, None) == 1
+    assert f(128, 256, 64, FAKE, FAKE, FAKE, 10**4, FAKE, None) == 1
+    assert f(128, 256, 64, FAKE, FAKE, FAKE, 3 * 10**9, FAKE, None) == 1

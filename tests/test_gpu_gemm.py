@@ -106,3 +106,47 @@ def test_gemm_k_block_argument_checked():
     with pytest.raises(sbp.SbpError) as ei:
         sbp.debug_gemm_bf16(A, 0, B, 0, C, kblk=100)
     assert ei.value.code == 1
+
+
+@pytest.mark.parametrize("wait_ms", [2, 20])
+def test_bounded_wait_times_out_and_context_survives(wait_ms):
+    """Failure detection without a GPU fault: the single-CTA GEMM launched with a producer that
+    issues no copy, so its MMA issuer's operand wait can never complete.  The bounded wait must
+    give up after the stated limit with nothing in flight, every role must wind down and free
+    TMEM, the status word must report SBP_ERR_DEVICE_TIMEOUT (and be cleared by the read), C
+    must be left untouched, and a normal GEMM on the same device and workspace right after
+    must still match fp64."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(wait_ms)
+    A = torch.randn(256, 128, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(512, 128, generator=g).to(torch.bfloat16).cuda()
+    C = torch.full((256, 512), float("nan"), device="cuda")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    ws = sbp.debug_gemm_stall_bf16(A, B, C, wait_ms * 1_000_000)
+    t1.record()
+    with pytest.raises(sbp.SbpError) as e:
+        sbp.device_status(ws)
+    assert e.value.code == 5, e.value
+    elapsed = t0.elapsed_time(t1)
+    assert 0.9 * wait_ms <= elapsed <= wait_ms + 500.0, elapsed
+    assert torch.isnan(C).all()
+    sbp.device_status(ws)                       # the read cleared the word
+    sbp.debug_gemm_bf16(A, 0, B, 1, C, path=3, ws=ws)
+    sbp.device_status(ws)
+    ref = A.double().cpu() @ B.double().cpu().t()
+    err = ((C.double().cpu() - ref).norm() / ref.norm()).item()
+    assert err <= 1e-5, err
+
+
+def test_stall_entry_rejects_bad_limits():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    A = torch.zeros(128, 64, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(256, 64, dtype=torch.bfloat16, device="cuda")
+    C = torch.zeros(128, 256, device="cuda")
+    for bad in (0, 99_999, 2_000_000_001):
+        with pytest.raises(sbp.SbpError) as e:
+            sbp.debug_gemm_stall_bf16(A, B, C, bad)
+        assert e.value.code == 1
