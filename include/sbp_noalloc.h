@@ -20,14 +20,20 @@ extern "C" {
 /*
  * Same computation, arguments, layouts and accumulate rules as sbp_lmhead_ce_backward_stream,
  * without the workspace: the scratch is a 32 MiB array inside the library (a static device
- * array; every GPU that loads the library holds it until the process exits).  Nothing is
+ * array; a GPU holds it from the first call made on it until the process exits).  Nothing is
  * allocated: no cudaMalloc, no cudaFree, no allocating library routine.
  *
  *   - Size limit: sizes whose sbp_lmhead_ce_workspace_size() exceeds 32 MiB are rejected with
  *     SBP_ERR_WORKSPACE and a message in sbp_last_error(); raise num_chunks to shrink the
  *     per-chunk scratch (it scales with n_tokens / num_chunks), or use the workspace entry.
- *   - First call on a device: it looks up the device address of the scratch for the current
- *     device (once per device).  Make that first call before any stream capture begins.
+ *   - First call on a device does one-time set-up there, with that device current: it looks
+ *     up the device address of the scratch, which also makes the CUDA runtime load the module
+ *     holding the array (the driver reserves its 32 MiB at that moment, not when the library
+ *     is opened), and, like the first call of any libsbp entry point on a device, it creates
+ *     the library's side streams and events.  Neither may happen under stream capture: make
+ *     that first call before any capture begins.
+ *   - Invalid sizes (n_tokens, hidden or vocab <= 0, num_chunks outside [1, n_tokens]) return
+ *     SBP_ERR_INVALID_ARG before any device work or set-up.
  *   - Shared scratch: every call on a device uses the same scratch, which keeps the last call's
  *     contents; the call clears what must start at zero.  Calls whose GPU work overlaps
  *     (different streams or threads) race on it -- serialise them on one stream.

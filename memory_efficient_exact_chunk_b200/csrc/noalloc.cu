@@ -11,7 +11,10 @@
 // library holds kNoAllocScratchBytes of device memory for it until the process exits.
 //
 // The scratch is shared by every call on a device and keeps the last call's contents; the
-// library clears what must start at zero (its status word) at the start of each call.  Two
+// library clears what must start at zero (its status word) at the start of each call.  The
+// array lives in this file's module, which the CUDA runtime loads lazily: the driver reserves
+// its 32 MiB on a device at the first call there (the symbol lookup below), not when the
+// library is opened.  Two
 // calls whose GPU work overlaps (different streams, or different host threads) race on the
 // scratch: serialise them on one stream.
 #include <cstdio>
@@ -51,7 +54,14 @@ sbp_status sbp_lmhead_ce_backward_noalloc(int64_t n_tokens, int64_t hidden, int6
     sbp::set_last_error(msg);
     return SBP_ERR_WORKSPACE;
   }
-  // (need == 0 means invalid arguments: the call below reports them without touching memory.)
+  if (need == 0) {
+    // invalid sizes: reported before any device or symbol lookup, so that even a first call
+    // on a device returns the argument error itself
+    sbp::set_last_error(
+        "sbp_lmhead_ce_backward_noalloc: invalid sizes (n_tokens, hidden and vocab must be "
+        "positive and 1 <= num_chunks <= n_tokens)");
+    return SBP_ERR_INVALID_ARG;
+  }
   // Set-up, once per device, with that device current: the device address of the scratch.
   // (The array's name in host code is only a host-side stand-in, never a device address.)
   int dev = 0;

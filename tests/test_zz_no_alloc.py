@@ -27,6 +27,9 @@ def _outputs(N, d, V):
 
 @pytest.mark.parametrize("dtype,N,d,V,D", [("bf16", 640, 128, 3000, 4), ("f32", 300, 64, 1000, 3)])
 def test_noalloc_matches_workspace_entry_twice(dtype, N, d, V, D):
+    """Two calls in a row match the workspace entry point, and the calls allocate no device
+    memory: after the first call (which may do the per-device set-up) the driver's free memory
+    and torch's allocated bytes stay the same across the second call."""
     import torch
     from memory_efficient_exact_chunk_b200 import sbp
     h, W, y, w = synth.lmhead_inputs(21, N, d, V, bf16=(dtype == "bf16"))
@@ -34,10 +37,18 @@ def test_noalloc_matches_workspace_entry_twice(dtype, N, d, V, D):
     loss0, dH0, dW0 = _outputs(N, d, V)
     sbp.lmhead_ce_backward(hd, Wd, yd, wd, D, loss0, dH0, dW0)
     torch.cuda.synchronize()
-    for _ in range(2):
-        loss, dH, dW = _outputs(N, d, V)
+    outs = [_outputs(N, d, V) for _ in range(2)]
+    free_before = alloc_before = None
+    for i, (loss, dH, dW) in enumerate(outs):
+        if i == 1:
+            torch.cuda.synchronize()
+            free_before = torch.cuda.mem_get_info()[0]
+            alloc_before = torch.cuda.memory_allocated()
         sbp.lmhead_ce_backward_noalloc(hd, Wd, yd, wd, D, loss, dH, dW)
         torch.cuda.synchronize()
+        if i == 1:
+            assert torch.cuda.mem_get_info()[0] == free_before
+            assert torch.cuda.memory_allocated() == alloc_before
         assert abs(loss.item() - loss0.item()) <= 1e-5 * abs(loss0.item())
         assert rel_fro(to_np(dH), to_np(dH0)) <= 1e-5
         assert rel_fro(to_np(dW), to_np(dW0)) <= 1e-5
