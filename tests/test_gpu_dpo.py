@@ -113,29 +113,33 @@ def _bf16_store(a):
     return synth.bf16_round(np.asarray(a, np.float32)).astype(np.float64)
 
 
-def _oracle_dpo(L, inp, beta, bf16):
+def _oracle_dpo(L, inp, beta, bf16, store=True):
     layers, E, fg, lm, ids, y, m, ref = inp
     loss, g, _ = O.stack_dpo(oracle_cfg(O, L), f64(E),
                              [{n: f64(W.get(n)) for n in NAMES} for W in layers], f64(fg),
                              f64(lm), ids, y, f64(m), f64(ref), beta,
-                             store=_bf16_store if bf16 else None)
+                             store=_bf16_store if (bf16 and store) else None)
     out = {"lm_head": g["lm_head"], "final_g": g["final_g"], "embed": g["embed"]}
     for n, v in g["layers"][0].items():
         out[f"L0.{n}"] = v
     return loss, out
 
 
-@pytest.mark.parametrize("dtype,L,P,T,D,tol", [
-    ("f32", synth.LayerShape(64, 4, 4, 16, 172, 1e-6, 10000.0), 1, 128, 4, 1e-5),
-    ("bf16", synth.LayerShape(128, 4, 2, 32, 192, 1e-5, 500000.0), 2, 256, 4, 1e-2),
+@pytest.mark.parametrize("dtype,L,P,T,D,tol,store", [
+    ("f32", synth.LayerShape(64, 4, 4, 16, 172, 1e-6, 10000.0), 1, 128, 4, 1e-5, False),
+    ("bf16", synth.LayerShape(128, 4, 2, 32, 192, 1e-5, 500000.0), 2, 256, 4, 1e-2, True),
+    ("bf16", synth.LayerShape(128, 4, 2, 32, 192, 1e-5, 500000.0), 2, 256, 4, 1e-2, False),
 ])
-def test_stack_dpo_step_matches_oracle(dtype, L, P, T, D, tol):
+def test_stack_dpo_step_matches_oracle(dtype, L, P, T, D, tol, store):
+    """store=False: the oracle keeps every tensor in fp64 (no bf16 rounding of the stored
+    checkpoints), so the whole bf16 error is measured."""
     inp = _dpo_inputs(7, L, 600, P, T, dtype == "bf16")
     beta = 0.5
     loss, g = _gpu_dpo(L, inp, D, dtype, beta)
-    l0, g0 = _oracle_dpo(L, inp, beta, dtype == "bf16")
+    l0, g0 = _oracle_dpo(L, inp, beta, dtype == "bf16", store)
     assert abs(loss - l0) <= tol * abs(l0), (loss, l0)
     errs = {k: rel_fro(v, g0[k]) for k, v in g.items()}
+    print("dpo errors:", {k: float(f"{v:.3g}") for k, v in errs.items()})
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, errs
 

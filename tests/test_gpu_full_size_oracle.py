@@ -1,0 +1,168 @@
+"""Oracle checks at the 32K-token length of the Llama-3-8B-shaped layer, in the launch
+configuration of its D = 8 chunks (4096 queries per chunk over a key prefix of up to 32768).
+
+The oracle cannot run these sizes whole, so each check is on outputs it can compute one by one
+(the paper page's Abstract claims gradients identical to full backprop; these are the pieces
+of that claim the oracle can reach at full length):
+  * attention output and log-sum-exp of single query rows over their whole causal prefix;
+  * dQ of single query rows (a query row's gradient depends on its own score row only);
+  * dK / dV of the last key rows, whose queries all lie in the last chunk;
+  * rows of the layer forward's output;
+  * dX of the last rows of the sequence, which no later token depends on.
+Two attention inputs: plain N(0, 1) rows, and keys with a drift that makes the scores of a
+query rise along the sequence (its running maximum grows over the 256 key tiles, so the
+forward's deferred rescaling of O and the backward's P = exp(S - lse) are exercised at full
+length)."""
+import numpy as np
+import pytest
+
+from oracle import sbp_oracle as O
+from memory_efficient_exact_chunk_b200 import synth
+from tests.helpers import f64, oracle_cfg
+
+pytestmark = pytest.mark.gpu
+
+T, H, HKV, HD, D = 32768, 32, 8, 128, 8
+TC = T // D
+Q_ROWS = (0, 1, 4095, 4096, 12345, 20000, 28672, 32767)
+HEADS = (0, 13, 31)
+
+
+def _rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def _attention_inputs(seed, drift):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H, HD), dtype=np.float32)
+    k = rng.standard_normal((T, HKV, HD), dtype=np.float32)
+    v = rng.standard_normal((T, HKV, HD), dtype=np.float32)
+    dO = rng.standard_normal((T, H, HD), dtype=np.float32)
+    if drift:
+        # scores q.k/sqrt(hd) gain about 40 * u / T along the keys u: a shared direction in
+        # every query and a key component that grows with the position
+        e = np.zeros(HD, np.float32)
+        e[:4] = 0.5
+        q += 4.0 * e
+        k += (np.float32(40.0 * np.sqrt(HD) / 4.0) * (np.arange(T, dtype=np.float32) / T))[
+            :, None, None] * e
+    return tuple(synth.bf16_round(a) for a in (q, k, v, dO))
+
+
+def _gpu_attention(q, k, v, dO):
+    """All D chunks through the debug entries, as the layer's chunk loop issues them."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
+    qd, dOd = bf(q), bf(dO)
+    Kp, Vp = bf(k)[None], bf(v)[None]
+    o = torch.empty(T, H, HD, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(T, H, device="cuda")
+    dq = torch.full((T, H, HD), float("nan"), device="cuda")
+    dK = torch.zeros(1, T, HKV, HD, device="cuda")
+    dV = torch.zeros(1, T, HKV, HD, device="cuda")
+    for i in range(D):
+        s = i * TC
+        ws = sbp.debug_attn_fwd_bf16(qd[s:s + TC], Kp, Vp, o[s:s + TC], lse[s:s + TC], s, path=2)
+        sbp.device_status(ws)
+    for i in range(D):
+        s = i * TC
+        ws = sbp.debug_attn_bwd_bf16(qd[s:s + TC], Kp, Vp, o[s:s + TC], dOd[s:s + TC],
+                                     lse[s:s + TC], dq[s:s + TC], dK, dV, s, path=2)
+        sbp.device_status(ws)
+    torch.cuda.synchronize()
+    return (o.float().cpu().numpy(), lse.cpu().numpy(), dq.cpu().numpy(),
+            dK[0].cpu().numpy(), dV[0].cpu().numpy())
+
+
+@pytest.mark.parametrize("drift", [False, True])
+def test_attention_rows_at_32k(drift):
+    q, k, v, dO = _attention_inputs(91 + drift, drift)
+    o, lse, dq, dK, dV = _gpu_attention(q, k, v, dO)
+    q64, k64, v64, dO64 = (a.astype(np.float64) for a in (q, k, v, dO))
+    grp = H // HKV
+    worst = {"o": 0.0, "lse": 0.0, "dq": 0.0}
+    for t in Q_ROWS:
+        for h in HEADS:
+            g = h // grp
+            qs = q64[t:t + 1, h:h + 1]
+            ks, vs = k64[:t + 1, g:g + 1], v64[:t + 1, g:g + 1]
+            out, p = O.attention_forward(qs, ks, vs, q_start=t)
+            l0 = O.attention_logsumexp(qs, ks, q_start=t)[0, 0]
+            dq0, _, _ = O.attention_backward(dO64[t:t + 1, h:h + 1], qs, ks, vs, p)
+            e = {"o": _rel(o[t, h], out[0, 0]), "lse": abs(float(lse[t, h]) - l0),
+                 "dq": _rel(dq[t, h], dq0[0, 0])}
+            for n in worst:
+                worst[n] = max(worst[n], e[n])
+            assert e["o"] <= 1e-2 and e["dq"] <= 1e-2, (t, h, e)
+            assert e["lse"] <= 2e-3 * max(1.0, abs(l0)), (t, h, e, l0)
+    # dK / dV of the last key rows: every query that reads them lies in [u0, T)
+    u0 = T - 256
+    for g in (0, 5):
+        heads = slice(g * grp, (g + 1) * grp)
+        qs = q64[u0:, heads]
+        out, p = O.attention_forward(qs, k64[:, g:g + 1], v64[:, g:g + 1], q_start=u0)
+        _, dk0, dv0 = O.attention_backward(dO64[u0:, heads], qs, k64[:, g:g + 1],
+                                           v64[:, g:g + 1], p)
+        for u in (u0, u0 + 100, T - 2, T - 1):
+            ek, ev = _rel(dK[u, g], dk0[u, 0]), _rel(dV[u, g], dv0[u, 0])
+            worst["dk"] = max(worst.get("dk", 0.0), ek)
+            worst["dv"] = max(worst.get("dv", 0.0), ev)
+            assert ek <= 1e-2 and ev <= 1e-2, (g, u, ek, ev)
+    print(f"attention at T={T} (drift={drift}) worst errors:", worst)
+
+
+def _layer_setup():
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    wl = synth.WORKLOADS["llama3_8b_layer_32k"]
+    L = wl.layer
+    W, x, dy = synth.layer_inputs(79, L, 1, wl.seq_len, bf16=True, dy_std=1e-3)
+    Wd = {n: (torch.from_numpy(W[n]).to(torch.bfloat16).cuda() if W.get(n) is not None else None)
+          for n in sbp.WEIGHT_FIELDS}
+    cfg = sbp.layer_cfg(1, wl.seq_len, L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
+                        L.rms_eps, L.rope_theta, sbp.SBP_BF16, wl.num_chunks)
+    W64 = {n: f64(W.get(n)) for n in sbp.WEIGHT_FIELDS}
+    return wl, L, W, x, dy, Wd, cfg, W64
+
+
+def test_llama_layer_rows_at_32k():
+    """Layer forward output rows (D = 8) and the last rows of the layer backward's dX, forward
+    and reverse chunk order, against the oracle over their whole causal prefix."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    wl, L, W, x, dy, Wd, cfg, W64 = _layer_setup()
+    xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    y = torch.empty_like(xd)
+    ws = sbp.decoder_layer_forward(cfg, Wd, xd, y)
+    sbp.device_status(ws)
+    y = y.float().cpu().numpy()[0]
+    del ws
+    ocfg = oracle_cfg(O, L)
+    x64 = x[0].astype(np.float64)
+    errs = {}
+    for t in (0, 4095, 4096, 20000, T - 1):
+        y0, _ = O.layer_forward_rows(ocfg, W64, x64[:t + 1], t)
+        e_y = _rel(y[t], y0[0])
+        e_delta = _rel(y[t] - x64[t], y0[0] - x64[t])     # the layer's own contribution
+        errs[t] = (e_y, e_delta)
+        assert e_y <= 4e-3 and e_delta <= 1e-2, (t, e_y, e_delta)
+    print("layer forward rows (y, y - x):", errs)
+    # dX of the last 8 rows: only queries t >= those rows read their keys/values
+    r0 = T - 8
+    _, cache = O.layer_forward_rows(ocfg, W64, x64, r0)
+    dx0, _ = O.layer_backward_rows(ocfg, W64, cache, dy[0, r0:].astype(np.float64))
+    dyd = torch.from_numpy(dy).cuda()
+    for run in (sbp.decoder_layer_backward, sbp.decoder_layer_backward_reverse):
+        dx = torch.full(xd.shape, float("nan"), device="cuda")
+        g = {n: (torch.zeros(v.shape, device="cuda") if v is not None else None)
+             for n, v in Wd.items()}
+        ws = run(cfg, Wd, xd, dyd, dx, g)
+        sbp.device_status(ws)
+        got = dx[0, r0:].double().cpu().numpy()
+        del ws, g
+        e = _rel(got, dx0[r0:])
+        print(f"{run.__name__}: last-row dX error {e:.3g}")
+        assert e <= 1e-2, (run.__name__, e)

@@ -47,22 +47,38 @@ def _oracle(L, W, x, dy, sum_scales=None):
 
 
 def _check(L, W, x, dy, D, dtype, tol=None, reverse=False):
+    """Every output against the oracle in the plain per-tensor relative Frobenius error, bias
+    gradients included.  On the bf16 path the key-bias gradient is the one tensor held to a
+    looser plain bound (BK_BF16_PLAIN): it is a column sum over tokens with heavy cancellation
+    (softmax is shift invariant, so without RoPE sum_t dk_t is exactly 0), and the bf16
+    rounding of the attention operands, ~2^-9 per summand, is amplified by the cancellation
+    ratio sum|dk| / |sum dk|.  There it must also meet the stated tolerance against the sum of
+    the absolute summands, the error scale of a rounded sum."""
     tol = tol or TOL[dtype]
     dx, g = _gpu_layer(L, W, x, dy, D, dtype, reverse=reverse)
     scales = {}
     dx0, g0 = _oracle(L, W, x, dy, scales)
     errs = {"dx": rel_fro(dx, dx0)}
     for n in g:
-        if n in ("bq", "bk", "bv"):
-            # a bias gradient is a column sum over tokens with heavy cancellation (softmax is
-            # shift invariant: without RoPE sum_t dk_t = 0), so its rounding error is measured
-            # against the sum of the absolute summands, the error scale of a sum
-            errs[n] = float(np.linalg.norm(f64(g[n]) - g0[n]) / np.linalg.norm(scales[n]))
-        else:
-            errs[n] = rel_fro(g[n], g0[n])
-    bad = {k: v for k, v in errs.items() if not v <= tol}
-    assert not bad, (errs, tol)
+        errs[n] = rel_fro(g[n], g0[n])
+    limits = {k: tol for k in errs}
+    summand = {}
+    if dtype == "bf16" and "bk" in g:
+        limits["bk"] = BK_BF16_PLAIN
+        summand["bk"] = float(np.linalg.norm(f64(g["bk"]) - g0["bk"]) / np.linalg.norm(scales["bk"]))
+    print("layer errors:", {k: float(f"{v:.3g}") for k, v in errs.items()},
+          "bk vs summands:", summand, "cancellation:",
+          {n: float(f"{np.linalg.norm(scales[n]) / max(np.linalg.norm(g0[n]), 1e-300):.3g}")
+           for n in ("bq", "bk", "bv") if n in g})
+    bad = {k: v for k, v in errs.items() if not v <= limits[k]}
+    bad.update({f"{k}/summands": v for k, v in summand.items() if not v <= tol})
+    assert not bad, (errs, summand, tol)
     return dx, g
+
+
+# Plain relative error allowed for the bf16 key-bias gradient (see _check); every other tensor
+# of the bf16 path meets 1e-2 plainly.
+BK_BF16_PLAIN = 5e-2
 
 
 TINY = synth.LayerShape(64, 4, 4, 16, 172, 1e-6, 10000.0)           # the fp32 tiny model

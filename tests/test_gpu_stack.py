@@ -51,31 +51,38 @@ def _bf16_store(a):
     return synth.bf16_round(np.asarray(a, np.float32)).astype(np.float64)
 
 
-def check(L, stack_in, D, dtype, tol):
+def check(L, stack_in, D, dtype, tol, store=True):
+    """Every gradient against the oracle in the plain per-tensor relative Frobenius error.
+    ``store``: on the bf16 path, give the oracle the bf16 rounding of the tensors the stack
+    keeps between its passes (layer-input checkpoints, final-norm output); False runs the
+    oracle on its own fp64 values throughout.  The bf16 key-bias gradients are held to the
+    looser plain bound of test_gpu_layer (a sum with heavy cancellation) and, in addition, to
+    ``tol`` against the sum of their absolute summands."""
+    from tests.test_gpu_layer import BK_BF16_PLAIN
     layers, E, fg, lm, ids, y, w = stack_in
     loss, dlm, dfg, dE, dls = run_gpu(L, layers, E, fg, lm, ids, y, w, D, dtype)
     scales = []
     l0, g0 = O.stack_forward_backward(oracle_cfg(O, L), f64(E),
                                       [{n: f64(W.get(n)) for n in NAMES} for W in layers],
                                       f64(fg), f64(lm), ids, y, f64(w),
-                                      store=_bf16_store if dtype == "bf16" else None,
+                                      store=_bf16_store if (dtype == "bf16" and store) else None,
                                       sum_scales=scales)
     assert abs(loss - l0) <= tol * abs(l0)
     errs = {"lm_head": rel_fro(dlm, g0["lm_head"]), "final_g": rel_fro(dfg, g0["final_g"]),
             "embed": rel_fro(dE, g0["embed"])}
+    limits = {}
+    summand = {}
     for i, lg in enumerate(dls):
         for n, v in lg.items():
-            if n in ("bq", "bk", "bv"):
-                # a bias gradient is a column sum over tokens with heavy cancellation (softmax
-                # is shift invariant: without RoPE sum_t dk_t = 0), so its rounding error is
-                # measured against the sum of the absolute summands, the error scale of a sum
-                ref = g0["layers"][i][n]
-                errs[f"L{i}.{n}"] = float(np.linalg.norm(f64(v) - ref) /
-                                          np.linalg.norm(scales[i][n]))
-            else:
-                errs[f"L{i}.{n}"] = rel_fro(v, g0["layers"][i][n])
-    print("stack errors:", {k: float(f"{v:.3g}") for k, v in errs.items()})
-    bad = {k: v for k, v in errs.items() if not v <= tol}
+            errs[f"L{i}.{n}"] = rel_fro(v, g0["layers"][i][n])
+            if n == "bk" and dtype == "bf16":
+                limits[f"L{i}.{n}"] = BK_BF16_PLAIN
+                summand[f"L{i}.{n}"] = float(np.linalg.norm(f64(v) - g0["layers"][i][n]) /
+                                             np.linalg.norm(scales[i][n]))
+    print("stack errors:", {k: float(f"{v:.3g}") for k, v in errs.items()},
+          "bk vs summands:", {k: float(f"{v:.3g}") for k, v in summand.items()})
+    bad = {k: v for k, v in errs.items() if not v <= limits.get(k, tol)}
+    bad.update({f"{k}/summands": v for k, v in summand.items() if not v <= tol})
     assert not bad, bad
 
 
@@ -87,17 +94,19 @@ def test_tiny_fp32_stack_full_size():
     check(wl.layer, s, wl.num_chunks, "f32", 1e-5)
 
 
-def test_bf16_gqa_stack_shifted_targets():
+@pytest.mark.parametrize("store", [True, False])
+def test_bf16_gqa_stack_shifted_targets(store):
     L = synth.LayerShape(128, 4, 2, 32, 192, 1e-5, 500000.0)
     s = make_stack(1, L, 2, 700, 1, 256, "bf16", "shifted_tail", from_frac=0.25)
-    check(L, s, 4, "bf16", 1e-2)
+    check(L, s, 4, "bf16", 1e-2, store=store)
 
 
-def test_bf16_grpo_batched_stack():
+@pytest.mark.parametrize("store", [True, False])
+def test_bf16_grpo_batched_stack(store):
     L = synth.LayerShape(128, 4, 1, 32, 160, 1e-6, 1e6, qkv_bias=True)
     rng = np.random.default_rng(9)
     B, T, V = 3, 128, 600
     layers, E, fg, lm, ids, y, _ = make_stack(2, L, 2, V, B, T, "bf16", "shifted_tail",
                                               from_frac=0.25)
     w = synth.loss_weights("grpo", B, T, prompt_len=32, advantages=rng.standard_normal(B))
-    check(L, (layers, E, fg, lm, ids, y, w), 4, "bf16", 1e-2)
+    check(L, (layers, E, fg, lm, ids, y, w), 4, "bf16", 1e-2, store=store)
