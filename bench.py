@@ -2,14 +2,20 @@
 """Benchmark of the streamed exact backward (StreamBP) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sbp|reference]
-                    [--workload lmhead_ce_32k|llama3_8b_layer_32k] [--chunks D] [--no-sweep]
+                    [--workload llama3_8b_stack4_64k|lmhead_ce_32k|llama3_8b_layer_32k]
+                    [--chunks D] [--no-sweep] [--no-e2e] [--no-lmhead] [--no-layer] [--no-stack]
 
-Default workload: the chunked LM-head + cross-entropy backward of a 32K-token SFT sequence
-(hidden 3584 = an RMSNorm output ~ N(0,1), vocabulary 152064, weight ~ N(0, 0.02), uniform
-targets, first 30 % of tokens loss-masked), bf16 operands with fp32 accumulation, D = 8.
-One step = one call of sbp_lmhead_ce_backward_stream over the whole sequence (all chunks).
-Inputs are resident in HBM and larger than L2 (the 1.09 GB LM-head weight is streamed by
-every chunk), so no explicit L2 flush is used.  Prints ONE JSON line on rank 0.
+Default workload, the largest configuration that fits one GPU: a 4-layer Llama-3-8B-shaped
+decoder stack (d 4096, 32 query / 8 KV heads of 128, SwiGLU 14336, RoPE theta 5e5) with an
+untied LM head (vocabulary 128256), bf16 operands with fp32 accumulation, one 65536-token
+sequence, next-token targets, mean CE over the last 75 % of tokens, D = 16.  One step = the
+streamed backward of the whole stack from its layer-input checkpoints (LM-head CE, final norm,
+four layers, embedding), all chunks.  Inputs are resident in HBM and larger than L2 (every
+chunk re-reads each layer's weights and the LM-head weight), so no explicit L2 flush is used.
+The line's `e2e` times the whole training step through the public API with the token data in
+pinned host memory (copied in, forward + backward, loss read back).  Prints ONE JSON line on
+rank 0; the LM-head workload (32K tokens, vocabulary 152064, D = 8), the single layer (32K
+tokens, D = 8) and the GRPO / DPO stacks follow under `also`.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own independent sequence
 (weak scaling, no data-path collective); the time is the max over ranks.
@@ -130,26 +136,37 @@ def lmhead_workload(T):
     return wl, T or wl.seq_len
 
 
-def traffic_from_profiles(kernel_src: str, workload: str):
-    """DRAM bytes per launch recorded by an ncu capture in profiles/, if neither the kernel
-    source nor the vocabulary block that shapes the LM head's launches has changed since (the
-    summary stores a hash of the kernel file and of the block constant)."""
-    path = os.path.join(ROOT, "profiles", f"{workload}_gemm_tc.md")
-    csrc = os.path.join(ROOT, "memory_efficient_exact_chunk_b200", "csrc")
-    src, api = os.path.join(csrc, kernel_src), os.path.join(csrc, "sbp_api.cu")
-    if not (os.path.exists(path) and os.path.exists(src) and os.path.exists(api)):
+def sources_hash(rel_paths) -> str:
+    """First 16 hex digits of the sha256 over the files (repo-relative paths, in order)."""
+    h = hashlib.sha256()
+    for rel in rel_paths:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(key: str):
+    """DRAM bytes per launch of the kernel `key` recorded in profiles/traffic.json (the figure
+    of an ncu capture summarised in profiles/), or None if the sources it was captured on have
+    changed since (the entry stores their hash, and literal lines that fix the launch shapes,
+    such as the vocabulary block of the LM head, which must still be present)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
         return None
-    blk = re.search(r"constexpr int64_t kVocabBlock = (\d+);", open(api).read())
-    if not blk:
+    with open(path) as fh:
+        ent = json.load(fh).get(key)
+    if not ent:
         return None
-    h = hashlib.sha256(open(src, "rb").read() +
-                       f"kVocabBlock={blk.group(1)}".encode()).hexdigest()[:16]
-    txt = open(path).read()
-    mh = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", txt)
-    mb = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", txt)
-    if not (mh and mb) or mh.group(1) != h:
+    try:
+        if sources_hash(ent["sources"]) != ent["sources_sha256_16"]:
+            return None
+        for rel, line in ent.get("requires", []):
+            with open(os.path.join(ROOT, rel)) as fh:
+                if line not in fh.read():
+                    return None
+    except OSError:
         return None
-    return float(mb.group(1))
+    return float(ent["dram_bytes_per_launch"])
 
 
 def run_lmhead(args, rank, world, device):
@@ -157,7 +174,7 @@ def run_lmhead(args, rank, world, device):
     from memory_efficient_exact_chunk_b200 import sbp, synth
     wl = synth.WORKLOADS["lmhead_ce_32k"]
     T, d, V = (args.tokens or wl.seq_len), wl.hidden, wl.vocab
-    D = args.chunks or wl.num_chunks
+    D = (args.chunks if args.workload == "lmhead_ce_32k" else 0) or wl.num_chunks
     h, W, y, w = synth.lmhead_inputs(1000 + rank, T, d, V, bf16=True, from_frac=wl.loss_from_frac)
     n_valid = int(np.count_nonzero(w))
     hd = torch.from_numpy(h).to(torch.bfloat16).to(device)
@@ -185,7 +202,7 @@ def run_lmhead(args, rank, world, device):
     torch.cuda.synchronize()
     peak_alloc = torch.cuda.max_memory_allocated(device)
     out = {
-        "tokens_per_step": T, "n_loss_tokens": n_valid, "flops_step": flops_step,
+        "tokens_per_step": T, "world": world, "n_loss_tokens": n_valid, "flops_step": flops_step,
         "flops_min_step": flops_min, "res": res, "ws_bytes": ws.numel(),
         "peak_act_gb": (peak_alloc - resident) / 1e9, "D": D,
         "config": {"workload": "lmhead_ce_32k" if T == wl.seq_len else f"lmhead_ce_{T}",
@@ -401,7 +418,7 @@ def run_dpo_stack(args, rank, world, device, name="qwen25_7b_stack2_dpo"):
     }
 
 
-def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k"):
+def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k", steps=1, e2e=False):
     """A decoder stack + untied LM head, bf16, through the streamed entry points:
     llama3_8b_stack4_64k: four Llama-3-8B-shaped layers, vocabulary 128256, T = 65536, D = 16,
         targets = next token, mean CE over the last 75 % of tokens;
@@ -410,13 +427,16 @@ def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k"):
         the response tokens after a 2048-token prompt).
     Weights are drawn on the device from a seeded generator (N(0, 0.02), gains 1).  The
     forward (layer-input checkpoints) and the streamed backward are timed separately; the
-    metric is the backward."""
+    metric is the backward (`steps` timed steps after args.warmup warm-ups).  With `e2e`, the
+    whole training step is also timed through the public API from pinned host memory: the
+    step's token ids, targets and loss weights are copied in, the forward and the streamed
+    backward run, and the loss is read back."""
     import torch
     from memory_efficient_exact_chunk_b200 import sbp, stack, synth
     wl = synth.WORKLOADS[name]
     L, B, V = wl.layer, wl.batch, wl.vocab
     T = (args.stack_tokens or wl.seq_len) if name.startswith("llama") else wl.seq_len
-    D = wl.num_chunks
+    D = (args.chunks or wl.num_chunks) if args.workload == name else wl.num_chunks
     gen = torch.Generator(device=device).manual_seed(3000 + rank)
 
     def rnd(*shape):
@@ -458,36 +478,96 @@ def run_stack(args, rank, world, device, name="llama3_8b_stack4_64k"):
 
     def bwd():
         xs, hf, rstd = state["ck"]
-        stack.stack_backward_from(cfg, layers, final_g, lm_w, ids_d, y_d, w_d, xs, hf, rstd, ws,
-                                  grads=grads)
+        state["r"] = stack.stack_backward_from(cfg, layers, final_g, lm_w, ids_d, y_d, w_d, xs,
+                                               hf, rstd, ws, grads=grads)
 
+    torch.cuda.synchronize(device)
+    base = torch.cuda.memory_allocated(device)     # weights, gradients, inputs
     fwd()
-    sargs = argparse.Namespace(steps=1, warmup=args.warmup)
+    sargs = argparse.Namespace(steps=steps, warmup=args.warmup)
     rb = timed(sargs, bwd, world, device, profile=True)
     rf = timed(argparse.Namespace(steps=1, warmup=1), fwd, world, device, profile=False)
+    torch.cuda.synchronize(device)
+    torch.cuda.reset_peak_memory_stats(device)
+    bwd()
+    torch.cuda.synchronize(device)
+    peak_total = torch.cuda.max_memory_allocated(device)
+    xs, hf, rstd = state["ck"]
+    ck = sum(t.numel() * t.element_size() for t in list(xs) + [hf, rstd])
+    ws_gb = sum(t.numel() for t in ws.bufs.values()) / 1e9
+    from memory_efficient_exact_chunk_b200 import memory_model as MM
+    model = MM.stack_step_bytes(MM.StackShape.from_workload(wl), T, D) if B == 1 else None
     P = sum(int(layers[0][n].numel()) for n in ("wq", "wk", "wv", "wo", "w_gate", "w_up",
                                                 "w_down"))
+    pairs = B * T * (T + 1) / 2 * L.n_heads * wl.n_layers     # causal (query, key, head) pairs
     lin = 6.0 * P * B * T * wl.n_layers
-    att = 14.0 * L.head_dim * L.n_heads * B * T * (T + 1) / 2 * wl.n_layers
+    att = 14.0 * L.head_dim * pairs
     head = 8.0 * n_loss * d * V
     prof = rb["prof"]
-    return {
-        "workload": wl.name if T == wl.seq_len else f"{wl.name[:-4]}_{T}",
+    k = steps
+
+    def tf(flops, ms):
+        return flops * k / (ms / 1e3) / 1e12 if ms > 0 else None
+
+    out = {
+        "workload": wl.name if T == wl.seq_len and D == wl.num_chunks
+        else f"{wl.name.rsplit('_', 1)[0]}_{T}_d{D}",
         "value": B * T * world / (rb["ms"] / 1e3), "unit": "tokens/s",
-        "ms_per_step": rb["ms"], "forward_ms": rf["ms"],
+        "ms_per_step": rb["ms"], "steps": k, "forward_ms": rf["ms"],
         "fwd_bwd_tokens_per_s": B * T * world / ((rb["ms"] + rf["ms"]) / 1e3),
-        "config": {"batch": B, "seq_len": T, "n_layers": wl.n_layers, "vocab": V,
-                   "num_chunks": D, "n_loss_tokens": n_loss},
+        "config": stack_config_dict(wl, T, D, n_loss),
         "flops_step": {"layers_linear_6P": lin, "layers_attention_14hd": att,
                        "lmhead_8NdV": head},
         "achieved_tflops_step": (lin + att + head) / (rb["ms"] / 1e3) / 1e12,
-        "kernels": {n: {"launches_per_step": v["launches"], "ms_per_step": v["ms"],
-                        "busy_ms_per_step": v["busy_ms"],
+        "kernels": {n: {"launches_per_step": v["launches"] / k, "ms_per_step": v["ms"] / k,
+                        "busy_ms_per_step": v["busy_ms"] / k,
                         "share": v["busy_ms"] / rb["ms_total"] if rb["ms_total"] else None}
                     for n, v in prof.items() if v["launches"]},
+        "attn_bwd_flops_step": 10.0 * L.head_dim * pairs,
+        "attn_fwd_flops_step": 4.0 * L.head_dim * pairs,
+        "gemm_tc_tflops": tf(lin + head, prof["gemm_tc"]["busy_ms"]),
+        "attn_fwd_tflops": tf(4.0 * L.head_dim * pairs, prof["attn_fwd"]["busy_ms"]),
+        "attn_bwd_tflops": tf(10.0 * L.head_dim * pairs, prof["attn_bwd"]["busy_ms"]),
+        "attn_bwd_busy_ms_total": prof["attn_bwd"]["busy_ms"],
+        "attn_bwd_launches_per_step": prof["attn_bwd"]["launches"] / k,
         "gpu_launches": rb["launches"], "clocks": rb["clocks"],
-        "workspace_gb": sum(t.numel() for t in ws.bufs.values()) / 1e9,
+        # transient memory of the streamed backward: its peak minus weights, gradients,
+        # inputs and the forward's checkpoints
+        "peak_act_gb": (peak_total - base - ck) / 1e9, "workspace_gb": ws_gb,
+        "peak_total_gb": peak_total / 1e9, "checkpoints_gb": ck / 1e9,
+        "model_total_gb": model["total"] / 1e9 if model else None,
+        "model_transient_gb": MM.transient_bytes(model) / 1e9 if model else None,
     }
+    if e2e:
+        ids_h = torch.from_numpy(ids.reshape(-1)).pin_memory()
+        y_h = torch.from_numpy(y.reshape(-1)).pin_memory()
+        w_h = torch.from_numpy(w.reshape(-1)).pin_memory()
+        loss_h = torch.zeros(1).pin_memory()
+
+        def e2e_step():
+            ids_d.copy_(ids_h, non_blocking=True)
+            y_d.copy_(y_h, non_blocking=True)
+            w_d.copy_(w_h, non_blocking=True)
+            fwd()
+            bwd()
+            loss_h.copy_(state["r"].loss, non_blocking=True)
+
+        # fewer timed steps than the device-resident timing: each e2e step also runs the
+        # forward, and the whole bench should stay within a few minutes
+        e2e_steps = min(steps, 8)
+        re_ = timed(argparse.Namespace(steps=e2e_steps, warmup=args.warmup), e2e_step, world,
+                    device, profile=False)
+        out["e2e"] = {"value": B * T * world / (re_["ms"] / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": ids_h.numel() * 4 + y_h.numel() * 4 +
+                      w_h.numel() * 4,
+                      "d2h_bytes_per_step": 4,
+                      "ms_per_step": re_["ms"], "steps": e2e_steps,
+                      "what": "training step through the public API: token ids, targets and "
+                              "loss weights copied from pinned host memory, forward "
+                              "(layer-input checkpoints) + streamed backward on the device, "
+                              "loss read back; weights and fp32 gradients stay resident in "
+                              "HBM (a device-resident training step fed with host token data)"}
+    return out
 
 
 def max_over_ranks(ms: float, world: int) -> float:
@@ -564,28 +644,108 @@ def cpu_baseline(n_rows=2048):
                       f"152064), fp64 numpy, {dt:.1f} s"}
 
 
+class OracleStackSample:
+    """The fp64 oracle on a bounded sample of the 4-layer Llama-3-8B-shaped stack workload:
+    one layer at full width (d 4096, 32/8 heads of 128, MLP 14336) on T_layer tokens (forward
+    recompute + backward, as the streamed backward does per chunk), and the LM head at full
+    width (vocabulary 128256) on `rows` loss rows.  Inputs are drawn once; run() times one pass
+    and returns the stack's tokens/s implied by it: per token, four layers plus the LM head on
+    the workload's share of loss tokens (75 %).  Attention is quadratic in T, so the reduced T
+    understates the oracle's cost per token at 64K tokens."""
+
+    def __init__(self, T_layer=512, rows=256, seed=7):
+        from memory_efficient_exact_chunk_b200 import synth
+        from oracle import sbp_oracle as O
+        self.O = O
+        wl = synth.WORKLOADS["llama3_8b_stack4_64k"]
+        self.wl, L = wl, wl.layer
+        self.T, self.rows = T_layer, rows
+        W, x, dy = synth.layer_inputs(seed, L, 1, T_layer, bf16=True, dy_std=1e-3)
+        self.W = {n: (None if v is None else v.astype(np.float64)) for n, v in W.items()}
+        self.x, self.dy = x.astype(np.float64), dy.astype(np.float64)
+        self.cfg = O.LayerConfig(L.d_model, L.n_heads, L.n_kv_heads, L.head_dim, L.ffn,
+                                 L.rms_eps, L.rope_theta)
+        self.h, self.Wh, self.y, self.w = synth.lmhead_inputs(seed, rows, L.d_model, wl.vocab,
+                                                              bf16=True, from_frac=0.0)
+        self.Wh = self.Wh.astype(np.float64)
+        self.loss_share = 1.0 - wl.loss_from_frac
+
+    def run(self):
+        t0 = time.perf_counter()
+        self.O.decoder_layer_backward(self.cfg, self.W, self.x, self.dy)
+        t1 = time.perf_counter()
+        self.O.lmhead_ce_forward_backward(self.h, self.Wh, self.y, self.w)
+        t2 = time.perf_counter()
+        per_token = (self.wl.n_layers * (t1 - t0) / self.T +
+                     self.loss_share * (t2 - t1) / self.rows)
+        return 1.0 / per_token, t2 - t0
+
+    def describe(self):
+        return (f"fp64 numpy oracle: one Llama-3-8B-shaped layer (forward + backward) on "
+                f"{self.T} tokens and the 128256-word LM head on {self.rows} loss rows, both at "
+                f"full width; tokens/s of the 4-layer stack + head implied per token "
+                f"(4 x layer + {self.loss_share:.2f} x head)")
+
+
+def cpu_baseline_stack():
+    smp = OracleStackSample()
+    smp.run()                                     # warm the BLAS threads
+    vals, secs = [], 0.0
+    while secs < 10.0 and len(vals) < 5:
+        v, dt = smp.run()
+        vals.append(v)
+        secs += dt
+    return {"value": statistics.median(vals), "unit": "tokens/s", "cores": cpu_cores(),
+            "kind": "oracle", "sample": f"{smp.describe()}; median of {len(vals)} passes, "
+                                        f"{secs:.1f} s"}
+
+
+def stack_config_dict(wl, T, D, n_loss):
+    """Shapes of a stack workload as the line's config reports them (both arms)."""
+    L = wl.layer
+    return {"batch": wl.batch, "seq_len": T, "n_layers": wl.n_layers, "d_model": L.d_model,
+            "n_heads": L.n_heads, "n_kv_heads": L.n_kv_heads, "head_dim": L.head_dim,
+            "ffn": L.ffn, "vocab": wl.vocab, "num_chunks": D, "n_loss_tokens": n_loss,
+            "loss": wl.loss}
+
+
+def stack_config(o):
+    """The line's config for a stack workload (the same keys as the reference arm's)."""
+    return dict(workload=o["workload"], **o["config"], l2=STACK_L2_NOTE)
+
+
+STACK_L2_NOTE = ("inputs larger than L2 (each layer's 0.44 GB of weights and the 1.05 GB "
+                 "LM-head weight are re-read per chunk)")
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on the host cores of rank 0, on a
+    bounded sample of the 4-layer stack workload per step (the other ranks exit at once)."""
     if rank != 0:
         return 0
-    n_rows = 16
-    oracle_lmhead_sample(4)                       # warm the BLAS threads
-    for _ in range(args.warmup):
-        oracle_lmhead_sample(n_rows)
-    t = 0.0
+    from memory_efficient_exact_chunk_b200 import synth
+    smp = OracleStackSample(T_layer=128, rows=64)
+    wl = synth.WORKLOADS["llama3_8b_stack4_64k"]
+    for _ in range(max(args.warmup, 1)):
+        smp.run()
+    t, vals = 0.0, []
     for _ in range(args.steps):
-        t += oracle_lmhead_sample(n_rows)
-    value = n_rows * args.steps / t
+        v, dt = smp.run()
+        vals.append(v)
+        t += dt
+    value = statistics.median(vals)
+    w = synth.loss_weights("shifted_tail", wl.batch, wl.seq_len, from_frac=wl.loss_from_frac)
+    cfg = dict(workload=wl.name, **stack_config_dict(wl, wl.seq_len, wl.num_chunks,
+                                                     int(np.count_nonzero(w))), l2=STACK_L2_NOTE)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "lmhead_ce_32k", "batch": 1, "seq_len": 32768, "hidden": 3584,
-                   "vocab": 152064, "num_chunks": 8},
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
                          "kind": "oracle",
-                         "sample": f"{n_rows} loss tokens per step of the 32K LM-head workload, "
-                                   "on the host cores of rank 0 (no GPU work)"},
+                         "sample": smp.describe() + " per step, on the host cores of rank 0 "
+                                                    "(no GPU work)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -619,27 +779,232 @@ def layer_main(args, rank, world, device):
     return 0
 
 
+# ----------------------------------------------------------------------------- memory
+def maxlen_main(args, rank, world, device):
+    """Longest sequence of the 4-layer Llama-3-8B-shaped stack + LM head that one GPU holds, by
+    the library's memory model (memory_model.py) at D = 1, 2, 4, 8, 16, 32, with the budget =
+    the device memory free after the CUDA context is up; then one streamed training step
+    (forward + backward) at T = --stack-tokens and D = --chunks, whose
+    torch.cuda.max_memory_allocated is compared with the model's prediction.  Prints one JSON
+    line (not the bench contract's line)."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import memory_model as MM
+    from memory_efficient_exact_chunk_b200 import sbp, stack, synth
+    wl = synth.WORKLOADS["llama3_8b_stack4_64k"]
+    shape = MM.StackShape.from_workload(wl)
+    free0, total = torch.cuda.mem_get_info(device)
+    budget = free0 - (1 << 30)          # 1 GiB for torch's allocator slack and the kernels' own
+    model = {D: MM.max_tokens(shape, D, budget) for D in (1, 2, 4, 8, 16, 32)}
+    T = args.stack_tokens or model[args.chunks or 1]
+    T = T // 128 * 128
+    D = args.chunks or 1
+    L = wl.layer
+    gen = torch.Generator(device=device).manual_seed(5000 + rank)
+
+    def rnd(*sh):
+        return (torch.randn(*sh, generator=gen, device=device) * 0.02).to(torch.bfloat16)
+
+    d, dq, dkv, f, V = (L.d_model, L.n_heads * L.head_dim, L.n_kv_heads * L.head_dim, L.ffn,
+                        wl.vocab)
+    layers = [{"ln1_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+               "wq": rnd(dq, d), "wk": rnd(dkv, d), "wv": rnd(dkv, d), "wo": rnd(d, dq),
+               "ln2_g": torch.ones(d, dtype=torch.bfloat16, device=device),
+               "w_gate": rnd(f, d), "w_up": rnd(f, d), "w_down": rnd(d, f),
+               "bq": None, "bk": None, "bv": None} for _ in range(wl.n_layers)]
+    embed, lm_w = rnd(V, d), rnd(V, d)
+    final_g = torch.ones(d, dtype=torch.bfloat16, device=device)
+    rng = np.random.default_rng(5000 + rank)
+    ids = synth.token_ids(rng, 1, T, V)
+    y = synth.shifted_targets(ids)
+    w = synth.loss_weights("shifted_tail", 1, T, from_frac=wl.loss_from_frac)
+    ids_d = torch.from_numpy(ids.reshape(-1)).to(device)
+    y_d = torch.from_numpy(y.reshape(-1)).to(device)
+    w_d = torch.from_numpy(w.reshape(-1)).to(device)
+    cfg = sbp.layer_cfg(1, T, d, L.n_heads, L.n_kv_heads, L.head_dim, f, L.rms_eps,
+                        L.rope_theta, sbp.SBP_BF16, D)
+    grads = stack.zero_grads(layers, lm_w, final_g, device, embed_shape=embed.shape)
+    ws = stack.Workspaces(device)
+    torch.cuda.synchronize(device)
+    torch.cuda.reset_peak_memory_stats(device)
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record()
+    xs, hf, rstd = stack.stack_forward(cfg, embed, layers, final_g, ids_d, ws)
+    e1.record()
+    r = stack.stack_backward_from(cfg, layers, final_g, lm_w, ids_d, y_d, w_d, xs, hf, rstd, ws,
+                                  grads=grads)
+    e2.record()
+    torch.cuda.synchronize(device)
+    peak = torch.cuda.max_memory_allocated(device)
+    pred = MM.stack_step_bytes(shape, T, D)
+    loss = float(r.loss.item())
+    line = {
+        "mode": "maxlen", "workload": "llama3_8b_stack4 + LM head 128256", "device_total_gb":
+        total / 1e9, "budget_gb": budget / 1e9,
+        "model_max_tokens": {str(k): v for k, v in model.items()},
+        "run": {"seq_len": T, "num_chunks": D, "measured_peak_gb": peak / 1e9,
+                "model_gb": pred["total"] / 1e9,
+                "model_parts_gb": {k: v / 1e9 for k, v in pred.items()},
+                "forward_ms": e0.elapsed_time(e1), "backward_ms": e1.elapsed_time(e2),
+                "loss": loss, "finite": bool(np.isfinite(loss))},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
+def lmhead_summary(out, args, peaks, peak_src):
+    """The LM-head workload's numbers with the roofline of its dominant kernel, the tcgen05
+    GEMM: all GEMM launches of a step, timed as the union of their CUDA-event intervals (the dH
+    and dW products overlap on side streams)."""
+    res = out["res"]
+    prof = res["prof"]["gemm_tc"]
+    tc_ms = prof["busy_ms"]
+    n_l = max(prof["launches"], 1)
+    achieved = (out["flops_step"] * args.steps) / (tc_ms / 1e3) / 1e12 if tc_ms > 0 else 0.0
+    peak = float(peaks["bf16_tflops_sustained"])
+    o = {
+        "workload": out["config"]["workload"],
+        "value": out["tokens_per_step"] * out["world"] / (res["ms"] / 1e3), "unit": "tokens/s",
+        "ms_per_step": res["ms"], "steps": args.steps, "config": out["config"],
+        "roofline": {
+            "bound": "tensor", "kernel": "gemm_tc2_kernel (tcgen05, all GEMM launches of a step)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak if peak else None,
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "flops_per_launch": out["flops_step"] / (n_l / args.steps),
+            "launch_ms": prof["ms"] / n_l, "launches_per_step": n_l / args.steps,
+            "gemm_busy_ms_per_step": tc_ms / args.steps,
+            "share_of_step": tc_ms / res["ms_total"] if res["ms_total"] else None,
+            "achieved_min_flops": (out["flops_min_step"] * args.steps) / (tc_ms / 1e3) / 1e12
+            if tc_ms > 0 else 0.0,
+            "traffic": traffic_from_profiles("gemm_tc2_kernel@lmhead_ce_32k"),
+        },
+        "gpu_launches": res["launches"], "clocks": res["clocks"],
+        "peak_act_gb": out["peak_act_gb"], "workspace_gb": out["ws_bytes"] / 1e9,
+    }
+    for k in ("sweep", "memory_fit", "e2e"):
+        if k in out:
+            o[k] = out[k]
+    return o
+
+
+def base_line(world, args, o):
+    return {"metric": METRIC, "value": o["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": o.get("steps", args.steps), "warmup": args.warmup,
+            "ms_per_step": o["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+
+
+def stack_main(args, rank, world, device):
+    """Default line: the 4-layer Llama-3-8B-shaped stack + LM head (T = 65536, D = 16), the
+    largest configuration that fits one GPU.  value = streamed-backward tokens/s."""
+    import torch
+    import torch.distributed as dist
+    peaks, peak_src = load_peaks()
+    o = run_stack(args, rank, world, device, "llama3_8b_stack4_64k", steps=args.steps,
+                  e2e=args.e2e)
+    peak = float(peaks["bf16_tflops_sustained"])
+    k = o["steps"]
+    busy = o["attn_bwd_busy_ms_total"]
+    n_l = max(o["attn_bwd_launches_per_step"], 1)
+    achieved = o["attn_bwd_tflops"] or 0.0
+    line = base_line(world, args, o)
+    line.update({
+        "config": stack_config(o),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attention backward (attn_bwd_kv_kernel + attn_bwd_q_kernel, tcgen05; "
+                      "one call per chunk and layer, its two kernels side by side)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak if peak else None,
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long "
+                           "step)",
+            "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
+            "flops_per_unit": "10 * head_dim per causal (query, key, head) pair",
+            "flops_per_launch": o["attn_bwd_flops_step"] / n_l,
+            "launches_per_step": n_l,
+            "launch_ms": busy / k / n_l,
+            "share_of_step": o["kernels"]["attn_bwd"]["share"],
+            "traffic": traffic_from_profiles("attn_bwd@llama3_8b_stack4_64k"),
+        },
+        "gpu_launches": o["gpu_launches"], "clocks": o["clocks"],
+        "peak_act_gb": o["peak_act_gb"], "stack": o,
+    })
+    if "e2e" in o:
+        line["e2e"] = o.pop("e2e")
+    also = []
+    if args.lmhead:
+        torch.cuda.empty_cache()
+        out = run_lmhead(args, rank, world, device)
+        also.append(lmhead_summary(out, args, peaks, peak_src))
+        del out
+    if args.layer:
+        torch.cuda.empty_cache()
+        also.append(run_layer(args, rank, world, device, sweep=args.sweep))
+    if args.stack:
+        torch.cuda.empty_cache()
+        also.append(run_stack(args, rank, world, device, "qwen25_7b_stack2_grpo"))
+        torch.cuda.empty_cache()
+        also.append(run_dpo_stack(args, rank, world, device))
+    if also:
+        line["also"] = also
+    line["cpu_baseline"] = cpu_baseline_stack() if (args.cpu and rank == 0 and world == 1) \
+        else None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def lmhead_main(args, rank, world, device):
+    """The LM-head workload as the line's own workload."""
+    import torch.distributed as dist
+    peaks, peak_src = load_peaks()
+    out = run_lmhead(args, rank, world, device)
+    o = lmhead_summary(out, args, peaks, peak_src)
+    line = base_line(world, args, o)
+    line.update({k: o[k] for k in ("config", "roofline", "gpu_launches", "clocks",
+                                   "peak_act_gb", "workspace_gb")})
+    for k in ("sweep", "memory_fit", "e2e"):
+        if k in o:
+            line[k] = o[k]
+    line["cpu_baseline"] = cpu_baseline() if (args.cpu and rank == 0 and world == 1) else None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sbp", choices=["sbp", "reference"])
-    ap.add_argument("--workload", default="lmhead_ce_32k",
-                    choices=["lmhead_ce_32k", "llama3_8b_layer_32k"])
-    ap.add_argument("--chunks", type=int, default=0)
+    ap.add_argument("--workload", default="llama3_8b_stack4_64k",
+                    choices=["llama3_8b_stack4_64k", "lmhead_ce_32k", "llama3_8b_layer_32k",
+                             "maxlen"])
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="override D of the line's own workload")
     ap.add_argument("--tokens", type=int, default=0,
-                    help="override the sequence length (small cases for profiling)")
+                    help="override the LM head's sequence length (small cases for profiling)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--no-lmhead", dest="lmhead", action="store_false",
+                    help="skip the LM-head measurement added to the stack line")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the decoder-layer measurement added to the line")
     ap.add_argument("--layer-tokens", type=int, default=0)
     ap.add_argument("--no-stack", dest="stack", action="store_false",
-                    help="skip the 4-layer stack measurement added to the line")
-    ap.add_argument("--stack-tokens", type=int, default=0)
+                    help="skip the GRPO / DPO stack measurements added to the line")
+    ap.add_argument("--stack-tokens", type=int, default=0,
+                    help="override the 4-layer stack's sequence length (small cases)")
     ap.add_argument("--layer-chunks", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -662,70 +1027,11 @@ def main():
     sbp.load()
     if args.workload == "llama3_8b_layer_32k":
         return layer_main(args, rank, world, device)
-    out = run_lmhead(args, rank, world, device)
-    res = out["res"]
-    peaks, peak_src = load_peaks()
-    prof = res["prof"]["gemm_tc"]
-    # GEMMs of one step run side by side on the library's streams: the time the GPU spent
-    # with at least one GEMM running (union of the launch intervals) is the denominator
-    tc_ms = prof["busy_ms"]
-    n_l = max(prof["launches"], 1)
-    achieved = (out["flops_step"] * args.steps) / (tc_ms / 1e3) / 1e12 if tc_ms > 0 else 0.0
-    peak = float(peaks["bf16_tflops_sustained"])
-    traffic = traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k")
-    line = {
-        "metric": METRIC,
-        "value": out["tokens_per_step"] * world / (res["ms"] / 1e3),
-        "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": out["config"],
-        "roofline": {
-            "bound": "tensor", "kernel": "gemm_tc_kernel (tcgen05, all GEMM launches of a step)",
-            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak if peak else None,
-            "peak_source": f"{peak_src} bf16_tflops_sustained",
-            "flops_per_launch": out["flops_step"] / (n_l / args.steps),
-            "launch_ms": prof["ms"] / n_l, "launches_per_step": n_l / args.steps,
-            "gemm_busy_ms_per_step": tc_ms / args.steps,
-            "share_of_step": tc_ms / res["ms_total"] if res["ms_total"] else None,
-            "achieved_min_flops": (out["flops_min_step"] * args.steps) / (tc_ms / 1e3) / 1e12
-            if tc_ms > 0 else 0.0,
-            "traffic": traffic,
-        },
-        "gpu_launches": res["launches"],
-        "clocks": res["clocks"],
-        "peak_act_gb": out["peak_act_gb"],
-        "workspace_gb": out["ws_bytes"] / 1e9,
-    }
-    if "sweep" in out:
-        line["sweep"] = out["sweep"]
-        line["memory_fit"] = out["memory_fit"]
-    also = []
-    if args.layer:
-        also.append(run_layer(args, rank, world, device, sweep=args.sweep))
-    if args.stack:
-        import torch
-        for name in ("llama3_8b_stack4_64k", "qwen25_7b_stack2_grpo"):
-            torch.cuda.empty_cache()
-            also.append(run_stack(args, rank, world, device, name))
-        torch.cuda.empty_cache()
-        also.append(run_dpo_stack(args, rank, world, device))
-    if also:
-        line["also"] = also
-    if "e2e" in out:
-        line["e2e"] = out["e2e"]
-    if args.cpu and rank == 0 and world == 1:
-        line["cpu_baseline"] = cpu_baseline()
-    else:
-        line["cpu_baseline"] = None
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    if args.workload == "lmhead_ce_32k":
+        return lmhead_main(args, rank, world, device)
+    if args.workload == "maxlen":
+        return maxlen_main(args, rank, world, device)
+    return stack_main(args, rank, world, device)
 
 
 if __name__ == "__main__":

@@ -1,7 +1,9 @@
-"""Host-side logic of bench.py on CPU: the a / D + b fit of the activation memory, and the
-per-launch DRAM traffic that the line reports only while the kernel file and the vocabulary
-block it was captured with are unchanged."""
+"""Host-side logic of bench.py on CPU: the a / D + b fit of the activation memory, the clock
+record parsing, and the per-launch DRAM traffic that the line reports only while the kernel
+sources and the launch shapes it was captured with are unchanged."""
 import hashlib
+import json
+import os
 
 import bench
 
@@ -14,35 +16,51 @@ def test_fit_inverse_d_recovers_a_and_b():
     assert bench.fit_inverse_d(sweep[:1]) is None and bench.fit_inverse_d([]) is None
 
 
-def _tree(tmp_path, src_text, api_block, stored_hash, bytes_per_launch="4.9e8"):
+def _tree(tmp_path, src_text, api_line, entry):
     root = tmp_path / "r"
     csrc = root / "memory_efficient_exact_chunk_b200" / "csrc"
     csrc.mkdir(parents=True)
     (root / "profiles").mkdir()
     (csrc / "gemm_tc.cu").write_text(src_text)
-    (csrc / "sbp_api.cu").write_text(f"constexpr int64_t kVocabBlock = {api_block};\n")
-    (root / "profiles" / "lmhead_ce_32k_gemm_tc.md").write_text(
-        f"dram_bytes_per_launch = {bytes_per_launch}\nkernel_source_sha256_16 = {stored_hash}\n")
+    (csrc / "sbp_api.cu").write_text(api_line)
+    (root / "profiles" / "traffic.json").write_text(json.dumps({"k@w": entry}))
     return str(root)
 
 
-def test_traffic_only_for_the_captured_kernel_and_block(tmp_path, monkeypatch):
+def test_traffic_only_for_the_captured_sources_and_shapes(tmp_path, monkeypatch):
     src = "// kernel\n"
-    good = hashlib.sha256(src.encode() + b"kVocabBlock=16384").hexdigest()[:16]
-    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "a", src, 16384, good))
-    assert bench.traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k") == 4.9e8
+    rel = "memory_efficient_exact_chunk_b200/csrc/gemm_tc.cu"
+    api = "memory_efficient_exact_chunk_b200/csrc/sbp_api.cu"
+    good = hashlib.sha256(src.encode()).hexdigest()[:16]
+    entry = {"sources": [rel], "sources_sha256_16": good, "dram_bytes_per_launch": 4.9e8,
+             "requires": [[api, "kVocabBlock = 16384;"]]}
+    line = "constexpr int64_t kVocabBlock = 16384;\n"
+    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "a", src, line, entry))
+    assert bench.traffic_from_profiles("k@w") == 4.9e8
+    assert bench.traffic_from_profiles("other@w") is None
     # another vocabulary block, or an edited kernel file: the stored figure no longer applies
-    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "b", src, 8192, good))
-    assert bench.traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k") is None
-    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "c", src + " ", 16384, good))
-    assert bench.traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k") is None
+    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "b", src, line.replace("16384", "8192"),
+                                             entry))
+    assert bench.traffic_from_profiles("k@w") is None
+    monkeypatch.setattr(bench, "ROOT", _tree(tmp_path / "c", src + " ", line, entry))
+    assert bench.traffic_from_profiles("k@w") is None
 
 
-def test_committed_traffic_matches_the_kernel_file():
-    """The committed profile was captured on the committed kernel file: after an edit of
-    gemm_tc.cu the DRAM-traffic capture in profiles/ has to be taken again (until then the
-    bench line reports traffic null)."""
-    assert bench.traffic_from_profiles("gemm_tc.cu", "lmhead_ce_32k") is not None
+def test_committed_traffic_entries_are_well_formed():
+    """Every entry of profiles/traffic.json names existing sources, a summary under profiles/
+    that exists, and a positive per-launch figure.  (Whether the sources still match is what
+    the bench checks at run time: a stale entry reports traffic null.)"""
+    path = os.path.join(bench.ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return
+    with open(path) as fh:
+        entries = json.load(fh)
+    for key, e in entries.items():
+        assert "@" in key
+        assert e["dram_bytes_per_launch"] > 0
+        assert os.path.exists(os.path.join(bench.ROOT, e["summary"])), key
+        for rel in e["sources"]:
+            assert os.path.exists(os.path.join(bench.ROOT, rel)), (key, rel)
 
 
 def test_parse_clocks_reasons_and_median():

@@ -22,7 +22,9 @@ def test_reference_arm_line():
     assert j["impl"] == "reference" and j["metric"] == bench.METRIC
     assert j["unit"] == "tokens/s" and j["higher_is_better"] is True and j["value"] > 0
     assert j["steps"] == 1 and j["warmup"] >= 3 and j["n_gpus"] == 1
-    assert j["config"]["workload"] == "lmhead_ce_32k"
+    assert j["config"]["workload"] == "llama3_8b_stack4_64k"
+    assert j["config"]["seq_len"] == 65536 and j["config"]["num_chunks"] == 16
+    assert j["config"]["n_loss_tokens"] == 49151
     assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     cb = j["cpu_baseline"]
