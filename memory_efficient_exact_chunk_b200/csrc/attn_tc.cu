@@ -1,18 +1,28 @@
 // Causal GQA attention forward of one query chunk over its key prefix on the tcgen05 tensor
 // cores (head_dim 128, bf16 operands, fp32 softmax statistics and accumulation).
 //
-// One CTA per (sequence b, query head h, 128-row query tile).  Warp roles:
-//   warp 0      : TMA producer (Q once; K and V tiles of 128 keys through 2-stage rings)
-//   warp 1      : TMEM owner + MMA issuer: S_j = Q K_j^T into one of two TMEM score buffers,
-//                 O += P_j V_j into the TMEM output accumulator
-//   warps 2..5  : softmax, one thread per query row: read S_j from TMEM, causal mask, online
-//                 max / sum in the exp2 domain, P_j (bf16) into shared memory in the layout the
-//                 next MMA reads, lazy rescale of O in TMEM, final O / l and log-sum-exp.
+// One CTA per (sequence b, query head h, pair of adjacent 128-row query tiles).  The two tiles
+// share every K / V tile the CTA loads and take turns on the tensor cores: while one tile's
+// softmax warps turn its scores into probabilities, the tensor cores run the other tile's
+// products, so neither the tensor pipe nor the exponential unit waits for the other.
+//   warp 0      : TMA producer (both Q tiles once; K and V tiles of 128 keys through 2-stage
+//                 rings, one load per key tile for both query tiles)
+//   warp 1      : TMEM owner + MMA issuer, in the order
+//                   S0_j S1_j | PV0_j S0_{j+1} PV1_j S1_{j+1} | PV0_{j+1} ...
+//                 S_t = Q_t K_j^T into tile t's score columns; PV_t: O_t += P_t V_j with P_t
+//                 read from TMEM (written by the softmax over the scores it replaces)
+//   warps 2..5  : softmax of tile 0, warps 6..9: softmax of tile 1, one thread per query row:
+//                 read S from TMEM, causal mask, online max / sum in the exp2 domain, P (bf16)
+//                 back into TMEM, lazy rescale of O in TMEM, final O / l and log-sum-exp.
 // The running maximum used as the exponent reference is only raised when the row maximum
 // exceeds it by more than 2^8 (P <= 256), so O is rescaled rarely; the result is exact up to
 // rounding because P, l and O share that reference.
-// Key tiles are visited in order 0, 1, ... up to the query tile's diagonal; masked entries are
-// exactly zero, so each query row's result does not depend on how the sequence was chunked.
+// Key tiles are visited in order 0, 1, ... up to each query tile's diagonal; masked entries
+// are exactly zero, so each query row's result does not depend on how the sequence was
+// chunked (or on which tile of a pair it sits in).
+// Ordering: S_t(j + 1) is issued after PV_t(j), whose P it overwrites; the tensor cores run a
+// CTA's MMAs in issue order, and the commit that signals S_t(j + 1) also covers PV_t(j), so a
+// softmax warp that has seen S_t(j + 1) may rescale O_t.
 #include <cuda.h>
 
 #include <mutex>
@@ -29,18 +39,19 @@ constexpr int BQ = 128, BKV = 128;      // query rows / keys per tile
 constexpr int TILE_BYTES = 128 * HD * 2;  // 32 KB: a 128 x 128 bf16 tile (two 64-wide chunks)
 constexpr int CHUNK_BYTES = TILE_BYTES / 2;
 constexpr int KV_STAGES = 2;
-constexpr int SMEM_BYTES = TILE_BYTES                 // Q
+constexpr int SMEM_BYTES = 2 * TILE_BYTES                // Q0, Q1
                            + 2 * KV_STAGES * TILE_BYTES  // K, V rings
-                           + TILE_BYTES                // P
                            + 1024;                     // alignment slack
-constexpr int kThreads = 192;
-constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O [256,384)
+constexpr int kSoftmaxWarps = 8;        // two warpgroups, one per query tile
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
+constexpr uint32_t TMEM_COLS = 512;     // S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512)
 constexpr uint32_t O_COL = 256;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 struct FwdArgs {
   int64_t B, T, Tc, s, H, Hkv;
   int nq;                 // query tiles per sequence
+  int np;                 // query-tile pairs per sequence
   void* o;                // [B*Tc, H, HD] bf16
   float* lse;             // [B*Tc, H]  natural log
   float scale_log2;       // log2(e) / sqrt(hd)
@@ -65,12 +76,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// generic-proxy shared-memory writes -> visible to the tensor cores (async proxy)
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -78,12 +94,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
-// Store 8 bf16 (16 bytes) of row r, 16-byte unit u (0..15 over 128 columns) of a 128 x 128
-// K-major tile with 128-byte swizzle (two 64-column chunks).
-__device__ __forceinline__ void st_tile_unit(uint8_t* tile, int r, int u, uint4 v) {
-  const int chunk = u >> 3, uu = u & 7;
-  uint8_t* p = tile + chunk * CHUNK_BYTES + r * 128 + ((uu ^ (r & 7)) << 4);
-  *reinterpret_cast<uint4*>(p) = v;
+// D[tmem] (+)= A[tmem] * B[smem], bf16 inputs, f32 accumulate (A: 128 lanes x K/2 columns of
+// packed bf16 pairs, K-major).
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -91,27 +111,34 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full, k_full[KV_STAGES], k_empty[KV_STAGES], v_full[KV_STAGES],
-      v_empty[KV_STAGES], s_full[2], s_empty[2], p_full, pv_done, drain_bar;
+      v_empty[KV_STAGES], s_full[2], p_full[2], o_done[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE_BYTES;
+  uint8_t* sQ = smem;                                  // tile t at sQ + t * TILE_BYTES
+  uint8_t* sK = sQ + 2 * TILE_BYTES;
   uint8_t* sV = sK + KV_STAGES * TILE_BYTES;
-  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
 
-  // heavy (late) query tiles first
-  const int qt = a.nq - 1 - (int)(blockIdx.x % a.nq);
-  const int64_t h = (blockIdx.x / a.nq) % a.H;
-  const int64_t b = blockIdx.x / (a.nq * a.H);
+  // heavy (late) query-tile pairs first
+  const int qp = a.np - 1 - (int)(blockIdx.x % a.np);
+  const int64_t h = (blockIdx.x / a.np) % a.H;
+  const int64_t b = blockIdx.x / (a.np * a.H);
   const int64_t g = h / (a.H / a.Hkv);
-  const int64_t q_lo = a.s + (int64_t)qt * BQ;                 // absolute position of row 0
-  const int64_t q_hi = a.s + imin((int64_t)(qt + 1) * BQ, a.Tc);  // one past the last valid row
-  const int nkv = (int)((q_hi + BKV - 1) / BKV);              // key tiles 0 .. nkv-1
+  const bool has1 = 2 * qp + 1 < a.nq;
+  int nkv_t[2];
+  int64_t q_lo_t[2], q_hi_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * qp + t;
+    q_lo_t[t] = a.s + (int64_t)qt * BQ;                            // position of row 0
+    q_hi_t[t] = a.s + imin((int64_t)(qt + 1) * BQ, a.Tc);          // one past the last row
+    nkv_t[t] = (t == 1 && !has1) ? 0 : (int)((q_hi_t[t] + BKV - 1) / BKV);
+  }
+  const int nkv = nkv_t[0] > nkv_t[1] ? nkv_t[0] : nkv_t[1];     // key tiles 0 .. nkv-1
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
@@ -121,12 +148,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::mbar_init(&v_full[i], 1);
       tc::mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&s_full[i], 1);
-      tc::mbar_init(&s_empty[i], 4);
+    for (int t = 0; t < 2; ++t) {
+      tc::mbar_init(&s_full[t], 1);
+      tc::mbar_init(&p_full[t], kSoftmaxWarps / 2);
+      tc::mbar_init(&o_done[t], 1);
     }
-    tc::mbar_init(&p_full, 4);
-    tc::mbar_init(&pv_done, 1);
     tc::mbar_init(&drain_bar, 1);
     abort_sh = 0;
     tc::fence_barrier_init();
@@ -144,10 +170,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       bool ok = true;
-      const int32_t qrow = (int32_t)(b * a.Tc + (int64_t)qt * BQ);
-      tc::mbar_expect_tx(&q_full, TILE_BYTES);
-      tc::tma_load_3d(sQ, &tmQ, &q_full, 0, (int32_t)h, qrow);
-      tc::tma_load_3d(sQ + CHUNK_BYTES, &tmQ, &q_full, 64, (int32_t)h, qrow);
+      const int32_t qrow = (int32_t)(b * a.Tc + (int64_t)(2 * qp) * BQ);
+      tc::mbar_expect_tx(&q_full, (has1 ? 2 : 1) * TILE_BYTES);
+      for (int t = 0; t < (has1 ? 2 : 1); ++t) {
+        tc::tma_load_3d(sQ + t * TILE_BYTES, &tmQ, &q_full, 0, (int32_t)h, qrow + t * BQ);
+        tc::tma_load_3d(sQ + t * TILE_BYTES + CHUNK_BYTES, &tmQ, &q_full, 64, (int32_t)h,
+                        qrow + t * BQ);
+      }
       uint32_t issued = 0;
       for (int j = 0; j < nkv && ok; ++j) {
         const int st = j % KV_STAGES;
@@ -182,55 +211,86 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // ---------------------------------------------------------------- MMA issuer
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T: both K-major
       const uint32_t id_o = tc::idesc_bf16_f32(128, 128, 0, 1);   // P V: V is MN-major
-      const uint32_t aQ = tc::smem_u32(sQ), aK = tc::smem_u32(sK), aV = tc::smem_u32(sV),
-                     aP = tc::smem_u32(sP);
+      const uint32_t aQ = tc::smem_u32(sQ), aK = tc::smem_u32(sK), aV = tc::smem_u32(sV);
+      // shared-memory descriptors built once; a k-step, a query tile or a ring stage adds its
+      // byte offset / 16 to the start address field (the tiles sit below 256 KB)
+      static_assert(KV_STAGES == 2, "stage descriptors are selected between two stages");
+      const uint64_t dQ0 = tc::smem_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = tc::smem_desc_sw128(aK, 16, 1024);
+      const uint64_t dV0 = tc::smem_desc_sw128(aV, CHUNK_BYTES, 1024);
+      constexpr uint64_t kTile = (uint64_t)(TILE_BYTES >> 4);
       bool ok = tc::mbar_wait(&q_full, 0, abort_flag);
       bool issued = false;
-      // shared-memory descriptors built once; a k-step or a ring stage adds its byte offset / 16
-      // to the start address field (the tiles sit below 256 KB, so the field cannot carry over)
-      static_assert(KV_STAGES == 2, "stage descriptors are selected between two stages");
-      const uint64_t dQ = tc::smem_desc_sw128(aQ, 16, 1024);
-      const uint64_t dK0 = tc::smem_desc_sw128(aK, 16, 1024);
-      const uint64_t dP = tc::smem_desc_sw128(aP, 16, 1024);
-      const uint64_t dV0 = tc::smem_desc_sw128(aV, CHUNK_BYTES, 1024);
-      constexpr uint64_t kStage = (uint64_t)(TILE_BYTES >> 4);
-      auto do_pv = [&](int jj) -> bool {
-        const int st = jj % KV_STAGES;
-        const uint32_t ph = (uint32_t)(jj / KV_STAGES) & 1u;
-        if (!tc::mbar_wait(&p_full, (uint32_t)jj & 1u, abort_flag)) return false;
-        if (!tc::mbar_wait(&v_full[st], ph, abort_flag)) return false;
+      int k_waited = -1;                 // last key tile whose K load this thread has seen
+      auto wait_k = [&](int j) -> bool {
+        if (k_waited >= j) return true;
+        if (!tc::mbar_wait(&k_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, abort_flag))
+          return false;
         tc::fence_after_sync();
-        const uint64_t vb = dV0 + (st ? kStage : 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = dP + (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
-          const uint64_t bd = vb + (uint64_t)((kk * 2048) >> 4);
-          tc::mma_f16_ss(tmem + O_COL, ad, bd, id_o, (jj | kk) != 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&pv_done);
-        tc::mma_commit(&v_empty[st]);
+        k_waited = j;
         return true;
       };
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % KV_STAGES;
-        const uint32_t ph = (uint32_t)(j / KV_STAGES) & 1u;
-        const int sb = j & 1;
-        const uint32_t sph = (uint32_t)(j >> 1) & 1u;
-        if (!tc::mbar_wait(&k_full[st], ph, abort_flag)) { ok = false; break; }
-        if (!tc::mbar_wait(&s_empty[sb], sph ^ 1u, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-        const uint64_t kb = dK0 + (st ? kStage : 0);
+      // S_t(j) = Q_t K_j^T
+      auto scores = [&](int t, int j) {
+        const uint64_t kb = dK0 + ((j % KV_STAGES) ? kTile : 0);
+        const uint64_t qb = dQ0 + (t ? kTile : 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + (uint32_t)(sb * 128), dQ + off, kb + off, id_s, kk != 0 ? 1u : 0u);
+          tc::mma_f16_ss(tmem + (uint32_t)(t * 128), qb + off, kb + off, id_s, kk != 0 ? 1u : 0u);
         }
+        tc::mma_commit(&s_full[t]);
         issued = true;
-        tc::mma_commit(&s_full[sb]);
-        tc::mma_commit(&k_empty[st]);
-        if (j >= 1 && !do_pv(j - 1)) { ok = false; break; }
+      };
+      // O_t += P_t(j) V_j; P_t packed two keys per column over S_t's first 64 columns
+      auto pv = [&](int t, int j) -> bool {
+        if (!tc::mbar_wait(&p_full[t], (uint32_t)j & 1u, abort_flag)) return false;
+        tc::fence_after_sync();
+        const uint64_t vb = dV0 + ((j % KV_STAGES) ? kTile : 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ts(tmem + O_COL + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kk),
+                     vb + (uint64_t)((kk * 2048) >> 4), id_o, (j | kk) != 0 ? 1u : 0u);
+        if (j == (t ? nkv_t[1] : nkv_t[0]) - 1) tc::mma_commit(&o_done[t]);
+        return true;
+      };
+      if (ok && nkv > 0) {
+        ok = wait_k(0);
+        if (ok) {
+          if (nkv_t[0] > 0) scores(0, 0);
+          if (nkv_t[1] > 0) scores(1, 0);
+          tc::mma_commit(&k_empty[0]);
+        }
       }
-      if (ok && nkv >= 1) ok = do_pv(nkv - 1);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j % KV_STAGES;
+        if (!tc::mbar_wait(&v_full[st], (uint32_t)(j / KV_STAGES) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const bool more = j + 1 < nkv;
+        if (j < nkv_t[0]) {
+          if (!pv(0, j)) { ok = false; break; }
+        }
+        if (j + 1 < nkv_t[0]) {
+          if (!wait_k(j + 1)) { ok = false; break; }
+          scores(0, j + 1);
+        }
+        if (j < nkv_t[1]) {
+          if (!pv(1, j)) { ok = false; break; }
+        }
+        tc::mma_commit(&v_empty[st]);
+        if (j + 1 < nkv_t[1]) {
+          if (!wait_k(j + 1)) { ok = false; break; }
+          scores(1, j + 1);
+        }
+        if (more) {
+          // every product that reads K_{j+1} is issued (a tile past its diagonal reads none)
+          if (!wait_k(j + 1)) { ok = false; break; }
+          tc::mma_commit(&k_empty[(j + 1) % KV_STAGES]);
+        }
+      }
       if (issued) {
         tc::mma_commit(&drain_bar);
         const uint64_t t0 = tc::globaltimer_ns();
@@ -239,35 +299,35 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const int q4 = warp & 3;
+    const int t = (warp - 2) >> 2;                // query tile of this warpgroup
+    const int q4 = warp & 3;                      // TMEM lane quarter
     const int r = q4 * 32 + lane;                 // query row within the tile
-    const int64_t t = q_lo + r;                   // absolute position
+    const int64_t q_lo = t ? q_lo_t[1] : q_lo_t[0], q_hi = t ? q_hi_t[1] : q_hi_t[0];
+    const int64_t tq = q_lo + r;                  // absolute position
+    const int n_kv = t ? nkv_t[1] : nkv_t[0];
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t s_col = (uint32_t)(t * 128), o_col = O_COL + (uint32_t)(t * 128);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!tc::mbar_wait_warp(&s_full[sb], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
+    for (int j = 0; j < n_kv; ++j) {
+      if (!tc::mbar_wait_warp(&s_full[t], (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
-        tc::tmem_ld32(tmem + lane_off + (uint32_t)(sb * 128 + c * 32), rr);
+        tc::tmem_ld32(tmem + lane_off + s_col + (uint32_t)(c * 32), rr);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(rr[i]);
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&s_empty[sb]);
       // scale into the exp2 domain; only tiles that reach past the first query need the
       // causal mask
       const int64_t k0 = (int64_t)j * BKV;
       const bool diag = k0 + BKV - 1 > q_lo;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (diag) {
-        const int lim = (int)(t - k0);             // keys k0 + i with i > lim are masked
+        const int lim = (int)(tq - k0);            // keys k0 + i with i > lim are masked
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           const float x = (i <= lim) ? sv[i] * a.scale_log2 : -INFINITY;
@@ -286,63 +346,57 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       float corr = 1.f;
       bool rescale = false;
       if (mx > m_ref + kRescaleThreshold) {
-        const float mn = mx;
-        corr = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mn);
+        corr = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
         rescale = (j > 0);
-        m_ref = mn;
+        m_ref = mx;
         l *= corr;
       }
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = fast_exp2(sv[2 * i] - m_ref);
-        const float p1 = fast_exp2(sv[2 * i + 1] - m_ref);
-        s4[i & 3] += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(sv[32 * c + 2 * i] - m_ref);
+          const float p1 = fast_exp2(sv[32 * c + 2 * i + 1] - m_ref);
+          s4[i & 3] += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        // P over the first 64 score columns (already read into registers)
+        tmem_st16(tmem + lane_off + s_col + (uint32_t)(c * 16), pk);
       }
-      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      l += sum;
-      // P_j may overwrite P_{j-1} (and O may be rescaled) once O += P_{j-1} V_{j-1} is done
-      if (j >= 1) {
-        if (!tc::mbar_wait_warp(&pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-      }
-      // warp-uniform decision: any lane that needs a rescale makes the warp do it
+      // O_t += P(j - 1) V(j - 1) has completed (the commit that announced S(j) covers it), so
+      // O may be rescaled before P(j) is announced; any lane that needs it makes the warp do it
       if (__any_sync(0xffffffffu, rescale)) {
         const float f = rescale ? corr : 1.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t rr[32];
-          const uint32_t ta = tmem + lane_off + O_COL + (uint32_t)(c * 32);
+          const uint32_t ta = tmem + lane_off + o_col + (uint32_t)(c * 32);
           tc::tmem_ld32(ta, rr);
           tc::tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
           tmem_st32(ta, rr);
         }
-        tmem_st_wait();
       }
-#pragma unroll
-      for (int u = 0; u < 16; ++u)
-        st_tile_unit(sP, r, u, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
-      fence_proxy_async_smem();
+      l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&p_full);
+      if (lane == 0) tc::mbar_arrive(&p_full[t]);
     }
-    // final: wait for the last O += P V, normalise, store
-    if (ok && nkv >= 1 &&
-        tc::mbar_wait_warp(&pv_done, (uint32_t)(nkv - 1) & 1u, abort_flag)) {
+    // final: wait for the tile's last O += P V, normalise, store
+    if (ok && n_kv >= 1 && tc::mbar_wait_warp(&o_done[t], 0, abort_flag)) {
       tc::fence_after_sync();
-      const bool row_ok = t < q_hi;
+      const bool row_ok = tq < q_hi;
       const float inv = 1.f / l;
-      const int64_t grow = b * a.Tc + (t - a.s);
+      const int64_t grow = b * a.Tc + (tq - a.s);
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(a.o) + (grow * a.H + h) * HD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
-        tc::tmem_ld32(tmem + lane_off + O_COL + (uint32_t)(c * 32), rr);
+        tc::tmem_ld32(tmem + lane_off + o_col + (uint32_t)(c * 32), rr);
         tc::tmem_ld_wait();
         if (row_ok) {
 #pragma unroll
@@ -428,11 +482,12 @@ cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   FwdArgs a;
   a.B = B; a.T = T; a.Tc = Tc; a.s = s; a.H = H; a.Hkv = Hkv;
   a.nq = (int)((Tc + BQ - 1) / BQ);
+  a.np = (a.nq + 1) / 2;
   a.o = o;
   a.lse = lse;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.err = err;
-  const int64_t grid = B * H * a.nq;
+  const int64_t grid = B * H * a.np;
   launch(attn_fwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)SMEM_BYTES, st, mq, mk,
          mv, a);
   return cudaGetLastError();
