@@ -795,7 +795,8 @@ def maxlen_main(args, rank, world, device):
     free0, total = torch.cuda.mem_get_info(device)
     budget = free0 - (1 << 30)          # 1 GiB for torch's allocator slack and the kernels' own
     model = {D: MM.max_tokens(shape, D, budget) for D in (1, 2, 4, 8, 16, 32)}
-    T = args.stack_tokens or model[args.chunks or 1]
+    # by default 97 % of the model's longest sequence at this D (a margin for the allocator)
+    T = args.stack_tokens or int(0.97 * model[args.chunks or 1])
     T = T // 128 * 128
     D = args.chunks or 1
     L = wl.layer
@@ -842,6 +843,7 @@ def maxlen_main(args, rank, world, device):
         total / 1e9, "budget_gb": budget / 1e9,
         "model_max_tokens": {str(k): v for k, v in model.items()},
         "run": {"seq_len": T, "num_chunks": D, "measured_peak_gb": peak / 1e9,
+                "fraction_of_model_max": T / max(model.get(D, 0), 1) if D in model else None,
                 "model_gb": pred["total"] / 1e9,
                 "model_parts_gb": {k: v / 1e9 for k, v in pred.items()},
                 "forward_ms": e0.elapsed_time(e1), "backward_ms": e1.elapsed_time(e2),

@@ -6,8 +6,8 @@ Each .cu under csrc/ is compiled to an object in _build/ (in parallel) and linke
 memory_efficient_exact_chunk_b200/libsbp.so with the CUDA runtime linked statically, so the
 library loads on a machine without a GPU (symbols can be listed, nothing is launched).
 `--timing` builds a separate instrumented library, libsbp_timing.so (objects in
-_build_timing/), whose pair GEMM and attention dK/dV kernel print per-launch cycle accounts
-(SBP_GEMM_TIMING, SBP_ATTN_TIMING); the product library is not touched.
+_build_timing/), whose pair GEMM prints per-launch cycle accounts (SBP_GEMM_TIMING); the
+product library is not touched.
 """
 from __future__ import annotations
 
@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     srcs = _sources()
     lib_path, build_dir = (LIB_TIMING, BUILD_TIMING) if timing else (LIB, BUILD)
     if timing:
-        extra = (extra or []) + ["-DSBP_GEMM_TIMING", "-DSBP_ATTN_TIMING"]
+        extra = (extra or []) + ["-DSBP_GEMM_TIMING"]
     if not force and os.path.exists(lib_path) and os.path.getmtime(lib_path) >= _deps_mtime():
         return lib_path
     os.makedirs(build_dir, exist_ok=True)

@@ -1,5 +1,5 @@
-"""Cycle accounting of the pair GEMM and of the attention dK/dV kernel, from the instrumented
-library (libsbp_timing.so, built with SBP_GEMM_TIMING and SBP_ATTN_TIMING).
+"""Cycle accounting of the pair GEMM from the instrumented library (libsbp_timing.so, built
+with SBP_GEMM_TIMING).
 
     python -m memory_efficient_exact_chunk_b200.build --timing
     python -m memory_efficient_exact_chunk_b200.timing lmhead > lmhead_timing.log
@@ -11,10 +11,11 @@ library (libsbp_timing.so, built with SBP_GEMM_TIMING and SBP_ATTN_TIMING).
 pair-GEMM launch prints, for CTA 0 (and CTA 1 for the producer): the producer's cycles waiting
 for a free ring stage, the MMA issuer's cycles waiting for operands (full stage) and for a free
 accumulator, and two epilogue warps' cycles waiting for a full accumulator and working.
-`layer` runs the Llama-3-8B-shaped layer backward twice (16384 tokens, D = 2); the dK/dV
-kernel's CTA 0 prints its producer's, MMA issuer's and two element-wise warps' accounts (and
-the layer's GEMMs print theirs).  `summarize` keeps the second call (warm) of each kind and
-averages per launch shape.  Measurement only: the product library is not involved.
+`layer` runs the Llama-3-8B-shaped layer backward twice (16384 tokens, D = 2); the layer's
+GEMMs print their accounts.  (The summary also reads the records of an attention dK/dV kernel
+that prints "SBPT KV..." lines; the current attention kernels print none.)  `summarize` keeps
+the second call (warm) of each kind and averages per launch shape.  Measurement only: the
+product library is not involved.
 """
 from __future__ import annotations
 
