@@ -1,51 +1,44 @@
 // Causal GQA attention backward of one query chunk over its key prefix on the tcgen05 tensor
 // cores (head_dim 128, bf16 operands, fp32 accumulation), as two kernels that each keep their
 // accumulator in TMEM and write it once (no atomics; both results are deterministic and do not
-// depend on how the sequence was chunked):
+// depend on how the sequence was chunked).
 //
-// dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile) and loops over the query
-// heads of g's group and the chunk's query tiles that can see those keys.  Each (head, query
-// tile) pair is taken as two halves of 64 queries; per half h:
-//   S^T_h  = K Q_h^T   (TMEM c_s(h), 64 columns)     dP^T_h = V dO_h^T  (TMEM c_dp(h))
-//   P^T_h  = exp(S^T_h * scale - lse) -> bf16, written back into TMEM over the dP^T_h columns
-//            the same warp has already read (the A operand of the dV product)
-//   dS^T_h = P^T_h (dP^T_h - delta)    -> bf16, shared-memory buffer h
-//   dV    += P^T_h dO_h (TMEM [256,384))            dK += dS^T_h Q_h (TMEM [384,512))
-// The two halves have their own TMEM columns and dS^T buffers, so the tensor cores compute the
-// scores of one half (and the dV / dK products of the other) while the element-wise warps
-// turn the scores of a half into P^T and dS^T.
+// Every product reads its A operand from TMEM (the tcgen05.mma form with A in tensor memory)
+// and only its B operand from shared memory: measured on B200, an M = 128, N = 128, K = 16
+// instruction then takes about 74 cycles against about 126 with both operands in shared
+// memory (64 at the nominal rate), and N = 64 instructions are no faster than N = 128 ones.
+// So the tile a CTA owns is copied into TMEM once (packed bf16 pairs), scores are computed
+// 128 x 128 at a time, and P^T / dS^T (or dS) are written back into TMEM as packed bf16 over
+// the scores they are computed from.
+//
+// dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile); K and V live in TMEM.  It
+// loops over the query heads of g's group and the chunk's query tiles that can see those
+// keys; per (head, query tile) pair, with one 128-column score region SP:
+//   S^T  = K Q^T                  -> SP   (the element-wise warps read it out)
+//   dP^T = V dO^T                 -> SP   (while the warps compute P^T = exp(S^T - lse))
+//   P^T, dS^T = P^T (dP^T - delta) -> SP as packed bf16 (each warp over its own columns)
+//   dV += P^T dO,  dK += dS^T Q   (A = P^T, dS^T from TMEM; B = dO, Q from shared memory)
 // The query tiles are taken in blocks of a fixed number of tiles counted from the chunk start
 // (all heads of the group within a block); after each block dK, dV are added into the fp32
 // prefix accumulators (single owner, no atomics).  A chunk whose length is a multiple of the
 // block therefore adds exactly the partial sums the same queries give inside a longer chunk.
 //
-// dQ kernel: one CTA owns (sequence b, query head h, 128-query tile) and loops over the key
-// tiles of its causal prefix, each as two halves of 64 keys:  S_h = Q K_h^T, dP_h = dO V_h^T,
-// dS_h = P_h (dP_h - delta) -> shared-memory buffer h, dQ += dS_h K_h (TMEM), stored once at
-// the end; the halves are pipelined the same way.
+// dQ kernel: one CTA owns (sequence b, query head h, 128-query tile); Q and dO live in TMEM.
+// It loops over the key tiles of its causal prefix with two score regions used alternately,
+// so the tensor cores compute the scores of key tile j + 1 while the element-wise warps work
+// on tile j:  S = Q K^T, dP = dO V^T, dS = P (dP - delta) -> packed bf16 over S / dP,
+// dQ += dS K (TMEM), stored once at the end.
 //
 // Entries with key > query, queries outside the chunk and keys outside the prefix are masked
 // by selection (not by multiplication), so stale values never reach an accumulator.
 // Warp roles (both kernels): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..9
 // element-wise (the warp's TMEM lane quarter is its index mod 4; the two warps of a quarter
-// split the 64 columns of a half).
+// split the 128 columns of a score tile into halves of 64).
 #include <cuda.h>
 
 #include <mutex>
 
 #include "sbp_internal.cuh"
-
-// Cycle accounting of the dK/dV kernel, compiled in only with -DSBP_ATTN_TIMING (the build's
-// --timing library): CTA 0 prints, per launch, the producer's cycles waiting for a free Q/dO
-// stage, the MMA issuer's cycles waiting for dS / Q,dO / the accumulator flush and issuing,
-// and two element-wise warps' cycles waiting for Q,dO and for the scores, working, and
-// flushing.  Off by default: no cost.
-#ifdef SBP_ATTN_TIMING
-#include <cstdio>
-#define SBP_ATTN_TIMED(...) __VA_ARGS__
-#else
-#define SBP_ATTN_TIMED(...)
-#endif
 #include "tc_ptx.cuh"
 
 namespace sbp {
@@ -56,36 +49,43 @@ constexpr int HD = 128;
 constexpr int BT = 128;                     // keys per key tile, queries per query tile
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
-constexpr int QD_STAGES = 2;
+constexpr int QD_STAGES = 2;                // Q/dO stages of the dK/dV kernel
+constexpr int KV_RING = 2;                  // K/V stages of the dQ kernel
 // All shared state lives in the dynamic allocation (no static shared memory), whose start is
 // 1024-byte aligned as the 128-byte swizzle needs: the tiles first, then the statistics and
 // the barriers.
 struct KvShared {
-  float stat[2 /*QD_STAGES*/][2][BT];   // per stage: lse (log2 units), delta
-  uint64_t kv_full, qd_full[2], qd_empty[2], sdp_full[2], ds_full[2], kv_free, drain;
+  float stat[QD_STAGES][2][BT];   // per stage: lse (log2 units), delta of the pair's queries
+  uint64_t kv_full, kv_tmem, qd_full[QD_STAGES], qd_empty[QD_STAGES], s_full, s_read, dp_full,
+      ds_full, kv_free, drain;
   uint32_t tmem;
   int abort;
 };
-constexpr int KV_TILES_BYTES = (3 + 2 * QD_STAGES) * TILE;        // K, V, dS^T, 2 x (Q, dO)
+constexpr int KV_TILES_BYTES = (2 + 2 * QD_STAGES) * TILE;        // K, V, 2 x (Q, dO)
 constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
-constexpr int KV_RING = 2;                                         // K/V stages of the dQ kernel
 struct QShared {
-  uint64_t qd_full, kv_full[KV_RING], kv_empty[KV_RING], sdp_full[2], ds_full[2], dq_done, drain;
+  uint64_t qd_full, q_tmem, kv_full[KV_RING], kv_empty[KV_RING], s_full[2], s_read[2],
+      dp_full[2], ds_full[2], dq_done, drain;
   uint32_t tmem;
   int abort;
 };
-constexpr int Q_TILES_BYTES = (3 + 2 * KV_RING) * TILE;           // Q, dO, dS, 2 x (K, V)
+constexpr int Q_TILES_BYTES = (2 + 2 * KV_RING) * TILE;           // Q, dO, 2 x (K, V)
 constexpr int Q_SMEM_BYTES = Q_TILES_BYTES + (int)sizeof(QShared);
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns: half h of a tile keeps its scores at c_s(h) and their gradient at c_dp(h)
-// (64 columns each); the fp32 accumulators dV, dK (key-tile kernel) or dQ (query-tile kernel)
-// take the upper columns.
-constexpr uint32_t C_DV = 256, C_DK = 384, C_DQ = 256;
-__device__ __forceinline__ uint32_t c_s(int h) { return 128u * (uint32_t)h; }
-__device__ __forceinline__ uint32_t c_dp(int h) { return 128u * (uint32_t)h + 64u; }
-constexpr int HALF = TILE / 4;              // 64 rows x 128 bytes: a 64-row slice of a chunk
+// TMEM columns.  dK/dV kernel: K and V (packed bf16, 64 columns each), the score region SP,
+// the fp32 accumulators dV and dK.  dQ kernel: Q and dO (packed), two score regions, dQ.
+constexpr uint32_t KV_KT = 0, KV_VT = 64, KV_SP = 128, KV_DV = 256, KV_DK = 384;
+constexpr uint32_t Q_QT = 0, Q_OT = 64, Q_SP0 = 128, Q_DQ = 384;
+__device__ __forceinline__ uint32_t q_sp(int x) { return Q_SP0 + 128u * (uint32_t)x; }
+// Packed-bf16 A operand written back over a score region: the warps of column half wh own
+// score columns [64 wh, 64 wh + 64) and put their packed values at the start of that range
+// (P^T at +0, dS^T at +32 in the dK/dV kernel; dS at +0 in the dQ kernel).  The k-step kk of
+// a K = 128 product (16 rows of K each) therefore starts at column 64 (kk / 4) + 8 (kk % 4).
+__device__ __forceinline__ uint32_t packed_col(int kk) {
+  return 64u * (uint32_t)(kk >> 2) + 8u * (uint32_t)(kk & 3);
+}
 
 struct BwdArgs {
   int64_t B, T, Tc, s, H, Hkv;
@@ -105,10 +105,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
 }
-__device__ __forceinline__ void st_unit(uint8_t* tile, int r, int u, uint4 v) {
-  const int chunk = u >> 3, uu = u & 7;
-  *reinterpret_cast<uint4*>(tile + chunk * CHUNK + r * 128 + ((uu ^ (r & 7)) << 4)) = v;
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -118,10 +114,22 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, f32 accumulate (A: 128 lanes x K/2 columns of
+// D[tmem] (+)= A[tmem] * B[smem], bf16 inputs, f32 accumulate (A: 128 lanes x K/2 columns of
 // packed bf16 pairs, K-major).
 __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
                                            uint32_t idesc, uint32_t accumulate) {
@@ -140,9 +148,24 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// Copy this thread's row r of a 128 x 128 bf16 tile staged by TMA (two 64-column chunks, each
+// 128 rows of 128 bytes with the 128-byte swizzle) into TMEM as packed bf16 pairs: chunk c
+// (columns 64 c ..) goes to TMEM columns col0 + 32 c ..; the caller's warp owns the lane.
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int r, int c,
+                                                 uint32_t taddr) {
+  uint32_t w[32];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + c * CHUNK + r * 128 +
+                                                    ((u ^ (r & 7)) << 4));
+    w[4 * u] = v.x;
+    w[4 * u + 1] = v.y;
+    w[4 * u + 2] = v.z;
+    w[4 * u + 3] = v.w;
+  }
+  tmem_st32(taddr, w);
 }
+
 // ================================================================== dK / dV kernel
 // The work of a key tile, pair by pair: (query head hh of the group, query tile qi) for the
 // query tiles i0 .. nq - 1, ordered block by block (qb tiles, counted from the chunk start)
@@ -192,8 +215,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   KvShared& sh = *reinterpret_cast<KvShared*>(smem_raw + KV_TILES_BYTES);
   uint8_t* sK = smem_raw;
   uint8_t* sV = sK + TILE;
-  uint8_t* sdSt = sV + TILE;                     // half h: dS^T [128 keys x 64 queries] at h*CHUNK
-  uint8_t* sQ0 = sdSt + TILE;                    // stage st: Q at sQ0 + 2 st TILE, dO after it
+  uint8_t* sQ0 = sV + TILE;                      // stage st: Q at sQ0 + 2 st TILE, dO after it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
 
@@ -213,14 +235,15 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&sh.kv_full, 1);
+    tc::mbar_init(&sh.kv_tmem, kEwWarps);
     for (int i = 0; i < QD_STAGES; ++i) {
       tc::mbar_init(&sh.qd_full[i], 1);
       tc::mbar_init(&sh.qd_empty[i], 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      tc::mbar_init(&sh.sdp_full[h], 1);
-      tc::mbar_init(&sh.ds_full[h], kEwWarps);
-    }
+    tc::mbar_init(&sh.s_full, 1);
+    tc::mbar_init(&sh.s_read, kEwWarps);
+    tc::mbar_init(&sh.dp_full, 1);
+    tc::mbar_init(&sh.ds_full, kEwWarps);
     tc::mbar_init(&sh.kv_free, kEwWarps);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -246,16 +269,13 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full, 64, (int32_t)g, krow);
       bool ok = true;
       int issued = 0;
-      SBP_ATTN_TIMED(long long w_empty = 0, tp0 = clock64(), c0;)
       PairIter it;
       it.init((int)i0, a.nq, (int)grp, a.qb);
       for (int j = 0; j < npairs; ++j, it.next()) {
         const PairPos pos = it.pos(g);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
-        SBP_ATTN_TIMED(c0 = clock64();)
         if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
-        SBP_ATTN_TIMED(w_empty += clock64() - c0;)
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
@@ -269,9 +289,6 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
         issued = j + 1;
       }
-      SBP_ATTN_TIMED(if (blockIdx.x == 0) printf(
-          "SBPT KVPROD s %lld Tc %lld pairs %d total %lld w_empty %lld\n", (long long)a.s,
-          (long long)a.Tc, npairs, clock64() - tp0, w_empty);)
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
@@ -283,111 +300,67 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 1) {
     if (lane == 0 && npairs > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      // Two 64-query halves per pair, each with its own S^T / dP^T columns and dS^T buffer,
-      // so the scores of one half are computed while the element-wise warps work on the other.
-      const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);     // S^T, dP^T: N = 64 queries
+      const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: B K-major
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dV, dK: B MN-major
-      const uint32_t aK = tc::smem_u32(sK), aV = tc::smem_u32(sV), adS = tc::smem_u32(sdSt),
-                     aQ0 = tc::smem_u32(sQ0);
-      bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag);
-      bool issued = false;
-      // Shared-memory descriptors built once; a k-step adds its byte offset / 16 to the start
-      // address field (the tiles sit below 256 KB, so the field cannot carry over).  This keeps
-      // the single issuing thread fast enough for the 128 x 64 x 16 products.
-      const uint64_t dK = tc::smem_desc_sw128(aK, 16, 1024), dV = tc::smem_desc_sw128(aV, 16, 1024);
-      const uint64_t dS = tc::smem_desc_sw128(adS, 16, 1024);
-      // the two Q/dO stages differ by a constant: stage 1's start address field is stage 0's
-      // plus 2 TILE / 16 (selected, not indexed, so the descriptors stay in registers)
+      const uint32_t aQ0 = tc::smem_u32(sQ0);
+      // shared-memory descriptors built once; a k-step adds its byte offset / 16 to the start
+      // address field (the tiles sit below 256 KB, so the field cannot carry over)
       static_assert(QD_STAGES == 2, "stage descriptors are selected between two stages");
       const uint64_t dQk0 = tc::smem_desc_sw128(aQ0, 16, 1024);
       const uint64_t dOk0 = tc::smem_desc_sw128(aQ0 + TILE, 16, 1024);
       const uint64_t dQm0 = tc::smem_desc_sw128(aQ0, CHUNK, 1024);
       const uint64_t dOm0 = tc::smem_desc_sw128(aQ0 + TILE, CHUNK, 1024);
       constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
-      // S^T_h = K Q_h^T and dP^T_h = V dO_h^T of pair j's half h
-      auto scores = [&](int j, int h) {
-        const uint64_t so = (j & 1) ? kStage : 0;
-        const uint64_t bq = dQk0 + so + (uint64_t)((h * HALF) >> 4);
-        const uint64_t bo = dOk0 + so + (uint64_t)((h * HALF) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + c_s(h), dK + off, bq + off, id_s, kk != 0);
-          tc::mma_f16_ss(tmem + c_dp(h), dV + off, bo + off, id_s, kk != 0);
-        }
-        tc::mma_commit(&sh.sdp_full[h]);
-      };
-      // dV += P^T_h dO_h (P^T from TMEM), dK += dS^T_h Q_h; `first`: the block's first product
-      auto grads = [&](int j, int h, bool first) {
-        const uint64_t so = (j & 1) ? kStage : 0;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries of the half
-          const uint64_t offm = so + (uint64_t)(((4 * h + kk) * 2048) >> 4);  // MN-major k-step
-          const uint32_t acc = (!first || kk != 0) ? 1u : 0u;
-          // packed P^T of queries 32 w.. of half h sits at c_dp(h) + 32 w (w = column half)
-          const uint32_t pcol = c_dp(h) + 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_f16_ts(tmem + C_DV, tmem + pcol, dOm0 + offm, id_g, acc);
-          tc::mma_f16_ss(tmem + C_DK, dS + (uint64_t)((h * CHUNK + kk * 32) >> 4), dQm0 + offm,
-                         id_g, acc);
-        }
-      };
+      bool ok = tc::mbar_wait(&sh.kv_tmem, 0, abort_flag);      // K, V copied into TMEM
+      bool issued = false;
       int nflush = 0;
-      SBP_ATTN_TIMED(long long w_ds = 0, w_qd = 0, w_free = 0, t_iss = 0, ti0 = clock64(), c0;)
-      if (ok && tc::mbar_wait(&sh.qd_full[0], 0, abort_flag)) {
-        tc::fence_after_sync();
-        scores(0, 0);
-        scores(0, 1);
-        issued = true;
-      } else {
-        ok = false;
-      }
       PairIter it;
       it.init((int)i0, a.nq, (int)grp, a.qb);
       for (int j = 0; j < npairs && ok; ++j, it.next()) {
         const PairPos pos = it.pos(g);
+        const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)j & 1u;
-        SBP_ATTN_TIMED(c0 = clock64();)
-        if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
-        SBP_ATTN_TIMED(w_ds += clock64() - c0;)
-        // a new block overwrites dK / dV: the element-wise warps must have added the last one
+        const uint64_t so = st ? kStage : 0;
+        if (!tc::mbar_wait(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        // S^T = K Q^T (the previous pair's dV / dK products, issued before, have read SP)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
+          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          mma_f16_ts(tmem + KV_SP, tmem + KV_KT + 8 * kk, dQk0 + off, id_s, kk != 0);
+        }
+        tc::mma_commit(&sh.s_full);
+        issued = true;
+        // dP^T = V dO^T, over S^T once the element-wise warps have read it
+        if (!tc::mbar_wait(&sh.s_read, ph, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          mma_f16_ts(tmem + KV_SP, tmem + KV_VT + 8 * kk, dOk0 + off, id_s, kk != 0);
+        }
+        tc::mma_commit(&sh.dp_full);
+        // dV += P^T dO, dK += dS^T Q once P^T, dS^T are in TMEM; a new block overwrites dK / dV,
+        // so the element-wise warps must have added the last one
+        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
         if (pos.first && j > 0) {
-          SBP_ATTN_TIMED(c0 = clock64();)
           if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
-          SBP_ATTN_TIMED(w_free += clock64() - c0;)
           ++nflush;
         }
         tc::fence_after_sync();
-        SBP_ATTN_TIMED(c0 = clock64();)
-        grads(j, 0, pos.first);
-        SBP_ATTN_TIMED(t_iss += clock64() - c0;)
-        const bool more = j + 1 < npairs;
-        if (more) {
-          const int st1 = (j + 1) % QD_STAGES;
-          SBP_ATTN_TIMED(c0 = clock64();)
-          if (!tc::mbar_wait(&sh.qd_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          SBP_ATTN_TIMED(w_qd += clock64() - c0;)
-          tc::fence_after_sync();
-          SBP_ATTN_TIMED(c0 = clock64();)
-          scores(j + 1, 0);
-          SBP_ATTN_TIMED(t_iss += clock64() - c0;)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = 128 queries
+          const uint64_t offm = so + (uint64_t)((kk * 2048) >> 4);     // MN-major k-step
+          const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
+          const uint32_t pc = KV_SP + packed_col(kk);
+          mma_f16_ts(tmem + KV_DV, tmem + pc, dOm0 + offm, id_g, acc);
+          mma_f16_ts(tmem + KV_DK, tmem + pc + 32, dQm0 + offm, id_g, acc);
         }
-        SBP_ATTN_TIMED(c0 = clock64();)
-        if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
-        SBP_ATTN_TIMED(w_ds += clock64() - c0;)
-        tc::fence_after_sync();
-        SBP_ATTN_TIMED(c0 = clock64();)
-        grads(j, 1, false);
-        tc::mma_commit(&sh.qd_empty[j % QD_STAGES]);
-        if (more) scores(j + 1, 1);
-        SBP_ATTN_TIMED(t_iss += clock64() - c0;)
+        tc::mma_commit(&sh.qd_empty[st]);
       }
-      SBP_ATTN_TIMED(if (blockIdx.x == 0) printf(
-          "SBPT KVISSUE s %lld Tc %lld pairs %d total %lld w_ds %lld w_qd %lld w_free %lld "
-          "issue %lld\n", (long long)a.s, (long long)a.Tc, npairs, clock64() - ti0, w_ds, w_qd,
-          w_free, t_iss);)
       if (issued) {
         tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
@@ -397,16 +370,25 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (npairs > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
-    const int wh = (warp - 2) >> 2;                  // column half: queries 32 wh .. of a half
+    const int wh = (warp - 2) >> 2;                  // column half: queries 64 wh .. 64 wh + 63
     const int r = q4 * 32 + lane;                    // TMEM lane = key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t sp = tmem + lane_off + KV_SP + 64u * (uint32_t)wh;   // this warp's columns
     const int kpos = (int)(k_lo + r);
     const float scale_log2 = a.scale * 1.4426950408889634f;
     const int e32 = (int)e;
     const bool kv = kpos < e32;
     const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
-    bool ok = true;
-    SBP_ATTN_TIMED(long long w_q = 0, w_sdp = 0, t_work = 0, t_flush = 0, te0 = clock64(), c0;)
+    bool ok = tc::mbar_wait_warp(&sh.kv_full, 0, abort_flag);
+    if (ok) {
+      // K and V rows of this lane into TMEM (packed), this warp's 64-column half of each
+      tile_row_to_tmem(sK, r, wh, tmem + lane_off + KV_KT + 32u * (uint32_t)wh);
+      tile_row_to_tmem(sV, r, wh, tmem + lane_off + KV_VT + 32u * (uint32_t)wh);
+      tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.kv_tmem);
+    }
     PairIter it;
     it.init((int)i0, a.nq, (int)grp, a.qb);
     for (int j = 0; j < npairs && ok; ++j, it.next()) {
@@ -421,76 +403,86 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
       const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
-      // acquire the bulk copies of this stage (already complete once the scores are ready)
-      SBP_ATTN_TIMED(c0 = clock64();)
       if (!tc::mbar_wait_warp(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
         break;
       }
-      SBP_ATTN_TIMED(w_q += clock64() - c0;)
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int qoff = 64 * h + 32 * wh;             // this warp's queries within the tile
-        const int q0 = (int)(a.s + pos.qi * BT) + qoff;  // absolute position of its first query
-        // no masking needed when every key of the tile precedes every (valid) query here
-        const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 32 <= a.Tc);
-        const float* lse_s = sh.stat[st][0] + qoff;
-        const float* delta_s = sh.stat[st][1] + qoff;
-        SBP_ATTN_TIMED(c0 = clock64();)
-        if (!tc::mbar_wait_warp(&sh.sdp_full[h], ph, abort_flag)) { ok = false; break; }
-        SBP_ATTN_TIMED(w_sdp += clock64() - c0; c0 = clock64();)
-        tc::fence_after_sync();
-        uint32_t rs[32], rd[32];
-        tc::tmem_ld32(tmem + lane_off + c_s(h) + 32 * wh, rs);
-        tc::tmem_ld32(tmem + lane_off + c_dp(h) + 32 * wh, rd);
+      const int qoff = 64 * wh;                        // this warp's queries within the tile
+      const int q0 = (int)(a.s + pos.qi * BT) + qoff;  // absolute position of its first query
+      // no masking needed when every key of the tile precedes every (valid) query here
+      const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 64 <= a.Tc);
+      const float* lse_s = sh.stat[st][0] + qoff;
+      const float* delta_s = sh.stat[st][1] + qoff;
+      // S^T of this warp's 64 queries
+      if (!tc::mbar_wait_warp(&sh.s_full, ph, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      float p[64];
+      {
+        uint32_t rs[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tc::tmem_ld32(sp + 32u * (uint32_t)c, rs);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) p[32 * c + i] = __uint_as_float(rs[i]);
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.s_read);        // SP may take dP^T now
+      // P^T = exp(S^T * scale - lse) while the tensor cores compute dP^T
+#pragma unroll
+      for (int i4 = 0; i4 < 16; ++i4) {
+        const float4 lv = reinterpret_cast<const float4*>(lse_s)[i4];
+        const float la[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = i4 * 4 + k;
+          float x = ex2(fmaf(p[i], scale_log2, -la[k]));
+          if (!full) {
+            const int qpos = q0 + i;
+            x = ((kpos <= qpos) && (qpos < e32)) ? x : 0.f;
+          }
+          p[i] = x;
+        }
+      }
+      if (!tc::mbar_wait_warp(&sh.dp_full, ph, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      // dS^T = P^T (dP^T - delta); P^T and dS^T go back over this warp's own columns as packed
+      // bf16 (P^T at +0, dS^T at +32), each written only after the values it replaces are read
+      uint32_t dsw[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rd[32];
+        tc::tmem_ld32(sp + 32u * (uint32_t)c, rd);
         tc::tmem_ld_wait();
-        uint32_t pp[16], dd[16];
-        const float4* l4 = reinterpret_cast<const float4*>(lse_s);
-        const float4* d4 = reinterpret_cast<const float4*>(delta_s);
+        uint32_t pw[16];
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 lv = l4[i4], dv = d4[i4];
-          const float la[4] = {lv.x, lv.y, lv.z, lv.w};
+          const float4 dv = reinterpret_cast<const float4*>(delta_s)[8 * c + i4];
           const float da[4] = {dv.x, dv.y, dv.z, dv.w};
-          float p[4], gg[4];
+          float gg[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int i = i4 * 4 + k;
-            p[k] = ex2(fmaf(__uint_as_float(rs[i]), scale_log2, -la[k]));
-            gg[k] = p[k] * (__uint_as_float(rd[i]) - da[k]);
-            if (!full) {
-              const int qpos = q0 + i;
-              const bool live = (kpos <= qpos) && (qpos < e32);
-              p[k] = live ? p[k] : 0.f;
-              gg[k] = live ? gg[k] : 0.f;
-            }
+            const int i = 32 * c + i4 * 4 + k;
+            gg[k] = p[i] * (__uint_as_float(rd[i4 * 4 + k]) - da[k]);
           }
-          pp[i4 * 2] = pack2(p[0], p[1]);
-          pp[i4 * 2 + 1] = pack2(p[2], p[3]);
-          dd[i4 * 2] = pack2(gg[0], gg[1]);
-          dd[i4 * 2 + 1] = pack2(gg[2], gg[3]);
+          pw[2 * i4] = pack2(p[32 * c + 4 * i4], p[32 * c + 4 * i4 + 1]);
+          pw[2 * i4 + 1] = pack2(p[32 * c + 4 * i4 + 2], p[32 * c + 4 * i4 + 3]);
+          dsw[16 * c + 2 * i4] = pack2(gg[0], gg[1]);
+          dsw[16 * c + 2 * i4 + 1] = pack2(gg[2], gg[3]);
         }
-        // packed P^T over the dP^T columns this warp has just read
-        tmem_st16(tmem + lane_off + c_dp(h) + 32 * wh, pp);
-        // dS^T of this half (the previous pair's dK product of this half has read the buffer:
-        // its completion precedes the scores this warp has waited for)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_unit(sdSt + h * CHUNK, r, 4 * wh + u,
-                  make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
-        tmem_st_wait();
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sh.ds_full[h]);
-        SBP_ATTN_TIMED(t_work += clock64() - c0;)
+        tmem_st16(sp + 16u * (uint32_t)c, pw);          // over dP^T columns already read
       }
-      if (!ok || !pos.last) continue;
-      SBP_ATTN_TIMED(c0 = clock64();)
-      // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner)
-      // the release of this pair's Q/dO stage is committed after its last dK / dV product
-      if (!tc::mbar_wait_warp(&sh.qd_empty[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u,
-                              abort_flag)) {
+      tmem_st32(sp + 32u, dsw);                         // over the second half, now read too
+      tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
+      if (!pos.last) continue;
+      // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner); the
+      // release of this pair's Q/dO stage is committed after its last dK / dV product
+      if (!tc::mbar_wait_warp(&sh.qd_empty[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -499,8 +491,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int cc = 0; cc < 2; ++cc) {
         const int c = wh * 2 + cc;
         uint32_t rk[32], rv[32];
-        tc::tmem_ld32(tmem + lane_off + C_DK + c * 32, rk);
-        tc::tmem_ld32(tmem + lane_off + C_DV + c * 32, rv);
+        tc::tmem_ld32(tmem + lane_off + KV_DK + c * 32, rk);
+        tc::tmem_ld32(tmem + lane_off + KV_DV + c * 32, rv);
         tc::tmem_ld_wait();
         if (kv) {
           // all loads first (one memory latency), then the adds and the stores
@@ -533,12 +525,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0 && j + 1 < npairs) tc::mbar_arrive(&sh.kv_free);
-      SBP_ATTN_TIMED(t_flush += clock64() - c0;)
     }
-    SBP_ATTN_TIMED(if (blockIdx.x == 0 && (warp == 2 || warp == 9) && lane == 0) printf(
-        "SBPT KVEW warp %d s %lld Tc %lld pairs %d total %lld w_qd %lld w_sdp %lld work %lld "
-        "flush %lld\n", warp, (long long)a.s, (long long)a.Tc, npairs, clock64() - te0, w_q,
-        w_sdp, t_work, t_flush);)
   }
 
   tc::fence_before_sync();
@@ -560,8 +547,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   QShared& sh = *reinterpret_cast<QShared*>(smem_raw + Q_TILES_BYTES);
   uint8_t* sQ = smem_raw;
   uint8_t* sdO = sQ + TILE;
-  uint8_t* sdS = sdO + TILE;                     // half h: dS [128 queries x 64 keys] at h*CHUNK
-  uint8_t* sKV0 = sdS + TILE;                    // ring stage st: K at sKV0 + 2 st TILE, V after
+  uint8_t* sKV0 = sdO + TILE;                    // ring stage st: K at sKV0 + 2 st TILE, V after
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
 
@@ -577,13 +563,16 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&sh.qd_full, 1);
+    tc::mbar_init(&sh.q_tmem, kEwWarps);
     for (int i = 0; i < KV_RING; ++i) {
       tc::mbar_init(&sh.kv_full[i], 1);
       tc::mbar_init(&sh.kv_empty[i], 1);
     }
-    for (int hh = 0; hh < 2; ++hh) {
-      tc::mbar_init(&sh.sdp_full[hh], 1);
-      tc::mbar_init(&sh.ds_full[hh], kEwWarps);
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(&sh.s_full[x], 1);
+      tc::mbar_init(&sh.s_read[x], kEwWarps);
+      tc::mbar_init(&sh.dp_full[x], 1);
+      tc::mbar_init(&sh.ds_full[x], kEwWarps);
     }
     tc::mbar_init(&sh.dq_done, 1);
     tc::mbar_init(&sh.drain, 1);
@@ -635,71 +624,65 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else if (warp == 1) {
     if (lane == 0 && nkv > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      // Two 64-key halves per key tile, each with its own S / dP columns and dS buffer.
-      const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);     // S, dP: N = 64 keys
+      // order: S_0 | dP_j S_{j+1} dQ_j | ...  (S_{j+1} goes into the other score region, whose
+      // previous dS has been read by dQ_{j-1}, issued before it)
+      const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S, dP: B K-major
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dQ: B MN-major
-      const uint32_t aQ = tc::smem_u32(sQ), adO = tc::smem_u32(sdO), adS = tc::smem_u32(sdS),
-                     aKV0 = tc::smem_u32(sKV0);
-      // descriptors built once; k-steps add their offset / 16 (see the key-tile kernel)
-      const uint64_t dQ = tc::smem_desc_sw128(aQ, 16, 1024), dO = tc::smem_desc_sw128(adO, 16, 1024);
-      const uint64_t dS = tc::smem_desc_sw128(adS, 16, 1024);
+      const uint32_t aKV0 = tc::smem_u32(sKV0);
       static_assert(KV_RING == 2, "stage descriptors are selected between two stages");
       const uint64_t dKk0 = tc::smem_desc_sw128(aKV0, 16, 1024);
       const uint64_t dVk0 = tc::smem_desc_sw128(aKV0 + TILE, 16, 1024);
       const uint64_t dKm0 = tc::smem_desc_sw128(aKV0, CHUNK, 1024);
       constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
-      // S_h = Q K_h^T and dP_h = dO V_h^T of key tile j's half hh
-      auto scores = [&](int j, int hh) {
-        const uint64_t so = (j & 1) ? kStage : 0;
-        const uint64_t bk = dKk0 + so + (uint64_t)((hh * HALF) >> 4);
-        const uint64_t bv = dVk0 + so + (uint64_t)((hh * HALF) >> 4);
+      // S_j = Q K_j^T into score region j & 1
+      auto scores = [&](int j) {
+        const uint64_t so = (j % KV_RING) ? kStage : 0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + c_s(hh), dQ + off, bk + off, id_s, kk != 0);
-          tc::mma_f16_ss(tmem + c_dp(hh), dO + off, bv + off, id_s, kk != 0);
+          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          mma_f16_ts(tmem + q_sp(j & 1), tmem + Q_QT + 8 * kk, dKk0 + off, id_s, kk != 0);
         }
-        tc::mma_commit(&sh.sdp_full[hh]);
+        tc::mma_commit(&sh.s_full[j & 1]);
       };
-      // dQ += dS_h K_h
-      auto dq_prod = [&](int j, int hh) {
-        const uint64_t so = (j & 1) ? kStage : 0;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {   // K = 64 keys of the half
-          tc::mma_f16_ss(tmem + C_DQ, dS + (uint64_t)((hh * CHUNK + kk * 32) >> 4),
-                         dKm0 + so + (uint64_t)(((4 * hh + kk) * 2048) >> 4), id_g,
-                         (j | hh | kk) != 0 ? 1u : 0u);
-        }
-      };
-      bool ok = tc::mbar_wait(&sh.qd_full, 0, abort_flag) &&
+      bool ok = tc::mbar_wait(&sh.q_tmem, 0, abort_flag) &&        // Q, dO copied into TMEM
                 tc::mbar_wait(&sh.kv_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
-        scores(0, 0);
-        scores(0, 1);
+        scores(0);
         issued = true;
       }
       for (int j = 0; j < nkv && ok; ++j) {
-        const uint32_t ph = (uint32_t)j & 1u;
-        if (!tc::mbar_wait(&sh.ds_full[0], ph, abort_flag)) { ok = false; break; }
+        const int x = j & 1;
+        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+        const uint64_t so = (j % KV_RING) ? kStage : 0;
+        // dP_j = dO V_j^T over S_j once the element-wise warps have read S_j
+        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
-        dq_prod(j, 0);
-        const bool more = j + 1 < nkv;
-        if (more) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          mma_f16_ts(tmem + q_sp(x), tmem + Q_OT + 8 * kk, dVk0 + off, id_s, kk != 0);
+        }
+        tc::mma_commit(&sh.dp_full[x]);
+        if (j + 1 < nkv) {
           const int st1 = (j + 1) % KV_RING;
           if (!tc::mbar_wait(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          scores(j + 1, 0);
+          scores(j + 1);
         }
-        if (!tc::mbar_wait(&sh.ds_full[1], ph, abort_flag)) { ok = false; break; }
+        // dQ += dS_j K_j
+        if (!tc::mbar_wait(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
-        dq_prod(j, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = 128 keys
+          mma_f16_ts(tmem + Q_DQ, tmem + q_sp(x) + packed_col(kk),
+                     dKm0 + so + (uint64_t)((kk * 2048) >> 4), id_g, (j | kk) != 0 ? 1u : 0u);
+        }
         tc::mma_commit(&sh.kv_empty[j % KV_RING]);
-        if (more) scores(j + 1, 1);
       }
       if (ok) tc::mma_commit(&sh.dq_done);
       if (issued) {
@@ -711,7 +694,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else if (nkv > 0) {
     // ------------------------------------------------------------------ element-wise warps
     const int q4 = warp & 3;
-    const int wh = (warp - 2) >> 2;                  // column half: keys 32 wh .. of a half
+    const int wh = (warp - 2) >> 2;                  // column half: keys 64 wh .. of a tile
     const int r = q4 * 32 + lane;                    // TMEM lane = query row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int t = (int)(q_lo + r);                   // absolute query position
@@ -720,44 +703,63 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const float lse_r = a.lse_t[srow];               // log2 units (0 in the padding)
     const float dl_r = a.delta_t[srow];
     const float scale_log2 = a.scale * 1.4426950408889634f;
-    bool ok = true;
+    bool ok = tc::mbar_wait_warp(&sh.qd_full, 0, abort_flag);
+    if (ok) {
+      // Q and dO rows of this lane into TMEM (packed), this warp's 64-column half of each
+      tile_row_to_tmem(sQ, r, wh, tmem + lane_off + Q_QT + 32u * (uint32_t)wh);
+      tile_row_to_tmem(sdO, r, wh, tmem + lane_off + Q_OT + 32u * (uint32_t)wh);
+      tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.q_tmem);
+    }
     for (int j = 0; j < nkv && ok; ++j) {
-      const uint32_t ph = (uint32_t)j & 1u;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int k0 = j * BT + 64 * hh + 32 * wh;   // this warp's first key
-        const bool diag = k0 + 31 > (int)q_lo;       // some key may follow some query
-        if (!tc::mbar_wait_warp(&sh.sdp_full[hh], ph, abort_flag)) { ok = false; break; }
-        tc::fence_after_sync();
-        uint32_t rs[32], rd[32];
-        tc::tmem_ld32(tmem + lane_off + c_s(hh) + 32 * wh, rs);
-        tc::tmem_ld32(tmem + lane_off + c_dp(hh) + 32 * wh, rd);
-        tc::tmem_ld_wait();
-        uint32_t dd[16];
+      const int x = j & 1;
+      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      const uint32_t sp = tmem + lane_off + q_sp(x) + 64u * (uint32_t)wh;
+      const int k0 = j * BT + 64 * wh;               // this warp's first key
+      const bool diag = k0 + 63 > (int)q_lo;         // some key may follow some query
+      if (!tc::mbar_wait_warp(&sh.s_full[x], ph, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      float p[64];
+      {
+        uint32_t rs[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float gg[2];
+        for (int c = 0; c < 2; ++c) {
+          tc::tmem_ld32(sp + 32u * (uint32_t)c, rs);
+          tc::tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const float p = ex2(fmaf(__uint_as_float(rs[i + k]), scale_log2, -lse_r));
-            float v = p * (__uint_as_float(rd[i + k]) - dl_r);
-            if (diag) v = (k0 + i + k <= t && qv) ? v : 0.f;
-            else v = qv ? v : 0.f;
-            gg[k] = v;
-          }
-          dd[i >> 1] = pack2(gg[0], gg[1]);
+          for (int i = 0; i < 32; ++i) p[32 * c + i] = __uint_as_float(rs[i]);
         }
-        // dS of this half (the previous tile's dQ product of this half has read the buffer:
-        // its completion precedes the scores this warp has waited for)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_unit(sdS + hh * CHUNK, r, 4 * wh + u,
-                  make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]));
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sh.ds_full[hh]);
       }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.s_read[x]);   // the region may take dP_j now
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float v = ex2(fmaf(p[i], scale_log2, -lse_r));
+        if (diag) v = (k0 + i <= t && qv) ? v : 0.f;
+        else v = qv ? v : 0.f;
+        p[i] = v;
+      }
+      if (!tc::mbar_wait_warp(&sh.dp_full[x], ph, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      // dS = P (dP - delta), packed over this warp's first 32 columns (already read)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rd[32], dw[16];
+        tc::tmem_ld32(sp + 32u * (uint32_t)c, rd);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          dw[i] = pack2(p[32 * c + 2 * i] * (__uint_as_float(rd[2 * i]) - dl_r),
+                        p[32 * c + 2 * i + 1] * (__uint_as_float(rd[2 * i + 1]) - dl_r));
+        tmem_st16(sp + 16u * (uint32_t)c, dw);
+      }
+      tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.ds_full[x]);
     }
     // dQ of this query tile, written once
     if (ok && tc::mbar_wait_warp(&sh.dq_done, 0, abort_flag)) {
@@ -767,7 +769,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       for (int cc = 0; cc < 2; ++cc) {
         const int c = wh * 2 + cc;
         uint32_t rq[32];
-        tc::tmem_ld32(tmem + lane_off + C_DQ + c * 32, rq);
+        tc::tmem_ld32(tmem + lane_off + Q_DQ + c * 32, rq);
         tc::tmem_ld_wait();
         if (qv) {
 #pragma unroll

@@ -420,6 +420,29 @@ __global__ void gather_chunk_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s,
     static_cast<float*>(dst)[i] = static_cast<const float*>(src)[so];
 }
 
+// Row copy between the chunk buffer [B * Tc, cols] and the sequence layout [B, T, cols] in
+// 16-byte units: one CTA per chunk row (token s + r % Tc of sequence r / Tc), threads over the
+// row's units.  to_seq: chunk -> sequence (optionally adding fp32 rows), else sequence -> chunk.
+__global__ void chunk_rows_vec_kernel(int64_t Tc, int64_t s, int64_t T, int units,
+                                      const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                      int to_seq, int accumulate_f32) {
+  const int64_t r = blockIdx.x;
+  const int64_t srow = (r / Tc) * T + s + r % Tc;
+  const uint4* sp = src + (to_seq ? r : srow) * units;
+  uint4* dp = dst + (to_seq ? srow : r) * units;
+  for (int u = threadIdx.x; u < units; u += blockDim.x) {
+    uint4 v = sp[u];
+    if (accumulate_f32) {
+      const uint4 o = dp[u];
+      v.x = __float_as_uint(__uint_as_float(v.x) + __uint_as_float(o.x));
+      v.y = __float_as_uint(__uint_as_float(v.y) + __uint_as_float(o.y));
+      v.z = __float_as_uint(__uint_as_float(v.z) + __uint_as_float(o.z));
+      v.w = __float_as_uint(__uint_as_float(v.w) + __uint_as_float(o.w));
+    }
+    dp[u] = v;
+  }
+}
+
 __global__ void scatter_chunk_kernel(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
                                      int dt, const void* __restrict__ src, void* __restrict__ dst,
                                      int accumulate) {
@@ -691,10 +714,29 @@ cudaError_t swiglu_bwd(int64_t R, int64_t f, int dt, const void* gu, const float
   return cudaGetLastError();
 }
 
+namespace {
+// The 16-byte row path applies when rows are whole 16-byte units and both buffers aligned.
+bool rows_vec_ok(int64_t cols, int dt, const void* a, const void* b) {
+  const int64_t bytes = cols * (int64_t)dt_size(dt);
+  return bytes % 16 == 0 && bytes / 16 <= (1 << 20) &&
+         (reinterpret_cast<uintptr_t>(a) & 15u) == 0 && (reinterpret_cast<uintptr_t>(b) & 15u) == 0;
+}
+cudaError_t chunk_rows_vec(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
+                           const void* src, void* dst, int to_seq, int accumulate_f32,
+                           cudaStream_t st) {
+  const int units = (int)(cols * (int64_t)dt_size(dt) / 16);
+  const int threads = units >= 256 ? 256 : ((units + 31) / 32) * 32;
+  launch(chunk_rows_vec_kernel, dim3((unsigned)(B * Tc)), dim3(threads), 0, st, Tc, s, T, units,
+         static_cast<const uint4*>(src), static_cast<uint4*>(dst), to_seq, accumulate_f32);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t gather_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols, int dt,
                          const void* src, void* dst, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
+  if (rows_vec_ok(cols, dt, src, dst)) return chunk_rows_vec(B, T, Tc, s, cols, dt, src, dst, 0, 0, st);
   launch(gather_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, dt, src, dst);
   return cudaGetLastError();
 }
@@ -703,6 +745,8 @@ cudaError_t scatter_chunk_f32(int64_t B, int64_t T, int64_t Tc, int64_t s, int64
                               const float* src, float* dst, int accumulate, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
+  if (rows_vec_ok(cols, DT_F32, src, dst))
+    return chunk_rows_vec(B, T, Tc, s, cols, DT_F32, src, dst, 1, accumulate, st);
   launch(scatter_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, DT_F32, src, dst,
                                                      accumulate);
   return cudaGetLastError();
@@ -712,6 +756,7 @@ cudaError_t scatter_chunk(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t c
                           const void* src, void* dst, cudaStream_t st) {
   const int64_t n = B * Tc * cols;
   if (n <= 0) return cudaSuccess;
+  if (rows_vec_ok(cols, dt, src, dst)) return chunk_rows_vec(B, T, Tc, s, cols, dt, src, dst, 1, 0, st);
   launch(scatter_chunk_kernel, nblk(n, 256), 256, 0, st, B, T, Tc, s, cols, dt, src, dst, 0);
   return cudaGetLastError();
 }

@@ -19,7 +19,8 @@ cudaError_t gemm(const GemmDesc& g, cudaStream_t st) {
   if (g.kblk < 0 || (g.kblk > 0 && (g.kblk % 64 != 0 || (g.epi != EPI_STORE && g.epi != EPI_ACC))))
     return cudaErrorInvalidValue;
   const bool tc = g.path != 1 && gemm_tc_supported(g);
-  if (!tc && g.path >= 2) return cudaErrorNotSupported;
+  if (!tc && (g.path >= 2 || g.epi == EPI_ROPE || g.epi == EPI_SWIGLU_FWD))
+    return cudaErrorNotSupported;
   const int kind = tc ? PROF_GEMM_TC : PROF_GEMM_SIMT;
   prof_mark_begin(kind, st);
   const cudaError_t e = tc ? ((g.path == 4 || (g.path == 0 && use_pair(g))) ? gemm_tc_pair(g, g.err, st)

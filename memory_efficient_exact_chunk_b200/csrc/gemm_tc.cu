@@ -167,6 +167,39 @@ __device__ __forceinline__ void epi_swiglu_bwd32(const GemmDesc& g, int64_t m, i
   }
 }
 
+// SwiGLU forward for 32 consecutive columns: v = u, g from aux (bf16); u (rounded to bf16) to
+// C and m = silu(g) u of the rounded u to C2 (bf16) -- the values the separate SwiGLU kernel
+// computes from the stored g and u, bit for bit, and the ones the backward differentiates.
+__device__ __forceinline__ void epi_swiglu_fwd32(const GemmDesc& g, int64_t m, int64_t n,
+                                                 int64_t N, const float (&v)[32]) {
+  const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(g.aux) + m * g.aux_ld + n;
+  __nv_bfloat16* up = static_cast<__nv_bfloat16*>(g.C) + m * g.ldc + n;
+  __nv_bfloat16* mp = static_cast<__nv_bfloat16*>(g.C2) + m * g.ldc2 + n;
+  if (n + 32 <= N) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 gq = *reinterpret_cast<const uint4*>(gp + 8 * q);
+      const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
+      float mv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float gv = __bfloat162float(gb[i]);
+        const float uv = __bfloat162float(__float2bfloat16_rn(v[8 * q + i]));
+        mv[i] = gv / (1.f + expf(-gv)) * uv;
+      }
+      store8_bf16(up + 8 * q, v + 8 * q);
+      store8_bf16(mp + 8 * q, mv);
+    }
+  } else {
+    for (int i = 0; i < 32 && n + i < N; ++i) {
+      const float gv = __bfloat162float(gp[i]);
+      const __nv_bfloat16 ub = __float2bfloat16_rn(v[i]);
+      up[i] = ub;
+      mp[i] = __float2bfloat16_rn(gv / (1.f + expf(-gv)) * __bfloat162float(ub));
+    }
+  }
+}
+
 // Epilogue of one accumulator tile for the calling thread's row m: tile columns
 // [c_lo, c_lo + BN / 2) (this warp's half) starting at global column n0, read from TMEM at
 // tbase (this warp's lane quarter, accumulator base column).  nk = the k-steps summed into
@@ -216,6 +249,51 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
         g.zy[m] = nk ? z : 0.f;
       }
     }
+  } else if (g.epi == EPI_ROPE) {
+    // this warp's 128 columns are one head: rotate pairs (i, i + 64) with the row's position
+    const int64_t rr = m % g.r_Tc;
+    const int64_t pos = g.r_s + rr;
+    const int64_t drow = g.r_T > 0 ? (m / g.r_Tc) * g.r_T + pos : m;
+    const int64_t nh = n0 + c_lo;                 // the head's first column
+#pragma unroll 1
+    for (int c = 0; c < 64; c += 32) {
+      uint32_t lo[32], hi[32];
+      tc::tmem_ld32(tbase + c_lo + c, lo);
+      tc::tmem_ld32(tbase + c_lo + 64 + c, hi);
+      tc::tmem_ld_wait();
+      if (!row_ok || nh >= N) continue;
+      float a[32], bb[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        a[j] = nk ? u2f(lo[j]) : 0.f;
+        bb[j] = nk ? u2f(hi[j]) : 0.f;
+      }
+      if (g.bias) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          a[j] += ld_dt(g.bias, g.bias_dt, nh + c + j);
+          bb[j] += ld_dt(g.bias, g.bias_dt, nh + 64 + c + j);
+        }
+      }
+      if (g.cosb) {
+        const float* cr = g.cosb + pos * 64 + c;
+        const float* sr = g.sinb + pos * 64 + c;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float cs = cr[j], sn = sr[j];
+          const float y1 = a[j] * cs - bb[j] * sn;
+          const float y2 = bb[j] * cs + a[j] * sn;
+          a[j] = y1;
+          bb[j] = y2;
+        }
+      }
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.C) + drow * g.ldc + nh + c;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        store8_bf16(out + j, a + j);
+        store8_bf16(out + 64 + j, bb + j);
+      }
+    }
   } else {
     float w = 0.f, l = 0.f;
     int64_t ycol = -1;
@@ -240,6 +318,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmDesc& g, uint32_t tbase,
       for (int j = 0; j < 32; ++j) v[j] = nk ? u2f(r[j]) : 0.f;
       if (g.epi == EPI_SWIGLU_BWD) {
         epi_swiglu_bwd32(g, m, nc, N, v);
+        continue;
+      }
+      if (g.epi == EPI_SWIGLU_FWD) {
+        epi_swiglu_fwd32(g, m, nc, N, v);
         continue;
       }
       if (g.epi == EPI_CEGRAD) {
@@ -735,6 +817,14 @@ bool gemm_tc_supported(const GemmDesc& g) {
   }
   if (g.epi == EPI_SWIGLU_BWD &&
       (g.cdt != DT_BF16 || !al16(g.aux) || g.aux_ld % 8 != 0 || g.aux_off % 8 != 0))
+    return false;
+  if (g.epi == EPI_SWIGLU_FWD &&
+      (g.cdt != DT_BF16 || !al16(g.C) || g.ldc % 8 != 0 || !al16(g.aux) || g.aux_ld % 8 != 0 ||
+       !al16(g.C2) || g.ldc2 % 8 != 0 || g.kblk != 0))
+    return false;
+  if (g.epi == EPI_ROPE &&
+      (g.cdt != DT_BF16 || !al16(g.C) || g.ldc % 8 != 0 || g.N % 128 != 0 || g.kblk != 0 ||
+       g.r_Tc <= 0))
     return false;
   if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX)
     return false;

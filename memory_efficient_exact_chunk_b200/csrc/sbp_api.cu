@@ -117,6 +117,13 @@ struct LayerPlan {
   int64_t R;
 };
 
+// The Q / K / V projections get their bias, the rotate-half RoPE, the cast to bf16 and the
+// append to the K/V prefix in the tensor-core GEMM's epilogue (no fp32 staging of the
+// projections) on the bf16 path with head_dim 128.
+bool qkv_fused(const sbp_layer_cfg& L) {
+  return L.dtype == SBP_BF16 && L.head_dim == 128 && L.d_model % 8 == 0;
+}
+
 void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   const int dt = L.dtype;
   const size_t es = dt_size(dt);
@@ -135,7 +142,8 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.dyg = c.take<float>((size_t)R * d);
   p.n1 = c.take_bytes((size_t)R * d * es);
   p.rstd1 = c.take<float>(R);
-  p.qkv = c.take<float>((size_t)R * (dq + 2 * dkv));
+  // fp32 staging of the Q/K/V projections: only where RoPE is not done in the GEMM epilogue
+  p.qkv = c.take<float>(qkv_fused(L) ? 0 : (size_t)R * (dq + 2 * dkv));
   p.q = c.take_bytes((size_t)R * dq * es);
   p.o = c.take_bytes((size_t)R * dq * es);
   p.alse = c.take<float>((size_t)R * L.n_heads);
@@ -231,6 +239,33 @@ sbp_status check_weights(const sbp_layer_weights* w, bool* has_bias) {
   return SBP_OK;
 }
 
+// Fused Q / K / V projections of a chunk (qkv_fused): part QKV_Q, QKV_KV or QKV_ALL.
+sbp_status qkv_project(const sbp_layer_cfg& L, const sbp_layer_weights& w, const LayerPlan& p,
+                       int64_t s, int64_t Tc, int part, cudaStream_t st) {
+  const int dt = L.dtype;
+  const int64_t B = L.batch, T = L.seq_len, d = L.d_model;
+  const int64_t dq = L.n_heads * L.head_dim, dkv = L.n_kv_heads * L.head_dim;
+  const int64_t R = B * Tc;
+  (void)B;
+  auto proj = [&](int64_t N, const void* W, const void* bias, void* out, int64_t rT,
+                  bool rope) -> sbp_status {
+    GemmDesc g = mk_gemm(R, N, d, dt, p.n1, false, d, dt, W, true, d, DT_BF16, out, N, EPI_ROPE);
+    g.bias = bias; g.bias_dt = dt;
+    g.cosb = rope ? p.cosb : nullptr;
+    g.sinb = rope ? p.sinb : nullptr;
+    g.r_Tc = Tc; g.r_s = s; g.r_T = rT;
+    SBP_CK(gemm(g, st));
+    return SBP_OK;
+  };
+  sbp_status r = SBP_OK;
+  if (part != QKV_KV && (r = proj(dq, w.wq, w.bq, p.q, 0, true)) != SBP_OK) return r;
+  if (part != QKV_Q) {
+    if ((r = proj(dkv, w.wk, w.bk, p.Kp, T, true)) != SBP_OK) return r;
+    if ((r = proj(dkv, w.wv, w.bv, p.Vp, T, false)) != SBP_OK) return r;
+  }
+  return SBP_OK;
+}
+
 // RMSNorm-1 and the K/V projections of one chunk: fills n1, rstd1 and the chunk's rows of the
 // K/V prefix.  xc is the chunk's input rows [B * Tc, d] (contiguous).
 sbp_status layer_chunk_kv(const sbp_layer_cfg& L, const sbp_layer_weights& w, const LayerPlan& p,
@@ -241,6 +276,7 @@ sbp_status layer_chunk_kv(const sbp_layer_cfg& L, const sbp_layer_weights& w, co
   const int64_t dq = H * hd, dkv = Hkv * hd, W3 = dq + 2 * dkv;
   const int64_t R = B * Tc;
   SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
+  if (qkv_fused(L)) return qkv_project(L, w, p, s, Tc, QKV_KV, st);
   GemmDesc g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
                        EPI_STORE);
   g.bias = w.bk; g.bias_dt = dt;
@@ -266,25 +302,28 @@ sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& 
   const int64_t dq = H * hd, dkv = Hkv * hd, W3 = dq + 2 * dkv;
   const int64_t R = B * Tc;
   SBP_CK(rmsnorm_fwd(R, d, dt, xc, dt, w.ln1_g, dt, p.n1, p.rstd1, L.rms_eps, st));
-  {
+  if (qkv_fused(L)) {
+    const sbp_status r = qkv_project(L, w, p, s, Tc, kv_ready ? QKV_Q : QKV_ALL, st);
+    if (r != SBP_OK) return r;
+  } else {
     GemmDesc g = mk_gemm(R, dq, d, dt, p.n1, false, d, dt, w.wq, true, d, DT_F32, p.qkv, W3,
                          EPI_STORE);
     g.bias = w.bq; g.bias_dt = dt;
     SBP_CK(gemm(g, st));
-  }
-  if (kv_ready) {
-    SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st,
-                    QKV_Q));
-  } else {
-    GemmDesc g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
-                         EPI_STORE);
-    g.bias = w.bk; g.bias_dt = dt;
-    SBP_CK(gemm(g, st));
-    g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wv, true, d, DT_F32, p.qkv + dq + dkv, W3,
-                EPI_STORE);
-    g.bias = w.bv; g.bias_dt = dt;
-    SBP_CK(gemm(g, st));
-    SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
+    if (kv_ready) {
+      SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st,
+                      QKV_Q));
+    } else {
+      g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wk, true, d, DT_F32, p.qkv + dq, W3,
+                  EPI_STORE);
+      g.bias = w.bk; g.bias_dt = dt;
+      SBP_CK(gemm(g, st));
+      g = mk_gemm(R, dkv, d, dt, p.n1, false, d, dt, w.wv, true, d, DT_F32, p.qkv + dq + dkv,
+                  W3, EPI_STORE);
+      g.bias = w.bv; g.bias_dt = dt;
+      SBP_CK(gemm(g, st));
+      SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
+    }
   }
   SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, st));
   SBP_CK(copy_cast(R * d, dt, xc, DT_F32, p.hbuf, st));
@@ -293,9 +332,18 @@ sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& 
   SBP_CK(rmsnorm_fwd(R, d, DT_F32, p.hbuf, dt, w.ln2_g, dt, p.n2, p.rstd2, L.rms_eps, st));
   SBP_CK(gemm(mk_gemm(R, f, d, dt, p.n2, false, d, dt, w.w_gate, true, d, dt, p.gu, 2 * f,
                       EPI_STORE), st));
-  SBP_CK(gemm(mk_gemm(R, f, d, dt, p.n2, false, d, dt, w.w_up, true, d, dt,
-                      static_cast<char*>(p.gu) + f * dt_size(dt), 2 * f, EPI_STORE), st));
-  SBP_CK(swiglu_fwd(R, f, dt, p.gu, p.m, st));
+  // the up projection; on the tensor-core path its epilogue also forms m = silu(g) u
+  GemmDesc gup = mk_gemm(R, f, d, dt, p.n2, false, d, dt, w.w_up, true, d, dt,
+                         static_cast<char*>(p.gu) + f * dt_size(dt), 2 * f, EPI_SWIGLU_FWD);
+  gup.aux = p.gu; gup.aux_ld = 2 * f;
+  gup.C2 = p.m; gup.ldc2 = f;
+  if (dt == DT_BF16 && gemm_tc_supported(gup)) {
+    SBP_CK(gemm(gup, st));
+  } else {
+    gup.epi = EPI_STORE;
+    SBP_CK(gemm(gup, st));
+    SBP_CK(swiglu_fwd(R, f, dt, p.gu, p.m, st));
+  }
   return SBP_OK;
 }
 

@@ -108,10 +108,18 @@ __device__ __forceinline__ float warp_max(float v) {
 //   EPI_SWIGLU_BWD : acc = dM (gradient of m = silu(g) u); with g = aux[m, n] and
 //                u = aux[m, aux_off + n] (aux row stride aux_ld, C dtype):
 //                C[m, n] = dM u silu'(g),  C[m, aux_off + n] = dM silu(g).
+//   EPI_SWIGLU_FWD : acc = u (the up projection); with g = aux[m, n] (bf16, row stride aux_ld):
+//                C[m, n] = u (bf16) and C2[m, n] = silu(g) u (bf16, row stride ldc2).
+//   EPI_ROPE   : the Q / K / V projection of a chunk (head_dim 128, bf16 C): y = acc (+ bias),
+//                rotated per 128-column head by the rotate-half RoPE at position
+//                r_s + m % r_Tc when cosb is set (cos / sin tables [T, 64]), written to row
+//                (m / r_Tc) r_T + r_s + m % r_Tc of C when r_T > 0 (the K/V prefix of the
+//                sequence), else to row m.
 // dynM / dynK (nullable) give the true M / K on the device (<= the static M / K).
 // crow (nullable) maps row m of the result to row crow[m] of C.
 // ---------------------------------------------------------------------------------------------
-enum Epi : int { EPI_STORE = 0, EPI_ACC = 1, EPI_LSE = 2, EPI_CEGRAD = 3, EPI_SWIGLU_BWD = 4 };
+enum Epi : int { EPI_STORE = 0, EPI_ACC = 1, EPI_LSE = 2, EPI_CEGRAD = 3, EPI_SWIGLU_BWD = 4,
+                 EPI_ROPE = 5, EPI_SWIGLU_FWD = 6 };
 
 struct GemmDesc {
   int64_t M = 0, N = 0, K = 0;
@@ -138,9 +146,15 @@ struct GemmDesc {
   float* psum = nullptr;
   int64_t pld = 0;
   float* zy = nullptr;
-  // SwiGLU-backward epilogue operand
+  // SwiGLU-backward / -forward epilogue operand, and the forward's second output
   const void* aux = nullptr;
   int64_t aux_ld = 0, aux_off = 0;
+  void* C2 = nullptr;
+  int64_t ldc2 = 0;
+  // RoPE epilogue: cos / sin tables (nullable: no rotation) and the row map
+  const float* cosb = nullptr;
+  const float* sinb = nullptr;
+  int64_t r_Tc = 0, r_s = 0, r_T = 0;
   // > 0: the accumulator is flushed into C after every kblk elements of K (a multiple of 64),
   // so C is a left-to-right fp32 sum of partial products over consecutive K blocks that
   // start at the GEMM's first K row.  Used on the reductions over tokens (weight gradients):

@@ -24,6 +24,7 @@ pytestmark = pytest.mark.gpu
 
 T, H, HKV, HD, D = 32768, 32, 8, 128, 8
 TC = T // D
+BT = 128                     # keys per tile
 Q_ROWS = (0, 1, 4095, 4096, 12345, 20000, 28672, 32767)
 HEADS = (0, 13, 31)
 
@@ -84,7 +85,7 @@ def test_attention_rows_at_32k(drift):
     q64, k64, v64, dO64 = (a.astype(np.float64) for a in (q, k, v, dO))
     grp = H // HKV
     worst = {"o": 0.0, "lse": 0.0, "dq": 0.0}
-    dq_norms = []
+    dq_ref = {}
     for t in Q_ROWS:
         for h in HEADS:
             g = h // grp
@@ -93,18 +94,22 @@ def test_attention_rows_at_32k(drift):
             out, p = O.attention_forward(qs, ks, vs, q_start=t)
             l0 = O.attention_logsumexp(qs, ks, q_start=t)[0, 0]
             dq0, _, _ = O.attention_backward(dO64[t:t + 1, h:h + 1], qs, ks, vs, p)
+            dq_ref[(t, h)] = dq0[0, 0]
             e = {"o": _rel(o[t, h], out[0, 0]), "lse": abs(float(lse[t, h]) - l0)}
-            if t > 0:
-                # (query 0 sees one key: its softmax is constant and its exact dq is 0)
-                e["dq"] = _rel(dq[t, h], dq0[0, 0])
-                dq_norms.append(float(np.linalg.norm(dq0[0, 0])))
             for n in e:
                 worst[n] = max(worst[n], e[n])
-            assert e["o"] <= 1e-2 and e.get("dq", 0.0) <= 1e-2, (t, h, e)
+            assert e["o"] <= 1e-2, (t, h, e)
             assert e["lse"] <= 2e-3 * max(1.0, abs(l0)), (t, h, e, l0)
-    # the degenerate row: rounding-level dq against the typical dq of the sampled rows
-    for h in HEADS:
-        assert np.linalg.norm(dq[0, h]) <= 1e-2 * np.median(dq_norms), h
+    # dQ: rows that see at least a key tile are held to 1e-2 of their own norm; a row with a
+    # handful of keys has a dq that is a sum of a few terms which can cancel (query 0 sees one
+    # key: its softmax is constant and its exact dq is 0), so its error is measured against the
+    # typical dq norm of the other sampled rows
+    typical = float(np.median([np.linalg.norm(v) for (t, _), v in dq_ref.items() if t >= BT]))
+    for (t, h), v in dq_ref.items():
+        den = np.linalg.norm(v) if t >= BT else max(np.linalg.norm(v), typical)
+        e_dq = float(np.linalg.norm(dq[t, h] - v) / den)
+        worst["dq"] = max(worst["dq"], e_dq)
+        assert e_dq <= 1e-2, (t, h, e_dq)
     # dK / dV of the last key rows: every query that reads them lies in [u0, T)
     u0 = T - 256
     for g in (0, 5):
