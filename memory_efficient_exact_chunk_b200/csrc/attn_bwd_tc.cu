@@ -11,13 +11,16 @@
 // 128 x 128 at a time, and P^T / dS^T (or dS) are written back into TMEM as packed bf16 over
 // the scores they are computed from.
 //
-// dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile); K and V live in TMEM.  It
-// loops over the query heads of g's group and the chunk's query tiles that can see those
-// keys; per (head, query tile) pair, with one 128-column score region SP:
+// dK/dV kernel: one CTA owns (sequence b, KV head g, 128-key tile).  It loops over the query
+// heads of g's group and the chunk's query tiles that can see those keys; per (head, query
+// tile) pair, in one of two 128-column score regions SP used alternately:
 //   S^T  = K Q^T                  -> SP   (the element-wise warps read it out)
 //   dP^T = V dO^T                 -> SP   (while the warps compute P^T = exp(S^T - lse))
-//   P^T, dS^T = P^T (dP^T - delta) -> SP as packed bf16 (each warp over its own columns)
+//   P^T, dS^T = P^T (dP^T - delta) -> SP as packed bf16 (each warp over columns it has read)
 //   dV += P^T dO,  dK += dS^T Q   (A = P^T, dS^T from TMEM; B = dO, Q from shared memory)
+// K and V stay in shared memory as the A operands of the score products: the two score
+// regions, not a TMEM copy of K and V, take the TMEM beside the dK / dV accumulators, so the
+// tensor cores compute the next pair's scores while the element-wise warps work on this one.
 // The query tiles are taken in blocks of a fixed number of tiles counted from the chunk start
 // (all heads of the group within a block); after each block dK, dV are added into the fp32
 // prefix accumulators (single owner, no atomics).  A chunk whose length is a multiple of the
@@ -56,8 +59,8 @@ constexpr int KV_RING = 2;                  // K/V stages of the dQ kernel
 // the barriers.
 struct KvShared {
   float stat[QD_STAGES][2][BT];   // per stage: lse (log2 units), delta of the pair's queries
-  uint64_t kv_full, kv_tmem, qd_full[QD_STAGES], qd_empty[QD_STAGES], s_full, s_read, dp_full,
-      ds_full, kv_free, drain;
+  uint64_t kv_full, qd_full[QD_STAGES], qd_empty[QD_STAGES], s_full[2], s_read[2], dp_full[2],
+      ds_full[2], kv_free, drain;
   uint32_t tmem;
   int abort;
 };
@@ -74,17 +77,23 @@ constexpr int Q_SMEM_BYTES = Q_TILES_BYTES + (int)sizeof(QShared);
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns.  dK/dV kernel: K and V (packed bf16, 64 columns each), the score region SP,
-// the fp32 accumulators dV and dK.  dQ kernel: Q and dO (packed), two score regions, dQ.
-constexpr uint32_t KV_KT = 0, KV_VT = 64, KV_SP = 128, KV_DV = 256, KV_DK = 384;
+// TMEM columns.  dK/dV kernel: two score regions, the fp32 accumulators dV and dK.  dQ
+// kernel: Q and dO (packed bf16, 64 columns each), two score regions, dQ.
+constexpr uint32_t KV_SP0 = 0, KV_DV = 256, KV_DK = 384;
 constexpr uint32_t Q_QT = 0, Q_OT = 64, Q_SP0 = 128, Q_DQ = 384;
+__device__ __forceinline__ uint32_t kv_sp(int x) { return KV_SP0 + 128u * (uint32_t)x; }
 __device__ __forceinline__ uint32_t q_sp(int x) { return Q_SP0 + 128u * (uint32_t)x; }
-// Packed-bf16 A operand written back over a score region: the warps of column half wh own
-// score columns [64 wh, 64 wh + 64) and put their packed values at the start of that range
-// (P^T at +0, dS^T at +32 in the dK/dV kernel; dS at +0 in the dQ kernel).  The k-step kk of
-// a K = 128 product (16 rows of K each) therefore starts at column 64 (kk / 4) + 8 (kk % 4).
+// Packed-bf16 A operands written back over a score region: the warps of column half wh own
+// score columns [64 wh, 64 wh + 64).  dQ kernel: dS of those 64 keys at the start of the range,
+// so the k-step kk of a K = 128 product (16 keys) starts at column 64 (kk / 4) + 8 (kk % 4).
+// dK/dV kernel: per 32 queries (columns [32 c, 32 c + 32) of the range), P^T at +0 and dS^T at
+// +16, so the k-step kk (16 queries) of P^T starts at 64 (kk / 4) + 32 ((kk / 2) % 2) +
+// 8 (kk % 2) and that of dS^T 16 columns later.
 __device__ __forceinline__ uint32_t packed_col(int kk) {
   return 64u * (uint32_t)(kk >> 2) + 8u * (uint32_t)(kk & 3);
+}
+__device__ __forceinline__ uint32_t kv_packed_col(int kk) {
+  return 64u * (uint32_t)(kk >> 2) + 32u * (uint32_t)((kk >> 1) & 1) + 8u * (uint32_t)(kk & 1);
 }
 
 struct BwdArgs {
@@ -235,15 +244,16 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&sh.kv_full, 1);
-    tc::mbar_init(&sh.kv_tmem, kEwWarps);
     for (int i = 0; i < QD_STAGES; ++i) {
       tc::mbar_init(&sh.qd_full[i], 1);
       tc::mbar_init(&sh.qd_empty[i], 1);
     }
-    tc::mbar_init(&sh.s_full, 1);
-    tc::mbar_init(&sh.s_read, kEwWarps);
-    tc::mbar_init(&sh.dp_full, 1);
-    tc::mbar_init(&sh.ds_full, kEwWarps);
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(&sh.s_full[x], 1);
+      tc::mbar_init(&sh.s_read[x], kEwWarps);
+      tc::mbar_init(&sh.dp_full[x], 1);
+      tc::mbar_init(&sh.ds_full[x], kEwWarps);
+    }
     tc::mbar_init(&sh.kv_free, kEwWarps);
     tc::mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -300,52 +310,69 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 1) {
     if (lane == 0 && npairs > 0) {
       // ---------------------------------------------------------------- MMA issuer
+      // order: S^T_0 | dP^T_j S^T_{j+1} grads_j | ...  (S^T_{j+1} goes into the other score
+      // region, whose P^T / dS^T the grads of pair j - 1, issued before it, have read)
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: B K-major
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dV, dK: B MN-major
       const uint32_t aQ0 = tc::smem_u32(sQ0);
       // shared-memory descriptors built once; a k-step adds its byte offset / 16 to the start
       // address field (the tiles sit below 256 KB, so the field cannot carry over)
       static_assert(QD_STAGES == 2, "stage descriptors are selected between two stages");
+      const uint64_t dK = tc::smem_desc_sw128(tc::smem_u32(sK), 16, 1024);
+      const uint64_t dV = tc::smem_desc_sw128(tc::smem_u32(sV), 16, 1024);
       const uint64_t dQk0 = tc::smem_desc_sw128(aQ0, 16, 1024);
       const uint64_t dOk0 = tc::smem_desc_sw128(aQ0 + TILE, 16, 1024);
       const uint64_t dQm0 = tc::smem_desc_sw128(aQ0, CHUNK, 1024);
       const uint64_t dOm0 = tc::smem_desc_sw128(aQ0 + TILE, CHUNK, 1024);
       constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
-      bool ok = tc::mbar_wait(&sh.kv_tmem, 0, abort_flag);      // K, V copied into TMEM
+      // S^T_j = K Q_j^T into score region j & 1
+      auto scores = [&](int j) {
+        const uint64_t so = (j % QD_STAGES) ? kStage : 0;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
+          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(tmem + kv_sp(j & 1), dK + off, dQk0 + so + off, id_s, kk != 0);
+        }
+        tc::mma_commit(&sh.s_full[j & 1]);
+      };
+      bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag) &&
+                tc::mbar_wait(&sh.qd_full[0], 0, abort_flag);
       bool issued = false;
+      if (ok) {
+        tc::fence_after_sync();
+        scores(0);
+        issued = true;
+      }
       int nflush = 0;
       PairIter it;
       it.init((int)i0, a.nq, (int)grp, a.qb);
       for (int j = 0; j < npairs && ok; ++j, it.next()) {
         const PairPos pos = it.pos(g);
+        const int x = j & 1;
+        const uint32_t ph = (uint32_t)(j >> 1) & 1u;
         const int st = j % QD_STAGES;
-        const uint32_t ph = (uint32_t)j & 1u;
         const uint64_t so = st ? kStage : 0;
-        if (!tc::mbar_wait(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        // S^T = K Q^T (the previous pair's dV / dK products, issued before, have read SP)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          mma_f16_ts(tmem + KV_SP, tmem + KV_KT + 8 * kk, dQk0 + off, id_s, kk != 0);
-        }
-        tc::mma_commit(&sh.s_full);
-        issued = true;
-        // dP^T = V dO^T, over S^T once the element-wise warps have read it
-        if (!tc::mbar_wait(&sh.s_read, ph, abort_flag)) { ok = false; break; }
+        // dP^T_j = V dO_j^T over S^T_j once the element-wise warps have read S^T_j
+        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          mma_f16_ts(tmem + KV_SP, tmem + KV_VT + 8 * kk, dOk0 + off, id_s, kk != 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(tmem + kv_sp(x), dV + off, dOk0 + so + off, id_s, kk != 0);
         }
-        tc::mma_commit(&sh.dp_full);
+        tc::mma_commit(&sh.dp_full[x]);
+        if (j + 1 < npairs) {
+          const int st1 = (j + 1) % QD_STAGES;
+          if (!tc::mbar_wait(&sh.qd_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          scores(j + 1);
+        }
         // dV += P^T dO, dK += dS^T Q once P^T, dS^T are in TMEM; a new block overwrites dK / dV,
         // so the element-wise warps must have added the last one
-        if (!tc::mbar_wait(&sh.ds_full, ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
         if (pos.first && j > 0) {
           if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
           ++nflush;
@@ -355,9 +382,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int kk = 0; kk < 8; ++kk) {   // K = 128 queries
           const uint64_t offm = so + (uint64_t)((kk * 2048) >> 4);     // MN-major k-step
           const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
-          const uint32_t pc = KV_SP + packed_col(kk);
+          const uint32_t pc = kv_sp(x) + kv_packed_col(kk);
           mma_f16_ts(tmem + KV_DV, tmem + pc, dOm0 + offm, id_g, acc);
-          mma_f16_ts(tmem + KV_DK, tmem + pc + 32, dQm0 + offm, id_g, acc);
+          mma_f16_ts(tmem + KV_DK, tmem + pc + 16, dQm0 + offm, id_g, acc);
         }
         tc::mma_commit(&sh.qd_empty[st]);
       }
@@ -373,27 +400,19 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int wh = (warp - 2) >> 2;                  // column half: queries 64 wh .. 64 wh + 63
     const int r = q4 * 32 + lane;                    // TMEM lane = key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t sp = tmem + lane_off + KV_SP + 64u * (uint32_t)wh;   // this warp's columns
     const int kpos = (int)(k_lo + r);
     const float scale_log2 = a.scale * 1.4426950408889634f;
     const int e32 = (int)e;
     const bool kv = kpos < e32;
     const int64_t ko = ((b * a.T + kpos) * a.Hkv + g) * HD;
-    bool ok = tc::mbar_wait_warp(&sh.kv_full, 0, abort_flag);
-    if (ok) {
-      // K and V rows of this lane into TMEM (packed), this warp's 64-column half of each
-      tile_row_to_tmem(sK, r, wh, tmem + lane_off + KV_KT + 32u * (uint32_t)wh);
-      tile_row_to_tmem(sV, r, wh, tmem + lane_off + KV_VT + 32u * (uint32_t)wh);
-      tmem_st_wait();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.kv_tmem);
-    }
+    bool ok = true;
     PairIter it;
     it.init((int)i0, a.nq, (int)grp, a.qb);
     for (int j = 0; j < npairs && ok; ++j, it.next()) {
-      const uint32_t ph = (uint32_t)j & 1u;
+      const int x = j & 1;
+      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       const PairPos pos = it.pos(g);
+      const uint32_t sp = tmem + lane_off + kv_sp(x) + 64u * (uint32_t)wh;  // this warp's columns
       if (pos.first && kv) {
         // bring this row's dK / dV accumulator lines into L2 ahead of the block's flush
 #pragma unroll
@@ -413,23 +432,15 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 64 <= a.Tc);
       const float* lse_s = sh.stat[st][0] + qoff;
       const float* delta_s = sh.stat[st][1] + qoff;
-      // S^T of this warp's 64 queries
-      if (!tc::mbar_wait_warp(&sh.s_full, ph, abort_flag)) { ok = false; break; }
+      // S^T of this warp's 64 queries, one TMEM load
+      if (!tc::mbar_wait_warp(&sh.s_full[x], ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
-      float p[64];
-      {
-        uint32_t rs[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(sp + 32u * (uint32_t)c, rs);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) p[32 * c + i] = __uint_as_float(rs[i]);
-        }
-      }
+      uint32_t p[64];
+      tc::tmem_ld64(sp, p);
+      tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.s_read);        // SP may take dP^T now
+      if (lane == 0) tc::mbar_arrive(&sh.s_read[x]);     // SP may take dP^T now
       // P^T = exp(S^T * scale - lse) while the tensor cores compute dP^T
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
@@ -438,47 +449,46 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int i = i4 * 4 + k;
-          float x = ex2(fmaf(p[i], scale_log2, -la[k]));
+          float v = ex2(fmaf(__uint_as_float(p[i]), scale_log2, -la[k]));
           if (!full) {
             const int qpos = q0 + i;
-            x = ((kpos <= qpos) && (qpos < e32)) ? x : 0.f;
+            v = ((kpos <= qpos) && (qpos < e32)) ? v : 0.f;
           }
-          p[i] = x;
+          p[i] = __float_as_uint(v);
         }
       }
-      if (!tc::mbar_wait_warp(&sh.dp_full, ph, abort_flag)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&sh.dp_full[x], ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
-      // dS^T = P^T (dP^T - delta); P^T and dS^T go back over this warp's own columns as packed
-      // bf16 (P^T at +0, dS^T at +32), each written only after the values it replaces are read
-      uint32_t dsw[32];
+      // dS^T = P^T (dP^T - delta), per 32 queries: P^T and dS^T of those queries go back as
+      // packed bf16 over the 32 dP^T columns just read (P^T at +0, dS^T at +16)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t rd[32];
         tc::tmem_ld32(sp + 32u * (uint32_t)c, rd);
         tc::tmem_ld_wait();
-        uint32_t pw[16];
+        uint32_t pw[16], dsw[16];
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 dv = reinterpret_cast<const float4*>(delta_s)[8 * c + i4];
           const float da[4] = {dv.x, dv.y, dv.z, dv.w};
-          float gg[4];
+          float pp[4], gg[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int i = 32 * c + i4 * 4 + k;
-            gg[k] = p[i] * (__uint_as_float(rd[i4 * 4 + k]) - da[k]);
+            pp[k] = __uint_as_float(p[32 * c + 4 * i4 + k]);
+            gg[k] = pp[k] * (__uint_as_float(rd[4 * i4 + k]) - da[k]);
           }
-          pw[2 * i4] = pack2(p[32 * c + 4 * i4], p[32 * c + 4 * i4 + 1]);
-          pw[2 * i4 + 1] = pack2(p[32 * c + 4 * i4 + 2], p[32 * c + 4 * i4 + 3]);
-          dsw[16 * c + 2 * i4] = pack2(gg[0], gg[1]);
-          dsw[16 * c + 2 * i4 + 1] = pack2(gg[2], gg[3]);
+          pw[2 * i4] = pack2(pp[0], pp[1]);
+          pw[2 * i4 + 1] = pack2(pp[2], pp[3]);
+          dsw[2 * i4] = pack2(gg[0], gg[1]);
+          dsw[2 * i4 + 1] = pack2(gg[2], gg[3]);
         }
-        tmem_st16(sp + 16u * (uint32_t)c, pw);          // over dP^T columns already read
+        tmem_st16(sp + 32u * (uint32_t)c, pw);
+        tmem_st16(sp + 32u * (uint32_t)c + 16u, dsw);
       }
-      tmem_st32(sp + 32u, dsw);                         // over the second half, now read too
       tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.ds_full);
+      if (lane == 0) tc::mbar_arrive(&sh.ds_full[x]);
       if (!pos.last) continue;
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner); the
       // release of this pair's Q/dO stage is committed after its last dK / dV product
@@ -488,38 +498,30 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       tc::fence_after_sync();
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = wh * 2 + cc;
-        uint32_t rk[32], rv[32];
-        tc::tmem_ld32(tmem + lane_off + KV_DK + c * 32, rk);
-        tc::tmem_ld32(tmem + lane_off + KV_DV + c * 32, rv);
+      for (int cc = 0; cc < 4; ++cc) {
+        // cc 0, 1: dK columns, cc 2, 3: dV columns of this warp's half (one accumulator at a
+        // time keeps the registers of the flush low)
+        const int c = wh * 2 + (cc & 1);
+        const bool isk = cc < 2;
+        uint32_t rv[32];
+        tc::tmem_ld32(tmem + lane_off + (isk ? KV_DK : KV_DV) + c * 32, rv);
         tc::tmem_ld_wait();
         if (kv) {
           // all loads first (one memory latency), then the adds and the stores
-          float4* pk = reinterpret_cast<float4*>(a.dKp + ko + c * 32);
-          float4* pv = reinterpret_cast<float4*>(a.dVp + ko + c * 32);
-          float4 x[8], y[8];
+          float4* pa = reinterpret_cast<float4*>((isk ? a.dKp : a.dVp) + ko + c * 32);
+          const float f = isk ? a.scale : 1.f;
+          float4 xa[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xa[i] = pa[i];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            x[i] = pk[i];
-            y[i] = pv[i];
+            xa[i].x += __uint_as_float(rv[4 * i]) * f;
+            xa[i].y += __uint_as_float(rv[4 * i + 1]) * f;
+            xa[i].z += __uint_as_float(rv[4 * i + 2]) * f;
+            xa[i].w += __uint_as_float(rv[4 * i + 3]) * f;
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            x[i].x += __uint_as_float(rk[4 * i]) * a.scale;
-            x[i].y += __uint_as_float(rk[4 * i + 1]) * a.scale;
-            x[i].z += __uint_as_float(rk[4 * i + 2]) * a.scale;
-            x[i].w += __uint_as_float(rk[4 * i + 3]) * a.scale;
-            y[i].x += __uint_as_float(rv[4 * i]);
-            y[i].y += __uint_as_float(rv[4 * i + 1]);
-            y[i].z += __uint_as_float(rv[4 * i + 2]);
-            y[i].w += __uint_as_float(rv[4 * i + 3]);
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            pk[i] = x[i];
-            pv[i] = y[i];
-          }
+          for (int i = 0; i < 8; ++i) pa[i] = xa[i];
         }
       }
       tc::fence_before_sync();
@@ -721,41 +723,31 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       const bool diag = k0 + 63 > (int)q_lo;         // some key may follow some query
       if (!tc::mbar_wait_warp(&sh.s_full[x], ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
-      float p[64];
-      {
-        uint32_t rs[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc::tmem_ld32(sp + 32u * (uint32_t)c, rs);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) p[32 * c + i] = __uint_as_float(rs[i]);
-        }
-      }
+      uint32_t p[64];
+      tc::tmem_ld64(sp, p);                            // this warp's 64 scores, one load
+      tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sh.s_read[x]);   // the region may take dP_j now
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        float v = ex2(fmaf(p[i], scale_log2, -lse_r));
+        float v = ex2(fmaf(__uint_as_float(p[i]), scale_log2, -lse_r));
         if (diag) v = (k0 + i <= t && qv) ? v : 0.f;
         else v = qv ? v : 0.f;
-        p[i] = v;
+        p[i] = __float_as_uint(v);
       }
       if (!tc::mbar_wait_warp(&sh.dp_full[x], ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
-      // dS = P (dP - delta), packed over this warp's first 32 columns (already read)
+      // dS = P (dP - delta), packed over this warp's first 32 columns (all 64 read above)
+      uint32_t rd[64];
+      tc::tmem_ld64(sp, rd);
+      tc::tmem_ld_wait();
+      uint32_t dw[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rd[32], dw[16];
-        tc::tmem_ld32(sp + 32u * (uint32_t)c, rd);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          dw[i] = pack2(p[32 * c + 2 * i] * (__uint_as_float(rd[2 * i]) - dl_r),
-                        p[32 * c + 2 * i + 1] * (__uint_as_float(rd[2 * i + 1]) - dl_r));
-        tmem_st16(sp + 16u * (uint32_t)c, dw);
-      }
+      for (int i = 0; i < 32; ++i)
+        dw[i] = pack2(__uint_as_float(p[2 * i]) * (__uint_as_float(rd[2 * i]) - dl_r),
+                      __uint_as_float(p[2 * i + 1]) * (__uint_as_float(rd[2 * i + 1]) - dl_r));
+      tmem_st32(sp, dw);
       tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
