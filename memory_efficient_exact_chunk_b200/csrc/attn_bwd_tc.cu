@@ -53,26 +53,31 @@ constexpr int BT = 128;                     // keys per key tile, queries per qu
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
 constexpr int QD_STAGES = 2;                // Q/dO stages of the dK/dV kernel
-constexpr int KV_RING = 2;                  // K/V stages of the dQ kernel
+constexpr int KV_RING = 3;                  // K/V stages of the dQ kernel (the Q/dO staging
+                                            // copy lands in the last one before K/V do)
 // All shared state lives in the dynamic allocation (no static shared memory), whose start is
 // 1024-byte aligned as the 128-byte swizzle needs: the tiles first, then the statistics and
 // the barriers.
 struct KvShared {
   float stat[QD_STAGES][2][BT];   // per stage: lse (log2 units), delta of the pair's queries
-  uint64_t kv_full, qd_full[QD_STAGES], qd_empty[QD_STAGES], s_full[2], s_read[2], dp_full[2],
-      ds_full[2], kv_free, drain;
+  // per stage: q_full (Q and the statistics), do_full (dO) -- S^T needs only Q, so its copy
+  // lands first -- and qd_empty (the stage may be refilled)
+  uint64_t kv_full, q_full[QD_STAGES], do_full[QD_STAGES], qd_empty[QD_STAGES], s_full[2],
+      s_read[2], dp_full[2], ds_full[2], kv_free, drain;
   uint32_t tmem;
   int abort;
 };
 constexpr int KV_TILES_BYTES = (2 + 2 * QD_STAGES) * TILE;        // K, V, 2 x (Q, dO)
 constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
 struct QShared {
-  uint64_t qd_full, q_tmem, kv_full[KV_RING], kv_empty[KV_RING], s_full[2], s_read[2],
-      dp_full[2], ds_full[2], dq_done, drain;
+  // per ring stage: k_full (K), v_full (V) -- S needs only K, so its copy lands first -- and
+  // kv_empty (the stage may be refilled)
+  uint64_t qd_full, q_tmem, k_full[KV_RING], v_full[KV_RING], kv_empty[KV_RING], s_full[2],
+      s_read[2], dp_full[2], ds_full[2], dq_done, drain;
   uint32_t tmem;
   int abort;
 };
-constexpr int Q_TILES_BYTES = (2 + 2 * KV_RING) * TILE;           // Q, dO, 2 x (K, V)
+constexpr int Q_TILES_BYTES = 2 * KV_RING * TILE;                 // KV_RING x (K, V)
 constexpr int Q_SMEM_BYTES = Q_TILES_BYTES + (int)sizeof(QShared);
 constexpr int kEwWarps = 8;                 // element-wise warps: 4 lane quarters x 2 column halves
 constexpr int kThreads = 64 + 32 * kEwWarps;
@@ -245,7 +250,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (threadIdx.x == 0) {
     tc::mbar_init(&sh.kv_full, 1);
     for (int i = 0; i < QD_STAGES; ++i) {
-      tc::mbar_init(&sh.qd_full[i], 1);
+      tc::mbar_init(&sh.q_full[i], 1);
+      tc::mbar_init(&sh.do_full[i], 1);
       tc::mbar_init(&sh.qd_empty[i], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -289,22 +295,27 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
-        tc::mbar_expect_tx(&sh.qd_full[st], 2 * TILE + 2 * BT * 4);
+        tc::mbar_expect_tx(&sh.q_full[st], TILE + 2 * BT * 4);
         const int64_t srow = (pos.hh * a.B + b) * a.Tcp + pos.qi * BT;
-        tc::bulk_load(&sh.stat[st][0][0], a.lse_t + srow, BT * 4, &sh.qd_full[st]);
-        tc::bulk_load(&sh.stat[st][1][0], a.delta_t + srow, BT * 4, &sh.qd_full[st]);
-        tc::tma_load_3d(sQ, &tmQ, &sh.qd_full[st], 0, (int32_t)pos.hh, qrow);
-        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
-        tc::tma_load_3d(sdO, &tmdO, &sh.qd_full[st], 0, (int32_t)pos.hh, qrow);
-        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.qd_full[st], 64, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sQ, &tmQ, &sh.q_full[st], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.q_full[st], 64, (int32_t)pos.hh, qrow);
+        tc::bulk_load(&sh.stat[st][0][0], a.lse_t + srow, BT * 4, &sh.q_full[st]);
+        tc::bulk_load(&sh.stat[st][1][0], a.delta_t + srow, BT * 4, &sh.q_full[st]);
+        tc::mbar_expect_tx(&sh.do_full[st], TILE);
+        tc::tma_load_3d(sdO, &tmdO, &sh.do_full[st], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.do_full[st], 64, (int32_t)pos.hh, qrow);
         issued = j + 1;
       }
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-        for (int j = issued > QD_STAGES ? issued - QD_STAGES : 0; j < issued; ++j)
-          while (!tc::mbar_try_wait(&sh.qd_full[j % QD_STAGES], (uint32_t)(j / QD_STAGES) & 1u) &&
+        for (int j = issued > QD_STAGES ? issued - QD_STAGES : 0; j < issued; ++j) {
+          const uint32_t pj = (uint32_t)(j / QD_STAGES) & 1u;
+          while (!tc::mbar_try_wait(&sh.q_full[j % QD_STAGES], pj) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+          while (!tc::mbar_try_wait(&sh.do_full[j % QD_STAGES], pj) &&
+                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+        }
       }
     }
   } else if (warp == 1) {
@@ -336,7 +347,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::mma_commit(&sh.s_full[j & 1]);
       };
       bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag) &&
-                tc::mbar_wait(&sh.qd_full[0], 0, abort_flag);
+                tc::mbar_wait(&sh.q_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
@@ -353,7 +364,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int st = j % QD_STAGES;
         const uint64_t so = st ? kStage : 0;
         // dP^T_j = V dO_j^T over S^T_j once the element-wise warps have read S^T_j
-        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag) ||
+            !tc::mbar_wait(&sh.do_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -363,7 +378,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tc::mma_commit(&sh.dp_full[x]);
         if (j + 1 < npairs) {
           const int st1 = (j + 1) % QD_STAGES;
-          if (!tc::mbar_wait(&sh.qd_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
+          if (!tc::mbar_wait(&sh.q_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -422,7 +437,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
       const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
-      if (!tc::mbar_wait_warp(&sh.qd_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+      if (!tc::mbar_wait_warp(&sh.q_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -547,9 +562,11 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                   const BwdArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   QShared& sh = *reinterpret_cast<QShared*>(smem_raw + Q_TILES_BYTES);
-  uint8_t* sQ = smem_raw;
+  uint8_t* sKV0 = smem_raw;                      // ring stage st: K at sKV0 + 2 st TILE, V after
+  // Q and dO are staged in the last ring stage; the producer refills that stage with K/V only
+  // once the element-wise warps have copied them into TMEM
+  uint8_t* sQ = sKV0 + 2 * (KV_RING - 1) * TILE;
   uint8_t* sdO = sQ + TILE;
-  uint8_t* sKV0 = sdO + TILE;                    // ring stage st: K at sKV0 + 2 st TILE, V after
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
 
@@ -567,7 +584,8 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     tc::mbar_init(&sh.qd_full, 1);
     tc::mbar_init(&sh.q_tmem, kEwWarps);
     for (int i = 0; i < KV_RING; ++i) {
-      tc::mbar_init(&sh.kv_full[i], 1);
+      tc::mbar_init(&sh.k_full[i], 1);
+      tc::mbar_init(&sh.v_full[i], 1);
       tc::mbar_init(&sh.kv_empty[i], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -605,22 +623,29 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int st = j % KV_RING;
         const uint32_t ph = (uint32_t)(j / KV_RING) & 1u;
         if (!tc::mbar_wait(&sh.kv_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        // the last stage holds the Q / dO staging copy until it is in TMEM
+        if (j == KV_RING - 1 && !tc::mbar_wait(&sh.q_tmem, 0, abort_flag)) { ok = false; break; }
         uint8_t* sK = sKV0 + 2 * st * TILE;
         uint8_t* sV = sK + TILE;
         const int32_t krow = (int32_t)(b * a.T + (int64_t)j * BT);
-        tc::mbar_expect_tx(&sh.kv_full[st], 2 * TILE);
-        tc::tma_load_3d(sK, &tmK, &sh.kv_full[st], 0, (int32_t)g, krow);
-        tc::tma_load_3d(sK + CHUNK, &tmK, &sh.kv_full[st], 64, (int32_t)g, krow);
-        tc::tma_load_3d(sV, &tmV, &sh.kv_full[st], 0, (int32_t)g, krow);
-        tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full[st], 64, (int32_t)g, krow);
+        tc::mbar_expect_tx(&sh.k_full[st], TILE);
+        tc::tma_load_3d(sK, &tmK, &sh.k_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sK + CHUNK, &tmK, &sh.k_full[st], 64, (int32_t)g, krow);
+        tc::mbar_expect_tx(&sh.v_full[st], TILE);
+        tc::tma_load_3d(sV, &tmV, &sh.v_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sV + CHUNK, &tmV, &sh.v_full[st], 64, (int32_t)g, krow);
         issued = j + 1;
       }
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.qd_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-        for (int j = issued > KV_RING ? issued - KV_RING : 0; j < issued; ++j)
-          while (!tc::mbar_try_wait(&sh.kv_full[j % KV_RING], (uint32_t)(j / KV_RING) & 1u) &&
+        for (int j = issued > KV_RING ? issued - KV_RING : 0; j < issued; ++j) {
+          const uint32_t pj = (uint32_t)(j / KV_RING) & 1u;
+          while (!tc::mbar_try_wait(&sh.k_full[j % KV_RING], pj) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+          while (!tc::mbar_try_wait(&sh.v_full[j % KV_RING], pj) &&
+                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
+        }
       }
     }
   } else if (warp == 1) {
@@ -631,14 +656,13 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S, dP: B K-major
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dQ: B MN-major
       const uint32_t aKV0 = tc::smem_u32(sKV0);
-      static_assert(KV_RING == 2, "stage descriptors are selected between two stages");
       const uint64_t dKk0 = tc::smem_desc_sw128(aKV0, 16, 1024);
       const uint64_t dVk0 = tc::smem_desc_sw128(aKV0 + TILE, 16, 1024);
       const uint64_t dKm0 = tc::smem_desc_sw128(aKV0, CHUNK, 1024);
-      constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
+      constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);   // 192 KB of stages < 256 KB
       // S_j = Q K_j^T into score region j & 1
       auto scores = [&](int j) {
-        const uint64_t so = (j % KV_RING) ? kStage : 0;
+        const uint64_t so = (uint64_t)(j % KV_RING) * kStage;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // K = head dim
           const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
@@ -647,7 +671,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc::mma_commit(&sh.s_full[j & 1]);
       };
       bool ok = tc::mbar_wait(&sh.q_tmem, 0, abort_flag) &&        // Q, dO copied into TMEM
-                tc::mbar_wait(&sh.kv_full[0], 0, abort_flag);
+                tc::mbar_wait(&sh.k_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
@@ -657,9 +681,13 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       for (int j = 0; j < nkv && ok; ++j) {
         const int x = j & 1;
         const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-        const uint64_t so = (j % KV_RING) ? kStage : 0;
+        const uint64_t so = (uint64_t)(j % KV_RING) * kStage;
         // dP_j = dO V_j^T over S_j once the element-wise warps have read S_j
-        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag) ||
+            !tc::mbar_wait(&sh.v_full[j % KV_RING], (uint32_t)(j / KV_RING) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -669,7 +697,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc::mma_commit(&sh.dp_full[x]);
         if (j + 1 < nkv) {
           const int st1 = (j + 1) % KV_RING;
-          if (!tc::mbar_wait(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
+          if (!tc::mbar_wait(&sh.k_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
             ok = false;
             break;
           }
