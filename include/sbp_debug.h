@@ -24,7 +24,9 @@ extern "C" {
  * path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores (either kernel), 3 = tensor cores with
  * one CTA per 128 x 256 tile, 4 = tensor cores with a CTA pair per 256 x 256 tile
  * (SBP_ERR_UNSUPPORTED for 2..4 if the layout is not one the tensor-core kernels
- * take).  kblk = 0 sums all of K in one accumulator; kblk > 0 (a multiple of 64, else
+ * take, and for 4 if kblk is not a multiple of 128, the pair kernel's stage depth; path 0 and
+ * 2 then take the single-CTA kernel).  kblk = 0 sums all of K in one accumulator; kblk > 0
+ * (a multiple of 64, else
  * SBP_ERR_INVALID_ARG) adds the partial products of consecutive K blocks of that length into
  * C one after another, in fp32 (the rounding the weight-gradient products over tokens use).
  * `workspace` (>= 256 bytes, device) receives the device status word (see

@@ -249,9 +249,10 @@ __global__ void rmsnorm_bwd_kernel(int64_t rows, int64_t cols, int xdt,
     partial[(int64_t)blockIdx.x * cols + c] = dgs[c];
 }
 
-// dst[c] += sum_p partial[p, c].  A CTA of 256 threads takes 32 columns; its 8 warps sum
-// interleaved eighths of the partial rows, and warp 0 adds the eight sums in a fixed order.
-constexpr int kColsumCols = 32, kColsumGroups = 8;
+// dst[c] += sum_p partial[p, c].  A CTA of 1024 threads takes 32 columns; its 32 warps sum
+// interleaved 32nds of the partial rows (a dozen independent loads per thread for the 444
+// partial rows of the RMSNorm backward), and warp 0 adds the 32 sums in a fixed order.
+constexpr int kColsumCols = 32, kColsumGroups = 32;
 __global__ void __launch_bounds__(kColsumCols * kColsumGroups)
 colsum_partials_kernel(int64_t nparts, int64_t cols, const float* __restrict__ partial,
                        float* __restrict__ dst) {
@@ -259,8 +260,10 @@ colsum_partials_kernel(int64_t nparts, int64_t cols, const float* __restrict__ p
   const int lc = threadIdx.x % kColsumCols, grp = threadIdx.x / kColsumCols;
   const int64_t c = (int64_t)blockIdx.x * kColsumCols + lc;
   float s = 0.f;
-  if (c < cols)
-    for (int64_t p = grp; p < nparts; p += kColsumGroups) s += partial[p * cols + c];
+  if (c < cols) {
+#pragma unroll 4
+    for (int64_t p = grp; p < nparts; p += kColsumGroups) s += __ldg(partial + p * cols + c);
+  }
   red[grp][lc] = s;
   __syncthreads();
   if (grp == 0 && c < cols) {
@@ -377,6 +380,39 @@ __global__ void gather_rope_inv_kernel(int64_t T, int64_t Tc, int64_t s, int hea
     const float c = cr[j], sn = sr[j];
     drow[hh * hd + j] = d1 * c + d2 * sn;
     drow[hh * hd + j + half] = d2 * c - d1 * sn;
+  }
+}
+
+// The same inverse rotation with 16-byte accesses (hd % 8 == 0, rows and tables 16-byte
+// aligned): a thread rotates four consecutive pairs (x_j..x_j+3, x_j+half..x_j+half+3) of one
+// head.  dst row r = rotation of src row (r / Tc) T + s + r % Tc when gather, else of src row r
+// (in place when src == dst).
+__global__ void rope_inv_vec_kernel(int64_t T, int64_t Tc, int64_t s, int heads, int hd,
+                                    int gather, const float* src, float* dst,
+                                    const float* __restrict__ cosb,
+                                    const float* __restrict__ sinb) {
+  const int64_t r = blockIdx.x;
+  const int half = hd / 2, q4 = half / 4;
+  const int64_t b = r / Tc, t = s + r % Tc;
+  const float* srow = src + (gather ? b * T + t : r) * (int64_t)heads * hd;
+  float* drow = dst + r * (int64_t)heads * hd;
+  const float4* cr = reinterpret_cast<const float4*>(cosb + t * half);
+  const float4* sr = reinterpret_cast<const float4*>(sinb + t * half);
+  const int n = heads * q4;
+  for (int p = threadIdx.x; p < n; p += blockDim.x) {
+    const int hh = p / q4;
+    const int j4 = p - hh * q4;
+    const int o1 = hh * hd + 4 * j4, o2 = o1 + half;
+    const float4 a = *reinterpret_cast<const float4*>(srow + o1);
+    const float4 e = *reinterpret_cast<const float4*>(srow + o2);
+    const float4 c = cr[j4], sn = sr[j4];
+    float4 u, w;
+    u.x = a.x * c.x + e.x * sn.x;  w.x = e.x * c.x - a.x * sn.x;
+    u.y = a.y * c.y + e.y * sn.y;  w.y = e.y * c.y - a.y * sn.y;
+    u.z = a.z * c.z + e.z * sn.z;  w.z = e.z * c.z - a.z * sn.z;
+    u.w = a.w * c.w + e.w * sn.w;  w.w = e.w * c.w - a.w * sn.w;
+    *reinterpret_cast<float4*>(drow + o1) = u;
+    *reinterpret_cast<float4*>(drow + o2) = w;
   }
 }
 
@@ -680,6 +716,11 @@ cudaError_t qkv_post(int64_t R, int64_t Tc, int64_t s, int64_t T, int64_t H, int
 cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_t hd, float* x,
                          const float* cosb, const float* sinb, cudaStream_t st) {
   if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
+  if (hd % 8 == 0 && al16p(x) && al16p(cosb) && al16p(sinb)) {
+    launch(rope_inv_vec_kernel, dim3((unsigned)R), dim3(128), 0, st, (int64_t)0, Tc, s,
+           (int)heads, (int)hd, 0, (const float*)x, x, cosb, sinb);
+    return cudaGetLastError();
+  }
   launch(rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, Tc, s, (int)heads, (int)hd, x,
          cosb, sinb);
   return cudaGetLastError();
@@ -690,6 +731,11 @@ cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t
                             const float* sinb, cudaStream_t st) {
   const int64_t R = B * Tc;
   if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
+  if (hd % 8 == 0 && al16p(src) && al16p(dst) && al16p(cosb) && al16p(sinb)) {
+    launch(rope_inv_vec_kernel, dim3((unsigned)R), dim3(128), 0, st, T, Tc, s, (int)heads,
+           (int)hd, 1, src, dst, cosb, sinb);
+    return cudaGetLastError();
+  }
   launch(gather_rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, T, Tc, s, (int)heads,
          (int)hd, src, dst, cosb, sinb);
   return cudaGetLastError();

@@ -8,10 +8,11 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t st);
 cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st);
 cudaError_t gemm_tc_pair(const GemmDesc& g, int* err, cudaStream_t st);
 
-// The CTA-pair kernel needs enough 256 x 256 tiles to occupy every SM pair.
+// The CTA-pair kernel needs enough 256 x 256 tiles to occupy every SM pair, and K blocks
+// (kblk) that are whole 128-column stages.
 static bool use_pair(const GemmDesc& g) {
   const int64_t tiles = ((g.M + 255) / 256) * ((g.N + 255) / 256);
-  return g.path != 3 && tiles >= 74;
+  return g.path != 3 && tiles >= 74 && g.kblk % 128 == 0;
 }
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st) {

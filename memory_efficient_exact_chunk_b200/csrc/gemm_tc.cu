@@ -446,6 +446,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, args.a_mn, args.b_mn);
       const uint32_t smem_base = tc::smem_u32(smem);
+      // descriptors of stage 0 / k-step 0 and their increments (16-byte units): the loop
+      // below only adds loop-invariant values, so the issuing thread keeps up with the
+      // tensor pipe (computing each descriptor afresh costs it more than an N = 256 MMA)
+      const uint64_t a_desc0 = args.a_mn ? tc::smem_desc_sw128(smem_base, 8192, 1024)
+                                         : tc::smem_desc_sw128(smem_base, 16, 1024);
+      const uint64_t b_desc0 = args.b_mn ? tc::smem_desc_sw128(smem_base + A_BYTES, 8192, 1024)
+                                         : tc::smem_desc_sw128(smem_base + A_BYTES, 16, 1024);
+      const uint64_t a_kstep = args.a_mn ? (2048 >> 4) : (32 >> 4);
+      const uint64_t b_kstep = args.b_mn ? (2048 >> 4) : (32 >> 4);
       int s = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       bool ok = true;
@@ -462,16 +471,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int kb = kb0; kb < kb1; ++kb) {
             if (!tc::mbar_wait(&full_bar[s], ph, abort_flag, wait_ns)) { ok = false; break; }
             tc::fence_after_sync();
-            const uint32_t sa = smem_base + s * STAGE_BYTES;
-            const uint32_t sb = sa + A_BYTES;
+            const uint64_t soff = (uint64_t)(s * (STAGE_BYTES >> 4));
+            const uint64_t ad = a_desc0 + soff, bd = b_desc0 + soff;
+            tc::mma_f16_ss(d_tmem, ad, bd, idesc, kb != kb0 ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
-                                            : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                            : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
-              tc::mma_f16_ss(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0 ? 1u : 0u);
-            }
+            for (int kk = 1; kk < BK / 16; ++kk)
+              tc::mma_f16_ss(d_tmem, ad + kk * a_kstep, bd + kk * b_kstep, idesc, 1u);
             issued = true;
             tc::mma_commit(&empty_bar[s]);
             if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -531,17 +536,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // the even CTA issues M=256 N=256 MMAs that read both CTAs' shared memory, and each CTA keeps
 // its 128 accumulator rows in its own TMEM.  Shared-memory traffic per MMA is half that of the
 // single-CTA kernel, which is what lets the tensor cores run closer to their peak.
-constexpr int BM2 = 256, STAGES2 = 6;
-constexpr int A2_BYTES = 128 * BK * 2;              // 16 KB per CTA
-constexpr int B2_BYTES = 128 * BK * 2;              // 16 KB per CTA (half of N)
-constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
-constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024;
+// Operands stream through six slots of 64 k-columns (per CTA: 128 rows of A and 128 rows of
+// B, 16 KB each), consumed in pairs: one mbarrier completes when both slots of a pair hold
+// data, so the MMA thread waits once per eight K = 16 MMAs (a wait costs the issuing thread
+// about as long as an N = 256 MMA runs, and the tensor pipe idles meanwhile), while the
+// producer refills each slot as soon as its own MMAs complete (up to five slots in flight
+// ahead of the one being consumed).
+constexpr int BM2 = 256, NSLOT2 = 6, NPAIR2 = NSLOT2 / 2, BK2 = 2 * BK;
+constexpr int A2_BYTES = 128 * BK * 2;              // 16 KB per CTA per slot
+constexpr int B2_BYTES = 128 * BK * 2;              // 16 KB per CTA per slot (half of N)
+constexpr int SLOT2_BYTES = A2_BYTES + B2_BYTES;
+constexpr int SMEM2_BYTES = NSLOT2 * SLOT2_BYTES + 1024;
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t full_bar[STAGES2], empty_bar[STAGES2], tfull_bar[2], tempty_bar[2];
+  __shared__ uint64_t full_bar[NPAIR2], empty_bar[NSLOT2], tfull_bar[2], tempty_bar[2];
   __shared__ uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -556,10 +567,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES2; ++s) {
-      tc::mbar_init(&full_bar[s], 1);
-      tc::mbar_init(&empty_bar[s], 1);
-    }
+    for (int s = 0; s < NPAIR2; ++s) tc::mbar_init(&full_bar[s], 1);
+    for (int s = 0; s < NSLOT2; ++s) tc::mbar_init(&empty_bar[s], 1);
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tfull_bar[a], 1);
       tc::mbar_init(&tempty_bar[a], 2 * kEpiWarps);   // epilogue warps of both CTAs
@@ -583,9 +592,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int64_t M = g.dynM ? (int64_t)*g.dynM : g.M;
   const int64_t K = g.dynK ? (int64_t)*g.dynK : g.K;
   const int64_t N = g.N;
-  const int nk = (int)((K + BK - 1) / BK);
+  const int nk = (int)((K + BK2 - 1) / BK2);
   const int ntiles = args.nM * args.nN;      // nM counts 256-row tiles here
-  const int kpb = g.kblk > 0 ? (int)(g.kblk / BK) : (nk > 0 ? nk : 1);
+  const int kpb = g.kblk > 0 ? (int)(g.kblk / BK2) : (nk > 0 ? nk : 1);
   const int nblk = nk > 0 ? (nk + kpb - 1) / kpb : 1;
 
   if (warp == 0) {
@@ -603,30 +612,36 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (m0 >= M) continue;
         SBP_TIMED(++ntl;)
         const int ma = m0 + 128 * (int)rank, nb = n0 + 128 * (int)rank;
-        for (int kb = 0; kb < nk; ++kb) {
-          SBP_TIMED(c0 = clock64();)
-          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag)) { ok = false; break; }
-          SBP_TIMED(w_empty += clock64() - c0;)
-          uint8_t* sa = smem + s * STAGE2_BYTES;
-          uint8_t* sb = sa + A2_BYTES;
+        for (int kb = 0; kb < nk && ok; ++kb) {
           const uint32_t fb = tc::mapa(tc::smem_u32(&full_bar[s]), 0);
-          if (rank == 0) tc::mbar_expect_tx(&full_bar[s], 2 * STAGE2_BYTES);
-          const int k0 = kb * BK;
-          if (!args.a_mn) {
-            tc::tma_load_2d_pair(sa, &tmA, fb, k0, ma);
-          } else {
-            tc::tma_load_2d_pair(sa, &tmA, fb, ma, k0);
-            tc::tma_load_2d_pair(sa + 8192, &tmA, fb, ma + 64, k0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = 2 * s + h;
+            SBP_TIMED(c0 = clock64();)
+            if (!tc::mbar_wait(&empty_bar[q], ph ^ 1u, abort_flag)) { ok = false; break; }
+            SBP_TIMED(w_empty += clock64() - c0;)
+            uint8_t* sa = smem + q * SLOT2_BYTES;
+            uint8_t* sb = sa + A2_BYTES;
+            if (h == 0) {
+              if (rank == 0) tc::mbar_expect_tx(&full_bar[s], 2 * 2 * SLOT2_BYTES);
+              issued_mask |= 1u << s;
+              issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
+            }
+            const int k0 = kb * BK2 + h * BK;
+            if (!args.a_mn) {
+              tc::tma_load_2d_pair(sa, &tmA, fb, k0, ma);
+            } else {
+              tc::tma_load_2d_pair(sa, &tmA, fb, ma, k0);
+              tc::tma_load_2d_pair(sa + 8192, &tmA, fb, ma + 64, k0);
+            }
+            if (!args.b_mn) {
+              tc::tma_load_2d_pair(sb, &tmB, fb, k0, nb);
+            } else {
+              tc::tma_load_2d_pair(sb, &tmB, fb, nb, k0);
+              tc::tma_load_2d_pair(sb + 8192, &tmB, fb, nb + 64, k0);
+            }
           }
-          if (!args.b_mn) {
-            tc::tma_load_2d_pair(sb, &tmB, fb, k0, nb);
-          } else {
-            tc::tma_load_2d_pair(sb, &tmB, fb, nb, k0);
-            tc::tma_load_2d_pair(sb + 8192, &tmB, fb, nb + 64, k0);
-          }
-          issued_mask |= 1u << s;
-          issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
-          if (++s == STAGES2) { s = 0; ph ^= 1u; }
+          if (++s == NPAIR2) { s = 0; ph ^= 1u; }
         }
       }
       SBP_TIMED(if (blockIdx.x < 2) printf(
@@ -636,7 +651,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       if (!ok && rank == 0) {
         // wind down: wait (bounded) for the pair's copies in flight on this CTA's barriers
         const uint64_t t0 = tc::globaltimer_ns();
-        for (int q = 0; q < STAGES2; ++q) {
+        for (int q = 0; q < NPAIR2; ++q) {
           if (!(issued_mask & (1u << q))) continue;
           const uint32_t p = (issued_phase >> q) & 1u;
           while (!tc::mbar_try_wait(&full_bar[q], p) &&
@@ -650,6 +665,14 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(BM2, BN, args.a_mn, args.b_mn);
       const uint32_t smem_base = tc::smem_u32(smem);
+      // slot-0 descriptors and the k-step increments (16-byte units), as in the single-CTA
+      // kernel: the loop below only adds loop-invariant values
+      const uint64_t a_desc0 = args.a_mn ? tc::smem_desc_sw128(smem_base, 8192, 1024)
+                                         : tc::smem_desc_sw128(smem_base, 16, 1024);
+      const uint64_t b_desc0 = args.b_mn ? tc::smem_desc_sw128(smem_base + A2_BYTES, 8192, 1024)
+                                         : tc::smem_desc_sw128(smem_base + A2_BYTES, 16, 1024);
+      const uint64_t a_kstep = args.a_mn ? (2048 >> 4) : (32 >> 4);
+      const uint64_t b_kstep = args.b_mn ? (2048 >> 4) : (32 >> 4);
       int s = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       bool ok = true;
@@ -671,19 +694,18 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (!tc::mbar_wait(&full_bar[s], ph, abort_flag)) { ok = false; break; }
             SBP_TIMED(w_full += clock64() - c0; ++nkbt;)
             tc::fence_after_sync();
-            const uint32_t sa = smem_base + s * STAGE2_BYTES;
-            const uint32_t sb = sa + A2_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = args.a_mn ? tc::smem_desc_sw128(sa + kk * 2048, 8192, 1024)
-                                            : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t bd = args.b_mn ? tc::smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                            : tc::smem_desc_sw128(sb + kk * 32, 16, 1024);
-              tc::mma_f16_ss_pair(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0 ? 1u : 0u);
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t soff = (uint64_t)((2 * s + h) * (SLOT2_BYTES >> 4));
+              const uint64_t ad = a_desc0 + soff, bd = b_desc0 + soff;
+              tc::mma_f16_ss_pair(d_tmem, ad, bd, idesc, (kb != kb0 || h) ? 1u : 0u);
+#pragma unroll
+              for (int kk = 1; kk < BK / 16; ++kk)
+                tc::mma_f16_ss_pair(d_tmem, ad + kk * a_kstep, bd + kk * b_kstep, idesc, 1u);
+              tc::mma_commit_pair(&empty_bar[2 * s + h], 0x3);
             }
             issued = true;
-            tc::mma_commit_pair(&empty_bar[s], 0x3);
-            if (++s == STAGES2) { s = 0; ph ^= 1u; }
+            if (++s == NPAIR2) { s = 0; ph ^= 1u; }
           }
           if (!ok) break;
           tc::mma_commit_pair(&tfull_bar[acc], 0x3);
@@ -863,6 +885,7 @@ cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st) {
 
 // The CTA-pair kernel: 256 x 256 tiles; B boxes hold 128 rows (half of N) per CTA.
 cudaError_t gemm_tc_pair(const GemmDesc& g, int* err, cudaStream_t st) {
+  if (g.kblk % BK2 != 0) return cudaErrorNotSupported;   // K blocks are whole stages
   TcArgs args;
   args.g = g;
   args.a_mn = (g.sak == 1) ? 0 : 1;

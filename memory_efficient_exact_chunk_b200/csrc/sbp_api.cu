@@ -1083,6 +1083,8 @@ sbp_status sbp_debug_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
   g.kblk = kblk;
   if (path >= 2 && !gemm_tc_supported(g))
     return fail(SBP_ERR_UNSUPPORTED, "layout not supported by the tensor-core GEMM");
+  if (path == 4 && kblk % 128 != 0)
+    return fail(SBP_ERR_UNSUPPORTED, "the CTA-pair GEMM takes K blocks of whole 128-column stages");
   SBP_CK(gemm(g, st));
   return SBP_OK;
 }

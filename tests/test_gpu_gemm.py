@@ -97,6 +97,30 @@ def test_gemm_k_blocks_match_sliced_products(path, at, K):
     assert ((C.double().cpu() - ref).norm() / ref.norm()).item() <= 1e-5
 
 
+def test_gemm_k_blocks_of_half_a_pair_stage():
+    """kblk = 320 (a multiple of 64, not of the pair kernel's 128-column stage): the automatic
+    choice takes the single-CTA kernel for a product the pair kernel would otherwise take, the
+    result equals the sliced products bit for bit, and an explicit pair request is refused."""
+    import torch
+    from memory_efficient_exact_chunk_b200 import sbp
+    g = torch.Generator().manual_seed(5)
+    M, N, K, kb = 2048, 2560, 1000, 320
+    A = torch.randn(K, M, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16).cuda()
+    C = torch.full((M, N), float("nan"), device="cuda")
+    ws = sbp.debug_gemm_bf16(A, 1, B, 0, C, path=0, kblk=kb)
+    sbp.device_status(ws)
+    Cs = torch.full((M, N), float("nan"), device="cuda")
+    for k0 in range(0, K, kb):
+        k1 = min(K, k0 + kb)
+        sbp.debug_gemm_bf16(A[k0:k1], 1, B[k0:k1], 0, Cs, accumulate=k0 > 0, path=3, ws=ws)
+    sbp.device_status(ws)
+    assert torch.equal(C, Cs)
+    with pytest.raises(sbp.SbpError) as ei:
+        sbp.debug_gemm_bf16(A, 1, B, 0, C, path=4, kblk=kb)
+    assert ei.value.code == 2
+
+
 def test_gemm_k_block_argument_checked():
     import torch
     from memory_efficient_exact_chunk_b200 import sbp

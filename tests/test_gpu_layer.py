@@ -92,7 +92,13 @@ def test_layer_fp32_tiny(D):
     _check(TINY, W, x, dy, D, "f32")
 
 
-@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 200, 3), (QWEN_LIKE, 1, 256, 4)])
+# head_dim 12 (not a multiple of 8): the RoPE kernels' per-pair forms instead of the
+# 16-byte ones
+HD12_BIAS = synth.LayerShape(48, 4, 2, 12, 100, 1e-6, 10000.0, qkv_bias=True)
+
+
+@pytest.mark.parametrize("L,B,T,D", [(GQA, 2, 200, 3), (QWEN_LIKE, 1, 256, 4),
+                                     (HD12_BIAS, 2, 150, 3)])
 def test_layer_fp32_gqa_bias_ragged(L, B, T, D):
     W, x, dy = synth.layer_inputs(1, L, B, T, bf16=False, dy_std=1.0, gamma_std=0.1)
     _check(L, W, x, dy, D, "f32")
