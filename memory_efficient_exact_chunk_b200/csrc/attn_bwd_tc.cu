@@ -62,8 +62,10 @@ struct KvShared {
   float stat[QD_STAGES][2][BT];   // per stage: lse (log2 units), delta of the pair's queries
   // per stage: q_full (Q and the statistics), do_full (dO) -- S^T needs only Q, so its copy
   // lands first -- and qd_empty (the stage may be refilled)
-  uint64_t kv_full, q_full[QD_STAGES], do_full[QD_STAGES], qd_empty[QD_STAGES], s_full[2],
-      s_read[2], dp_full[2], ds_full[2], kv_free, drain;
+  // st_free: the element-wise warps are done with the stage (its statistics, and at the end
+  // of a block the dK / dV rows staged there for the bulk reduce-adds)
+  uint64_t kv_full, q_full[QD_STAGES], do_full[QD_STAGES], qd_empty[QD_STAGES],
+      st_free[QD_STAGES], s_full[2], s_read[2], dp_full[2], ds_full[2], kv_free, drain;
   uint32_t tmem;
   int abort;
 };
@@ -162,6 +164,25 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
+// Bulk asynchronous reduce-add of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// fp32 values from shared memory into global memory, tracked in the calling thread's bulk
+// groups; the shared-memory writes it reads must precede it behind fence.proxy.async.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const float* ssrc,
+                                                    uint32_t bytes) {
+  asm volatile("fence.proxy.async.shared::cta;\n\t"
+               "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;\n\t"
+               "cp.async.bulk.commit_group;" ::"l"(reinterpret_cast<uint64_t>(gdst)),
+               "r"(tc::smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+// the calling thread's bulk operations have read their shared-memory sources
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// the calling thread's bulk operations have completed (global writes done)
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 // Copy this thread's row r of a 128 x 128 bf16 tile staged by TMA (two 64-column chunks, each
 // 128 rows of 128 bytes with the 128-byte swizzle) into TMEM as packed bf16 pairs: chunk c
 // (columns 64 c ..) goes to TMEM columns col0 + 32 c ..; the caller's warp owns the lane.
@@ -183,11 +204,13 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int r, int
 // ================================================================== dK / dV kernel
 // The work of a key tile, pair by pair: (query head hh of the group, query tile qi) for the
 // query tiles i0 .. nq - 1, ordered block by block (qb tiles, counted from the chunk start)
-// and head-major inside a block; first / last: the pair opens / closes its block.  Every role
-// of the CTA walks the same sequence with its own iterator (no divisions per pair).
+// and head-major inside a block; first / last: the pair opens / closes its block, left: pairs
+// after it in its block.  Every role of the CTA walks the same sequence with its own iterator
+// (no divisions per pair).
 struct PairPos {
   int64_t hh, qi;
   bool first, last;
+  int left;
 };
 struct PairIter {
   int qs, nbt, hi, t;       // block start tile, tiles in the block, head in group, tile in block
@@ -206,7 +229,8 @@ struct PairIter {
     p.hh = g * grp + hi;
     p.qi = qs + t;
     p.first = hi == 0 && t == 0;
-    p.last = hi == grp - 1 && t == nbt - 1;
+    p.left = (grp - 1 - hi) * nbt + (nbt - 1 - t);
+    p.last = p.left == 0;
     return p;
   }
   __device__ __forceinline__ void next() {
@@ -253,6 +277,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::mbar_init(&sh.q_full[i], 1);
       tc::mbar_init(&sh.do_full[i], 1);
       tc::mbar_init(&sh.qd_empty[i], 1);
+      tc::mbar_init(&sh.st_free[i], kEwWarps);
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(&sh.s_full[x], 1);
@@ -291,7 +316,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const PairPos pos = it.pos(g);
         const int st = j % QD_STAGES;
         const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
-        if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag) ||
+            !tc::mbar_wait(&sh.st_free[st], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         uint8_t* sQ = sQ0 + 2 * st * TILE;
         uint8_t* sdO = sQ + TILE;
         const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
@@ -428,14 +457,6 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       const PairPos pos = it.pos(g);
       const uint32_t sp = tmem + lane_off + kv_sp(x) + 64u * (uint32_t)wh;  // this warp's columns
-      if (pos.first && kv) {
-        // bring this row's dK / dV accumulator lines into L2 ahead of the block's flush
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          prefetch_l2(a.dKp + ko + wh * 64 + u * 32);
-          prefetch_l2(a.dVp + ko + wh * 64 + u * 32);
-        }
-      }
       const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
       if (!tc::mbar_wait_warp(&sh.q_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
         ok = false;
@@ -504,7 +525,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sh.ds_full[x]);
-      if (!pos.last) continue;
+      if (!pos.last) {
+        if (lane == 0) tc::mbar_arrive(&sh.st_free[st]);   // statistics read
+        continue;
+      }
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner); the
       // release of this pair's Q/dO stage is committed after its last dK / dV product
       if (!tc::mbar_wait_warp(&sh.qd_empty[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
@@ -512,37 +536,46 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         break;
       }
       tc::fence_after_sync();
+      // The stage's Q / dO tiles (64 KB) are free: dK, then dV, of the block are staged there
+      // as fp32 rows (512 B per key row; this lane's row, this warp's 64 columns) and added
+      // into the prefix accumulators by bulk asynchronous reduce-adds, one per (row, column
+      // half), so the flush does not wait for global memory.  This CTA is the only writer of
+      // these rows; the previous block's reduce-adds into them have completed before these
+      // are issued, so every element receives its block sums in block order.
+      float* srow = reinterpret_cast<float*>(sQ0 + 2 * st * TILE) + r * HD + wh * 64;
+      bulk_wait_all();
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        // cc 0, 1: dK columns, cc 2, 3: dV columns of this warp's half (one accumulator at a
-        // time keeps the registers of the flush low)
-        const int c = wh * 2 + (cc & 1);
-        const bool isk = cc < 2;
-        uint32_t rv[32];
-        tc::tmem_ld32(tmem + lane_off + (isk ? KV_DK : KV_DV) + c * 32, rv);
-        tc::tmem_ld_wait();
-        if (kv) {
-          // all loads first (one memory latency), then the adds and the stores
-          float4* pa = reinterpret_cast<float4*>((isk ? a.dKp : a.dVp) + ko + c * 32);
-          const float f = isk ? a.scale : 1.f;
-          float4 xa[8];
+      for (int acc = 0; acc < 2; ++acc) {
+        const bool isk = acc == 0;
+        const float f = isk ? a.scale : 1.f;
+        if (!isk) bulk_wait_read();                    // the dK rows have been read
 #pragma unroll
-          for (int i = 0; i < 8; ++i) xa[i] = pa[i];
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t rv[32];
+          tc::tmem_ld32(tmem + lane_off + (isk ? KV_DK : KV_DV) + (wh * 2 + c2) * 32, rv);
+          tc::tmem_ld_wait();
+          // rows past the prefix end are not staged (nothing reads them; a stray generic
+          // write could also land after the next TMA write of the stage)
+          if (kv) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            xa[i].x += __uint_as_float(rv[4 * i]) * f;
-            xa[i].y += __uint_as_float(rv[4 * i + 1]) * f;
-            xa[i].z += __uint_as_float(rv[4 * i + 2]) * f;
-            xa[i].w += __uint_as_float(rv[4 * i + 3]) * f;
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4*>(srow + c2 * 32)[i] =
+                  make_float4(__uint_as_float(rv[4 * i]) * f, __uint_as_float(rv[4 * i + 1]) * f,
+                              __uint_as_float(rv[4 * i + 2]) * f,
+                              __uint_as_float(rv[4 * i + 3]) * f);
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pa[i] = xa[i];
         }
+        if (kv) bulk_reduce_add_f32((isk ? a.dKp : a.dVp) + ko + wh * 64, srow, 64 * 4);
       }
+      // dK / dV are out of TMEM: the next block's products may overwrite them
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0 && j + 1 < npairs) tc::mbar_arrive(&sh.kv_free);
+      bulk_wait_read();                                // the staged rows have been read
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sh.st_free[st]);
     }
+    bulk_wait_all();                                   // the last block's adds have landed
   }
 
   tc::fence_before_sync();
