@@ -72,10 +72,10 @@ struct KvShared {
 constexpr int KV_TILES_BYTES = (2 + 2 * QD_STAGES) * TILE;        // K, V, 2 x (Q, dO)
 constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
 struct QShared {
-  // per ring stage: k_full (K), v_full (V) -- S needs only K, so its copy lands first -- and
-  // kv_empty (the stage may be refilled)
-  uint64_t qd_full, q_tmem, k_full[KV_RING], v_full[KV_RING], kv_empty[KV_RING], s_full[2],
-      s_read[2], dp_full[2], ds_full[2], dq_done, drain;
+  // per ring stage: kv_full (K and V; one wait per key tile in the MMA thread) and kv_empty
+  // (the stage may be refilled)
+  uint64_t qd_full, q_tmem, kv_full[KV_RING], kv_empty[KV_RING], s_full[2], s_read[2],
+      dp_full[2], ds_full[2], dq_done, drain;
   uint32_t tmem;
   int abort;
 };
@@ -617,8 +617,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     tc::mbar_init(&sh.qd_full, 1);
     tc::mbar_init(&sh.q_tmem, kEwWarps);
     for (int i = 0; i < KV_RING; ++i) {
-      tc::mbar_init(&sh.k_full[i], 1);
-      tc::mbar_init(&sh.v_full[i], 1);
+      tc::mbar_init(&sh.kv_full[i], 1);
       tc::mbar_init(&sh.kv_empty[i], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -661,12 +660,11 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         uint8_t* sK = sKV0 + 2 * st * TILE;
         uint8_t* sV = sK + TILE;
         const int32_t krow = (int32_t)(b * a.T + (int64_t)j * BT);
-        tc::mbar_expect_tx(&sh.k_full[st], TILE);
-        tc::tma_load_3d(sK, &tmK, &sh.k_full[st], 0, (int32_t)g, krow);
-        tc::tma_load_3d(sK + CHUNK, &tmK, &sh.k_full[st], 64, (int32_t)g, krow);
-        tc::mbar_expect_tx(&sh.v_full[st], TILE);
-        tc::tma_load_3d(sV, &tmV, &sh.v_full[st], 0, (int32_t)g, krow);
-        tc::tma_load_3d(sV + CHUNK, &tmV, &sh.v_full[st], 64, (int32_t)g, krow);
+        tc::mbar_expect_tx(&sh.kv_full[st], 2 * TILE);
+        tc::tma_load_3d(sK, &tmK, &sh.kv_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sK + CHUNK, &tmK, &sh.kv_full[st], 64, (int32_t)g, krow);
+        tc::tma_load_3d(sV, &tmV, &sh.kv_full[st], 0, (int32_t)g, krow);
+        tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full[st], 64, (int32_t)g, krow);
         issued = j + 1;
       }
       if (!ok) {
@@ -674,9 +672,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         while (!tc::mbar_try_wait(&sh.qd_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
         for (int j = issued > KV_RING ? issued - KV_RING : 0; j < issued; ++j) {
           const uint32_t pj = (uint32_t)(j / KV_RING) & 1u;
-          while (!tc::mbar_try_wait(&sh.k_full[j % KV_RING], pj) &&
-                 tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-          while (!tc::mbar_try_wait(&sh.v_full[j % KV_RING], pj) &&
+          while (!tc::mbar_try_wait(&sh.kv_full[j % KV_RING], pj) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
         }
       }
@@ -704,7 +700,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc::mma_commit(&sh.s_full[j & 1]);
       };
       bool ok = tc::mbar_wait(&sh.q_tmem, 0, abort_flag) &&        // Q, dO copied into TMEM
-                tc::mbar_wait(&sh.k_full[0], 0, abort_flag);
+                tc::mbar_wait(&sh.kv_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
@@ -715,12 +711,9 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int x = j & 1;
         const uint32_t ph = (uint32_t)(j >> 1) & 1u;
         const uint64_t so = (uint64_t)(j % KV_RING) * kStage;
-        // dP_j = dO V_j^T over S_j once the element-wise warps have read S_j
-        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag) ||
-            !tc::mbar_wait(&sh.v_full[j % KV_RING], (uint32_t)(j / KV_RING) & 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
+        // dP_j = dO V_j^T over S_j once the element-wise warps have read S_j (V_j arrived with
+        // K_j, whose barrier was waited for before S_j)
+        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -730,7 +723,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc::mma_commit(&sh.dp_full[x]);
         if (j + 1 < nkv) {
           const int st1 = (j + 1) % KV_RING;
-          if (!tc::mbar_wait(&sh.k_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
+          if (!tc::mbar_wait(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
             ok = false;
             break;
           }

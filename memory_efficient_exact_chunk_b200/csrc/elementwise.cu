@@ -158,6 +158,42 @@ __global__ void copy_cast_vec_kernel(int64_t n8, const TS* __restrict__ src, TD*
   store8(dst + 8 * i, v);
 }
 
+// hi = bf16(v), lo = bf16(v - hi) of four values, stored as 4 + 4 bf16 (8-byte aligned)
+__device__ __forceinline__ void split4_store(__nv_bfloat16* hi, __nv_bfloat16* lo, float4 v) {
+  const float f[4] = {v.x, v.y, v.z, v.w};
+  float h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    h[k] = __bfloat162float(__float2bfloat16_rn(f[k]));
+    l[k] = f[k] - h[k];
+  }
+  __nv_bfloat162 hh[2] = {__floats2bfloat162_rn(h[0], h[1]), __floats2bfloat162_rn(h[2], h[3])};
+  __nv_bfloat162 ll[2] = {__floats2bfloat162_rn(l[0], l[1]), __floats2bfloat162_rn(l[2], l[3])};
+  *reinterpret_cast<uint2*>(hi) = *reinterpret_cast<const uint2*>(hh);
+  *reinterpret_cast<uint2*>(lo) = *reinterpret_cast<const uint2*>(ll);
+}
+
+// hi + lo split of the chunk's rows of a [B, T, cols] fp32 prefix: row r of hi / lo is row
+// (r / Tc) T + s + r % Tc of src (8 values per thread; cols % 8 == 0, 16-byte aligned rows)
+__global__ void gather_split_bf16_kernel(int64_t n8, int64_t cols8, int64_t Tc, int64_t s,
+                                         int64_t T, const float* __restrict__ src,
+                                         __nv_bfloat16* __restrict__ hi,
+                                         __nv_bfloat16* __restrict__ lo) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const int64_t r = i / cols8, c8 = i - r * cols8;
+  const int64_t srow = (r / Tc) * T + s + r % Tc;
+  float v[8], h[8], l[8];
+  load8(src + (srow * cols8 + c8) * 8, v);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    h[k] = __bfloat162float(__float2bfloat16_rn(v[k]));
+    l[k] = v[k] - h[k];
+  }
+  store8(hi + i * 8, h);
+  store8(lo + i * 8, l);
+}
+
 __global__ void split_bf16_vec_kernel(int64_t n8, const float* __restrict__ x,
                                       __nv_bfloat16* __restrict__ hi,
                                       __nv_bfloat16* __restrict__ lo) {
@@ -390,7 +426,9 @@ __global__ void gather_rope_inv_kernel(int64_t T, int64_t Tc, int64_t s, int hea
 __global__ void rope_inv_vec_kernel(int64_t T, int64_t Tc, int64_t s, int heads, int hd,
                                     int gather, const float* src, float* dst,
                                     const float* __restrict__ cosb,
-                                    const float* __restrict__ sinb) {
+                                    const float* __restrict__ sinb,
+                                    __nv_bfloat16* __restrict__ hi,
+                                    __nv_bfloat16* __restrict__ lo) {
   const int64_t r = blockIdx.x;
   const int half = hd / 2, q4 = half / 4;
   const int64_t b = r / Tc, t = s + r % Tc;
@@ -411,8 +449,15 @@ __global__ void rope_inv_vec_kernel(int64_t T, int64_t Tc, int64_t s, int heads,
     u.y = a.y * c.y + e.y * sn.y;  w.y = e.y * c.y - a.y * sn.y;
     u.z = a.z * c.z + e.z * sn.z;  w.z = e.z * c.z - a.z * sn.z;
     u.w = a.w * c.w + e.w * sn.w;  w.w = e.w * c.w - a.w * sn.w;
-    *reinterpret_cast<float4*>(drow + o1) = u;
-    *reinterpret_cast<float4*>(drow + o2) = w;
+    if (hi) {
+      // the rotated values go out as their hi + lo bf16 split (the fp32 row is not stored)
+      const int64_t ro = r * (int64_t)heads * hd;
+      split4_store(hi + ro + o1, lo + ro + o1, u);
+      split4_store(hi + ro + o2, lo + ro + o2, w);
+    } else {
+      *reinterpret_cast<float4*>(drow + o1) = u;
+      *reinterpret_cast<float4*>(drow + o2) = w;
+    }
   }
 }
 
@@ -718,7 +763,8 @@ cudaError_t rope_inv_f32(int64_t R, int64_t Tc, int64_t s, int64_t heads, int64_
   if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
   if (hd % 8 == 0 && al16p(x) && al16p(cosb) && al16p(sinb)) {
     launch(rope_inv_vec_kernel, dim3((unsigned)R), dim3(128), 0, st, (int64_t)0, Tc, s,
-           (int)heads, (int)hd, 0, (const float*)x, x, cosb, sinb);
+           (int)heads, (int)hd, 0, (const float*)x, x, cosb, sinb,
+           static_cast<__nv_bfloat16*>(nullptr), static_cast<__nv_bfloat16*>(nullptr));
     return cudaGetLastError();
   }
   launch(rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, Tc, s, (int)heads, (int)hd, x,
@@ -733,11 +779,38 @@ cudaError_t gather_rope_inv(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t
   if (R <= 0 || heads <= 0 || hd < 2) return cudaSuccess;
   if (hd % 8 == 0 && al16p(src) && al16p(dst) && al16p(cosb) && al16p(sinb)) {
     launch(rope_inv_vec_kernel, dim3((unsigned)R), dim3(128), 0, st, T, Tc, s, (int)heads,
-           (int)hd, 1, src, dst, cosb, sinb);
+           (int)hd, 1, src, dst, cosb, sinb, static_cast<__nv_bfloat16*>(nullptr),
+           static_cast<__nv_bfloat16*>(nullptr));
     return cudaGetLastError();
   }
   launch(gather_rope_inv_kernel, dim3((unsigned)R), dim3(256), 0, st, T, Tc, s, (int)heads,
          (int)hd, src, dst, cosb, sinb);
+  return cudaGetLastError();
+}
+
+bool gather_split_ok(int64_t hd, int64_t cols, const void* src, const void* hi, const void* lo,
+                     const float* cosb, const float* sinb) {
+  return hd % 8 == 0 && cols % 8 == 0 && al16p(src) && al16p(hi) && al16p(lo) && al16p(cosb) &&
+         al16p(sinb);
+}
+
+cudaError_t gather_rope_inv_split(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t heads,
+                                  int64_t hd, const float* src, void* hi, void* lo,
+                                  const float* cosb, const float* sinb, cudaStream_t st) {
+  const int64_t R = B * Tc;
+  if (R <= 0 || heads <= 0) return cudaSuccess;
+  launch(rope_inv_vec_kernel, dim3((unsigned)R), dim3(128), 0, st, T, Tc, s, (int)heads, (int)hd,
+         1, src, static_cast<float*>(nullptr), cosb, sinb, static_cast<__nv_bfloat16*>(hi),
+         static_cast<__nv_bfloat16*>(lo));
+  return cudaGetLastError();
+}
+
+cudaError_t gather_split_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                              const float* src, void* hi, void* lo, cudaStream_t st) {
+  const int64_t n8 = B * Tc * cols / 8;
+  if (n8 <= 0) return cudaSuccess;
+  launch(gather_split_bf16_kernel, dim3(nblk(n8, 256)), dim3(256), 0, st, n8, cols / 8, Tc, s, T,
+         src, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
   return cudaGetLastError();
 }
 

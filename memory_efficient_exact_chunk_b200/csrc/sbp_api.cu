@@ -776,13 +776,25 @@ static sbp_status layer_backward_run(const sbp_layer_cfg* cfg, const sbp_layer_w
   // dK_pre W_k + dV W_v is stored into dn1 or, with acc, added to it.
   auto kv_backward = [&](int64_t s, int64_t Tc, bool acc) -> sbp_status {
     const int64_t R = B * Tc;
-    SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
-    SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
+    // without biases the fp32 chunk rows of dK / dV are not needed: the bf16 path reads the
+    // prefix rows, rotates dK and writes the hi + lo operands in one pass each
+    const bool fused = dt == DT_BF16 && !has_bias &&
+                       gather_split_ok(hd, dkv, p.dKp, p.khi, p.klo, p.cosb, p.sinb) &&
+                       gather_split_ok(hd, dkv, p.dVp, p.vhi, p.vlo, p.cosb, p.sinb);
+    if (fused) {
+      SBP_CK(gather_rope_inv_split(B, T, Tc, s, Hkv, hd, p.dKp, p.khi, p.klo, p.cosb, p.sinb, st));
+      SBP_CK(gather_split_bf16(B, T, Tc, s, dkv, p.dVp, p.vhi, p.vlo, st));
+    } else {
+      SBP_CK(gather_rope_inv(B, T, Tc, s, Hkv, hd, p.dKp, p.dkpre, p.cosb, p.sinb, st));
+      SBP_CK(gather_chunk(B, T, Tc, s, dkv, DT_F32, p.dVp, p.dvg, st));
+    }
     if (dt == DT_BF16) {
       // dK/dV are fp32 sums over chunks; their bf16 operands carry a hi + lo pair so that the
       // products do not depend on where the fp32 sum happened to round
-      SBP_CK(split_bf16(R * dkv, p.dkpre, p.khi, p.klo, st));
-      SBP_CK(split_bf16(R * dkv, p.dvg, p.vhi, p.vlo, st));
+      if (!fused) {
+        SBP_CK(split_bf16(R * dkv, p.dkpre, p.khi, p.klo, st));
+        SBP_CK(split_bf16(R * dkv, p.dvg, p.vhi, p.vlo, st));
+      }
       const void* parts[4] = {p.khi, p.klo, p.vhi, p.vlo};
       const void* wts[4] = {w->wk, w->wk, w->wv, w->wv};
       float* grs[4] = {gr->wk, gr->wk, gr->wv, gr->wv};

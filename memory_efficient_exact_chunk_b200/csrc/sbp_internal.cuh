@@ -243,6 +243,17 @@ cudaError_t add_residual(int64_t n, int xdt, const void* x, const float* z, int 
 cudaError_t copy_cast(int64_t n, int sdt, const void* src, int ddt, void* dst, cudaStream_t st);
 // hi = bf16(x), lo = bf16(x - hi)
 cudaError_t split_bf16(int64_t n, const float* x, void* hi, void* lo, cudaStream_t st);
+// The two steps above fused for the chunk's rows of a [B, T, ...] fp32 prefix: hi / lo rows r
+// of the inverse-rotated (gather_rope_inv_split) or plain (gather_split_bf16) row
+// (r / Tc) T + s + r % Tc; both need gather_split_ok (head_dim and cols multiples of 8,
+// 16-byte aligned buffers).
+bool gather_split_ok(int64_t hd, int64_t cols, const void* src, const void* hi, const void* lo,
+                     const float* cosb, const float* sinb);
+cudaError_t gather_rope_inv_split(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t heads,
+                                  int64_t hd, const float* src, void* hi, void* lo,
+                                  const float* cosb, const float* sinb, cudaStream_t st);
+cudaError_t gather_split_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t cols,
+                              const float* src, void* hi, void* lo, cudaStream_t st);
 
 // LM head helpers (lmhead.cu)
 // Stable compaction of chunk rows [s, e) with w != 0 (and a valid target) into idx[0..n),
