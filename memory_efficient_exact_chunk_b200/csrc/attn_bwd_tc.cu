@@ -348,8 +348,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && npairs > 0) {
+    if (npairs > 0) {
       // ---------------------------------------------------------------- MMA issuer
+      // the whole warp runs the issue loop; one elected lane issues the MMAs and commits (as in
+      // the dQ kernel)
+      const bool leader = tc::elect_one_sync();
       // order: S^T_0 | dP^T_j S^T_{j+1} grads_j | ...  (S^T_{j+1} goes into the other score
       // region, whose P^T / dS^T the grads of pair j - 1, issued before it, have read)
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: B K-major
@@ -368,15 +371,18 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // S^T_j = K Q_j^T into score region j & 1
       auto scores = [&](int j) {
         const uint64_t so = (j % QD_STAGES) ? kStage : 0;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + kv_sp(j & 1), dK + off, dQk0 + so + off, id_s, kk != 0);
+          for (int kk = 0; kk < 8; ++kk) {   // K = head dim
+            const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+            tc::mma_f16_ss(tmem + kv_sp(j & 1), dK + off, dQk0 + so + off, id_s, kk != 0);
+          }
+          tc::mma_commit(&sh.s_full[j & 1]);
         }
-        tc::mma_commit(&sh.s_full[j & 1]);
+        __syncwarp();
       };
-      bool ok = tc::mbar_wait(&sh.kv_full, 0, abort_flag) &&
-                tc::mbar_wait(&sh.q_full[0], 0, abort_flag);
+      bool ok = tc::mbar_wait_warp(&sh.kv_full, 0, abort_flag) &&
+                tc::mbar_wait_warp(&sh.q_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
@@ -393,21 +399,25 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int st = j % QD_STAGES;
         const uint64_t so = st ? kStage : 0;
         // dP^T_j = V dO_j^T over S^T_j once the element-wise warps have read S^T_j
-        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag) ||
-            !tc::mbar_wait(&sh.do_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+        if (!tc::mbar_wait_warp(&sh.s_read[x], ph, abort_flag) ||
+            !tc::mbar_wait_warp(&sh.do_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + kv_sp(x), dV + off, dOk0 + so + off, id_s, kk != 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+            tc::mma_f16_ss(tmem + kv_sp(x), dV + off, dOk0 + so + off, id_s, kk != 0);
+          }
+          tc::mma_commit(&sh.dp_full[x]);
         }
-        tc::mma_commit(&sh.dp_full[x]);
+        __syncwarp();
         if (j + 1 < npairs) {
           const int st1 = (j + 1) % QD_STAGES;
-          if (!tc::mbar_wait(&sh.q_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u, abort_flag)) {
+          if (!tc::mbar_wait_warp(&sh.q_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u,
+                                  abort_flag)) {
             ok = false;
             break;
           }
@@ -416,24 +426,30 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         // dV += P^T dO, dK += dS^T Q once P^T, dS^T are in TMEM; a new block overwrites dK / dV,
         // so the element-wise warps must have added the last one
-        if (!tc::mbar_wait(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
         if (pos.first && j > 0) {
-          if (!tc::mbar_wait(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait_warp(&sh.kv_free, (uint32_t)nflush & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
           ++nflush;
         }
         tc::fence_after_sync();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = 128 queries
-          const uint64_t offm = so + (uint64_t)((kk * 2048) >> 4);     // MN-major k-step
-          const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
-          const uint32_t pc = kv_sp(x) + kv_packed_col(kk);
-          mma_f16_ts(tmem + KV_DV, tmem + pc, dOm0 + offm, id_g, acc);
-          mma_f16_ts(tmem + KV_DK, tmem + pc + 16, dQm0 + offm, id_g, acc);
+          for (int kk = 0; kk < 8; ++kk) {   // K = 128 queries
+            const uint64_t offm = so + (uint64_t)((kk * 2048) >> 4);     // MN-major k-step
+            const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
+            const uint32_t pc = kv_sp(x) + kv_packed_col(kk);
+            mma_f16_ts(tmem + KV_DV, tmem + pc, dOm0 + offm, id_g, acc);
+            mma_f16_ts(tmem + KV_DK, tmem + pc + 16, dQm0 + offm, id_g, acc);
+          }
+          tc::mma_commit(&sh.qd_empty[st]);
         }
-        tc::mma_commit(&sh.qd_empty[st]);
+        __syncwarp();
       }
       if (issued) {
-        tc::mma_commit(&sh.drain);
+        if (leader) tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.drain, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }
@@ -678,7 +694,11 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && nkv > 0) {
+    if (nkv > 0) {
+      // the whole warp runs the issue loop (waits, bookkeeping); one elected lane issues the
+      // MMAs and their commits: a lone lane in a divergent branch gets far fewer issue slots
+      // while the element-wise warps of its sub-partition issue back to back
+      const bool leader = tc::elect_one_sync();
       // ---------------------------------------------------------------- MMA issuer
       // order: S_0 | dP_j S_{j+1} dQ_j | ...  (S_{j+1} goes into the other score region, whose
       // previous dS has been read by dQ_{j-1}, issued before it)
@@ -692,15 +712,18 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // S_j = Q K_j^T into score region j & 1
       auto scores = [&](int j) {
         const uint64_t so = (uint64_t)(j % KV_RING) * kStage;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = head dim
-          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          mma_f16_ts(tmem + q_sp(j & 1), tmem + Q_QT + 8 * kk, dKk0 + off, id_s, kk != 0);
+          for (int kk = 0; kk < 8; ++kk) {   // K = head dim
+            const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+            mma_f16_ts(tmem + q_sp(j & 1), tmem + Q_QT + 8 * kk, dKk0 + off, id_s, kk != 0);
+          }
+          tc::mma_commit(&sh.s_full[j & 1]);
         }
-        tc::mma_commit(&sh.s_full[j & 1]);
+        __syncwarp();
       };
-      bool ok = tc::mbar_wait(&sh.q_tmem, 0, abort_flag) &&        // Q, dO copied into TMEM
-                tc::mbar_wait(&sh.kv_full[0], 0, abort_flag);
+      bool ok = tc::mbar_wait_warp(&sh.q_tmem, 0, abort_flag) &&   // Q, dO copied into TMEM
+                tc::mbar_wait_warp(&sh.kv_full[0], 0, abort_flag);
       bool issued = false;
       if (ok) {
         tc::fence_after_sync();
@@ -713,17 +736,21 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const uint64_t so = (uint64_t)(j % KV_RING) * kStage;
         // dP_j = dO V_j^T over S_j once the element-wise warps have read S_j (V_j arrived with
         // K_j, whose barrier was waited for before S_j)
-        if (!tc::mbar_wait(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&sh.s_read[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-          mma_f16_ts(tmem + q_sp(x), tmem + Q_OT + 8 * kk, dVk0 + off, id_s, kk != 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t off = so + (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
+            mma_f16_ts(tmem + q_sp(x), tmem + Q_OT + 8 * kk, dVk0 + off, id_s, kk != 0);
+          }
+          tc::mma_commit(&sh.dp_full[x]);
         }
-        tc::mma_commit(&sh.dp_full[x]);
+        __syncwarp();
         if (j + 1 < nkv) {
           const int st1 = (j + 1) % KV_RING;
-          if (!tc::mbar_wait(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u, abort_flag)) {
+          if (!tc::mbar_wait_warp(&sh.kv_full[st1], (uint32_t)((j + 1) / KV_RING) & 1u,
+                                  abort_flag)) {
             ok = false;
             break;
           }
@@ -731,18 +758,21 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           scores(j + 1);
         }
         // dQ += dS_j K_j
-        if (!tc::mbar_wait(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&sh.ds_full[x], ph, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = 128 keys
-          mma_f16_ts(tmem + Q_DQ, tmem + q_sp(x) + packed_col(kk),
-                     dKm0 + so + (uint64_t)((kk * 2048) >> 4), id_g, (j | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {   // K = 128 keys
+            mma_f16_ts(tmem + Q_DQ, tmem + q_sp(x) + packed_col(kk),
+                       dKm0 + so + (uint64_t)((kk * 2048) >> 4), id_g, (j | kk) != 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&sh.kv_empty[j % KV_RING]);
         }
-        tc::mma_commit(&sh.kv_empty[j % KV_RING]);
+        __syncwarp();
       }
-      if (ok) tc::mma_commit(&sh.dq_done);
+      if (ok && leader) tc::mma_commit(&sh.dq_done);
       if (issued) {
-        tc::mma_commit(&sh.drain);
+        if (leader) tc::mma_commit(&sh.drain);
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.drain, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }

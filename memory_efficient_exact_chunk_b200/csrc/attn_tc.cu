@@ -207,8 +207,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ---------------------------------------------------------------- MMA issuer
+      // the whole warp runs the issue loop (waits, bookkeeping); one elected lane issues the
+      // MMAs and commits: a lone lane in a divergent branch gets far fewer issue slots while
+      // the softmax warps of its sub-partition issue back to back
+      const bool leader = tc::elect_one_sync();
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T: both K-major
       const uint32_t id_o = tc::idesc_bf16_f32(128, 128, 0, 1);   // P V: V is MN-major
       const uint32_t aQ = tc::smem_u32(sQ), aK = tc::smem_u32(sK), aV = tc::smem_u32(sV);
@@ -219,12 +223,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint64_t dK0 = tc::smem_desc_sw128(aK, 16, 1024);
       const uint64_t dV0 = tc::smem_desc_sw128(aV, CHUNK_BYTES, 1024);
       constexpr uint64_t kTile = (uint64_t)(TILE_BYTES >> 4);
-      bool ok = tc::mbar_wait(&q_full, 0, abort_flag);
+      bool ok = tc::mbar_wait_warp(&q_full, 0, abort_flag);
       bool issued = false;
       int k_waited = -1;                 // last key tile whose K load this thread has seen
       auto wait_k = [&](int j) -> bool {
         if (k_waited >= j) return true;
-        if (!tc::mbar_wait(&k_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, abort_flag))
+        if (!tc::mbar_wait_warp(&k_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u,
+                                abort_flag))
           return false;
         tc::fence_after_sync();
         k_waited = j;
@@ -234,24 +239,31 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       auto scores = [&](int t, int j) {
         const uint64_t kb = dK0 + ((j % KV_STAGES) ? kTile : 0);
         const uint64_t qb = dQ0 + (t ? kTile : 0);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(tmem + (uint32_t)(t * 128), qb + off, kb + off, id_s, kk != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
+            tc::mma_f16_ss(tmem + (uint32_t)(t * 128), qb + off, kb + off, id_s,
+                           kk != 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&s_full[t]);
         }
-        tc::mma_commit(&s_full[t]);
+        __syncwarp();
         issued = true;
       };
       // O_t += P_t(j) V_j; P_t packed two keys per column over S_t's first 64 columns
       auto pv = [&](int t, int j) -> bool {
-        if (!tc::mbar_wait(&p_full[t], (uint32_t)j & 1u, abort_flag)) return false;
+        if (!tc::mbar_wait_warp(&p_full[t], (uint32_t)j & 1u, abort_flag)) return false;
         tc::fence_after_sync();
         const uint64_t vb = dV0 + ((j % KV_STAGES) ? kTile : 0);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ts(tmem + O_COL + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kk),
-                     vb + (uint64_t)((kk * 2048) >> 4), id_o, (j | kk) != 0 ? 1u : 0u);
-        if (j == (t ? nkv_t[1] : nkv_t[0]) - 1) tc::mma_commit(&o_done[t]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(tmem + O_COL + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kk),
+                       vb + (uint64_t)((kk * 2048) >> 4), id_o, (j | kk) != 0 ? 1u : 0u);
+          if (j == (t ? nkv_t[1] : nkv_t[0]) - 1) tc::mma_commit(&o_done[t]);
+        }
+        __syncwarp();
         return true;
       };
       if (ok && nkv > 0) {
@@ -259,12 +271,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (ok) {
           if (nkv_t[0] > 0) scores(0, 0);
           if (nkv_t[1] > 0) scores(1, 0);
-          tc::mma_commit(&k_empty[0]);
+          if (leader) tc::mma_commit(&k_empty[0]);
         }
       }
       for (int j = 0; j < nkv && ok; ++j) {
         const int st = j % KV_STAGES;
-        if (!tc::mbar_wait(&v_full[st], (uint32_t)(j / KV_STAGES) & 1u, abort_flag)) {
+        if (!tc::mbar_wait_warp(&v_full[st], (uint32_t)(j / KV_STAGES) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -280,7 +292,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (j < nkv_t[1]) {
           if (!pv(1, j)) { ok = false; break; }
         }
-        tc::mma_commit(&v_empty[st]);
+        if (leader) tc::mma_commit(&v_empty[st]);
         if (j + 1 < nkv_t[1]) {
           if (!wait_k(j + 1)) { ok = false; break; }
           scores(1, j + 1);
@@ -288,11 +300,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (more) {
           // every product that reads K_{j+1} is issued (a tile past its diagonal reads none)
           if (!wait_k(j + 1)) { ok = false; break; }
-          tc::mma_commit(&k_empty[(j + 1) % KV_STAGES]);
+          if (leader) tc::mma_commit(&k_empty[(j + 1) % KV_STAGES]);
         }
       }
       if (issued) {
-        tc::mma_commit(&drain_bar);
+        if (leader) tc::mma_commit(&drain_bar);
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&drain_bar, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }

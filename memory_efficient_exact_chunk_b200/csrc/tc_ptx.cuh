@@ -71,6 +71,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return mbar_wait(bar, parity, abort_flag, kWaitLimitNs);
 }
 
+// One lane of the (converged) warp: the same lane on every call with all 32 lanes active.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t p;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+               : "=r"(p));
+  return p != 0;
+}
+
 // Warp-uniform bounded wait: every lane waits, and the warp proceeds only if all lanes saw the
 // phase complete (so that the .sync.aligned tcgen05 instructions that follow run converged).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
