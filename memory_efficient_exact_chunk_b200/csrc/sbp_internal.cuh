@@ -184,7 +184,7 @@ int64_t gemm_lse_tiles(int64_t N);
 // these blocks bound it, and a chunk whose length is a multiple of the block adds the same
 // partial sums as a longer chunk.
 constexpr int64_t kTokenBlock = 4096;
-constexpr int64_t kKvTokenBlock = 1024;
+constexpr int64_t kKvTokenBlock = 2048;
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
 bool gemm_tc_supported(const GemmDesc& g);
