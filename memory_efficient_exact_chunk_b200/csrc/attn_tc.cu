@@ -211,8 +211,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // ---------------------------------------------------------------- MMA issuer
       // the whole warp runs the issue loop (waits, bookkeeping); one elected lane issues the
       // MMAs and commits: a lone lane in a divergent branch gets far fewer issue slots while
-      // the softmax warps of its sub-partition issue back to back
-      const bool leader = tc::elect_one_sync();
+      // the softmax warps of its sub-partition issue back to back.  The lane is elected at each
+      // use (the same lane every time, the warp being converged), which keeps a register free.
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T: both K-major
       const uint32_t id_o = tc::idesc_bf16_f32(128, 128, 0, 1);   // P V: V is MN-major
       const uint32_t aQ = tc::smem_u32(sQ), aK = tc::smem_u32(sK), aV = tc::smem_u32(sV);
@@ -239,7 +239,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       auto scores = [&](int t, int j) {
         const uint64_t kb = dK0 + ((j % KV_STAGES) ? kTile : 0);
         const uint64_t qb = dQ0 + (t ? kTile : 0);
-        if (leader) {
+        if (tc::elect_one_sync()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
@@ -256,7 +256,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!tc::mbar_wait_warp(&p_full[t], (uint32_t)j & 1u, abort_flag)) return false;
         tc::fence_after_sync();
         const uint64_t vb = dV0 + ((j % KV_STAGES) ? kTile : 0);
-        if (leader) {
+        if (tc::elect_one_sync()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_f16_ts(tmem + O_COL + (uint32_t)(t * 128), tmem + (uint32_t)(t * 128 + 8 * kk),
@@ -271,7 +271,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (ok) {
           if (nkv_t[0] > 0) scores(0, 0);
           if (nkv_t[1] > 0) scores(1, 0);
-          if (leader) tc::mma_commit(&k_empty[0]);
+          if (tc::elect_one_sync()) tc::mma_commit(&k_empty[0]);
         }
       }
       for (int j = 0; j < nkv && ok; ++j) {
@@ -292,7 +292,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (j < nkv_t[1]) {
           if (!pv(1, j)) { ok = false; break; }
         }
-        if (leader) tc::mma_commit(&v_empty[st]);
+        if (tc::elect_one_sync()) tc::mma_commit(&v_empty[st]);
         if (j + 1 < nkv_t[1]) {
           if (!wait_k(j + 1)) { ok = false; break; }
           scores(1, j + 1);
@@ -300,11 +300,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (more) {
           // every product that reads K_{j+1} is issued (a tile past its diagonal reads none)
           if (!wait_k(j + 1)) { ok = false; break; }
-          if (leader) tc::mma_commit(&k_empty[(j + 1) % KV_STAGES]);
+          if (tc::elect_one_sync()) tc::mma_commit(&k_empty[(j + 1) % KV_STAGES]);
         }
       }
       if (issued) {
-        if (leader) tc::mma_commit(&drain_bar);
+        if (tc::elect_one_sync()) tc::mma_commit(&drain_bar);
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&drain_bar, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
       }
