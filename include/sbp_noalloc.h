@@ -4,9 +4,8 @@
  *
  * Who needs it: code that may not call cudaMalloc (or any allocating routine) where it runs the
  * backward -- a plug-in inside a framework that owns all device memory through its own pool and
- * hands it only tensors, code running while a CUDA graph is captured, or an embedded runtime
- * with a memory budget fixed in advance.  Such a caller can pass inputs and outputs but no
- * workspace.
+ * hands it only tensors, or an embedded runtime with a memory budget fixed in advance.  Such a
+ * caller can pass inputs and outputs but no workspace.
  */
 #ifndef SBP_NOALLOC_H_
 #define SBP_NOALLOC_H_
@@ -30,8 +29,7 @@ extern "C" {
  *     up the device address of the scratch, which also makes the CUDA runtime load the module
  *     holding the array (the driver reserves its 32 MiB at that moment, not when the library
  *     is opened), and, like the first call of any libsbp entry point on a device, it creates
- *     the library's side streams and events.  Neither may happen under stream capture: make
- *     that first call before any capture begins.
+ *     the library's side streams and events.
  *   - Invalid sizes (n_tokens, hidden or vocab <= 0, num_chunks outside [1, n_tokens]) return
  *     SBP_ERR_INVALID_ARG before any device work or set-up.
  *   - Shared scratch: every call on a device uses the same scratch, which keeps the last call's

@@ -3,9 +3,8 @@
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the point where they run
 // the backward: code inside a framework that owns every device allocation through its own
-// pool and hands plug-ins only tensors, code running while a CUDA graph is being captured
-// (where a fresh allocation would be baked into the graph or is forbidden outright), or
-// embedded runtimes with a fixed memory budget decided before they start.  Such callers can
+// pool and hands plug-ins only tensors, or embedded runtimes with a fixed memory budget
+// decided before they start.  Such callers can
 // still pass their inputs and outputs, but not a workspace.  This entry point therefore keeps
 // its scratch in a fixed-size array that belongs to the library: every GPU that loads the
 // library holds kNoAllocScratchBytes of device memory for it until the process exits.
