@@ -1,7 +1,7 @@
 // Side streams: per device, a few streams on which the library runs independent work of one
 // call next to the caller's stream.  Work is forked from and joined back into the caller's
-// stream with events, so a call stays ordered on the caller's stream (and can be captured in a
-// CUDA graph once the pool exists).  Created on the first call on a device, kept until exit.
+// stream with events, so a call stays ordered on the caller's stream.  Created on the first
+// call on a device, kept until exit.
 #include <mutex>
 
 #include "sbp_internal.cuh"
