@@ -333,8 +333,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(rr[i]);
       }
-      // scale into the exp2 domain; only tiles that reach past the first query need the
-      // causal mask
+      // row maximum of the raw scores (the scale is positive and rounding is monotonic, so
+      // the scaled maximum equals the maximum of the scaled scores); the scale is folded into
+      // the exponent's FMA below.  Only tiles that reach past the first query need the causal
+      // mask (masked scores become -inf).
       const int64_t k0 = (int64_t)j * BKV;
       const bool diag = k0 + BKV - 1 > q_lo;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -342,19 +344,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int lim = (int)(tq - k0);            // keys k0 + i with i > lim are masked
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
-          const float x = (i <= lim) ? sv[i] * a.scale_log2 : -INFINITY;
+          const float x = (i <= lim) ? sv[i] : -INFINITY;
           sv[i] = x;
           m4[i & 3] = fmaxf(m4[i & 3], x);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float x = sv[i] * a.scale_log2;
-          sv[i] = x;
-          m4[i & 3] = fmaxf(m4[i & 3], x);
-        }
+        for (int i = 0; i < 128; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
       }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       float corr = 1.f;
       bool rescale = false;
       if (mx > m_ref + kRescaleThreshold) {
@@ -369,8 +367,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(sv[32 * c + 2 * i] - m_ref);
-          const float p1 = fast_exp2(sv[32 * c + 2 * i + 1] - m_ref);
+          const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * i], a.scale_log2, -m_ref));
+          const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * i + 1], a.scale_log2, -m_ref));
           s4[i & 3] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
