@@ -23,8 +23,11 @@
 // tensor cores compute the next pair's scores while the element-wise warps work on this one.
 // The query tiles are taken in blocks of a fixed number of tiles counted from the chunk start
 // (all heads of the group within a block); after each block dK, dV are added into the fp32
-// prefix accumulators (single owner, no atomics).  A chunk whose length is a multiple of the
-// block therefore adds exactly the partial sums the same queries give inside a longer chunk.
+// prefix accumulators (single owner; bulk asynchronous reduce-adds from shared memory, in
+// block order).  A chunk whose length is a multiple of the block therefore adds exactly the
+// partial sums the same queries give inside a longer chunk.  Q tiles flow through a 3-slot
+// ring and dO tiles (with the pair's lse and delta) through a 2-slot ring: the scores of the
+// next pair read Q first, so its copy starts a pair earlier than dO's.
 //
 // dQ kernel: one CTA owns (sequence b, query head h, 128-query tile); Q and dO live in TMEM.
 // It loops over the key tiles of its causal prefix with two score regions used alternately,
@@ -52,24 +55,28 @@ constexpr int HD = 128;
 constexpr int BT = 128;                     // keys per key tile, queries per query tile
 constexpr int TILE = 128 * HD * 2;          // 32 KB bf16 tile: two 64-column swizzled chunks
 constexpr int CHUNK = TILE / 2;
-constexpr int QD_STAGES = 2;                // Q/dO stages of the dK/dV kernel
+constexpr int Q_SLOTS = 3;                  // Q ring of the dK/dV kernel (S^T reads Q first:
+                                            // a third slot lets its copy start a pair earlier)
+constexpr int DO_SLOTS = 2;                 // dO ring of the dK/dV kernel (with the statistics)
 constexpr int KV_RING = 3;                  // K/V stages of the dQ kernel (the Q/dO staging
                                             // copy lands in the last one before K/V do)
 // All shared state lives in the dynamic allocation (no static shared memory), whose start is
 // 1024-byte aligned as the 128-byte swizzle needs: the tiles first, then the statistics and
 // the barriers.
 struct KvShared {
-  float stat[QD_STAGES][2][BT];   // per stage: lse (log2 units), delta of the pair's queries
-  // per stage: q_full (Q and the statistics), do_full (dO) -- S^T needs only Q, so its copy
-  // lands first -- and qd_empty (the stage may be refilled)
-  // st_free: the element-wise warps are done with the stage (its statistics, and at the end
-  // of a block the dK / dV rows staged there for the bulk reduce-adds)
-  uint64_t kv_full, q_full[QD_STAGES], do_full[QD_STAGES], qd_empty[QD_STAGES],
-      st_free[QD_STAGES], s_full[2], s_read[2], dp_full[2], ds_full[2], kv_free, drain;
+  float stat[DO_SLOTS][2][BT];    // per dO slot: lse (log2 units), delta of the pair's queries
+  // per Q slot: q_full, q_empty (the MMAs reading it have completed), q_free (the element-wise
+  // warps are done with it); per dO slot: do_full (dO and the statistics), do_empty, st_free.
+  // The element-wise warps use a slot only for the statistics and, at the end of a block, to
+  // stage the dK / dV rows for the bulk reduce-adds (rows 0-63 in the Q slot, 64-127 in the dO
+  // slot of the block's last pair).
+  uint64_t kv_full, q_full[Q_SLOTS], q_empty[Q_SLOTS], q_free[Q_SLOTS], do_full[DO_SLOTS],
+      do_empty[DO_SLOTS], st_free[DO_SLOTS], s_full[2], s_read[2], dp_full[2], ds_full[2],
+      kv_free, drain;
   uint32_t tmem;
   int abort;
 };
-constexpr int KV_TILES_BYTES = (2 + 2 * QD_STAGES) * TILE;        // K, V, 2 x (Q, dO)
+constexpr int KV_TILES_BYTES = (2 + Q_SLOTS + DO_SLOTS) * TILE;   // K, V, Q ring, dO ring
 constexpr int KV_SMEM_BYTES = KV_TILES_BYTES + (int)sizeof(KvShared);
 struct QShared {
   // per ring stage: kv_full (K and V; one wait per key tile in the MMA thread) and kv_empty
@@ -253,7 +260,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   KvShared& sh = *reinterpret_cast<KvShared*>(smem_raw + KV_TILES_BYTES);
   uint8_t* sK = smem_raw;
   uint8_t* sV = sK + TILE;
-  uint8_t* sQ0 = sV + TILE;                      // stage st: Q at sQ0 + 2 st TILE, dO after it
+  uint8_t* sQ0 = sV + TILE;                      // Q slot i at sQ0 + i TILE
+  uint8_t* sdO0 = sQ0 + Q_SLOTS * TILE;          // dO slot i at sdO0 + i TILE
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sh.abort;
 
@@ -273,10 +281,14 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&sh.kv_full, 1);
-    for (int i = 0; i < QD_STAGES; ++i) {
+    for (int i = 0; i < Q_SLOTS; ++i) {
       tc::mbar_init(&sh.q_full[i], 1);
+      tc::mbar_init(&sh.q_empty[i], 1);
+      tc::mbar_init(&sh.q_free[i], kEwWarps);
+    }
+    for (int i = 0; i < DO_SLOTS; ++i) {
       tc::mbar_init(&sh.do_full[i], 1);
-      tc::mbar_init(&sh.qd_empty[i], 1);
+      tc::mbar_init(&sh.do_empty[i], 1);
       tc::mbar_init(&sh.st_free[i], kEwWarps);
     }
     for (int x = 0; x < 2; ++x) {
@@ -309,40 +321,49 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::tma_load_3d(sV, &tmV, &sh.kv_full, 0, (int32_t)g, krow);
       tc::tma_load_3d(sV + CHUNK, &tmV, &sh.kv_full, 64, (int32_t)g, krow);
       bool ok = true;
-      int issued = 0;
+      int issued_q = 0, issued_do = 0;
       PairIter it;
       it.init((int)i0, a.nq, (int)grp, a.qb);
       for (int j = 0; j < npairs; ++j, it.next()) {
         const PairPos pos = it.pos(g);
-        const int st = j % QD_STAGES;
-        const uint32_t ph = (uint32_t)(j / QD_STAGES) & 1u;
-        if (!tc::mbar_wait(&sh.qd_empty[st], ph ^ 1u, abort_flag) ||
-            !tc::mbar_wait(&sh.st_free[st], ph ^ 1u, abort_flag)) {
+        const int qs = j % Q_SLOTS, ds = j % DO_SLOTS;
+        const uint32_t qph = (uint32_t)(j / Q_SLOTS) & 1u, dph = (uint32_t)(j / DO_SLOTS) & 1u;
+        const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
+        if (!tc::mbar_wait(&sh.q_empty[qs], qph ^ 1u, abort_flag) ||
+            !tc::mbar_wait(&sh.q_free[qs], qph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* sQ = sQ0 + 2 * st * TILE;
-        uint8_t* sdO = sQ + TILE;
-        const int32_t qrow = (int32_t)(b * a.Tc + pos.qi * BT);
-        tc::mbar_expect_tx(&sh.q_full[st], TILE + 2 * BT * 4);
+        uint8_t* sQ = sQ0 + qs * TILE;
+        tc::mbar_expect_tx(&sh.q_full[qs], TILE);
+        tc::tma_load_3d(sQ, &tmQ, &sh.q_full[qs], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.q_full[qs], 64, (int32_t)pos.hh, qrow);
+        issued_q = j + 1;
+        if (!tc::mbar_wait(&sh.do_empty[ds], dph ^ 1u, abort_flag) ||
+            !tc::mbar_wait(&sh.st_free[ds], dph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sdO = sdO0 + ds * TILE;
         const int64_t srow = (pos.hh * a.B + b) * a.Tcp + pos.qi * BT;
-        tc::tma_load_3d(sQ, &tmQ, &sh.q_full[st], 0, (int32_t)pos.hh, qrow);
-        tc::tma_load_3d(sQ + CHUNK, &tmQ, &sh.q_full[st], 64, (int32_t)pos.hh, qrow);
-        tc::bulk_load(&sh.stat[st][0][0], a.lse_t + srow, BT * 4, &sh.q_full[st]);
-        tc::bulk_load(&sh.stat[st][1][0], a.delta_t + srow, BT * 4, &sh.q_full[st]);
-        tc::mbar_expect_tx(&sh.do_full[st], TILE);
-        tc::tma_load_3d(sdO, &tmdO, &sh.do_full[st], 0, (int32_t)pos.hh, qrow);
-        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.do_full[st], 64, (int32_t)pos.hh, qrow);
-        issued = j + 1;
+        tc::mbar_expect_tx(&sh.do_full[ds], TILE + 2 * BT * 4);
+        tc::tma_load_3d(sdO, &tmdO, &sh.do_full[ds], 0, (int32_t)pos.hh, qrow);
+        tc::tma_load_3d(sdO + CHUNK, &tmdO, &sh.do_full[ds], 64, (int32_t)pos.hh, qrow);
+        tc::bulk_load(&sh.stat[ds][0][0], a.lse_t + srow, BT * 4, &sh.do_full[ds]);
+        tc::bulk_load(&sh.stat[ds][1][0], a.delta_t + srow, BT * 4, &sh.do_full[ds]);
+        issued_do = j + 1;
       }
       if (!ok) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(&sh.kv_full, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-        for (int j = issued > QD_STAGES ? issued - QD_STAGES : 0; j < issued; ++j) {
-          const uint32_t pj = (uint32_t)(j / QD_STAGES) & 1u;
-          while (!tc::mbar_try_wait(&sh.q_full[j % QD_STAGES], pj) &&
+        for (int j = issued_q > Q_SLOTS ? issued_q - Q_SLOTS : 0; j < issued_q; ++j) {
+          const uint32_t pj = (uint32_t)(j / Q_SLOTS) & 1u;
+          while (!tc::mbar_try_wait(&sh.q_full[j % Q_SLOTS], pj) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
-          while (!tc::mbar_try_wait(&sh.do_full[j % QD_STAGES], pj) &&
+        }
+        for (int j = issued_do > DO_SLOTS ? issued_do - DO_SLOTS : 0; j < issued_do; ++j) {
+          const uint32_t pj = (uint32_t)(j / DO_SLOTS) & 1u;
+          while (!tc::mbar_try_wait(&sh.do_full[j % DO_SLOTS], pj) &&
                  tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {}
         }
       }
@@ -357,20 +378,19 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // region, whose P^T / dS^T the grads of pair j - 1, issued before it, have read)
       const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: B K-major
       const uint32_t id_g = tc::idesc_bf16_f32(128, 128, 0, 1);    // dV, dK: B MN-major
-      const uint32_t aQ0 = tc::smem_u32(sQ0);
-      // shared-memory descriptors built once; a k-step adds its byte offset / 16 to the start
-      // address field (the tiles sit below 256 KB, so the field cannot carry over)
-      static_assert(QD_STAGES == 2, "stage descriptors are selected between two stages");
+      const uint32_t aQ0 = tc::smem_u32(sQ0), adO0 = tc::smem_u32(sdO0);
+      // shared-memory descriptors built once; a k-step or a slot adds its byte offset / 16 to
+      // the start address field (the tiles sit below 256 KB, so the field cannot carry over)
       const uint64_t dK = tc::smem_desc_sw128(tc::smem_u32(sK), 16, 1024);
       const uint64_t dV = tc::smem_desc_sw128(tc::smem_u32(sV), 16, 1024);
       const uint64_t dQk0 = tc::smem_desc_sw128(aQ0, 16, 1024);
-      const uint64_t dOk0 = tc::smem_desc_sw128(aQ0 + TILE, 16, 1024);
+      const uint64_t dOk0 = tc::smem_desc_sw128(adO0, 16, 1024);
       const uint64_t dQm0 = tc::smem_desc_sw128(aQ0, CHUNK, 1024);
-      const uint64_t dOm0 = tc::smem_desc_sw128(aQ0 + TILE, CHUNK, 1024);
-      constexpr uint64_t kStage = (uint64_t)((2 * TILE) >> 4);
+      const uint64_t dOm0 = tc::smem_desc_sw128(adO0, CHUNK, 1024);
+      constexpr uint64_t kSlot = (uint64_t)(TILE >> 4);
       // S^T_j = K Q_j^T into score region j & 1
       auto scores = [&](int j) {
-        const uint64_t so = (j % QD_STAGES) ? kStage : 0;
+        const uint64_t so = (uint64_t)(j % Q_SLOTS) * kSlot;
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {   // K = head dim
@@ -396,11 +416,11 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const PairPos pos = it.pos(g);
         const int x = j & 1;
         const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-        const int st = j % QD_STAGES;
-        const uint64_t so = st ? kStage : 0;
+        const int qs = j % Q_SLOTS, ds = j % DO_SLOTS;
+        const uint64_t sq = (uint64_t)qs * kSlot, sd = (uint64_t)ds * kSlot;
         // dP^T_j = V dO_j^T over S^T_j once the element-wise warps have read S^T_j
         if (!tc::mbar_wait_warp(&sh.s_read[x], ph, abort_flag) ||
-            !tc::mbar_wait_warp(&sh.do_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+            !tc::mbar_wait_warp(&sh.do_full[ds], (uint32_t)(j / DO_SLOTS) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -409,15 +429,14 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4);
-            tc::mma_f16_ss(tmem + kv_sp(x), dV + off, dOk0 + so + off, id_s, kk != 0);
+            tc::mma_f16_ss(tmem + kv_sp(x), dV + off, dOk0 + sd + off, id_s, kk != 0);
           }
           tc::mma_commit(&sh.dp_full[x]);
         }
         __syncwarp();
         if (j + 1 < npairs) {
-          const int st1 = (j + 1) % QD_STAGES;
-          if (!tc::mbar_wait_warp(&sh.q_full[st1], (uint32_t)((j + 1) / QD_STAGES) & 1u,
-                                  abort_flag)) {
+          if (!tc::mbar_wait_warp(&sh.q_full[(j + 1) % Q_SLOTS],
+                                  (uint32_t)((j + 1) / Q_SLOTS) & 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -436,15 +455,21 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         tc::fence_after_sync();
         if (leader) {
+          // dK first: its completion releases the Q slot, whose next copy is two pairs ahead
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {   // K = 128 queries
-            const uint64_t offm = so + (uint64_t)((kk * 2048) >> 4);     // MN-major k-step
-            const uint32_t acc = (!pos.first || kk != 0) ? 1u : 0u;
-            const uint32_t pc = kv_sp(x) + kv_packed_col(kk);
-            mma_f16_ts(tmem + KV_DV, tmem + pc, dOm0 + offm, id_g, acc);
-            mma_f16_ts(tmem + KV_DK, tmem + pc + 16, dQm0 + offm, id_g, acc);
+            const uint64_t offm = (uint64_t)((kk * 2048) >> 4);          // MN-major k-step
+            mma_f16_ts(tmem + KV_DK, tmem + kv_sp(x) + kv_packed_col(kk) + 16,
+                       dQm0 + sq + offm, id_g, (!pos.first || kk != 0) ? 1u : 0u);
           }
-          tc::mma_commit(&sh.qd_empty[st]);
+          tc::mma_commit(&sh.q_empty[qs]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t offm = (uint64_t)((kk * 2048) >> 4);
+            mma_f16_ts(tmem + KV_DV, tmem + kv_sp(x) + kv_packed_col(kk), dOm0 + sd + offm, id_g,
+                       (!pos.first || kk != 0) ? 1u : 0u);
+          }
+          tc::mma_commit(&sh.do_empty[ds]);
         }
         __syncwarp();
       }
@@ -473,8 +498,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       const PairPos pos = it.pos(g);
       const uint32_t sp = tmem + lane_off + kv_sp(x) + 64u * (uint32_t)wh;  // this warp's columns
-      const int st = j % QD_STAGES;     // this pair's Q/dO stage also holds lse and delta
-      if (!tc::mbar_wait_warp(&sh.q_full[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+      const int qs = j % Q_SLOTS, ds = j % DO_SLOTS;   // the dO slot holds lse and delta
+      if (!tc::mbar_wait_warp(&sh.do_full[ds], (uint32_t)(j / DO_SLOTS) & 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -482,8 +507,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int q0 = (int)(a.s + pos.qi * BT) + qoff;  // absolute position of its first query
       // no masking needed when every key of the tile precedes every (valid) query here
       const bool full = (k_lo + BT - 1 <= q0) && (pos.qi * BT + qoff + 64 <= a.Tc);
-      const float* lse_s = sh.stat[st][0] + qoff;
-      const float* delta_s = sh.stat[st][1] + qoff;
+      const float* lse_s = sh.stat[ds][0] + qoff;
+      const float* delta_s = sh.stat[ds][1] + qoff;
       // S^T of this warp's 64 queries, one TMEM load
       if (!tc::mbar_wait_warp(&sh.s_full[x], ph, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
@@ -542,23 +567,28 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sh.ds_full[x]);
       if (!pos.last) {
-        if (lane == 0) tc::mbar_arrive(&sh.st_free[st]);   // statistics read
+        if (lane == 0) {
+          tc::mbar_arrive(&sh.st_free[ds]);                // statistics read
+          tc::mbar_arrive(&sh.q_free[qs]);                 // the Q slot is not staged
+        }
         continue;
       }
       // end of a block: add its dK, dV into the fp32 prefix accumulators (single owner); the
       // release of this pair's Q/dO stage is committed after its last dK / dV product
-      if (!tc::mbar_wait_warp(&sh.qd_empty[st], (uint32_t)(j / QD_STAGES) & 1u, abort_flag)) {
+      if (!tc::mbar_wait_warp(&sh.do_empty[ds], (uint32_t)(j / DO_SLOTS) & 1u, abort_flag)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      // The stage's Q / dO tiles (64 KB) are free: dK, then dV, of the block are staged there
-      // as fp32 rows (512 B per key row; this lane's row, this warp's 64 columns) and added
+      // The Q and dO slots of the block's last pair (32 KB each) are free: dK, then dV, of the
+      // block are staged there as fp32 rows (512 B per key row, rows 0-63 in the Q slot and
+      // 64-127 in the dO slot; this lane's row, this warp's 64 columns) and added
       // into the prefix accumulators by bulk asynchronous reduce-adds, one per (row, column
       // half), so the flush does not wait for global memory.  This CTA is the only writer of
       // these rows; the previous block's reduce-adds into them have completed before these
       // are issued, so every element receives its block sums in block order.
-      float* srow = reinterpret_cast<float*>(sQ0 + 2 * st * TILE) + r * HD + wh * 64;
+      float* srow = reinterpret_cast<float*>(r < 64 ? sQ0 + qs * TILE : sdO0 + ds * TILE) +
+                    (r & 63) * HD + wh * 64;
       bulk_wait_all();
 #pragma unroll 1
       for (int acc = 0; acc < 2; ++acc) {
@@ -589,7 +619,10 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (lane == 0 && j + 1 < npairs) tc::mbar_arrive(&sh.kv_free);
       bulk_wait_read();                                // the staged rows have been read
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh.st_free[st]);
+      if (lane == 0) {
+        tc::mbar_arrive(&sh.st_free[ds]);
+        tc::mbar_arrive(&sh.q_free[qs]);
+      }
     }
     bulk_wait_all();                                   // the last block's adds have landed
   }
