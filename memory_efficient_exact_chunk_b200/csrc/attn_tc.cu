@@ -89,6 +89,14 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32; a NaN input is ignored,
+// as fmaxf does)
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -325,13 +333,21 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (!tc::mbar_wait_warp(&s_full[t], (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
       float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tc::tmem_ld32(tmem + lane_off + s_col + (uint32_t)(c * 32), rr);
+      {
+        // the four 32-column loads in flight together, one wait
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tc::tmem_ld32(tmem + lane_off + s_col, r0);
+        tc::tmem_ld32(tmem + lane_off + s_col + 32u, r1);
+        tc::tmem_ld32(tmem + lane_off + s_col + 64u, r2);
+        tc::tmem_ld32(tmem + lane_off + s_col + 96u, r3);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(rr[i]);
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = __uint_as_float(r0[i]);
+          sv[32 + i] = __uint_as_float(r1[i]);
+          sv[64 + i] = __uint_as_float(r2[i]);
+          sv[96 + i] = __uint_as_float(r3[i]);
+        }
       }
       // row maximum of the raw scores (the scale is positive and rounding is monotonic, so
       // the scaled maximum equals the maximum of the scaled scores); the scale is folded into
@@ -343,15 +359,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (diag) {
         const int lim = (int)(tq - k0);            // keys k0 + i with i > lim are masked
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float x = (i <= lim) ? sv[i] : -INFINITY;
-          sv[i] = x;
-          m4[i & 3] = fmaxf(m4[i & 3], x);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+        for (int i = 0; i < 128; ++i) sv[i] = (i <= lim) ? sv[i] : -INFINITY;
       }
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) m4[(i >> 1) & 3] = fmax3f(m4[(i >> 1) & 3], sv[i], sv[i + 1]);
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       float corr = 1.f;
       bool rescale = false;

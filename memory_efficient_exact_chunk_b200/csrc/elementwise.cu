@@ -78,6 +78,54 @@ __global__ void rmsnorm_fwd_vec_kernel(int64_t cols, const TX* __restrict__ x,
   if (rstd && threadIdx.x == 0) rstd[r] = rs;
 }
 
+// RMSNorm forward with the row held in registers (NCH 8-column chunks per thread): x and g are
+// read once, all loads of a thread in flight together; the sum of squares and the products
+// are formed in the same order as in rmsnorm_fwd_vec_kernel, so the results are identical.
+template <typename TX, typename TG, typename TY, int NCH>
+__global__ void __launch_bounds__(kRowThreads)
+rmsnorm_fwd_reg_kernel(int64_t rows, int64_t cols, const TX* __restrict__ x,
+                       const TG* __restrict__ g, TY* __restrict__ y, float* __restrict__ rstd,
+                       float eps) {
+  __shared__ float red[32];
+  float gv[NCH][8];
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+    if (c < cols) load8(g + c, gv[k]);
+  }
+  // a few CTAs per SM take the rows in turn (block_sum synchronises before reusing red)
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const TX* xr = x + r * cols;
+    float v[NCH][8];
+  #pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+      if (c < cols) load8(xr + c, v[k]);
+    }
+    float ss = 0.f;
+  #pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+      if (c < cols) {
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(v[k][i], v[k][i], ss);
+      }
+    }
+    ss = block_sum(ss, red);
+    const float rs = rsqrtf(ss / (float)cols + eps);
+  #pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int64_t c = 8 * (threadIdx.x + (int64_t)k * blockDim.x);
+      if (c < cols) {
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) v[k][i] = v[k][i] * rs * gv[k][i];
+        store8(y + r * cols + c, v[k]);
+      }
+    }
+    if (rstd && threadIdx.x == 0) rstd[r] = rs;
+  }
+}
+
 // RMSNorm backward, 8 columns per access; each thread keeps the dg partial of its columns in
 // registers (NCH <= kVecChunks 8-column chunks per thread, sized to the row so that three CTAs
 // fit on an SM).
@@ -665,13 +713,34 @@ cudaError_t rmsnorm_fwd(int64_t rows, int64_t cols, int xdt, const void* x, int 
   if (cols % 8 == 0 && gdt == DT_BF16 && ydt == DT_BF16 && al16p(x) && al16p(g) && al16p(y)) {
     const auto* gb = static_cast<const __nv_bfloat16*>(g);
     auto* yb = static_cast<__nv_bfloat16*>(y);
-    if (xdt == DT_BF16)
-      launch(rmsnorm_fwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>,
-             dim3((unsigned)rows), dim3(kRowThreads), 0, st, cols,
-             static_cast<const __nv_bfloat16*>(x), gb, yb, rstd, eps);
-    else
-      launch(rmsnorm_fwd_vec_kernel<float, __nv_bfloat16, __nv_bfloat16>, dim3((unsigned)rows),
-             dim3(kRowThreads), 0, st, cols, static_cast<const float*>(x), gb, yb, rstd, eps);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* xf = static_cast<const float*>(x);
+    const int64_t nch = (cols + 8 * kRowThreads - 1) / (8 * kRowThreads);
+    const dim3 grid((unsigned)rows), block(kRowThreads);
+    const int64_t rcap = (int64_t)sm_count() * 8;   // 8 CTAs of 256 threads per SM
+    const dim3 rgrid((unsigned)(rows < rcap ? rows : rcap));
+    if (nch > 4) {
+      if (xdt == DT_BF16)
+        launch(rmsnorm_fwd_vec_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>, grid, block,
+               0, st, cols, xb, gb, yb, rstd, eps);
+      else
+        launch(rmsnorm_fwd_vec_kernel<float, __nv_bfloat16, __nv_bfloat16>, grid, block, 0, st,
+               cols, xf, gb, yb, rstd, eps);
+    } else if (xdt == DT_BF16) {
+      if (nch == 1)
+        launch(rmsnorm_fwd_reg_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, 1>, rgrid, block, 0, st, rows, cols, xb, gb, yb, rstd, eps);
+      else if (nch == 2)
+        launch(rmsnorm_fwd_reg_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, 2>, rgrid, block, 0, st, rows, cols, xb, gb, yb, rstd, eps);
+      else
+        launch(rmsnorm_fwd_reg_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, 4>, rgrid, block, 0, st, rows, cols, xb, gb, yb, rstd, eps);
+    } else {
+      if (nch == 1)
+        launch(rmsnorm_fwd_reg_kernel<float, __nv_bfloat16, __nv_bfloat16, 1>, rgrid, block, 0, st, rows, cols, xf, gb, yb, rstd, eps);
+      else if (nch == 2)
+        launch(rmsnorm_fwd_reg_kernel<float, __nv_bfloat16, __nv_bfloat16, 2>, rgrid, block, 0, st, rows, cols, xf, gb, yb, rstd, eps);
+      else
+        launch(rmsnorm_fwd_reg_kernel<float, __nv_bfloat16, __nv_bfloat16, 4>, rgrid, block, 0, st, rows, cols, xf, gb, yb, rstd, eps);
+    }
     return cudaGetLastError();
   }
   launch(rmsnorm_fwd_kernel, (unsigned)rows, kRowThreads, 0, st, cols, xdt, x, gdt, g, ydt, y, rstd,

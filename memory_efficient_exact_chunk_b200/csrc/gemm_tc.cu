@@ -791,18 +791,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  });
-  return n;
-}
-
 // 2-D bf16 tensor map: inner dimension `inner` (contiguous), outer dimension `outer` with a
 // stride of `ld` elements; box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
@@ -822,6 +810,18 @@ bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  });
+  return n;
+}
 
 // Can the tensor-core kernel take this GEMM?
 bool gemm_tc_supported(const GemmDesc& g) {

@@ -188,6 +188,8 @@ constexpr int64_t kKvTokenBlock = 2048;
 
 cudaError_t gemm(const GemmDesc& g, cudaStream_t st);
 bool gemm_tc_supported(const GemmDesc& g);
+// SMs of the device current at the first call (cached)
+int sm_count();
 
 // ---------------------------------------------------------------------------------------------
 // element-wise / row kernels (elementwise.cu)
