@@ -49,14 +49,17 @@ struct TcArgs {
   GemmDesc g;
   int a_mn, b_mn;
   int nM, nN;
+  int gm;               // row tiles per rasterisation group
   int* err;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int nM, int nN, int& mt, int& nt) {
-  const int per_group = kGroupM * nN;
+// Tile t of a launch: groups of gm row tiles, row tiles fastest within a group, so the CTAs
+// running at the same time share a few A row panels and B column panels in L2.
+__device__ __forceinline__ void tile_coords(int t, int nM, int nN, int gm, int& mt, int& nt) {
+  const int per_group = gm * nN;
   const int group = t / per_group;
-  const int first_m = group * kGroupM;
-  const int gsz = min(nM - first_m, kGroupM);
+  const int first_m = group * gm;
+  const int gsz = min(nM - first_m, gm);
   const int r = t % per_group;
   mt = first_m + r % gsz;
   nt = r / gsz;
@@ -401,7 +404,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok && !stall; t += gridDim.x) {
         int mt, nt;
-        tile_coords(t, args.nM, args.nN, mt, nt);
+        tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
         const int m0 = mt * BM, n0 = nt * BN;
         if (m0 >= M) continue;
         for (int kb = 0; kb < nk; ++kb) {
@@ -461,7 +464,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool issued = false;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int mt, nt;
-        tile_coords(t, args.nM, args.nN, mt, nt);
+        tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
         if ((int64_t)mt * BM >= M) continue;
         for (int b = 0; b < nblk && ok; ++b) {
           if (!tc::mbar_wait(&tempty_bar[acc], aph ^ 1u, abort_flag, wait_ns)) { ok = false; break; }
@@ -503,7 +506,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int mt, nt;
-      tile_coords(t, args.nM, args.nN, mt, nt);
+      tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
       const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
       if (m0 >= M) continue;
       bool ok = true;
@@ -607,7 +610,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       SBP_TIMED(long long w_empty = 0, tp0 = clock64(), c0; int ntl = 0;)
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
         int mt, nt;
-        tile_coords(t, args.nM, args.nN, mt, nt);
+        tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
         const int m0 = mt * BM2, n0 = nt * BN;
         if (m0 >= M) continue;
         SBP_TIMED(++ntl;)
@@ -680,7 +683,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       SBP_TIMED(long long w_full = 0, w_temp = 0, ti0 = clock64(), c0; int nkbt = 0;)
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
         int mt, nt;
-        tile_coords(t, args.nM, args.nN, mt, nt);
+        tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
         if ((int64_t)mt * BM2 >= M) continue;
         for (int b = 0; b < nblk && ok; ++b) {
           SBP_TIMED(c0 = clock64();)
@@ -734,7 +737,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     SBP_TIMED(long long w_tf = 0, t_ep = 0, te0 = clock64(), c0;)
     for (int t = cluster; t < ntiles; t += nclusters) {
       int mt, nt;
-      tile_coords(t, args.nM, args.nN, mt, nt);
+      tile_coords(t, args.nM, args.nN, args.gm, mt, nt);
       const int64_t m0 = (int64_t)mt * BM2, n0 = (int64_t)nt * BN;
       if (m0 >= M) continue;
       bool ok = true;
@@ -809,6 +812,15 @@ bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, 
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Row tiles per rasterisation group.  When all of A fits well inside L2 (126 MB), one group
+// spans every row tile: each B column panel is then read from DRAM once while A stays
+// resident (with groups of kGroupM rows, B is read once per group).  Otherwise groups of
+// kGroupM rows keep the panels the CTAs share at one time small.
+int group_rows(const GemmDesc& g, int nM) {
+  constexpr int64_t kResidentA = 48ll << 20;
+  return g.M * g.K * 2 <= kResidentA ? nM : kGroupM;
+}
+
 }  // namespace
 
 int sm_count() {
@@ -860,6 +872,7 @@ cudaError_t gemm_tc(const GemmDesc& g, int* err, cudaStream_t st) {
   args.b_mn = (g.sbk == 1) ? 0 : 1;
   args.nM = (int)((g.M + BM - 1) / BM);
   args.nN = (int)((g.N + BN - 1) / BN);
+  args.gm = group_rows(g, args.nM);
   args.err = err;
   CUtensorMap ma, mb;
   bool ok;
@@ -892,6 +905,7 @@ cudaError_t gemm_tc_pair(const GemmDesc& g, int* err, cudaStream_t st) {
   args.b_mn = (g.sbk == 1) ? 0 : 1;
   args.nM = (int)((g.M + BM2 - 1) / BM2);
   args.nN = (int)((g.N + BN - 1) / BN);
+  args.gm = group_rows(g, args.nM);
   args.err = err;
   CUtensorMap ma, mb;
   bool ok;
