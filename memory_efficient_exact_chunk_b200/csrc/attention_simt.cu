@@ -178,12 +178,12 @@ inline unsigned warps_blocks(int64_t warps) { return (unsigned)((warps * 32 + 25
 
 cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp, void* o,
-                     float* lse, cudaStream_t st, int path) {
+                     float* lse, const AttnFwdSplit& sc, cudaStream_t st, int path) {
   const int64_t w = B * Tc * H;
   if (w <= 0) return cudaSuccess;
   if (path != 1 && attn_tc_supported(hd, dt, q, Kp, Vp, o)) {
     prof_mark_begin(PROF_ATTN_FWD, st);
-    const cudaError_t e = attn_fwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, lse, status_word(), st);
+    const cudaError_t e = attn_fwd_tc(B, T, Tc, s, H, Hkv, q, Kp, Vp, o, lse, sc, status_word(), st);
     prof_mark_end(PROF_ATTN_FWD, st);
     return e;
   }

@@ -23,6 +23,14 @@
 // Ordering: S_t(j + 1) is issued after PV_t(j), whose P it overwrites; the tensor cores run a
 // CTA's MMAs in issue order, and the commit that signals S_t(j + 1) also covers PV_t(j), so a
 // softmax warp that has seen S_t(j + 1) may rescale O_t.
+// Key-range split: a chunk of 4096 queries has 32 heads x 16 pairs = 512 CTAs of nearly equal
+// work, 3.46 waves of the 148 SMs.  Pairs whose keys reach past the middle of the sequence
+// (key tile segt, fixed by the sequence length) therefore run as two CTAs, one per segment
+// [0, segt) and [segt, end).  The CTA that finishes second combines both partials (maximum,
+// sum, unnormalised O) in segment order, the other parks its partial in scratch; a row whose
+// keys all precede the split gets exactly the unsplit result (its second partial is empty), and
+// the split point does not depend on the chunking, so each row's result is still the same at
+// every D.
 #include <cuda.h>
 
 #include <mutex>
@@ -56,6 +64,12 @@ struct FwdArgs {
   float* lse;             // [B*Tc, H]  natural log
   float scale_log2;       // log2(e) / sqrt(hd)
   int* err;
+  // Key-range split (segt > 0): a pair whose keys reach past key tile segt runs as two CTAs,
+  // keys [0, 128 segt) and [128 segt, end); units = pairs of the launch (the grid is 2 units).
+  int segt, units;
+  float* part;            // [B*Tc, H, HD] fp32: the first-finished segment's unnormalised O
+  float* ml;              // [B*Tc, H, 2]: its running maximum (log2 units) and sum
+  int* flags;             // [units, 2]: finish counter, partial-ready flag (zeroed per launch)
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -119,9 +133,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full, k_full[KV_STAGES], k_empty[KV_STAGES], v_full[KV_STAGES],
-      v_empty[KV_STAGES], s_full[2], p_full[2], o_done[2], drain_bar;
+      v_empty[KV_STAGES], s_full[2], p_full[2], o_done[2], drain_bar, sm_sync;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
+  __shared__ int abort_sh, role_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -131,10 +145,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
 
-  // heavy (late) query-tile pairs first
-  const int qp = a.np - 1 - (int)(blockIdx.x % a.np);
-  const int64_t h = (blockIdx.x / a.np) % a.H;
-  const int64_t b = blockIdx.x / (a.np * a.H);
+  // heavy (late) query-tile pairs first; the second segments of split pairs after all first
+  // segments
+  const int unit = (int)(blockIdx.x % (unsigned)a.units);
+  const int seg = (int)(blockIdx.x / (unsigned)a.units);
+  const int qp = a.np - 1 - (unit % a.np);
+  const int64_t h = (unit / a.np) % a.H;
+  const int64_t b = unit / (a.np * a.H);
   const int64_t g = h / (a.H / a.Hkv);
   const bool has1 = 2 * qp + 1 < a.nq;
   int nkv_t[2];
@@ -146,7 +163,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     q_hi_t[t] = a.s + imin((int64_t)(qt + 1) * BQ, a.Tc);          // one past the last row
     nkv_t[t] = (t == 1 && !has1) ? 0 : (int)((q_hi_t[t] + BKV - 1) / BKV);
   }
-  const int nkv = nkv_t[0] > nkv_t[1] ? nkv_t[0] : nkv_t[1];     // key tiles 0 .. nkv-1
+  // The key range is split at the fixed key tile segt (a function of the sequence length
+  // only), so each query row's two partial results do not depend on the chunking; a row that
+  // sees no key past the split gets exactly its unsplit result.  From here on nkv_t counts the
+  // key tiles of this CTA's segment, from key tile j0.
+  const bool split = a.segt > 0 && (nkv_t[0] > a.segt || nkv_t[1] > a.segt);
+  if (seg == 1 && !split) return;                  // whole CTA, before any set-up
+  const int j0 = (split && seg == 1) ? a.segt : 0;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int end = (split && seg == 0) ? imin(nkv_t[t], a.segt) : nkv_t[t];
+    nkv_t[t] = end > j0 ? end - j0 : 0;
+  }
+  const int nkv = nkv_t[0] > nkv_t[1] ? nkv_t[0] : nkv_t[1];     // key tiles j0 .. j0+nkv-1
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
@@ -162,6 +191,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::mbar_init(&o_done[t], 1);
     }
     tc::mbar_init(&drain_bar, 1);
+    tc::mbar_init(&sm_sync, kSoftmaxWarps);
     abort_sh = 0;
     tc::fence_barrier_init();
   }
@@ -189,7 +219,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int j = 0; j < nkv && ok; ++j) {
         const int st = j % KV_STAGES;
         const uint32_t ph = (uint32_t)(j / KV_STAGES) & 1u;
-        const int32_t krow = (int32_t)(b * a.T + (int64_t)j * BKV);
+        const int32_t krow = (int32_t)(b * a.T + (int64_t)(j0 + j) * BKV);
         if (!tc::mbar_wait(&k_empty[st], ph ^ 1u, abort_flag)) { ok = false; break; }
         tc::mbar_expect_tx(&k_full[st], TILE_BYTES);
         tc::tma_load_3d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, (int32_t)g, krow);
@@ -353,7 +383,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // the scaled maximum equals the maximum of the scaled scores); the scale is folded into
       // the exponent's FMA below.  Only tiles that reach past the first query need the causal
       // mask (masked scores become -inf).
-      const int64_t k0 = (int64_t)j * BKV;
+      const int64_t k0 = (int64_t)(j0 + j) * BKV;
       const bool diag = k0 + BKV - 1 > q_lo;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (diag) {
@@ -372,14 +402,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         m_ref = mx;
         l *= corr;
       }
+      // a row that has seen no key yet (only in a second segment: its keys all precede the
+      // split) keeps P = 0 instead of exp2(-inf + inf)
+      const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * i], a.scale_log2, -m_ref));
-          const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * i + 1], a.scale_log2, -m_ref));
+          const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * i], a.scale_log2, nm));
+          const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * i + 1], a.scale_log2, nm));
           s4[i & 3] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
@@ -407,6 +440,128 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&p_full[t]);
     }
+    if (split) {
+      // ---- a split pair: the CTA that finishes first parks its partial (unnormalised O, its
+      // reference and sum); the other combines both in segment order and writes the result
+      const bool have = n_kv >= 1;
+      if (ok && have && tc::mbar_wait_warp(&o_done[t], 0, abort_flag)) tc::fence_after_sync();
+      else if (have) ok = false;
+      // the eight softmax warps meet on an mbarrier (bounded waits), phases 0, 1, 2 in turn
+      int sync_phase = 0;
+      auto softmax_sync = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm_sync);
+        return tc::mbar_wait_warp(&sm_sync, (uint32_t)(sync_phase++) & 1u, abort_flag);
+      };
+      bool synced = softmax_sync();
+      if (warp == 2) {
+        if (lane == 0) role_sh = (ok && synced) ? atomicAdd(&a.flags[2 * unit], 1) : -1;
+        __syncwarp();
+      }
+      synced = softmax_sync() && synced;
+      const int role = synced ? role_sh : -1;
+      const bool row_ok = tq < q_hi;
+      const int64_t grow = b * a.Tc + (tq - a.s);
+      float* prow = a.part + (grow * a.H + h) * HD;
+      float* mlrow = a.ml + (grow * a.H + h) * 2;
+      const float m_own = have ? m_ref : -INFINITY, l_own = have ? l : 0.f;
+      if (role == 0) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          if (have) {
+            tc::tmem_ld32(tmem + lane_off + o_col + (uint32_t)(c * 32), rr);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = 0u;
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<uint4*>(prow + c * 32 + i) =
+                  make_uint4(rr[i], rr[i + 1], rr[i + 2], rr[i + 3]);
+          }
+        }
+        if (row_ok) *reinterpret_cast<float2*>(mlrow) = make_float2(m_own, l_own);
+        __threadfence();
+        if (softmax_sync() && warp == 2) {
+          if (lane == 0) atomicExch(&a.flags[2 * unit + 1], 1);
+          __syncwarp();
+        }
+      } else if (role == 1) {
+        // the other CTA has taken its turn and is writing its partial: bounded wait for it, the
+        // whole warp looping on lane 0's reading
+        if (warp == 2) {
+          const volatile int* ready = a.flags + 2 * unit + 1;
+          const uint64_t t0 = tc::globaltimer_ns();
+          for (;;) {
+            int stop = 0;
+            if (lane == 0) {
+              if (*ready != 0) stop = 1;
+              else if (tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) stop = 2;
+            }
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop == 2 && lane == 0) *abort_flag = 1;
+            if (stop != 0) break;
+          }
+          __syncwarp();
+        }
+        const bool got = softmax_sync();
+        __threadfence();
+        // warp-uniform from here: the TMEM loads are warp-collective; only the global accesses
+        // of rows past the chunk's end are skipped
+        if (__all_sync(0xffffffffu, got && *abort_flag == 0)) {
+          const float2 mo = row_ok ? __ldcg(reinterpret_cast<const float2*>(mlrow))
+                                   : make_float2(-INFINITY, 0.f);
+          // segment 0 first: (m0, l0, O0) and (m1, l1, O1) in that order whichever is own
+          const float m0 = seg == 0 ? m_own : mo.x, l0 = seg == 0 ? l_own : mo.y;
+          const float m1 = seg == 0 ? mo.x : m_own, l1 = seg == 0 ? mo.y : l_own;
+          const float m = fmaxf(m0, m1);
+          const float a0 = m0 == m ? 1.f : (m0 == -INFINITY ? 0.f : fast_exp2(m0 - m));
+          const float a1 = m1 == m ? 1.f : (m1 == -INFINITY ? 0.f : fast_exp2(m1 - m));
+          const float ls = a0 * l0 + a1 * l1;
+          const float inv = 1.f / ls;
+          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(a.o) + (grow * a.H + h) * HD;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t rr[32];
+            if (have) {
+              tc::tmem_ld32(tmem + lane_off + o_col + (uint32_t)(c * 32), rr);
+              tc::tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) rr[i] = 0u;
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                float v[8];
+#pragma unroll
+                for (int k = 0; k < 8; k += 4) {
+                  const float4 q =
+                      __ldcg(reinterpret_cast<const float4*>(prow + c * 32 + i + k));
+                  const float ot[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float ow = __uint_as_float(rr[i + k + e]);
+                    const float o0 = seg == 0 ? ow : ot[e], o1 = seg == 0 ? ot[e] : ow;
+                    v[k + e] = (a0 * o0 + a1 * o1) * inv;
+                  }
+                }
+                uint4 w;
+                w.x = pack_bf16(v[0], v[1]);
+                w.y = pack_bf16(v[2], v[3]);
+                w.z = pack_bf16(v[4], v[5]);
+                w.w = pack_bf16(v[6], v[7]);
+                *reinterpret_cast<uint4*>(op + c * 32 + i) = w;
+              }
+            }
+          }
+          if (row_ok) a.lse[grow * a.H + h] = (m + __log2f(ls)) * 0.69314718055994531f;
+        }
+      }
+    } else
     // final: wait for the tile's last O += P V, normalise, store
     if (ok && n_kv >= 1 && tc::mbar_wait_warp(&o_done[t], 0, abort_flag)) {
       tc::fence_after_sync();
@@ -486,9 +641,14 @@ bool attn_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, const 
          encode_fn_attn() != nullptr;
 }
 
+size_t attn_fwd_split_flags(int64_t B, int64_t Tc, int64_t H) {
+  const int64_t nq = (Tc + BQ - 1) / BQ, np = (nq + 1) / 2;
+  return (size_t)2 * B * H * np;
+}
+
 cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                         const void* q, const void* Kp, const void* Vp, void* o, float* lse,
-                        int* err, cudaStream_t st) {
+                        const AttnFwdSplit& sc, int* err, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map3(&mq, q, H, B * Tc) || !make_map3(&mk, Kp, Hkv, B * T) ||
       !make_map3(&mv, Vp, Hkv, B * T))
@@ -508,7 +668,26 @@ cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   a.lse = lse;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.err = err;
-  const int64_t grid = B * H * a.np;
+  // Pairs whose keys reach past the middle of the sequence (key tile segt, a function of T
+  // only) run as two CTAs, so that a chunk's 32 heads x 16 pairs fill whole waves of the SMs.
+  const int64_t units = B * H * a.np;
+  const int64_t nkv_max = (s + Tc + BKV - 1) / BKV;
+  a.segt = (int)(((T + BKV - 1) / BKV + 1) / 2);
+  a.units = (int)units;
+  a.part = nullptr;
+  a.ml = nullptr;
+  a.flags = nullptr;
+  const bool split = sc.part && sc.ml && sc.flags && nkv_max > a.segt;
+  if (split) {
+    a.part = sc.part;
+    a.ml = sc.ml;
+    a.flags = sc.flags;
+    cudaError_t e = cudaMemsetAsync(a.flags, 0, sizeof(int) * 2 * (size_t)units, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    a.segt = 0;
+  }
+  const int64_t grid = units * (split ? 2 : 1);
   launch(attn_fwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)SMEM_BYTES, st, mq, mk,
          mv, a);
   return cudaGetLastError();

@@ -112,6 +112,7 @@ struct LayerPlan {
   void *xg, *n1, *q, *o, *n2, *gu, *m, *dgu, *dO;
   float *dyg, *rstd1, *qkv, *alse, *hbuf, *rstd2, *dn2, *dh, *delta, *dq, *dn1, *dxg;
   float *dkpre, *dvg, *rpart, *cpart;
+  int* aflags;   // the attention forward's split flags (its partials use dq and delta)
   // bf16 operand copies of fp32 gradients (bf16 path only)
   void *dyg16, *dh16, *dq16, *khi, *klo, *vhi, *vlo;
   int64_t R;
@@ -163,6 +164,7 @@ void layer_carve(Carver& c, const sbp_layer_cfg& L, LayerPlan& p) {
   p.dkpre = c.take<float>((size_t)R * dkv);
   p.dvg = c.take<float>((size_t)R * dkv);
   p.rpart = c.take<float>(rmsnorm_bwd_partial_floats(d));
+  p.aflags = c.take<int>(attn_fwd_split_flags(B, chunk_max(T, L.num_chunks), L.n_heads));
   int64_t wmax = dq > dkv ? dq : dkv;
   p.cpart = c.take<float>(colsum_partial_floats(wmax));
   p.dyg16 = p.dh16 = p.dq16 = p.khi = p.klo = p.vhi = p.vlo = nullptr;
@@ -325,7 +327,13 @@ sbp_status layer_chunk_forward(const sbp_layer_cfg& L, const sbp_layer_weights& 
       SBP_CK(qkv_post(R, Tc, s, T, H, Hkv, hd, p.qkv, dt, p.q, p.Kp, p.Vp, p.cosb, p.sinb, st));
     }
   }
-  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, st));
+  // the forward's key-range split parks partials in dq and delta, which only the backward
+  // of the same chunk fills, after this call
+  AttnFwdSplit sc;
+  sc.part = p.dq;
+  sc.ml = p.delta;
+  sc.flags = p.aflags;
+  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, dt, p.q, p.Kp, p.Vp, p.o, p.alse, sc, st));
   SBP_CK(copy_cast(R * d, dt, xc, DT_F32, p.hbuf, st));
   SBP_CK(gemm(mk_gemm(R, d, dq, dt, p.o, false, dq, dt, w.wo, true, dq, DT_F32, p.hbuf, d,
                       EPI_ACC), st));
@@ -1132,7 +1140,12 @@ sbp_status sbp_debug_attn_fwd_bf16(int64_t B, int64_t T, int64_t Tc, int64_t s, 
   if (path == 2 && !attn_tc_supported(hd, DT_BF16, q, Kp, Vp, o))
     return fail(SBP_ERR_UNSUPPORTED, "the tensor-core attention needs head_dim 128 and aligned rows");
   tl_status = static_cast<int*>(workspace);
-  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, lse,
+  // the split scratch follows the status word: part, ml, flags
+  AttnFwdSplit sc;
+  sc.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  sc.ml = sc.part + B * Tc * H * hd;
+  sc.flags = reinterpret_cast<int*>(sc.ml + 2 * B * Tc * H);
+  SBP_CK(attn_fwd(B, T, Tc, s, H, Hkv, hd, DT_BF16, q, Kp, Vp, o, lse, sc,
                   static_cast<cudaStream_t>(stream), path));
   return SBP_OK;
 }

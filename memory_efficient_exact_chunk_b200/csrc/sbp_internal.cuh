@@ -285,13 +285,23 @@ cudaError_t dpo_weights(int64_t P, int64_t T, const float* token_ce, const float
 // path: 0 = automatic, 1 = CUDA cores, 2 = tensor cores.
 bool attn_tc_supported(int64_t hd, int dt, const void* q, const void* Kp, const void* Vp,
                        const void* o);
+// Scratch of the tensor-core forward's key-range split: part [B*Tc, H, 128] fp32, ml
+// [B*Tc, H, 2] fp32, flags attn_fwd_split_flags() ints (zeroed by the launch).  Null pointers:
+// no split (then results differ in rounding from calls that split, so every caller of a
+// sequence passes them).
+struct AttnFwdSplit {
+  float* part = nullptr;
+  float* ml = nullptr;
+  int* flags = nullptr;
+};
+size_t attn_fwd_split_flags(int64_t B, int64_t Tc, int64_t H);
 cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                         const void* q, const void* Kp, const void* Vp, void* o, float* lse,
-                        int* err, cudaStream_t st);
+                        const AttnFwdSplit& sc, int* err, cudaStream_t st);
 // Forward for chunk queries q [B*Tc, H, hd] at positions s.. over prefix keys [0, s + Tc).
 cudaError_t attn_fwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,
                      int64_t hd, int dt, const void* q, const void* Kp, const void* Vp, void* o,
-                     float* lse, cudaStream_t st, int path = 0);
+                     float* lse, const AttnFwdSplit& sc, cudaStream_t st, int path = 0);
 // Backward: dq [B*Tc, H, hd] fp32 (overwritten); dKp/dVp [B, T, Hkv, hd] fp32 (+= rows < s+Tc);
 // delta: scratch of attn_bwd_scratch_floats() floats.
 cudaError_t attn_bwd(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, int64_t Hkv,

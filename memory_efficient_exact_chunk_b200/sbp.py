@@ -394,15 +394,25 @@ def profile_end() -> dict:
             for i, n in enumerate(names)}
 
 
+def debug_attn_fwd_workspace_bytes(B, Tc, H, hd):
+    """Workspace of sbp_debug_attn_fwd_bf16: the status word, then the key-range split's
+    partial O (fp32), its maxima and sums, and two flags per query-tile pair."""
+    pairs = ((Tc + 127) // 128 + 1) // 2
+    return 256 + 4 * B * Tc * H * (hd + 2) + 8 * B * H * pairs
+
+
 def debug_attn_fwd_bf16(q, Kp, Vp, o, lse, s, path=0, ws=None, stream=None):
     """Attention forward of a chunk (include/sbp_debug.h); q/o [B*Tc, H, hd], Kp/Vp
     [B, T, Hkv, hd] bf16, lse [B*Tc, H] fp32."""
     B, T, Hkv, hd = Kp.shape
     R, H, _ = q.shape
     Tc = R // B
+    need = debug_attn_fwd_workspace_bytes(B, Tc, H, hd)
     if ws is None:
-        ws = workspace(256, q.device)
+        ws = workspace(need, q.device)
         ws.zero_()
+    elif ws.numel() * ws.element_size() < need:
+        raise ValueError(f"attention forward workspace needs {need} bytes")
     _check(load().sbp_debug_attn_fwd_bf16(B, T, Tc, s, H, Hkv, hd, _ptr(q), _ptr(Kp), _ptr(Vp),
                                           _ptr(o), _ptr(lse), int(path), _ptr(ws),
                                           _stream(stream)))
