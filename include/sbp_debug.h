@@ -60,8 +60,8 @@ sbp_status sbp_debug_gemm_stall_bf16(int64_t M, int64_t N, int64_t K, const void
  * path: 0 automatic, 1 CUDA cores, 2 tensor cores (head_dim 128 only).
  * `workspace` (device, 16-byte aligned) holds the 256-byte status word and then the scratch
  * of the tensor-core path's key-range split: 256 + 4 * B * Tc * H * (hd + 2) + 8 * B * H * P
- * bytes, P = ceil(ceil(Tc / 128) / 2) query-tile pairs.  Query rows whose keys reach past the
- * middle of the sequence (key tile ceil(ceil(T / 128) / 2)) are computed as two partial
+ * bytes, P = ceil(ceil(Tc / 128) / 2) query-tile pairs.  Query rows whose keys reach past a
+ * quarter of the sequence (key tile ceil(ceil(T / 128) / 4)) are computed as two partial
  * softmaxes over the keys before and after that point and combined, in that order, by the
  * second of the two CTAs to finish; the split point depends on T only, so a row's result does
  * not depend on the chunking.

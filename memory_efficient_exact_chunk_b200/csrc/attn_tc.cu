@@ -24,9 +24,9 @@
 // CTA's MMAs in issue order, and the commit that signals S_t(j + 1) also covers PV_t(j), so a
 // softmax warp that has seen S_t(j + 1) may rescale O_t.
 // Key-range split: a chunk of 4096 queries has 32 heads x 16 pairs = 512 CTAs of nearly equal
-// work, 3.46 waves of the 148 SMs.  Pairs whose keys reach past the middle of the sequence
+// work, 3.46 waves of the 148 SMs.  Pairs whose keys reach past a quarter of the sequence
 // (key tile segt, fixed by the sequence length) therefore run as two CTAs, one per segment
-// [0, segt) and [segt, end).  The CTA that finishes second combines both partials (maximum,
+// [0, segt) and [segt, end), the heavier segments launched first.  The CTA that finishes second combines both partials (maximum,
 // sum, unnormalised O) in segment order, the other parks its partial in scratch; a row whose
 // keys all precede the split gets exactly the unsplit result (its second partial is empty), and
 // the split point does not depend on the chunking, so each row's result is still the same at
@@ -67,6 +67,7 @@ struct FwdArgs {
   // Key-range split (segt > 0): a pair whose keys reach past key tile segt runs as two CTAs,
   // keys [0, 128 segt) and [128 segt, end); units = pairs of the launch (the grid is 2 units).
   int segt, units;
+  int seg1_first;         // the grid's first half runs the second segments (the heavier ones)
   float* part;            // [B*Tc, H, HD] fp32: the first-finished segment's unnormalised O
   float* ml;              // [B*Tc, H, 2]: its running maximum (log2 units) and sum
   int* flags;             // [units, 2]: finish counter, partial-ready flag (zeroed per launch)
@@ -145,10 +146,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
 
-  // heavy (late) query-tile pairs first; the second segments of split pairs after all first
-  // segments
+  // heavy (late) query-tile pairs first, and the heavier segment of the split pairs first
   const int unit = (int)(blockIdx.x % (unsigned)a.units);
-  const int seg = (int)(blockIdx.x / (unsigned)a.units);
+  const int seg = (int)(blockIdx.x / (unsigned)a.units) ^ a.seg1_first;
   const int qp = a.np - 1 - (unit % a.np);
   const int64_t h = (unit / a.np) % a.H;
   const int64_t b = unit / (a.np * a.H);
@@ -668,11 +668,13 @@ cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
   a.lse = lse;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.err = err;
-  // Pairs whose keys reach past the middle of the sequence (key tile segt, a function of T
-  // only) run as two CTAs, so that a chunk's 32 heads x 16 pairs fill whole waves of the SMs.
+  // Pairs whose keys reach past a quarter of the sequence (key tile segt, a function of T only)
+  // run as two CTAs, so that a chunk's 32 heads x 16 pairs fill whole waves of the SMs; the
+  // heavier segment's CTAs are launched first and the lighter ones fill the last wave.
   const int64_t units = B * H * a.np;
   const int64_t nkv_max = (s + Tc + BKV - 1) / BKV;
-  a.segt = (int)(((T + BKV - 1) / BKV + 1) / 2);
+  a.segt = (int)(((T + BKV - 1) / BKV + 3) / 4);
+  a.seg1_first = nkv_max - a.segt > a.segt ? 1 : 0;
   a.units = (int)units;
   a.part = nullptr;
   a.ml = nullptr;
@@ -686,6 +688,7 @@ cudaError_t attn_fwd_tc(int64_t B, int64_t T, int64_t Tc, int64_t s, int64_t H, 
     if (e != cudaSuccess) return e;
   } else {
     a.segt = 0;
+    a.seg1_first = 0;
   }
   const int64_t grid = units * (split ? 2 : 1);
   launch(attn_fwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)SMEM_BYTES, st, mq, mk,

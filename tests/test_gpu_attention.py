@@ -35,7 +35,7 @@ def _reference(q, Kp, Vp, s):
     (1, 300, 100, 150, 2, 2, 1.0),      # ragged chunk and sequence
     (1, 1024, 512, 512, 8, 2, 1.0),
     (1, 512, 128, 256, 2, 1, 12.0),     # peaked softmax: exercises the output rescale
-    # the key range split at the middle of the sequence (key tile ceil(ceil(T / 128) / 2)):
+    # the key range split at a quarter of the sequence (key tile ceil(ceil(T / 128) / 4)):
     (2, 512, 256, 256, 4, 2, 1.0),      # two sequences, every pair split
     (1, 600, 250, 350, 2, 1, 1.0),      # unaligned chunk: a tile straddles the split (rows
                                         # before it see no key in the second segment) and a
