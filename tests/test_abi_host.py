@@ -187,3 +187,21 @@ def test_stall_hook_argument_errors(lib):
     assert f(128, 256, 64, None, FAKE, FAKE, 10**6, FAKE, None) == 1
     assert f(128, 256, 64, FAKE, FAKE, FAKE, 10**4, FAKE, None) == 1
     assert f(128, 256, 64, FAKE, FAKE, FAKE, 3 * 10**9, FAKE, None) == 1
+
+
+def test_attention_forward_workspace_size_is_checked_before_any_call():
+    """The debug attention forward's workspace holds the status word and the key-range split's
+    scratch (partial O, maxima and sums, two flags per query-tile pair); a smaller buffer is
+    refused on the host, before the library is called."""
+    import torch
+    B, T, Tc, H, Hkv, hd = 2, 1024, 384, 4, 2, 128
+    pairs = ((Tc + 127) // 128 + 1) // 2
+    need = sbp.debug_attn_fwd_workspace_bytes(B, Tc, H, hd)
+    assert need == 256 + 4 * B * Tc * H * hd + 8 * B * Tc * H + 8 * B * H * pairs
+    q = torch.empty(B * Tc, H, hd, dtype=torch.bfloat16)
+    Kp = torch.empty(B, T, Hkv, hd, dtype=torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty(B * Tc, H)
+    small = torch.empty(need - 16, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        sbp.debug_attn_fwd_bf16(q, Kp, Kp, o, lse, 0, path=2, ws=small)
